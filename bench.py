@@ -1,0 +1,531 @@
+"""Benchmark of the EP MoE dispatch / combine hot path on B200.
+
+One step = one pass of the whole path over one batch of the ``cfg2`` workload (W=8
+virtual EP ranks x T=256 tokens, H=4096 bf16, E=64, K=8): dispatch layout (2 kernels),
+exchange plan of the layout's send counts (1 kernel), dispatch copy (1 kernel), combine
+(1 kernel) with the dispatched rows as the experts' outputs (identity expert). Inputs are
+resident in HBM when the timed region starts; L2 is flushed (a 256 MiB write) before
+every timed step, outside the per-step CUDA-event pair.
+
+Prints ONE JSON line (rank 0). ``value`` = tokens/s over all ranks (each rank runs an
+independent replica: weak scaling, no data-path collective); ``e2e`` = the same metric
+with the step's inputs copied host->device from pinned memory and the result copied
+back inside the timed region. ``roofline`` = the dominant kernel's algorithmic bytes /
+its CUDA-event duration against the measured HBM copy bandwidth; ``ops`` = per-kernel
+figures for the other workloads (int8 / fp8 dispatch, the W=64 all-to-all-v).
+
+``--impl reference`` times the plain CPU oracle (the reference arm of this build) on the
+same workload and metric instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "dispatch+combine tokens/s and achieved HBM GB/s (% of B200 peak), 1 GPU"
+UNIT = "tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+LAUNCHES_PER_STEP = 5          # layout (2 kernels), plan, dispatch, combine
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        try:
+            d = json.load(open(p))
+            return float(d["hbm_gbs"]), "measured"
+        except Exception:
+            pass
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_sha(path):
+    return hashlib.sha256(open(os.path.join(ROOT, path), "rb").read()).hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key):
+    """dram read+write bytes per launch from a committed ncu capture, when the kernel's
+    source has not changed since (else None)."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p)).get(kernel_key)
+        if not d or d.get("source_sha") != source_sha(d["source"]):
+            return None
+        return float(d["bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    def __init__(self, enabled=True):
+        self.enabled = enabled
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        if not self.enabled:
+            return
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        q = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self, uuids):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        mhz, maxes, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            if uuids and not any(u and u in f[1] for u in uuids):
+                continue
+            try:
+                mhz.append(float(f[2]))
+                maxes.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not mhz:
+            return None
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max(maxes),
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+# --------------------------------------------------------------- workloads
+
+def algorithmic_bytes(op, w=None, R=None, a2a=None):
+    """Bytes an op must move at minimum (each input byte read once, each output byte
+    written once)."""
+    if op == "a2a_v":
+        return 2 * a2a.moved_rows() * a2a.row_bytes
+    G, K, H = w.G, w.K, w.H
+    n_act = G if w.active is None else int(w.active.sum())
+    out_elem = 2 if w.quant_mode == 0 else 1
+    if op == "dispatch":
+        return (n_act * H * 2 + R * H * out_elem + (R * 4 if w.quant_mode else 0)
+                + G * K * 4)
+    if op == "combine":
+        return R * H * 2 + G * H * 2 + G * K * 8
+    if op == "layout":
+        return G * K * 4 + (0 if w.active is None else G) + 2 * G * K * 4 + R * 4
+    raise ValueError(op)
+
+
+class MoEStep:
+    """Device-resident buffers of one workload and the five launches of one step."""
+
+    def __init__(self, md, torch, w, device):
+        self.md, self.torch, self.w = md, torch, w
+        t = torch
+        self.ids = t.from_numpy(w.expert_ids.reshape(-1)).to(device)
+        self.active = None if w.active is None else t.from_numpy(w.active).to(device)
+        self.x = t.from_numpy(w.x_bits.view(np.int16)).to(device).view(t.bfloat16)
+        self.wts = t.from_numpy(w.weights.reshape(-1)).to(device)
+        self.L = md.LayoutBuffers.allocate(w.W, w.T, w.K, w.E, device=device)
+        cap = self.L.rows_cap
+        if w.quant_mode == 0:
+            self.ex = t.empty((cap, w.H), dtype=t.bfloat16, device=device)
+            self.scales = None
+            self.expert_out = self.ex                    # identity expert
+        else:
+            self.ex = t.empty((cap, w.H), dtype=t.uint8, device=device)
+            self.scales = t.empty(cap, dtype=t.float32, device=device)
+            g = t.Generator(device=device).manual_seed(7)
+            self.expert_out = t.randn((cap, w.H), generator=g, device=device).to(t.bfloat16)
+        ne = w.E // w.W
+        self.etn = t.empty((w.W, ne), dtype=t.int64, device=device)
+        self.erc = t.empty((w.W, ne, w.W), dtype=t.int32, device=device)
+        self.plan = [t.empty((w.W, w.W), dtype=t.int64, device=device) for _ in range(3)]
+        self.y = t.empty((w.G, w.H), dtype=t.bfloat16, device=device)
+        self.status = t.zeros(1, dtype=t.int32, device=device)
+
+    def run(self, events=None):
+        md, L, w = self.md, self.L, self.w
+        md.moe_dispatch_layout(self.ids, self.active, L, self.status)
+        if events:
+            events[0].record()
+        md.a2a_exchange_plan(L.send_splits, self.plan[0], self.plan[1], self.plan[2], self.status)
+        if events:
+            events[1].record()
+        md.moe_dispatch(self.x, w.H, L, w.quant_mode, self.ex, self.scales, self.status,
+                        expert_token_nums=self.etn, expert_token_nums_type=0,
+                        ep_recv_counts=self.erc)
+        if events:
+            events[2].record()
+        md.moe_combine(self.expert_out, w.H, L, self.wts, self.y, self.status)
+
+
+def time_steps(torch, step, steps, warmup, flush):
+    """Per-step CUDA-event times (ms) of the whole step and of each op."""
+    E = torch.cuda.Event
+    for _ in range(warmup):
+        flush.zero_()
+        step.run()
+    torch.cuda.synchronize()
+    rec = []
+    for _ in range(steps):
+        flush.zero_()
+        ev = [E(enable_timing=True) for _ in range(5)]
+        ev[0].record()
+        step.run(events=ev[1:4])
+        ev[4].record()
+        rec.append(ev)
+    torch.cuda.synchronize()
+    out = {"step": [], "layout": [], "plan": [], "dispatch": [], "combine": []}
+    for ev in rec:
+        out["step"].append(ev[0].elapsed_time(ev[4]))
+        out["layout"].append(ev[0].elapsed_time(ev[1]))
+        out["plan"].append(ev[1].elapsed_time(ev[2]))
+        out["dispatch"].append(ev[2].elapsed_time(ev[3]))
+        out["combine"].append(ev[3].elapsed_time(ev[4]))
+    return out
+
+
+def time_e2e(torch, step, steps, warmup, flush, device):
+    """Same step with its inputs copied in from pinned host memory and y copied out."""
+    w = step.w
+    h_x = torch.from_numpy(w.x_bits.view(np.int16)).pin_memory()
+    h_ids = torch.from_numpy(w.expert_ids.reshape(-1)).pin_memory()
+    h_w = torch.from_numpy(w.weights.reshape(-1)).pin_memory()
+    h_act = None if w.active is None else torch.from_numpy(w.active).pin_memory()
+    h_y = torch.empty((w.G, w.H), dtype=torch.int16).pin_memory()
+    h2d = h_x.numel() * 2 + h_ids.numel() * 4 + h_w.numel() * 4 + (0 if h_act is None else h_act.numel())
+    d2h = h_y.numel() * 2
+    x16 = step.x.view(torch.int16)
+    y16 = step.y.view(torch.int16)
+
+    def one():
+        x16.copy_(h_x, non_blocking=True)
+        step.ids.copy_(h_ids, non_blocking=True)
+        step.wts.copy_(h_w, non_blocking=True)
+        if h_act is not None:
+            step.active.copy_(h_act, non_blocking=True)
+        step.run()
+        h_y.copy_(y16, non_blocking=True)
+
+    for _ in range(warmup):
+        flush.zero_()
+        one()
+    torch.cuda.synchronize()
+    times = []
+    E = torch.cuda.Event
+    for _ in range(steps):
+        flush.zero_()
+        a, b = E(enable_timing=True), E(enable_timing=True)
+        a.record()
+        one()
+        b.record()
+        times.append((a, b))
+    torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in times]
+    return statistics.mean(ms), h2d, d2h
+
+
+def oracle_step(oracle, w):
+    lay = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active)
+    oracle.a2a_exchange_plan(lay["send_splits"])
+    ex, sc, _ = oracle.moe_dispatch(w.x_bits, lay["dst_row"], w.K, lay["rows_cap"], w.quant_mode)
+    oracle.moe_recv_counts(w.W, w.E, lay["cnt"], 0)
+    if w.quant_mode == 0:
+        oracle.moe_combine_f32(ex, lay["dst_row"], w.weights, w.K)
+    else:
+        eo = np.zeros((lay["rows_cap"], w.H), np.uint16)
+        oracle.moe_combine_f32(eo, lay["dst_row"], w.weights, w.K)
+
+
+def cpu_baseline(w, budget_s=10.0):
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    oracle_step(oracle, w)                       # warm-up (builds the library if needed)
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        oracle_step(oracle, w)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return {"value": n * w.G / el, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{n} full {w.name} steps (layout, plan, dispatch, fp32 combine) on one "
+                      f"host thread, {el:.1f} s; {cores} cores visible"}
+
+
+def config_of(w, flush_note=True):
+    c = {"workload": f"{w.name}: W={w.W} virtual EP ranks x T={w.T} tokens, H={w.H} bf16, "
+                     f"E={w.E}, K={w.K}, quant={'none' if w.quant_mode == 0 else w.quant_mode}",
+         "global_batch": w.G, "seq_len": 1, "parallelism": "ep-virtual (one GPU)"}
+    if flush_note:
+        c["l2"] = "flushed (256 MiB write) before every timed step"
+    return c
+
+
+# --------------------------------------------------------------- per-op sweep
+
+def op_sweep(md, torch, device, hbm, reps=10):
+    import workloads as wl
+    out = []
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=device)
+    for name in ("cfg3", "cfg4"):
+        w = wl.moe_workload(name, seed=0)
+        st = MoEStep(md, torch, w, device)
+        t = time_steps(torch, st, reps, 3, flush)
+        R = int(st.L.expert_base[-1].item())
+        for op in ("layout", "dispatch", "combine"):
+            ms = statistics.mean(t[op])
+            b = algorithmic_bytes(op, w, R)
+            out.append({"workload": name, "op": op, "us": round(ms * 1e3, 2),
+                        "bytes": b, "GB/s": round(b / ms / 1e6, 1),
+                        "frac": round(b / ms / 1e6 / hbm, 4)})
+        out.append({"workload": name, "op": "step", "us": round(statistics.mean(t["step"]) * 1e3, 2),
+                    "tokens/s": round(w.G / (statistics.mean(t["step"]) / 1e3), 1)})
+        assert int(st.status.item()) == 0, md.status_string(int(st.status.item()))
+        del st
+        torch.cuda.empty_cache()
+    # raw all-to-all-v, W = 64
+    a = wl.a2a_workload(seed=0)
+    W, E_ = a.W, a.row_elems
+    cap_in, cap_out = a.cap_in, a.cap_out
+    S = torch.from_numpy(a.in_splits).to(device)
+    plan = [torch.empty((W, W), dtype=torch.int64, device=device) for _ in range(3)]
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    i = torch.arange(W, device=device, dtype=torch.float32)[:, None]
+    k = torch.arange(cap_in, device=device, dtype=torch.float32)[None, :]
+    inp = (10.0 * i + k).to(torch.bfloat16)[:, :, None].expand(W, cap_in, E_).contiguous()
+    outb = torch.empty((W, cap_out, E_), dtype=torch.bfloat16, device=device)
+    Ev = torch.cuda.Event
+    times_plan, times_a2a = [], []
+    for r in range(reps + 3):
+        flush.zero_()
+        e0, e1, e2 = Ev(enable_timing=True), Ev(enable_timing=True), Ev(enable_timing=True)
+        e0.record()
+        md.a2a_exchange_plan(S, plan[0], plan[1], plan[2], status)
+        e1.record()
+        md.a2a_v(inp, cap_in, outb, cap_out, 2 * E_, W, plan[0], plan[1], plan[2], status)
+        e2.record()
+        if r >= 3:
+            times_plan.append((e0, e1))
+            times_a2a.append((e1, e2))
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ms_p = statistics.mean(a.elapsed_time(b) for a, b in times_plan)
+    ms_a = statistics.mean(x.elapsed_time(y) for x, y in times_a2a)
+    b = algorithmic_bytes("a2a_v", a2a=a)
+    out.append({"workload": "a2a64", "op": "plan", "us": round(ms_p * 1e3, 2)})
+    out.append({"workload": "a2a64", "op": "a2a_v", "us": round(ms_a * 1e3, 2), "bytes": b,
+                "GB/s": round(b / ms_a / 1e6, 1), "frac": round(b / ms_a / 1e6 / hbm, 4),
+                "rows/s": round(a.moved_rows() / (ms_a / 1e3), 1)})
+    del inp, outb
+    torch.cuda.empty_cache()
+    return out
+
+
+# ---------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="cfg2")
+    ap.add_argument("--no-ops", action="store_true", help="skip the per-op sweep of other workloads")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    import workloads as wl
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        return run_reference(args, wl)
+
+    import torch
+    import torch.distributed as dist
+    import combine_a2a_exchange_b200 as md
+
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=device)
+
+    hbm, peak_src = measured_peaks()
+    w = wl.moe_workload(args.workload, seed=rank)
+    step = MoEStep(md, torch, w, device)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=device)
+
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(device).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(enabled=(rank == 0))
+
+    # warm-up
+    for _ in range(args.warmup):
+        flush.zero_()
+        step.run()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    t = time_steps(torch, step, args.steps, 0, flush)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = sampler.stop([uuid.replace("GPU-", "")] if uuid else None) if rank == 0 else None
+    status = int(step.status.item())
+    if status != 0:
+        raise RuntimeError(f"device status after the timed steps: {md.status_string(status)}")
+
+    ms_step = statistics.mean(t["step"])
+    if world > 1:
+        tt = torch.tensor([ms_step], device=device, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_step = float(tt.item())
+    R = int(step.L.expert_base[-1].item())
+    per_op = {op: statistics.mean(t[op]) for op in ("layout", "plan", "dispatch", "combine")}
+    dom = max(("dispatch", "combine"), key=lambda o: per_op[o])
+    dom_bytes = algorithmic_bytes(dom, w, R)
+    achieved = dom_bytes / (per_op[dom] * 1e-3) / 1e9
+    kernel_key = {"dispatch": "dispatch_kernel<0>", "combine": "combine_kernel<8>"}[dom]
+    traffic = ncu_traffic(kernel_key)
+
+    e2e = None
+    if not args.no_e2e:
+        ms_e2e, h2d, d2h = time_e2e(torch, step, args.steps, args.warmup, flush, device)
+        if world > 1:
+            tt = torch.tensor([ms_e2e], device=device, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            ms_e2e = float(tt.item())
+        e2e = {"value": round(world * w.G / (ms_e2e / 1e3), 1), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": round(ms_e2e, 4)}
+
+    ops = None
+    if rank == 0 and world == 1 and not args.no_ops:
+        del step
+        torch.cuda.empty_cache()
+        ops = op_sweep(md, torch, device, hbm)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    step_bytes = sum(algorithmic_bytes(op, w, R) for op in ("layout", "dispatch", "combine"))
+    line = {
+        "metric": METRIC,
+        "value": round(world * w.G / (ms_step / 1e3), 1),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded generator; no dataset)",
+        "config": config_of(w),
+        "hbm_GBps_step": round(step_bytes / (ms_step * 1e-3) / 1e9, 1),
+        "frac_of_peak_step": round(step_bytes / (ms_step * 1e-3) / 1e9 / hbm, 4),
+        "per_op_us": {k: round(v * 1e3, 2) for k, v in per_op.items()},
+        "per_op_frac": {op: round(algorithmic_bytes(op, w, R) / (per_op[op] * 1e-3) / 1e9 / hbm, 4)
+                        for op in ("dispatch", "combine")},
+        "roofline": {"bound": "hbm", "kernel": kernel_key, "achieved": round(achieved, 1),
+                     "peak": hbm, "peak_source": peak_src, "unit": "GB/s",
+                     "frac": round(achieved / hbm, 4), "traffic": traffic,
+                     "algorithmic_bytes": dom_bytes},
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "clocks": clocks,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+        "ops": ops,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_reference(args, wl):
+    import oracle
+    w = wl.moe_workload(args.workload, seed=0)
+    cores = len(os.sched_getaffinity(0))
+    for _ in range(args.warmup):
+        oracle_step(oracle, w)
+    ts = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle_step(oracle, w)
+        ts.append(time.perf_counter() - t0)
+    ms = statistics.mean(ts) * 1e3
+    value = round(w.G / (ms / 1e3), 1)
+    line = {
+        "impl": "reference",
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded generator; no dataset)", "config": config_of(w, False),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"each step one full {w.name} pass (layout, plan, dispatch, "
+                                   f"fp32 combine) on one host thread; {cores} cores visible"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

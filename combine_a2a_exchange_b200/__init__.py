@@ -1,0 +1,227 @@
+"""Python binding of libmoedisp: EP MoE dispatch / combine and the all-to-all-v exchange
+on NVIDIA B200 (sm_100a).
+
+This module only marshals arguments: torch tensors (device memory allocated by torch)
+become raw pointers, the current torch CUDA stream becomes the cudaStream_t, and every
+step of the path runs in the CUDA kernels of ``libmoedisp.so``. The functions carry the
+names of the C ABI (``include/moedisp.h``) without its ``moedisp_`` prefix. There is no
+CPU fallback: importing this package fails if the library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIBRARY_PATH = os.path.join(_HERE, "libmoedisp.so")
+
+if not os.path.exists(LIBRARY_PATH):
+    raise ImportError(
+        f"{LIBRARY_PATH} is missing: build it with `python -m combine_a2a_exchange_b200._build` "
+        "(or __graft_entry__.build()); this package has no fallback implementation")
+
+_lib = ctypes.CDLL(LIBRARY_PATH)
+
+MOEDISP_OK = 0
+MOEDISP_ERR_NULLPTR = -1
+MOEDISP_ERR_INVALID = -2
+MOEDISP_ERR_MISALIGNED = -3
+MOEDISP_ERR_ALIASED = -4
+MOEDISP_ERR_UNSUPPORTED = -5
+MOEDISP_ERR_WORKSPACE = -6
+MOEDISP_ERR_CUDA = -7
+
+STATUS_CAPACITY = 1
+STATUS_BAD_EXPERT_ID = 2
+STATUS_TIMEOUT = 4
+STATUS_BAD_SPLIT = 8
+
+QUANT_NONE = 0
+QUANT_INT8 = 2
+QUANT_FP8_E4M3 = 3
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_I64 = ctypes.c_int64
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("W", _I), ("T", _I), ("K", _I), ("E", _I)]
+
+
+class Layout(ctypes.Structure):
+    _fields_ = [("cnt", _P), ("occ", _P), ("dst_row", _P), ("assist_info", _P),
+                ("expert_base", _P), ("rank_base", _P), ("send_splits", _P),
+                ("rows_cap", _I64)]
+
+
+def _sig(name, argtypes, restype=ctypes.c_int):
+    f = getattr(_lib, name)
+    f.argtypes = argtypes
+    f.restype = restype
+    return f
+
+
+_status_string = _sig("moedisp_status_string", [_I], ctypes.c_char_p)
+_version = _sig("moedisp_version", [])
+_plan = _sig("moedisp_a2a_exchange_plan", [_P, _I, _P, _P, _P, _P, _P])
+_a2a_v = _sig("moedisp_a2a_v", [_P, _I64, _P, _I64, _I64, _I, _P, _P, _P, _P, _P])
+_ws_size = _sig("moedisp_layout_workspace_size", [Dims, ctypes.POINTER(ctypes.c_size_t)])
+_layout = _sig("moedisp_moe_dispatch_layout",
+               [_P, _P, Dims, ctypes.POINTER(Layout), _P, ctypes.c_size_t, _P, _P])
+_dispatch = _sig("moedisp_moe_dispatch",
+                 [_P, _I, Dims, ctypes.POINTER(Layout), _I, _P, _P, _P, _I, _P, _P, _P])
+_combine = _sig("moedisp_moe_combine", [_P, _I, Dims, ctypes.POINTER(Layout), _P, _P, _P, _P])
+
+
+class MoedispError(RuntimeError):
+    def __init__(self, code: int, call: str):
+        super().__init__(f"{call} failed: {status_string(code)} ({code})")
+        self.code = code
+
+
+def status_string(code: int) -> str:
+    return _status_string(int(code)).decode()
+
+
+def version() -> int:
+    return int(_version())
+
+
+def _ptr(t):
+    """Device pointer of a tensor (None stays NULL; ints pass through)."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(rc: int, call: str, raise_on_error: bool) -> int:
+    if rc < 0 and raise_on_error:
+        raise MoedispError(rc, call)
+    return rc
+
+
+# ------------------------------------------------------------------ exchange
+
+def a2a_exchange_plan(in_splits, src_offsets, out_splits, dst_offsets, status, W=None,
+                      stream=None, raise_on_error=True) -> int:
+    W = int(in_splits.shape[0]) if W is None else W
+    rc = _plan(_ptr(in_splits), W, _ptr(src_offsets), _ptr(out_splits), _ptr(dst_offsets),
+               _ptr(status), _stream(stream))
+    return _check(rc, "a2a_exchange_plan", raise_on_error)
+
+
+def a2a_v(inp, in_rank_stride_rows, out, out_cap_rows, row_bytes, W, src_offsets, out_splits,
+          dst_offsets, status, stream=None, raise_on_error=True) -> int:
+    rc = _a2a_v(_ptr(inp), int(in_rank_stride_rows), _ptr(out), int(out_cap_rows),
+                int(row_bytes), int(W), _ptr(src_offsets), _ptr(out_splits), _ptr(dst_offsets),
+                _ptr(status), _stream(stream))
+    return _check(rc, "a2a_v", raise_on_error)
+
+
+# -------------------------------------------------------------------- layout
+
+def layout_workspace_size(W: int, T: int, K: int, E: int) -> int:
+    n = ctypes.c_size_t(0)
+    rc = _ws_size(Dims(W, T, K, E), ctypes.byref(n))
+    _check(rc, "layout_workspace_size", True)
+    return int(n.value)
+
+
+@dataclass
+class LayoutBuffers:
+    """The caller-owned device buffers of one dispatch layout (allocated with torch)."""
+    W: int
+    T: int
+    K: int
+    E: int
+    rows_cap: int
+    cnt: object
+    occ: object
+    dst_row: object
+    assist_info: object
+    expert_base: object
+    rank_base: object
+    send_splits: object
+    workspace: object
+
+    @classmethod
+    def allocate(cls, W, T, K, E, rows_cap=None, device="cuda"):
+        import torch
+        G = W * T
+        rows_cap = G * K if rows_cap is None else rows_cap
+        z = dict(device=device)
+        return cls(W=W, T=T, K=K, E=E, rows_cap=rows_cap,
+                   cnt=torch.zeros((W, E), dtype=torch.int32, **z),
+                   occ=torch.zeros(G * K, dtype=torch.int32, **z),
+                   dst_row=torch.zeros(G * K, dtype=torch.int32, **z),
+                   assist_info=torch.zeros(max(rows_cap, 1), dtype=torch.int32, **z),
+                   expert_base=torch.zeros(E + 1, dtype=torch.int64, **z),
+                   rank_base=torch.zeros(W + 1, dtype=torch.int64, **z),
+                   send_splits=torch.zeros((W, W), dtype=torch.int64, **z),
+                   workspace=torch.zeros(layout_workspace_size(W, T, K, E), dtype=torch.uint8, **z))
+
+    @property
+    def dims(self) -> Dims:
+        return Dims(self.W, self.T, self.K, self.E)
+
+    def struct(self) -> Layout:
+        return Layout(_ptr(self.cnt), _ptr(self.occ), _ptr(self.dst_row), _ptr(self.assist_info),
+                      _ptr(self.expert_base), _ptr(self.rank_base), _ptr(self.send_splits),
+                      int(self.rows_cap))
+
+
+def moe_dispatch_layout(expert_ids, active_mask, layout: LayoutBuffers, status, stream=None,
+                        raise_on_error=True, workspace=None, workspace_bytes=None) -> int:
+    ws = layout.workspace if workspace is None else workspace
+    nbytes = (ws.numel() * ws.element_size()) if workspace_bytes is None else workspace_bytes
+    L = layout.struct()
+    rc = _layout(_ptr(expert_ids), _ptr(active_mask), layout.dims, ctypes.byref(L), _ptr(ws),
+                 int(nbytes), _ptr(status), _stream(stream))
+    return _check(rc, "moe_dispatch_layout", raise_on_error)
+
+
+def moe_dispatch(x, H, layout: LayoutBuffers, quant_mode, expand_x, dynamic_scales, status,
+                 expert_token_nums=None, expert_token_nums_type=1, ep_recv_counts=None,
+                 stream=None, raise_on_error=True) -> int:
+    L = layout.struct()
+    rc = _dispatch(_ptr(x), int(H), layout.dims, ctypes.byref(L), int(quant_mode), _ptr(expand_x),
+                   _ptr(dynamic_scales), _ptr(expert_token_nums), int(expert_token_nums_type),
+                   _ptr(ep_recv_counts), _ptr(status), _stream(stream))
+    return _check(rc, "moe_dispatch", raise_on_error)
+
+
+def moe_combine(expert_out, H, layout: LayoutBuffers, expert_scales, y, status, stream=None,
+                raise_on_error=True) -> int:
+    L = layout.struct()
+    rc = _combine(_ptr(expert_out), int(H), layout.dims, ctypes.byref(L), _ptr(expert_scales),
+                  _ptr(y), _ptr(status), _stream(stream))
+    return _check(rc, "moe_combine", raise_on_error)
+
+
+def raw_call(name: str, *args) -> int:
+    """Calls an exported C function with already-marshalled arguments (for ABI tests)."""
+    return int({"moedisp_a2a_exchange_plan": _plan, "moedisp_a2a_v": _a2a_v,
+                "moedisp_moe_dispatch_layout": _layout, "moedisp_moe_dispatch": _dispatch,
+                "moedisp_moe_combine": _combine}[name](*args))
+
+
+__all__ = [
+    "a2a_exchange_plan", "a2a_v", "layout_workspace_size", "LayoutBuffers",
+    "moe_dispatch_layout", "moe_dispatch", "moe_combine", "status_string", "version",
+    "Dims", "Layout", "MoedispError", "LIBRARY_PATH",
+    "QUANT_NONE", "QUANT_INT8", "QUANT_FP8_E4M3",
+    "STATUS_CAPACITY", "STATUS_BAD_EXPERT_ID", "STATUS_TIMEOUT", "STATUS_BAD_SPLIT",
+]

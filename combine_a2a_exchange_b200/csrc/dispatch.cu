@@ -1,0 +1,302 @@
+// MoE dispatch copy: every token row goes to the K rows its active slots were given by
+// the layout, optionally quantised per token (int8 or fp8-e4m3, dynamic scale).
+//
+// The PyTorch symm_mem index push sends one row per (token, expert) with a remote put
+// from the source buffer. On one GPU the K destinations are rows of one expand_x buffer,
+// so each token row is read from HBM exactly once: a persistent block brings the row
+// into shared memory with a 1-D bulk (TMA) load, quantises it there if asked, and the
+// K copies leave shared memory as K bulk stores issued by K lanes in parallel. Warp 0
+// runs the pipeline: it looks ahead through its tokens (skipping tokens with no active
+// slot), keeps up to kStages-1 row loads in flight, and reuses a stage only after the
+// bulk stores that read it have drained.
+#include "common.cuh"
+#include "kernels.h"
+
+#include <algorithm>
+
+namespace moedisp {
+
+namespace {
+constexpr int kMaxStages = 8;
+
+struct DispatchArgs {
+    const uint8_t* x;
+    int64_t G;
+    int K, H;
+    const int32_t* dst_row;
+    int64_t rows_cap;
+    uint8_t* expand_x;
+    float* scales;
+    int stages;
+    uint32_t in_bytes, out_bytes;
+    // receive counts (optional)
+    const int32_t* cnt;
+    const int64_t* expert_base;
+    const int64_t* rank_base;
+    int W, E, ne;
+    int64_t* etn;
+    int etn_type;
+    int32_t* erc;
+    int32_t* status;
+};
+
+template <int Q>
+struct Threads {
+    static constexpr int value = Q == MOEDISP_QUANT_NONE ? 32 : 256;
+};
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ float absmax8(const uint4& v) {
+    float m = fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x)));
+    m = fmaxf(m, fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y))));
+    m = fmaxf(m, fmaxf(fabsf(bf16_lo(v.z)), fabsf(bf16_hi(v.z))));
+    m = fmaxf(m, fmaxf(fabsf(bf16_lo(v.w)), fabsf(bf16_hi(v.w))));
+    return m;
+}
+
+// q = clamp(rint(x / scale), -127, 127), x / scale an IEEE fp32 divide.
+__device__ __forceinline__ uint32_t q_int8_pair(uint32_t w, float scale) {
+    int a = __float2int_rn(__fdiv_rn(bf16_lo(w), scale));
+    int b = __float2int_rn(__fdiv_rn(bf16_hi(w), scale));
+    a = max(-127, min(127, a));
+    b = max(-127, min(127, b));
+    return (uint32_t)(a & 0xff) | ((uint32_t)(b & 0xff) << 8);
+}
+
+// e4m3(x / scale), round to nearest even, saturating to +-448 (hardware conversion).
+__device__ __forceinline__ uint32_t q_e4m3_pair(uint32_t w, float scale) {
+    const float2 f = make_float2(__fdiv_rn(bf16_lo(w), scale), __fdiv_rn(bf16_hi(w), scale));
+    return (uint32_t)__nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3);
+}
+
+template <int Q>
+__device__ __forceinline__ uint2 quant8(const uint4& v, float scale, bool zero) {
+    if (zero) return make_uint2(0u, 0u);
+    uint32_t p0, p1, p2, p3;
+    if (Q == MOEDISP_QUANT_INT8) {
+        p0 = q_int8_pair(v.x, scale); p1 = q_int8_pair(v.y, scale);
+        p2 = q_int8_pair(v.z, scale); p3 = q_int8_pair(v.w, scale);
+    } else {
+        p0 = q_e4m3_pair(v.x, scale); p1 = q_e4m3_pair(v.y, scale);
+        p2 = q_e4m3_pair(v.z, scale); p3 = q_e4m3_pair(v.w, scale);
+    }
+    return make_uint2(p0 | (p1 << 16), p2 | (p3 << 16));
+}
+
+__device__ void write_recv_counts(const DispatchArgs& a) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t first = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (a.erc != nullptr) {
+        const int64_t n = (int64_t)a.W * a.ne * a.W;
+        for (int64_t idx = first; idx < n; idx += stride) {
+            const int64_t e = idx / a.W;                  // = d*ne + le
+            const int r = (int)(idx - e * a.W);
+            a.erc[idx] = a.cnt[(int64_t)r * a.E + e];
+        }
+    }
+    if (a.etn != nullptr) {
+        for (int64_t e = first; e < a.E; e += stride) {
+            const int d = (int)(e / a.ne);
+            a.etn[e] = a.etn_type == 0 ? a.expert_base[e + 1] - a.rank_base[d]
+                                       : a.expert_base[e + 1] - a.expert_base[e];
+        }
+    }
+}
+
+template <int Q>
+__global__ void __launch_bounds__(Threads<Q>::value) dispatch_kernel(DispatchArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ __align__(8) uint64_t bars[kMaxStages];
+    __shared__ int64_t tok[kMaxStages];
+    __shared__ int32_t drow[kMaxStages][MOEDISP_MAX_K];
+    __shared__ float red[8];
+    __shared__ int ok_s[2];
+    constexpr int NT = Threads<Q>::value;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int S = a.stages, K = a.K;
+    uint8_t* inbuf = smem;
+    uint8_t* outbuf = smem + (size_t)S * a.in_bytes;
+
+    write_recv_counts(a);
+
+    if (tid == 0) {
+        for (int s = 0; s < S; ++s) mbar_init(&bars[s], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    int64_t next_g = blockIdx.x;     // warp 0's look-ahead cursor over this block's tokens
+    // Warp 0: arm stage `st` with the next token that has an active slot (or the end).
+    auto fill = [&](int st) {
+        while (true) {
+            if (next_g >= a.G) {
+                if (lane == 0) {
+                    tok[st] = -1;
+                    mbar_arrive(&bars[st]);
+                }
+                return;
+            }
+            int32_t d = -1;
+            if (lane < K) {
+                d = __ldg(a.dst_row + next_g * K + lane);
+                if (d >= a.rows_cap) {
+                    raise_status(a.status, MOEDISP_STATUS_CAPACITY);
+                    d = -1;
+                }
+                if (d < 0) d = -1;
+            }
+            const unsigned any = __ballot_sync(0xffffffffu, d >= 0);
+            if (any) {
+                int32_t dk[MOEDISP_MAX_K];
+#pragma unroll
+                for (int k = 0; k < MOEDISP_MAX_K; ++k) dk[k] = __shfl_sync(0xffffffffu, d, k);
+                if (lane == 0) {
+#pragma unroll
+                    for (int k = 0; k < MOEDISP_MAX_K; ++k)
+                        if (k < K) drow[st][k] = dk[k];
+                    tok[st] = next_g;
+                    mbar_arrive_expect_tx(&bars[st], a.in_bytes);
+                    bulk_load(inbuf + (size_t)st * a.in_bytes, a.x + next_g * a.in_bytes, a.in_bytes,
+                              &bars[st]);
+                }
+                next_g += gridDim.x;
+                return;
+            }
+            next_g += gridDim.x;
+        }
+    };
+
+    if (warp == 0)
+        for (int st = 0; st < S; ++st) fill(st);
+
+    const bool issuer = warp == 0 && lane < K;
+    for (int it = 0;; ++it) {
+        const int st = it % S;
+        const uint32_t par = (uint32_t)((it / S) & 1);
+        // One thread waits with a time limit and shares the verdict (double-buffered: a
+        // thread can lag by at most one iteration); then every thread observes the
+        // already completed phase itself.
+        if (tid == 0) ok_s[it & 1] = mbar_wait(&bars[st], par) ? 1 : 0;
+        __syncthreads();
+        if (!ok_s[it & 1]) {
+            if (tid == 0) raise_status(a.status, MOEDISP_STATUS_TIMEOUT);
+            break;
+        }
+        (void)mbar_wait(&bars[st], par);
+        const int64_t g = tok[st];
+        if (g < 0) break;
+        const uint8_t* row_in = inbuf + (size_t)st * a.in_bytes;
+
+        if constexpr (Q == MOEDISP_QUANT_NONE) {
+            if (issuer) {
+                const int32_t d = drow[st][lane];
+                if (d >= 0) bulk_store(a.expand_x + (int64_t)d * a.out_bytes, row_in, a.in_bytes);
+                bulk_commit();
+            }
+            if (it >= 1) {
+                if (issuer) bulk_wait_read<1>();
+                __syncwarp();
+                fill((it - 1) % S);
+            }
+        } else {
+            constexpr float kQmax = Q == MOEDISP_QUANT_INT8 ? 127.0f : 448.0f;
+            const uint4* v = reinterpret_cast<const uint4*>(row_in);
+            const int nvec = a.H >> 3;
+            float m = 0.0f;
+            for (int c = tid; c < nvec; c += NT) m = fmaxf(m, absmax8(v[c]));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            if (lane == 0) red[warp] = m;
+            if (issuer) bulk_wait_read<1>();      // output buffer it % 2 is free again
+            __syncthreads();
+            float amax = red[0];
+#pragma unroll
+            for (int w = 1; w < NT / 32; ++w) amax = fmaxf(amax, red[w]);
+            const float scale = __fdiv_rn(amax, kQmax);
+            const bool zero = amax == 0.0f;
+            uint8_t* ob = outbuf + (size_t)(it & 1) * a.out_bytes;
+            uint2* o2 = reinterpret_cast<uint2*>(ob);
+            for (int c = tid; c < nvec; c += NT) o2[c] = quant8<Q>(v[c], scale, zero);
+            fence_proxy_async_smem();
+            __syncthreads();
+            if (warp == 0) {
+                if (issuer) {
+                    const int32_t d = drow[st][lane];
+                    if (d >= 0) {
+                        bulk_store(a.expand_x + (int64_t)d * a.out_bytes, ob, a.out_bytes);
+                        a.scales[d] = scale;
+                    }
+                    bulk_commit();
+                }
+                __syncwarp();
+                fill(st);                           // every thread is done reading stage st
+            }
+        }
+    }
+    if (issuer) bulk_wait<0>();
+}
+
+template <int Q>
+cudaError_t launch_q(const DispatchArgs& a0, cudaStream_t stream) {
+    DispatchArgs a = a0;
+    constexpr int NT = Threads<Q>::value;
+    const size_t budget = Q == MOEDISP_QUANT_NONE ? 64 * 1024 : 96 * 1024;
+    const size_t per_stage = a.in_bytes;
+    const size_t fixed = Q == MOEDISP_QUANT_NONE ? 0 : 2 * (size_t)a.out_bytes;
+    int S = (int)std::min<size_t>(kMaxStages, (budget - std::min(budget, fixed)) / per_stage);
+    S = std::max(S, 2);
+    a.stages = S;
+    const size_t smem = (size_t)S * per_stage + fixed;
+    cudaError_t err = cudaFuncSetAttribute(dispatch_kernel<Q>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    int per_sm = 1;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dispatch_kernel<Q>, NT, smem);
+    if (err != cudaSuccess) return err;
+    per_sm = std::max(per_sm, 1);
+    int64_t grid = (int64_t)current_sm_count() * per_sm;
+    grid = std::min<int64_t>(grid, std::max<int64_t>(a.G, 1));
+    dispatch_kernel<Q><<<(unsigned)grid, NT, smem, stream>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch(const void* x, int H, const moedisp_dims& dims,
+                            const moedisp_layout& L, int quant_mode, void* expand_x,
+                            float* dynamic_scales, int64_t* expert_token_nums,
+                            int expert_token_nums_type, int32_t* ep_recv_counts,
+                            int32_t* status, cudaStream_t stream) {
+    DispatchArgs a;
+    a.x = static_cast<const uint8_t*>(x);
+    a.G = (int64_t)dims.W * dims.T;
+    a.K = dims.K;
+    a.H = H;
+    a.dst_row = L.dst_row;
+    a.rows_cap = L.rows_cap;
+    a.expand_x = static_cast<uint8_t*>(expand_x);
+    a.scales = dynamic_scales;
+    a.stages = 2;
+    a.in_bytes = (uint32_t)H * 2u;
+    a.out_bytes = quant_mode == MOEDISP_QUANT_NONE ? (uint32_t)H * 2u : (uint32_t)H;
+    a.cnt = L.cnt;
+    a.expert_base = L.expert_base;
+    a.rank_base = L.rank_base;
+    a.W = dims.W;
+    a.E = dims.E;
+    a.ne = dims.E / dims.W;
+    a.etn = expert_token_nums;
+    a.etn_type = expert_token_nums_type;
+    a.erc = ep_recv_counts;
+    a.status = status;
+    switch (quant_mode) {
+        case MOEDISP_QUANT_NONE: return launch_q<MOEDISP_QUANT_NONE>(a, stream);
+        case MOEDISP_QUANT_INT8: return launch_q<MOEDISP_QUANT_INT8>(a, stream);
+        case MOEDISP_QUANT_FP8_E4M3: return launch_q<MOEDISP_QUANT_FP8_E4M3>(a, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace moedisp

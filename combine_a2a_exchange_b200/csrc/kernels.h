@@ -1,0 +1,47 @@
+// Internal host-side launchers of libmoedisp (called by abi.cu after validation).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "moedisp.h"
+
+namespace moedisp {
+
+// Streaming-multiprocessor count of the current device (cached per device).
+int current_sm_count();
+
+cudaError_t launch_a2a_plan(const int64_t* in_splits, int W, int64_t* src_offsets,
+                            int64_t* out_splits, int64_t* dst_offsets, int32_t* status,
+                            cudaStream_t stream);
+
+cudaError_t launch_a2a_v(const void* in, int64_t in_rank_stride_rows, void* out,
+                         int64_t out_cap_rows, int64_t row_bytes, int W,
+                         const int64_t* src_offsets, const int64_t* out_splits,
+                         const int64_t* dst_offsets, int32_t* status, cudaStream_t stream);
+
+// Layout tiling, shared by the workspace-size query and the launcher.
+struct LayoutGeometry {
+    int64_t slots_per_rank;   // T*K
+    int tiles_per_rank;
+    int64_t n_tiles;
+    size_t off_tile_hist, off_lookback, off_colprefix, total_bytes;
+};
+LayoutGeometry layout_geometry(const moedisp_dims& d);
+
+cudaError_t launch_layout(const int32_t* expert_ids, const uint8_t* active,
+                          const moedisp_dims& dims, const moedisp_layout& layout,
+                          void* workspace, int32_t* status, cudaStream_t stream);
+
+cudaError_t launch_dispatch(const void* x, int H, const moedisp_dims& dims,
+                            const moedisp_layout& layout, int quant_mode, void* expand_x,
+                            float* dynamic_scales, int64_t* expert_token_nums,
+                            int expert_token_nums_type, int32_t* ep_recv_counts,
+                            int32_t* status, cudaStream_t stream);
+
+cudaError_t launch_combine(const void* expert_out, int H, const moedisp_dims& dims,
+                           const moedisp_layout& layout, const float* expert_scales, void* y,
+                           int32_t* status, cudaStream_t stream);
+
+}  // namespace moedisp

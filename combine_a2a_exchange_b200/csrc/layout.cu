@@ -1,0 +1,367 @@
+// MoE dispatch layout: a stable counting sort of the G*K (token, expert) slots by expert.
+//
+// The PyTorch symm_mem change computes the same thing in three separate pieces: a
+// per-rank histogram of the top-k ids (torch.histc), the 0-based occurrence number of
+// every slot (get_occurrence_numbers, an n_unique x n indicator matrix and a cumsum) and
+// a one-block 2-D exchange plan (make2dExchangePlan) whose per-expert destination offsets
+// the index-push kernel adds to the occurrence number. Here one pass does all of it:
+//
+//  kernel 1 (layout_hist_kernel): slots are cut into tiles of kTile slots that never
+//    straddle a source rank. Each block counts its tile per expert with a
+//    warp-aggregated shared-memory histogram (__match_any_sync groups the lanes that
+//    share an expert; the group's lowest lane adds the group size), writes the tile's
+//    counts and clears the tile's look-back words. The last block to finish (atomic
+//    ticket after a fence) reduces the tiles to cnt[r][e], scans over source ranks
+//    (colprefix) and over experts (expert_base, rank_base), and forms send_splits.
+//  kernel 2 (layout_scatter_kernel): blocks take tiles in ticket order. Each warp ranks
+//    its part of the tile with __match_any_sync + popcount of the lower peers, on top of
+//    a per-warp running count; the warps' counts are scanned per expert; the tile's
+//    per-expert offset among all earlier tiles comes from a decoupled look-back (each
+//    tile publishes its aggregate, then walks back over predecessors' status words in
+//    windows of kWindow until it meets an inclusive prefix); finally every slot is
+//    scattered: dst_row, occ and assist_info.
+#include "common.cuh"
+#include "kernels.h"
+
+#include <algorithm>
+
+namespace moedisp {
+
+namespace {
+constexpr int kTile = 2048;
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kSlotsPerWarp = kTile / kWarps;
+constexpr int kSteps = kSlotsPerWarp / 32;
+constexpr int kWindow = 16;
+constexpr uint32_t kFlagAggregate = 1u << 30;
+constexpr uint32_t kFlagInclusive = 2u << 30;
+constexpr uint32_t kValueMask = (1u << 30) - 1;
+// Shared memory that kernel 1's last block may use to hold cnt while it scans.
+constexpr size_t kFinalizeSmemLimit = 160 * 1024;
+
+struct LayoutArgs {
+    const int32_t* ids;
+    const uint8_t* active;
+    int W, T, K, E, ne;
+    int64_t P;                 // slots per source rank, T*K
+    int tiles_per_rank;
+    int n_tiles;
+    int cnt_in_smem;
+    int32_t* cnt;
+    int32_t* occ;
+    int32_t* dst_row;
+    int32_t* assist;
+    int64_t* expert_base;
+    int64_t* rank_base;
+    int64_t* send_splits;
+    int64_t rows_cap;
+    uint32_t* counters;        // [0] blocks done in kernel 1, [1] tile ticket of kernel 2
+    int32_t* tile_hist;        // [n_tiles][E]
+    uint32_t* lookback;        // [n_tiles][E]
+    int32_t* colprefix;        // [W][E] slots of expert e in source ranks < r
+    int32_t* status;
+};
+
+__device__ __forceinline__ void st_relaxed(uint32_t* p, uint32_t v) {
+    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_relaxed(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Expert of slot s if the slot is active, else -1. `bad` is set for an active token's
+// out-of-range id.
+__device__ __forceinline__ int slot_expert(const LayoutArgs& a, int64_t s, bool& bad) {
+    const int e = __ldg(a.ids + s);
+    if (a.active != nullptr && __ldg(a.active + s / a.K) == 0) return -1;
+    if (e < 0 || e >= a.E) {
+        bad = true;
+        return -1;
+    }
+    return e;
+}
+
+__device__ void layout_finalize(const LayoutArgs& a, int32_t* smem) {
+    __shared__ int64_t warp_tot[32];
+    const int W = a.W, E = a.E, tpr = a.tiles_per_rank;
+    int64_t* ebase = reinterpret_cast<int64_t*>(smem);            // [E + 1]
+    int32_t* cnt_s = reinterpret_cast<int32_t*>(ebase + E + 1);   // [W * E] if it fits
+    int32_t* cnt_src = a.cnt_in_smem ? cnt_s : a.cnt;
+
+    // cnt[r][e]: sum of the tile counts of rank r.
+    for (int idx = threadIdx.x; idx < W * E; idx += blockDim.x) {
+        const int r = idx / E, e = idx - r * E;
+        const int32_t* th = a.tile_hist + (int64_t)r * tpr * E + e;
+        int32_t sum = 0;
+#pragma unroll 8
+        for (int c = 0; c < tpr; ++c) sum += __ldcg(th + (int64_t)c * E);
+        a.cnt[idx] = sum;
+        if (a.cnt_in_smem) cnt_s[idx] = sum;
+    }
+    __syncthreads();
+    // Per expert: prefix over source ranks, total; then exclusive scan over experts.
+    int64_t carry = 0;
+    for (int base = 0; base < E; base += blockDim.x) {
+        const int e = base + threadIdx.x;
+        int64_t tot = 0;
+        if (e < E) {
+            for (int r = 0; r < W; ++r) {
+                a.colprefix[(int64_t)r * E + e] = (int32_t)tot;
+                tot += a.cnt_in_smem ? cnt_s[r * E + e] : __ldcg(cnt_src + (int64_t)r * E + e);
+            }
+        }
+        int64_t chunk;
+        const int64_t ex = block_exclusive_scan(tot, warp_tot, chunk);
+        if (e < E) ebase[e] = carry + ex;
+        carry += chunk;
+    }
+    if (threadIdx.x == 0) ebase[E] = carry;
+    __syncthreads();
+    const int64_t R = ebase[E];
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) a.expert_base[e] = ebase[e];
+    for (int d = threadIdx.x; d <= W; d += blockDim.x) a.rank_base[d] = d < W ? ebase[d * a.ne] : R;
+    for (int idx = threadIdx.x; idx < W * W; idx += blockDim.x) {
+        const int r = idx / W, d = idx - r * W;
+        int64_t sum = 0;
+        for (int le = 0; le < a.ne; ++le) {
+            const int e = d * a.ne + le;
+            sum += a.cnt_in_smem ? cnt_s[r * E + e] : __ldcg(cnt_src + (int64_t)r * E + e);
+        }
+        a.send_splits[idx] = sum;
+    }
+    if (threadIdx.x == 0) {
+        if (R > a.rows_cap) raise_status(a.status, MOEDISP_STATUS_CAPACITY);
+        a.counters[0] = 0;   // ready for the next call
+        a.counters[1] = 0;   // tile ticket of kernel 2
+    }
+}
+
+__global__ void __launch_bounds__(kThreads) layout_hist_kernel(LayoutArgs a) {
+    extern __shared__ __align__(16) int32_t smem[];
+    __shared__ int is_last;
+    const int tile = blockIdx.x;
+    const int r = tile / a.tiles_per_rank, c = tile - r * a.tiles_per_rank;
+    const int64_t base = (int64_t)r * a.P;
+    const int64_t lo = (int64_t)c * kTile, hi = min64(lo + kTile, a.P);
+    const int lane = threadIdx.x & 31;
+
+    int32_t* hist = smem;
+    for (int e = threadIdx.x; e < a.E; e += blockDim.x) hist[e] = 0;
+    __syncthreads();
+    bool bad = false;
+    for (int64_t l0 = lo; l0 < hi; l0 += blockDim.x) {
+        const int64_t l = l0 + threadIdx.x;
+        const int e = l < hi ? slot_expert(a, base + l, bad) : -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        if (e >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[e], __popc(peers));
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) raise_status(a.status, MOEDISP_STATUS_BAD_EXPERT_ID);
+    __syncthreads();
+    int32_t* th = a.tile_hist + (int64_t)tile * a.E;
+    uint32_t* lb = a.lookback + (int64_t)tile * a.E;
+    for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+        th[e] = hist[e];
+        lb[e] = 0;
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) is_last = atomicAdd(&a.counters[0], 1u) == (unsigned)(a.n_tiles - 1);
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    layout_finalize(a, smem);
+}
+
+__global__ void __launch_bounds__(kThreads) layout_scatter_kernel(LayoutArgs a) {
+    extern __shared__ __align__(16) int32_t smem[];
+    __shared__ int tile_s;
+    const int E = a.E;
+    int32_t* warp_cnt = smem;                    // [kWarps][E]
+    int32_t* tile_off = smem + kWarps * E;       // [E]
+    if (threadIdx.x == 0) tile_s = (int)atomicAdd(&a.counters[1], 1u);
+    for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) warp_cnt[i] = 0;
+    __syncthreads();
+    const int tile = tile_s;
+    const int r = tile / a.tiles_per_rank, c = tile - r * a.tiles_per_rank;
+    const int64_t base = (int64_t)r * a.P;
+    const int64_t lo = (int64_t)c * kTile, hi = min64(lo + kTile, a.P);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const unsigned lower = (1u << lane) - 1u;
+    int32_t* mine = warp_cnt + warp * E;
+    const int64_t wlo = lo + (int64_t)warp * kSlotsPerWarp;
+
+    int ev[kSteps];
+    int rk[kSteps];
+    bool bad = false;
+#pragma unroll
+    for (int st = 0; st < kSteps; ++st) {
+        const int64_t l = wlo + st * 32 + lane;
+        ev[st] = l < hi ? slot_expert(a, base + l, bad) : -1;
+    }
+    // Rank within the warp's part, in slot order, on top of the warp's running counts.
+#pragma unroll
+    for (int st = 0; st < kSteps; ++st) {
+        const int e = ev[st];
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        const int before = e >= 0 ? mine[e] : 0;
+        __syncwarp();
+        if (e >= 0 && lane == __ffs(peers) - 1) mine[e] = before + __popc(peers);
+        __syncwarp();
+        rk[st] = before + __popc(peers & lower);
+    }
+    __syncthreads();
+    // Exclusive scan of the warps' counts per expert; the tile's count per expert.
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int32_t run = 0;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            const int32_t t = warp_cnt[w * E + e];
+            warp_cnt[w * E + e] = run;
+            run += t;
+        }
+        tile_off[e] = run;
+    }
+    __syncthreads();
+    // Decoupled look-back: the number of slots of expert e in all earlier tiles.
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        const uint32_t count = (uint32_t)tile_off[e];
+        uint32_t* my_word = a.lookback + (int64_t)tile * E + e;
+        uint32_t excl = 0;
+        if (tile == 0) {
+            st_relaxed(my_word, kFlagInclusive | count);
+        } else {
+            st_relaxed(my_word, kFlagAggregate | count);
+            int p = tile - 1;
+            uint64_t t0 = 0;
+            while (p >= 0) {
+                const int n = min(kWindow, p + 1);
+                uint32_t w[kWindow];
+#pragma unroll
+                for (int i = 0; i < kWindow; ++i)
+                    w[i] = i < n ? ld_relaxed(a.lookback + (int64_t)(p - i) * E + e) : 0u;
+                int used = 0;
+                bool stop = false, found = false;
+#pragma unroll
+                for (int i = 0; i < kWindow; ++i) {
+                    if (!stop && i < n) {
+                        const uint32_t f = w[i] & ~kValueMask;
+                        if (f == 0) {
+                            stop = true;
+                        } else {
+                            excl += w[i] & kValueMask;
+                            used = i + 1;
+                            if (f == kFlagInclusive) found = stop = true;
+                        }
+                    }
+                }
+                if (found) break;
+                p -= used;
+                if (used < n) {           // predecessor p has not published yet
+                    const uint64_t now = global_timer_ns();
+                    if (t0 == 0) t0 = now;
+                    else if (now - t0 > kWaitLimitNs) {
+                        raise_status(a.status, MOEDISP_STATUS_TIMEOUT);
+                        break;
+                    }
+                    __nanosleep(64);
+                }
+            }
+            st_relaxed(my_word, kFlagInclusive | ((excl + count) & kValueMask));
+        }
+        tile_off[e] = (int32_t)excl;
+    }
+    __syncthreads();
+    // Stable scatter.
+    const int32_t* colp = a.colprefix + (int64_t)r * E;
+#pragma unroll
+    for (int st = 0; st < kSteps; ++st) {
+        const int64_t l = wlo + st * 32 + lane;
+        if (l >= hi) continue;
+        const int64_t s = base + l;
+        const int e = ev[st];
+        if (e < 0) {
+            a.dst_row[s] = -1;
+            a.occ[s] = -1;
+            continue;
+        }
+        const int32_t within = tile_off[e] + mine[e] + rk[st];   // earlier slots of e, all ranks
+        const int64_t row = __ldg(a.expert_base + e) + within;
+        a.occ[s] = within - __ldg(colp + e);
+        a.dst_row[s] = (int32_t)row;
+        if (row < a.rows_cap) a.assist[row] = (int32_t)s;
+    }
+}
+
+}  // namespace
+
+LayoutGeometry layout_geometry(const moedisp_dims& d) {
+    LayoutGeometry g{};
+    g.slots_per_rank = (int64_t)d.T * d.K;
+    g.tiles_per_rank = (int)std::max<int64_t>(1, (g.slots_per_rank + kTile - 1) / kTile);
+    g.n_tiles = (int64_t)d.W * g.tiles_per_rank;
+    auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    size_t off = 256;                                       // counters
+    g.off_tile_hist = off;
+    off += al((size_t)g.n_tiles * d.E * sizeof(int32_t));
+    g.off_lookback = off;
+    off += al((size_t)g.n_tiles * d.E * sizeof(uint32_t));
+    g.off_colprefix = off;
+    off += al((size_t)d.W * d.E * sizeof(int32_t));
+    g.total_bytes = off;
+    return g;
+}
+
+cudaError_t launch_layout(const int32_t* expert_ids, const uint8_t* active,
+                          const moedisp_dims& dims, const moedisp_layout& L, void* workspace,
+                          int32_t* status, cudaStream_t stream) {
+    const LayoutGeometry g = layout_geometry(dims);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    LayoutArgs a;
+    a.ids = expert_ids;
+    a.active = active;
+    a.W = dims.W;
+    a.T = dims.T;
+    a.K = dims.K;
+    a.E = dims.E;
+    a.ne = dims.E / dims.W;
+    a.P = g.slots_per_rank;
+    a.tiles_per_rank = g.tiles_per_rank;
+    a.n_tiles = (int)g.n_tiles;
+    a.cnt = L.cnt;
+    a.occ = L.occ;
+    a.dst_row = L.dst_row;
+    a.assist = L.assist_info;
+    a.expert_base = L.expert_base;
+    a.rank_base = L.rank_base;
+    a.send_splits = L.send_splits;
+    a.rows_cap = L.rows_cap;
+    a.counters = reinterpret_cast<uint32_t*>(ws);
+    a.tile_hist = reinterpret_cast<int32_t*>(ws + g.off_tile_hist);
+    a.lookback = reinterpret_cast<uint32_t*>(ws + g.off_lookback);
+    a.colprefix = reinterpret_cast<int32_t*>(ws + g.off_colprefix);
+    a.status = status;
+
+    const size_t fin_base = (size_t)(dims.E + 1) * sizeof(int64_t);
+    const size_t fin_cnt = (size_t)dims.W * dims.E * sizeof(int32_t);
+    a.cnt_in_smem = fin_base + fin_cnt <= kFinalizeSmemLimit;
+    size_t smem1 = std::max((size_t)dims.E * sizeof(int32_t), fin_base + (a.cnt_in_smem ? fin_cnt : 0));
+    smem1 = (smem1 + 15) & ~(size_t)15;
+    const size_t smem2 = (size_t)(kWarps + 1) * dims.E * sizeof(int32_t);
+
+    cudaError_t err = cudaFuncSetAttribute(layout_hist_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
+    if (err != cudaSuccess) return err;
+    err = cudaFuncSetAttribute(layout_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem2);
+    if (err != cudaSuccess) return err;
+    layout_hist_kernel<<<(unsigned)g.n_tiles, kThreads, smem1, stream>>>(a);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    layout_scatter_kernel<<<(unsigned)g.n_tiles, kThreads, smem2, stream>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace moedisp

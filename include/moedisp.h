@@ -1,0 +1,220 @@
+/*
+ * moedisp.h -- C ABI of libmoedisp: expert-parallel (EP) MoE token dispatch / combine
+ * and the uneven all-to-all-v exchange, for NVIDIA B200 (sm_100a).
+ *
+ * The W EP ranks of the exchange are "virtual ranks": slices of one GPU's memory.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Ownership: the caller allocates and owns every buffer. All pointers named
+ *    "device" point to device memory of the current CUDA device. The library never
+ *    allocates, frees or synchronises; each call validates its arguments on the host,
+ *    enqueues its kernels on `stream` and returns.
+ *  - Host-detected errors return a negative MOEDISP_ERR_* code and enqueue nothing.
+ *  - Device-detected errors are OR-ed into `*status` (an int32 in device memory that the
+ *    caller zeroes) as MOEDISP_STATUS_* bits; read it after the stream completes. No
+ *    kernel traps, asserts or waits without bound: every device-side wait gives up after
+ *    about two seconds and sets MOEDISP_STATUS_TIMEOUT.
+ *  - Empty inputs (no rows, no tokens, all splits 0) are valid no-ops.
+ *  - Integer, index, copy and quantisation outputs are deterministic and bit-exact
+ *    against a plain CPU implementation; combine sums each token's K rows in fp32 in
+ *    ascending k with fused multiply-adds, so it is deterministic too.
+ *
+ * Notation: W ranks, T tokens per rank, G = W*T global tokens (token g = r*T + t lives on
+ * source rank r), K experts per token, E experts, ne = E/W experts per rank,
+ * owner(e) = e / ne. Slot s = g*K + k is the k-th expert choice of token g.
+ */
+#ifndef MOEDISP_H
+#define MOEDISP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream (cudaStream_t); NULL is the legacy default stream. */
+typedef struct CUstream_st *moedisp_stream_t;
+
+/* Host-side return codes. The error classes follow the status-code convention of the
+ * Ascend aclnnMoeDistributeDispatchV2 API (Returns: null pointer, invalid parameter,
+ * unsupported shape or value). */
+#define MOEDISP_OK                0
+#define MOEDISP_ERR_NULLPTR      -1  /* a required pointer is NULL */
+#define MOEDISP_ERR_INVALID      -2  /* a size, count or mode is out of range */
+#define MOEDISP_ERR_MISALIGNED   -3  /* a pointer or row size breaks the 16-byte rule */
+#define MOEDISP_ERR_ALIASED      -4  /* an output overlaps an input or another output */
+#define MOEDISP_ERR_UNSUPPORTED  -5  /* valid but outside this build's limits */
+#define MOEDISP_ERR_WORKSPACE    -6  /* workspace missing or too small */
+#define MOEDISP_ERR_CUDA         -7  /* a CUDA runtime call or kernel launch failed */
+
+/* Device-side status bits (OR-ed into *status). */
+#define MOEDISP_STATUS_CAPACITY      1  /* rows beyond the receive capacity were dropped */
+#define MOEDISP_STATUS_BAD_EXPERT_ID 2  /* an active slot named an expert outside [0, E) */
+#define MOEDISP_STATUS_TIMEOUT       4  /* a bounded device-side wait gave up */
+#define MOEDISP_STATUS_BAD_SPLIT     8  /* a negative split or a segment outside its buffer */
+
+/* Limits of this build. */
+#define MOEDISP_MAX_K        16      /* Ascend dispatch: 0 < K <= 16 */
+#define MOEDISP_MAX_E        1024    /* Ascend A3: moeExpertNum <= 1024 */
+#define MOEDISP_MAX_H        16384   /* hidden size (elements) for dispatch staging */
+#define MOEDISP_MAX_W        65536   /* ranks of an exchange plan */
+
+/* Returns a static, human-readable name for a return code (< 0) or status bits (> 0). */
+const char *moedisp_status_string(int code);
+
+/* ABI version, currently 1. */
+int moedisp_version(void);
+
+/* ------------------------------------------------------------------------------------
+ * a2a_exchange_plan
+ *
+ * The all-to-all-v exchange plan of the PyTorch symm_mem change ("ExchangePlan" doc
+ * comment, make_a2a_exchange_plan, and the checks in test_make_a2a_exchange_plan), for
+ * all W virtual ranks at once. With S = in_splits (S[i][j] = rows rank i sends to j):
+ *     out_splits[i][j]  = S[j][i]                  rows rank i receives from j
+ *     src_offsets[i][j] = sum_{k<i} S[j][k]        where i's rows start in j's input
+ *     dst_offsets[i][j] = sum_{k<j} out_splits[i][k]   where j's rows land in i's output
+ * All five arrays are int64 [W][W], row-major, device memory; the three outputs must not
+ * overlap each other or in_splits. A negative split sets MOEDISP_STATUS_BAD_SPLIT (the
+ * outputs are then computed from the values as given). One kernel, W blocks.
+ * ---------------------------------------------------------------------------------- */
+int moedisp_a2a_exchange_plan(const int64_t *in_splits, int W, int64_t *src_offsets,
+                              int64_t *out_splits, int64_t *dst_offsets, int32_t *status,
+                              moedisp_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * a2a_v
+ *
+ * The uneven all-to-all-v row exchange driven by a plan (PyTorch symm_mem all_to_all_v,
+ * get style: rank i fetches its rows from each peer j), between W virtual ranks:
+ *     for every i, j and q < out_splits[i][j]:
+ *       out row (i*out_cap_rows + dst_offsets[i][j] + q) =
+ *       in  row (j*in_rank_stride_rows + src_offsets[i][j] + q)
+ * `in` holds W send buffers of in_rank_stride_rows rows each, `out` W receive buffers of
+ * out_cap_rows rows each; rows are `row_bytes` opaque bytes (the copy is dtype-agnostic).
+ * Output rows no segment covers are left untouched. A segment whose source or
+ * destination range leaves its rank's buffer (or has a negative size/offset) is skipped
+ * and sets MOEDISP_STATUS_BAD_SPLIT.
+ * Requirements: row_bytes > 0 and a multiple of 16; in and out 16-byte aligned and not
+ * overlapping; plan arrays int64 [W][W] device memory (e.g. from a2a_exchange_plan).
+ * ---------------------------------------------------------------------------------- */
+int moedisp_a2a_v(const void *in, int64_t in_rank_stride_rows, void *out,
+                  int64_t out_cap_rows, int64_t row_bytes, int W,
+                  const int64_t *src_offsets, const int64_t *out_splits,
+                  const int64_t *dst_offsets, int32_t *status, moedisp_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * MoE dispatch layout
+ * ---------------------------------------------------------------------------------- */
+typedef struct {
+    int W;   /* EP ranks, >= 1 */
+    int T;   /* tokens per rank, >= 0 */
+    int K;   /* experts per token, 1..MOEDISP_MAX_K */
+    int E;   /* experts, 1..MOEDISP_MAX_E, E % W == 0 */
+} moedisp_dims;
+
+/* Caller-owned device buffers that one moe_dispatch_layout call fills and that
+ * moe_dispatch / moe_combine read. */
+typedef struct {
+    int32_t *cnt;          /* [W][E]   active slots of source rank r choosing expert e   */
+    int32_t *occ;          /* [G*K]    0-based occurrence of slot s among the earlier
+                                       active slots of its source rank with its expert;
+                                       -1 for an inactive slot                           */
+    int32_t *dst_row;      /* [G*K]    row of expand_x that slot s is dispatched to; -1
+                                       for an inactive slot                              */
+    int32_t *assist_info;  /* [rows_cap] slot s = g*K + k that row r holds (r < R)        */
+    int64_t *expert_base;  /* [E+1]    first row of expert e; expert_base[E] = R         */
+    int64_t *rank_base;    /* [W+1]    first row of destination rank d; rank_base[W] = R */
+    int64_t *send_splits;  /* [W][W]   rows source rank r sends to destination rank d
+                                       (the in_splits of a 1-D exchange plan)            */
+    int64_t  rows_cap;     /* rows that expand_x / assist_info hold                       */
+} moedisp_layout;
+
+/* Bytes of device workspace moe_dispatch_layout needs for `dims`. */
+int moedisp_layout_workspace_size(moedisp_dims dims, size_t *bytes);
+
+/* moe_dispatch_layout
+ *
+ * Routes the G*K (token, expert) slots into an expert-grouped layout, following the
+ * PyTorch symm_mem 2-D exchange plan and index-push dispatch (get_occurrence_numbers,
+ * make2dExchangePlan, _allToAllV_2d_index_push_kernel) and the Ascend
+ * aclnnMoeDistributeDispatchV2 inputs (expertIds int32 [Bs][K], 1-D xActiveMask):
+ *   cnt[r][e]   = active slots of rank r with expert e (the 2-D plan's in_splits);
+ *   occ[s]      = earlier active slots of s's rank with s's expert (0-based);
+ *   rows of expand_x are ordered by destination rank, then local expert, then source
+ *   rank, then token, then k -- i.e. dst_row[s] is the position of s in a stable sort of
+ *   all active slots by expert id:
+ *     dst_row[s] = expert_base[e] + sum_{r' < r} cnt[r'][e] + occ[s];
+ *   assist_info[dst_row[s]] = s.
+ * expert_ids: int32 [G][K] device; active_mask: uint8 [G] device or NULL (all active; any
+ * pattern of active tokens is accepted). A slot is active when its token is active and
+ * its expert id lies in [0, E); an active token's out-of-range id sets
+ * MOEDISP_STATUS_BAD_EXPERT_ID and that slot is dropped. If R > rows_cap,
+ * MOEDISP_STATUS_CAPACITY is set, every output is still computed, and assist_info is
+ * written only below rows_cap.
+ * workspace: device memory of at least moedisp_layout_workspace_size() bytes, 16-byte
+ * aligned, ZERO-FILLED BEFORE ITS FIRST USE; every call leaves it ready for the next.
+ * Calls sharing one workspace must not run concurrently.
+ * Two kernels: a tiled, warp-aggregated histogram whose last block scans the counts,
+ * then a tiled ranking/scatter pass whose per-expert tile offsets come from a decoupled
+ * look-back over the tiles. */
+int moedisp_moe_dispatch_layout(const int32_t *expert_ids, const uint8_t *active_mask,
+                                moedisp_dims dims, const moedisp_layout *layout,
+                                void *workspace, size_t workspace_bytes, int32_t *status,
+                                moedisp_stream_t stream);
+
+/* Quantisation modes of moe_dispatch (the Ascend quantMode values; 3 is this library's
+ * fp8 variant of the same per-token dynamic scheme). */
+#define MOEDISP_QUANT_NONE      0
+#define MOEDISP_QUANT_INT8      2
+#define MOEDISP_QUANT_FP8_E4M3  3
+
+/* moe_dispatch
+ *
+ * Copies every token row to the rows its active slots were given by
+ * moe_dispatch_layout (Ascend expandXOut; PyTorch symm_mem index push), optionally
+ * quantised per token (Ascend quantMode 2, per-token dynamic):
+ *   NONE: expand_x[dst_row[s]] = x[g]                            (bf16, H*2 bytes/row)
+ *   INT8: a = max_h |x[g,h]|, scale = a / 127 (fp32, IEEE divide),
+ *         q = a == 0 ? 0 : clamp(rint(x / scale), -127, 127)     (int8, H bytes/row)
+ *   FP8_E4M3: scale = a / 448, q = a == 0 ? 0 : e4m3(x / scale), round to nearest even,
+ *         saturating to +-448                                    (e4m3, H bytes/row)
+ *   dynamic_scales[dst_row[s]] = scale (quant modes).
+ * x: bf16 [G][H] device, 16-byte aligned; expand_x: [layout->rows_cap][H] elements of
+ * the output type, 16-byte aligned, not overlapping x; dynamic_scales: fp32
+ * [rows_cap] (required for quant modes, ignored otherwise). H % 8 == 0 (NONE) or
+ * H % 16 == 0 (quant), H <= MOEDISP_MAX_H.
+ * Optional (NULL to skip), per destination rank d and local expert le:
+ *   expert_token_nums int64 [W][ne]: rows of expert d*ne+le (type 1), or the running sum
+ *     over the rank's local experts up to and including le (type 0);
+ *   ep_recv_counts int32 [W][ne][W]: rows expert d*ne+le receives from source rank r.
+ * Rows at or beyond rows_cap are not written (MOEDISP_STATUS_CAPACITY).
+ * One persistent kernel: each token row is brought into shared memory once by a bulk
+ * (TMA) copy, quantised there if asked, and written to its K rows by bulk copies. */
+int moedisp_moe_dispatch(const void *x, int H, moedisp_dims dims,
+                         const moedisp_layout *layout, int quant_mode, void *expand_x,
+                         float *dynamic_scales, int64_t *expert_token_nums,
+                         int expert_token_nums_type, int32_t *ep_recv_counts,
+                         int32_t *status, moedisp_stream_t stream);
+
+/* moe_combine
+ *
+ * The weighted combine back (Ascend aclnnMoeDistributeCombineV2 inputs expandX,
+ * expertIds / assist info, expertScales; FlashInfer MoE finalize, where a routed index
+ * of -1 means "not routed"):
+ *   y[g] = bf16_rn( acc ),  acc = 0; for k = 0..K-1 with a routed slot:
+ *                                    acc = fmaf(expert_scales[g,k], expert_out[dst_row[g*K+k]], acc)
+ * A token with no routed slot gets y[g] = 0.
+ * expert_out: bf16 [layout->rows_cap][H] device (the experts' outputs, rows in the
+ * dispatch layout); expert_scales: fp32 [G][K] device; y: bf16 [G][H] device, not
+ * overlapping expert_out. H % 8 == 0; all row pointers 16-byte aligned. */
+int moedisp_moe_combine(const void *expert_out, int H, moedisp_dims dims,
+                        const moedisp_layout *layout, const float *expert_scales, void *y,
+                        int32_t *status, moedisp_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOEDISP_H */

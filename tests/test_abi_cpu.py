@@ -1,0 +1,168 @@
+"""Host-side tests of the C ABI: the library loads without a GPU, exports every function
+include/*.h declares, and rejects bad arguments before touching the GPU (so these run on
+a CPU-only machine; the pointers below are never dereferenced)."""
+import ctypes
+import glob
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="session")
+def md():
+    from combine_a2a_exchange_b200 import _build
+    _build.build_library()
+    import combine_a2a_exchange_b200 as md
+    return md
+
+
+def declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"\b(moedisp_\w+)\s*\(", text):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("moedisp_a2a_exchange_plan", "moedisp_a2a_v", "moedisp_moe_dispatch_layout",
+                     "moedisp_moe_dispatch", "moedisp_moe_combine",
+                     "moedisp_layout_workspace_size", "moedisp_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(md):
+    lib = ctypes.CDLL(md.LIBRARY_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", md.LIBRARY_PATH], capture_output=True,
+                         text=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    assert set(declared_functions()) <= exported
+
+
+def test_status_strings(md):
+    assert md.version() == 1
+    assert md.status_string(0) == "ok"
+    assert md.status_string(-1) == "null pointer"
+    assert md.status_string(md.STATUS_CAPACITY | md.STATUS_TIMEOUT) == "capacity | timeout"
+    assert md.status_string(12345) == "unknown code"
+
+
+FAKE = 0x7f0000000000          # 16-byte aligned, never dereferenced on the host paths
+
+
+def test_plan_rejections(md):
+    call = lambda *a: md.raw_call("moedisp_a2a_exchange_plan", *a)
+    ok = [FAKE, 4, FAKE + 0x1000, FAKE + 0x2000, FAKE + 0x3000, FAKE + 0x4000, None]
+    a = list(ok); a[0] = None
+    assert call(*a) == md.MOEDISP_ERR_NULLPTR
+    a = list(ok); a[5] = None
+    assert call(*a) == md.MOEDISP_ERR_NULLPTR
+    a = list(ok); a[1] = 0
+    assert call(*a) == md.MOEDISP_ERR_INVALID
+    a = list(ok); a[1] = 70000
+    assert call(*a) == md.MOEDISP_ERR_UNSUPPORTED
+    a = list(ok); a[2] = FAKE + 0x1004
+    assert call(*a) == md.MOEDISP_ERR_MISALIGNED
+    a = list(ok); a[3] = FAKE + 0x1008          # out_splits overlaps src_offsets
+    assert call(*a) == md.MOEDISP_ERR_ALIASED
+    a = list(ok); a[2] = FAKE + 0x10            # src_offsets overlaps in_splits
+    assert call(*a) == md.MOEDISP_ERR_ALIASED
+
+
+def test_a2a_v_rejections(md):
+    call = lambda *a: md.raw_call("moedisp_a2a_v", *a)
+    # in, stride, out, cap, row_bytes, W, src, splits, dst, status, stream
+    ok = [FAKE, 10, FAKE + (1 << 30), 10, 64, 2, FAKE + (2 << 30), FAKE + (2 << 30) + 64,
+          FAKE + (2 << 30) + 128, FAKE + (2 << 30) + 256, None]
+    a = list(ok); a[4] = 24
+    assert call(*a) == md.MOEDISP_ERR_MISALIGNED
+    a = list(ok); a[0] = FAKE + 8
+    assert call(*a) == md.MOEDISP_ERR_MISALIGNED
+    a = list(ok); a[4] = 0
+    assert call(*a) == md.MOEDISP_ERR_INVALID
+    a = list(ok); a[1] = -1
+    assert call(*a) == md.MOEDISP_ERR_INVALID
+    a = list(ok); a[0] = None
+    assert call(*a) == md.MOEDISP_ERR_NULLPTR
+    a = list(ok); a[2] = FAKE + 640            # out overlaps in (2 ranks x 10 rows x 64 B)
+    assert call(*a) == md.MOEDISP_ERR_ALIASED
+    a = list(ok); a[7] = None
+    assert call(*a) == md.MOEDISP_ERR_NULLPTR
+
+
+def _layout(md, base=FAKE, rows_cap=64):
+    step = 1 << 20
+    return md.Layout(base, base + step, base + 2 * step, base + 3 * step, base + 4 * step,
+                     base + 5 * step, base + 6 * step, rows_cap)
+
+
+def test_layout_rejections(md):
+    ws_ok = md.layout_workspace_size(4, 8, 2, 8)
+    assert ws_ok > 0
+    with pytest.raises(md.MoedispError):
+        md.layout_workspace_size(3, 8, 2, 8)                 # E % W != 0
+    with pytest.raises(md.MoedispError):
+        md.layout_workspace_size(4, 8, 17, 8)                # K > 16
+    L = _layout(md)
+    call = lambda ids, dims, L, ws, nws, st: md.raw_call(
+        "moedisp_moe_dispatch_layout", ids, None, dims, ctypes.byref(L), ws, nws, st, None)
+    ids, ws, st = FAKE + (64 << 20), FAKE + (128 << 20), FAKE + (256 << 20)
+    d = md.Dims(4, 8, 2, 8)
+    assert call(ids, d, L, ws, ws_ok - 1, st) == md.MOEDISP_ERR_WORKSPACE
+    assert call(ids, d, L, None, ws_ok, st) == md.MOEDISP_ERR_WORKSPACE
+    assert call(None, d, L, ws, ws_ok, st) == md.MOEDISP_ERR_NULLPTR
+    assert call(ids, md.Dims(4, 8, 0, 8), L, ws, ws_ok, st) == md.MOEDISP_ERR_INVALID
+    assert call(ids, md.Dims(4, 8, 2, 2048), L, ws, ws_ok, st) == md.MOEDISP_ERR_UNSUPPORTED
+    assert call(ids, md.Dims(4, 1 << 28, 2, 8), L, ws, ws_ok, st) == md.MOEDISP_ERR_UNSUPPORTED
+    assert call(ids + 2, d, L, ws, ws_ok, st) == md.MOEDISP_ERR_MISALIGNED
+    bad = _layout(md); bad.dst_row = bad.occ + 16       # dst_row overlaps occ
+    assert call(ids, d, bad, ws, ws_ok, st) == md.MOEDISP_ERR_ALIASED
+    bad = _layout(md, rows_cap=-1)
+    assert call(ids, d, bad, ws, ws_ok, st) == md.MOEDISP_ERR_INVALID
+    assert call(ids, d, L, L.cnt, ws_ok, st) == md.MOEDISP_ERR_ALIASED   # workspace over cnt
+
+
+def test_dispatch_and_combine_rejections(md):
+    L = _layout(md)
+    d = md.Dims(4, 8, 2, 8)
+    x, ex, sc, st = FAKE + (64 << 20), FAKE + (128 << 20), FAKE + (192 << 20), FAKE + (256 << 20)
+    disp = lambda x, H, q, ex, sc, st, etn=None, t=1: md.raw_call(
+        "moedisp_moe_dispatch", x, H, d, ctypes.byref(L), q, ex, sc, etn, t, None, st, None)
+    assert disp(x, 128, 1, ex, sc, st) == md.MOEDISP_ERR_INVALID           # quant mode
+    assert disp(x, 120, 2, ex, sc, st) == md.MOEDISP_ERR_MISALIGNED        # H % 16 (quant)
+    assert disp(x, 124, 0, ex, sc, st) == md.MOEDISP_ERR_MISALIGNED        # H % 8
+    assert disp(x, 32768, 0, ex, sc, st) == md.MOEDISP_ERR_UNSUPPORTED
+    assert disp(x, 128, 2, ex, None, st) == md.MOEDISP_ERR_NULLPTR          # scales needed
+    assert disp(None, 128, 0, ex, None, st) == md.MOEDISP_ERR_NULLPTR
+    assert disp(x, 128, 0, x + 256, None, st) == md.MOEDISP_ERR_ALIASED     # out over x
+    assert disp(x + 8, 128, 0, ex, None, st) == md.MOEDISP_ERR_MISALIGNED
+    assert disp(x, 128, 0, ex, None, None) == md.MOEDISP_ERR_NULLPTR
+    assert disp(x, 128, 0, ex, None, st, etn=FAKE + (300 << 20), t=5) == md.MOEDISP_ERR_INVALID
+    comb = lambda eo, H, w, y, st: md.raw_call(
+        "moedisp_moe_combine", eo, H, d, ctypes.byref(L), w, y, st, None)
+    assert comb(ex, 100, x, sc, st) == md.MOEDISP_ERR_MISALIGNED
+    assert comb(ex, 0, x, sc, st) == md.MOEDISP_ERR_INVALID
+    assert comb(ex, 128, None, sc, st) == md.MOEDISP_ERR_NULLPTR
+    assert comb(ex, 128, x, ex + 512, st) == md.MOEDISP_ERR_ALIASED        # y over expert_out
+    assert comb(ex + 4, 128, x, sc, st) == md.MOEDISP_ERR_MISALIGNED
+    # no tokens: a valid no-op that launches nothing
+    assert md.raw_call("moedisp_moe_combine", None, 128, md.Dims(4, 0, 2, 8), ctypes.byref(L),
+                       None, None, st, None) == md.MOEDISP_OK
+
+
+def test_binding_has_no_fallback():
+    """The package refuses to import without the compiled library."""
+    src = open(os.path.join(ROOT, "combine_a2a_exchange_b200", "__init__.py")).read()
+    assert "raise ImportError" in src
+    for f in glob.glob(os.path.join(ROOT, "combine_a2a_exchange_b200", "**", "*.py"), recursive=True):
+        text = open(f).read()
+        assert "import oracle" not in text and "from oracle" not in text, f

@@ -1,0 +1,491 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the same seeded
+inputs. Bit-exact for counts, offsets, indices, copied rows, quantised bytes and scales;
+combine bit-exact against the fixed-order fp32 oracle and within max-abs 1e-2 / rel 1e-2
+of the fp64 oracle."""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as wl
+from tests.gpu_cases import (alloc_expand, assert_layout_equal, bf16_dev, bits_host, dev,
+                             layout_host, new_status, run_layout)
+
+pytestmark = pytest.mark.gpu
+
+ATOL = 1e-2
+RTOL = 1e-2
+
+
+@pytest.fixture(scope="module")
+def md():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import combine_a2a_exchange_b200 as md
+    return md
+
+
+# ---------------------------------------------------------------- exchange plan
+
+def run_plan(md, S):
+    W = S.shape[0]
+    Sd = dev(S.astype(np.int64))
+    outs = [torch.full((W, W), -99, dtype=torch.int64, device="cuda") for _ in range(3)]
+    st = new_status()
+    md.a2a_exchange_plan(Sd, outs[0], outs[1], outs[2], st)
+    torch.cuda.synchronize()
+    return [o.cpu().numpy() for o in outs], int(st.item())
+
+
+@pytest.mark.parametrize("W,seed", [(1, 0), (2, 1), (7, 2), (64, 3), (300, 4)])
+def test_plan_parity(md, W, seed):
+    rng = np.random.default_rng(seed)
+    S = rng.integers(0, 512, size=(W, W))
+    S[rng.random((W, W)) < 0.1] = 0
+    (src, out, dst), st = run_plan(md, S)
+    rs, ro, rd, fl = oracle.a2a_exchange_plan(S)
+    assert st == 0 and fl == 0
+    assert np.array_equal(src, rs) and np.array_equal(out, ro) and np.array_equal(dst, rd)
+
+
+def test_plan_flags_negative_split(md):
+    S = np.array([[1, -2], [3, 4]])
+    (_, out, _), st = run_plan(md, S)
+    assert st & md.STATUS_BAD_SPLIT
+    assert np.array_equal(out, S.T)
+
+
+# --------------------------------------------------------------------- a2a_v
+
+def run_a2a(md, S, rows_u8: np.ndarray, cap_out: int, fill=0xEE):
+    """rows_u8: [W, cap_in, row_bytes] uint8 send buffers. Returns out [W, cap_out, row_bytes]."""
+    W, cap_in, rb = rows_u8.shape
+    (src, out_s, dst), st = run_plan(md, S)
+    assert st == 0
+    ind = dev(rows_u8)
+    outd = torch.full((W, cap_out, rb), fill, dtype=torch.uint8, device="cuda")
+    plan = [dev(a.astype(np.int64)) for a in (src, out_s, dst)]
+    st = new_status()
+    md.a2a_v(ind, cap_in, outd, cap_out, rb, W, plan[0], plan[1], plan[2], st)
+    torch.cuda.synchronize()
+    return outd.cpu().numpy(), int(st.item()), (src, out_s, dst)
+
+
+def test_a2a_p3_worked_example(md):
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "p3_uneven_a2a_2rank.json")))
+    S = np.array(g["in_splits"])
+    rows = np.zeros((2, g["rows_per_rank"], g["cols"]), np.float32)
+    for i in range(2):
+        for k in range(g["rows_per_rank"]):
+            rows[i, k] = 10 * i + k
+    out, st, _ = run_a2a(md, S, rows.view(np.uint8).reshape(2, g["rows_per_rank"], -1), 5)
+    assert st == 0
+    outf = out.view(np.float32).reshape(2, 5, g["cols"])
+    for i, exp in enumerate(g["expected_rows"]):
+        assert (outf[i, :len(exp)] == np.array(exp, np.float32)[:, None]).all()
+        assert (out[i, len(exp):] == 0xEE).all()
+
+
+@pytest.mark.parametrize("W,max_split,row_bytes,seed", [
+    (3, 6, 16, 0), (5, 40, 48, 1), (16, 64, 16, 2), (64, 64, 32, 3), (8, 300, 8192, 4)])
+def test_a2a_parity_small(md, W, max_split, row_bytes, seed):
+    rng = np.random.default_rng(seed)
+    S = rng.integers(0, max_split, size=(W, W))
+    S[rng.random((W, W)) < 0.1] = 0
+    cap_in = max(1, int(S.sum(axis=1).max()))
+    cap_out = max(1, int(S.sum(axis=0).max())) + 3
+    rows = rng.integers(0, 256, size=(W, cap_in, row_bytes), dtype=np.uint8)
+    out, st, (src, out_s, dst) = run_a2a(md, S, rows, cap_out)
+    assert st == 0
+    ref = np.full_like(out, 0xEE)
+    assert oracle.a2a_v(rows, ref, src, out_s, dst) == 0
+    assert np.array_equal(out, ref)
+
+
+def test_a2a_bad_plan_is_skipped_and_flagged(md):
+    W, rb = 2, 32
+    S = np.array([[3, 2], [1, 4]])
+    rows = np.arange(W * 5 * rb, dtype=np.uint8).reshape(W, 5, rb)
+    (src, out_s, dst), _ = run_plan(md, S)
+    out_s = out_s.copy()
+    out_s[1, 1] = 100                                  # segment far beyond both buffers
+    outd = torch.full((W, 6, rb), 0xEE, dtype=torch.uint8, device="cuda")
+    plan = [dev(a.astype(np.int64)) for a in (src, out_s, dst)]
+    st = new_status()
+    md.a2a_v(dev(rows), 5, outd, 6, rb, W, plan[0], plan[1], plan[2], st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & md.STATUS_BAD_SPLIT
+    ref = np.full((W, 6, rb), 0xEE, np.uint8)
+    assert oracle.a2a_v(rows, ref, src, out_s, dst) & oracle.ORC_BAD_SPLIT
+    assert np.array_equal(outd.cpu().numpy(), ref)
+
+
+@pytest.mark.slow
+def test_a2a_full_size_w64_sampled(md):
+    """W=64, splits ~ randint[0,512) with 10 % zeros, 4096-element bf16 rows labelled
+    10*i+k, the first two lanes carrying the raw (i, k). Every received row is checked
+    through its provenance lanes on the GPU; 2000 sampled rows are compared whole with
+    the oracle's prediction; rows beyond each rank's receive count keep their fill."""
+    a = wl.a2a_workload(seed=0)
+    W, E_ = a.W, a.row_elems
+    S = a.in_splits
+    cap_in, cap_out = a.cap_in, a.cap_out
+    (src, out_s, dst), st = run_plan(md, S)
+    assert st == 0
+    # send buffers built on the device: label bf16(10*i + k) everywhere, lanes 0/1 = (i, k)
+    i = torch.arange(W, device="cuda", dtype=torch.float32)[:, None]
+    k = torch.arange(cap_in, device="cuda", dtype=torch.float32)[None, :]
+    lab = (10.0 * i + k).to(torch.bfloat16).view(torch.int16)
+    inp = lab[:, :, None].expand(W, cap_in, E_).contiguous()
+    inp[:, :, 0] = torch.arange(W, device="cuda", dtype=torch.int16)[:, None]
+    inp[:, :, 1] = (torch.arange(cap_in, device="cuda", dtype=torch.int64) & 0xFFFF).to(torch.int16)[None, :]
+    outd = torch.full((W, cap_out, E_), -1, dtype=torch.int16, device="cuda")
+    plan = [dev(x.astype(np.int64)) for x in (src, out_s, dst)]
+    st = new_status()
+    md.a2a_v(inp, cap_in, outd, cap_out, 2 * E_, W, plan[0], plan[1], plan[2], st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    # expected provenance of every output row, from the oracle's plan
+    exp_src = np.full((W, cap_out), -1, np.int64)
+    exp_row = np.full((W, cap_out), -1, np.int64)
+    for ii in range(W):
+        for jj in range(W):
+            n = out_s[ii, jj]
+            exp_src[ii, dst[ii, jj]:dst[ii, jj] + n] = jj
+            exp_row[ii, dst[ii, jj]:dst[ii, jj] + n] = src[ii, jj] + np.arange(n)
+    got_i = outd[:, :, 0].cpu().numpy().astype(np.int64)
+    got_k = outd[:, :, 1].cpu().numpy().astype(np.int64) & 0xFFFF
+    filled = exp_src >= 0
+    assert np.array_equal(got_i[filled], exp_src[filled])
+    assert np.array_equal(got_k[filled], exp_row[filled] & 0xFFFF)
+    assert (got_i[~filled] == -1).all()
+    rng = np.random.default_rng(1)
+    rr = np.argwhere(filled)
+    pick = rr[rng.choice(len(rr), size=2000, replace=False)]
+    lab_h = wl.f32_to_bf16_bits(10.0 * np.arange(W, dtype=np.float32)[:, None]
+                                + np.arange(cap_in, dtype=np.float32)[None, :])
+    got_rows = outd[torch.from_numpy(pick[:, 0]).cuda(), torch.from_numpy(pick[:, 1]).cuda()]
+    got_rows = got_rows.cpu().numpy().view(np.uint16)
+    for n, (ii, q) in enumerate(pick):
+        jj, kk = exp_src[ii, q], exp_row[ii, q]
+        assert (got_rows[n, 2:] == lab_h[jj, kk]).all()
+
+
+# -------------------------------------------------------------------- layout
+
+LAYOUT_CASES = [
+    ("tiny", {}),
+    ("tiny", dict(W=3, T=1000, K=3, E=12)),               # 2 tiles per rank, ragged
+    ("tiny", dict(W=5, T=700, K=6, E=40, active_p=0.6)),  # ragged tiles, inactive tokens
+    ("tiny", dict(W=2, T=513, K=4, E=6, routing="dup")),  # duplicate experts in a token
+    ("tiny", dict(W=1, T=37, K=1, E=1)),
+    ("tiny", dict(W=8, T=0, K=2, E=16)),                  # no tokens
+    ("tiny", dict(W=64, T=33, K=8, E=1024)),              # many experts and ranks
+    ("cfg2", {}), ("cfg3", {}), ("cfg4", {}),
+]
+
+
+@pytest.mark.parametrize("name,over", LAYOUT_CASES)
+def test_layout_parity(md, name, over):
+    w = wl.moe_workload(name, seed=21, **over)
+    L, st = run_layout(md, w)
+    ref = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active)
+    assert st == 0 and ref["flags"] == 0
+    assert_layout_equal(layout_host(L), ref, ref["R"], ref["rows_cap"])
+
+
+def test_layout_repeated_calls_reuse_workspace(md):
+    w = wl.moe_workload("tiny", seed=5, W=4, T=900, K=4, E=16)
+    L, _ = run_layout(md, w)
+    st = new_status()
+    for seed in range(3):
+        w2 = wl.moe_workload("tiny", seed=100 + seed, W=4, T=900, K=4, E=16, active_p=0.5)
+        md.moe_dispatch_layout(dev(w2.expert_ids.reshape(-1)), dev(w2.active), L, st)
+        torch.cuda.synchronize()
+        ref = oracle.moe_dispatch_layout(w2.W, w2.T, w2.K, w2.E, w2.expert_ids, w2.active)
+        assert_layout_equal(layout_host(L), ref, ref["R"], ref["rows_cap"])
+    assert int(st.item()) == 0
+
+
+def test_layout_bad_expert_ids(md):
+    w = wl.moe_workload("tiny", seed=6, W=2, T=300, K=3, E=8)
+    ids = w.expert_ids.copy()
+    ids[5, 1] = 8
+    ids[77, 0] = -3
+    L, st = run_layout(md, w, ids=ids)
+    ref = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, ids, w.active)
+    assert st == md.STATUS_BAD_EXPERT_ID and ref["flags"] == oracle.ORC_BAD_EXPERT
+    assert_layout_equal(layout_host(L), ref, ref["R"], ref["rows_cap"])
+
+
+def test_layout_capacity_overflow(md):
+    w = wl.moe_workload("tiny", seed=7, W=2, T=300, K=3, E=8)
+    cap = 1000                                                     # R = 1800
+    L, st = run_layout(md, w, rows_cap=cap)
+    ref = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active, rows_cap=cap)
+    assert st == md.STATUS_CAPACITY and ref["flags"] == oracle.ORC_CAPACITY
+    assert_layout_equal(layout_host(L), ref, ref["R"], cap)
+
+
+# ------------------------------------------------------------------ dispatch
+
+def run_dispatch(md, w, L, quant_mode, etn_type=1):
+    x = bf16_dev(w.x_bits)
+    full, scales, gr = alloc_expand(L, w.H, quant_mode)
+    ex = full[gr:gr + L.rows_cap]
+    sc = scales[gr:gr + L.rows_cap]
+    ne = w.E // w.W
+    etn = torch.full((w.W, ne), -1, dtype=torch.int64, device="cuda")
+    erc = torch.full((w.W, ne, w.W), -1, dtype=torch.int32, device="cuda")
+    st = new_status()
+    md.moe_dispatch(x, w.H, L, quant_mode, ex, sc if quant_mode else None, st,
+                    expert_token_nums=etn, expert_token_nums_type=etn_type, ep_recv_counts=erc)
+    torch.cuda.synchronize()
+    return full, scales, gr, etn.cpu().numpy(), erc.cpu().numpy(), int(st.item())
+
+
+DISPATCH_CASES = [
+    ("tiny", {}, 0), ("tiny", {}, 2), ("tiny", {}, 3),
+    ("tiny", dict(W=3, T=400, K=3, E=12, H=144, active_p=0.7), 0),
+    ("tiny", dict(W=3, T=400, K=3, E=12, H=144, active_p=0.7, zero_rows=0.05), 2),
+    ("tiny", dict(W=3, T=400, K=3, E=12, H=144, active_p=0.7, zero_rows=0.05,
+                  outlier_frac=0.05), 3),
+    ("tiny", dict(W=2, T=64, K=16, E=32, H=16384), 0),                # largest H, K
+    ("tiny", dict(W=2, T=64, K=16, E=32, H=16384), 2),
+    ("tiny", dict(W=4, T=50, K=5, E=8, H=8, routing="dup"), 0),       # smallest H
+]
+
+
+@pytest.mark.parametrize("name,over,q", DISPATCH_CASES)
+def test_dispatch_parity_full(md, name, over, q):
+    w = wl.moe_workload(name, seed=31, **over)
+    L, st0 = run_layout(md, w)
+    assert st0 == 0
+    ref = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active)
+    full, scales, gr, etn, erc, st = run_dispatch(md, w, L, q)
+    assert st == 0
+    R = ref["R"]
+    rex, rsc, fl = oracle.moe_dispatch(w.x_bits, ref["dst_row"], w.K, ref["rows_cap"], q)
+    assert fl == 0
+    got = full.cpu().numpy()
+    if q == 0:
+        got = got.view(np.uint16)
+        assert np.array_equal(got[gr:gr + R], rex[:R])
+        assert (got[:gr] == np.uint16(-12345 & 0xFFFF)).all()
+        assert (got[gr + R:] == np.uint16(-12345 & 0xFFFF)).all()   # rows >= R untouched
+    else:
+        assert np.array_equal(got[gr:gr + R], rex[:R])
+        assert (got[:gr] == 0x5A).all() and (got[gr + R:] == 0x5A).all()
+        s = scales.cpu().numpy()
+        assert np.array_equal(s[gr:gr + R].view(np.uint32), rsc[:R].view(np.uint32))
+        assert (s[:gr] == -1).all() and (s[gr + R:] == -1).all()
+    retn, rerc, _ = oracle.moe_recv_counts(w.W, w.E, ref["cnt"], 1)
+    assert np.array_equal(etn, retn) and np.array_equal(erc, rerc)
+
+
+@pytest.mark.parametrize("name,q", [("cfg2", 0), ("cfg3", 2), ("cfg4", 3)])
+def test_dispatch_parity_full_size_sampled(md, name, q):
+    """Full-size workloads in the benchmark's launch configuration: every output row of
+    512 sampled tokens (all K destinations) and its scale, against the oracle."""
+    w = wl.moe_workload(name, seed=0)
+    L, st0 = run_layout(md, w)
+    ref = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active)
+    full, scales, gr, etn, erc, st = run_dispatch(md, w, L, q, etn_type=0)
+    assert st0 == 0 and st == 0
+    rng = np.random.default_rng(0)
+    toks = rng.choice(w.G, size=512, replace=False)
+    drow = ref["dst_row"].reshape(w.G, w.K)
+    for g in toks:
+        rows = drow[g][drow[g] >= 0]
+        if rows.size == 0:
+            continue
+        got = full[torch.from_numpy(rows + gr).cuda()].cpu().numpy()
+        if q == 0:
+            assert (got.view(np.uint16) == w.x_bits[g][None, :]).all()
+        else:
+            qr, s = oracle.quant_row(w.x_bits[g], q)
+            assert (got == qr[None, :]).all()
+            gs = scales[torch.from_numpy(rows + gr).cuda()].cpu().numpy()
+            assert (gs.view(np.uint32) == np.float32(s).view(np.uint32)).all()
+    retn, rerc, _ = oracle.moe_recv_counts(w.W, w.E, ref["cnt"], 0)
+    assert np.array_equal(etn, retn) and np.array_equal(erc, rerc)
+    R = ref["R"]
+    tail = full[gr + R:].cpu().numpy()                  # rows >= R and the guard rows
+    assert (tail == (0x5A if q else -12345)).all()
+
+
+def test_fp8_conversion_exhaustive_over_bf16(md):
+    """Every finite bf16 value with |v| <= 448 goes through the dispatch's e4m3 path with
+    scale exactly 1 (each row holds 448 as its largest magnitude) and must give the
+    oracle's OCP E4M3 code."""
+    allb = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    f = wl.bf16_bits_to_f32(allb)
+    vals = allb[np.isfinite(f) & (np.abs(f) <= 448)]
+    H = 256
+    per = H - 1
+    n_rows = -(-vals.size // per)
+    x = np.zeros((n_rows, H), np.uint16)
+    x[:, 0] = wl.f32_to_bf16_bits(np.float32(448.0))
+    flat = np.zeros(n_rows * per, np.uint16)
+    flat[:vals.size] = vals
+    x[:, 1:] = flat.reshape(n_rows, per)
+    T = n_rows
+    w = wl.MoEWorkload(name="e4m3", W=1, T=T, H=H, E=1, K=1, quant_mode=3, x_bits=x,
+                       expert_ids=np.zeros((T, 1), np.int32),
+                       weights=np.ones((T, 1), np.float32), active=None)
+    L, _ = run_layout(md, w)
+    full, scales, gr, _, _, st = run_dispatch(md, w, L, 3)
+    assert st == 0
+    got = full.cpu().numpy()[gr:gr + T]
+    assert (scales.cpu().numpy()[gr:gr + T] == 1.0).all()
+    exp = np.array([oracle.e4m3_from_f32(float(v)) for v in wl.bf16_bits_to_f32(x.reshape(-1))],
+                   np.uint8).reshape(T, H)
+    assert np.array_equal(got, exp)
+
+
+def test_dispatch_capacity_guard(md):
+    w = wl.moe_workload("tiny", seed=8, W=2, T=100, K=4, E=8, H=64)
+    cap = 500                                                      # R = 800
+    L, st = run_layout(md, w, rows_cap=cap)
+    assert st == md.STATUS_CAPACITY
+    full, scales, gr, _, _, st = run_dispatch(md, w, L, 2)
+    assert st & md.STATUS_CAPACITY
+    got = full.cpu().numpy()
+    assert (got[:gr] == 0x5A).all() and (got[gr + cap:] == 0x5A).all()
+    ref = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, None, rows_cap=cap)
+    rex, rsc, fl = oracle.moe_dispatch(w.x_bits, ref["dst_row"], w.K, cap, 2)
+    assert fl & oracle.ORC_CAPACITY
+    assert np.array_equal(got[gr:gr + cap], rex[:cap])
+
+
+# ------------------------------------------------------------------- combine
+
+def run_combine(md, L, eo_bits, w):
+    eo = bf16_dev(eo_bits)
+    y = torch.full((w.G, w.H), 7, dtype=torch.int16, device="cuda").view(torch.bfloat16)
+    st = new_status()
+    md.moe_combine(eo, w.H, L, dev(w.weights.reshape(-1)), y, st)
+    torch.cuda.synchronize()
+    return bits_host(y), int(st.item())
+
+
+def check_combine(y_bits, eo_bits, dst_row, weights, K, rows_cap):
+    y32, fl = oracle.moe_combine_f32(eo_bits, dst_row, weights, K, rows_cap)
+    y64, _ = oracle.moe_combine_f64(eo_bits, dst_row, weights, K, rows_cap)
+    assert np.array_equal(y_bits, y32), "not bit-exact against the fixed-order fp32 oracle"
+    yf = wl.bf16_bits_to_f32(y_bits).astype(np.float64)
+    err = np.abs(yf - y64)
+    assert (err <= ATOL + RTOL * np.abs(y64)).all(), err.max()
+    return fl
+
+
+COMBINE_CASES = [
+    ("tiny", {}), ("tiny", dict(W=3, T=400, K=3, E=12, H=1032, active_p=0.7)),
+    ("tiny", dict(W=2, T=64, K=16, E=32, H=16384)), ("tiny", dict(W=4, T=50, K=1, E=8, H=8)),
+    ("tiny", dict(W=4, T=90, K=5, E=8, H=136, routing="dup")),
+]
+
+
+@pytest.mark.parametrize("name,over", COMBINE_CASES)
+def test_combine_parity_full(md, name, over):
+    w = wl.moe_workload(name, seed=41, **over)
+    L, _ = run_layout(md, w)
+    ref = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active)
+    eo = wl.expert_rows(L.rows_cap, w.H, seed=42)
+    y, st = run_combine(md, L, eo, w)
+    assert st == 0
+    check_combine(y, eo, ref["dst_row"], w.weights, w.K, L.rows_cap)
+
+
+def test_combine_association_order(md):
+    """Rows 2^24, 1, -2^24 with unit weights: fixed ascending-k fp32 FMAs give 0."""
+    w = wl.moe_workload("tiny", seed=1, W=1, T=1, K=3, E=3, H=8)
+    w.weights[:] = 1.0
+    w.expert_ids[:] = np.array([[0, 1, 2]], np.int32)
+    L, _ = run_layout(md, w)
+    vals = wl.f32_to_bf16_bits(np.array([2.0 ** 24, 1.0, -(2.0 ** 24)], np.float32))
+    eo = np.repeat(vals[:, None], 8, axis=1)
+    y, st = run_combine(md, L, eo, w)
+    assert st == 0 and (wl.bf16_bits_to_f32(y) == 0).all()
+
+
+@pytest.mark.parametrize("name", ["cfg2", "cfg3", "cfg4"])
+def test_combine_parity_full_size_sampled(md, name):
+    w = wl.moe_workload(name, seed=0)
+    L, _ = run_layout(md, w)
+    ref = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active)
+    R = ref["R"]
+    # expert outputs: N(0,1) rows generated on the device from a seeded generator
+    gen = torch.Generator(device="cuda").manual_seed(5)
+    eo = torch.randn((L.rows_cap, w.H), generator=gen, device="cuda").to(torch.bfloat16)
+    y = torch.empty((w.G, w.H), dtype=torch.bfloat16, device="cuda")
+    st = new_status()
+    md.moe_combine(eo, w.H, L, dev(w.weights.reshape(-1)), y, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    rng = np.random.default_rng(3)
+    toks = rng.choice(w.G, size=256, replace=False)
+    drow = ref["dst_row"].reshape(w.G, w.K)
+    sel = drow[toks]
+    rows = np.unique(sel[sel >= 0])
+    # compact copy of just the rows these tokens read, with dst_row remapped onto it
+    remap = np.full(L.rows_cap, -1, np.int64)
+    remap[rows] = np.arange(rows.size)
+    sub_dr = np.where(sel >= 0, remap[np.maximum(sel, 0)], -1).astype(np.int32)
+    sub_eo = bits_host(eo[torch.from_numpy(rows).cuda()]) if rows.size else np.zeros((1, w.H), np.uint16)
+    yt = bits_host(y[torch.from_numpy(toks).cuda()])
+    check_combine(yt, sub_eo, sub_dr, w.weights[toks], w.K, max(rows.size, 1))
+    if w.active is not None:
+        assert (yt[w.active[toks] == 0] == 0).all()
+
+
+# --------------------------------------------------------------- end to end
+
+@pytest.mark.parametrize("name,over,q", [("tiny", {}, 0), ("cfg2", {}, 0),
+                                         ("tiny", dict(W=4, T=300, K=4, E=16, H=256, active_p=0.8), 2),
+                                         ("tiny", dict(W=4, T=300, K=4, E=16, H=256, active_p=0.8), 3)])
+def test_dispatch_then_combine(md, name, over, q):
+    """Layout -> dispatch -> identity expert -> combine. For bf16 the expert output is
+    expand_x itself; for the quant modes the harness dequantises (q * scale, bf16), on
+    the GPU through torch, as the experts' input would be. Checked against the oracle
+    composition and against sum_k w_k * x."""
+    w = wl.moe_workload(name, seed=51, **over)
+    L, _ = run_layout(md, w)
+    full, scales, gr, _, _, st = run_dispatch(md, w, L, q)
+    assert st == 0
+    ref = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active)
+    R = ref["R"]
+    if q == 0:
+        eo_d = full[gr:gr + L.rows_cap].view(torch.bfloat16)
+    elif q == 2:
+        eo_d = (full[gr:gr + L.rows_cap].view(torch.int8).float()
+                * scales[gr:gr + L.rows_cap, None]).to(torch.bfloat16)
+    else:
+        eo_d = (full[gr:gr + L.rows_cap].view(torch.float8_e4m3fn).float()
+                * scales[gr:gr + L.rows_cap, None]).to(torch.bfloat16)
+    eo_d = eo_d.contiguous()
+    y = torch.empty((w.G, w.H), dtype=torch.bfloat16, device="cuda")
+    st2 = new_status()
+    md.moe_combine(eo_d, w.H, L, dev(w.weights.reshape(-1)), y, st2)
+    torch.cuda.synchronize()
+    assert int(st2.item()) == 0
+    rex, rsc, _ = oracle.moe_dispatch(w.x_bits, ref["dst_row"], w.K, ref["rows_cap"], q)
+    if q == 0:
+        eo_ref = rex
+    else:
+        deq = (rex.view(np.int8).astype(np.float32) if q == 2 else
+               torch.from_numpy(rex).view(torch.float8_e4m3fn).float().numpy())
+        eo_ref = wl.f32_to_bf16_bits(deq * rsc[:, None])
+    assert np.array_equal(bits_host(eo_d)[:R], eo_ref[:R])
+    yb = bits_host(y)
+    check_combine(yb, eo_ref, ref["dst_row"], w.weights, w.K, L.rows_cap)
+    if q == 0:
+        xf = wl.bf16_bits_to_f32(w.x_bits).astype(np.float64)
+        act = np.ones(w.G, bool) if w.active is None else w.active.astype(bool)
+        wsum = w.weights.astype(np.float64).sum(axis=1)
+        exp = xf * (wsum * act)[:, None]
+        yf = wl.bf16_bits_to_f32(yb).astype(np.float64)
+        assert (np.abs(yf - exp) <= ATOL + RTOL * np.abs(exp)).all()
