@@ -178,45 +178,67 @@ class MoEStep:
         self.y = t.empty((w.G, w.H), dtype=t.bfloat16, device=device)
         self.status = t.zeros(1, dtype=t.int32, device=device)
 
-    def run(self, events=None):
-        md, L, w = self.md, self.L, self.w
-        md.moe_dispatch_layout(self.ids, self.active, L, self.status)
-        if events:
-            events[0].record()
-        md.a2a_exchange_plan(L.send_splits, self.plan[0], self.plan[1], self.plan[2], self.status)
-        if events:
-            events[1].record()
-        md.moe_dispatch(self.x, w.H, L, w.quant_mode, self.ex, self.scales, self.status,
-                        expert_token_nums=self.etn, expert_token_nums_type=0,
-                        ep_recv_counts=self.erc)
-        if events:
-            events[2].record()
-        md.moe_combine(self.expert_out, w.H, L, self.wts, self.y, self.status)
+    def op_layout(self):
+        self.md.moe_dispatch_layout(self.ids, self.active, self.L, self.status)
+
+    def op_plan(self):
+        L = self.L
+        self.md.a2a_exchange_plan(L.send_splits, self.plan[0], self.plan[1], self.plan[2],
+                                  self.status)
+
+    def op_dispatch(self):
+        w = self.w
+        self.md.moe_dispatch(self.x, w.H, self.L, w.quant_mode, self.ex, self.scales, self.status,
+                             expert_token_nums=self.etn, expert_token_nums_type=0,
+                             ep_recv_counts=self.erc)
+
+    def op_combine(self):
+        self.md.moe_combine(self.expert_out, self.w.H, self.L, self.wts, self.y, self.status)
+
+    def run(self):
+        self.op_layout()
+        self.op_plan()
+        self.op_dispatch()
+        self.op_combine()
 
 
-def time_steps(torch, step, steps, warmup, flush):
-    """Per-step CUDA-event times (ms) of the whole step and of each op."""
+def capture(torch, fn):
+    """CUDA graph of fn's launches (one eager run first, outside the capture)."""
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def time_graph(torch, g, reps, warmup, flush):
+    """CUDA-event time (ms) of each of `reps` replays, L2 flushed before each."""
     E = torch.cuda.Event
     for _ in range(warmup):
         flush.zero_()
-        step.run()
+        g.replay()
     torch.cuda.synchronize()
-    rec = []
-    for _ in range(steps):
+    evs = []
+    for _ in range(reps):
         flush.zero_()
-        ev = [E(enable_timing=True) for _ in range(5)]
-        ev[0].record()
-        step.run(events=ev[1:4])
-        ev[4].record()
-        rec.append(ev)
+        a, b = E(enable_timing=True), E(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        evs.append((a, b))
     torch.cuda.synchronize()
-    out = {"step": [], "layout": [], "plan": [], "dispatch": [], "combine": []}
-    for ev in rec:
-        out["step"].append(ev[0].elapsed_time(ev[4]))
-        out["layout"].append(ev[0].elapsed_time(ev[1]))
-        out["plan"].append(ev[1].elapsed_time(ev[2]))
-        out["dispatch"].append(ev[2].elapsed_time(ev[3]))
-        out["combine"].append(ev[3].elapsed_time(ev[4]))
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def time_ops(torch, step, reps, warmup, flush):
+    """Per-op CUDA-event times (ms), each op replayed alone from its own graph."""
+    out = {}
+    for op in ("layout", "plan", "dispatch", "combine"):
+        g = capture(torch, getattr(step, "op_" + op))
+        out[op] = time_graph(torch, g, reps, warmup, flush)
+        del g
     return out
 
 
@@ -307,7 +329,10 @@ def op_sweep(md, torch, device, hbm, reps=10):
     for name in ("cfg3", "cfg4"):
         w = wl.moe_workload(name, seed=0)
         st = MoEStep(md, torch, w, device)
-        t = time_steps(torch, st, reps, 3, flush)
+        g = capture(torch, st.run)
+        t_step = time_graph(torch, g, reps, 3, flush)
+        del g
+        t = time_ops(torch, st, reps, 3, flush)
         R = int(st.L.expert_base[-1].item())
         for op in ("layout", "dispatch", "combine"):
             ms = statistics.mean(t[op])
@@ -315,8 +340,8 @@ def op_sweep(md, torch, device, hbm, reps=10):
             out.append({"workload": name, "op": op, "us": round(ms * 1e3, 2),
                         "bytes": b, "GB/s": round(b / ms / 1e6, 1),
                         "frac": round(b / ms / 1e6 / hbm, 4)})
-        out.append({"workload": name, "op": "step", "us": round(statistics.mean(t["step"]) * 1e3, 2),
-                    "tokens/s": round(w.G / (statistics.mean(t["step"]) / 1e3), 1)})
+        out.append({"workload": name, "op": "step", "us": round(statistics.mean(t_step) * 1e3, 2),
+                    "tokens/s": round(w.G / (statistics.mean(t_step) / 1e3), 1)})
         assert int(st.status.item()) == 0, md.status_string(int(st.status.item()))
         del st
         torch.cuda.empty_cache()
@@ -407,26 +432,28 @@ def main():
         pass
     sampler = ClockSampler(enabled=(rank == 0))
 
-    # warm-up
+    g_step = capture(torch, step.run)
     for _ in range(args.warmup):
         flush.zero_()
-        step.run()
+        g_step.replay()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     sampler.start()
-    t = time_steps(torch, step, args.steps, 0, flush)
+    t_step = time_graph(torch, g_step, args.steps, 0, flush)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     clocks = sampler.stop([uuid.replace("GPU-", "")] if uuid else None) if rank == 0 else None
+    del g_step
+    t = time_ops(torch, step, args.steps, args.warmup, flush)
     status = int(step.status.item())
     if status != 0:
         raise RuntimeError(f"device status after the timed steps: {md.status_string(status)}")
 
-    ms_step = statistics.mean(t["step"])
+    ms_step = statistics.mean(t_step)
     if world > 1:
         tt = torch.tensor([ms_step], device=device, dtype=torch.float64)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
@@ -480,6 +507,7 @@ def main():
         "dtype": "bf16",
         "data": "synthetic (seeded generator; no dataset)",
         "config": config_of(w),
+        "timing": "CUDA-graph replay of the step's launches; per-op times from per-op graphs",
         "hbm_GBps_step": round(step_bytes / (ms_step * 1e-3) / 1e9, 1),
         "frac_of_peak_step": round(step_bytes / (ms_step * 1e-3) / 1e9 / hbm, 4),
         "per_op_us": {k: round(v * 1e3, 2) for k, v in per_op.items()},

@@ -89,10 +89,8 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a) {
 template <int K>
 cudaError_t launch_k(const CombineArgs& a, cudaStream_t stream) {
     int per_sm = 1;
-    cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, combine_kernel<K>,
-                                                                    kThreads, 0);
+    cudaError_t err = blocks_per_sm((const void*)combine_kernel<K>, kThreads, 0, &per_sm);
     if (err != cudaSuccess) return err;
-    per_sm = std::max(per_sm, 1);
     const int chunks = (a.H8 + kThreads - 1) / kThreads;
     int64_t grid = (int64_t)current_sm_count() * per_sm;
     grid = std::min<int64_t>(grid, std::max<int64_t>(1, a.G * chunks));

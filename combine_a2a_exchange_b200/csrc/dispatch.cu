@@ -249,13 +249,9 @@ cudaError_t launch_q(const DispatchArgs& a0, cudaStream_t stream) {
     S = std::max(S, 2);
     a.stages = S;
     const size_t smem = (size_t)S * per_stage + fixed;
-    cudaError_t err = cudaFuncSetAttribute(dispatch_kernel<Q>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
     int per_sm = 1;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dispatch_kernel<Q>, NT, smem);
+    cudaError_t err = blocks_per_sm((const void*)dispatch_kernel<Q>, NT, smem, &per_sm);
     if (err != cudaSuccess) return err;
-    per_sm = std::max(per_sm, 1);
     int64_t grid = (int64_t)current_sm_count() * per_sm;
     grid = std::min<int64_t>(grid, std::max<int64_t>(a.G, 1));
     dispatch_kernel<Q><<<(unsigned)grid, NT, smem, stream>>>(a);

@@ -16,7 +16,6 @@
 #include "kernels.h"
 
 #include <algorithm>
-#include <mutex>
 
 namespace moedisp {
 
@@ -127,22 +126,6 @@ a2a_v_kernel(const uint8_t* __restrict__ in, int64_t in_stride_rows, uint8_t* __
 
 // ------------------------------------------------------------------ launchers
 
-int current_sm_count() {
-    static std::mutex mu;
-    static int cache[64] = {0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-    if (dev < 0 || dev >= 64) dev = 0;
-    std::lock_guard<std::mutex> lock(mu);
-    if (cache[dev] == 0) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-            n = 148;
-        cache[dev] = n;
-    }
-    return cache[dev];
-}
-
 cudaError_t launch_a2a_plan(const int64_t* in_splits, int W, int64_t* src_offsets,
                             int64_t* out_splits, int64_t* dst_offsets, int32_t* status,
                             cudaStream_t stream) {
@@ -156,13 +139,9 @@ cudaError_t launch_a2a_v(const void* in, int64_t in_rank_stride_rows, void* out,
                          const int64_t* src_offsets, const int64_t* out_splits,
                          const int64_t* dst_offsets, int32_t* status, cudaStream_t stream) {
     const size_t smem = (size_t)kA2AStages * kA2APiece;
-    cudaError_t err = cudaFuncSetAttribute(a2a_v_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)smem);
-    if (err != cudaSuccess) return err;
     int per_sm = 1;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, a2a_v_kernel, kA2AThreads, smem);
+    cudaError_t err = blocks_per_sm((const void*)a2a_v_kernel, kA2AThreads, smem, &per_sm);
     if (err != cudaSuccess) return err;
-    per_sm = std::max(per_sm, 1);
     const int64_t segs = (int64_t)W * W;
     const int64_t target = (int64_t)current_sm_count() * per_sm * 2;
     // No segment holds more rows than either its source or its destination buffer.

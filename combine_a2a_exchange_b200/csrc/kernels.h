@@ -12,6 +12,13 @@ namespace moedisp {
 // Streaming-multiprocessor count of the current device (cached per device).
 int current_sm_count();
 
+// Lets `kernel` use the device's full opt-in dynamic shared memory (once per device).
+cudaError_t allow_dynamic_smem(const void* kernel);
+
+// Resident blocks per SM of `kernel` at this block size and dynamic shared memory
+// (at least 1; cached per device). Also calls allow_dynamic_smem.
+cudaError_t blocks_per_sm(const void* kernel, int threads, size_t smem, int* out);
+
 cudaError_t launch_a2a_plan(const int64_t* in_splits, int W, int64_t* src_offsets,
                             int64_t* out_splits, int64_t* dst_offsets, int32_t* status,
                             cudaStream_t stream);

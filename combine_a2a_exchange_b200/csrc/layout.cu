@@ -351,11 +351,9 @@ cudaError_t launch_layout(const int32_t* expert_ids, const uint8_t* active,
     smem1 = (smem1 + 15) & ~(size_t)15;
     const size_t smem2 = (size_t)(kWarps + 1) * dims.E * sizeof(int32_t);
 
-    cudaError_t err = cudaFuncSetAttribute(layout_hist_kernel,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
+    cudaError_t err = allow_dynamic_smem((const void*)layout_hist_kernel);
     if (err != cudaSuccess) return err;
-    err = cudaFuncSetAttribute(layout_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)smem2);
+    err = allow_dynamic_smem((const void*)layout_scatter_kernel);
     if (err != cudaSuccess) return err;
     layout_hist_kernel<<<(unsigned)g.n_tiles, kThreads, smem1, stream>>>(a);
     err = cudaGetLastError();
