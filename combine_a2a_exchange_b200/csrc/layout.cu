@@ -20,10 +20,24 @@
 //    tile publishes its aggregate, then walks back over predecessors' status words in
 //    windows of kWindow until it meets an inclusive prefix); finally every slot is
 //    scattered: dst_row, occ and assist_info.
+//
+// When the whole problem fits one thread-block cluster (at most 16 rank-aligned tiles of
+// at most 16384 slots), a single kernel replaces both: one 1024-thread block per tile
+// ranks its slots as above, the blocks exchange their per-expert tile counts through
+// distributed shared memory across the cluster barrier, and every block derives its
+// tile offsets, the expert bases and the per-rank counts from those counts directly --
+// no global scratch, no second launch, no look-back.
 #include "common.cuh"
 #include "kernels.h"
 
+#include <cooperative_groups.h>
+
 #include <algorithm>
+#include <map>
+#include <mutex>
+#include <tuple>
+
+namespace cg = cooperative_groups;
 
 namespace moedisp {
 
@@ -39,6 +53,12 @@ constexpr uint32_t kFlagInclusive = 2u << 30;
 constexpr uint32_t kValueMask = (1u << 30) - 1;
 // Shared memory that kernel 1's last block may use to hold cnt while it scans.
 constexpr size_t kFinalizeSmemLimit = 160 * 1024;
+// Single-kernel cluster path.
+constexpr int kCThreads = 1024;
+constexpr int kCWarps = kCThreads / 32;
+constexpr int kCMaxSteps = 16;                          // 32-slot steps per warp
+constexpr int64_t kCMaxTile = (int64_t)kCWarps * 32 * kCMaxSteps;   // 16384 slots
+constexpr int kCMaxCluster = 16;
 
 struct LayoutArgs {
     const int32_t* ids;
@@ -295,6 +315,187 @@ __global__ void __launch_bounds__(kThreads) layout_scatter_kernel(LayoutArgs a) 
     }
 }
 
+
+__global__ void __launch_bounds__(kCThreads, 1)
+layout_cluster_kernel(LayoutArgs a, int64_t tile_len, int steps) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    __shared__ int64_t warp_tot[32];
+    cg::cluster_group cluster = cg::this_cluster();
+    const int E = a.E, W = a.W, tpr = a.tiles_per_rank;
+    int64_t* ebase = reinterpret_cast<int64_t*>(smem_raw);      // [E + 1]
+    int32_t* wc = reinterpret_cast<int32_t*>(ebase + E + 1);    // [kCWarps][E]
+    int32_t* tcnt = wc + kCWarps * E;                            // [E] this tile's counts
+    int32_t* tpre = tcnt + E;                                    // [E] counts in earlier tiles
+    int32_t* colp = tpre + E;                                    // [E] counts in earlier ranks
+    int32_t* cntr = colp + E;                                    // [E] counts of this rank
+
+    const int tile = (int)cluster.block_rank();
+    const int C = (int)cluster.num_blocks();
+    const int r = tile / tpr, c = tile - r * tpr;
+    const int64_t base = (int64_t)r * a.P;
+    const int64_t lo = (int64_t)c * tile_len, hi = min64(lo + tile_len, a.P);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const unsigned lower = (1u << lane) - 1u;
+    for (int i = threadIdx.x; i < kCWarps * E; i += blockDim.x) wc[i] = 0;
+    __syncthreads();
+
+    // Rank every slot within its warp's contiguous part of the tile.
+    int32_t* mine = wc + warp * E;
+    const int64_t wlo = lo + (int64_t)warp * steps * 32;
+    int ev[kCMaxSteps];
+    int rk[kCMaxSteps];
+    bool bad = false;
+#pragma unroll
+    for (int st = 0; st < kCMaxSteps; ++st) {
+        const int64_t l = wlo + st * 32 + lane;
+        ev[st] = (st < steps && l < hi) ? slot_expert(a, base + l, bad) : -1;
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) raise_status(a.status, MOEDISP_STATUS_BAD_EXPERT_ID);
+#pragma unroll
+    for (int st = 0; st < kCMaxSteps; ++st) {
+        rk[st] = 0;
+        if (st < steps) {
+            const int e = ev[st];
+            const unsigned peers = __match_any_sync(0xffffffffu, e);
+            const int before = e >= 0 ? mine[e] : 0;
+            __syncwarp();
+            if (e >= 0 && lane == __ffs(peers) - 1) mine[e] = before + __popc(peers);
+            __syncwarp();
+            rk[st] = before + __popc(peers & lower);
+        }
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int32_t run = 0;
+        for (int w = 0; w < kCWarps; ++w) {
+            const int32_t t = wc[w * E + e];
+            wc[w * E + e] = run;
+            run += t;
+        }
+        tcnt[e] = run;
+    }
+    cluster.sync();   // every tile's counts are final and visible across the cluster
+
+    // Counts of every tile, read from the other blocks' shared memory: offsets of this
+    // tile and of this rank, this rank's row of cnt, and the expert totals (scanned).
+    int64_t carry = 0;
+    for (int b0 = 0; b0 < E; b0 += blockDim.x) {
+        const int e = b0 + threadIdx.x;
+        int64_t tot = 0;
+        if (e < E) {
+            int32_t pre = 0, cp = 0, cr = 0;
+            for (int t = 0; t < C; ++t) {
+                const int32_t v = cluster.map_shared_rank(tcnt, t)[e];
+                tot += v;
+                pre += t < tile ? v : 0;
+                cp += t < r * tpr ? v : 0;
+                cr += t / tpr == r ? v : 0;
+            }
+            tpre[e] = pre;
+            colp[e] = cp;
+            cntr[e] = cr;
+        }
+        int64_t chunk;
+        const int64_t ex = block_exclusive_scan(tot, warp_tot, chunk);
+        if (e < E) ebase[e] = carry + ex;
+        carry += chunk;
+    }
+    if (threadIdx.x == 0) ebase[E] = carry;
+    cluster.sync();   // no block reads another block's shared memory past this point
+
+    const int64_t R = ebase[E];
+    if (tile == 0) {
+        for (int e = threadIdx.x; e <= E; e += blockDim.x) a.expert_base[e] = ebase[e];
+        for (int d = threadIdx.x; d <= W; d += blockDim.x) a.rank_base[d] = d < W ? ebase[d * a.ne] : R;
+        if (threadIdx.x == 0 && R > a.rows_cap) raise_status(a.status, MOEDISP_STATUS_CAPACITY);
+    }
+    if (c == 0) {
+        for (int e = threadIdx.x; e < E; e += blockDim.x) a.cnt[(int64_t)r * E + e] = cntr[e];
+        for (int d = threadIdx.x; d < W; d += blockDim.x) {
+            int64_t sum = 0;
+            for (int le = 0; le < a.ne; ++le) sum += cntr[d * a.ne + le];
+            a.send_splits[(int64_t)r * W + d] = sum;
+        }
+    }
+#pragma unroll
+    for (int st = 0; st < kCMaxSteps; ++st) {
+        const int64_t l = wlo + st * 32 + lane;
+        if (st >= steps || l >= hi) continue;
+        const int64_t s = base + l;
+        const int e = ev[st];
+        if (e < 0) {
+            a.dst_row[s] = -1;
+            a.occ[s] = -1;
+            continue;
+        }
+        const int32_t within = tpre[e] + mine[e] + rk[st];
+        const int64_t row = ebase[e] + within;
+        a.occ[s] = within - colp[e];
+        a.dst_row[s] = (int32_t)row;
+        if (row < a.rows_cap) a.assist[row] = (int32_t)s;
+    }
+}
+
+// Cluster path geometry: tiles per rank and slots per tile, or false if the problem does
+// not fit one cluster.
+bool cluster_geometry(const moedisp_dims& d, int* tpr, int64_t* tile_len, int* steps) {
+    const int64_t P = (int64_t)d.T * d.K;
+    const int64_t need = std::max<int64_t>(1, (P + kCMaxTile - 1) / kCMaxTile);
+    const int64_t want = std::min<int64_t>((P + 4095) / 4096, kCMaxCluster / std::max(1, d.W));
+    const int64_t t = std::max(need, want);
+    if ((int64_t)d.W * t > kCMaxCluster) return false;
+    *tpr = (int)t;
+    *tile_len = (P + t - 1) / t;
+    *steps = (int)((*tile_len + kCThreads - 1) / kCThreads);
+    return *steps <= kCMaxSteps;
+}
+
+size_t cluster_smem(int E) {
+    return (size_t)(E + 1) * sizeof(int64_t) + (size_t)(kCWarps + 4) * E * sizeof(int32_t);
+}
+
+// Whether a cluster of C blocks of this kernel can be resident on the current device.
+cudaError_t cluster_fits(int C, size_t smem, bool* ok) {
+    static std::mutex mu;
+    static std::map<std::tuple<int, int, size_t>, bool> cache;
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        auto it = cache.find({dev, C, smem});
+        if (it != cache.end()) {
+            *ok = it->second;
+            return cudaSuccess;
+        }
+    }
+    err = allow_dynamic_smem((const void*)layout_cluster_kernel);
+    if (err != cudaSuccess) return err;
+    err = cudaFuncSetAttribute(layout_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (err != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(C);
+    cfg.blockDim = dim3(kCThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    err = cudaOccupancyMaxActiveClusters(&n, (const void*)layout_cluster_kernel, &cfg);
+    if (err != cudaSuccess) {
+        (void)cudaGetLastError();
+        n = 0;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    cache[{dev, C, smem}] = n > 0;
+    *ok = n > 0;
+    return cudaSuccess;
+}
+
 }  // namespace
 
 LayoutGeometry layout_geometry(const moedisp_dims& d) {
@@ -343,6 +544,35 @@ cudaError_t launch_layout(const int32_t* expert_ids, const uint8_t* active,
     a.lookback = reinterpret_cast<uint32_t*>(ws + g.off_lookback);
     a.colprefix = reinterpret_cast<int32_t*>(ws + g.off_colprefix);
     a.status = status;
+
+    int tpr_c = 0, steps_c = 0;
+    int64_t tile_c = 0;
+    if (cluster_geometry(dims, &tpr_c, &tile_c, &steps_c)) {
+        const int C = dims.W * tpr_c;
+        const size_t smem = cluster_smem(dims.E);
+        bool ok = false;
+        cudaError_t err = cluster_fits(C, smem, &ok);
+        if (err != cudaSuccess) return err;
+        if (ok) {
+            a.tiles_per_rank = tpr_c;
+            a.n_tiles = C;
+            cudaLaunchConfig_t cfg = {};
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = C;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.gridDim = dim3(C);
+            cfg.blockDim = dim3(kCThreads);
+            cfg.dynamicSmemBytes = smem;
+            cfg.stream = stream;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            err = cudaLaunchKernelEx(&cfg, layout_cluster_kernel, a, tile_c, steps_c);
+            if (err != cudaSuccess) return err;
+            return cudaGetLastError();
+        }
+    }
 
     const size_t fin_base = (size_t)(dims.E + 1) * sizeof(int64_t);
     const size_t fin_cnt = (size_t)dims.W * dims.E * sizeof(int32_t);

@@ -184,6 +184,13 @@ LAYOUT_CASES = [
     ("tiny", dict(W=1, T=37, K=1, E=1)),
     ("tiny", dict(W=8, T=0, K=2, E=16)),                  # no tokens
     ("tiny", dict(W=64, T=33, K=8, E=1024)),              # many experts and ranks
+    # beyond one 16-block cluster: the two-kernel path with the decoupled look-back
+    ("tiny", dict(W=2, T=40000, K=8, E=16)),              # 157 tiles, long look-back chains
+    ("tiny", dict(W=20, T=300, K=4, E=40, active_p=0.5)),
+    ("tiny", dict(W=3, T=30000, K=6, E=300, routing="zipf", zipf_zero=30)),
+    # one cluster, two tiles per rank and the largest tile
+    ("tiny", dict(W=8, T=2048, K=8, E=256, routing="zipf")),
+    ("tiny", dict(W=1, T=2048, K=8, E=1024)),
     ("cfg2", {}), ("cfg3", {}), ("cfg4", {}),
 ]
 
