@@ -38,6 +38,8 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 
 template <int K>
 __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a) {
+    grid_dep_wait();
+    grid_dep_launch_dependents();
     const int chunks = (a.H8 + kThreads - 1) / kThreads;
     const int64_t items = a.G * chunks;
     for (int64_t item = blockIdx.x; item < items; item += gridDim.x) {
@@ -94,8 +96,7 @@ cudaError_t launch_k(const CombineArgs& a, cudaStream_t stream) {
     const int chunks = (a.H8 + kThreads - 1) / kThreads;
     int64_t grid = (int64_t)current_sm_count() * per_sm;
     grid = std::min<int64_t>(grid, std::max<int64_t>(1, a.G * chunks));
-    combine_kernel<K><<<(unsigned)grid, kThreads, 0, stream>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(combine_kernel<K>, dim3((unsigned)grid), dim3(kThreads), 0, stream, 1, a);
 }
 
 }  // namespace

@@ -119,12 +119,13 @@ __global__ void __launch_bounds__(Threads<Q>::value) dispatch_kernel(DispatchArg
     uint8_t* inbuf = smem;
     uint8_t* outbuf = smem + (size_t)S * a.in_bytes;
 
-    write_recv_counts(a);
-
     if (tid == 0) {
         for (int s = 0; s < S; ++s) mbar_init(&bars[s], 1);
         fence_mbar_init();
     }
+    grid_dep_wait();
+    grid_dep_launch_dependents();
+    write_recv_counts(a);
     __syncthreads();
 
     int64_t next_g = blockIdx.x;     // warp 0's look-ahead cursor over this block's tokens
@@ -254,8 +255,7 @@ cudaError_t launch_q(const DispatchArgs& a0, cudaStream_t stream) {
     if (err != cudaSuccess) return err;
     int64_t grid = (int64_t)current_sm_count() * per_sm;
     grid = std::min<int64_t>(grid, std::max<int64_t>(a.G, 1));
-    dispatch_kernel<Q><<<(unsigned)grid, NT, smem, stream>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(dispatch_kernel<Q>, dim3((unsigned)grid), dim3(NT), smem, stream, 1, a);
 }
 
 }  // namespace

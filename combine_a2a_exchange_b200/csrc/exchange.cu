@@ -31,6 +31,8 @@ a2a_plan_kernel(const int64_t* __restrict__ S, int W, int64_t* __restrict__ src_
                 int64_t* __restrict__ out_splits, int64_t* __restrict__ dst_offsets,
                 int32_t* status) {
     __shared__ int64_t warp_tot[32];
+    grid_dep_wait();
+    grid_dep_launch_dependents();
     const int b = blockIdx.x;
     bool bad = false;
     // Row b of S is what rank b sends; its exclusive scan at k is where rank k's rows
@@ -69,6 +71,8 @@ a2a_v_kernel(const uint8_t* __restrict__ in, int64_t in_stride_rows, uint8_t* __
              int blocks_per_seg, int32_t* status) {
     extern __shared__ __align__(128) uint8_t stage_buf[];
     __shared__ __align__(8) uint64_t bars[kA2AStages];
+    grid_dep_wait();
+    grid_dep_launch_dependents();
     if (threadIdx.x != 0) return;
 
     const int64_t seg = blockIdx.x / blocks_per_seg;
@@ -129,9 +133,8 @@ a2a_v_kernel(const uint8_t* __restrict__ in, int64_t in_stride_rows, uint8_t* __
 cudaError_t launch_a2a_plan(const int64_t* in_splits, int W, int64_t* src_offsets,
                             int64_t* out_splits, int64_t* dst_offsets, int32_t* status,
                             cudaStream_t stream) {
-    a2a_plan_kernel<<<W, kPlanThreads, 0, stream>>>(in_splits, W, src_offsets, out_splits,
-                                                      dst_offsets, status);
-    return cudaGetLastError();
+    return launch_pdl(a2a_plan_kernel, dim3(W), dim3(kPlanThreads), 0, stream, 1, in_splits, W,
+                      src_offsets, out_splits, dst_offsets, status);
 }
 
 cudaError_t launch_a2a_v(const void* in, int64_t in_rank_stride_rows, void* out,
@@ -151,10 +154,10 @@ cudaError_t launch_a2a_v(const void* in, int64_t in_rank_stride_rows, void* out,
     bps = std::min(bps, max_pieces);
     const int64_t grid = segs * bps;
     if (grid > 0x7fffffffll) return cudaErrorInvalidConfiguration;
-    a2a_v_kernel<<<(unsigned)grid, kA2AThreads, smem, stream>>>(
-        static_cast<const uint8_t*>(in), in_rank_stride_rows, static_cast<uint8_t*>(out),
-        out_cap_rows, row_bytes, W, src_offsets, out_splits, dst_offsets, (int)bps, status);
-    return cudaGetLastError();
+    return launch_pdl(a2a_v_kernel, dim3((unsigned)grid), dim3(kA2AThreads), smem, stream, 1,
+                      static_cast<const uint8_t*>(in), in_rank_stride_rows,
+                      static_cast<uint8_t*>(out), out_cap_rows, row_bytes, W, src_offsets,
+                      out_splits, dst_offsets, (int)bps, status);
 }
 
 }  // namespace moedisp

@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "moedisp.h"
 
 namespace moedisp {
@@ -18,6 +20,35 @@ cudaError_t allow_dynamic_smem(const void* kernel);
 // Resident blocks per SM of `kernel` at this block size and dynamic shared memory
 // (at least 1; cached per device). Also calls allow_dynamic_smem.
 cudaError_t blocks_per_sm(const void* kernel, int threads, size_t smem, int* out);
+
+// Launches `kernel` with programmatic stream serialization (and a 1-D cluster of
+// `cluster` blocks when cluster > 1) and returns the launch status.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, int cluster, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+    if (cluster > 1) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = (unsigned)cluster;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = (unsigned)n;
+    cudaError_t err = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+    if (err != cudaSuccess) return err;
+    return cudaGetLastError();
+}
 
 cudaError_t launch_a2a_plan(const int64_t* in_splits, int W, int64_t* src_offsets,
                             int64_t* out_splits, int64_t* dst_offsets, int32_t* status,

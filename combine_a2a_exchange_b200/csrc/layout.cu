@@ -162,6 +162,8 @@ __device__ void layout_finalize(const LayoutArgs& a, int32_t* smem) {
 __global__ void __launch_bounds__(kThreads) layout_hist_kernel(LayoutArgs a) {
     extern __shared__ __align__(16) int32_t smem[];
     __shared__ int is_last;
+    grid_dep_wait();
+    grid_dep_launch_dependents();
     const int tile = blockIdx.x;
     const int r = tile / a.tiles_per_rank, c = tile - r * a.tiles_per_rank;
     const int64_t base = (int64_t)r * a.P;
@@ -198,6 +200,8 @@ __global__ void __launch_bounds__(kThreads) layout_hist_kernel(LayoutArgs a) {
 __global__ void __launch_bounds__(kThreads) layout_scatter_kernel(LayoutArgs a) {
     extern __shared__ __align__(16) int32_t smem[];
     __shared__ int tile_s;
+    grid_dep_wait();
+    grid_dep_launch_dependents();
     const int E = a.E;
     int32_t* warp_cnt = smem;                    // [kWarps][E]
     int32_t* tile_off = smem + kWarps * E;       // [E]
@@ -322,9 +326,10 @@ layout_cluster_kernel(LayoutArgs a, int64_t tile_len, int steps) {
     __shared__ int64_t warp_tot[32];
     cg::cluster_group cluster = cg::this_cluster();
     const int E = a.E, W = a.W, tpr = a.tiles_per_rank;
+    const int ES = E | 1;                                        // odd row stride: no bank conflicts
     int64_t* ebase = reinterpret_cast<int64_t*>(smem_raw);      // [E + 1]
-    int32_t* wc = reinterpret_cast<int32_t*>(ebase + E + 1);    // [kCWarps][E]
-    int32_t* tcnt = wc + kCWarps * E;                            // [E] this tile's counts
+    int32_t* wc = reinterpret_cast<int32_t*>(ebase + E + 1);    // [kCWarps][ES]
+    int32_t* tcnt = wc + kCWarps * ES;                           // [E] this tile's counts
     int32_t* tpre = tcnt + E;                                    // [E] counts in earlier tiles
     int32_t* colp = tpre + E;                                    // [E] counts in earlier ranks
     int32_t* cntr = colp + E;                                    // [E] counts of this rank
@@ -336,11 +341,13 @@ layout_cluster_kernel(LayoutArgs a, int64_t tile_len, int steps) {
     const int64_t lo = (int64_t)c * tile_len, hi = min64(lo + tile_len, a.P);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const unsigned lower = (1u << lane) - 1u;
-    for (int i = threadIdx.x; i < kCWarps * E; i += blockDim.x) wc[i] = 0;
+    for (int i = threadIdx.x; i < kCWarps * ES; i += blockDim.x) wc[i] = 0;
+    grid_dep_wait();
+    grid_dep_launch_dependents();
     __syncthreads();
 
     // Rank every slot within its warp's contiguous part of the tile.
-    int32_t* mine = wc + warp * E;
+    int32_t* mine = wc + warp * ES;
     const int64_t wlo = lo + (int64_t)warp * steps * 32;
     int ev[kCMaxSteps];
     int rk[kCMaxSteps];
@@ -365,14 +372,13 @@ layout_cluster_kernel(LayoutArgs a, int64_t tile_len, int steps) {
         }
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int32_t run = 0;
-        for (int w = 0; w < kCWarps; ++w) {
-            const int32_t t = wc[w * E + e];
-            wc[w * E + e] = run;
-            run += t;
-        }
-        tcnt[e] = run;
+    // Per expert, an exclusive scan over the 32 warps' counts: one warp per expert,
+    // lane w holding warp w's count.
+    for (int e = warp; e < E; e += kCWarps) {
+        const int32_t v = wc[lane * ES + e];
+        const int32_t inc = warp_inclusive_scan_i32(v);
+        wc[lane * ES + e] = inc - v;
+        if (lane == 31) tcnt[e] = inc;
     }
     cluster.sync();   // every tile's counts are final and visible across the cluster
 
@@ -384,12 +390,13 @@ layout_cluster_kernel(LayoutArgs a, int64_t tile_len, int steps) {
         int64_t tot = 0;
         if (e < E) {
             int32_t pre = 0, cp = 0, cr = 0;
+#pragma unroll 4
             for (int t = 0; t < C; ++t) {
                 const int32_t v = cluster.map_shared_rank(tcnt, t)[e];
                 tot += v;
                 pre += t < tile ? v : 0;
                 cp += t < r * tpr ? v : 0;
-                cr += t / tpr == r ? v : 0;
+                cr += (t >= r * tpr && t < (r + 1) * tpr) ? v : 0;
             }
             tpre[e] = pre;
             colp[e] = cp;
@@ -441,7 +448,7 @@ layout_cluster_kernel(LayoutArgs a, int64_t tile_len, int steps) {
 bool cluster_geometry(const moedisp_dims& d, int* tpr, int64_t* tile_len, int* steps) {
     const int64_t P = (int64_t)d.T * d.K;
     const int64_t need = std::max<int64_t>(1, (P + kCMaxTile - 1) / kCMaxTile);
-    const int64_t want = std::min<int64_t>((P + 4095) / 4096, kCMaxCluster / std::max(1, d.W));
+    const int64_t want = std::min<int64_t>((P + 1023) / 1024, kCMaxCluster / std::max(1, d.W));
     const int64_t t = std::max(need, want);
     if ((int64_t)d.W * t > kCMaxCluster) return false;
     *tpr = (int)t;
@@ -451,7 +458,7 @@ bool cluster_geometry(const moedisp_dims& d, int* tpr, int64_t* tile_len, int* s
 }
 
 size_t cluster_smem(int E) {
-    return (size_t)(E + 1) * sizeof(int64_t) + (size_t)(kCWarps + 4) * E * sizeof(int32_t);
+    return (size_t)(E + 1) * sizeof(int64_t) + ((size_t)kCWarps * (E | 1) + 4 * (size_t)E) * sizeof(int32_t);
 }
 
 // Whether a cluster of C blocks of this kernel can be resident on the current device.
@@ -556,21 +563,8 @@ cudaError_t launch_layout(const int32_t* expert_ids, const uint8_t* active,
         if (ok) {
             a.tiles_per_rank = tpr_c;
             a.n_tiles = C;
-            cudaLaunchConfig_t cfg = {};
-            cudaLaunchAttribute attr[1];
-            attr[0].id = cudaLaunchAttributeClusterDimension;
-            attr[0].val.clusterDim.x = C;
-            attr[0].val.clusterDim.y = 1;
-            attr[0].val.clusterDim.z = 1;
-            cfg.gridDim = dim3(C);
-            cfg.blockDim = dim3(kCThreads);
-            cfg.dynamicSmemBytes = smem;
-            cfg.stream = stream;
-            cfg.attrs = attr;
-            cfg.numAttrs = 1;
-            err = cudaLaunchKernelEx(&cfg, layout_cluster_kernel, a, tile_c, steps_c);
-            if (err != cudaSuccess) return err;
-            return cudaGetLastError();
+            return launch_pdl(layout_cluster_kernel, dim3(C), dim3(kCThreads), smem, stream, C, a,
+                              tile_c, steps_c);
         }
     }
 
@@ -585,11 +579,10 @@ cudaError_t launch_layout(const int32_t* expert_ids, const uint8_t* active,
     if (err != cudaSuccess) return err;
     err = allow_dynamic_smem((const void*)layout_scatter_kernel);
     if (err != cudaSuccess) return err;
-    layout_hist_kernel<<<(unsigned)g.n_tiles, kThreads, smem1, stream>>>(a);
-    err = cudaGetLastError();
+    err = launch_pdl(layout_hist_kernel, dim3((unsigned)g.n_tiles), dim3(kThreads), smem1, stream, 1, a);
     if (err != cudaSuccess) return err;
-    layout_scatter_kernel<<<(unsigned)g.n_tiles, kThreads, smem2, stream>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(layout_scatter_kernel, dim3((unsigned)g.n_tiles), dim3(kThreads), smem2, stream,
+                      1, a);
 }
 
 }  // namespace moedisp
