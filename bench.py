@@ -177,6 +177,7 @@ class MoEStep:
         self.plan = [t.empty((w.W, w.W), dtype=t.int64, device=device) for _ in range(3)]
         self.y = t.empty((w.G, w.H), dtype=t.bfloat16, device=device)
         self.status = t.zeros(1, dtype=t.int32, device=device)
+        self.side = t.cuda.Stream(device=device)
 
     def op_layout(self):
         self.md.moe_dispatch_layout(self.ids, self.active, self.L, self.status)
@@ -196,10 +197,18 @@ class MoEStep:
         self.md.moe_combine(self.expert_out, self.w.H, self.L, self.wts, self.y, self.status)
 
     def run(self):
+        """layout -> dispatch -> combine on the current stream; the exchange plan of the
+        layout's send counts runs beside dispatch on a side stream (nothing in the step
+        consumes it), joined before the step ends."""
+        torch = self.torch
+        main = torch.cuda.current_stream()
         self.op_layout()
-        self.op_plan()
+        self.side.wait_stream(main)
+        with torch.cuda.stream(self.side):
+            self.op_plan()
         self.op_dispatch()
         self.op_combine()
+        main.wait_stream(self.side)
 
 
 def capture(torch, fn):
@@ -392,6 +401,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="cfg2")
+    ap.add_argument("--T", type=int, default=None,
+                    help="tokens per rank override (smaller cases for profiling)")
     ap.add_argument("--no-ops", action="store_true", help="skip the per-op sweep of other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -421,7 +432,8 @@ def main():
                                 device_id=device)
 
     hbm, peak_src = measured_peaks()
-    w = wl.moe_workload(args.workload, seed=rank)
+    over = {} if args.T is None else {"T": args.T}
+    w = wl.moe_workload(args.workload, seed=rank, **over)
     step = MoEStep(md, torch, w, device)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=device)
 
@@ -507,7 +519,8 @@ def main():
         "dtype": "bf16",
         "data": "synthetic (seeded generator; no dataset)",
         "config": config_of(w),
-        "timing": "CUDA-graph replay of the step's launches; per-op times from per-op graphs",
+        "timing": "CUDA-graph replay of the step (exchange plan on a side-stream branch beside "
+                  "dispatch); per-op times from per-op graphs",
         "hbm_GBps_step": round(step_bytes / (ms_step * 1e-3) / 1e9, 1),
         "frac_of_peak_step": round(step_bytes / (ms_step * 1e-3) / 1e9 / hbm, 4),
         "per_op_us": {k: round(v * 1e3, 2) for k, v in per_op.items()},
