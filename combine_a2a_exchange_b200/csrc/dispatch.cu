@@ -5,10 +5,10 @@
 // from the source buffer. On one GPU the K destinations are rows of one expand_x buffer,
 // so each token row is read from HBM exactly once: a persistent block brings the row
 // into shared memory with a 1-D bulk (TMA) load, quantises it there if asked, and the
-// K copies leave shared memory as K bulk stores issued by K lanes in parallel. Warp 0
-// runs the pipeline: it looks ahead through its tokens (skipping tokens with no active
-// slot), keeps up to kStages-1 row loads in flight, and reuses a stage only after the
-// bulk stores that read it have drained.
+// K copies leave shared memory as K bulk stores issued by K lanes in parallel. Each warp
+// runs its own pipeline: it looks ahead through its tokens (skipping tokens with no
+// active slot), keeps up to stages-1 row loads in flight, and reuses a stage only after
+// the bulk stores that read it have drained.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -40,10 +40,8 @@ struct DispatchArgs {
     int32_t* status;
 };
 
-template <int Q>
-struct Threads {
-    static constexpr int value = Q == MOEDISP_QUANT_NONE ? 32 : 256;
-};
+constexpr int kCopyThreads = 32;        // bf16 copy: one warp per block
+constexpr int kQuantWarps = 4;          // quantising copy: independent warps per block
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
@@ -105,31 +103,28 @@ __device__ void write_recv_counts(const DispatchArgs& a) {
     }
 }
 
-template <int Q>
-__global__ void __launch_bounds__(Threads<Q>::value) dispatch_kernel(DispatchArgs a) {
+// bf16 dispatch: one warp per block; lane 0 streams token rows in, lanes 0..K-1 write
+// them out.
+__global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t bars[kMaxStages];
     __shared__ int64_t tok[kMaxStages];
     __shared__ int32_t drow[kMaxStages][MOEDISP_MAX_K];
-    __shared__ float red[8];
-    __shared__ int ok_s[2];
-    constexpr int NT = Threads<Q>::value;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int lane = threadIdx.x & 31;
     const int S = a.stages, K = a.K;
     uint8_t* inbuf = smem;
-    uint8_t* outbuf = smem + (size_t)S * a.in_bytes;
 
-    if (tid == 0) {
+    if (lane == 0) {
         for (int s = 0; s < S; ++s) mbar_init(&bars[s], 1);
         fence_mbar_init();
     }
+    __syncwarp();
     grid_dep_wait();
     grid_dep_launch_dependents();
     write_recv_counts(a);
-    __syncthreads();
 
-    int64_t next_g = blockIdx.x;     // warp 0's look-ahead cursor over this block's tokens
-    // Warp 0: arm stage `st` with the next token that has an active slot (or the end).
+    int64_t next_g = blockIdx.x;     // look-ahead cursor over this block's tokens
+    // Arm stage `st` with the next token that has an active slot (or the end).
     auto fill = [&](int st) {
         while (true) {
             if (next_g >= a.G) {
@@ -169,20 +164,19 @@ __global__ void __launch_bounds__(Threads<Q>::value) dispatch_kernel(DispatchArg
         }
     };
 
-    if (warp == 0)
-        for (int st = 0; st < S; ++st) fill(st);
+    for (int st = 0; st < S; ++st) fill(st);
 
-    const bool issuer = warp == 0 && lane < K;
+    const bool issuer = lane < K;
     for (int it = 0;; ++it) {
         const int st = it % S;
         const uint32_t par = (uint32_t)((it / S) & 1);
-        // One thread waits with a time limit and shares the verdict (double-buffered: a
-        // thread can lag by at most one iteration); then every thread observes the
-        // already completed phase itself.
-        if (tid == 0) ok_s[it & 1] = mbar_wait(&bars[st], par) ? 1 : 0;
-        __syncthreads();
-        if (!ok_s[it & 1]) {
-            if (tid == 0) raise_status(a.status, MOEDISP_STATUS_TIMEOUT);
+        // Lane 0 waits with a time limit and shares the verdict; then every lane observes
+        // the already completed phase itself.
+        int ok = 1;
+        if (lane == 0) ok = mbar_wait(&bars[st], par) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+            if (lane == 0) raise_status(a.status, MOEDISP_STATUS_TIMEOUT);
             break;
         }
         (void)mbar_wait(&bars[st], par);
@@ -190,72 +184,163 @@ __global__ void __launch_bounds__(Threads<Q>::value) dispatch_kernel(DispatchArg
         if (g < 0) break;
         const uint8_t* row_in = inbuf + (size_t)st * a.in_bytes;
 
-        if constexpr (Q == MOEDISP_QUANT_NONE) {
-            if (issuer) {
-                const int32_t d = drow[st][lane];
-                if (d >= 0) bulk_store(a.expand_x + (int64_t)d * a.out_bytes, row_in, a.in_bytes);
-                bulk_commit();
-            }
-            if (it >= 1) {
-                if (issuer) bulk_wait_read<1>();
-                __syncwarp();
-                fill((it - 1) % S);
-            }
-        } else {
-            constexpr float kQmax = Q == MOEDISP_QUANT_INT8 ? 127.0f : 448.0f;
-            const uint4* v = reinterpret_cast<const uint4*>(row_in);
-            const int nvec = a.H >> 3;
-            float m = 0.0f;
-            for (int c = tid; c < nvec; c += NT) m = fmaxf(m, absmax8(v[c]));
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-            if (lane == 0) red[warp] = m;
-            if (issuer) bulk_wait_read<1>();      // output buffer it % 2 is free again
-            __syncthreads();
-            float amax = red[0];
-#pragma unroll
-            for (int w = 1; w < NT / 32; ++w) amax = fmaxf(amax, red[w]);
-            const float scale = __fdiv_rn(amax, kQmax);
-            const bool zero = amax == 0.0f;
-            uint8_t* ob = outbuf + (size_t)(it & 1) * a.out_bytes;
-            uint2* o2 = reinterpret_cast<uint2*>(ob);
-            for (int c = tid; c < nvec; c += NT) o2[c] = quant8<Q>(v[c], scale, zero);
-            fence_proxy_async_smem();
-            __syncthreads();
-            if (warp == 0) {
-                if (issuer) {
-                    const int32_t d = drow[st][lane];
-                    if (d >= 0) {
-                        bulk_store(a.expand_x + (int64_t)d * a.out_bytes, ob, a.out_bytes);
-                        a.scales[d] = scale;
-                    }
-                    bulk_commit();
-                }
-                __syncwarp();
-                fill(st);                           // every thread is done reading stage st
-            }
+        if (issuer) {
+            const int32_t d = drow[st][lane];
+            if (d >= 0) bulk_store(a.expand_x + (int64_t)d * a.out_bytes, row_in, a.in_bytes);
+            bulk_commit();
+        }
+        // Refill the stage of the previous token once its stores have read it.
+        if (it >= 1) {
+            if (issuer) bulk_wait_read<1>();
+            __syncwarp();
+            fill((it - 1) % S);
         }
     }
     if (issuer) bulk_wait<0>();
 }
 
+// Quantising dispatch: every warp is an independent pipeline over its own tokens, with
+// its own stages, barriers and output buffers, so no block-wide barrier is needed per
+// token. Lane 0 streams token rows in; the warp reduces the row's max |x| with
+// shuffles, quantises the row into one of its two output buffers, and lanes 0..K-1
+// write the quantised row (and the scale) to the token's K rows.
 template <int Q>
-cudaError_t launch_q(const DispatchArgs& a0, cudaStream_t stream) {
-    DispatchArgs a = a0;
-    constexpr int NT = Threads<Q>::value;
-    const size_t budget = Q == MOEDISP_QUANT_NONE ? 64 * 1024 : 96 * 1024;
-    const size_t per_stage = a.in_bytes;
-    const size_t fixed = Q == MOEDISP_QUANT_NONE ? 0 : 2 * (size_t)a.out_bytes;
-    int S = (int)std::min<size_t>(kMaxStages, (budget - std::min(budget, fixed)) / per_stage);
-    S = std::max(S, 2);
+__global__ void __launch_bounds__(kQuantWarps * 32) dispatch_quant_kernel(DispatchArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ __align__(8) uint64_t bars[kQuantWarps][kMaxStages];
+    __shared__ int64_t tok[kQuantWarps][kMaxStages];
+    __shared__ int32_t drow[kQuantWarps][kMaxStages][MOEDISP_MAX_K];
+    constexpr float kQmax = Q == MOEDISP_QUANT_INT8 ? 127.0f : 448.0f;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int S = a.stages, K = a.K;
+    uint8_t* inbuf = smem + (size_t)warp * (S * a.in_bytes + 2 * a.out_bytes);
+    uint8_t* outbuf = inbuf + (size_t)S * a.in_bytes;
+    uint64_t* wbar = bars[warp];
+
+    if (lane == 0) {
+        for (int s = 0; s < S; ++s) mbar_init(&wbar[s], 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+    grid_dep_wait();
+    grid_dep_launch_dependents();
+    write_recv_counts(a);
+
+    const int64_t n_warps = (int64_t)gridDim.x * kQuantWarps;
+    int64_t next_g = (int64_t)blockIdx.x * kQuantWarps + warp;
+    auto fill = [&](int st) {
+        while (true) {
+            if (next_g >= a.G) {
+                if (lane == 0) {
+                    tok[warp][st] = -1;
+                    mbar_arrive(&wbar[st]);
+                }
+                return;
+            }
+            int32_t d = -1;
+            if (lane < K) {
+                d = __ldg(a.dst_row + next_g * K + lane);
+                if (d >= a.rows_cap) {
+                    raise_status(a.status, MOEDISP_STATUS_CAPACITY);
+                    d = -1;
+                }
+                if (d < 0) d = -1;
+            }
+            if (__ballot_sync(0xffffffffu, d >= 0)) {
+                int32_t dk[MOEDISP_MAX_K];
+#pragma unroll
+                for (int k = 0; k < MOEDISP_MAX_K; ++k) dk[k] = __shfl_sync(0xffffffffu, d, k);
+                if (lane == 0) {
+#pragma unroll
+                    for (int k = 0; k < MOEDISP_MAX_K; ++k)
+                        if (k < K) drow[warp][st][k] = dk[k];
+                    tok[warp][st] = next_g;
+                    mbar_arrive_expect_tx(&wbar[st], a.in_bytes);
+                    bulk_load(inbuf + (size_t)st * a.in_bytes, a.x + next_g * a.in_bytes,
+                              a.in_bytes, &wbar[st]);
+                }
+                next_g += n_warps;
+                return;
+            }
+            next_g += n_warps;
+        }
+    };
+
+    for (int st = 0; st < S; ++st) fill(st);
+    const bool issuer = lane < K;
+    const int nvec = a.H >> 3;
+    for (int it = 0;; ++it) {
+        const int st = it % S;
+        const uint32_t par = (uint32_t)((it / S) & 1);
+        int ok = 1;
+        if (lane == 0) ok = mbar_wait(&wbar[st], par) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+            if (lane == 0) raise_status(a.status, MOEDISP_STATUS_TIMEOUT);
+            break;
+        }
+        (void)mbar_wait(&wbar[st], par);
+        const int64_t g = tok[warp][st];
+        if (g < 0) break;
+        const uint4* v = reinterpret_cast<const uint4*>(inbuf + (size_t)st * a.in_bytes);
+        float m = 0.0f;
+        for (int c = lane; c < nvec; c += 32) m = fmaxf(m, absmax8(v[c]));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        const float scale = __fdiv_rn(m, kQmax);
+        const bool zero = m == 0.0f;
+        if (issuer) bulk_wait_read<1>();      // output buffer it % 2 is free again
+        __syncwarp();
+        uint8_t* ob = outbuf + (size_t)(it & 1) * a.out_bytes;
+        uint2* o2 = reinterpret_cast<uint2*>(ob);
+        for (int c = lane; c < nvec; c += 32) o2[c] = quant8<Q>(v[c], scale, zero);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (issuer) {
+            const int32_t d = drow[warp][st][lane];
+            if (d >= 0) {
+                bulk_store(a.expand_x + (int64_t)d * a.out_bytes, ob, a.out_bytes);
+                a.scales[d] = scale;
+            }
+            bulk_commit();
+        }
+        __syncwarp();
+        fill(st);                               // the warp is done reading stage st
+    }
+    if (issuer) bulk_wait<0>();
+}
+
+cudaError_t launch_copy(DispatchArgs a, cudaStream_t stream) {
+    const size_t budget = 64 * 1024;
+    const int S = (int)std::max<size_t>(2, std::min<size_t>(kMaxStages, budget / a.in_bytes));
     a.stages = S;
-    const size_t smem = (size_t)S * per_stage + fixed;
+    const size_t smem = (size_t)S * a.in_bytes;
     int per_sm = 1;
-    cudaError_t err = blocks_per_sm((const void*)dispatch_kernel<Q>, NT, smem, &per_sm);
+    cudaError_t err = blocks_per_sm((const void*)dispatch_copy_kernel, kCopyThreads, smem, &per_sm);
     if (err != cudaSuccess) return err;
     int64_t grid = (int64_t)current_sm_count() * per_sm;
     grid = std::min<int64_t>(grid, std::max<int64_t>(a.G, 1));
-    return launch_pdl(dispatch_kernel<Q>, dim3((unsigned)grid), dim3(NT), smem, stream, 1, a);
+    return launch_pdl(dispatch_copy_kernel, dim3((unsigned)grid), dim3(kCopyThreads), smem, stream,
+                      1, a);
+}
+
+template <int Q>
+cudaError_t launch_quant(DispatchArgs a, cudaStream_t stream) {
+    // Per warp: S input stages and two output buffers; aim for two blocks per SM.
+    const size_t per_warp_budget = 110 * 1024 / kQuantWarps;
+    const size_t fixed = 2 * (size_t)a.out_bytes;
+    int S = (int)((per_warp_budget - std::min(per_warp_budget, fixed)) / a.in_bytes);
+    S = std::max(2, std::min(S, 4));
+    a.stages = S;
+    const size_t smem = (size_t)kQuantWarps * ((size_t)S * a.in_bytes + fixed);
+    int per_sm = 1;
+    cudaError_t err = blocks_per_sm((const void*)dispatch_quant_kernel<Q>, kQuantWarps * 32, smem,
+                                    &per_sm);
+    if (err != cudaSuccess) return err;
+    int64_t grid = (int64_t)current_sm_count() * per_sm;
+    grid = std::min<int64_t>(grid, std::max<int64_t>((a.G + kQuantWarps - 1) / kQuantWarps, 1));
+    return launch_pdl(dispatch_quant_kernel<Q>, dim3((unsigned)grid), dim3(kQuantWarps * 32), smem,
+                      stream, 1, a);
 }
 
 }  // namespace
@@ -288,9 +373,9 @@ cudaError_t launch_dispatch(const void* x, int H, const moedisp_dims& dims,
     a.erc = ep_recv_counts;
     a.status = status;
     switch (quant_mode) {
-        case MOEDISP_QUANT_NONE: return launch_q<MOEDISP_QUANT_NONE>(a, stream);
-        case MOEDISP_QUANT_INT8: return launch_q<MOEDISP_QUANT_INT8>(a, stream);
-        case MOEDISP_QUANT_FP8_E4M3: return launch_q<MOEDISP_QUANT_FP8_E4M3>(a, stream);
+        case MOEDISP_QUANT_NONE: return launch_copy(a, stream);
+        case MOEDISP_QUANT_INT8: return launch_quant<MOEDISP_QUANT_INT8>(a, stream);
+        case MOEDISP_QUANT_FP8_E4M3: return launch_quant<MOEDISP_QUANT_FP8_E4M3>(a, stream);
         default: return cudaErrorInvalidValue;
     }
 }

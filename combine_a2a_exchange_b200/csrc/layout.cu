@@ -320,8 +320,17 @@ __global__ void __launch_bounds__(kThreads) layout_scatter_kernel(LayoutArgs a) 
 }
 
 
+__device__ __forceinline__ void cluster_arrive_release() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// STEPS = 32-slot steps per warp (a power of two, at most kCMaxSteps).
+template <int STEPS>
 __global__ void __launch_bounds__(kCThreads, 1)
-layout_cluster_kernel(LayoutArgs a, int64_t tile_len, int steps) {
+layout_cluster_kernel(LayoutArgs a, int64_t tile_len) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ int64_t warp_tot[32];
     cg::cluster_group cluster = cg::this_cluster();
@@ -344,32 +353,30 @@ layout_cluster_kernel(LayoutArgs a, int64_t tile_len, int steps) {
     for (int i = threadIdx.x; i < kCWarps * ES; i += blockDim.x) wc[i] = 0;
     grid_dep_wait();
     grid_dep_launch_dependents();
-    __syncthreads();
 
-    // Rank every slot within its warp's contiguous part of the tile.
+    // Each warp owns STEPS*32 consecutive slots of the tile.
     int32_t* mine = wc + warp * ES;
-    const int64_t wlo = lo + (int64_t)warp * steps * 32;
-    int ev[kCMaxSteps];
-    int rk[kCMaxSteps];
+    const int64_t wlo = lo + (int64_t)warp * STEPS * 32;
+    int ev[STEPS];
     bool bad = false;
 #pragma unroll
-    for (int st = 0; st < kCMaxSteps; ++st) {
+    for (int st = 0; st < STEPS; ++st) {
         const int64_t l = wlo + st * 32 + lane;
-        ev[st] = (st < steps && l < hi) ? slot_expert(a, base + l, bad) : -1;
+        ev[st] = l < hi ? slot_expert(a, base + l, bad) : -1;
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) raise_status(a.status, MOEDISP_STATUS_BAD_EXPERT_ID);
+    __syncthreads();
+    // Rank within the warp's slots, in slot order: packed as (rank << 11) | (expert + 1).
+    uint32_t pk[STEPS];
 #pragma unroll
-    for (int st = 0; st < kCMaxSteps; ++st) {
-        rk[st] = 0;
-        if (st < steps) {
-            const int e = ev[st];
-            const unsigned peers = __match_any_sync(0xffffffffu, e);
-            const int before = e >= 0 ? mine[e] : 0;
-            __syncwarp();
-            if (e >= 0 && lane == __ffs(peers) - 1) mine[e] = before + __popc(peers);
-            __syncwarp();
-            rk[st] = before + __popc(peers & lower);
-        }
+    for (int st = 0; st < STEPS; ++st) {
+        const int e = ev[st];
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        const int before = e >= 0 ? mine[e] : 0;
+        __syncwarp();
+        if (e >= 0 && lane == __ffs(peers) - 1) mine[e] = before + __popc(peers);
+        __syncwarp();
+        pk[st] = e >= 0 ? ((uint32_t)(before + __popc(peers & lower)) << 11) | (uint32_t)(e + 1) : 0u;
     }
     __syncthreads();
     // Per expert, an exclusive scan over the 32 warps' counts: one warp per expert,
@@ -382,21 +389,25 @@ layout_cluster_kernel(LayoutArgs a, int64_t tile_len, int steps) {
     }
     cluster.sync();   // every tile's counts are final and visible across the cluster
 
-    // Counts of every tile, read from the other blocks' shared memory: offsets of this
-    // tile and of this rank, this rank's row of cnt, and the expert totals (scanned).
+    // Counts of every tile, read from the other blocks' shared memory (all reads issued
+    // together): offsets of this tile and of this rank, this rank's row of cnt, and the
+    // expert totals, scanned into expert bases.
     int64_t carry = 0;
     for (int b0 = 0; b0 < E; b0 += blockDim.x) {
         const int e = b0 + threadIdx.x;
         int64_t tot = 0;
         if (e < E) {
+            int32_t v[kCMaxCluster];
+#pragma unroll
+            for (int t = 0; t < kCMaxCluster; ++t)
+                v[t] = t < C ? cluster.map_shared_rank(tcnt, t)[e] : 0;
             int32_t pre = 0, cp = 0, cr = 0;
-#pragma unroll 4
-            for (int t = 0; t < C; ++t) {
-                const int32_t v = cluster.map_shared_rank(tcnt, t)[e];
-                tot += v;
-                pre += t < tile ? v : 0;
-                cp += t < r * tpr ? v : 0;
-                cr += (t >= r * tpr && t < (r + 1) * tpr) ? v : 0;
+#pragma unroll
+            for (int t = 0; t < kCMaxCluster; ++t) {
+                tot += v[t];
+                pre += t < tile ? v[t] : 0;
+                cp += t < r * tpr ? v[t] : 0;
+                cr += (t >= r * tpr && t < (r + 1) * tpr) ? v[t] : 0;
             }
             tpre[e] = pre;
             colp[e] = cp;
@@ -408,7 +419,10 @@ layout_cluster_kernel(LayoutArgs a, int64_t tile_len, int steps) {
         carry += chunk;
     }
     if (threadIdx.x == 0) ebase[E] = carry;
-    cluster.sync();   // no block reads another block's shared memory past this point
+    // This block reads no other block's shared memory from here on; it keeps its own
+    // (which the others may still be reading) until the matching wait at the end.
+    cluster_arrive_release();
+    __syncthreads();
 
     const int64_t R = ebase[E];
     if (tile == 0) {
@@ -425,22 +439,23 @@ layout_cluster_kernel(LayoutArgs a, int64_t tile_len, int steps) {
         }
     }
 #pragma unroll
-    for (int st = 0; st < kCMaxSteps; ++st) {
+    for (int st = 0; st < STEPS; ++st) {
         const int64_t l = wlo + st * 32 + lane;
-        if (st >= steps || l >= hi) continue;
+        if (l >= hi) continue;
         const int64_t s = base + l;
-        const int e = ev[st];
-        if (e < 0) {
+        if (pk[st] == 0u) {
             a.dst_row[s] = -1;
             a.occ[s] = -1;
             continue;
         }
-        const int32_t within = tpre[e] + mine[e] + rk[st];
+        const int e = (int)(pk[st] & 2047u) - 1;
+        const int32_t within = tpre[e] + mine[e] + (int32_t)(pk[st] >> 11);
         const int64_t row = ebase[e] + within;
         a.occ[s] = within - colp[e];
         a.dst_row[s] = (int32_t)row;
         if (row < a.rows_cap) a.assist[row] = (int32_t)s;
     }
+    cluster_wait_acquire();
 }
 
 // Cluster path geometry: tiles per rank and slots per tile, or false if the problem does
@@ -453,8 +468,11 @@ bool cluster_geometry(const moedisp_dims& d, int* tpr, int64_t* tile_len, int* s
     if ((int64_t)d.W * t > kCMaxCluster) return false;
     *tpr = (int)t;
     *tile_len = (P + t - 1) / t;
-    *steps = (int)((*tile_len + kCThreads - 1) / kCThreads);
-    return *steps <= kCMaxSteps;
+    const int need_steps = (int)((*tile_len + kCThreads - 1) / kCThreads);
+    int p2 = 1;
+    while (p2 < need_steps) p2 <<= 1;
+    *steps = p2;
+    return p2 <= kCMaxSteps;
 }
 
 size_t cluster_smem(int E) {
@@ -462,23 +480,23 @@ size_t cluster_smem(int E) {
 }
 
 // Whether a cluster of C blocks of this kernel can be resident on the current device.
-cudaError_t cluster_fits(int C, size_t smem, bool* ok) {
+cudaError_t cluster_fits(const void* kernel, int C, size_t smem, bool* ok) {
     static std::mutex mu;
-    static std::map<std::tuple<int, int, size_t>, bool> cache;
+    static std::map<std::tuple<int, const void*, int, size_t>, bool> cache;
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
     {
         std::lock_guard<std::mutex> lock(mu);
-        auto it = cache.find({dev, C, smem});
+        auto it = cache.find({dev, kernel, C, smem});
         if (it != cache.end()) {
             *ok = it->second;
             return cudaSuccess;
         }
     }
-    err = allow_dynamic_smem((const void*)layout_cluster_kernel);
+    err = allow_dynamic_smem(kernel);
     if (err != cudaSuccess) return err;
-    err = cudaFuncSetAttribute(layout_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    err = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
@@ -492,13 +510,13 @@ cudaError_t cluster_fits(int C, size_t smem, bool* ok) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    err = cudaOccupancyMaxActiveClusters(&n, (const void*)layout_cluster_kernel, &cfg);
+    err = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg);
     if (err != cudaSuccess) {
         (void)cudaGetLastError();
         n = 0;
     }
     std::lock_guard<std::mutex> lock(mu);
-    cache[{dev, C, smem}] = n > 0;
+    cache[{dev, kernel, C, smem}] = n > 0;
     *ok = n > 0;
     return cudaSuccess;
 }
@@ -557,14 +575,17 @@ cudaError_t launch_layout(const int32_t* expert_ids, const uint8_t* active,
     if (cluster_geometry(dims, &tpr_c, &tile_c, &steps_c)) {
         const int C = dims.W * tpr_c;
         const size_t smem = cluster_smem(dims.E);
+        void (*kernel)(LayoutArgs, int64_t) =
+            steps_c == 1 ? layout_cluster_kernel<1> : steps_c == 2 ? layout_cluster_kernel<2>
+            : steps_c == 4 ? layout_cluster_kernel<4> : steps_c == 8 ? layout_cluster_kernel<8>
+                           : layout_cluster_kernel<16>;
         bool ok = false;
-        cudaError_t err = cluster_fits(C, smem, &ok);
+        cudaError_t err = cluster_fits((const void*)kernel, C, smem, &ok);
         if (err != cudaSuccess) return err;
         if (ok) {
             a.tiles_per_rank = tpr_c;
             a.n_tiles = C;
-            return launch_pdl(layout_cluster_kernel, dim3(C), dim3(kCThreads), smem, stream, C, a,
-                              tile_c, steps_c);
+            return launch_pdl(kernel, dim3(C), dim3(kCThreads), smem, stream, C, a, tile_c);
         }
     }
 
