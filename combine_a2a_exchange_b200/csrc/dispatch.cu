@@ -41,7 +41,7 @@ struct DispatchArgs {
 };
 
 constexpr int kCopyThreads = 32;        // bf16 copy: one warp per block
-constexpr int kQuantWarps = 4;          // quantising copy: independent warps per block
+constexpr int kQuantMaxWarps = 8;       // quantising copy: up to 8 independent warps per block
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
@@ -205,11 +205,11 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
 // shuffles, quantises the row into one of its two output buffers, and lanes 0..K-1
 // write the quantised row (and the scale) to the token's K rows.
 template <int Q>
-__global__ void __launch_bounds__(kQuantWarps * 32) dispatch_quant_kernel(DispatchArgs a) {
+__global__ void __launch_bounds__(kQuantMaxWarps * 32) dispatch_quant_kernel(DispatchArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ __align__(8) uint64_t bars[kQuantWarps][kMaxStages];
-    __shared__ int64_t tok[kQuantWarps][kMaxStages];
-    __shared__ int32_t drow[kQuantWarps][kMaxStages][MOEDISP_MAX_K];
+    __shared__ __align__(8) uint64_t bars[kQuantMaxWarps][kMaxStages];
+    __shared__ int64_t tok[kQuantMaxWarps][kMaxStages];
+    __shared__ int32_t drow[kQuantMaxWarps][kMaxStages][MOEDISP_MAX_K];
     constexpr float kQmax = Q == MOEDISP_QUANT_INT8 ? 127.0f : 448.0f;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int S = a.stages, K = a.K;
@@ -226,8 +226,9 @@ __global__ void __launch_bounds__(kQuantWarps * 32) dispatch_quant_kernel(Dispat
     grid_dep_launch_dependents();
     write_recv_counts(a);
 
-    const int64_t n_warps = (int64_t)gridDim.x * kQuantWarps;
-    int64_t next_g = (int64_t)blockIdx.x * kQuantWarps + warp;
+    const int wpb = blockDim.x >> 5;
+    const int64_t n_warps = (int64_t)gridDim.x * wpb;
+    int64_t next_g = (int64_t)blockIdx.x * wpb + warp;
     auto fill = [&](int st) {
         while (true) {
             if (next_g >= a.G) {
@@ -326,21 +327,24 @@ cudaError_t launch_copy(DispatchArgs a, cudaStream_t stream) {
 
 template <int Q>
 cudaError_t launch_quant(DispatchArgs a, cudaStream_t stream) {
-    // Per warp: S input stages and two output buffers; aim for two blocks per SM.
-    const size_t per_warp_budget = 110 * 1024 / kQuantWarps;
+    // Per warp: S input stages and two output buffers. Two stages when a row is large,
+    // up to four when it is small; then as many warps per block as fit about 200 KB.
     const size_t fixed = 2 * (size_t)a.out_bytes;
-    int S = (int)((per_warp_budget - std::min(per_warp_budget, fixed)) / a.in_bytes);
-    S = std::max(2, std::min(S, 4));
+    const size_t small = 25 * 1024;
+    int S = 2;
+    if (2 * (size_t)a.in_bytes + fixed <= small)
+        S = (int)std::min<size_t>(4, (small - fixed) / a.in_bytes);
     a.stages = S;
-    const size_t smem = (size_t)kQuantWarps * ((size_t)S * a.in_bytes + fixed);
+    const size_t per_warp = (size_t)S * a.in_bytes + fixed;
+    const int wpb = (int)std::max<size_t>(1, std::min<size_t>(kQuantMaxWarps, (200 * 1024) / per_warp));
+    const size_t smem = (size_t)wpb * per_warp;
     int per_sm = 1;
-    cudaError_t err = blocks_per_sm((const void*)dispatch_quant_kernel<Q>, kQuantWarps * 32, smem,
-                                    &per_sm);
+    cudaError_t err = blocks_per_sm((const void*)dispatch_quant_kernel<Q>, wpb * 32, smem, &per_sm);
     if (err != cudaSuccess) return err;
     int64_t grid = (int64_t)current_sm_count() * per_sm;
-    grid = std::min<int64_t>(grid, std::max<int64_t>((a.G + kQuantWarps - 1) / kQuantWarps, 1));
-    return launch_pdl(dispatch_quant_kernel<Q>, dim3((unsigned)grid), dim3(kQuantWarps * 32), smem,
-                      stream, 1, a);
+    grid = std::min<int64_t>(grid, std::max<int64_t>((a.G + wpb - 1) / wpb, 1));
+    return launch_pdl(dispatch_quant_kernel<Q>, dim3((unsigned)grid), dim3(wpb * 32), smem, stream,
+                      1, a);
 }
 
 }  // namespace
