@@ -4,8 +4,9 @@ One step = one pass of the whole path over one batch of the ``cfg2`` workload (W
 virtual EP ranks x T=256 tokens, H=4096 bf16, E=64, K=8): dispatch layout (2 kernels),
 exchange plan of the layout's send counts (1 kernel), dispatch copy (1 kernel), combine
 (1 kernel) with the dispatched rows as the experts' outputs (identity expert). Inputs are
-resident in HBM when the timed region starts; L2 is flushed (a 512 MiB write) before
-every timed step, outside the per-step CUDA-event pair.
+resident in HBM when the timed region starts; L2 is flushed before every timed step
+(a 512 MiB write, then a 256 MiB read of another buffer so no dirty line is left to be
+written back), outside the per-step CUDA-event pair.
 
 Prints ONE JSON line (rank 0). ``value`` = tokens/s over all ranks (each rank runs an
 independent replica: weak scaling, no data-path collective); ``e2e`` = the same metric
@@ -37,7 +38,8 @@ import numpy as np  # noqa: E402
 METRIC = "dispatch+combine tokens/s and achieved HBM GB/s (% of B200 peak), 1 GPU"
 UNIT = "tokens/s"
 FALLBACK_HBM_GBS = 6650.0
-L2_FLUSH_BYTES = 512 << 20
+L2_FLUSH_BYTES = 512 << 20     # written, then a separate 256 MiB buffer is read
+L2_READ_BYTES = 256 << 20
 LAUNCHES_PER_STEP = 5          # layout (2 kernels), plan, dispatch, combine
 
 
@@ -222,6 +224,22 @@ def capture(torch, fn):
     return g
 
 
+class L2Flush:
+    """Writes a 512 MiB buffer (> 4x L2), then reads a separate 256 MiB one: the read
+    evicts the dirty lines of the write, so the timed region starts with L2 holding
+    nothing of ours and nothing left to write back."""
+
+    def __init__(self, torch, device):
+        self.w = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=device)
+        self.r = torch.ones(L2_READ_BYTES // 4, dtype=torch.int32, device=device)
+        self.sink = torch.empty((), dtype=torch.int64, device=device)
+
+    def zero_(self):
+        self.w.zero_()
+        torch_sum = self.r.sum()
+        self.sink.copy_(torch_sum)
+
+
 def time_graph(torch, g, reps, warmup, flush):
     """CUDA-event time (ms) of each of `reps` replays, L2 flushed before each."""
     E = torch.cuda.Event
@@ -340,7 +358,7 @@ def config_of(w, flush_note=True):
                      f"E={w.E}, K={w.K}, quant={'none' if w.quant_mode == 0 else w.quant_mode}",
          "global_batch": w.G, "seq_len": 1, "parallelism": "ep-virtual (one GPU)"}
     if flush_note:
-        c["l2"] = "flushed (512 MiB write) before every timed step"
+        c["l2"] = "flushed before every timed step (512 MiB write, then 256 MiB read of another buffer)"
     return c
 
 
@@ -349,7 +367,7 @@ def config_of(w, flush_note=True):
 def op_sweep(md, torch, device, hbm, reps=10):
     import workloads as wl
     out = []
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=device)
+    flush = L2Flush(torch, device)
     for name in ("cfg3", "cfg4"):
         w = wl.moe_workload(name, seed=0)
         st = MoEStep(md, torch, w, device)
@@ -450,7 +468,7 @@ def main():
     over = {} if args.T is None else {"T": args.T}
     w = wl.moe_workload(args.workload, seed=rank, **over)
     step = MoEStep(md, torch, w, device)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=device)
+    flush = L2Flush(torch, device)
 
     uuid = None
     try:

@@ -41,7 +41,7 @@ struct DispatchArgs {
 };
 
 constexpr int kCopyThreads = 32;        // bf16 copy: one warp per block
-constexpr int kQuantMaxWarps = 8;       // quantising copy: up to 8 independent warps per block
+constexpr int kQuantThreads = 128;      // quantising copy: block size
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
@@ -54,31 +54,61 @@ __device__ __forceinline__ float absmax8(const uint4& v) {
     return m;
 }
 
-// q = clamp(rint(x / scale), -127, 127), x / scale an IEEE fp32 divide.
-__device__ __forceinline__ uint32_t q_int8_pair(uint32_t w, float scale) {
-    int a = __float2int_rn(__fdiv_rn(bf16_lo(w), scale));
-    int b = __float2int_rn(__fdiv_rn(bf16_hi(w), scale));
-    a = max(-127, min(127, a));
-    b = max(-127, min(127, b));
+// Quantisation. The definition is q = clamp(rint(x / scale), -127, 127) for int8 and
+// q = e4m3_rn_satfinite(x / scale) for fp8, with x / scale one IEEE fp32 division. The
+// quotient is only needed near a rounding boundary of q, so it is first approximated
+// by r = x * inv, inv = 1 / scale (both correctly rounded): then
+//   |r - x/scale| <= |x/scale| * (2^-23 + 2^-48)  and  |fl(x/scale) - x/scale| <= |x/scale| * 2^-24,
+// i.e. r and the IEEE quotient differ by at most ~3 units in the last place of fp32.
+// When r is farther than that from every rounding boundary of q, both round to the same
+// q; otherwise (and for inv or r not finite) the IEEE quotient is computed. The result
+// is the definition's bit for bit; the fast test only decides which path gives it.
+
+// int8 boundaries are the half-integers; |x/scale| <= ~127, so the bound above is below
+// 2.3e-5 and a margin of 2^-14 from k + 0.5 is safe.
+__device__ __forceinline__ int q_int8(float x, float scale, float inv) {
+    float v = __fmul_rn(x, inv);
+    const float t = v - floorf(v);
+    if (!(fabsf(t - 0.5f) >= 0.00006103515625f)) v = __fdiv_rn(x, scale);
+    const int q = __float2int_rn(v);
+    return max(-127, min(127, q));
+}
+
+// E4M3 keeps 3 mantissa bits: for 2^-6 <= |v| < 448 its rounding boundaries are the fp32
+// values whose 20 low mantissa bits are exactly 0x80000; r is used when it is more than
+// 16 fp32 ulps from one. E4M3's subnormal range and the saturation edge take the exact
+// path.
+__device__ __forceinline__ float q_e4m3_value(float x, float scale, float inv) {
+    const float r = __fmul_rn(x, inv);
+    const uint32_t u = __float_as_uint(r) & 0x7fffffffu;
+    const int32_t d = (int32_t)(u & 0xfffffu) - 0x80000;
+    const bool clear = u >= 0x3c800000u && u < 0x43e00000u && (d > 16 || d < -16);
+    return clear ? r : __fdiv_rn(x, scale);
+}
+
+__device__ __forceinline__ uint32_t q_int8_pair(uint32_t w, float scale, float inv) {
+    const int a = q_int8(bf16_lo(w), scale, inv);
+    const int b = q_int8(bf16_hi(w), scale, inv);
     return (uint32_t)(a & 0xff) | ((uint32_t)(b & 0xff) << 8);
 }
 
-// e4m3(x / scale), round to nearest even, saturating to +-448 (hardware conversion).
-__device__ __forceinline__ uint32_t q_e4m3_pair(uint32_t w, float scale) {
-    const float2 f = make_float2(__fdiv_rn(bf16_lo(w), scale), __fdiv_rn(bf16_hi(w), scale));
+// Round to nearest even, saturating to +-448 (hardware conversion).
+__device__ __forceinline__ uint32_t q_e4m3_pair(uint32_t w, float scale, float inv) {
+    const float2 f = make_float2(q_e4m3_value(bf16_lo(w), scale, inv),
+                                 q_e4m3_value(bf16_hi(w), scale, inv));
     return (uint32_t)__nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3);
 }
 
 template <int Q>
-__device__ __forceinline__ uint2 quant8(const uint4& v, float scale, bool zero) {
+__device__ __forceinline__ uint2 quant8(const uint4& v, float scale, float inv, bool zero) {
     if (zero) return make_uint2(0u, 0u);
     uint32_t p0, p1, p2, p3;
     if (Q == MOEDISP_QUANT_INT8) {
-        p0 = q_int8_pair(v.x, scale); p1 = q_int8_pair(v.y, scale);
-        p2 = q_int8_pair(v.z, scale); p3 = q_int8_pair(v.w, scale);
+        p0 = q_int8_pair(v.x, scale, inv); p1 = q_int8_pair(v.y, scale, inv);
+        p2 = q_int8_pair(v.z, scale, inv); p3 = q_int8_pair(v.w, scale, inv);
     } else {
-        p0 = q_e4m3_pair(v.x, scale); p1 = q_e4m3_pair(v.y, scale);
-        p2 = q_e4m3_pair(v.z, scale); p3 = q_e4m3_pair(v.w, scale);
+        p0 = q_e4m3_pair(v.x, scale, inv); p1 = q_e4m3_pair(v.y, scale, inv);
+        p2 = q_e4m3_pair(v.z, scale, inv); p3 = q_e4m3_pair(v.w, scale, inv);
     }
     return make_uint2(p0 | (p1 << 16), p2 | (p3 << 16));
 }
@@ -199,42 +229,44 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
     if (issuer) bulk_wait<0>();
 }
 
-// Quantising dispatch: every warp is an independent pipeline over its own tokens, with
-// its own stages, barriers and output buffers, so no block-wide barrier is needed per
-// token. Lane 0 streams token rows in; the warp reduces the row's max |x| with
-// shuffles, quantises the row into one of its two output buffers, and lanes 0..K-1
-// write the quantised row (and the scale) to the token's K rows.
+// Quantising dispatch: a block of kQuantThreads threads takes its tokens one at a time.
+// Warp 0's lane 0 streams token rows into kMaxStages-deep shared-memory stages; the block
+// reduces each row's max |x|, quantises the row into one of two output buffers, and
+// lanes 0..K-1 write the quantised row (and the scale) to the token's K rows with bulk
+// stores. Two block barriers per token: after the partial maxima (which also carries
+// the time-out verdict of the stage wait) and after the quantised row is complete.
 template <int Q>
-__global__ void __launch_bounds__(kQuantMaxWarps * 32) dispatch_quant_kernel(DispatchArgs a) {
+__global__ void __launch_bounds__(kQuantThreads) dispatch_quant_kernel(DispatchArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ __align__(8) uint64_t bars[kQuantMaxWarps][kMaxStages];
-    __shared__ int64_t tok[kQuantMaxWarps][kMaxStages];
-    __shared__ int32_t drow[kQuantMaxWarps][kMaxStages][MOEDISP_MAX_K];
+    __shared__ __align__(8) uint64_t bars[kMaxStages];
+    __shared__ int64_t tok[kMaxStages];
+    __shared__ int32_t drow[kMaxStages][MOEDISP_MAX_K];
+    __shared__ float red[kQuantThreads / 32];
+    __shared__ int abort_s;
     constexpr float kQmax = Q == MOEDISP_QUANT_INT8 ? 127.0f : 448.0f;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    constexpr int NW = kQuantThreads / 32;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int S = a.stages, K = a.K;
-    uint8_t* inbuf = smem + (size_t)warp * (S * a.in_bytes + 2 * a.out_bytes);
-    uint8_t* outbuf = inbuf + (size_t)S * a.in_bytes;
-    uint64_t* wbar = bars[warp];
+    uint8_t* inbuf = smem;
+    uint8_t* outbuf = smem + (size_t)S * a.in_bytes;
 
-    if (lane == 0) {
-        for (int s = 0; s < S; ++s) mbar_init(&wbar[s], 1);
+    if (tid == 0) {
+        for (int s = 0; s < S; ++s) mbar_init(&bars[s], 1);
         fence_mbar_init();
+        abort_s = 0;
     }
-    __syncwarp();
+    __syncthreads();
     grid_dep_wait();
     grid_dep_launch_dependents();
     write_recv_counts(a);
 
-    const int wpb = blockDim.x >> 5;
-    const int64_t n_warps = (int64_t)gridDim.x * wpb;
-    int64_t next_g = (int64_t)blockIdx.x * wpb + warp;
-    auto fill = [&](int st) {
+    int64_t next_g = blockIdx.x;
+    auto fill = [&](int st) {          // warp 0 only
         while (true) {
             if (next_g >= a.G) {
                 if (lane == 0) {
-                    tok[warp][st] = -1;
-                    mbar_arrive(&wbar[st]);
+                    tok[st] = -1;
+                    mbar_arrive(&bars[st]);
                 }
                 return;
             }
@@ -254,59 +286,62 @@ __global__ void __launch_bounds__(kQuantMaxWarps * 32) dispatch_quant_kernel(Dis
                 if (lane == 0) {
 #pragma unroll
                     for (int k = 0; k < MOEDISP_MAX_K; ++k)
-                        if (k < K) drow[warp][st][k] = dk[k];
-                    tok[warp][st] = next_g;
-                    mbar_arrive_expect_tx(&wbar[st], a.in_bytes);
+                        if (k < K) drow[st][k] = dk[k];
+                    tok[st] = next_g;
+                    mbar_arrive_expect_tx(&bars[st], a.in_bytes);
                     bulk_load(inbuf + (size_t)st * a.in_bytes, a.x + next_g * a.in_bytes,
-                              a.in_bytes, &wbar[st]);
+                              a.in_bytes, &bars[st]);
                 }
-                next_g += n_warps;
+                next_g += gridDim.x;
                 return;
             }
-            next_g += n_warps;
+            next_g += gridDim.x;
         }
     };
 
-    for (int st = 0; st < S; ++st) fill(st);
-    const bool issuer = lane < K;
+    if (warp == 0)
+        for (int st = 0; st < S; ++st) fill(st);
+    const bool issuer = warp == 0 && lane < K;
     const int nvec = a.H >> 3;
     for (int it = 0;; ++it) {
         const int st = it % S;
         const uint32_t par = (uint32_t)((it / S) & 1);
-        int ok = 1;
-        if (lane == 0) ok = mbar_wait(&wbar[st], par) ? 1 : 0;
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) {
-            if (lane == 0) raise_status(a.status, MOEDISP_STATUS_TIMEOUT);
-            break;
-        }
-        (void)mbar_wait(&wbar[st], par);
-        const int64_t g = tok[warp][st];
-        if (g < 0) break;
+        if (!mbar_wait(&bars[st], par)) abort_s = 1;
         const uint4* v = reinterpret_cast<const uint4*>(inbuf + (size_t)st * a.in_bytes);
         float m = 0.0f;
-        for (int c = lane; c < nvec; c += 32) m = fmaxf(m, absmax8(v[c]));
+        for (int c = tid; c < nvec; c += kQuantThreads) m = fmaxf(m, absmax8(v[c]));
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        const float scale = __fdiv_rn(m, kQmax);
-        const bool zero = m == 0.0f;
-        if (issuer) bulk_wait_read<1>();      // output buffer it % 2 is free again
-        __syncwarp();
-        uint8_t* ob = outbuf + (size_t)(it & 1) * a.out_bytes;
-        uint2* o2 = reinterpret_cast<uint2*>(ob);
-        for (int c = lane; c < nvec; c += 32) o2[c] = quant8<Q>(v[c], scale, zero);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (issuer) {
-            const int32_t d = drow[warp][st][lane];
-            if (d >= 0) {
-                bulk_store(a.expand_x + (int64_t)d * a.out_bytes, ob, a.out_bytes);
-                a.scales[d] = scale;
-            }
-            bulk_commit();
+        if (lane == 0) red[warp] = m;
+        if (issuer) bulk_wait_read<1>();        // output buffer it % 2 is free again
+        __syncthreads();
+        if (abort_s) {
+            if (tid == 0) raise_status(a.status, MOEDISP_STATUS_TIMEOUT);
+            break;
         }
-        __syncwarp();
-        fill(st);                               // the warp is done reading stage st
+        if (tok[st] < 0) break;
+        float amax = red[0];
+#pragma unroll
+        for (int w = 1; w < NW; ++w) amax = fmaxf(amax, red[w]);
+        const float scale = __fdiv_rn(amax, kQmax);
+        const float inv = __frcp_rn(scale);
+        const bool zero = amax == 0.0f;
+        uint2* o2 = reinterpret_cast<uint2*>(outbuf + (size_t)(it & 1) * a.out_bytes);
+        for (int c = tid; c < nvec; c += kQuantThreads) o2[c] = quant8<Q>(v[c], scale, inv, zero);
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (warp == 0) {
+            if (issuer) {
+                const int32_t d = drow[st][lane];
+                if (d >= 0) {
+                    bulk_store(a.expand_x + (int64_t)d * a.out_bytes, o2, a.out_bytes);
+                    a.scales[d] = scale;
+                }
+                bulk_commit();
+            }
+            __syncwarp();
+            fill(st);                           // every thread is done reading stage st
+        }
     }
     if (issuer) bulk_wait<0>();
 }
@@ -327,24 +362,22 @@ cudaError_t launch_copy(DispatchArgs a, cudaStream_t stream) {
 
 template <int Q>
 cudaError_t launch_quant(DispatchArgs a, cudaStream_t stream) {
-    // Per warp: S input stages and two output buffers. Two stages when a row is large,
-    // up to four when it is small; then as many warps per block as fit about 200 KB.
+    // S input stages (4 when a stage is small, down to 2) and two output buffers, about
+    // 56 KB per block for the largest rows here, so that four blocks share an SM.
     const size_t fixed = 2 * (size_t)a.out_bytes;
-    const size_t small = 25 * 1024;
-    int S = 2;
-    if (2 * (size_t)a.in_bytes + fixed <= small)
-        S = (int)std::min<size_t>(4, (small - fixed) / a.in_bytes);
+    const size_t budget = 56 * 1024;
+    int S = (int)((budget - std::min(budget, fixed)) / a.in_bytes);
+    S = std::max(2, std::min(S, 4));
     a.stages = S;
-    const size_t per_warp = (size_t)S * a.in_bytes + fixed;
-    const int wpb = (int)std::max<size_t>(1, std::min<size_t>(kQuantMaxWarps, (200 * 1024) / per_warp));
-    const size_t smem = (size_t)wpb * per_warp;
+    const size_t smem = (size_t)S * a.in_bytes + fixed;
     int per_sm = 1;
-    cudaError_t err = blocks_per_sm((const void*)dispatch_quant_kernel<Q>, wpb * 32, smem, &per_sm);
+    cudaError_t err = blocks_per_sm((const void*)dispatch_quant_kernel<Q>, kQuantThreads, smem,
+                                    &per_sm);
     if (err != cudaSuccess) return err;
     int64_t grid = (int64_t)current_sm_count() * per_sm;
-    grid = std::min<int64_t>(grid, std::max<int64_t>((a.G + wpb - 1) / wpb, 1));
-    return launch_pdl(dispatch_quant_kernel<Q>, dim3((unsigned)grid), dim3(wpb * 32), smem, stream,
-                      1, a);
+    grid = std::min<int64_t>(grid, std::max<int64_t>(a.G, 1));
+    return launch_pdl(dispatch_quant_kernel<Q>, dim3((unsigned)grid), dim3(kQuantThreads), smem,
+                      stream, 1, a);
 }
 
 }  // namespace

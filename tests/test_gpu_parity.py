@@ -353,6 +353,30 @@ def test_fp8_conversion_exhaustive_over_bf16(md):
     assert np.array_equal(got, exp)
 
 
+def test_int8_half_integer_ties(md):
+    """Rows whose largest magnitude is 127 have scale exactly 1, so x / scale = x: rows of
+    half-integers k + 0.5 sit exactly on int8 rounding boundaries (round half to even)
+    and values a few ulps off them sit next to one."""
+    rng = np.random.default_rng(0)
+    T, H = 96, 256
+    k = rng.integers(-127, 127, size=(T, H)).astype(np.float32)
+    vals = k + 0.5
+    near = rng.random((T, H)) < 0.3
+    vals[near] = np.nextafter(vals[near], np.where(rng.random(near.sum()) < 0.5, -1e9, 1e9)).astype(np.float32)
+    x = wl.f32_to_bf16_bits(vals)
+    x[:, 0] = wl.f32_to_bf16_bits(np.float32(127.0))
+    w = wl.MoEWorkload(name="ties", W=1, T=T, H=H, E=2, K=2, quant_mode=2, x_bits=x,
+                       expert_ids=np.tile(np.array([[0, 1]], np.int32), (T, 1)),
+                       weights=np.full((T, 2), 0.5, np.float32), active=None)
+    L, _ = run_layout(md, w)
+    ref = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, None)
+    full, scales, gr, _, _, st = run_dispatch(md, w, L, 2)
+    assert st == 0
+    rex, rsc, _ = oracle.moe_dispatch(x, ref["dst_row"], w.K, ref["rows_cap"], 2)
+    assert (rsc == 1.0).all()
+    assert np.array_equal(full.cpu().numpy()[gr:gr + ref["R"]], rex[:ref["R"]])
+
+
 def test_dispatch_capacity_guard(md):
     w = wl.moe_workload("tiny", seed=8, W=2, T=100, K=4, E=8, H=64)
     cap = 500                                                      # R = 800
