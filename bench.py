@@ -231,8 +231,8 @@ class L2Flush:
 
     def __init__(self, torch, device):
         self.w = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=device)
-        self.r = torch.ones(L2_READ_BYTES // 4, dtype=torch.int32, device=device)
-        self.sink = torch.empty((), dtype=torch.int64, device=device)
+        self.r = torch.ones(L2_READ_BYTES // 4, dtype=torch.float32, device=device)
+        self.sink = torch.empty((), dtype=torch.float32, device=device)
 
     def zero_(self):
         self.w.zero_()
