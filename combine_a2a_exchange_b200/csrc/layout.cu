@@ -8,13 +8,14 @@
 //
 //  kernel 1 (layout_hist_kernel): slots are cut into tiles of kTile slots that never
 //    straddle a source rank. Each block counts its tile per expert with a
-//    warp-aggregated shared-memory histogram (__match_any_sync groups the lanes that
-//    share an expert; the group's lowest lane adds the group size), writes the tile's
+//    warp-aggregated shared-memory histogram (the lanes that share an expert are found
+//    with one ballot per bit of the expert id; the group's lowest lane adds the group
+//    size), writes the tile's
 //    counts and clears the tile's look-back words. The last block to finish (atomic
 //    ticket after a fence) reduces the tiles to cnt[r][e], scans over source ranks
 //    (colprefix) and over experts (expert_base, rank_base), and forms send_splits.
 //  kernel 2 (layout_scatter_kernel): blocks take tiles in ticket order. Each warp ranks
-//    its part of the tile with __match_any_sync + popcount of the lower peers, on top of
+//    its part of the tile by the popcount of its lower peers (same ballots), on top of
 //    a per-warp running count; the warps' counts are scanned per expert; the tile's
 //    per-expert offset among all earlier tiles comes from a decoupled look-back (each
 //    tile publishes its aggregate, then walks back over predecessors' status words in
@@ -96,12 +97,36 @@ __device__ __forceinline__ uint32_t ld_relaxed(const uint32_t* p) {
 // out-of-range id.
 __device__ __forceinline__ int slot_expert(const LayoutArgs& a, int64_t s, bool& bad) {
     const int e = __ldg(a.ids + s);
-    if (a.active != nullptr && __ldg(a.active + s / a.K) == 0) return -1;
+    // s < 2^30 (checked on the host), so a 32-bit division finds the token.
+    if (a.active != nullptr && __ldg(a.active + (uint32_t)s / (uint32_t)a.K) == 0) return -1;
     if (e < 0 || e >= a.E) {
         bad = true;
         return -1;
     }
     return e;
+}
+
+// Lanes of the warp whose key equals this lane's key (0 <= key < 2^bits): the AND, over
+// the key's bits, of the ballot of lanes agreeing with this lane on that bit. `bits` must
+// be the same in every lane. One ballot per bit, no match instruction.
+__device__ __forceinline__ unsigned peers_by_ballot(unsigned key, int bits) {
+    unsigned m = 0xffffffffu;
+#pragma unroll
+    for (int b = 0; b < 11; ++b) {
+        if (b < bits) {
+            const unsigned bit = (key >> b) & 1u;
+            const unsigned bal = __ballot_sync(0xffffffffu, bit);
+            m &= bit ? bal : ~bal;
+        }
+    }
+    return m;
+}
+
+// Bits needed for the keys 0..E (expert + 1, 0 = no expert).
+__host__ __device__ __forceinline__ int key_bits(int E) {
+    int b = 1;
+    while ((1 << b) <= E) ++b;
+    return b;
 }
 
 __device__ void layout_finalize(const LayoutArgs& a, int32_t* smem) {
@@ -171,13 +196,14 @@ __global__ void __launch_bounds__(kThreads) layout_hist_kernel(LayoutArgs a) {
     const int lane = threadIdx.x & 31;
 
     int32_t* hist = smem;
+    const int kb = key_bits(a.E);
     for (int e = threadIdx.x; e < a.E; e += blockDim.x) hist[e] = 0;
     __syncthreads();
     bool bad = false;
     for (int64_t l0 = lo; l0 < hi; l0 += blockDim.x) {
         const int64_t l = l0 + threadIdx.x;
         const int e = l < hi ? slot_expert(a, base + l, bad) : -1;
-        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        const unsigned peers = peers_by_ballot((unsigned)(e + 1), kb);
         if (e >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[e], __popc(peers));
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) raise_status(a.status, MOEDISP_STATUS_BAD_EXPERT_ID);
@@ -226,10 +252,11 @@ __global__ void __launch_bounds__(kThreads) layout_scatter_kernel(LayoutArgs a) 
         ev[st] = l < hi ? slot_expert(a, base + l, bad) : -1;
     }
     // Rank within the warp's part, in slot order, on top of the warp's running counts.
+    const int kb = key_bits(E);
 #pragma unroll
     for (int st = 0; st < kSteps; ++st) {
         const int e = ev[st];
-        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        const unsigned peers = peers_by_ballot((unsigned)(e + 1), kb);
         const int before = e >= 0 ? mine[e] : 0;
         __syncwarp();
         if (e >= 0 && lane == __ffs(peers) - 1) mine[e] = before + __popc(peers);
@@ -368,10 +395,11 @@ layout_cluster_kernel(LayoutArgs a, int64_t tile_len) {
     __syncthreads();
     // Rank within the warp's slots, in slot order: packed as (rank << 11) | (expert + 1).
     uint32_t pk[STEPS];
+    const int kb = key_bits(E);
 #pragma unroll
     for (int st = 0; st < STEPS; ++st) {
         const int e = ev[st];
-        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        const unsigned peers = peers_by_ballot((unsigned)(e + 1), kb);
         const int before = e >= 0 ? mine[e] : 0;
         __syncwarp();
         if (e >= 0 && lane == __ffs(peers) - 1) mine[e] = before + __popc(peers);
