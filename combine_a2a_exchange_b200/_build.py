@@ -1,6 +1,7 @@
 """Builds libmoedisp.so in-tree with nvcc for sm_100a (B200).
 
-Usage: ``python -m combine_a2a_exchange_b200._build [--force] [--verbose-ptxas]``.
+Usage: ``python combine_a2a_exchange_b200/_build.py [--force] [--verbose-ptxas]`` (run by
+path: importing the package needs the library this script builds).
 Objects go to ``_build/`` next to the sources; the shared library lands in the package
 directory so that it travels with the source tree.
 """

@@ -14,8 +14,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="session")
 def md():
-    from combine_a2a_exchange_b200 import _build
-    _build.build_library()
+    import __graft_entry__
+    __graft_entry__.build()
     import combine_a2a_exchange_b200 as md
     return md
 
