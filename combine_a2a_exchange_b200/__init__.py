@@ -18,7 +18,7 @@ LIBRARY_PATH = os.path.join(_HERE, "libmoedisp.so")
 
 if not os.path.exists(LIBRARY_PATH):
     raise ImportError(
-        f"{LIBRARY_PATH} is missing: build it with `python -m combine_a2a_exchange_b200._build` "
+        f"{LIBRARY_PATH} is missing: build it with `python combine_a2a_exchange_b200/_build.py` "
         "(or __graft_entry__.build()); this package has no fallback implementation")
 
 _lib = ctypes.CDLL(LIBRARY_PATH)
@@ -36,6 +36,8 @@ STATUS_CAPACITY = 1
 STATUS_BAD_EXPERT_ID = 2
 STATUS_TIMEOUT = 4
 STATUS_BAD_SPLIT = 8
+
+NOALLOC_SCRATCH_BYTES = 2 << 20
 
 QUANT_NONE = 0
 QUANT_INT8 = 2
@@ -70,6 +72,8 @@ _a2a_v = _sig("moedisp_a2a_v", [_P, _I64, _P, _I64, _I64, _I, _P, _P, _P, _P, _P
 _ws_size = _sig("moedisp_layout_workspace_size", [Dims, ctypes.POINTER(ctypes.c_size_t)])
 _layout = _sig("moedisp_moe_dispatch_layout",
                [_P, _P, Dims, ctypes.POINTER(Layout), _P, ctypes.c_size_t, _P, _P])
+_layout_noalloc = _sig("moedisp_moe_dispatch_layout_noalloc",
+                       [_P, _P, Dims, ctypes.POINTER(Layout), _P, _P])
 _dispatch = _sig("moedisp_moe_dispatch",
                  [_P, _I, Dims, ctypes.POINTER(Layout), _I, _P, _P, _P, _I, _P, _P, _P])
 _combine = _sig("moedisp_moe_combine", [_P, _I, Dims, ctypes.POINTER(Layout), _P, _P, _P, _P])
@@ -193,6 +197,16 @@ def moe_dispatch_layout(expert_ids, active_mask, layout: LayoutBuffers, status, 
     return _check(rc, "moe_dispatch_layout", raise_on_error)
 
 
+def moe_dispatch_layout_noalloc(expert_ids, active_mask, layout: LayoutBuffers, status,
+                                stream=None, raise_on_error=True) -> int:
+    """moe_dispatch_layout without a workspace argument: the scratch lives in the
+    library's own device memory (see include/moedisp.h). Allocates nothing."""
+    L = layout.struct()
+    rc = _layout_noalloc(_ptr(expert_ids), _ptr(active_mask), layout.dims, ctypes.byref(L),
+                         _ptr(status), _stream(stream))
+    return _check(rc, "moe_dispatch_layout_noalloc", raise_on_error)
+
+
 def moe_dispatch(x, H, layout: LayoutBuffers, quant_mode, expand_x, dynamic_scales, status,
                  expert_token_nums=None, expert_token_nums_type=1, ep_recv_counts=None,
                  stream=None, raise_on_error=True) -> int:
@@ -214,13 +228,15 @@ def moe_combine(expert_out, H, layout: LayoutBuffers, expert_scales, y, status, 
 def raw_call(name: str, *args) -> int:
     """Calls an exported C function with already-marshalled arguments (for ABI tests)."""
     return int({"moedisp_a2a_exchange_plan": _plan, "moedisp_a2a_v": _a2a_v,
-                "moedisp_moe_dispatch_layout": _layout, "moedisp_moe_dispatch": _dispatch,
-                "moedisp_moe_combine": _combine}[name](*args))
+                "moedisp_moe_dispatch_layout": _layout,
+                "moedisp_moe_dispatch_layout_noalloc": _layout_noalloc,
+                "moedisp_moe_dispatch": _dispatch, "moedisp_moe_combine": _combine}[name](*args))
 
 
 __all__ = [
     "a2a_exchange_plan", "a2a_v", "layout_workspace_size", "LayoutBuffers",
-    "moe_dispatch_layout", "moe_dispatch", "moe_combine", "status_string", "version",
+    "moe_dispatch_layout", "moe_dispatch_layout_noalloc", "moe_dispatch", "moe_combine",
+    "status_string", "version", "NOALLOC_SCRATCH_BYTES",
     "Dims", "Layout", "MoedispError", "LIBRARY_PATH",
     "QUANT_NONE", "QUANT_INT8", "QUANT_FP8_E4M3",
     "STATUS_CAPACITY", "STATUS_BAD_EXPERT_ID", "STATUS_TIMEOUT", "STATUS_BAD_SPLIT",

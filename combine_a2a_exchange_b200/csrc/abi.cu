@@ -178,6 +178,38 @@ int moedisp_moe_dispatch_layout(const int32_t* expert_ids, const uint8_t* active
     return rc(moedisp::launch_layout(expert_ids, active_mask, dims, L, workspace, status, stream));
 }
 
+int moedisp_moe_dispatch_layout_noalloc(const int32_t* expert_ids, const uint8_t* active_mask,
+                                        moedisp_dims dims, const moedisp_layout* layout,
+                                        int32_t* status, moedisp_stream_t stream) {
+    if (!layout || !status) return MOEDISP_ERR_NULLPTR;
+    int c = check_dims(dims);
+    if (c != MOEDISP_OK) return c;
+    const moedisp_layout& L = *layout;
+    if ((c = check_rows_cap(L.rows_cap)) != MOEDISP_OK) return c;
+    const int64_t slots = (int64_t)dims.W * dims.T * dims.K;
+    if (!L.cnt || !L.expert_base || !L.rank_base || !L.send_splits) return MOEDISP_ERR_NULLPTR;
+    if (slots > 0 && (!expert_ids || !L.occ || !L.dst_row)) return MOEDISP_ERR_NULLPTR;
+    if (L.rows_cap > 0 && !L.assist_info) return MOEDISP_ERR_NULLPTR;
+    if (moedisp::layout_geometry(dims).total_bytes > moedisp::layout_noalloc_scratch_bytes())
+        return MOEDISP_ERR_UNSUPPORTED;
+    if (!aligned(expert_ids, 4) || !aligned(L.cnt, 4) || !aligned(L.occ, 4) ||
+        !aligned(L.dst_row, 4) || !aligned(L.assist_info, 4) || !aligned(L.expert_base, 8) ||
+        !aligned(L.rank_base, 8) || !aligned(L.send_splits, 8) || !aligned(status, 4))
+        return MOEDISP_ERR_MISALIGNED;
+    const int64_t G = (int64_t)dims.W * dims.T;
+    if (any_alias({{L.cnt, (size_t)dims.W * dims.E * 4},
+                   {L.occ, (size_t)slots * 4},
+                   {L.dst_row, (size_t)slots * 4},
+                   {L.assist_info, (size_t)L.rows_cap * 4},
+                   {L.expert_base, (size_t)(dims.E + 1) * 8},
+                   {L.rank_base, (size_t)(dims.W + 1) * 8},
+                   {L.send_splits, (size_t)dims.W * dims.W * 8},
+                   {status, 4}},
+                  {{expert_ids, (size_t)slots * 4}, {active_mask, (size_t)G}}))
+        return MOEDISP_ERR_ALIASED;
+    return rc(moedisp::launch_layout_noalloc(expert_ids, active_mask, dims, L, status, stream));
+}
+
 int moedisp_moe_dispatch(const void* x, int H, moedisp_dims dims,
                          const moedisp_layout* layout, int quant_mode, void* expand_x,
                          float* dynamic_scales, int64_t* expert_token_nums,

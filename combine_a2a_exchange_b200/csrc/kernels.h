@@ -72,6 +72,12 @@ cudaError_t launch_layout(const int32_t* expert_ids, const uint8_t* active,
                           const moedisp_dims& dims, const moedisp_layout& layout,
                           void* workspace, int32_t* status, cudaStream_t stream);
 
+// Allocation-free layout: the two-kernel path on the library's static scratch array.
+size_t layout_noalloc_scratch_bytes();
+cudaError_t launch_layout_noalloc(const int32_t* expert_ids, const uint8_t* active,
+                                  const moedisp_dims& dims, const moedisp_layout& layout,
+                                  int32_t* status, cudaStream_t stream);
+
 cudaError_t launch_dispatch(const void* x, int H, const moedisp_dims& dims,
                             const moedisp_layout& layout, int quant_mode, void* expand_x,
                             float* dynamic_scales, int64_t* expert_token_nums,

@@ -549,6 +549,27 @@ cudaError_t cluster_fits(const void* kernel, int C, size_t smem, bool* ok) {
     return cudaSuccess;
 }
 
+// Launches the two-kernel path (histogram, then ranking + look-back + scatter) on the
+// workspace pointers already in `a`.
+cudaError_t launch_tiled(LayoutArgs& a, const moedisp_dims& dims, const LayoutGeometry& g,
+                         cudaStream_t stream) {
+    const size_t fin_base = (size_t)(dims.E + 1) * sizeof(int64_t);
+    const size_t fin_cnt = (size_t)dims.W * dims.E * sizeof(int32_t);
+    a.cnt_in_smem = fin_base + fin_cnt <= kFinalizeSmemLimit;
+    size_t smem1 = std::max((size_t)dims.E * sizeof(int32_t), fin_base + (a.cnt_in_smem ? fin_cnt : 0));
+    smem1 = (smem1 + 15) & ~(size_t)15;
+    const size_t smem2 = (size_t)(kWarps + 1) * dims.E * sizeof(int32_t);
+
+    cudaError_t err = allow_dynamic_smem((const void*)layout_hist_kernel);
+    if (err != cudaSuccess) return err;
+    err = allow_dynamic_smem((const void*)layout_scatter_kernel);
+    if (err != cudaSuccess) return err;
+    err = launch_pdl(layout_hist_kernel, dim3((unsigned)g.n_tiles), dim3(kThreads), smem1, stream, 1, a);
+    if (err != cudaSuccess) return err;
+    return launch_pdl(layout_scatter_kernel, dim3((unsigned)g.n_tiles), dim3(kThreads), smem2, stream,
+                      1, a);
+}
+
 }  // namespace
 
 LayoutGeometry layout_geometry(const moedisp_dims& d) {
@@ -568,10 +589,10 @@ LayoutGeometry layout_geometry(const moedisp_dims& d) {
     return g;
 }
 
-cudaError_t launch_layout(const int32_t* expert_ids, const uint8_t* active,
-                          const moedisp_dims& dims, const moedisp_layout& L, void* workspace,
-                          int32_t* status, cudaStream_t stream) {
-    const LayoutGeometry g = layout_geometry(dims);
+namespace {
+LayoutArgs make_args(const int32_t* expert_ids, const uint8_t* active, const moedisp_dims& dims,
+                     const moedisp_layout& L, void* workspace, int32_t* status,
+                     const LayoutGeometry& g) {
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     LayoutArgs a;
     a.ids = expert_ids;
@@ -597,6 +618,15 @@ cudaError_t launch_layout(const int32_t* expert_ids, const uint8_t* active,
     a.lookback = reinterpret_cast<uint32_t*>(ws + g.off_lookback);
     a.colprefix = reinterpret_cast<int32_t*>(ws + g.off_colprefix);
     a.status = status;
+    return a;
+}
+}  // namespace
+
+cudaError_t launch_layout(const int32_t* expert_ids, const uint8_t* active,
+                          const moedisp_dims& dims, const moedisp_layout& L, void* workspace,
+                          int32_t* status, cudaStream_t stream) {
+    const LayoutGeometry g = layout_geometry(dims);
+    LayoutArgs a = make_args(expert_ids, active, dims, L, workspace, status, g);
 
     int tpr_c = 0, steps_c = 0;
     int64_t tile_c = 0;
@@ -617,21 +647,56 @@ cudaError_t launch_layout(const int32_t* expert_ids, const uint8_t* active,
         }
     }
 
-    const size_t fin_base = (size_t)(dims.E + 1) * sizeof(int64_t);
-    const size_t fin_cnt = (size_t)dims.W * dims.E * sizeof(int32_t);
-    a.cnt_in_smem = fin_base + fin_cnt <= kFinalizeSmemLimit;
-    size_t smem1 = std::max((size_t)dims.E * sizeof(int32_t), fin_base + (a.cnt_in_smem ? fin_cnt : 0));
-    smem1 = (smem1 + 15) & ~(size_t)15;
-    const size_t smem2 = (size_t)(kWarps + 1) * dims.E * sizeof(int32_t);
+    return launch_tiled(a, dims, g, stream);
+}
 
-    cudaError_t err = allow_dynamic_smem((const void*)layout_hist_kernel);
+// ------------------------------------------------------------ allocation-free variant
+//
+// Scratch of moedisp_moe_dispatch_layout_noalloc: the two-kernel path's workspace kept in
+// this library's own device memory (present on every GPU that loads the library, until
+// the process exits), so the caller passes no workspace and nothing is allocated.
+static __device__ __align__(256) unsigned char g_layout_scratch[MOEDISP_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+// Device address of g_layout_scratch on the current device. The host-side name of a
+// __device__ array is only a stand-in, so the address is looked up once per device
+// (with that device current) and cached.
+cudaError_t layout_scratch_address(void** out) {
+    static std::mutex mu;
+    static std::map<int, void*> cache;
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
-    err = allow_dynamic_smem((const void*)layout_scatter_kernel);
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(dev);
+    if (it != cache.end()) {
+        *out = it->second;
+        return cudaSuccess;
+    }
+    void* p = nullptr;
+    err = cudaGetSymbolAddress(&p, g_layout_scratch);
     if (err != cudaSuccess) return err;
-    err = launch_pdl(layout_hist_kernel, dim3((unsigned)g.n_tiles), dim3(kThreads), smem1, stream, 1, a);
+    cache[dev] = p;
+    *out = p;
+    return cudaSuccess;
+}
+}  // namespace
+
+size_t layout_noalloc_scratch_bytes() { return MOEDISP_NOALLOC_SCRATCH_BYTES; }
+
+cudaError_t launch_layout_noalloc(const int32_t* expert_ids, const uint8_t* active,
+                                  const moedisp_dims& dims, const moedisp_layout& L,
+                                  int32_t* status, cudaStream_t stream) {
+    const LayoutGeometry g = layout_geometry(dims);
+    void* scratch = nullptr;
+    cudaError_t err = layout_scratch_address(&scratch);
     if (err != cudaSuccess) return err;
-    return launch_pdl(layout_scatter_kernel, dim3((unsigned)g.n_tiles), dim3(kThreads), smem2, stream,
-                      1, a);
+    // The array keeps whatever the previous call left: clear the two counters that must
+    // start at zero (every other scratch word is written before it is read).
+    err = cudaMemsetAsync(scratch, 0, 256, stream);
+    if (err != cudaSuccess) return err;
+    LayoutArgs a = make_args(expert_ids, active, dims, L, scratch, status, g);
+    return launch_tiled(a, dims, g, stream);
 }
 
 }  // namespace moedisp

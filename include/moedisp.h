@@ -165,6 +165,32 @@ int moedisp_moe_dispatch_layout(const int32_t *expert_ids, const uint8_t *active
                                 void *workspace, size_t workspace_bytes, int32_t *status,
                                 moedisp_stream_t stream);
 
+/* moe_dispatch_layout_noalloc
+ *
+ * The same computation and outputs as moe_dispatch_layout, for callers that cannot
+ * allocate device memory for the workspace: code running under an allocator that owns
+ * all device memory and forbids side allocations, code inside a region where
+ * allocation is not allowed (for example while a stream is being captured), or embedded
+ * and real-time callers that must not allocate after start-up. (The source pages have no
+ * counterpart; their APIs always take a caller-allocated workspace.)
+ * Instead of a workspace argument it uses a scratch array of
+ * MOEDISP_NOALLOC_SCRATCH_BYTES that lives in this library's own device memory: every
+ * GPU that loads the library holds it until the process exits. It always runs the
+ * two-kernel path (histogram, then ranking + look-back + scatter) on that array.
+ *  - Dims whose workspace (moedisp_layout_workspace_size) exceeds
+ *    MOEDISP_NOALLOC_SCRATCH_BYTES are rejected with MOEDISP_ERR_UNSUPPORTED.
+ *  - It calls no allocating routine. The first call on a device looks up the array's
+ *    device address (once per device, with that device current); make that first call
+ *    before any stream capture.
+ *  - All calls share the one array, which keeps the last call's contents; each call
+ *    clears what must start at zero. Calls that overlap on the GPU (on different streams,
+ *    or from different threads) race on the array and must not be made.
+ * Other arguments and errors are those of moedisp_moe_dispatch_layout. */
+#define MOEDISP_NOALLOC_SCRATCH_BYTES (2u << 20)
+int moedisp_moe_dispatch_layout_noalloc(const int32_t *expert_ids, const uint8_t *active_mask,
+                                        moedisp_dims dims, const moedisp_layout *layout,
+                                        int32_t *status, moedisp_stream_t stream);
+
 /* Quantisation modes of moe_dispatch (the Ascend quantMode values; 3 is this library's
  * fp8 variant of the same per-token dynamic scheme). */
 #define MOEDISP_QUANT_NONE      0

@@ -1,0 +1,69 @@
+"""The allocation-free layout entry point, moedisp_moe_dispatch_layout_noalloc.
+
+It serves callers that cannot allocate device memory for a workspace (an allocator that
+owns all device memory, a region where allocation is not allowed, a real-time caller
+that allocates nothing after start-up): its scratch is an array inside the library's own
+device memory. The test calls it through the C ABI and checks that every output equals
+what the regular entry point (with a caller-allocated workspace) produces, on two calls
+in a row with different inputs -- so a stale counter or flag left in the shared array by
+the first call would show up in the second. The file's name makes pytest collect it last.
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def md():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import combine_a2a_exchange_b200 as md
+    return md
+
+
+def _outputs(L):
+    return {k: getattr(L, k).cpu().numpy() for k in
+            ("cnt", "occ", "dst_row", "assist_info", "expert_base", "rank_base", "send_splits")}
+
+
+def test_noalloc_layout_matches_regular_entry_point(md):
+    shapes = [dict(W=4, T=1500, K=6, E=24, active_p=0.7), dict(W=4, T=1500, K=6, E=24)]
+    for call, over in enumerate(shapes):
+        w = wl.moe_workload("tiny", seed=900 + call, **over)
+        ids = torch.from_numpy(w.expert_ids.reshape(-1)).cuda()
+        act = None if w.active is None else torch.from_numpy(w.active).cuda()
+
+        ref = md.LayoutBuffers.allocate(w.W, w.T, w.K, w.E)
+        st_ref = torch.zeros(1, dtype=torch.int32, device="cuda")
+        md.moe_dispatch_layout(ids, act, ref, st_ref)
+
+        got = md.LayoutBuffers.allocate(w.W, w.T, w.K, w.E)
+        for t in (got.cnt, got.occ, got.dst_row, got.assist_info, got.expert_base,
+                  got.rank_base, got.send_splits):
+            t.fill_(-7)
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        md.moe_dispatch_layout_noalloc(ids, act, got, st)
+        torch.cuda.synchronize()
+
+        assert int(st.item()) == 0 and int(st_ref.item()) == 0
+        a, b = _outputs(got), _outputs(ref)
+        R = int(b["expert_base"][-1])
+        for k in ("cnt", "occ", "dst_row", "expert_base", "rank_base", "send_splits"):
+            assert np.array_equal(a[k], b[k]), (call, k)
+        assert np.array_equal(a["assist_info"][:R], b["assist_info"][:R]), call
+
+
+def test_noalloc_layout_rejects_oversized_problems(md):
+    # E = 1024 experts over 8 ranks with 2^20 slots needs more scratch than the array holds
+    W, T, K, E = 8, 16384, 8, 1024
+    assert md.layout_workspace_size(W, T, K, E) > md.NOALLOC_SCRATCH_BYTES
+    L = md.Layout(1 << 40, 1 << 41, 1 << 42, 1 << 43, 1 << 44, 1 << 45, 1 << 46, W * T * K)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    import ctypes
+    rc = md.raw_call("moedisp_moe_dispatch_layout_noalloc", 1 << 47, None, md.Dims(W, T, K, E),
+                     ctypes.byref(L), st.data_ptr(), None)
+    assert rc == md.MOEDISP_ERR_UNSUPPORTED
