@@ -63,8 +63,10 @@ cudaError_t launch_a2a_v(const void* in, int64_t in_rank_stride_rows, void* out,
 struct LayoutGeometry {
     int64_t slots_per_rank;   // T*K
     int tiles_per_rank;
+    int64_t tile_len;         // slots per tile
+    int steps;                // 32-slot steps per warp (a power of two)
     int64_t n_tiles;
-    size_t off_tile_hist, off_lookback, off_colprefix, total_bytes;
+    size_t off_tile_hist, off_tile_prefix, total_bytes;
 };
 LayoutGeometry layout_geometry(const moedisp_dims& d);
 
@@ -72,7 +74,7 @@ cudaError_t launch_layout(const int32_t* expert_ids, const uint8_t* active,
                           const moedisp_dims& dims, const moedisp_layout& layout,
                           void* workspace, int32_t* status, cudaStream_t stream);
 
-// Allocation-free layout: the two-kernel path on the library's static scratch array.
+// Allocation-free layout: the tiled path on the library's static scratch array.
 size_t layout_noalloc_scratch_bytes();
 cudaError_t launch_layout_noalloc(const int32_t* expert_ids, const uint8_t* active,
                                   const moedisp_dims& dims, const moedisp_layout& layout,

@@ -1,33 +1,32 @@
 // MoE dispatch layout: a stable counting sort of the G*K (token, expert) slots by expert.
 //
-// The PyTorch symm_mem change computes the same thing in three separate pieces: a
-// per-rank histogram of the top-k ids (torch.histc), the 0-based occurrence number of
-// every slot (get_occurrence_numbers, an n_unique x n indicator matrix and a cumsum) and
-// a one-block 2-D exchange plan (make2dExchangePlan) whose per-expert destination offsets
-// the index-push kernel adds to the occurrence number. Here one pass does all of it:
+// The PyTorch symm_mem change computes the same thing in separate pieces: a per-rank
+// histogram of the top-k ids (torch.histc), the 0-based occurrence number of every slot
+// (get_occurrence_numbers, an n_unique x n indicator matrix and a cumsum) and a one-block
+// 2-D exchange plan (make2dExchangePlan) whose per-expert destination offsets the
+// index-push kernel adds to the occurrence number. Here the slots are cut into tiles that
+// never straddle a source rank, and:
 //
-//  kernel 1 (layout_hist_kernel): slots are cut into tiles of kTile slots that never
-//    straddle a source rank. Each block counts its tile per expert with a
-//    warp-aggregated shared-memory histogram (the lanes that share an expert are found
-//    with one ballot per bit of the expert id; the group's lowest lane adds the group
-//    size), writes the tile's
-//    counts and clears the tile's look-back words. The last block to finish (atomic
-//    ticket after a fence) reduces the tiles to cnt[r][e], scans over source ranks
-//    (colprefix) and over experts (expert_base, rank_base), and forms send_splits.
-//  kernel 2 (layout_scatter_kernel): blocks take tiles in ticket order. Each warp ranks
-//    its part of the tile by the popcount of its lower peers (same ballots), on top of
-//    a per-warp running count; the warps' counts are scanned per expert; the tile's
-//    per-expert offset among all earlier tiles comes from a decoupled look-back (each
-//    tile publishes its aggregate, then walks back over predecessors' status words in
-//    windows of kWindow until it meets an inclusive prefix); finally every slot is
-//    scattered: dst_row, occ and assist_info.
+//  * small problems (at most 16 tiles of at most 2048 slots): one kernel, one thread-block
+//    cluster. Each 1024-thread block ranks its tile (below), the blocks exchange their
+//    per-expert tile counts through distributed shared memory across the cluster barrier,
+//    and every block derives its tile offsets, the expert bases and the per-rank counts
+//    from them -- no global scratch, no second launch.
+//  * larger problems: three kernels, each spread over the whole GPU.
+//      count: one block per tile; a warp-aggregated shared-memory histogram -> the tile's
+//             counts per expert;
+//      scan:  one block per 32 experts; exclusive scans down the tiles -> per (tile,
+//             expert) offsets and the expert totals;
+//      rank:  one block per tile; ranks its slots (this needs only the inputs, so it runs
+//             before waiting for the scan), then reads four rows of offsets, scans the
+//             totals into expert bases and scatters dst_row, occ and assist_info.
 //
-// When the whole problem fits one thread-block cluster (at most 16 rank-aligned tiles of
-// at most 16384 slots), a single kernel replaces both: one 1024-thread block per tile
-// ranks its slots as above, the blocks exchange their per-expert tile counts through
-// distributed shared memory across the cluster barrier, and every block derives its
-// tile offsets, the expert bases and the per-rank counts from those counts directly --
-// no global scratch, no second launch, no look-back.
+// Ranking: each warp owns consecutive slots and walks them 32 at a time. The lanes that
+// share an expert are found with one ballot per bit of (expert + 1) (a warp-level
+// multisplit); a slot's rank is the popcount of its lower peers plus the warp's running
+// count of that expert in shared memory, which the group's lowest lane then advances.
+// Per expert, the warps' counts are scanned in warp order. Everything is in slot order,
+// so the sort is stable and the result deterministic.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -43,22 +42,17 @@ namespace cg = cooperative_groups;
 namespace moedisp {
 
 namespace {
-constexpr int kTile = 2048;
+// Tiled (three-kernel) path.
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kSlotsPerWarp = kTile / kWarps;
-constexpr int kSteps = kSlotsPerWarp / 32;
-constexpr int kWindow = 16;
-constexpr uint32_t kFlagAggregate = 1u << 30;
-constexpr uint32_t kFlagInclusive = 2u << 30;
-constexpr uint32_t kValueMask = (1u << 30) - 1;
-// Shared memory that kernel 1's last block may use to hold cnt while it scans.
-constexpr size_t kFinalizeSmemLimit = 160 * 1024;
+constexpr int64_t kTargetTiles = 296;         // about two blocks per SM
+constexpr int kScanThreads = 1024;
+constexpr int kScanRows = 256;                // tiles per pass of the scan kernel
 // Single-kernel cluster path.
 constexpr int kCThreads = 1024;
 constexpr int kCWarps = kCThreads / 32;
-constexpr int kCMaxSteps = 16;                          // 32-slot steps per warp
-constexpr int64_t kCMaxTile = (int64_t)kCWarps * 32 * kCMaxSteps;   // 16384 slots
+constexpr int kCMaxSteps = 2;                 // tiles <= 2048 slots
+constexpr int64_t kCMaxTile = (int64_t)kCWarps * 32 * kCMaxSteps;
 constexpr int kCMaxCluster = 16;
 
 struct LayoutArgs {
@@ -68,7 +62,7 @@ struct LayoutArgs {
     int64_t P;                 // slots per source rank, T*K
     int tiles_per_rank;
     int n_tiles;
-    int cnt_in_smem;
+    int64_t tile_len;          // slots per tile (the last tile of a rank may be shorter)
     int32_t* cnt;
     int32_t* occ;
     int32_t* dst_row;
@@ -77,21 +71,10 @@ struct LayoutArgs {
     int64_t* rank_base;
     int64_t* send_splits;
     int64_t rows_cap;
-    uint32_t* counters;        // [0] blocks done in kernel 1, [1] tile ticket of kernel 2
-    int32_t* tile_hist;        // [n_tiles][E]
-    uint32_t* lookback;        // [n_tiles][E]
-    int32_t* colprefix;        // [W][E] slots of expert e in source ranks < r
+    int32_t* tile_hist;        // [n_tiles][E]      counts of each tile
+    int32_t* tile_prefix;      // [n_tiles + 1][E]  counts in earlier tiles; last row = totals
     int32_t* status;
 };
-
-__device__ __forceinline__ void st_relaxed(uint32_t* p, uint32_t v) {
-    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ uint32_t ld_relaxed(const uint32_t* p) {
-    uint32_t v;
-    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
 
 // Expert of slot s if the slot is active, else -1. `bad` is set for an active token's
 // out-of-range id.
@@ -129,34 +112,181 @@ __host__ __device__ __forceinline__ int key_bits(int E) {
     return b;
 }
 
-__device__ void layout_finalize(const LayoutArgs& a, int32_t* smem) {
-    __shared__ int64_t warp_tot[32];
-    const int W = a.W, E = a.E, tpr = a.tiles_per_rank;
-    int64_t* ebase = reinterpret_cast<int64_t*>(smem);            // [E + 1]
-    int32_t* cnt_s = reinterpret_cast<int32_t*>(ebase + E + 1);   // [W * E] if it fits
-    int32_t* cnt_src = a.cnt_in_smem ? cnt_s : a.cnt;
+// Loads the expert of each of this lane's STEPS slots (-1 where none) and ranks them
+// within the warp: packed (rank << 11) | (expert + 1), 0 for no expert. `mine` is the
+// warp's running count per expert (shared memory, zeroed by the caller).
+template <int STEPS>
+__device__ __forceinline__ void rank_in_warp(const LayoutArgs& a, int64_t base, int64_t wlo,
+                                             int64_t hi, int32_t* mine, uint32_t (&pk)[STEPS]) {
+    const int lane = threadIdx.x & 31;
+    const unsigned lower = (1u << lane) - 1u;
+    int ev[STEPS];
+    bool bad = false;
+#pragma unroll
+    for (int st = 0; st < STEPS; ++st) {
+        const int64_t l = wlo + st * 32 + lane;
+        ev[st] = l < hi ? slot_expert(a, base + l, bad) : -1;
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) raise_status(a.status, MOEDISP_STATUS_BAD_EXPERT_ID);
+    const int kb = key_bits(a.E);
+#pragma unroll
+    for (int st = 0; st < STEPS; ++st) {
+        const int e = ev[st];
+        const unsigned peers = peers_by_ballot((unsigned)(e + 1), kb);
+        const int before = e >= 0 ? mine[e] : 0;
+        __syncwarp();
+        if (e >= 0 && lane == __ffs(peers) - 1) mine[e] = before + __popc(peers);
+        __syncwarp();
+        pk[st] = e >= 0 ? ((uint32_t)(before + __popc(peers & lower)) << 11) | (uint32_t)(e + 1) : 0u;
+    }
+}
 
-    // cnt[r][e]: sum of the tile counts of rank r.
-    for (int idx = threadIdx.x; idx < W * E; idx += blockDim.x) {
-        const int r = idx / E, e = idx - r * E;
-        const int32_t* th = a.tile_hist + (int64_t)r * tpr * E + e;
-        int32_t sum = 0;
-#pragma unroll 8
-        for (int c = 0; c < tpr; ++c) sum += __ldcg(th + (int64_t)c * E);
-        a.cnt[idx] = sum;
-        if (a.cnt_in_smem) cnt_s[idx] = sum;
+// Writes dst_row, occ and assist_info of this lane's slots. `pre` = slots of each expert
+// before this tile, `colp` = before this rank, `mine` = before this warp inside the tile.
+template <int STEPS>
+__device__ __forceinline__ void scatter_slots(const LayoutArgs& a, int64_t base, int64_t wlo,
+                                              int64_t hi, const uint32_t (&pk)[STEPS],
+                                              const int32_t* pre, const int32_t* colp,
+                                              const int32_t* mine, const int64_t* ebase) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int st = 0; st < STEPS; ++st) {
+        const int64_t l = wlo + st * 32 + lane;
+        if (l >= hi) continue;
+        const int64_t s = base + l;
+        if (pk[st] == 0u) {
+            a.dst_row[s] = -1;
+            a.occ[s] = -1;
+            continue;
+        }
+        const int e = (int)(pk[st] & 2047u) - 1;
+        const int32_t within = pre[e] + mine[e] + (int32_t)(pk[st] >> 11);
+        const int64_t row = ebase[e] + within;
+        a.occ[s] = within - colp[e];
+        a.dst_row[s] = (int32_t)row;
+        if (row < a.rows_cap) a.assist[row] = (int32_t)s;
+    }
+}
+
+// --------------------------------------------------------------- tiled path
+
+template <int STEPS>
+__global__ void __launch_bounds__(kThreads) layout_count_kernel(LayoutArgs a) {
+    extern __shared__ __align__(16) int32_t hist[];          // [E]
+    const int tile = blockIdx.x;
+    const int r = tile / a.tiles_per_rank, c = tile - r * a.tiles_per_rank;
+    const int64_t base = (int64_t)r * a.P;
+    const int64_t lo = (int64_t)c * a.tile_len, hi = min64(lo + a.tile_len, a.P);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int e = threadIdx.x; e < a.E; e += blockDim.x) hist[e] = 0;
+    __syncthreads();
+    grid_dep_wait();
+    grid_dep_launch_dependents();
+    const int64_t wlo = lo + (int64_t)warp * STEPS * 32;
+    int ev[STEPS];
+    bool bad = false;
+#pragma unroll
+    for (int st = 0; st < STEPS; ++st) {
+        const int64_t l = wlo + st * 32 + lane;
+        ev[st] = l < hi ? slot_expert(a, base + l, bad) : -1;
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) raise_status(a.status, MOEDISP_STATUS_BAD_EXPERT_ID);
+    const int kb = key_bits(a.E);
+#pragma unroll
+    for (int st = 0; st < STEPS; ++st) {
+        const int e = ev[st];
+        const unsigned peers = peers_by_ballot((unsigned)(e + 1), kb);
+        if (e >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[e], __popc(peers));
     }
     __syncthreads();
-    // Per expert: prefix over source ranks, total; then exclusive scan over experts.
+    int32_t* th = a.tile_hist + (int64_t)tile * a.E;
+    for (int e = threadIdx.x; e < a.E; e += blockDim.x) th[e] = hist[e];
+}
+
+// Exclusive scan of tile_hist down each column (expert), 32 columns per block, in
+// passes of kScanRows tiles; warp w scans column w of the pass, 32 tiles per step.
+__global__ void __launch_bounds__(kScanThreads) layout_scan_kernel(LayoutArgs a) {
+    __shared__ int32_t col[kScanRows][33];
+    grid_dep_wait();
+    grid_dep_launch_dependents();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int e = blockIdx.x * 32 + lane;
+    const bool valid = e < a.E;
+    const int n = a.n_tiles;
+    int32_t carry = 0;                                       // column `warp`'s running sum
+    for (int t0 = 0; t0 < n; t0 += kScanRows) {
+        const int rows = min(kScanRows, n - t0);
+        for (int i = warp; i < rows; i += kScanThreads / 32)
+            col[i][lane] = valid ? a.tile_hist[(int64_t)(t0 + i) * a.E + e] : 0;
+        __syncthreads();
+        for (int q = 0; q < rows; q += 32) {
+            const int i = q + lane;
+            const int32_t v = i < rows ? col[i][warp] : 0;
+            const int32_t inc = warp_inclusive_scan_i32(v);
+            if (i < rows) col[i][warp] = carry + inc - v;
+            carry += __shfl_sync(0xffffffffu, inc, 31);
+        }
+        __syncthreads();
+        for (int i = warp; i < rows; i += kScanThreads / 32)
+            if (valid) a.tile_prefix[(int64_t)(t0 + i) * a.E + e] = col[i][lane];
+        __syncthreads();
+    }
+    const int ec = blockIdx.x * 32 + warp;                   // totals row
+    if (lane == 0 && ec < a.E) a.tile_prefix[(int64_t)n * a.E + ec] = carry;
+}
+
+template <int STEPS>
+__global__ void __launch_bounds__(kThreads) layout_rank_kernel(LayoutArgs a) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    __shared__ int64_t warp_tot[32];
+    const int E = a.E, W = a.W, tpr = a.tiles_per_rank;
+    const int ES = E | 1;
+    int64_t* ebase = reinterpret_cast<int64_t*>(smem_raw);      // [E + 1]
+    int32_t* wc = reinterpret_cast<int32_t*>(ebase + E + 1);    // [kWarps][ES]
+    int32_t* pre = wc + kWarps * ES;                             // [E]
+    int32_t* colp = pre + E;                                     // [E]
+    int32_t* cntr = colp + E;                                    // [E]
+    const int tile = blockIdx.x;
+    const int r = tile / tpr, c = tile - r * tpr;
+    const int64_t base = (int64_t)r * a.P;
+    const int64_t lo = (int64_t)c * a.tile_len, hi = min64(lo + a.tile_len, a.P);
+    const int warp = threadIdx.x >> 5;
+    for (int i = threadIdx.x; i < kWarps * ES; i += blockDim.x) wc[i] = 0;
+    __syncthreads();
+
+    // Ranking reads only the layout's inputs. They were complete before the count kernel
+    // passed its own dependency wait, which precedes this kernel's start, so this part
+    // overlaps the count and scan kernels.
+    int32_t* mine = wc + warp * ES;
+    const int64_t wlo = lo + (int64_t)warp * STEPS * 32;
+    uint32_t pk[STEPS];
+    rank_in_warp<STEPS>(a, base, wlo, hi, mine, pk);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int32_t run = 0;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            const int32_t t = wc[w * ES + e];
+            wc[w * ES + e] = run;
+            run += t;
+        }
+    }
+
+    grid_dep_wait();
+    grid_dep_launch_dependents();
+    const int32_t* tp = a.tile_prefix;
+    const int64_t row_tile = (int64_t)tile * E, row_rank = (int64_t)r * tpr * E;
+    const int64_t row_next = (int64_t)(r + 1) * tpr * E, row_tot = (int64_t)a.n_tiles * E;
     int64_t carry = 0;
-    for (int base = 0; base < E; base += blockDim.x) {
-        const int e = base + threadIdx.x;
+    for (int b0 = 0; b0 < E; b0 += blockDim.x) {
+        const int e = b0 + threadIdx.x;
         int64_t tot = 0;
         if (e < E) {
-            for (int r = 0; r < W; ++r) {
-                a.colprefix[(int64_t)r * E + e] = (int32_t)tot;
-                tot += a.cnt_in_smem ? cnt_s[r * E + e] : __ldcg(cnt_src + (int64_t)r * E + e);
-            }
+            pre[e] = __ldcg(tp + row_tile + e);
+            const int32_t cp = __ldcg(tp + row_rank + e);
+            colp[e] = cp;
+            cntr[e] = __ldcg(tp + row_next + e) - cp;
+            tot = __ldcg(tp + row_tot + e);
         }
         int64_t chunk;
         const int64_t ex = block_exclusive_scan(tot, warp_tot, chunk);
@@ -165,187 +295,25 @@ __device__ void layout_finalize(const LayoutArgs& a, int32_t* smem) {
     }
     if (threadIdx.x == 0) ebase[E] = carry;
     __syncthreads();
+
     const int64_t R = ebase[E];
-    for (int e = threadIdx.x; e <= E; e += blockDim.x) a.expert_base[e] = ebase[e];
-    for (int d = threadIdx.x; d <= W; d += blockDim.x) a.rank_base[d] = d < W ? ebase[d * a.ne] : R;
-    for (int idx = threadIdx.x; idx < W * W; idx += blockDim.x) {
-        const int r = idx / W, d = idx - r * W;
-        int64_t sum = 0;
-        for (int le = 0; le < a.ne; ++le) {
-            const int e = d * a.ne + le;
-            sum += a.cnt_in_smem ? cnt_s[r * E + e] : __ldcg(cnt_src + (int64_t)r * E + e);
+    if (tile == 0) {
+        for (int e = threadIdx.x; e <= E; e += blockDim.x) a.expert_base[e] = ebase[e];
+        for (int d = threadIdx.x; d <= W; d += blockDim.x) a.rank_base[d] = d < W ? ebase[d * a.ne] : R;
+        if (threadIdx.x == 0 && R > a.rows_cap) raise_status(a.status, MOEDISP_STATUS_CAPACITY);
+    }
+    if (c == 0) {
+        for (int e = threadIdx.x; e < E; e += blockDim.x) a.cnt[(int64_t)r * E + e] = cntr[e];
+        for (int d = threadIdx.x; d < W; d += blockDim.x) {
+            int64_t sum = 0;
+            for (int le = 0; le < a.ne; ++le) sum += cntr[d * a.ne + le];
+            a.send_splits[(int64_t)r * W + d] = sum;
         }
-        a.send_splits[idx] = sum;
     }
-    if (threadIdx.x == 0) {
-        if (R > a.rows_cap) raise_status(a.status, MOEDISP_STATUS_CAPACITY);
-        a.counters[0] = 0;   // ready for the next call
-        a.counters[1] = 0;   // tile ticket of kernel 2
-    }
+    scatter_slots<STEPS>(a, base, wlo, hi, pk, pre, colp, mine, ebase);
 }
 
-__global__ void __launch_bounds__(kThreads) layout_hist_kernel(LayoutArgs a) {
-    extern __shared__ __align__(16) int32_t smem[];
-    __shared__ int is_last;
-    grid_dep_wait();
-    grid_dep_launch_dependents();
-    const int tile = blockIdx.x;
-    const int r = tile / a.tiles_per_rank, c = tile - r * a.tiles_per_rank;
-    const int64_t base = (int64_t)r * a.P;
-    const int64_t lo = (int64_t)c * kTile, hi = min64(lo + kTile, a.P);
-    const int lane = threadIdx.x & 31;
-
-    int32_t* hist = smem;
-    const int kb = key_bits(a.E);
-    for (int e = threadIdx.x; e < a.E; e += blockDim.x) hist[e] = 0;
-    __syncthreads();
-    bool bad = false;
-    for (int64_t l0 = lo; l0 < hi; l0 += blockDim.x) {
-        const int64_t l = l0 + threadIdx.x;
-        const int e = l < hi ? slot_expert(a, base + l, bad) : -1;
-        const unsigned peers = peers_by_ballot((unsigned)(e + 1), kb);
-        if (e >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[e], __popc(peers));
-    }
-    if (__any_sync(0xffffffffu, bad) && lane == 0) raise_status(a.status, MOEDISP_STATUS_BAD_EXPERT_ID);
-    __syncthreads();
-    int32_t* th = a.tile_hist + (int64_t)tile * a.E;
-    uint32_t* lb = a.lookback + (int64_t)tile * a.E;
-    for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
-        th[e] = hist[e];
-        lb[e] = 0;
-    }
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) is_last = atomicAdd(&a.counters[0], 1u) == (unsigned)(a.n_tiles - 1);
-    __syncthreads();
-    if (!is_last) return;
-    __threadfence();
-    layout_finalize(a, smem);
-}
-
-__global__ void __launch_bounds__(kThreads) layout_scatter_kernel(LayoutArgs a) {
-    extern __shared__ __align__(16) int32_t smem[];
-    __shared__ int tile_s;
-    grid_dep_wait();
-    grid_dep_launch_dependents();
-    const int E = a.E;
-    int32_t* warp_cnt = smem;                    // [kWarps][E]
-    int32_t* tile_off = smem + kWarps * E;       // [E]
-    if (threadIdx.x == 0) tile_s = (int)atomicAdd(&a.counters[1], 1u);
-    for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) warp_cnt[i] = 0;
-    __syncthreads();
-    const int tile = tile_s;
-    const int r = tile / a.tiles_per_rank, c = tile - r * a.tiles_per_rank;
-    const int64_t base = (int64_t)r * a.P;
-    const int64_t lo = (int64_t)c * kTile, hi = min64(lo + kTile, a.P);
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const unsigned lower = (1u << lane) - 1u;
-    int32_t* mine = warp_cnt + warp * E;
-    const int64_t wlo = lo + (int64_t)warp * kSlotsPerWarp;
-
-    int ev[kSteps];
-    int rk[kSteps];
-    bool bad = false;
-#pragma unroll
-    for (int st = 0; st < kSteps; ++st) {
-        const int64_t l = wlo + st * 32 + lane;
-        ev[st] = l < hi ? slot_expert(a, base + l, bad) : -1;
-    }
-    // Rank within the warp's part, in slot order, on top of the warp's running counts.
-    const int kb = key_bits(E);
-#pragma unroll
-    for (int st = 0; st < kSteps; ++st) {
-        const int e = ev[st];
-        const unsigned peers = peers_by_ballot((unsigned)(e + 1), kb);
-        const int before = e >= 0 ? mine[e] : 0;
-        __syncwarp();
-        if (e >= 0 && lane == __ffs(peers) - 1) mine[e] = before + __popc(peers);
-        __syncwarp();
-        rk[st] = before + __popc(peers & lower);
-    }
-    __syncthreads();
-    // Exclusive scan of the warps' counts per expert; the tile's count per expert.
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int32_t run = 0;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-            const int32_t t = warp_cnt[w * E + e];
-            warp_cnt[w * E + e] = run;
-            run += t;
-        }
-        tile_off[e] = run;
-    }
-    __syncthreads();
-    // Decoupled look-back: the number of slots of expert e in all earlier tiles.
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        const uint32_t count = (uint32_t)tile_off[e];
-        uint32_t* my_word = a.lookback + (int64_t)tile * E + e;
-        uint32_t excl = 0;
-        if (tile == 0) {
-            st_relaxed(my_word, kFlagInclusive | count);
-        } else {
-            st_relaxed(my_word, kFlagAggregate | count);
-            int p = tile - 1;
-            uint64_t t0 = 0;
-            while (p >= 0) {
-                const int n = min(kWindow, p + 1);
-                uint32_t w[kWindow];
-#pragma unroll
-                for (int i = 0; i < kWindow; ++i)
-                    w[i] = i < n ? ld_relaxed(a.lookback + (int64_t)(p - i) * E + e) : 0u;
-                int used = 0;
-                bool stop = false, found = false;
-#pragma unroll
-                for (int i = 0; i < kWindow; ++i) {
-                    if (!stop && i < n) {
-                        const uint32_t f = w[i] & ~kValueMask;
-                        if (f == 0) {
-                            stop = true;
-                        } else {
-                            excl += w[i] & kValueMask;
-                            used = i + 1;
-                            if (f == kFlagInclusive) found = stop = true;
-                        }
-                    }
-                }
-                if (found) break;
-                p -= used;
-                if (used < n) {           // predecessor p has not published yet
-                    const uint64_t now = global_timer_ns();
-                    if (t0 == 0) t0 = now;
-                    else if (now - t0 > kWaitLimitNs) {
-                        raise_status(a.status, MOEDISP_STATUS_TIMEOUT);
-                        break;
-                    }
-                    __nanosleep(64);
-                }
-            }
-            st_relaxed(my_word, kFlagInclusive | ((excl + count) & kValueMask));
-        }
-        tile_off[e] = (int32_t)excl;
-    }
-    __syncthreads();
-    // Stable scatter.
-    const int32_t* colp = a.colprefix + (int64_t)r * E;
-#pragma unroll
-    for (int st = 0; st < kSteps; ++st) {
-        const int64_t l = wlo + st * 32 + lane;
-        if (l >= hi) continue;
-        const int64_t s = base + l;
-        const int e = ev[st];
-        if (e < 0) {
-            a.dst_row[s] = -1;
-            a.occ[s] = -1;
-            continue;
-        }
-        const int32_t within = tile_off[e] + mine[e] + rk[st];   // earlier slots of e, all ranks
-        const int64_t row = __ldg(a.expert_base + e) + within;
-        a.occ[s] = within - __ldg(colp + e);
-        a.dst_row[s] = (int32_t)row;
-        if (row < a.rows_cap) a.assist[row] = (int32_t)s;
-    }
-}
-
+// ------------------------------------------------------------ cluster path
 
 __device__ __forceinline__ void cluster_arrive_release() {
     asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
@@ -354,10 +322,9 @@ __device__ __forceinline__ void cluster_wait_acquire() {
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// STEPS = 32-slot steps per warp (a power of two, at most kCMaxSteps).
 template <int STEPS>
 __global__ void __launch_bounds__(kCThreads, 1)
-layout_cluster_kernel(LayoutArgs a, int64_t tile_len) {
+layout_cluster_kernel(LayoutArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ int64_t warp_tot[32];
     cg::cluster_group cluster = cg::this_cluster();
@@ -374,38 +341,17 @@ layout_cluster_kernel(LayoutArgs a, int64_t tile_len) {
     const int C = (int)cluster.num_blocks();
     const int r = tile / tpr, c = tile - r * tpr;
     const int64_t base = (int64_t)r * a.P;
-    const int64_t lo = (int64_t)c * tile_len, hi = min64(lo + tile_len, a.P);
+    const int64_t lo = (int64_t)c * a.tile_len, hi = min64(lo + a.tile_len, a.P);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const unsigned lower = (1u << lane) - 1u;
     for (int i = threadIdx.x; i < kCWarps * ES; i += blockDim.x) wc[i] = 0;
     grid_dep_wait();
     grid_dep_launch_dependents();
+    __syncthreads();
 
-    // Each warp owns STEPS*32 consecutive slots of the tile.
     int32_t* mine = wc + warp * ES;
     const int64_t wlo = lo + (int64_t)warp * STEPS * 32;
-    int ev[STEPS];
-    bool bad = false;
-#pragma unroll
-    for (int st = 0; st < STEPS; ++st) {
-        const int64_t l = wlo + st * 32 + lane;
-        ev[st] = l < hi ? slot_expert(a, base + l, bad) : -1;
-    }
-    if (__any_sync(0xffffffffu, bad) && lane == 0) raise_status(a.status, MOEDISP_STATUS_BAD_EXPERT_ID);
-    __syncthreads();
-    // Rank within the warp's slots, in slot order: packed as (rank << 11) | (expert + 1).
     uint32_t pk[STEPS];
-    const int kb = key_bits(E);
-#pragma unroll
-    for (int st = 0; st < STEPS; ++st) {
-        const int e = ev[st];
-        const unsigned peers = peers_by_ballot((unsigned)(e + 1), kb);
-        const int before = e >= 0 ? mine[e] : 0;
-        __syncwarp();
-        if (e >= 0 && lane == __ffs(peers) - 1) mine[e] = before + __popc(peers);
-        __syncwarp();
-        pk[st] = e >= 0 ? ((uint32_t)(before + __popc(peers & lower)) << 11) | (uint32_t)(e + 1) : 0u;
-    }
+    rank_in_warp<STEPS>(a, base, wlo, hi, mine, pk);
     __syncthreads();
     // Per expert, an exclusive scan over the 32 warps' counts: one warp per expert,
     // lane w holding warp w's count.
@@ -466,24 +412,14 @@ layout_cluster_kernel(LayoutArgs a, int64_t tile_len) {
             a.send_splits[(int64_t)r * W + d] = sum;
         }
     }
-#pragma unroll
-    for (int st = 0; st < STEPS; ++st) {
-        const int64_t l = wlo + st * 32 + lane;
-        if (l >= hi) continue;
-        const int64_t s = base + l;
-        if (pk[st] == 0u) {
-            a.dst_row[s] = -1;
-            a.occ[s] = -1;
-            continue;
-        }
-        const int e = (int)(pk[st] & 2047u) - 1;
-        const int32_t within = tpre[e] + mine[e] + (int32_t)(pk[st] >> 11);
-        const int64_t row = ebase[e] + within;
-        a.occ[s] = within - colp[e];
-        a.dst_row[s] = (int32_t)row;
-        if (row < a.rows_cap) a.assist[row] = (int32_t)s;
-    }
+    scatter_slots<STEPS>(a, base, wlo, hi, pk, tpre, colp, mine, ebase);
     cluster_wait_acquire();
+}
+
+int pow2_at_least(int64_t x) {
+    int p = 1;
+    while (p < x) p <<= 1;
+    return p;
 }
 
 // Cluster path geometry: tiles per rank and slots per tile, or false if the problem does
@@ -496,11 +432,8 @@ bool cluster_geometry(const moedisp_dims& d, int* tpr, int64_t* tile_len, int* s
     if ((int64_t)d.W * t > kCMaxCluster) return false;
     *tpr = (int)t;
     *tile_len = (P + t - 1) / t;
-    const int need_steps = (int)((*tile_len + kCThreads - 1) / kCThreads);
-    int p2 = 1;
-    while (p2 < need_steps) p2 <<= 1;
-    *steps = p2;
-    return p2 <= kCMaxSteps;
+    *steps = pow2_at_least((*tile_len + kCThreads - 1) / kCThreads);
+    return *steps <= kCMaxSteps;
 }
 
 size_t cluster_smem(int E) {
@@ -549,25 +482,36 @@ cudaError_t cluster_fits(const void* kernel, int C, size_t smem, bool* ok) {
     return cudaSuccess;
 }
 
-// Launches the two-kernel path (histogram, then ranking + look-back + scatter) on the
-// workspace pointers already in `a`.
+// Launches the three-kernel path on the workspace pointers already in `a`.
 cudaError_t launch_tiled(LayoutArgs& a, const moedisp_dims& dims, const LayoutGeometry& g,
                          cudaStream_t stream) {
-    const size_t fin_base = (size_t)(dims.E + 1) * sizeof(int64_t);
-    const size_t fin_cnt = (size_t)dims.W * dims.E * sizeof(int32_t);
-    a.cnt_in_smem = fin_base + fin_cnt <= kFinalizeSmemLimit;
-    size_t smem1 = std::max((size_t)dims.E * sizeof(int32_t), fin_base + (a.cnt_in_smem ? fin_cnt : 0));
-    smem1 = (smem1 + 15) & ~(size_t)15;
-    const size_t smem2 = (size_t)(kWarps + 1) * dims.E * sizeof(int32_t);
-
-    cudaError_t err = allow_dynamic_smem((const void*)layout_hist_kernel);
+    a.tiles_per_rank = g.tiles_per_rank;
+    a.n_tiles = (int)g.n_tiles;
+    a.tile_len = g.tile_len;
+    const int E = dims.E;
+    const size_t smem_count = (size_t)E * sizeof(int32_t);
+    const size_t smem_rank = (size_t)(E + 1) * sizeof(int64_t) +
+                             ((size_t)kWarps * (E | 1) + 3 * (size_t)E) * sizeof(int32_t);
+    void (*count)(LayoutArgs) = nullptr;
+    void (*rank)(LayoutArgs) = nullptr;
+    switch (g.steps) {
+        case 1: count = layout_count_kernel<1>; rank = layout_rank_kernel<1>; break;
+        case 2: count = layout_count_kernel<2>; rank = layout_rank_kernel<2>; break;
+        case 4: count = layout_count_kernel<4>; rank = layout_rank_kernel<4>; break;
+        case 8: count = layout_count_kernel<8>; rank = layout_rank_kernel<8>; break;
+        default: count = layout_count_kernel<16>; rank = layout_rank_kernel<16>; break;
+    }
+    cudaError_t err = allow_dynamic_smem((const void*)count);
     if (err != cudaSuccess) return err;
-    err = allow_dynamic_smem((const void*)layout_scatter_kernel);
+    err = allow_dynamic_smem((const void*)rank);
     if (err != cudaSuccess) return err;
-    err = launch_pdl(layout_hist_kernel, dim3((unsigned)g.n_tiles), dim3(kThreads), smem1, stream, 1, a);
+    const unsigned tiles = (unsigned)g.n_tiles;
+    err = launch_pdl(count, dim3(tiles), dim3(kThreads), smem_count, stream, 1, a);
     if (err != cudaSuccess) return err;
-    return launch_pdl(layout_scatter_kernel, dim3((unsigned)g.n_tiles), dim3(kThreads), smem2, stream,
-                      1, a);
+    err = launch_pdl(layout_scan_kernel, dim3((unsigned)((E + 31) / 32)), dim3(kScanThreads), 0,
+                     stream, 1, a);
+    if (err != cudaSuccess) return err;
+    return launch_pdl(rank, dim3(tiles), dim3(kThreads), smem_rank, stream, 1, a);
 }
 
 }  // namespace
@@ -575,16 +519,19 @@ cudaError_t launch_tiled(LayoutArgs& a, const moedisp_dims& dims, const LayoutGe
 LayoutGeometry layout_geometry(const moedisp_dims& d) {
     LayoutGeometry g{};
     g.slots_per_rank = (int64_t)d.T * d.K;
-    g.tiles_per_rank = (int)std::max<int64_t>(1, (g.slots_per_rank + kTile - 1) / kTile);
+    const int64_t slots = (int64_t)d.W * g.slots_per_rank;
+    // Tile size: a power of two between 512 and 4096 slots, aiming at kTargetTiles tiles;
+    // tiles never straddle a rank, so a rank's last tile may be shorter.
+    const int64_t want = std::min<int64_t>(4096, std::max<int64_t>(512, pow2_at_least((slots + kTargetTiles - 1) / kTargetTiles)));
+    g.tiles_per_rank = (int)std::max<int64_t>(1, (g.slots_per_rank + want - 1) / want);
+    g.tile_len = (g.slots_per_rank + g.tiles_per_rank - 1) / g.tiles_per_rank;
+    g.steps = pow2_at_least(std::max<int64_t>(1, (g.tile_len + kThreads - 1) / kThreads));  // <= 16
     g.n_tiles = (int64_t)d.W * g.tiles_per_rank;
     auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
-    size_t off = 256;                                       // counters
-    g.off_tile_hist = off;
-    off += al((size_t)g.n_tiles * d.E * sizeof(int32_t));
-    g.off_lookback = off;
-    off += al((size_t)g.n_tiles * d.E * sizeof(uint32_t));
-    g.off_colprefix = off;
-    off += al((size_t)d.W * d.E * sizeof(int32_t));
+    g.off_tile_hist = 0;
+    size_t off = al((size_t)g.n_tiles * d.E * sizeof(int32_t));
+    g.off_tile_prefix = off;
+    off += al((size_t)(g.n_tiles + 1) * d.E * sizeof(int32_t));
     g.total_bytes = off;
     return g;
 }
@@ -605,6 +552,7 @@ LayoutArgs make_args(const int32_t* expert_ids, const uint8_t* active, const moe
     a.P = g.slots_per_rank;
     a.tiles_per_rank = g.tiles_per_rank;
     a.n_tiles = (int)g.n_tiles;
+    a.tile_len = g.tile_len;
     a.cnt = L.cnt;
     a.occ = L.occ;
     a.dst_row = L.dst_row;
@@ -613,10 +561,8 @@ LayoutArgs make_args(const int32_t* expert_ids, const uint8_t* active, const moe
     a.rank_base = L.rank_base;
     a.send_splits = L.send_splits;
     a.rows_cap = L.rows_cap;
-    a.counters = reinterpret_cast<uint32_t*>(ws);
     a.tile_hist = reinterpret_cast<int32_t*>(ws + g.off_tile_hist);
-    a.lookback = reinterpret_cast<uint32_t*>(ws + g.off_lookback);
-    a.colprefix = reinterpret_cast<int32_t*>(ws + g.off_colprefix);
+    a.tile_prefix = reinterpret_cast<int32_t*>(ws + g.off_tile_prefix);
     a.status = status;
     return a;
 }
@@ -633,26 +579,23 @@ cudaError_t launch_layout(const int32_t* expert_ids, const uint8_t* active,
     if (cluster_geometry(dims, &tpr_c, &tile_c, &steps_c)) {
         const int C = dims.W * tpr_c;
         const size_t smem = cluster_smem(dims.E);
-        void (*kernel)(LayoutArgs, int64_t) =
-            steps_c == 1 ? layout_cluster_kernel<1> : steps_c == 2 ? layout_cluster_kernel<2>
-            : steps_c == 4 ? layout_cluster_kernel<4> : steps_c == 8 ? layout_cluster_kernel<8>
-                           : layout_cluster_kernel<16>;
+        void (*kernel)(LayoutArgs) = steps_c == 1 ? layout_cluster_kernel<1> : layout_cluster_kernel<2>;
         bool ok = false;
         cudaError_t err = cluster_fits((const void*)kernel, C, smem, &ok);
         if (err != cudaSuccess) return err;
         if (ok) {
             a.tiles_per_rank = tpr_c;
             a.n_tiles = C;
-            return launch_pdl(kernel, dim3(C), dim3(kCThreads), smem, stream, C, a, tile_c);
+            a.tile_len = tile_c;
+            return launch_pdl(kernel, dim3(C), dim3(kCThreads), smem, stream, C, a);
         }
     }
-
     return launch_tiled(a, dims, g, stream);
 }
 
 // ------------------------------------------------------------ allocation-free variant
 //
-// Scratch of moedisp_moe_dispatch_layout_noalloc: the two-kernel path's workspace kept in
+// Scratch of moedisp_moe_dispatch_layout_noalloc: the tiled path's workspace kept in
 // this library's own device memory (present on every GPU that loads the library, until
 // the process exits), so the caller passes no workspace and nothing is allocated.
 static __device__ __align__(256) unsigned char g_layout_scratch[MOEDISP_NOALLOC_SCRATCH_BYTES];
@@ -691,10 +634,8 @@ cudaError_t launch_layout_noalloc(const int32_t* expert_ids, const uint8_t* acti
     void* scratch = nullptr;
     cudaError_t err = layout_scratch_address(&scratch);
     if (err != cudaSuccess) return err;
-    // The array keeps whatever the previous call left: clear the two counters that must
-    // start at zero (every other scratch word is written before it is read).
-    err = cudaMemsetAsync(scratch, 0, 256, stream);
-    if (err != cudaSuccess) return err;
+    // The array keeps whatever the previous call left; nothing in it has to start at
+    // zero: every scratch word is written (tile counts, then offsets) before it is read.
     LayoutArgs a = make_args(expert_ids, active, dims, L, scratch, status, g);
     return launch_tiled(a, dims, g, stream);
 }

@@ -155,11 +155,12 @@ int moedisp_layout_workspace_size(moedisp_dims dims, size_t *bytes);
  * MOEDISP_STATUS_CAPACITY is set, every output is still computed, and assist_info is
  * written only below rows_cap.
  * workspace: device memory of at least moedisp_layout_workspace_size() bytes, 16-byte
- * aligned, ZERO-FILLED BEFORE ITS FIRST USE; every call leaves it ready for the next.
- * Calls sharing one workspace must not run concurrently.
- * Two kernels: a tiled, warp-aggregated histogram whose last block scans the counts,
- * then a tiled ranking/scatter pass whose per-expert tile offsets come from a decoupled
- * look-back over the tiles. */
+ * aligned; its contents need no initialisation (every word is written before it is
+ * read). Calls sharing one workspace must not run concurrently.
+ * Kernels: for up to 16 tiles of up to 2048 slots, one thread-block cluster that ranks
+ * the tiles and exchanges their counts through distributed shared memory; otherwise
+ * three: per-tile warp-aggregated histograms, per-expert scans down the tiles, and a
+ * per-tile ranking + scatter. */
 int moedisp_moe_dispatch_layout(const int32_t *expert_ids, const uint8_t *active_mask,
                                 moedisp_dims dims, const moedisp_layout *layout,
                                 void *workspace, size_t workspace_bytes, int32_t *status,
@@ -176,15 +177,16 @@ int moedisp_moe_dispatch_layout(const int32_t *expert_ids, const uint8_t *active
  * Instead of a workspace argument it uses a scratch array of
  * MOEDISP_NOALLOC_SCRATCH_BYTES that lives in this library's own device memory: every
  * GPU that loads the library holds it until the process exits. It always runs the
- * two-kernel path (histogram, then ranking + look-back + scatter) on that array.
+ * three-kernel tiled path (histograms, scans, ranking + scatter) on that array.
  *  - Dims whose workspace (moedisp_layout_workspace_size) exceeds
  *    MOEDISP_NOALLOC_SCRATCH_BYTES are rejected with MOEDISP_ERR_UNSUPPORTED.
  *  - It calls no allocating routine. The first call on a device looks up the array's
  *    device address (once per device, with that device current); make that first call
  *    before any stream capture.
- *  - All calls share the one array, which keeps the last call's contents; each call
- *    clears what must start at zero. Calls that overlap on the GPU (on different streams,
- *    or from different threads) race on the array and must not be made.
+ *  - All calls share the one array, which keeps the last call's contents; nothing in it
+ *    needs to start at zero (every word is written before it is read). Calls that
+ *    overlap on the GPU (on different streams, or from different threads) race on the
+ *    array and must not be made.
  * Other arguments and errors are those of moedisp_moe_dispatch_layout. */
 #define MOEDISP_NOALLOC_SCRATCH_BYTES (2u << 20)
 int moedisp_moe_dispatch_layout_noalloc(const int32_t *expert_ids, const uint8_t *active_mask,

@@ -184,8 +184,9 @@ LAYOUT_CASES = [
     ("tiny", dict(W=1, T=37, K=1, E=1)),
     ("tiny", dict(W=8, T=0, K=2, E=16)),                  # no tokens
     ("tiny", dict(W=64, T=33, K=8, E=1024)),              # many experts and ranks
-    # beyond one 16-block cluster: the two-kernel path with the decoupled look-back
-    ("tiny", dict(W=2, T=40000, K=8, E=16)),              # 157 tiles, long look-back chains
+    # beyond one 16-block cluster: the tiled (count, scan, rank) path
+    ("tiny", dict(W=2, T=40000, K=8, E=16)),              # 158 tiles of up to 4096 slots
+    ("tiny", dict(W=4, T=70000, K=8, E=64)),              # > kScanRows tiles: multi-pass scan
     ("tiny", dict(W=20, T=300, K=4, E=40, active_p=0.5)),
     ("tiny", dict(W=3, T=30000, K=6, E=300, routing="zipf", zipf_zero=30)),
     # one cluster, two tiles per rank and the largest tile
