@@ -284,6 +284,54 @@ def time_ops(torch, step, reps, warmup, flush):
     return out
 
 
+def time_ops_in_graph(torch, step, reps, warmup, flush):
+    """Per-op device times (ms) inside one graph of the step (the plan serialised between
+    layout and dispatch): an external event-record node after each op, so each pair of
+    events brackets exactly that op's kernels as the graph runs them (no host launch
+    latency). Returns None if the runtime does not support event nodes."""
+    import ctypes
+    try:
+        rt = ctypes.CDLL("libcudart.so.12")
+        rec_fn = rt.cudaEventRecordWithFlags
+    except (OSError, AttributeError):
+        return None
+    rec_fn.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint]
+    rec_fn.restype = ctypes.c_int
+    ops = ("layout", "plan", "dispatch", "combine")
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(ops) + 1)]
+
+    def body():
+        s = torch.cuda.current_stream().cuda_stream
+        def rec(ev):
+            rc = rec_fn(ctypes.c_void_p(ev.cuda_event), ctypes.c_void_p(s), 1)  # external
+            if rc != 0:
+                raise RuntimeError(f"cudaEventRecordWithFlags failed ({rc})")
+        rec(evs[0])
+        for i, op in enumerate(ops):
+            getattr(step, "op_" + op)()
+            rec(evs[i + 1])
+
+    try:
+        body()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            body()
+        out = {op: [] for op in ops}
+        for it in range(warmup + reps):
+            flush.zero_()
+            g.replay()
+            torch.cuda.synchronize()
+            if it >= warmup:
+                for i, op in enumerate(ops):
+                    out[op].append(evs[i].elapsed_time(evs[i + 1]))
+        del g
+        return out
+    except RuntimeError:
+        torch.cuda.synchronize()
+        return None
+
+
 def time_e2e(torch, step, steps, warmup, flush, device):
     """Same step with its inputs copied in from pinned host memory and y copied out."""
     w = step.w
@@ -374,7 +422,7 @@ def op_sweep(md, torch, device, hbm, reps=10):
         g = capture(torch, st.run)
         t_step = time_graph(torch, g, reps, 3, flush)
         del g
-        t = time_ops(torch, st, reps, 3, flush)
+        t = time_ops_in_graph(torch, st, reps, 3, flush) or time_ops(torch, st, reps, 3, flush)
         R = int(st.L.expert_base[-1].item())
         for op in ("layout", "dispatch", "combine"):
             ms = statistics.mean(t[op])
@@ -493,7 +541,11 @@ def main():
     torch.cuda.synchronize()
     clocks = sampler.stop([uuid.replace("GPU-", "")] if uuid else None) if rank == 0 else None
     del g_step
-    t = time_ops(torch, step, args.steps, args.warmup, flush)
+    t = time_ops_in_graph(torch, step, args.steps, args.warmup, flush)
+    op_timing = "event-record nodes inside a graph of the step"
+    if t is None:
+        t = time_ops(torch, step, args.steps, args.warmup, flush)
+        op_timing = "eager launches right behind the L2 flush"
     status = int(step.status.item())
     if status != 0:
         raise RuntimeError(f"device status after the timed steps: {md.status_string(status)}")
@@ -553,7 +605,7 @@ def main():
         "data": "synthetic (seeded generator; no dataset)",
         "config": config_of(w),
         "timing": "CUDA-graph replay of the step (exchange plan on a side-stream branch beside "
-                  "dispatch); per-op times from eager launches right behind the L2 flush",
+                  "dispatch); per-op times from " + op_timing,
         "hbm_GBps_step": round(step_bytes / (ms_step * 1e-3) / 1e9, 1),
         "frac_of_peak_step": round(step_bytes / (ms_step * 1e-3) / 1e9 / hbm, 4),
         "per_op_us": {k: round(v * 1e3, 2) for k, v in per_op.items()},

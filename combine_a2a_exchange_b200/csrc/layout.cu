@@ -216,8 +216,18 @@ __global__ void __launch_bounds__(kScanThreads) layout_scan_kernel(LayoutArgs a)
     int32_t carry = 0;                                       // column `warp`'s running sum
     for (int t0 = 0; t0 < n; t0 += kScanRows) {
         const int rows = min(kScanRows, n - t0);
-        for (int i = warp; i < rows; i += kScanThreads / 32)
-            col[i][lane] = valid ? a.tile_hist[(int64_t)(t0 + i) * a.E + e] : 0;
+        constexpr int kPer = kScanRows / (kScanThreads / 32);       // rows per warp per pass
+        int32_t v[kPer];
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {                             // all loads in flight
+            const int i = warp + k * (kScanThreads / 32);
+            v[k] = (valid && i < rows) ? __ldcg(a.tile_hist + (int64_t)(t0 + i) * a.E + e) : 0;
+        }
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {
+            const int i = warp + k * (kScanThreads / 32);
+            if (i < rows) col[i][lane] = v[k];
+        }
         __syncthreads();
         for (int q = 0; q < rows; q += 32) {
             const int i = q + lane;
