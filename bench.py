@@ -297,8 +297,14 @@ def time_ops_in_graph(torch, step, reps, warmup, flush):
         return None
     rec_fn.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint]
     rec_fn.restype = ctypes.c_int
+    rt.cudaGetLastError.restype = ctypes.c_int
     ops = ("layout", "plan", "dispatch", "combine")
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(ops) + 1)]
+    for ev in evs:                 # torch creates the CUDA event at its first record
+        ev.record()
+    torch.cuda.synchronize()
+    if any(not ev.cuda_event for ev in evs):
+        return None
 
     def body():
         s = torch.cuda.current_stream().cuda_stream
@@ -328,6 +334,7 @@ def time_ops_in_graph(torch, step, reps, warmup, flush):
         del g
         return out
     except RuntimeError:
+        rt.cudaGetLastError()      # clear the refused call's error state
         torch.cuda.synchronize()
         return None
 
