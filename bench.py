@@ -306,10 +306,11 @@ def time_ops_in_graph(torch, step, reps, warmup, flush):
     if any(not ev.cuda_event for ev in evs):
         return None
 
-    def body():
+    def body(capturing):
         s = torch.cuda.current_stream().cuda_stream
+        flags = 1 if capturing else 0       # external (a graph node) only inside a capture
         def rec(ev):
-            rc = rec_fn(ctypes.c_void_p(ev.cuda_event), ctypes.c_void_p(s), 1)  # external
+            rc = rec_fn(ctypes.c_void_p(ev.cuda_event), ctypes.c_void_p(s), flags)
             if rc != 0:
                 raise RuntimeError(f"cudaEventRecordWithFlags failed ({rc})")
         rec(evs[0])
@@ -318,11 +319,11 @@ def time_ops_in_graph(torch, step, reps, warmup, flush):
             rec(evs[i + 1])
 
     try:
-        body()
+        body(False)
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            body()
+            body(True)
         out = {op: [] for op in ops}
         for it in range(warmup + reps):
             flush.zero_()

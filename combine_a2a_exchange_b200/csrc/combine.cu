@@ -42,6 +42,20 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a) {
     grid_dep_launch_dependents();
     const int chunks = (a.H8 + kThreads - 1) / kThreads;
     const int64_t items = a.G * chunks;
+    // The next item's routing (rows and weights) is loaded while this item's rows are in
+    // flight, so each item costs one dependent round trip instead of two.
+    int32_t nd[K];
+    float nw[K];
+    auto load_routing = [&](int64_t item) {
+        if (item >= items) return;
+        const int64_t g = item / chunks;
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+            nd[k] = __ldg(a.dst_row + g * K + k);
+            nw[k] = __ldg(a.w + g * K + k);
+        }
+    };
+    load_routing(blockIdx.x);
     for (int64_t item = blockIdx.x; item < items; item += gridDim.x) {
         const int64_t g = item / chunks;
         const int vec = (int)(item - g * chunks) * kThreads + threadIdx.x;
@@ -50,13 +64,14 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a) {
         bool over = false;
 #pragma unroll
         for (int k = 0; k < K; ++k) {
-            d[k] = __ldg(a.dst_row + g * K + k);
-            w[k] = __ldg(a.w + g * K + k);
+            d[k] = nd[k];
+            w[k] = nw[k];
             if (d[k] >= a.rows_cap) {
                 over = true;
                 d[k] = -1;
             }
         }
+        load_routing(item + gridDim.x);
         if (over && threadIdx.x == 0) raise_status(a.status, MOEDISP_STATUS_CAPACITY);
         if (vec >= a.H8) continue;
         uint4 v[K];

@@ -41,7 +41,7 @@ struct DispatchArgs {
 };
 
 constexpr int kCopyThreads = 32;        // bf16 copy: one warp per block
-constexpr int kQuantThreads = 128;      // quantising copy: block size
+constexpr int kQuantThreads = 256;      // quantising copy: block size
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
@@ -230,25 +230,25 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
 }
 
 // Quantising dispatch: a block of kQuantThreads threads takes its tokens one at a time.
-// Warp 0's lane 0 streams token rows into kMaxStages-deep shared-memory stages; the block
-// reduces each row's max |x|, quantises the row into one of two output buffers, and
-// lanes 0..K-1 write the quantised row (and the scale) to the token's K rows with bulk
-// stores. Two block barriers per token: after the partial maxima (which also carries
-// the time-out verdict of the stage wait) and after the quantised row is complete.
+// Warp 0's lane 0 streams token rows into shared-memory stages (bulk loads); the block
+// reduces each row's max |x| (one block barrier per token, which also carries the
+// time-out verdict of the stage wait), then every thread quantises its 16-byte chunks of
+// the row in registers and writes the 8-byte result straight to the token's K rows --
+// a warp covers 256 contiguous bytes of each row per store. The stage of token i is
+// refilled after the barrier of token i+1, when every thread is done reading it.
 template <int Q>
 __global__ void __launch_bounds__(kQuantThreads) dispatch_quant_kernel(DispatchArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t bars[kMaxStages];
     __shared__ int64_t tok[kMaxStages];
     __shared__ int32_t drow[kMaxStages][MOEDISP_MAX_K];
-    __shared__ float red[kQuantThreads / 32];
+    __shared__ float red[2][kQuantThreads / 32];
     __shared__ int abort_s;
     constexpr float kQmax = Q == MOEDISP_QUANT_INT8 ? 127.0f : 448.0f;
     constexpr int NW = kQuantThreads / 32;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int S = a.stages, K = a.K;
     uint8_t* inbuf = smem;
-    uint8_t* outbuf = smem + (size_t)S * a.in_bytes;
 
     if (tid == 0) {
         for (int s = 0; s < S; ++s) mbar_init(&bars[s], 1);
@@ -301,7 +301,6 @@ __global__ void __launch_bounds__(kQuantThreads) dispatch_quant_kernel(DispatchA
 
     if (warp == 0)
         for (int st = 0; st < S; ++st) fill(st);
-    const bool issuer = warp == 0 && lane < K;
     const int nvec = a.H >> 3;
     for (int it = 0;; ++it) {
         const int st = it % S;
@@ -312,49 +311,57 @@ __global__ void __launch_bounds__(kQuantThreads) dispatch_quant_kernel(DispatchA
         for (int c = tid; c < nvec; c += kQuantThreads) m = fmaxf(m, absmax8(v[c]));
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if (lane == 0) red[warp] = m;
-        if (issuer) bulk_wait_read<1>();        // output buffer it % 2 is free again
+        if (lane == 0) red[it & 1][warp] = m;
         __syncthreads();
         if (abort_s) {
             if (tid == 0) raise_status(a.status, MOEDISP_STATUS_TIMEOUT);
             break;
         }
+        // Every thread is past its reads of the previous token's stage: refill it.
+        if (warp == 0 && it >= 1) fill((it - 1) % S);
         if (tok[st] < 0) break;
-        float amax = red[0];
+        float amax = red[it & 1][0];
 #pragma unroll
-        for (int w = 1; w < NW; ++w) amax = fmaxf(amax, red[w]);
+        for (int w = 1; w < NW; ++w) amax = fmaxf(amax, red[it & 1][w]);
         const float scale = __fdiv_rn(amax, kQmax);
         const float inv = __frcp_rn(scale);
         const bool zero = amax == 0.0f;
-        uint2* o2 = reinterpret_cast<uint2*>(outbuf + (size_t)(it & 1) * a.out_bytes);
-        for (int c = tid; c < nvec; c += kQuantThreads) o2[c] = quant8<Q>(v[c], scale, inv, zero);
-        fence_proxy_async_smem();
-        __syncthreads();
-        if (warp == 0) {
-            if (issuer) {
-                const int32_t d = drow[st][lane];
-                if (d >= 0) {
-                    bulk_store(a.expand_x + (int64_t)d * a.out_bytes, o2, a.out_bytes);
-                    a.scales[d] = scale;
-                }
-                bulk_commit();
-            }
-            __syncwarp();
-            fill(st);                           // every thread is done reading stage st
+        int32_t d[MOEDISP_MAX_K];
+#pragma unroll
+        for (int k = 0; k < MOEDISP_MAX_K; ++k) d[k] = k < K ? drow[st][k] : -1;
+        for (int c = tid; c < nvec; c += kQuantThreads) {
+            const uint2 q = quant8<Q>(v[c], scale, inv, zero);
+#pragma unroll
+            for (int k = 0; k < MOEDISP_MAX_K; ++k)
+                if (d[k] >= 0)
+                    __stcs(reinterpret_cast<uint2*>(a.expand_x + (int64_t)d[k] * a.out_bytes) + c, q);
+        }
+        if (tid < K) {
+            const int32_t dt = drow[st][tid];
+            if (dt >= 0) a.scales[dt] = scale;
         }
     }
-    if (issuer) bulk_wait<0>();
 }
 
 cudaError_t launch_copy(DispatchArgs a, cudaStream_t stream) {
-    const size_t budget = 64 * 1024;
-    const int S = (int)std::max<size_t>(2, std::min<size_t>(kMaxStages, budget / a.in_bytes));
+    // Few tokens per block keep the pipeline's serial start short: use the fewest stages
+    // (2, 4 or 8) with which one wave of resident blocks gives each block at most about
+    // two tokens per stage... i.e. prefer many shallow blocks while the tokens are few.
+    const int sms = current_sm_count();
+    int S = 8, per_sm = 1;
+    for (int cand : {2, 4, 8}) {
+        if ((size_t)cand * a.in_bytes > 64 * 1024 && cand > 2) break;
+        int n = 1;
+        cudaError_t err = blocks_per_sm((const void*)dispatch_copy_kernel, kCopyThreads,
+                                        (size_t)cand * a.in_bytes, &n);
+        if (err != cudaSuccess) return err;
+        S = cand;
+        per_sm = n;
+        if ((int64_t)sms * n * cand * 2 >= a.G) break;     // one wave covers the tokens
+    }
     a.stages = S;
     const size_t smem = (size_t)S * a.in_bytes;
-    int per_sm = 1;
-    cudaError_t err = blocks_per_sm((const void*)dispatch_copy_kernel, kCopyThreads, smem, &per_sm);
-    if (err != cudaSuccess) return err;
-    int64_t grid = (int64_t)current_sm_count() * per_sm;
+    int64_t grid = (int64_t)sms * per_sm;
     grid = std::min<int64_t>(grid, std::max<int64_t>(a.G, 1));
     return launch_pdl(dispatch_copy_kernel, dim3((unsigned)grid), dim3(kCopyThreads), smem, stream,
                       1, a);
@@ -362,14 +369,13 @@ cudaError_t launch_copy(DispatchArgs a, cudaStream_t stream) {
 
 template <int Q>
 cudaError_t launch_quant(DispatchArgs a, cudaStream_t stream) {
-    // S input stages (4 when a stage is small, down to 2) and two output buffers, about
-    // 56 KB per block for the largest rows here, so that four blocks share an SM.
-    const size_t fixed = 2 * (size_t)a.out_bytes;
+    // S input stages (no output buffers: quantised rows go straight from registers to
+    // global memory); about 56 KB per block for the largest rows here.
     const size_t budget = 56 * 1024;
-    int S = (int)((budget - std::min(budget, fixed)) / a.in_bytes);
+    int S = (int)(budget / a.in_bytes);
     S = std::max(2, std::min(S, 4));
     a.stages = S;
-    const size_t smem = (size_t)S * a.in_bytes + fixed;
+    const size_t smem = (size_t)S * a.in_bytes;
     int per_sm = 1;
     cudaError_t err = blocks_per_sm((const void*)dispatch_quant_kernel<Q>, kQuantThreads, smem,
                                     &per_sm);
