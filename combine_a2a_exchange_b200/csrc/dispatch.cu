@@ -153,28 +153,30 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
     grid_dep_launch_dependents();
     write_recv_counts(a);
 
-    int64_t next_g = blockIdx.x;     // look-ahead cursor over this block's tokens
-    // Arm stage `st` with the next token that has an active slot (or the end).
+    // Look-ahead over this block's tokens. The routing (K destination rows) of the token
+    // after the one being armed is loaded one fill ahead, so arming a stage does not wait
+    // for a dependent load.
+    int64_t pf_g = blockIdx.x;
+    int32_t pf_d = (pf_g < a.G && lane < K) ? __ldg(a.dst_row + pf_g * K + lane) : -1;
     auto fill = [&](int st) {
         while (true) {
-            if (next_g >= a.G) {
+            const int64_t g = pf_g;
+            int32_t d = pf_d;
+            pf_g = g + gridDim.x;
+            pf_d = (pf_g < a.G && lane < K) ? __ldg(a.dst_row + pf_g * K + lane) : -1;
+            if (g >= a.G) {
                 if (lane == 0) {
                     tok[st] = -1;
                     mbar_arrive(&bars[st]);
                 }
                 return;
             }
-            int32_t d = -1;
-            if (lane < K) {
-                d = __ldg(a.dst_row + next_g * K + lane);
-                if (d >= a.rows_cap) {
-                    raise_status(a.status, MOEDISP_STATUS_CAPACITY);
-                    d = -1;
-                }
-                if (d < 0) d = -1;
+            if (d >= a.rows_cap) {
+                raise_status(a.status, MOEDISP_STATUS_CAPACITY);
+                d = -1;
             }
-            const unsigned any = __ballot_sync(0xffffffffu, d >= 0);
-            if (any) {
+            if (d < 0) d = -1;
+            if (__ballot_sync(0xffffffffu, d >= 0)) {
                 int32_t dk[MOEDISP_MAX_K];
 #pragma unroll
                 for (int k = 0; k < MOEDISP_MAX_K; ++k) dk[k] = __shfl_sync(0xffffffffu, d, k);
@@ -182,15 +184,13 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
 #pragma unroll
                     for (int k = 0; k < MOEDISP_MAX_K; ++k)
                         if (k < K) drow[st][k] = dk[k];
-                    tok[st] = next_g;
+                    tok[st] = g;
                     mbar_arrive_expect_tx(&bars[st], a.in_bytes);
-                    bulk_load(inbuf + (size_t)st * a.in_bytes, a.x + next_g * a.in_bytes, a.in_bytes,
+                    bulk_load(inbuf + (size_t)st * a.in_bytes, a.x + g * a.in_bytes, a.in_bytes,
                               &bars[st]);
                 }
-                next_g += gridDim.x;
                 return;
             }
-            next_g += gridDim.x;
         }
     };
 
@@ -260,25 +260,29 @@ __global__ void __launch_bounds__(kQuantThreads) dispatch_quant_kernel(DispatchA
     grid_dep_launch_dependents();
     write_recv_counts(a);
 
-    int64_t next_g = blockIdx.x;
+    // Look-ahead over this block's tokens. The routing (K destination rows) of the token
+    // after the one being armed is loaded one fill ahead, so arming a stage does not wait
+    // for a dependent load.
+    int64_t pf_g = blockIdx.x;
+    int32_t pf_d = (pf_g < a.G && lane < K) ? __ldg(a.dst_row + pf_g * K + lane) : -1;
     auto fill = [&](int st) {          // warp 0 only
         while (true) {
-            if (next_g >= a.G) {
+            const int64_t g = pf_g;
+            int32_t d = pf_d;
+            pf_g = g + gridDim.x;
+            pf_d = (pf_g < a.G && lane < K) ? __ldg(a.dst_row + pf_g * K + lane) : -1;
+            if (g >= a.G) {
                 if (lane == 0) {
                     tok[st] = -1;
                     mbar_arrive(&bars[st]);
                 }
                 return;
             }
-            int32_t d = -1;
-            if (lane < K) {
-                d = __ldg(a.dst_row + next_g * K + lane);
-                if (d >= a.rows_cap) {
-                    raise_status(a.status, MOEDISP_STATUS_CAPACITY);
-                    d = -1;
-                }
-                if (d < 0) d = -1;
+            if (d >= a.rows_cap) {
+                raise_status(a.status, MOEDISP_STATUS_CAPACITY);
+                d = -1;
             }
+            if (d < 0) d = -1;
             if (__ballot_sync(0xffffffffu, d >= 0)) {
                 int32_t dk[MOEDISP_MAX_K];
 #pragma unroll
@@ -287,15 +291,13 @@ __global__ void __launch_bounds__(kQuantThreads) dispatch_quant_kernel(DispatchA
 #pragma unroll
                     for (int k = 0; k < MOEDISP_MAX_K; ++k)
                         if (k < K) drow[st][k] = dk[k];
-                    tok[st] = next_g;
+                    tok[st] = g;
                     mbar_arrive_expect_tx(&bars[st], a.in_bytes);
-                    bulk_load(inbuf + (size_t)st * a.in_bytes, a.x + next_g * a.in_bytes,
-                              a.in_bytes, &bars[st]);
+                    bulk_load(inbuf + (size_t)st * a.in_bytes, a.x + g * a.in_bytes, a.in_bytes,
+                              &bars[st]);
                 }
-                next_g += gridDim.x;
                 return;
             }
-            next_g += gridDim.x;
         }
     };
 

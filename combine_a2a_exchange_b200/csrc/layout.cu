@@ -8,7 +8,7 @@
 // never straddle a source rank, and:
 //
 //  * small problems (at most 16 tiles of at most 2048 slots): one kernel, one thread-block
-//    cluster. Each 1024-thread block ranks its tile (below), the blocks exchange their
+//    cluster. Each 256-thread block ranks its tile (below), the blocks exchange their
 //    per-expert tile counts through distributed shared memory across the cluster barrier,
 //    and every block derives its tile offsets, the expert bases and the per-rank counts
 //    from them -- no global scratch, no second launch.
@@ -49,9 +49,9 @@ constexpr int64_t kTargetTiles = 296;         // about two blocks per SM
 constexpr int kScanThreads = 1024;
 constexpr int kScanRows = 256;                // tiles per pass of the scan kernel
 // Single-kernel cluster path.
-constexpr int kCThreads = 1024;
+constexpr int kCThreads = 256;
 constexpr int kCWarps = kCThreads / 32;
-constexpr int kCMaxSteps = 2;                 // tiles <= 2048 slots
+constexpr int kCMaxSteps = 8;                 // tiles <= 2048 slots
 constexpr int64_t kCMaxTile = (int64_t)kCWarps * 32 * kCMaxSteps;
 constexpr int kCMaxCluster = 16;
 
@@ -352,7 +352,7 @@ layout_cluster_kernel(LayoutArgs a) {
     const int r = tile / tpr, c = tile - r * tpr;
     const int64_t base = (int64_t)r * a.P;
     const int64_t lo = (int64_t)c * a.tile_len, hi = min64(lo + a.tile_len, a.P);
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int warp = threadIdx.x >> 5;
     for (int i = threadIdx.x; i < kCWarps * ES; i += blockDim.x) wc[i] = 0;
     grid_dep_wait();
     grid_dep_launch_dependents();
@@ -363,13 +363,16 @@ layout_cluster_kernel(LayoutArgs a) {
     uint32_t pk[STEPS];
     rank_in_warp<STEPS>(a, base, wlo, hi, mine, pk);
     __syncthreads();
-    // Per expert, an exclusive scan over the 32 warps' counts: one warp per expert,
-    // lane w holding warp w's count.
-    for (int e = warp; e < E; e += kCWarps) {
-        const int32_t v = wc[lane * ES + e];
-        const int32_t inc = warp_inclusive_scan_i32(v);
-        wc[lane * ES + e] = inc - v;
-        if (lane == 31) tcnt[e] = inc;
+    // Per expert, an exclusive scan over the warps' counts, in warp order.
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int32_t run = 0;
+#pragma unroll
+        for (int w = 0; w < kCWarps; ++w) {
+            const int32_t t = wc[w * ES + e];
+            wc[w * ES + e] = run;
+            run += t;
+        }
+        tcnt[e] = run;
     }
     cluster.sync();   // every tile's counts are final and visible across the cluster
 
@@ -589,7 +592,9 @@ cudaError_t launch_layout(const int32_t* expert_ids, const uint8_t* active,
     if (cluster_geometry(dims, &tpr_c, &tile_c, &steps_c)) {
         const int C = dims.W * tpr_c;
         const size_t smem = cluster_smem(dims.E);
-        void (*kernel)(LayoutArgs) = steps_c == 1 ? layout_cluster_kernel<1> : layout_cluster_kernel<2>;
+        void (*kernel)(LayoutArgs) =
+            steps_c == 1 ? layout_cluster_kernel<1> : steps_c == 2 ? layout_cluster_kernel<2>
+            : steps_c == 4 ? layout_cluster_kernel<4> : layout_cluster_kernel<8>;
         bool ok = false;
         cudaError_t err = cluster_fits((const void*)kernel, C, smem, &ok);
         if (err != cudaSuccess) return err;
