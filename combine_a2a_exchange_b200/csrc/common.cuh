@@ -91,13 +91,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete; false after kWaitLimitNs.
+// (try_wait itself suspends the thread for a while; the clock is read every 64 polls.)
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 63u) == 0u && global_timer_ns() - t0 > kWaitLimitNs) return false;
     }
-    return true;
 }
 
 // ------------------------------------------------------- 1-D bulk (TMA) copies

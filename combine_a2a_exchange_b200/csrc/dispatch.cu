@@ -65,25 +65,39 @@ __device__ __forceinline__ float absmax8(const uint4& v) {
 // is the definition's bit for bit; the fast test only decides which path gives it.
 
 // int8 boundaries are the half-integers; |x/scale| <= ~127, so the bound above is below
-// 2.3e-5 and a margin of 2^-14 from k + 0.5 is safe.
+// 2.3e-5 and a margin of 2^-14 from k + 0.5 is safe. Rounding to an integer uses the
+// floating-point adder: for |v| < 2^22, v + 1.5*2^23 rounds v's fraction away to the
+// nearest integer, ties to even, and the integer is read back from the sum's low bits.
 __device__ __forceinline__ int q_int8(float x, float scale, float inv) {
+    constexpr float kMagic = 12582912.0f;                    // 1.5 * 2^23
     float v = __fmul_rn(x, inv);
-    const float t = v - floorf(v);
-    if (!(fabsf(t - 0.5f) >= 0.00006103515625f)) v = __fdiv_rn(x, scale);
-    const int q = __float2int_rn(v);
+    float rr = __fadd_rn(v, kMagic);
+    const float t = __fsub_rn(v, __fsub_rn(rr, kMagic));      // v - round(v), in [-0.5, 0.5]
+    if (!(0.5f - fabsf(t) >= 0.00006103515625f)) {            // near k + 0.5, or not finite
+        v = __fdiv_rn(x, scale);
+        if (!(fabsf(v) < 4194304.0f)) return v > 0.0f ? 127 : -127;   // |v| >= 2^22 or NaN
+        rr = __fadd_rn(v, kMagic);
+    }
+    const int q = (int)(__float_as_uint(rr) - __float_as_uint(kMagic));
     return max(-127, min(127, q));
 }
 
 // E4M3 keeps 3 mantissa bits: for 2^-6 <= |v| < 448 its rounding boundaries are the fp32
-// values whose 20 low mantissa bits are exactly 0x80000; r is used when it is more than
-// 16 fp32 ulps from one. E4M3's subnormal range and the saturation edge take the exact
-// path.
-__device__ __forceinline__ float q_e4m3_value(float x, float scale, float inv) {
+// values whose 20 low mantissa bits are exactly 0x80000. When r is more than 16 fp32 ulps
+// from such a boundary, rounding to nearest is adding half an E4M3 step to the bits and
+// truncating: the code is sign | ((bits + 0x80000) >> 20) - ((127 - 7) << 3), the carry
+// moving into the exponent when the mantissa rounds up. Elsewhere (near a boundary, in
+// E4M3's subnormal range, at the saturation edge, not finite) the IEEE quotient goes
+// through the hardware conversion (round to nearest even, saturating to +-448).
+__device__ __forceinline__ uint32_t q_e4m3(float x, float scale, float inv) {
     const float r = __fmul_rn(x, inv);
-    const uint32_t u = __float_as_uint(r) & 0x7fffffffu;
+    const uint32_t b = __float_as_uint(r);
+    const uint32_t u = b & 0x7fffffffu;
     const int32_t d = (int32_t)(u & 0xfffffu) - 0x80000;
-    const bool clear = u >= 0x3c800000u && u < 0x43e00000u && (d > 16 || d < -16);
-    return clear ? r : __fdiv_rn(x, scale);
+    if (u >= 0x3c800000u && u < 0x43e00000u && (d > 16 || d < -16))
+        return ((b >> 24) & 0x80u) | (((u + 0x80000u) >> 20) - 0x3c0u);
+    const float v = __fdiv_rn(x, scale);
+    return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(v, 0.0f), __NV_SATFINITE, __NV_E4M3) & 0xffu;
 }
 
 __device__ __forceinline__ uint32_t q_int8_pair(uint32_t w, float scale, float inv) {
@@ -92,11 +106,8 @@ __device__ __forceinline__ uint32_t q_int8_pair(uint32_t w, float scale, float i
     return (uint32_t)(a & 0xff) | ((uint32_t)(b & 0xff) << 8);
 }
 
-// Round to nearest even, saturating to +-448 (hardware conversion).
 __device__ __forceinline__ uint32_t q_e4m3_pair(uint32_t w, float scale, float inv) {
-    const float2 f = make_float2(q_e4m3_value(bf16_lo(w), scale, inv),
-                                 q_e4m3_value(bf16_hi(w), scale, inv));
-    return (uint32_t)__nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3);
+    return q_e4m3(bf16_lo(w), scale, inv) | (q_e4m3(bf16_hi(w), scale, inv) << 8);
 }
 
 template <int Q>
@@ -236,7 +247,7 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
 // the row in registers and writes the 8-byte result straight to the token's K rows --
 // a warp covers 256 contiguous bytes of each row per store. The stage of token i is
 // refilled after the barrier of token i+1, when every thread is done reading it.
-template <int Q>
+template <int Q, int KT>
 __global__ void __launch_bounds__(kQuantThreads) dispatch_quant_kernel(DispatchArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t bars[kMaxStages];
@@ -246,8 +257,9 @@ __global__ void __launch_bounds__(kQuantThreads) dispatch_quant_kernel(DispatchA
     __shared__ int abort_s;
     constexpr float kQmax = Q == MOEDISP_QUANT_INT8 ? 127.0f : 448.0f;
     constexpr int NW = kQuantThreads / 32;
+    constexpr int K = KT;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int S = a.stages, K = a.K;
+    const int S = a.stages;
     uint8_t* inbuf = smem;
 
     if (tid == 0) {
@@ -328,15 +340,17 @@ __global__ void __launch_bounds__(kQuantThreads) dispatch_quant_kernel(DispatchA
         const float scale = __fdiv_rn(amax, kQmax);
         const float inv = __frcp_rn(scale);
         const bool zero = amax == 0.0f;
-        int32_t d[MOEDISP_MAX_K];
+        uint2* dst[K];
 #pragma unroll
-        for (int k = 0; k < MOEDISP_MAX_K; ++k) d[k] = k < K ? drow[st][k] : -1;
+        for (int k = 0; k < K; ++k) {
+            const int32_t d = drow[st][k];
+            dst[k] = d >= 0 ? reinterpret_cast<uint2*>(a.expand_x + (int64_t)d * a.out_bytes) : nullptr;
+        }
         for (int c = tid; c < nvec; c += kQuantThreads) {
             const uint2 q = quant8<Q>(v[c], scale, inv, zero);
 #pragma unroll
-            for (int k = 0; k < MOEDISP_MAX_K; ++k)
-                if (d[k] >= 0)
-                    __stcs(reinterpret_cast<uint2*>(a.expand_x + (int64_t)d[k] * a.out_bytes) + c, q);
+            for (int k = 0; k < K; ++k)
+                if (dst[k] != nullptr) __stcs(dst[k] + c, q);
         }
         if (tid < K) {
             const int32_t dt = drow[st][tid];
@@ -369,7 +383,7 @@ cudaError_t launch_copy(DispatchArgs a, cudaStream_t stream) {
                       1, a);
 }
 
-template <int Q>
+template <int Q, int KT>
 cudaError_t launch_quant(DispatchArgs a, cudaStream_t stream) {
     // S input stages (no output buffers: quantised rows go straight from registers to
     // global memory); about 56 KB per block for the largest rows here.
@@ -379,13 +393,26 @@ cudaError_t launch_quant(DispatchArgs a, cudaStream_t stream) {
     a.stages = S;
     const size_t smem = (size_t)S * a.in_bytes;
     int per_sm = 1;
-    cudaError_t err = blocks_per_sm((const void*)dispatch_quant_kernel<Q>, kQuantThreads, smem,
+    cudaError_t err = blocks_per_sm((const void*)dispatch_quant_kernel<Q, KT>, kQuantThreads, smem,
                                     &per_sm);
     if (err != cudaSuccess) return err;
     int64_t grid = (int64_t)current_sm_count() * per_sm;
     grid = std::min<int64_t>(grid, std::max<int64_t>(a.G, 1));
-    return launch_pdl(dispatch_quant_kernel<Q>, dim3((unsigned)grid), dim3(kQuantThreads), smem,
+    return launch_pdl(dispatch_quant_kernel<Q, KT>, dim3((unsigned)grid), dim3(kQuantThreads), smem,
                       stream, 1, a);
+}
+
+template <int Q>
+cudaError_t launch_quant_k(const DispatchArgs& a, cudaStream_t stream) {
+    switch (a.K) {
+#define MOEDISP_QK(n) \
+    case n: return launch_quant<Q, n>(a, stream);
+        MOEDISP_QK(1) MOEDISP_QK(2) MOEDISP_QK(3) MOEDISP_QK(4) MOEDISP_QK(5) MOEDISP_QK(6)
+        MOEDISP_QK(7) MOEDISP_QK(8) MOEDISP_QK(9) MOEDISP_QK(10) MOEDISP_QK(11) MOEDISP_QK(12)
+        MOEDISP_QK(13) MOEDISP_QK(14) MOEDISP_QK(15) MOEDISP_QK(16)
+#undef MOEDISP_QK
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace
@@ -419,8 +446,8 @@ cudaError_t launch_dispatch(const void* x, int H, const moedisp_dims& dims,
     a.status = status;
     switch (quant_mode) {
         case MOEDISP_QUANT_NONE: return launch_copy(a, stream);
-        case MOEDISP_QUANT_INT8: return launch_quant<MOEDISP_QUANT_INT8>(a, stream);
-        case MOEDISP_QUANT_FP8_E4M3: return launch_quant<MOEDISP_QUANT_FP8_E4M3>(a, stream);
+        case MOEDISP_QUANT_INT8: return launch_quant_k<MOEDISP_QUANT_INT8>(a, stream);
+        case MOEDISP_QUANT_FP8_E4M3: return launch_quant_k<MOEDISP_QUANT_FP8_E4M3>(a, stream);
         default: return cudaErrorInvalidValue;
     }
 }
