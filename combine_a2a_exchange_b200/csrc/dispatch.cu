@@ -240,53 +240,62 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
     if (issuer) bulk_wait<0>();
 }
 
-// Quantising dispatch: a block of kQuantThreads threads takes its tokens one at a time.
-// Warp 0's lane 0 streams token rows into shared-memory stages (bulk loads); the block
-// reduces each row's max |x| (one block barrier per token, which also carries the
-// time-out verdict of the stage wait), then every thread quantises its 16-byte chunks of
-// the row in registers and writes the 8-byte result straight to the token's K rows --
-// a warp covers 256 contiguous bytes of each row per store. The stage of token i is
-// refilled after the barrier of token i+1, when every thread is done reading it.
-template <int Q, int KT>
-__global__ void __launch_bounds__(kQuantThreads) dispatch_quant_kernel(DispatchArgs a) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ __align__(8) uint64_t bars[kMaxStages];
-    __shared__ int64_t tok[kMaxStages];
-    __shared__ int32_t drow[kMaxStages][MOEDISP_MAX_K];
-    __shared__ float red[2][kQuantThreads / 32];
-    __shared__ int abort_s;
-    constexpr float kQmax = Q == MOEDISP_QUANT_INT8 ? 127.0f : 448.0f;
-    constexpr int NW = kQuantThreads / 32;
-    constexpr int K = KT;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int S = a.stages;
-    uint8_t* inbuf = smem;
+// Quantising dispatch. A block of kQuantThreads threads is split into token groups of WPT
+// warps; each group is an independent pipeline over its own tokens, with its own
+// shared-memory stages and barriers. The group's first lane streams token rows into the
+// stages (bulk loads); the group reduces the row's max |x| (warp shuffles, plus a named
+// barrier across the group's warps when WPT > 1 -- that barrier also carries the
+// time-out verdict), then each thread quantises its 16-byte chunks of the row and writes
+// the 8-byte results straight to the token's K rows (a warp covers 256 contiguous bytes
+// of a row per store). The previous token's stage is refilled after the barrier.
+constexpr int kChunks = 8;
 
-    if (tid == 0) {
-        for (int s = 0; s < S; ++s) mbar_init(&bars[s], 1);
+__device__ __forceinline__ void group_barrier(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+template <int Q, int WPT>
+__global__ void __launch_bounds__(kQuantThreads, 2) dispatch_quant_kernel(DispatchArgs a) {
+    constexpr int NG = kQuantThreads / 32 / WPT;     // token groups per block
+    constexpr int GT = WPT * 32;                     // threads per group
+    constexpr float kQmax = Q == MOEDISP_QUANT_INT8 ? 127.0f : 448.0f;
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ __align__(8) uint64_t bars[NG][kMaxStages];
+    __shared__ int64_t tok[NG][kMaxStages];
+    __shared__ int32_t drow[NG][kMaxStages][MOEDISP_MAX_K];
+    __shared__ float red[NG][2][WPT];
+    __shared__ int abort_s[NG];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int grp = warp / WPT, gw = warp - grp * WPT, gt = tid - grp * GT;
+    const int S = a.stages, K = a.K;
+    uint8_t* inbuf = smem + (size_t)grp * S * a.in_bytes;
+    uint64_t* gbar = bars[grp];
+
+    if (gt == 0) {
+        for (int s = 0; s < S; ++s) mbar_init(&gbar[s], 1);
         fence_mbar_init();
-        abort_s = 0;
+        abort_s[grp] = 0;
     }
     __syncthreads();
     grid_dep_wait();
     grid_dep_launch_dependents();
     write_recv_counts(a);
 
-    // Look-ahead over this block's tokens. The routing (K destination rows) of the token
-    // after the one being armed is loaded one fill ahead, so arming a stage does not wait
-    // for a dependent load.
-    int64_t pf_g = blockIdx.x;
-    int32_t pf_d = (pf_g < a.G && lane < K) ? __ldg(a.dst_row + pf_g * K + lane) : -1;
-    auto fill = [&](int st) {          // warp 0 only
+    // The group's first warp arms stages. The routing (K destination rows) of the token
+    // after the one being armed is loaded one fill ahead.
+    const int64_t n_groups = (int64_t)gridDim.x * NG;
+    int64_t pf_g = (int64_t)blockIdx.x * NG + grp;
+    int32_t pf_d = (gw == 0 && pf_g < a.G && lane < K) ? __ldg(a.dst_row + pf_g * K + lane) : -1;
+    auto fill = [&](int st) {
         while (true) {
             const int64_t g = pf_g;
             int32_t d = pf_d;
-            pf_g = g + gridDim.x;
+            pf_g = g + n_groups;
             pf_d = (pf_g < a.G && lane < K) ? __ldg(a.dst_row + pf_g * K + lane) : -1;
             if (g >= a.G) {
                 if (lane == 0) {
-                    tok[st] = -1;
-                    mbar_arrive(&bars[st]);
+                    tok[grp][st] = -1;
+                    mbar_arrive(&gbar[st]);
                 }
                 return;
             }
@@ -302,58 +311,60 @@ __global__ void __launch_bounds__(kQuantThreads) dispatch_quant_kernel(DispatchA
                 if (lane == 0) {
 #pragma unroll
                     for (int k = 0; k < MOEDISP_MAX_K; ++k)
-                        if (k < K) drow[st][k] = dk[k];
-                    tok[st] = g;
-                    mbar_arrive_expect_tx(&bars[st], a.in_bytes);
+                        if (k < K) drow[grp][st][k] = dk[k];
+                    tok[grp][st] = g;
+                    mbar_arrive_expect_tx(&gbar[st], a.in_bytes);
                     bulk_load(inbuf + (size_t)st * a.in_bytes, a.x + g * a.in_bytes, a.in_bytes,
-                              &bars[st]);
+                              &gbar[st]);
                 }
                 return;
             }
         }
     };
-
-    if (warp == 0)
+    if (gw == 0)
         for (int st = 0; st < S; ++st) fill(st);
+
     const int nvec = a.H >> 3;
     for (int it = 0;; ++it) {
         const int st = it % S;
         const uint32_t par = (uint32_t)((it / S) & 1);
-        if (!mbar_wait(&bars[st], par)) abort_s = 1;
-        const uint4* v = reinterpret_cast<const uint4*>(inbuf + (size_t)st * a.in_bytes);
+        if (!mbar_wait(&gbar[st], par)) abort_s[grp] = 1;
+        const int64_t g = tok[grp][st];
+        int32_t d[MOEDISP_MAX_K];
+#pragma unroll
+        for (int k = 0; k < MOEDISP_MAX_K; ++k) d[k] = k < K ? drow[grp][st][k] : -1;
+        const uint4* row = reinterpret_cast<const uint4*>(inbuf + (size_t)st * a.in_bytes);
         float m = 0.0f;
-        for (int c = tid; c < nvec; c += kQuantThreads) m = fmaxf(m, absmax8(v[c]));
+        for (int c = gt; c < nvec; c += GT) m = fmaxf(m, absmax8(row[c]));
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if (lane == 0) red[it & 1][warp] = m;
-        __syncthreads();
-        if (abort_s) {
-            if (tid == 0) raise_status(a.status, MOEDISP_STATUS_TIMEOUT);
+        if (WPT > 1) {
+            if (lane == 0) red[grp][it & 1][gw] = m;
+            group_barrier(1 + grp, GT);
+#pragma unroll
+            for (int w = 0; w < WPT; ++w) m = fmaxf(m, red[grp][it & 1][w]);
+        } else {
+            __syncwarp();
+        }
+        if (abort_s[grp]) {
+            if (gt == 0) raise_status(a.status, MOEDISP_STATUS_TIMEOUT);
             break;
         }
-        // Every thread is past its reads of the previous token's stage: refill it.
-        if (warp == 0 && it >= 1) fill((it - 1) % S);
-        if (tok[st] < 0) break;
-        float amax = red[it & 1][0];
-#pragma unroll
-        for (int w = 1; w < NW; ++w) amax = fmaxf(amax, red[it & 1][w]);
-        const float scale = __fdiv_rn(amax, kQmax);
+        // Every thread of the group is past the previous token: its stage is free.
+        if (gw == 0 && it >= 1) fill((it - 1) % S);
+        if (g < 0) break;
+        const float scale = __fdiv_rn(m, kQmax);
         const float inv = __frcp_rn(scale);
-        const bool zero = amax == 0.0f;
-        uint2* dst[K];
+        const bool zero = m == 0.0f;
+        for (int c = gt; c < nvec; c += GT) {
+            const uint2 q = quant8<Q>(row[c], scale, inv, zero);
 #pragma unroll
-        for (int k = 0; k < K; ++k) {
-            const int32_t d = drow[st][k];
-            dst[k] = d >= 0 ? reinterpret_cast<uint2*>(a.expand_x + (int64_t)d * a.out_bytes) : nullptr;
+            for (int k = 0; k < MOEDISP_MAX_K; ++k)
+                if (d[k] >= 0)
+                    __stcs(reinterpret_cast<uint2*>(a.expand_x + (int64_t)d[k] * a.out_bytes) + c, q);
         }
-        for (int c = tid; c < nvec; c += kQuantThreads) {
-            const uint2 q = quant8<Q>(v[c], scale, inv, zero);
-#pragma unroll
-            for (int k = 0; k < K; ++k)
-                if (dst[k] != nullptr) __stcs(dst[k] + c, q);
-        }
-        if (tid < K) {
-            const int32_t dt = drow[st][tid];
+        if (gt < K) {
+            const int32_t dt = drow[grp][st][gt];
             if (dt >= 0) a.scales[dt] = scale;
         }
     }
@@ -383,36 +394,30 @@ cudaError_t launch_copy(DispatchArgs a, cudaStream_t stream) {
                       1, a);
 }
 
-template <int Q, int KT>
-cudaError_t launch_quant(DispatchArgs a, cudaStream_t stream) {
-    // S input stages (no output buffers: quantised rows go straight from registers to
-    // global memory); about 56 KB per block for the largest rows here.
-    const size_t budget = 56 * 1024;
-    int S = (int)(budget / a.in_bytes);
-    S = std::max(2, std::min(S, 4));
-    a.stages = S;
-    const size_t smem = (size_t)S * a.in_bytes;
+template <int Q, int WPT>
+cudaError_t launch_quant_w(DispatchArgs a, cudaStream_t stream) {
+    constexpr int NG = kQuantThreads / 32 / WPT;
+    // Three stages per group: one being read, one or two loading.
+    a.stages = 3;
+    const size_t smem = (size_t)NG * a.stages * a.in_bytes;
     int per_sm = 1;
-    cudaError_t err = blocks_per_sm((const void*)dispatch_quant_kernel<Q, KT>, kQuantThreads, smem,
+    cudaError_t err = blocks_per_sm((const void*)dispatch_quant_kernel<Q, WPT>, kQuantThreads, smem,
                                     &per_sm);
     if (err != cudaSuccess) return err;
     int64_t grid = (int64_t)current_sm_count() * per_sm;
-    grid = std::min<int64_t>(grid, std::max<int64_t>(a.G, 1));
-    return launch_pdl(dispatch_quant_kernel<Q, KT>, dim3((unsigned)grid), dim3(kQuantThreads), smem,
+    grid = std::min<int64_t>(grid, std::max<int64_t>((a.G + NG - 1) / NG, 1));
+    return launch_pdl(dispatch_quant_kernel<Q, WPT>, dim3((unsigned)grid), dim3(kQuantThreads), smem,
                       stream, 1, a);
 }
 
+// Warps per token: the fewest that hold a row in kChunks 16-byte chunks per thread.
 template <int Q>
-cudaError_t launch_quant_k(const DispatchArgs& a, cudaStream_t stream) {
-    switch (a.K) {
-#define MOEDISP_QK(n) \
-    case n: return launch_quant<Q, n>(a, stream);
-        MOEDISP_QK(1) MOEDISP_QK(2) MOEDISP_QK(3) MOEDISP_QK(4) MOEDISP_QK(5) MOEDISP_QK(6)
-        MOEDISP_QK(7) MOEDISP_QK(8) MOEDISP_QK(9) MOEDISP_QK(10) MOEDISP_QK(11) MOEDISP_QK(12)
-        MOEDISP_QK(13) MOEDISP_QK(14) MOEDISP_QK(15) MOEDISP_QK(16)
-#undef MOEDISP_QK
-        default: return cudaErrorInvalidValue;
-    }
+cudaError_t launch_quant(const DispatchArgs& a, cudaStream_t stream) {
+    const int nvec = a.H / 8;
+    if (nvec <= 1 * 32 * kChunks) return launch_quant_w<Q, 1>(a, stream);
+    if (nvec <= 2 * 32 * kChunks) return launch_quant_w<Q, 2>(a, stream);
+    if (nvec <= 4 * 32 * kChunks) return launch_quant_w<Q, 4>(a, stream);
+    return launch_quant_w<Q, 8>(a, stream);
 }
 
 }  // namespace
@@ -446,8 +451,8 @@ cudaError_t launch_dispatch(const void* x, int H, const moedisp_dims& dims,
     a.status = status;
     switch (quant_mode) {
         case MOEDISP_QUANT_NONE: return launch_copy(a, stream);
-        case MOEDISP_QUANT_INT8: return launch_quant_k<MOEDISP_QUANT_INT8>(a, stream);
-        case MOEDISP_QUANT_FP8_E4M3: return launch_quant_k<MOEDISP_QUANT_FP8_E4M3>(a, stream);
+        case MOEDISP_QUANT_INT8: return launch_quant<MOEDISP_QUANT_INT8>(a, stream);
+        case MOEDISP_QUANT_FP8_E4M3: return launch_quant<MOEDISP_QUANT_FP8_E4M3>(a, stream);
         default: return cudaErrorInvalidValue;
     }
 }
