@@ -93,8 +93,8 @@ __device__ __forceinline__ uint32_t q_e4m3(float x, float scale, float inv) {
     const float r = __fmul_rn(x, inv);
     const uint32_t b = __float_as_uint(r);
     const uint32_t u = b & 0x7fffffffu;
-    const int32_t d = (int32_t)(u & 0xfffffu) - 0x80000;
-    if (u >= 0x3c800000u && u < 0x43e00000u && (d > 16 || d < -16))
+    // (unsigned range tests: 2^-6 <= |r| < 448, and low bits outside [0x80000 +- 16])
+    if (u - 0x3c800000u < 0x43e00000u - 0x3c800000u && (u & 0xfffffu) - 0x7fff0u > 32u)
         return ((b >> 24) & 0x80u) | (((u + 0x80000u) >> 20) - 0x3c0u);
     const float v = __fdiv_rn(x, scale);
     return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(v, 0.0f), __NV_SATFINITE, __NV_E4M3) & 0xffu;
@@ -356,12 +356,26 @@ __global__ void __launch_bounds__(kQuantThreads, 2) dispatch_quant_kernel(Dispat
         const float scale = __fdiv_rn(m, kQmax);
         const float inv = __frcp_rn(scale);
         const bool zero = m == 0.0f;
-        for (int c = gt; c < nvec; c += GT) {
-            const uint2 q = quant8<Q>(row[c], scale, inv, zero);
+        if (K <= 8) {                          // row bases once per token, 8-way stores
+            uint2* dst[8];
 #pragma unroll
-            for (int k = 0; k < MOEDISP_MAX_K; ++k)
-                if (d[k] >= 0)
-                    __stcs(reinterpret_cast<uint2*>(a.expand_x + (int64_t)d[k] * a.out_bytes) + c, q);
+            for (int k = 0; k < 8; ++k)
+                dst[k] = d[k] >= 0 ? reinterpret_cast<uint2*>(a.expand_x + (int64_t)d[k] * a.out_bytes)
+                                   : nullptr;
+            for (int c = gt; c < nvec; c += GT) {
+                const uint2 q = quant8<Q>(row[c], scale, inv, zero);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    if (dst[k] != nullptr) __stcs(dst[k] + c, q);
+            }
+        } else {
+            for (int c = gt; c < nvec; c += GT) {
+                const uint2 q = quant8<Q>(row[c], scale, inv, zero);
+#pragma unroll
+                for (int k = 0; k < MOEDISP_MAX_K; ++k)
+                    if (d[k] >= 0)
+                        __stcs(reinterpret_cast<uint2*>(a.expand_x + (int64_t)d[k] * a.out_bytes) + c, q);
+            }
         }
         if (gt < K) {
             const int32_t dt = drow[grp][st][gt];
@@ -397,8 +411,8 @@ cudaError_t launch_copy(DispatchArgs a, cudaStream_t stream) {
 template <int Q, int WPT>
 cudaError_t launch_quant_w(DispatchArgs a, cudaStream_t stream) {
     constexpr int NG = kQuantThreads / 32 / WPT;
-    // Three stages per group: one being read, one or two loading.
-    a.stages = 3;
+    // Two stages per group: one being read while the next loads.
+    a.stages = 2;
     const size_t smem = (size_t)NG * a.stages * a.in_bytes;
     int per_sm = 1;
     cudaError_t err = blocks_per_sm((const void*)dispatch_quant_kernel<Q, WPT>, kQuantThreads, smem,
