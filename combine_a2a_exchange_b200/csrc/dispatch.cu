@@ -411,8 +411,9 @@ cudaError_t launch_copy(DispatchArgs a, cudaStream_t stream) {
 template <int Q, int WPT>
 cudaError_t launch_quant_w(DispatchArgs a, cudaStream_t stream) {
     constexpr int NG = kQuantThreads / 32 / WPT;
-    // Two stages per group: one being read while the next loads.
-    a.stages = 2;
+    // Stages per group: two for single-warp groups (small rows: more blocks per SM pays
+    // more), three for wider groups (large rows: deeper look-ahead pays more); measured.
+    a.stages = WPT == 1 ? 2 : 3;
     const size_t smem = (size_t)NG * a.stages * a.in_bytes;
     int per_sm = 1;
     cudaError_t err = blocks_per_sm((const void*)dispatch_quant_kernel<Q, WPT>, kQuantThreads, smem,
