@@ -213,6 +213,21 @@ class MoEStep:
         main.wait_stream(self.side)
 
 
+def max_over_ranks(torch, value: float, device=None) -> float:
+    """The largest of every rank's value (no-op without a multi-rank process group)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: int, world: int, ms: float) -> float:
+    """Units per second over all ranks, for a step time that is the max over ranks."""
+    return world * units_per_rank / (ms / 1e3)
+
+
 def capture(torch, fn):
     """CUDA graph of fn's launches (one eager run first, outside the capture)."""
     fn()
@@ -492,6 +507,8 @@ def main():
     ap.add_argument("--workload", default="cfg2")
     ap.add_argument("--T", type=int, default=None,
                     help="tokens per rank override (smaller cases for profiling)")
+    ap.add_argument("--a2a-W", type=int, default=64, help="ranks of the a2a64 workload")
+    ap.add_argument("--a2a-max-split", type=int, default=512, help="split bound of a2a64")
     ap.add_argument("--no-ops", action="store_true", help="skip the per-op sweep of other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -508,6 +525,8 @@ def main():
         if rank != 0:
             return 0
         return run_reference(args, wl)
+    if args.workload == "a2a64":
+        return run_a2a(args, wl, world, rank, local_rank)
 
     import torch
     import torch.distributed as dist
@@ -558,11 +577,7 @@ def main():
     if status != 0:
         raise RuntimeError(f"device status after the timed steps: {md.status_string(status)}")
 
-    ms_step = statistics.mean(t_step)
-    if world > 1:
-        tt = torch.tensor([ms_step], device=device, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_step = float(tt.item())
+    ms_step = max_over_ranks(torch, statistics.mean(t_step), device)
     R = int(step.L.expert_base[-1].item())
     per_op = {op: statistics.mean(t[op]) for op in ("layout", "plan", "dispatch", "combine")}
     dom = max(("dispatch", "combine"), key=lambda o: per_op[o])
@@ -574,11 +589,8 @@ def main():
     e2e = None
     if not args.no_e2e:
         ms_e2e, h2d, d2h = time_e2e(torch, step, args.steps, args.warmup, flush, device)
-        if world > 1:
-            tt = torch.tensor([ms_e2e], device=device, dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            ms_e2e = float(tt.item())
-        e2e = {"value": round(world * w.G / (ms_e2e / 1e3), 1), "unit": UNIT,
+        ms_e2e = max_over_ranks(torch, ms_e2e, device)
+        e2e = {"value": round(whole_job_rate(w.G, world, ms_e2e), 1), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": round(ms_e2e, 4)}
 
@@ -600,7 +612,7 @@ def main():
     step_bytes = sum(algorithmic_bytes(op, w, R) for op in ("layout", "dispatch", "combine"))
     line = {
         "metric": METRIC,
-        "value": round(world * w.G / (ms_step / 1e3), 1),
+        "value": round(whole_job_rate(w.G, world, ms_step), 1),
         "unit": UNIT,
         "n_gpus": world,
         "steps": args.steps,
@@ -630,6 +642,51 @@ def main():
         "ops": ops,
     }
     print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_a2a(args, wl, world, rank, local_rank):
+    """The raw uneven all-to-all-v workload as the step: exchange plan + a2a_v over W
+    virtual ranks (rows of 4096 bf16 labelled 10*i+k). Metric: moved rows/s and GB/s."""
+    import torch
+    import combine_a2a_exchange_b200 as md
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    hbm, peak_src = measured_peaks()
+    a = wl.a2a_workload(seed=rank, W=args.a2a_W, max_split=args.a2a_max_split)
+    W, E_ = a.W, a.row_elems
+    cap_in, cap_out = a.cap_in, a.cap_out
+    S = torch.from_numpy(a.in_splits).to(device)
+    plan = [torch.empty((W, W), dtype=torch.int64, device=device) for _ in range(3)]
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    i = torch.arange(W, device=device, dtype=torch.float32)[:, None]
+    k = torch.arange(cap_in, device=device, dtype=torch.float32)[None, :]
+    inp = (10.0 * i + k).to(torch.bfloat16)[:, :, None].expand(W, cap_in, E_).contiguous()
+    out = torch.empty((W, cap_out, E_), dtype=torch.bfloat16, device=device)
+
+    def step():
+        md.a2a_exchange_plan(S, plan[0], plan[1], plan[2], status)
+        md.a2a_v(inp, cap_in, out, cap_out, 2 * E_, W, plan[0], plan[1], plan[2], status)
+
+    flush = L2Flush(torch, device)
+    g = capture(torch, step)
+    ms = statistics.mean(time_graph(torch, g, args.steps, args.warmup, flush))
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise RuntimeError(md.status_string(int(status.item())))
+    ms = max_over_ranks(torch, ms, device)
+    if rank == 0:
+        b = algorithmic_bytes("a2a_v", a2a=a)
+        print(json.dumps({
+            "metric": "a2a_v moved rows/s (plan + exchange), 1 GPU", "value":
+            round(whole_job_rate(a.moved_rows(), world, ms), 1), "unit": "rows/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16 rows (copied as bytes)", "data": "synthetic",
+            "config": {"workload": f"a2a: W={W}, splits ~ randint[0,{args.a2a_max_split}) with 10% "
+                                   f"zeros, rows of {E_} bf16", "moved_rows": a.moved_rows()},
+            "hbm_GBps": round(b / (ms * 1e-3) / 1e9, 1), "peak": hbm, "peak_source": peak_src,
+            "gpu_launches": 2 * args.steps}), flush=True)
     return 0
 
 
