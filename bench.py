@@ -553,6 +553,7 @@ def main():
     sampler = ClockSampler(enabled=(rank == 0))
 
     g_step = capture(torch, step.run)
+    sampler.start()                    # clocks sampled over warm-up, timed steps, per-op timing
     for _ in range(args.warmup):
         flush.zero_()
         g_step.replay()
@@ -560,19 +561,18 @@ def main():
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    sampler.start()
     t_step = time_graph(torch, g_step, args.steps, 0, flush)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    clocks = sampler.stop([uuid.replace("GPU-", "")] if uuid else None) if rank == 0 else None
     del g_step
     t = time_ops_in_graph(torch, step, args.steps, args.warmup, flush)
     op_timing = "event-record nodes inside a graph of the step"
     if t is None:
         t = time_ops(torch, step, args.steps, args.warmup, flush)
         op_timing = "eager launches right behind the L2 flush"
+    clocks = sampler.stop([uuid.replace("GPU-", "")] if uuid else None) if rank == 0 else None
     status = int(step.status.item())
     if status != 0:
         raise RuntimeError(f"device status after the timed steps: {md.status_string(status)}")
@@ -583,7 +583,7 @@ def main():
     dom = max(("dispatch", "combine"), key=lambda o: per_op[o])
     dom_bytes = algorithmic_bytes(dom, w, R)
     achieved = dom_bytes / (per_op[dom] * 1e-3) / 1e9
-    kernel_key = {"dispatch": "dispatch_kernel<0>", "combine": "combine_kernel<8>"}[dom]
+    kernel_key = {"dispatch": "dispatch_copy_kernel", "combine": f"combine_kernel<{w.K}>"}[dom]
     traffic = ncu_traffic(kernel_key)
 
     e2e = None
