@@ -67,6 +67,7 @@ def _sig(name, argtypes, restype=ctypes.c_int):
 
 _status_string = _sig("moedisp_status_string", [_I], ctypes.c_char_p)
 _version = _sig("moedisp_version", [])
+_selftest_wait = _sig("moedisp_selftest_bounded_wait", [ctypes.c_uint32, _P, _P])
 _plan = _sig("moedisp_a2a_exchange_plan", [_P, _I, _P, _P, _P, _P, _P])
 _a2a_v = _sig("moedisp_a2a_v", [_P, _I64, _P, _I64, _I64, _I, _P, _P, _P, _P, _P])
 _ws_size = _sig("moedisp_layout_workspace_size", [Dims, ctypes.POINTER(ctypes.c_size_t)])
@@ -115,6 +116,12 @@ def _check(rc: int, call: str, raise_on_error: bool) -> int:
     if rc < 0 and raise_on_error:
         raise MoedispError(rc, call)
     return rc
+
+
+def selftest_bounded_wait(limit_us, status, stream=None, raise_on_error=True) -> int:
+    """Runs the device-side wait time-out diagnostic (see include/moedisp.h)."""
+    rc = _selftest_wait(int(limit_us), _ptr(status), _stream(stream))
+    return _check(rc, "selftest_bounded_wait", raise_on_error)
 
 
 # ------------------------------------------------------------------ exchange
@@ -225,6 +232,10 @@ def moe_combine(expert_out, H, layout: LayoutBuffers, expert_scales, y, status, 
     return _check(rc, "moe_combine", raise_on_error)
 
 
+def raw_selftest(limit_us, status_ptr) -> int:
+    return int(_selftest_wait(int(limit_us), status_ptr, None))
+
+
 def raw_call(name: str, *args) -> int:
     """Calls an exported C function with already-marshalled arguments (for ABI tests)."""
     return int({"moedisp_a2a_exchange_plan": _plan, "moedisp_a2a_v": _a2a_v,
@@ -236,6 +247,7 @@ def raw_call(name: str, *args) -> int:
 __all__ = [
     "a2a_exchange_plan", "a2a_v", "layout_workspace_size", "LayoutBuffers",
     "moe_dispatch_layout", "moe_dispatch_layout_noalloc", "moe_dispatch", "moe_combine",
+    "selftest_bounded_wait",
     "status_string", "version", "NOALLOC_SCRATCH_BYTES",
     "Dims", "Layout", "MoedispError", "LIBRARY_PATH",
     "QUANT_NONE", "QUANT_INT8", "QUANT_FP8_E4M3",

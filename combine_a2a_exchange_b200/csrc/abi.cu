@@ -91,6 +91,13 @@ const char* moedisp_status_string(int code) {
 
 int moedisp_version(void) { return 1; }
 
+int moedisp_selftest_bounded_wait(uint32_t limit_us, int32_t* status, moedisp_stream_t stream) {
+    if (!status) return MOEDISP_ERR_NULLPTR;
+    if (!aligned(status, 4)) return MOEDISP_ERR_MISALIGNED;
+    if (limit_us < 1 || limit_us > 10000000u) return MOEDISP_ERR_INVALID;
+    return rc(moedisp::launch_bounded_wait_selftest((uint64_t)limit_us * 1000ull, status, stream));
+}
+
 int moedisp_a2a_exchange_plan(const int64_t* in_splits, int W, int64_t* src_offsets,
                               int64_t* out_splits, int64_t* dst_offsets, int32_t* status,
                               moedisp_stream_t stream) {

@@ -90,15 +90,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return done != 0;
 }
 
-// Waits for the phase with the given parity to complete; false after kWaitLimitNs.
+// Waits for the phase with the given parity to complete; false after limit_ns.
 // (try_wait itself suspends the thread for a while; the clock is read every 64 polls.)
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 63u) == 0u && global_timer_ns() - t0 > kWaitLimitNs) return false;
+        if ((i & 63u) == 0u && global_timer_ns() - t0 > limit_ns) return false;
     }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+    return mbar_wait_for(bar, parity, kWaitLimitNs);
 }
 
 // ------------------------------------------------------- 1-D bulk (TMA) copies

@@ -241,8 +241,8 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
 }
 
 // Quantising dispatch. A block of kQuantThreads threads is split into token groups of WPT
-// warps; each group is an independent pipeline over its own tokens, with its own
-// shared-memory stages and barriers. The group's first lane streams token rows into the
+// warps; each group is an independent pipeline over the tokens it draws from the block's
+// share, with its own shared-memory stages and barriers. The group's first lane streams token rows into the
 // stages (bulk loads); the group reduces the row's max |x| (warp shuffles, plus a named
 // barrier across the group's warps when WPT > 1 -- that barrier also carries the
 // time-out verdict), then each thread quantises its 16-byte chunks of the row and writes
@@ -265,6 +265,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) dispatch_quant_kernel(Dispat
     __shared__ int32_t drow[NG][kMaxStages][MOEDISP_MAX_K];
     __shared__ float red[NG][2][WPT];
     __shared__ int abort_s[NG];
+    __shared__ unsigned next_s;                      // the block's next token index
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int grp = warp / WPT, gw = warp - grp * WPT, gt = tid - grp * GT;
     const int S = a.stages, K = a.K;
@@ -276,22 +277,36 @@ __global__ void __launch_bounds__(kQuantThreads, 2) dispatch_quant_kernel(Dispat
         fence_mbar_init();
         abort_s[grp] = 0;
     }
+    if (tid == 0) next_s = 0;
     __syncthreads();
     grid_dep_wait();
     grid_dep_launch_dependents();
     write_recv_counts(a);
 
-    // The group's first warp arms stages. The routing (K destination rows) of the token
+    // The group's first warp arms stages. The block's tokens are g = blockIdx.x + i *
+    // gridDim.x; the groups draw i from a shared counter, so a group that meets
+    // inactive tokens simply takes more. The routing (K destination rows) of the token
     // after the one being armed is loaded one fill ahead.
-    const int64_t n_groups = (int64_t)gridDim.x * NG;
-    int64_t pf_g = (int64_t)blockIdx.x * NG + grp;
-    int32_t pf_d = (gw == 0 && pf_g < a.G && lane < K) ? __ldg(a.dst_row + pf_g * K + lane) : -1;
+    auto next_token = [&]() -> int64_t {
+        unsigned i = 0;
+        if (lane == 0) i = atomicAdd(&next_s, 1u);
+        i = __shfl_sync(0xffffffffu, i, 0);
+        return (int64_t)blockIdx.x + (int64_t)i * gridDim.x;
+    };
+    int64_t pf_g = 0;
+    int32_t pf_d = -1;
+    if (gw == 0) {
+        pf_g = next_token();
+        pf_d = (pf_g < a.G && lane < K) ? __ldg(a.dst_row + pf_g * K + lane) : -1;
+    }
     auto fill = [&](int st) {
         while (true) {
             const int64_t g = pf_g;
             int32_t d = pf_d;
-            pf_g = g + n_groups;
-            pf_d = (pf_g < a.G && lane < K) ? __ldg(a.dst_row + pf_g * K + lane) : -1;
+            if (g < a.G) {
+                pf_g = next_token();
+                pf_d = (pf_g < a.G && lane < K) ? __ldg(a.dst_row + pf_g * K + lane) : -1;
+            }
             if (g >= a.G) {
                 if (lane == 0) {
                     tok[grp][st] = -1;

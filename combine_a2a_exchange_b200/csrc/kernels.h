@@ -80,6 +80,8 @@ cudaError_t launch_layout_noalloc(const int32_t* expert_ids, const uint8_t* acti
                                   const moedisp_dims& dims, const moedisp_layout& layout,
                                   int32_t* status, cudaStream_t stream);
 
+cudaError_t launch_bounded_wait_selftest(uint64_t limit_ns, int32_t* status, cudaStream_t stream);
+
 cudaError_t launch_dispatch(const void* x, int H, const moedisp_dims& dims,
                             const moedisp_layout& layout, int quant_mode, void* expand_x,
                             float* dynamic_scales, int64_t* expert_token_nums,

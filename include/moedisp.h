@@ -67,6 +67,14 @@ const char *moedisp_status_string(int code);
 /* ABI version, currently 1. */
 int moedisp_version(void);
 
+/* Diagnostic for the time-out path of the device-side waits (this library's own
+ * addition; the pages' kernels spin without a limit). Enqueues a one-thread kernel that
+ * waits, through the same bounded-wait helper every kernel uses, on a barrier phase that
+ * nothing completes; after limit_us microseconds (1..10^7) it must give up and OR
+ * MOEDISP_STATUS_TIMEOUT into *status (device memory). No fault, trap or hang: the
+ * context stays usable. */
+int moedisp_selftest_bounded_wait(uint32_t limit_us, int32_t *status, moedisp_stream_t stream);
+
 /* ------------------------------------------------------------------------------------
  * a2a_exchange_plan
  *

@@ -159,6 +159,12 @@ def test_dispatch_and_combine_rejections(md):
                        None, None, st, None) == md.MOEDISP_OK
 
 
+def test_selftest_rejections(md):
+    assert md.raw_selftest(10, None) == md.MOEDISP_ERR_NULLPTR
+    assert md.raw_selftest(0, FAKE) == md.MOEDISP_ERR_INVALID
+    assert md.raw_selftest(10, FAKE + 2) == md.MOEDISP_ERR_MISALIGNED
+
+
 def test_binding_has_no_fallback():
     """The package refuses to import without the compiled library."""
     src = open(os.path.join(ROOT, "combine_a2a_exchange_b200", "__init__.py")).read()

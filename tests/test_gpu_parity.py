@@ -521,3 +521,19 @@ def test_dispatch_then_combine(md, name, over, q):
         exp = xf * (wsum * act)[:, None]
         yf = wl.bf16_bits_to_f32(yb).astype(np.float64)
         assert (np.abs(yf - exp) <= ATOL + RTOL * np.abs(exp)).all()
+
+
+# ------------------------------------------------------- failure detection
+
+def test_bounded_wait_times_out_and_context_survives(md):
+    """A device-side wait on a barrier that nothing completes gives up after its limit
+    and reports TIMEOUT; the GPU context stays usable (a layout runs right after)."""
+    st = new_status()
+    md.selftest_bounded_wait(20000, st)                       # 20 ms
+    torch.cuda.synchronize()
+    assert int(st.item()) == md.STATUS_TIMEOUT
+    w = wl.moe_workload("tiny", seed=1)
+    L, st2 = run_layout(md, w)
+    ref = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active)
+    assert st2 == 0
+    assert_layout_equal(layout_host(L), ref, ref["R"], ref["rows_cap"])
