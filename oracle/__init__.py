@@ -68,7 +68,10 @@ def lib() -> ctypes.CDLL:
         L.orc_quant_row.restype = ctypes.c_float
         L.orc_moe_combine_f64.argtypes = [i32, i32, i32, P, i64, P, P, P]
         L.orc_moe_combine_f32.argtypes = [i32, i32, i32, P, i64, P, P, P]
-        for f in ("orc_a2a_exchange_plan", "orc_a2a_v", "orc_moe_dispatch_layout",
+        L.orc_moe_combine_rmsnorm_f64.argtypes = [i32, i32, i32, P, i64, P, P, P, P, ctypes.c_float, P, P]
+        L.orc_moe_combine_rmsnorm_f32.argtypes = [i32, i32, i32, P, i64, P, P, P, P, ctypes.c_float, P, P]
+        for f in ("orc_moe_combine_rmsnorm_f64", "orc_moe_combine_rmsnorm_f32",
+                  "orc_a2a_exchange_plan", "orc_a2a_v", "orc_moe_dispatch_layout",
                   "orc_moe_recv_counts", "orc_moe_dispatch", "orc_moe_combine_f64",
                   "orc_moe_combine_f32"):
             getattr(L, f).restype = ctypes.c_int
@@ -217,3 +220,29 @@ def moe_combine_f32(expert_out_bits, dst_row, weights, K: int, rows_cap: int | N
     y = np.zeros((G, H), np.uint16)
     fl = lib().orc_moe_combine_f32(G, K, H, _p(eo), rows_cap, _p(dr), _p(w), _p(y))
     return y, fl
+
+
+# ------------------------------------------------------------- fused tail
+
+def moe_combine_rmsnorm(expert_out_bits, dst_row, weights, K: int, residual_bits, gamma,
+                        eps: float, rows_cap: int | None = None, exact: str = "f64"):
+    """Returns (residual_out bf16 bits, y) with y fp64 (exact='f64') or bf16 bits ('f32')."""
+    eo = _c(expert_out_bits, np.uint16)
+    dr = _c(dst_row, np.int32).reshape(-1)
+    w = _c(weights, np.float32).reshape(-1)
+    res = _c(residual_bits, np.uint16)
+    gm = _c(gamma, np.float32)
+    G = dr.size // K
+    H = res.shape[1]
+    if rows_cap is None:
+        rows_cap = eo.shape[0]
+    rout = np.zeros((G, H), np.uint16)
+    if exact == "f64":
+        y = np.zeros((G, H), np.float64)
+        fl = lib().orc_moe_combine_rmsnorm_f64(G, K, H, _p(eo), rows_cap, _p(dr), _p(w), _p(res),
+                                               _p(gm), eps, _p(rout), _p(y))
+    else:
+        y = np.zeros((G, H), np.uint16)
+        fl = lib().orc_moe_combine_rmsnorm_f32(G, K, H, _p(eo), rows_cap, _p(dr), _p(w), _p(res),
+                                               _p(gm), eps, _p(rout), _p(y))
+    return rout, y, fl

@@ -377,3 +377,75 @@ int orc_moe_combine_f32(int G, int K, int H, const uint16_t *expert_out, int64_t
     free(acc);
     return flags;
 }
+
+/* ------------------------------------------------------- fused tail (RMSNorm) */
+
+/* [P5] MoE finalize followed by the residual add and RMSNorm: the prenorm row is the
+ * token's combined row plus its residual (kept as residual_out in bf16), normalised by
+ * the root mean square of that bf16 row (plus eps) and scaled by gamma. */
+int orc_moe_combine_rmsnorm_f64(int G, int K, int H, const uint16_t *expert_out,
+                                int64_t rows_cap, const int32_t *dst_row, const float *w,
+                                const uint16_t *residual, const float *gamma, float eps,
+                                uint16_t *residual_out, double *y64)
+{
+    int flags = 0;
+    double *s = (double *)malloc(sizeof(double) * (size_t)(H > 0 ? H : 1));
+    for (int64_t g = 0; g < G; g++) {
+        for (int h = 0; h < H; h++) s[h] = (double)orc_bf16_to_f32(residual[g * (int64_t)H + h]);
+        for (int k = 0; k < K; k++) {
+            int32_t row = dst_row[g * K + k];
+            if (row < 0) continue;
+            if (row >= rows_cap) { flags |= ORC_CAPACITY; continue; }
+            const uint16_t *v = expert_out + (int64_t)row * H;
+            double wk = (double)w[g * K + k];
+            for (int h = 0; h < H; h++) s[h] += wk * (double)orc_bf16_to_f32(v[h]);
+        }
+        double ss = 0.0;
+        for (int h = 0; h < H; h++) {
+            uint16_t r = orc_bf16_from_f32((float)s[h]);
+            residual_out[g * (int64_t)H + h] = r;
+            double rv = (double)orc_bf16_to_f32(r);
+            ss += rv * rv;
+        }
+        double inv = 1.0 / sqrt(ss / H + (double)eps);
+        for (int h = 0; h < H; h++)
+            y64[g * (int64_t)H + h] = (double)orc_bf16_to_f32(residual_out[g * (int64_t)H + h]) * inv *
+                                      (double)gamma[h];
+    }
+    free(s);
+    return flags;
+}
+
+int orc_moe_combine_rmsnorm_f32(int G, int K, int H, const uint16_t *expert_out,
+                                int64_t rows_cap, const int32_t *dst_row, const float *w,
+                                const uint16_t *residual, const float *gamma, float eps,
+                                uint16_t *residual_out, uint16_t *y)
+{
+    int flags = 0;
+    float *acc = (float *)malloc(sizeof(float) * (size_t)(H > 0 ? H : 1));
+    for (int64_t g = 0; g < G; g++) {
+        for (int h = 0; h < H; h++) acc[h] = 0.0f;
+        for (int k = 0; k < K; k++) {
+            int32_t row = dst_row[g * K + k];
+            if (row < 0) continue;
+            if (row >= rows_cap) { flags |= ORC_CAPACITY; continue; }
+            const uint16_t *v = expert_out + (int64_t)row * H;
+            float wk = w[g * K + k];
+            for (int h = 0; h < H; h++) acc[h] = fmaf(wk, orc_bf16_to_f32(v[h]), acc[h]);
+        }
+        float ss = 0.0f;
+        for (int h = 0; h < H; h++) {
+            float sv = acc[h] + orc_bf16_to_f32(residual[g * (int64_t)H + h]);
+            uint16_t r = orc_bf16_from_f32(sv);
+            residual_out[g * (int64_t)H + h] = r;
+            float rv = orc_bf16_to_f32(r);
+            ss = fmaf(rv, rv, ss);
+        }
+        float inv = 1.0f / sqrtf(ss / (float)H + eps);
+        for (int h = 0; h < H; h++)
+            y[g * (int64_t)H + h] =
+                orc_bf16_from_f32(orc_bf16_to_f32(residual_out[g * (int64_t)H + h]) * inv * gamma[h]);
+    }
+    free(acc);
+    return flags;
+}

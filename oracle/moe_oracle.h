@@ -74,6 +74,21 @@ int orc_moe_combine_f64(int G, int K, int H, const uint16_t *expert_out, int64_t
 int orc_moe_combine_f32(int G, int K, int H, const uint16_t *expert_out, int64_t rows_cap,
                         const int32_t *dst_row, const float *w, uint16_t *y);
 
+/* Fused tail, MoE finalize + residual + RMSNorm ([P5]), on one GPU:
+ *   s      = combine(g) + residual[g]           (the combine as in O5)
+ *   res    = bf16(s)                            residual_out
+ *   y[g,h] = bf16( res[h] / sqrt(mean_h res^2 + eps) * gamma[h] )
+ * _f64: every step in double (res rounded to bf16 as defined); _f32: the fixed-order fp32
+ * FMA chain, one fp32 add of the residual, the sum of squares in ascending h. */
+int orc_moe_combine_rmsnorm_f64(int G, int K, int H, const uint16_t *expert_out,
+                                int64_t rows_cap, const int32_t *dst_row, const float *w,
+                                const uint16_t *residual, const float *gamma, float eps,
+                                uint16_t *residual_out, double *y64);
+int orc_moe_combine_rmsnorm_f32(int G, int K, int H, const uint16_t *expert_out,
+                                int64_t rows_cap, const int32_t *dst_row, const float *w,
+                                const uint16_t *residual, const float *gamma, float eps,
+                                uint16_t *residual_out, uint16_t *y);
+
 #ifdef __cplusplus
 }
 #endif

@@ -470,3 +470,65 @@ def _round_f32(q: Fraction) -> float:
     best = min(cands, key=lambda c: (abs(Fraction(c) - q),
                                      int(np.float32(c).view(np.uint32)) & 1))
     return best
+
+
+# ----------------------------------------------------- fused tail pins (RMSNorm)
+
+def _rms_case(seed=12, G=6, K=3, H=48, R=20):
+    rng = np.random.default_rng(seed)
+    eo = wl.f32_to_bf16_bits(rng.standard_normal((R, H)).astype(np.float32))
+    dr = rng.integers(-1, R, size=(G, K)).astype(np.int32)
+    w = rng.random((G, K)).astype(np.float32)
+    res = wl.f32_to_bf16_bits(rng.standard_normal((G, H)).astype(np.float32))
+    gamma = (0.5 + rng.random(H)).astype(np.float32)
+    return eo, dr, w, res, gamma
+
+
+def test_rmsnorm_residual_out_brute_force():
+    """residual_out = bf16(fp32 FMA chain over k + fp32 residual), by exact rationals."""
+    eo, dr, w, res, gamma = _rms_case()
+    rout, _, fl = oracle.moe_combine_rmsnorm(eo, dr, w, 3, res, gamma, 1e-6, exact="f32")
+    assert fl == 0
+    G, H = res.shape
+    for g in range(G):
+        for h in range(H):
+            acc = np.float32(0)
+            for k in range(3):
+                if dr[g, k] >= 0:
+                    p = Fraction(float(w[g, k])) * Fraction(float(wl.bf16_bits_to_f32(eo[dr[g, k], h])))
+                    acc = np.float32(_round_f32(p + Fraction(float(acc))))
+            s = np.float32(acc) + np.float32(wl.bf16_bits_to_f32(res[g, h]))
+            ref = torch.tensor([float(s)], dtype=torch.float32).to(torch.bfloat16)
+            assert rout[g, h] == ref.view(torch.int16).numpy().view(np.uint16)[0]
+
+
+def test_rmsnorm_matches_torch_rms_norm():
+    """The normalisation step is torch's rms_norm (a library routine) of residual_out."""
+    eo, dr, w, res, gamma = _rms_case(seed=13, G=9, H=64)
+    eps = 1e-5
+    rout, y64, _ = oracle.moe_combine_rmsnorm(eo, dr, w, 3, res, gamma, eps, exact="f64")
+    r = torch.from_numpy(wl.bf16_bits_to_f32(rout).astype(np.float64))
+    ref = torch.nn.functional.rms_norm(r, (r.shape[1],), torch.from_numpy(gamma.astype(np.float64)), eps)
+    assert np.allclose(y64, ref.numpy(), rtol=1e-12, atol=1e-12)
+    rout32, y32, _ = oracle.moe_combine_rmsnorm(eo, dr, w, 3, res, gamma, eps, exact="f32")
+    assert np.array_equal(rout32, rout)
+    yf = wl.bf16_bits_to_f32(y32).astype(np.float64)
+    assert (np.abs(yf - y64) <= 1e-2 + 1e-2 * np.abs(y64)).all()
+
+
+def test_rmsnorm_closed_form_properties():
+    """With gamma = 1 every row's mean square is mean(r^2) / (mean(r^2) + eps); scaling
+    gamma scales y; the residual adds exactly into the combined row."""
+    eo, dr, w, res, gamma = _rms_case(seed=14, G=5, H=96)
+    ones = np.ones_like(gamma)
+    eps = 0.25
+    rout, y64, _ = oracle.moe_combine_rmsnorm(eo, dr, w, 3, res, ones, eps)
+    r = wl.bf16_bits_to_f32(rout).astype(np.float64)
+    ms = (r * r).mean(axis=1)
+    assert np.allclose((y64 * y64).mean(axis=1), ms / (ms + eps), rtol=1e-12)
+    _, y64b, _ = oracle.moe_combine_rmsnorm(eo, dr, w, 3, res, 3.0 * ones, eps)
+    assert np.allclose(y64b, 3.0 * y64, rtol=1e-12)
+    zero = np.zeros_like(res)
+    rz, _, _ = oracle.moe_combine_rmsnorm(eo, dr, w, 3, zero, ones, eps)
+    yc, _ = oracle.moe_combine_f64(eo, dr, w, 3)
+    assert np.allclose(wl.bf16_bits_to_f32(rz), yc, rtol=2 ** -8, atol=1e-30)
