@@ -149,6 +149,9 @@ def algorithmic_bytes(op, w=None, R=None, a2a=None):
         return R * H * 2 + G * H * 2 + G * K * 8
     if op == "layout":
         return G * K * 4 + (0 if w.active is None else G) + 2 * G * K * 4 + R * 4
+    if op == "combine_rmsnorm":
+        # expert rows + residual read, residual_out + y written, gamma, routing
+        return R * H * 2 + 3 * G * H * 2 + H * 4 + G * K * 8
     raise ValueError(op)
 
 
@@ -457,6 +460,37 @@ def op_sweep(md, torch, device, hbm, reps=10):
                     "tokens/s": round(w.G / (statistics.mean(t_step) / 1e3), 1)})
         assert int(st.status.item()) == 0, md.status_string(int(st.status.item()))
         del st
+        torch.cuda.empty_cache()
+    # fused tail: combine + residual add + RMSNorm (residual_out written), after the step's
+    # layout and dispatch
+    for name in ("cfg2", "cfg3"):
+        w = wl.moe_workload(name, seed=0)
+        st = MoEStep(md, torch, w, device)
+        st.run()
+        g = torch.Generator(device=device).manual_seed(11)
+        res = torch.randn((w.G, w.H), generator=g, device=device).to(torch.bfloat16)
+        gamma = 0.5 + torch.rand((w.H,), generator=g, device=device)
+        rout = torch.empty_like(res)
+        Ev = torch.cuda.Event
+        pairs = []
+        for r in range(reps + 3):
+            flush.zero_()
+            e0, e1 = Ev(enable_timing=True), Ev(enable_timing=True)
+            e0.record()
+            md.moe_combine_rmsnorm(st.expert_out, w.H, st.L, st.wts, res, gamma, 1e-6, st.y,
+                                   st.status, residual_out=rout)
+            e1.record()
+            if r >= 3:
+                pairs.append((e0, e1))
+        torch.cuda.synchronize()
+        assert int(st.status.item()) == 0, md.status_string(int(st.status.item()))
+        ms = statistics.mean(a.elapsed_time(b) for a, b in pairs)
+        R = int(st.L.expert_base[-1].item())
+        b = algorithmic_bytes("combine_rmsnorm", w, R)
+        out.append({"workload": name, "op": "combine_rmsnorm", "us": round(ms * 1e3, 2),
+                    "bytes": b, "GB/s": round(b / ms / 1e6, 1),
+                    "frac": round(b / ms / 1e6 / hbm, 4)})
+        del st, res, rout
         torch.cuda.empty_cache()
     # raw all-to-all-v, W = 64
     a = wl.a2a_workload(seed=0)

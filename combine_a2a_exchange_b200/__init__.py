@@ -78,6 +78,8 @@ _layout_noalloc = _sig("moedisp_moe_dispatch_layout_noalloc",
 _dispatch = _sig("moedisp_moe_dispatch",
                  [_P, _I, Dims, ctypes.POINTER(Layout), _I, _P, _P, _P, _I, _P, _P, _P])
 _combine = _sig("moedisp_moe_combine", [_P, _I, Dims, ctypes.POINTER(Layout), _P, _P, _P, _P])
+_combine_rms = _sig("moedisp_moe_combine_rmsnorm",
+                    [_P, _I, Dims, ctypes.POINTER(Layout), _P, _P, _P, ctypes.c_float, _P, _P, _P, _P])
 
 
 class MoedispError(RuntimeError):
@@ -232,6 +234,15 @@ def moe_combine(expert_out, H, layout: LayoutBuffers, expert_scales, y, status, 
     return _check(rc, "moe_combine", raise_on_error)
 
 
+def moe_combine_rmsnorm(expert_out, H, layout: LayoutBuffers, expert_scales, residual, gamma,
+                        eps, y, status, residual_out=None, stream=None, raise_on_error=True) -> int:
+    L = layout.struct()
+    rc = _combine_rms(_ptr(expert_out), int(H), layout.dims, ctypes.byref(L), _ptr(expert_scales),
+                      _ptr(residual), _ptr(gamma), float(eps), _ptr(residual_out), _ptr(y),
+                      _ptr(status), _stream(stream))
+    return _check(rc, "moe_combine_rmsnorm", raise_on_error)
+
+
 def raw_selftest(limit_us, status_ptr) -> int:
     return int(_selftest_wait(int(limit_us), status_ptr, None))
 
@@ -241,13 +252,14 @@ def raw_call(name: str, *args) -> int:
     return int({"moedisp_a2a_exchange_plan": _plan, "moedisp_a2a_v": _a2a_v,
                 "moedisp_moe_dispatch_layout": _layout,
                 "moedisp_moe_dispatch_layout_noalloc": _layout_noalloc,
-                "moedisp_moe_dispatch": _dispatch, "moedisp_moe_combine": _combine}[name](*args))
+                "moedisp_moe_dispatch": _dispatch, "moedisp_moe_combine": _combine,
+                "moedisp_moe_combine_rmsnorm": _combine_rms}[name](*args))
 
 
 __all__ = [
     "a2a_exchange_plan", "a2a_v", "layout_workspace_size", "LayoutBuffers",
     "moe_dispatch_layout", "moe_dispatch_layout_noalloc", "moe_dispatch", "moe_combine",
-    "selftest_bounded_wait",
+    "selftest_bounded_wait", "moe_combine_rmsnorm",
     "status_string", "version", "NOALLOC_SCRATCH_BYTES",
     "Dims", "Layout", "MoedispError", "LIBRARY_PATH",
     "QUANT_NONE", "QUANT_INT8", "QUANT_FP8_E4M3",

@@ -292,4 +292,37 @@ int moedisp_moe_combine(const void* expert_out, int H, moedisp_dims dims,
     return rc(moedisp::launch_combine(expert_out, H, dims, L, expert_scales, y, status, stream));
 }
 
+int moedisp_moe_combine_rmsnorm(const void* expert_out, int H, moedisp_dims dims,
+                                const moedisp_layout* layout, const float* expert_scales,
+                                const void* residual, const float* gamma, float eps,
+                                void* residual_out, void* y, int32_t* status,
+                                moedisp_stream_t stream) {
+    if (!layout || !status) return MOEDISP_ERR_NULLPTR;
+    int c = check_dims(dims);
+    if (c != MOEDISP_OK) return c;
+    const moedisp_layout& L = *layout;
+    if ((c = check_rows_cap(L.rows_cap)) != MOEDISP_OK) return c;
+    if (H <= 0 || !(eps >= 0.0f) || eps > 1.0e30f) return MOEDISP_ERR_INVALID;
+    if (H % 8 != 0) return MOEDISP_ERR_MISALIGNED;
+    if (H > MOEDISP_MAX_H) return MOEDISP_ERR_UNSUPPORTED;
+    const int64_t G = (int64_t)dims.W * dims.T;
+    if (G == 0) return MOEDISP_OK;
+    if (!y || !expert_scales || !L.dst_row || !residual || !gamma) return MOEDISP_ERR_NULLPTR;
+    if (L.rows_cap > 0 && !expert_out) return MOEDISP_ERR_NULLPTR;
+    if (!aligned(expert_out, 16) || !aligned(y, 16) || !aligned(residual, 16) ||
+        !aligned(residual_out, 16) || !aligned(gamma, 16) || !aligned(expert_scales, 4) ||
+        !aligned(L.dst_row, 4) || !aligned(status, 4))
+        return MOEDISP_ERR_MISALIGNED;
+    const size_t rowb = (size_t)G * H * 2;
+    if (any_alias({{y, rowb}, {residual_out, rowb}, {status, 4}},
+                  {{expert_out, (size_t)L.rows_cap * H * 2},
+                   {residual, rowb},
+                   {gamma, (size_t)H * 4},
+                   {expert_scales, (size_t)G * dims.K * 4},
+                   {L.dst_row, (size_t)G * dims.K * 4}}))
+        return MOEDISP_ERR_ALIASED;
+    return rc(moedisp::launch_combine_rmsnorm(expert_out, H, dims, L, expert_scales, residual, gamma,
+                                              eps, residual_out, y, status, stream));
+}
+
 }  // extern "C"

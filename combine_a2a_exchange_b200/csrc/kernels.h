@@ -92,4 +92,10 @@ cudaError_t launch_combine(const void* expert_out, int H, const moedisp_dims& di
                            const moedisp_layout& layout, const float* expert_scales, void* y,
                            int32_t* status, cudaStream_t stream);
 
+cudaError_t launch_combine_rmsnorm(const void* expert_out, int H, const moedisp_dims& dims,
+                                   const moedisp_layout& layout, const float* expert_scales,
+                                   const void* residual, const float* gamma, float eps,
+                                   void* residual_out, void* y, int32_t* status,
+                                   cudaStream_t stream);
+
 }  // namespace moedisp

@@ -250,6 +250,25 @@ int moedisp_moe_combine(const void *expert_out, int H, moedisp_dims dims,
                         const moedisp_layout *layout, const float *expert_scales, void *y,
                         int32_t *status, moedisp_stream_t stream);
 
+/* moe_combine_rmsnorm
+ *
+ * The combine fused with the residual add and RMSNorm that follow it (the FlashInfer
+ * MNNVL PR's "MoE finalize + residual + RMSNorm" tail, without its tensor-parallel
+ * all-reduce), one pass over HBM:
+ *   prenorm[g] = bf16_rn( acc + residual[g] )        acc as in moe_combine (fp32, k order),
+ *                                                    one fp32 add per element
+ *   y[g,h]     = bf16_rn( (prenorm[g,h] * rs) * gamma[h] ),
+ *                rs = 1/sqrt( sum_h prenorm[g,h]^2 / H + eps )   (fp32)
+ * residual: bf16 [G][H]; gamma: fp32 [H]; residual_out: bf16 [G][H] receiving prenorm, or
+ * NULL; y: bf16 [G][H]. Outputs must not overlap inputs. H % 8 == 0, H <= MOEDISP_MAX_H;
+ * all row pointers and gamma 16-byte aligned; eps >= 0. prenorm is bit-exact; y depends on
+ * the order of the sum of squares (a block reduction) within fp32 rounding. */
+int moedisp_moe_combine_rmsnorm(const void *expert_out, int H, moedisp_dims dims,
+                                const moedisp_layout *layout, const float *expert_scales,
+                                const void *residual, const float *gamma, float eps,
+                                void *residual_out, void *y, int32_t *status,
+                                moedisp_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

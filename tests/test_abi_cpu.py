@@ -33,7 +33,7 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for required in ("moedisp_a2a_exchange_plan", "moedisp_a2a_v", "moedisp_moe_dispatch_layout",
-                     "moedisp_moe_dispatch", "moedisp_moe_combine",
+                     "moedisp_moe_dispatch", "moedisp_moe_combine", "moedisp_moe_combine_rmsnorm",
                      "moedisp_layout_workspace_size", "moedisp_status_string"):
         assert required in names
 
@@ -157,6 +157,23 @@ def test_dispatch_and_combine_rejections(md):
     # no tokens: a valid no-op that launches nothing
     assert md.raw_call("moedisp_moe_combine", None, 128, md.Dims(4, 0, 2, 8), ctypes.byref(L),
                        None, None, st, None) == md.MOEDISP_OK
+    res, gm, ro = FAKE + (320 << 20), FAKE + (384 << 20), FAKE + (448 << 20)
+    rms = lambda eo, H, res, gm, eps, ro, y, st: md.raw_call(
+        "moedisp_moe_combine_rmsnorm", eo, H, d, ctypes.byref(L), x, res, gm, eps, ro, y, st, None)
+    assert rms(ex, 100, res, gm, 1e-6, ro, sc, st) == md.MOEDISP_ERR_MISALIGNED   # H % 8
+    assert rms(ex, 128, res, gm, -1.0, ro, sc, st) == md.MOEDISP_ERR_INVALID      # eps < 0
+    assert rms(ex, 128, res, gm, float("nan"), ro, sc, st) == md.MOEDISP_ERR_INVALID
+    assert rms(ex, 32768, res, gm, 1e-6, ro, sc, st) == md.MOEDISP_ERR_UNSUPPORTED
+    assert rms(ex, 128, None, gm, 1e-6, ro, sc, st) == md.MOEDISP_ERR_NULLPTR
+    assert rms(ex, 128, res, None, 1e-6, ro, sc, st) == md.MOEDISP_ERR_NULLPTR
+    assert rms(ex, 128, res, gm + 4, 1e-6, ro, sc, st) == md.MOEDISP_ERR_MISALIGNED
+    assert rms(ex, 128, res, gm, 1e-6, ro + 8, sc, st) == md.MOEDISP_ERR_MISALIGNED
+    assert rms(ex, 128, res, gm, 1e-6, res + 512, sc, st) == md.MOEDISP_ERR_ALIASED  # rout over residual
+    assert rms(ex, 128, res, gm, 1e-6, ro, ro + 1024, st) == md.MOEDISP_ERR_ALIASED  # y over rout
+    assert rms(ex, 128, res, gm, 1e-6, ro, gm, st) == md.MOEDISP_ERR_ALIASED         # y over gamma
+    assert rms(ex, 128, res, gm, 1e-6, ro, sc, None) == md.MOEDISP_ERR_NULLPTR
+    assert md.raw_call("moedisp_moe_combine_rmsnorm", None, 128, md.Dims(4, 0, 2, 8),
+                       ctypes.byref(L), None, None, None, 1e-6, None, None, st, None) == md.MOEDISP_OK
 
 
 def test_selftest_rejections(md):

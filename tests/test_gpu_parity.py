@@ -1,7 +1,8 @@
 """GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the same seeded
 inputs. Bit-exact for counts, offsets, indices, copied rows, quantised bytes and scales;
 combine bit-exact against the fixed-order fp32 oracle and within max-abs 1e-2 / rel 1e-2
-of the fp64 oracle."""
+of the fp64 oracle; the fused combine + residual + RMSNorm tail bit-exact in its residual
+output and within one bf16 ulp of the fp32 oracle (and the fp64 tolerance) in y."""
 import json
 import os
 
@@ -472,6 +473,116 @@ def test_combine_parity_full_size_sampled(md, name):
     check_combine(yt, sub_eo, sub_dr, w.weights[toks], w.K, max(rows.size, 1))
     if w.active is not None:
         assert (yt[w.active[toks] == 0] == 0).all()
+
+
+# ------------------------------------------- fused tail: combine + residual + RMSNorm
+
+RMS_EPS = 1e-6
+
+
+def run_combine_rmsnorm(md, L, eo_bits, w, residual, gamma, eps=RMS_EPS, want_rout=True):
+    y = torch.full((w.G, w.H), 7, dtype=torch.int16, device="cuda").view(torch.bfloat16)
+    rout = (torch.full((w.G, w.H), 9, dtype=torch.int16, device="cuda").view(torch.bfloat16)
+            if want_rout else None)
+    st = new_status()
+    md.moe_combine_rmsnorm(bf16_dev(eo_bits), w.H, L, dev(w.weights.reshape(-1)),
+                           bf16_dev(residual), dev(gamma), eps, y, st, residual_out=rout)
+    torch.cuda.synchronize()
+    return bits_host(y), (bits_host(rout) if want_rout else None), int(st.item())
+
+
+def check_combine_rmsnorm(y_bits, rout_bits, eo_bits, dst_row, weights, K, residual, gamma,
+                          rows_cap, eps=RMS_EPS):
+    """residual_out bit-exact against the fixed-order fp32 oracle; y within one bf16 ulp of
+    it (the sum of squares is a block reduction, its order differs) and within
+    max-abs 1e-2 / rel 1e-2 of the fp64 oracle."""
+    r32, y32, fl = oracle.moe_combine_rmsnorm(eo_bits, dst_row, weights, K, residual, gamma, eps,
+                                              rows_cap=rows_cap, exact="f32")
+    _, y64, _ = oracle.moe_combine_rmsnorm(eo_bits, dst_row, weights, K, residual, gamma, eps,
+                                           rows_cap=rows_cap, exact="f64")
+    if rout_bits is not None:
+        assert np.array_equal(rout_bits, r32), "residual_out not bit-exact"
+    same_sign = (y_bits >> 15) == (y32 >> 15)
+    ulps = np.abs(y_bits.astype(np.int64) - y32.astype(np.int64))
+    assert same_sign.all() and ulps.max(initial=0) <= 1, ulps.max(initial=0)
+    yf = wl.bf16_bits_to_f32(y_bits).astype(np.float64)
+    err = np.abs(yf - y64)
+    assert (err <= ATOL + RTOL * np.abs(y64)).all(), err.max()
+    return fl
+
+
+@pytest.mark.parametrize("name,over", COMBINE_CASES + [
+    ("tiny", dict(W=2, T=33, K=8, E=16, H=7168, active_p=0.5)),
+    ("tiny", dict(W=1, T=1, K=2, E=2, H=2048))])
+def test_combine_rmsnorm_parity_full(md, name, over):
+    w = wl.moe_workload(name, seed=43, **over)
+    L, _ = run_layout(md, w)
+    ref = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active)
+    eo = wl.expert_rows(L.rows_cap, w.H, seed=44)
+    residual, gamma = wl.rmsnorm_inputs(w.G, w.H, seed=45)
+    y, rout, st = run_combine_rmsnorm(md, L, eo, w, residual, gamma)
+    assert st == 0
+    check_combine_rmsnorm(y, rout, eo, ref["dst_row"], w.weights, w.K, residual, gamma, L.rows_cap)
+    y2, _, st2 = run_combine_rmsnorm(md, L, eo, w, residual, gamma, want_rout=False)
+    assert st2 == 0 and np.array_equal(y2, y), "y depends on whether residual_out is written"
+
+
+def test_combine_rmsnorm_inactive_tokens_normalise_the_residual(md):
+    """A token with no routed slot reduces to RMSNorm of its residual row."""
+    w = wl.moe_workload("tiny", seed=46, W=2, T=40, K=4, E=8, H=512)
+    w.active = np.zeros(w.G, np.uint8)
+    L, _ = run_layout(md, w)
+    eo = wl.expert_rows(max(L.rows_cap, 1), w.H, seed=47)
+    residual, gamma = wl.rmsnorm_inputs(w.G, w.H, seed=48)
+    y, rout, st = run_combine_rmsnorm(md, L, eo, w, residual, gamma)
+    assert st == 0 and np.array_equal(rout, residual)
+    r = torch.from_numpy(wl.bf16_bits_to_f32(residual).astype(np.float64))
+    ref = torch.nn.functional.rms_norm(r, (w.H,), torch.from_numpy(gamma.astype(np.float64)), RMS_EPS)
+    yf = wl.bf16_bits_to_f32(y).astype(np.float64)
+    assert (np.abs(yf - ref.numpy()) <= ATOL + RTOL * np.abs(ref.numpy())).all()
+
+
+def test_combine_rmsnorm_capacity_guard(md):
+    w = wl.moe_workload("tiny", seed=49, W=2, T=64, K=4, E=8, H=256)
+    ref = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active)
+    cap = ref["R"] // 2
+    L, _ = run_layout(md, w, rows_cap=cap)
+    eo = wl.expert_rows(cap, w.H, seed=50)
+    residual, gamma = wl.rmsnorm_inputs(w.G, w.H, seed=51)
+    y, rout, st = run_combine_rmsnorm(md, L, eo, w, residual, gamma)
+    assert st & md.STATUS_CAPACITY
+    capped = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active, rows_cap=cap)
+    fl = check_combine_rmsnorm(y, rout, eo, capped["dst_row"], w.weights, w.K, residual, gamma, cap)
+    assert fl & oracle.ORC_CAPACITY
+
+
+@pytest.mark.parametrize("name", ["cfg2", "cfg3"])
+def test_combine_rmsnorm_full_size_sampled(md, name):
+    w = wl.moe_workload(name, seed=0)
+    L, _ = run_layout(md, w)
+    ref = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active)
+    gen = torch.Generator(device="cuda").manual_seed(6)
+    eo = torch.randn((L.rows_cap, w.H), generator=gen, device="cuda").to(torch.bfloat16)
+    res = torch.randn((w.G, w.H), generator=gen, device="cuda").to(torch.bfloat16)
+    gamma = 0.5 + torch.rand((w.H,), generator=gen, device="cuda")
+    y = torch.empty((w.G, w.H), dtype=torch.bfloat16, device="cuda")
+    rout = torch.empty((w.G, w.H), dtype=torch.bfloat16, device="cuda")
+    st = new_status()
+    md.moe_combine_rmsnorm(eo, w.H, L, dev(w.weights.reshape(-1)), res, gamma, RMS_EPS, y, st,
+                           residual_out=rout)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    rng = np.random.default_rng(4)
+    toks = rng.choice(w.G, size=128, replace=False)
+    sel = ref["dst_row"].reshape(w.G, w.K)[toks]
+    rows = np.unique(sel[sel >= 0])
+    remap = np.full(L.rows_cap, -1, np.int64)
+    remap[rows] = np.arange(rows.size)
+    sub_dr = np.where(sel >= 0, remap[np.maximum(sel, 0)], -1).astype(np.int32)
+    sub_eo = bits_host(eo[torch.from_numpy(rows).cuda()]) if rows.size else np.zeros((1, w.H), np.uint16)
+    tk = torch.from_numpy(toks).cuda()
+    check_combine_rmsnorm(bits_host(y[tk]), bits_host(rout[tk]), sub_eo, sub_dr, w.weights[toks],
+                          w.K, bits_host(res[tk]), gamma.cpu().numpy(), max(rows.size, 1))
 
 
 # --------------------------------------------------------------- end to end

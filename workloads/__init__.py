@@ -192,6 +192,15 @@ def expert_rows(R: int, H: int, seed: int = 1) -> np.ndarray:
     return f32_to_bf16_bits(rng.standard_normal((R, H), dtype=np.float32))
 
 
+def rmsnorm_inputs(G: int, H: int, seed: int = 7):
+    """Inputs of the fused combine + residual + RMSNorm tail: the residual stream as bf16
+    bits [G, H], N(0,1), and the RMSNorm weight gamma, fp32 [H], uniform in [0.5, 1.5)."""
+    rng = _rng(seed)
+    residual = f32_to_bf16_bits(rng.standard_normal((G, H), dtype=np.float32))
+    gamma = (0.5 + rng.random(H, dtype=np.float32)).astype(np.float32)
+    return residual, gamma
+
+
 # --------------------------------------------------------------------------------------
 # raw uneven all-to-all-v
 
