@@ -61,11 +61,13 @@ def lib() -> ctypes.CDLL:
         L.orc_e4m3_to_f32.restype = ctypes.c_float
         L.orc_a2a_exchange_plan.argtypes = [i32, P, P, P, P]
         L.orc_a2a_v.argtypes = [i32, P, i64, P, i64, i64, P, P, P]
-        L.orc_moe_dispatch_layout.argtypes = [i32, i32, i32, i32, P, P, i64, P, P, P, P, P, P, P]
+        L.orc_moe_dispatch_layout.argtypes = [i32, i32, i32, i32, P, P, i32, i64, P, P, P, P, P, P, P]
         L.orc_moe_recv_counts.argtypes = [i32, i32, P, i32, P, P]
-        L.orc_moe_dispatch.argtypes = [i32, i32, i32, P, P, i64, i32, P, P]
+        L.orc_moe_dispatch.argtypes = [i32, i32, i32, P, P, i64, i32, P, P, P, i32, P]
         L.orc_quant_row.argtypes = [i32, P, i32, P]
         L.orc_quant_row.restype = ctypes.c_float
+        L.orc_quant_row_f32.argtypes = [i32, P, i32, P]
+        L.orc_quant_row_f32.restype = ctypes.c_float
         L.orc_moe_combine_f64.argtypes = [i32, i32, i32, P, i64, P, P, P]
         L.orc_moe_combine_f32.argtypes = [i32, i32, i32, P, i64, P, P, P]
         L.orc_moe_combine_rmsnorm_f64.argtypes = [i32, i32, i32, P, i64, P, P, P, P, ctypes.c_float, P, P]
@@ -136,10 +138,14 @@ def a2a_v(inp: np.ndarray, out: np.ndarray, src_offsets, out_splits, dst_offsets
 
 def moe_dispatch_layout(W: int, T: int, K: int, E: int, expert_ids, active=None,
                         rows_cap: int | None = None) -> dict:
+    """active: None, a per-token mask [G], or a per-slot mask [G, K] (told apart by size;
+    with K = 1 the two readings coincide)."""
     ids = _c(expert_ids, np.int32).reshape(-1)
     G = W * T
     assert ids.size == G * K
     act = None if active is None else _c(active, np.uint8).reshape(-1)
+    active_dims = 1 if act is None or act.size == G else 2
+    assert act is None or act.size == (G if active_dims == 1 else G * K)
     if rows_cap is None:
         rows_cap = G * K
     out = dict(
@@ -151,7 +157,7 @@ def moe_dispatch_layout(W: int, T: int, K: int, E: int, expert_ids, active=None,
         rank_base=np.zeros(W + 1, np.int64),
         send_splits=np.zeros((W, W), np.int64),
     )
-    fl = lib().orc_moe_dispatch_layout(W, T, K, E, _p(ids), _p(act), rows_cap,
+    fl = lib().orc_moe_dispatch_layout(W, T, K, E, _p(ids), _p(act), active_dims, rows_cap,
                                        _p(out["cnt"]), _p(out["occ"]), _p(out["dst_row"]),
                                        _p(out["assist_info"]), _p(out["expert_base"]),
                                        _p(out["rank_base"]), _p(out["send_splits"]))
@@ -179,18 +185,31 @@ def quant_row(x_bits_row, quant_mode: int):
     return q, float(np.float32(s))
 
 
+def quant_row_f32(x_row, quant_mode: int):
+    x = _c(x_row, np.float32)
+    q = np.zeros(x.size, np.uint8)
+    s = lib().orc_quant_row_f32(x.size, _p(x), quant_mode, _p(q))
+    return q, float(np.float32(s))
+
+
 def moe_dispatch(x_bits, dst_row, K: int, rows_cap: int, quant_mode: int = 0,
-                 expand_x=None, dynamic_scales=None):
+                 expand_x=None, dynamic_scales=None, smooth=None, expert_ids=None):
+    """smooth: per-expert smoothing factors [E, H] fp32 (quantising modes), with the
+    routing's expert_ids [G, K]."""
     x = _c(x_bits, np.uint16)
     G, H = x.shape
     dr = _c(dst_row, np.int32).reshape(-1)
+    sm = None if smooth is None else _c(smooth, np.float32)
+    ids = None if expert_ids is None else _c(expert_ids, np.int32).reshape(-1)
+    E = 0 if sm is None else sm.shape[0]
+    assert sm is None or (sm.shape == (E, H) and ids is not None and ids.size == G * K)
     if expand_x is None:
         expand_x = (np.zeros((rows_cap, H), np.uint16) if quant_mode == 0
                     else np.zeros((rows_cap, H), np.uint8))
     if dynamic_scales is None and quant_mode != 0:
         dynamic_scales = np.zeros(rows_cap, np.float32)
     fl = lib().orc_moe_dispatch(G, K, H, _p(x), _p(dr), rows_cap, quant_mode,
-                                _p(expand_x), _p(dynamic_scales))
+                                _p(expand_x), _p(dynamic_scales), _p(sm), E, _p(ids))
     return expand_x, dynamic_scales, fl
 
 

@@ -156,14 +156,16 @@ int orc_a2a_v(int W, const uint8_t *in, int64_t in_rank_stride_rows, uint8_t *ou
  *  3. the index push: slot s of rank r with expert e goes to row
  *        dst_offsets[r][e] + occ[s] of rank owner(e) = e / ne  ([P1]
  *        _allToAllV_2d_index_push_kernel), i.e. global row rank_base[d] + that.
- * Inactive tokens ([P4] xActiveMask, read as: any 1-D mask) and expert ids outside
- * [0, E) contribute no slot; both get occ = dst_row = -1. */
+ * Inactive slots ([P4] xActiveMask: a 1-D mask [G] of tokens, read as any pattern, or a
+ * 2-D mask [G][K] of slots, where a token whose K flags are all false sends nothing) and
+ * expert ids outside [0, E) contribute no slot; both get occ = dst_row = -1. */
 int orc_moe_dispatch_layout(int W, int T, int K, int E, const int32_t *expert_ids,
-                            const uint8_t *active, int64_t rows_cap, int32_t *cnt,
+                            const uint8_t *active, int active_dims, int64_t rows_cap, int32_t *cnt,
                             int32_t *occ, int32_t *dst_row, int32_t *assist_info,
                             int64_t *expert_base, int64_t *rank_base, int64_t *send_splits)
 {
     if (W <= 0 || T < 0 || K <= 0 || E <= 0 || E % W != 0) return ORC_BAD_ARG;
+    if (active && active_dims != 1 && active_dims != 2) return ORC_BAD_ARG;
     int flags = 0;
     int ne = E / W;
     int64_t G = (int64_t)W * T;
@@ -178,9 +180,9 @@ int orc_moe_dispatch_layout(int W, int T, int K, int E, const int32_t *expert_id
         memset(running, 0, sizeof(int64_t) * E);
         for (int t = 0; t < T; t++) {
             int64_t g = (int64_t)r * T + t;
-            int act = active ? (active[g] != 0) : 1;
             for (int k = 0; k < K; k++) {
                 int64_t s = g * K + k;
+                int act = !active ? 1 : active_dims == 1 ? (active[g] != 0) : (active[s] != 0);
                 int32_t e = expert_ids[s];
                 if (act && (e < 0 || e >= E)) flags |= ORC_BAD_EXPERT;
                 if (!act || e < 0 || e >= E) { occ[s] = -1; continue; }
@@ -276,18 +278,18 @@ int orc_moe_recv_counts(int W, int E, const int32_t *cnt, int expert_token_nums_
  * (QMAX = 127 for int8, 448 for e4m3), q = round(x / scale) with one IEEE fp32 divide;
  * int8 rounds half to even and clamps to [-127, 127]; e4m3 rounds to nearest even and
  * saturates. An all-zero row has scale 0 and q = 0. */
-float orc_quant_row(int H, const uint16_t *x, int quant_mode, uint8_t *q)
+float orc_quant_row_f32(int H, const float *x, int quant_mode, uint8_t *q)
 {
     float amax = 0.0f;
     for (int h = 0; h < H; h++) {
-        float a = fabsf(orc_bf16_to_f32(x[h]));
+        float a = fabsf(x[h]);
         if (a > amax) amax = a;
     }
     float qmax = quant_mode == 2 ? 127.0f : 448.0f;
     float scale = amax / qmax;
     for (int h = 0; h < H; h++) {
         if (amax == 0.0f) { q[h] = 0; continue; }
-        float v = orc_bf16_to_f32(x[h]) / scale;
+        float v = x[h] / scale;
         if (quant_mode == 2) {
             float r = rintf(v);
             if (r > 127.0f) r = 127.0f;
@@ -300,16 +302,30 @@ float orc_quant_row(int H, const uint16_t *x, int quant_mode, uint8_t *q)
     return scale;
 }
 
+float orc_quant_row(int H, const uint16_t *x, int quant_mode, uint8_t *q)
+{
+    float *v = (float *)malloc(sizeof(float) * (size_t)(H > 0 ? H : 1));
+    for (int h = 0; h < H; h++) v[h] = orc_bf16_to_f32(x[h]);
+    float scale = orc_quant_row_f32(H, v, quant_mode, q);
+    free(v);
+    return scale;
+}
+
 /* [P1] index push / [P4] expandXOut: every active slot s writes its token's row
  * (quantised or not) to row dst_row[s]. Rows at or beyond rows_cap are skipped and
- * flagged. */
+ * flagged. With smooth ([P4] scalesOptional, [E][H]; quantising modes only) the row sent
+ * to expert e = expert_ids[s] is first multiplied element-wise by smooth[e] (one fp32
+ * product per element) and quantised on its own, so each copy has its own scale. */
 int orc_moe_dispatch(int G, int K, int H, const uint16_t *x, const int32_t *dst_row,
-                     int64_t rows_cap, int quant_mode, void *expand_x, float *dynamic_scales)
+                     int64_t rows_cap, int quant_mode, void *expand_x, float *dynamic_scales,
+                     const float *smooth, int E, const int32_t *expert_ids)
 {
     if (quant_mode != 0 && quant_mode != 2 && quant_mode != 3) return ORC_BAD_ARG;
+    if (smooth && (quant_mode == 0 || !expert_ids || E <= 0)) return ORC_BAD_ARG;
     int flags = 0;
     size_t out_row = quant_mode == 0 ? (size_t)H * 2 : (size_t)H;
     uint8_t *q = (uint8_t *)malloc((size_t)H > 0 ? (size_t)H : 1);
+    float *xs = (float *)malloc(sizeof(float) * (size_t)(H > 0 ? H : 1));
     for (int64_t g = 0; g < G; g++) {
         const uint16_t *xr = x + g * (int64_t)H;
         float scale = 0.0f;
@@ -321,6 +337,13 @@ int orc_moe_dispatch(int G, int K, int H, const uint16_t *x, const int32_t *dst_
             uint8_t *dst = (uint8_t *)expand_x + (size_t)row * out_row;
             if (quant_mode == 0) {
                 memcpy(dst, xr, out_row);
+            } else if (smooth) {
+                int32_t e = expert_ids[g * K + k];
+                if (e < 0 || e >= E) { flags |= ORC_BAD_EXPERT; continue; }
+                for (int h = 0; h < H; h++)
+                    xs[h] = orc_bf16_to_f32(xr[h]) * smooth[(int64_t)e * H + h];
+                dynamic_scales[row] = orc_quant_row_f32(H, xs, quant_mode, q);
+                memcpy(dst, q, out_row);
             } else {
                 if (!have_q) { scale = orc_quant_row(H, xr, quant_mode, q); have_q = 1; }
                 memcpy(dst, q, out_row);
@@ -329,6 +352,7 @@ int orc_moe_dispatch(int G, int K, int H, const uint16_t *x, const int32_t *dst_
         }
     }
     free(q);
+    free(xs);
     return flags;
 }
 

@@ -45,10 +45,11 @@ int orc_a2a_v(int W, const uint8_t *in, int64_t in_rank_stride_rows, uint8_t *ou
               int64_t out_cap_rows, int64_t row_bytes, const int64_t *src_offsets,
               const int64_t *out_splits, const int64_t *dst_offsets);
 
-/* O3: dispatch layout. active may be NULL (all active). Inactive slots get occ = -1,
- * dst_row = -1. assist_info entries beyond R are left untouched. */
+/* O3: dispatch layout. active may be NULL (all active); active_dims 1: active[G] per
+ * token, 2: active[G][K] per slot. Inactive slots get occ = -1, dst_row = -1. assist_info
+ * entries beyond R are left untouched. */
 int orc_moe_dispatch_layout(int W, int T, int K, int E, const int32_t *expert_ids,
-                            const uint8_t *active, int64_t rows_cap, int32_t *cnt,
+                            const uint8_t *active, int active_dims, int64_t rows_cap, int32_t *cnt,
                             int32_t *occ, int32_t *dst_row, int32_t *assist_info,
                             int64_t *expert_base, int64_t *rank_base, int64_t *send_splits);
 
@@ -60,12 +61,15 @@ int orc_moe_recv_counts(int W, int E, const int32_t *cnt, int expert_token_nums_
                         int64_t *expert_token_nums, int32_t *ep_recv_counts);
 
 /* O4: dispatch copy with optional per-token dynamic quantisation (0 none, 2 int8,
- * 3 fp8-e4m3). dynamic_scales may be NULL for mode 0. */
+ * 3 fp8-e4m3). dynamic_scales may be NULL for mode 0. smooth ([E][H] fp32, quantising
+ * modes only; needs expert_ids [G][K]) or NULL: per-expert smoothing before quantisation. */
 int orc_moe_dispatch(int G, int K, int H, const uint16_t *x, const int32_t *dst_row,
-                     int64_t rows_cap, int quant_mode, void *expand_x, float *dynamic_scales);
+                     int64_t rows_cap, int quant_mode, void *expand_x, float *dynamic_scales,
+                     const float *smooth, int E, const int32_t *expert_ids);
 
 /* Per-token quantisation of one row (exposed for pins). Returns the scale. */
 float orc_quant_row(int H, const uint16_t *x, int quant_mode, uint8_t *q);
+float orc_quant_row_f32(int H, const float *x, int quant_mode, uint8_t *q);
 
 /* O5a: combine in double precision; y64[G][H]. */
 int orc_moe_combine_f64(int G, int K, int H, const uint16_t *expert_out, int64_t rows_cap,

@@ -175,9 +175,11 @@ def brute_layout(W, T, K, E, ids, active):
             for r in range(W):
                 for t in range(T):
                     g = r * T + t
-                    if active is not None and not active[g]:
-                        continue
                     for k in range(K):
+                        if active is not None:
+                            flag = active[g][k] if isinstance(active[g], (list, tuple)) else active[g]
+                            if not flag:
+                                continue
                         if ids[g][k] == e:
                             rows.append(g * K + k)
     dst_row = [-1] * (W * T * K)
@@ -198,8 +200,12 @@ def _check_layout(W, T, K, E, ids, active, lay):
     G = W * T
     ne = E // W
     ids2 = np.asarray(ids).reshape(G, K)
-    act = np.ones(G, bool) if active is None else np.asarray(active).astype(bool)
-    slot_active = np.repeat(act, K) & (ids2.reshape(-1) >= 0) & (ids2.reshape(-1) < E)
+    if active is None:
+        act = np.ones(G * K, bool)
+    else:
+        a = np.asarray(active).astype(bool)
+        act = np.repeat(a.reshape(-1), K) if a.ndim == 1 else a.reshape(-1)
+    slot_active = act & (ids2.reshape(-1) >= 0) & (ids2.reshape(-1) < E)
     R = int(slot_active.sum())
     assert lay["R"] == R
     # closed form: dst_row = position in a stable sort of the active slots by expert id
@@ -252,7 +258,39 @@ def test_layout_brute_force_tiny(seed):
     _check_layout(W, T, K, E, ids, active, lay)
 
 
+@pytest.mark.parametrize("seed", range(6))
+def test_layout_slot_mask_brute_force_tiny(seed):
+    """[P4] 2-D xActiveMask (Bs, K): each slot's own flag decides; nested-loop brute force."""
+    rng = np.random.default_rng(200 + seed)
+    W = int(rng.integers(1, 5))
+    ne = int(rng.integers(1, 4))
+    E = W * ne
+    T = int(rng.integers(1, 7))
+    K = int(rng.integers(2, 5))
+    ids = rng.integers(0, E, size=(W * T, K)).astype(np.int32)
+    active = (rng.random((W * T, K)) < 0.6).astype(np.uint8)
+    active[0] = 0                                                  # a token that sends nothing
+    lay = oracle.moe_dispatch_layout(W, T, K, E, ids, active)
+    assert lay["flags"] == 0
+    rows, dst_row = brute_layout(W, T, K, E, ids.tolist(), active.tolist())
+    assert lay["dst_row"].tolist() == dst_row
+    assert lay["assist_info"][:len(rows)].tolist() == rows
+    assert (lay["dst_row"][:K] == -1).all() and (lay["occ"][:K] == -1).all()
+    _check_layout(W, T, K, E, ids, active, lay)
+
+
+def test_layout_slot_mask_repeating_token_mask_equals_token_mask():
+    w = wl.moe_workload("tiny", seed=21, W=3, T=40, E=12, K=3, active_p=0.6)
+    one = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active)
+    two = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids,
+                                     np.repeat(w.active[:, None], w.K, axis=1))
+    for k in ("cnt", "occ", "dst_row", "expert_base", "rank_base", "send_splits"):
+        assert np.array_equal(one[k], two[k]), k
+    assert np.array_equal(one["assist_info"][:one["R"]], two["assist_info"][:two["R"]])
+
+
 @pytest.mark.parametrize("name,over", [("tiny", {}), ("tiny", dict(W=3, T=37, E=12, K=3)),
+                                       ("tiny", dict(W=4, T=50, E=16, K=4, slot_active_p=0.5)),
                                        ("cfg4", dict(T=64)), ("cfg3", dict(T=128, H=256))])
 def test_layout_closed_form_on_workloads(name, over):
     w = wl.moe_workload(name, seed=3, **over)
@@ -399,6 +437,54 @@ def test_dispatch_copy_and_scale_placement():
             else:
                 q, s = oracle.quant_row(w.x_bits[g], mode)
                 assert (ex[row] == q).all() and sc[row] == s
+
+
+@pytest.mark.parametrize("mode", [2, 3])
+def test_smoothing_brute_force(mode):
+    """[P4] scalesOptional: the copy for expert e is x * smooth[e] (fp32 products, here
+    numpy's) quantised on its own -- brute force through the independent quantiser."""
+    w = wl.moe_workload("tiny", seed=31, W=2, T=6, E=4, K=3, H=48, outlier_frac=0.1,
+                        zero_rows=0.1)
+    sm = wl.smooth_scales(w.E, w.H, seed=32)
+    lay = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active)
+    ex, sc, fl = oracle.moe_dispatch(w.x_bits, lay["dst_row"], w.K, lay["rows_cap"], mode,
+                                     smooth=sm, expert_ids=w.expert_ids)
+    assert fl == 0
+    for row in range(lay["R"]):
+        s_ = lay["assist_info"][row]
+        g, e = s_ // w.K, w.expert_ids.reshape(-1)[s_]
+        xs = wl.bf16_bits_to_f32(w.x_bits[g]).astype(np.float32) * sm[e]
+        qb, sb = _quant_brute(xs, mode)
+        assert sc[row] == np.float32(sb)
+        assert ex[row].tolist() == qb
+
+
+@pytest.mark.parametrize("mode", [2, 3])
+def test_smoothing_special_cases(mode):
+    """All-ones smoothing is no smoothing; a power-of-two factor c per expert leaves the
+    codes unchanged and multiplies the scale by c exactly."""
+    w = wl.moe_workload("tiny", seed=33, W=2, T=10, E=4, K=2, H=64, outlier_frac=0.1)
+    lay = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active)
+    plain, psc, _ = oracle.moe_dispatch(w.x_bits, lay["dst_row"], w.K, lay["rows_cap"], mode)
+    ones, osc, _ = oracle.moe_dispatch(w.x_bits, lay["dst_row"], w.K, lay["rows_cap"], mode,
+                                       smooth=np.ones((w.E, w.H), np.float32),
+                                       expert_ids=w.expert_ids)
+    assert np.array_equal(plain, ones) and np.array_equal(psc, osc)
+    c = np.array([0.25, 2.0, 8.0, 0.5], np.float32)
+    pw, pwsc, _ = oracle.moe_dispatch(w.x_bits, lay["dst_row"], w.K, lay["rows_cap"], mode,
+                                      smooth=np.repeat(c[:, None], w.H, axis=1),
+                                      expert_ids=w.expert_ids)
+    assert np.array_equal(pw, plain)
+    e_of_row = w.expert_ids.reshape(-1)[lay["assist_info"][:lay["R"]]]
+    assert np.array_equal(pwsc[:lay["R"]], psc[:lay["R"]] * c[e_of_row])
+
+
+def test_smoothing_needs_a_quantising_mode():
+    w = wl.moe_workload("tiny", seed=34)
+    lay = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active)
+    _, _, fl = oracle.moe_dispatch(w.x_bits, lay["dst_row"], w.K, lay["rows_cap"], 0,
+                                   smooth=np.ones((w.E, w.H), np.float32), expert_ids=w.expert_ids)
+    assert fl & oracle.ORC_BAD_ARG
 
 
 # --------------------------------------------------------------- O5 pins

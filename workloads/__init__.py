@@ -66,7 +66,7 @@ class MoEWorkload:
     x_bits: np.ndarray              # uint16 [G, H]  (bf16 bits)
     expert_ids: np.ndarray          # int32  [G, K]
     weights: np.ndarray             # fp32   [G, K]  gate weights (expert scales)
-    active: Optional[np.ndarray]    # uint8  [G] or None (all tokens active)
+    active: Optional[np.ndarray]    # uint8  [G] (tokens) or [G, K] (slots); None = all active
     recipe: dict = field(default_factory=dict)
 
     @property
@@ -80,7 +80,14 @@ class MoEWorkload:
     def n_active_slots(self) -> int:
         if self.active is None:
             return self.G * self.K
-        return int(self.active.astype(np.int64).sum()) * self.K
+        n = int(self.active.astype(np.int64).sum())
+        return n * self.K if self.active.ndim == 1 else n
+
+    def token_active(self) -> np.ndarray:
+        """uint8 [G]: tokens with at least one active slot."""
+        if self.active is None:
+            return np.ones(self.G, np.uint8)
+        return (self.active if self.active.ndim == 1 else self.active.max(axis=1, initial=0)).astype(np.uint8)
 
     def rows_cap(self) -> int:
         """Receive capacity for all ranks together: every (token, k) slot may land."""
@@ -136,8 +143,10 @@ def moe_workload(name: str = "cfg2", seed: int = 0, **over) -> MoEWorkload:
     ``name`` picks a configuration from ``MOE_CONFIGS``; keyword overrides change any
     of its fields (used for small parity cases that span several tiles with a ragged
     tail). Extra override keys: ``routing`` ("uniform" | "zipf" | "dup" — "dup" draws
-    experts with replacement, so a token can pick one expert twice), ``active_p``,
-    ``outlier_frac``, ``outlier_scale``, ``zero_rows`` (fraction of all-zero rows).
+    experts with replacement, so a token can pick one expert twice), ``active_p``
+    (per-token Bernoulli mask [G]), ``slot_active_p`` (per-slot Bernoulli mask [G, K], plus
+    5% of tokens with no active slot), ``outlier_frac``, ``outlier_scale``, ``zero_rows``
+    (fraction of all-zero rows).
     """
     cfg = dict(MOE_CONFIGS[name])
     cfg.update(over)
@@ -178,6 +187,12 @@ def moe_workload(name: str = "cfg2", seed: int = 0, **over) -> MoEWorkload:
     ap = cfg.get("active_p")
     if ap is not None:
         active = (rng.random(G) < float(ap)).astype(np.uint8)
+    sp = cfg.get("slot_active_p")
+    if sp is not None:
+        # per-slot mask [G, K]; a seeded 5% of tokens get all K flags false
+        active = (rng.random((G, K)) < float(sp)).astype(np.uint8)
+        if G > 0:
+            active[rng.choice(G, size=max(1, G // 20), replace=False)] = 0
 
     return MoEWorkload(name=name, W=W, T=T, H=H, E=E, K=K,
                        quant_mode=int(cfg["quant_mode"]), x_bits=x_bits,
@@ -190,6 +205,13 @@ def expert_rows(R: int, H: int, seed: int = 1) -> np.ndarray:
     """Synthetic expert outputs for combine: bf16 bits [R, H], N(0,1)."""
     rng = _rng(seed)
     return f32_to_bf16_bits(rng.standard_normal((R, H), dtype=np.float32))
+
+
+def smooth_scales(E: int, H: int, seed: int = 9) -> np.ndarray:
+    """Per-expert smoothing factors for quantisation, fp32 [E, H], log-uniform in
+    [1/4, 4)."""
+    rng = _rng(seed)
+    return np.exp2(rng.uniform(-2.0, 2.0, size=(E, H))).astype(np.float32)
 
 
 def rmsnorm_inputs(G: int, H: int, seed: int = 7):
