@@ -149,6 +149,9 @@ def algorithmic_bytes(op, w=None, R=None, a2a=None):
         return R * H * 2 + G * H * 2 + G * K * 8
     if op == "layout":
         return G * K * 4 + (0 if w.active is None else G) + 2 * G * K * 4 + R * 4
+    if op == "dispatch_smooth":
+        # the dispatch's bytes + the smoothing table (read once at least) + the expert ids
+        return algorithmic_bytes("dispatch", w, R) + w.E * H * 4 + G * K * 4
     if op == "combine_rmsnorm":
         # expert rows + residual read, residual_out + y written, gamma, routing
         return R * H * 2 + 3 * G * H * 2 + H * 4 + G * K * 8
@@ -491,6 +494,33 @@ def op_sweep(md, torch, device, hbm, reps=10):
                     "bytes": b, "GB/s": round(b / ms / 1e6, 1),
                     "frac": round(b / ms / 1e6 / hbm, 4)})
         del st, res, rout
+        torch.cuda.empty_cache()
+    # dispatch with per-expert smoothing before the dynamic quantisation
+    for name in ("cfg3", "cfg4"):
+        w = wl.moe_workload(name, seed=0)
+        st = MoEStep(md, torch, w, device)
+        st.run()
+        sm = torch.from_numpy(wl.smooth_scales(w.E, w.H, seed=1)).to(device)
+        Ev = torch.cuda.Event
+        pairs = []
+        for r in range(reps + 3):
+            flush.zero_()
+            e0, e1 = Ev(enable_timing=True), Ev(enable_timing=True)
+            e0.record()
+            md.moe_dispatch(st.x, w.H, st.L, w.quant_mode, st.ex, st.scales, st.status,
+                            smooth_scales=sm, expert_ids=st.ids)
+            e1.record()
+            if r >= 3:
+                pairs.append((e0, e1))
+        torch.cuda.synchronize()
+        assert int(st.status.item()) == 0, md.status_string(int(st.status.item()))
+        ms = statistics.mean(a.elapsed_time(b) for a, b in pairs)
+        R = int(st.L.expert_base[-1].item())
+        b = algorithmic_bytes("dispatch_smooth", w, R)
+        out.append({"workload": name, "op": "dispatch_smooth", "us": round(ms * 1e3, 2),
+                    "bytes": b, "GB/s": round(b / ms / 1e6, 1),
+                    "frac": round(b / ms / 1e6 / hbm, 4)})
+        del st, sm
         torch.cuda.empty_cache()
     # raw all-to-all-v, W = 64
     a = wl.a2a_workload(seed=0)

@@ -72,11 +72,11 @@ _plan = _sig("moedisp_a2a_exchange_plan", [_P, _I, _P, _P, _P, _P, _P])
 _a2a_v = _sig("moedisp_a2a_v", [_P, _I64, _P, _I64, _I64, _I, _P, _P, _P, _P, _P])
 _ws_size = _sig("moedisp_layout_workspace_size", [Dims, ctypes.POINTER(ctypes.c_size_t)])
 _layout = _sig("moedisp_moe_dispatch_layout",
-               [_P, _P, Dims, ctypes.POINTER(Layout), _P, ctypes.c_size_t, _P, _P])
+               [_P, _P, _I, Dims, ctypes.POINTER(Layout), _P, ctypes.c_size_t, _P, _P])
 _layout_noalloc = _sig("moedisp_moe_dispatch_layout_noalloc",
-                       [_P, _P, Dims, ctypes.POINTER(Layout), _P, _P])
+                       [_P, _P, _I, Dims, ctypes.POINTER(Layout), _P, _P])
 _dispatch = _sig("moedisp_moe_dispatch",
-                 [_P, _I, Dims, ctypes.POINTER(Layout), _I, _P, _P, _P, _I, _P, _P, _P])
+                 [_P, _I, Dims, ctypes.POINTER(Layout), _I, _P, _P, _P, _P, _P, _I, _P, _P, _P])
 _combine = _sig("moedisp_moe_combine", [_P, _I, Dims, ctypes.POINTER(Layout), _P, _P, _P, _P])
 _combine_rms = _sig("moedisp_moe_combine_rmsnorm",
                     [_P, _I, Dims, ctypes.POINTER(Layout), _P, _P, _P, ctypes.c_float, _P, _P, _P, _P])
@@ -196,31 +196,52 @@ class LayoutBuffers:
                       int(self.rows_cap))
 
 
+def _mask_dims(active_mask, dims: Dims, given) -> int:
+    """1 for a per-token mask [G], 2 for a per-slot mask [G, K]: from the tensor's shape
+    unless given (raw pointers need it given)."""
+    if given is not None:
+        return int(given)
+    if active_mask is None:
+        return 0
+    if isinstance(active_mask, int):
+        raise ValueError("active_mask_dims is required with a raw active_mask pointer")
+    if active_mask.dim() == 2:
+        return 2
+    return 2 if (dims.K > 1 and active_mask.numel() == dims.W * dims.T * dims.K) else 1
+
+
 def moe_dispatch_layout(expert_ids, active_mask, layout: LayoutBuffers, status, stream=None,
-                        raise_on_error=True, workspace=None, workspace_bytes=None) -> int:
+                        raise_on_error=True, workspace=None, workspace_bytes=None,
+                        active_mask_dims=None) -> int:
+    """active_mask: None, uint8 [G] (per token) or [G, K] (per slot)."""
     ws = layout.workspace if workspace is None else workspace
     nbytes = (ws.numel() * ws.element_size()) if workspace_bytes is None else workspace_bytes
     L = layout.struct()
-    rc = _layout(_ptr(expert_ids), _ptr(active_mask), layout.dims, ctypes.byref(L), _ptr(ws),
-                 int(nbytes), _ptr(status), _stream(stream))
+    rc = _layout(_ptr(expert_ids), _ptr(active_mask),
+                 _mask_dims(active_mask, layout.dims, active_mask_dims), layout.dims,
+                 ctypes.byref(L), _ptr(ws), int(nbytes), _ptr(status), _stream(stream))
     return _check(rc, "moe_dispatch_layout", raise_on_error)
 
 
 def moe_dispatch_layout_noalloc(expert_ids, active_mask, layout: LayoutBuffers, status,
-                                stream=None, raise_on_error=True) -> int:
+                                stream=None, raise_on_error=True, active_mask_dims=None) -> int:
     """moe_dispatch_layout without a workspace argument: the scratch lives in the
     library's own device memory (see include/moedisp.h). Allocates nothing."""
     L = layout.struct()
-    rc = _layout_noalloc(_ptr(expert_ids), _ptr(active_mask), layout.dims, ctypes.byref(L),
-                         _ptr(status), _stream(stream))
+    rc = _layout_noalloc(_ptr(expert_ids), _ptr(active_mask),
+                         _mask_dims(active_mask, layout.dims, active_mask_dims), layout.dims,
+                         ctypes.byref(L), _ptr(status), _stream(stream))
     return _check(rc, "moe_dispatch_layout_noalloc", raise_on_error)
 
 
 def moe_dispatch(x, H, layout: LayoutBuffers, quant_mode, expand_x, dynamic_scales, status,
                  expert_token_nums=None, expert_token_nums_type=1, ep_recv_counts=None,
-                 stream=None, raise_on_error=True) -> int:
+                 stream=None, raise_on_error=True, smooth_scales=None, expert_ids=None) -> int:
+    """smooth_scales: fp32 [E, H] per-expert smoothing before quantisation (quantising
+    modes), with the routing's expert_ids [G, K]."""
     L = layout.struct()
-    rc = _dispatch(_ptr(x), int(H), layout.dims, ctypes.byref(L), int(quant_mode), _ptr(expand_x),
+    rc = _dispatch(_ptr(x), int(H), layout.dims, ctypes.byref(L), int(quant_mode),
+                   _ptr(smooth_scales), _ptr(expert_ids), _ptr(expand_x),
                    _ptr(dynamic_scales), _ptr(expert_token_nums), int(expert_token_nums_type),
                    _ptr(ep_recv_counts), _ptr(status), _stream(stream))
     return _check(rc, "moe_dispatch", raise_on_error)

@@ -89,7 +89,7 @@ const char* moedisp_status_string(int code) {
     return "unknown code";
 }
 
-int moedisp_version(void) { return 1; }
+int moedisp_version(void) { return 2; }
 
 int moedisp_selftest_bounded_wait(uint32_t limit_us, int32_t* status, moedisp_stream_t stream) {
     if (!status) return MOEDISP_ERR_NULLPTR;
@@ -150,7 +150,7 @@ int moedisp_layout_workspace_size(moedisp_dims dims, size_t* bytes) {
 }
 
 int moedisp_moe_dispatch_layout(const int32_t* expert_ids, const uint8_t* active_mask,
-                                moedisp_dims dims, const moedisp_layout* layout,
+                                int active_mask_dims, moedisp_dims dims, const moedisp_layout* layout,
                                 void* workspace, size_t workspace_bytes, int32_t* status,
                                 moedisp_stream_t stream) {
     if (!layout || !status) return MOEDISP_ERR_NULLPTR;
@@ -162,6 +162,7 @@ int moedisp_moe_dispatch_layout(const int32_t* expert_ids, const uint8_t* active
     if (!L.cnt || !L.expert_base || !L.rank_base || !L.send_splits) return MOEDISP_ERR_NULLPTR;
     if (slots > 0 && (!expert_ids || !L.occ || !L.dst_row)) return MOEDISP_ERR_NULLPTR;
     if (L.rows_cap > 0 && !L.assist_info) return MOEDISP_ERR_NULLPTR;
+    if (active_mask && active_mask_dims != 1 && active_mask_dims != 2) return MOEDISP_ERR_INVALID;
     if (!workspace) return MOEDISP_ERR_WORKSPACE;
     const moedisp::LayoutGeometry g = moedisp::layout_geometry(dims);
     if (workspace_bytes < g.total_bytes) return MOEDISP_ERR_WORKSPACE;
@@ -180,13 +181,15 @@ int moedisp_moe_dispatch_layout(const int32_t* expert_ids, const uint8_t* active
                    {L.send_splits, (size_t)dims.W * dims.W * 8},
                    {workspace, g.total_bytes},
                    {status, 4}},
-                  {{expert_ids, (size_t)slots * 4}, {active_mask, (size_t)G}}))
+                  {{expert_ids, (size_t)slots * 4},
+                   {active_mask, (size_t)(active_mask_dims == 2 ? slots : G)}}))
         return MOEDISP_ERR_ALIASED;
-    return rc(moedisp::launch_layout(expert_ids, active_mask, dims, L, workspace, status, stream));
+    return rc(moedisp::launch_layout(expert_ids, active_mask, active_mask_dims, dims, L, workspace,
+                                     status, stream));
 }
 
 int moedisp_moe_dispatch_layout_noalloc(const int32_t* expert_ids, const uint8_t* active_mask,
-                                        moedisp_dims dims, const moedisp_layout* layout,
+                                        int active_mask_dims, moedisp_dims dims, const moedisp_layout* layout,
                                         int32_t* status, moedisp_stream_t stream) {
     if (!layout || !status) return MOEDISP_ERR_NULLPTR;
     int c = check_dims(dims);
@@ -197,6 +200,7 @@ int moedisp_moe_dispatch_layout_noalloc(const int32_t* expert_ids, const uint8_t
     if (!L.cnt || !L.expert_base || !L.rank_base || !L.send_splits) return MOEDISP_ERR_NULLPTR;
     if (slots > 0 && (!expert_ids || !L.occ || !L.dst_row)) return MOEDISP_ERR_NULLPTR;
     if (L.rows_cap > 0 && !L.assist_info) return MOEDISP_ERR_NULLPTR;
+    if (active_mask && active_mask_dims != 1 && active_mask_dims != 2) return MOEDISP_ERR_INVALID;
     if (moedisp::layout_geometry(dims).total_bytes > moedisp::layout_noalloc_scratch_bytes())
         return MOEDISP_ERR_UNSUPPORTED;
     if (!aligned(expert_ids, 4) || !aligned(L.cnt, 4) || !aligned(L.occ, 4) ||
@@ -212,13 +216,16 @@ int moedisp_moe_dispatch_layout_noalloc(const int32_t* expert_ids, const uint8_t
                    {L.rank_base, (size_t)(dims.W + 1) * 8},
                    {L.send_splits, (size_t)dims.W * dims.W * 8},
                    {status, 4}},
-                  {{expert_ids, (size_t)slots * 4}, {active_mask, (size_t)G}}))
+                  {{expert_ids, (size_t)slots * 4},
+                   {active_mask, (size_t)(active_mask_dims == 2 ? slots : G)}}))
         return MOEDISP_ERR_ALIASED;
-    return rc(moedisp::launch_layout_noalloc(expert_ids, active_mask, dims, L, status, stream));
+    return rc(moedisp::launch_layout_noalloc(expert_ids, active_mask, active_mask_dims, dims, L,
+                                             status, stream));
 }
 
 int moedisp_moe_dispatch(const void* x, int H, moedisp_dims dims,
-                         const moedisp_layout* layout, int quant_mode, void* expand_x,
+                         const moedisp_layout* layout, int quant_mode,
+                         const float* smooth_scales, const int32_t* expert_ids, void* expand_x,
                          float* dynamic_scales, int64_t* expert_token_nums,
                          int expert_token_nums_type, int32_t* ep_recv_counts,
                          int32_t* status, moedisp_stream_t stream) {
@@ -232,12 +239,14 @@ int moedisp_moe_dispatch(const void* x, int H, moedisp_dims dims,
         return MOEDISP_ERR_INVALID;
     if (expert_token_nums && expert_token_nums_type != 0 && expert_token_nums_type != 1)
         return MOEDISP_ERR_INVALID;
+    if (smooth_scales && quant_mode == MOEDISP_QUANT_NONE) return MOEDISP_ERR_INVALID;
     if (H <= 0) return MOEDISP_ERR_INVALID;
     if (H > MOEDISP_MAX_H) return MOEDISP_ERR_UNSUPPORTED;
     if (H % (quant_mode == MOEDISP_QUANT_NONE ? 8 : 16) != 0) return MOEDISP_ERR_MISALIGNED;
     const int64_t G = (int64_t)dims.W * dims.T;
     const int64_t slots = G * dims.K;
     if (G > 0 && (!x || !L.dst_row)) return MOEDISP_ERR_NULLPTR;
+    if (G > 0 && smooth_scales && !expert_ids) return MOEDISP_ERR_NULLPTR;
     if (L.rows_cap > 0 && !expand_x) return MOEDISP_ERR_NULLPTR;
     if (quant_mode != MOEDISP_QUANT_NONE && L.rows_cap > 0 && !dynamic_scales)
         return MOEDISP_ERR_NULLPTR;
@@ -245,7 +254,8 @@ int moedisp_moe_dispatch(const void* x, int H, moedisp_dims dims,
     if (ep_recv_counts && !L.cnt) return MOEDISP_ERR_NULLPTR;
     if (!aligned(x, 16) || !aligned(expand_x, 16) || !aligned(L.dst_row, 4) ||
         !aligned(dynamic_scales, 4) || !aligned(expert_token_nums, 8) ||
-        !aligned(ep_recv_counts, 4) || !aligned(status, 4))
+        !aligned(ep_recv_counts, 4) || !aligned(status, 4) || !aligned(smooth_scales, 16) ||
+        !aligned(expert_ids, 4))
         return MOEDISP_ERR_MISALIGNED;
     const size_t out_row = quant_mode == MOEDISP_QUANT_NONE ? (size_t)H * 2 : (size_t)H;
     const int ne = dims.E / dims.W;
@@ -258,11 +268,14 @@ int moedisp_moe_dispatch(const void* x, int H, moedisp_dims dims,
                    {status, 4}},
                   {{x, (size_t)G * H * 2},
                    {L.dst_row, (size_t)slots * 4},
+                   {smooth_scales, (size_t)dims.E * H * 4},
+                   {smooth_scales ? expert_ids : nullptr, (size_t)slots * 4},
                    {L.cnt, (size_t)dims.W * dims.E * 4},
                    {L.expert_base, (size_t)(dims.E + 1) * 8},
                    {L.rank_base, (size_t)(dims.W + 1) * 8}}))
         return MOEDISP_ERR_ALIASED;
-    return rc(moedisp::launch_dispatch(x, H, dims, L, quant_mode, expand_x, dynamic_scales,
+    return rc(moedisp::launch_dispatch(x, H, dims, L, quant_mode, smooth_scales,
+                                       smooth_scales ? expert_ids : nullptr, expand_x, dynamic_scales,
                                        expert_token_nums, expert_token_nums_type, ep_recv_counts,
                                        status, stream));
 }

@@ -27,6 +27,8 @@ struct DispatchArgs {
     int64_t rows_cap;
     uint8_t* expand_x;
     float* scales;
+    const float* smooth;       // [E][H] per-expert smoothing (quantising modes) or null
+    const int32_t* ids;        // [G][K] expert ids, with smooth
     int stages;
     uint32_t in_bytes, out_bytes;
     // receive counts (optional)
@@ -110,6 +112,29 @@ __device__ __forceinline__ uint32_t q_e4m3_pair(uint32_t w, float scale, float i
     return q_e4m3(bf16_lo(w), scale, inv) | (q_e4m3(bf16_hi(w), scale, inv) << 8);
 }
 
+// Eight fp32 values (a smoothed row chunk) to eight codes.
+template <int Q>
+__device__ __forceinline__ uint2 quant8f(const float (&v)[8], float scale, float inv, bool zero) {
+    if (zero) return make_uint2(0u, 0u);
+    uint32_t b[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        b[j] = Q == MOEDISP_QUANT_INT8 ? (uint32_t)(q_int8(v[j], scale, inv) & 0xff)
+                                       : q_e4m3(v[j], scale, inv);
+    return make_uint2(b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24),
+                      b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24));
+}
+
+// x chunk (8 bf16) times a smoothing chunk (8 fp32), one correctly rounded product each.
+__device__ __forceinline__ void smooth8(const uint4& v, const float* s, float (&o)[8]) {
+    const float4 s0 = __ldg(reinterpret_cast<const float4*>(s));
+    const float4 s1 = __ldg(reinterpret_cast<const float4*>(s) + 1);
+    o[0] = __fmul_rn(bf16_lo(v.x), s0.x); o[1] = __fmul_rn(bf16_hi(v.x), s0.y);
+    o[2] = __fmul_rn(bf16_lo(v.y), s0.z); o[3] = __fmul_rn(bf16_hi(v.y), s0.w);
+    o[4] = __fmul_rn(bf16_lo(v.z), s1.x); o[5] = __fmul_rn(bf16_hi(v.z), s1.y);
+    o[6] = __fmul_rn(bf16_lo(v.w), s1.z); o[7] = __fmul_rn(bf16_hi(v.w), s1.w);
+}
+
 template <int Q>
 __device__ __forceinline__ uint2 quant8(const uint4& v, float scale, float inv, bool zero) {
     if (zero) return make_uint2(0u, 0u);
@@ -160,6 +185,12 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
         fence_mbar_init();
     }
     __syncwarp();
+    // The first rows this block will load go to L2 while the kernel this one depends on
+    // (normally the layout, which moves little data) is still running.
+    if (lane < S) {
+        const int64_t g = (int64_t)blockIdx.x + (int64_t)lane * gridDim.x;
+        if (g < a.G) bulk_prefetch_l2(a.x + g * a.in_bytes, a.in_bytes);
+    }
     grid_dep_wait();
     grid_dep_launch_dependents();
     write_recv_counts(a);
@@ -254,16 +285,23 @@ __device__ __forceinline__ void group_barrier(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-template <int Q, int WPT>
+//
+// With per-expert smoothing (SM), the copy for slot k is x * smooth[e_k] quantised on its
+// own: the group reduces K maxima of |x * smooth[e_k]| in one pass over the row, then
+// recomputes the products chunk by chunk (the smoothing rows come from L2) and stores
+// each slot's codes and scale.
+template <int Q, int WPT, bool SM>
 __global__ void __launch_bounds__(kQuantThreads, 2) dispatch_quant_kernel(DispatchArgs a) {
     constexpr int NG = kQuantThreads / 32 / WPT;     // token groups per block
     constexpr int GT = WPT * 32;                     // threads per group
+    constexpr int KS = SM ? MOEDISP_MAX_K : 1;       // maxima reduced per token
     constexpr float kQmax = Q == MOEDISP_QUANT_INT8 ? 127.0f : 448.0f;
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t bars[NG][kMaxStages];
     __shared__ int64_t tok[NG][kMaxStages];
     __shared__ int32_t drow[NG][kMaxStages][MOEDISP_MAX_K];
-    __shared__ float red[NG][2][WPT];
+    __shared__ int32_t dexp[NG][kMaxStages][KS];     // expert of each slot (SM)
+    __shared__ float red[NG][2][KS][WPT];
     __shared__ int abort_s[NG];
     __shared__ unsigned next_s;                      // the block's next token index
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -277,8 +315,14 @@ __global__ void __launch_bounds__(kQuantThreads, 2) dispatch_quant_kernel(Dispat
         fence_mbar_init();
         abort_s[grp] = 0;
     }
+    if (SM && gt < S * KS) dexp[grp][gt / KS][gt % KS] = 0;   // always a valid expert id
     if (tid == 0) next_s = 0;
     __syncthreads();
+    // L2 prefetch of the block's first NG * S token rows (see dispatch_copy_kernel).
+    if (tid < NG * S) {
+        const int64_t g = (int64_t)blockIdx.x + (int64_t)tid * gridDim.x;
+        if (g < a.G) bulk_prefetch_l2(a.x + g * a.in_bytes, a.in_bytes);
+    }
     grid_dep_wait();
     grid_dep_launch_dependents();
     write_recv_counts(a);
@@ -294,18 +338,24 @@ __global__ void __launch_bounds__(kQuantThreads, 2) dispatch_quant_kernel(Dispat
         return (int64_t)blockIdx.x + (int64_t)i * gridDim.x;
     };
     int64_t pf_g = 0;
-    int32_t pf_d = -1;
+    int32_t pf_d = -1, pf_e = 0;
+    auto load_routing = [&]() {
+        const bool mine = pf_g < a.G && lane < K;
+        pf_d = mine ? __ldg(a.dst_row + pf_g * K + lane) : -1;
+        if (SM) pf_e = mine ? __ldg(a.ids + pf_g * K + lane) : 0;
+    };
     if (gw == 0) {
         pf_g = next_token();
-        pf_d = (pf_g < a.G && lane < K) ? __ldg(a.dst_row + pf_g * K + lane) : -1;
+        load_routing();
     }
     auto fill = [&](int st) {
         while (true) {
             const int64_t g = pf_g;
             int32_t d = pf_d;
+            const int32_t e = pf_e;
             if (g < a.G) {
                 pf_g = next_token();
-                pf_d = (pf_g < a.G && lane < K) ? __ldg(a.dst_row + pf_g * K + lane) : -1;
+                load_routing();
             }
             if (g >= a.G) {
                 if (lane == 0) {
@@ -318,11 +368,24 @@ __global__ void __launch_bounds__(kQuantThreads, 2) dispatch_quant_kernel(Dispat
                 raise_status(a.status, MOEDISP_STATUS_CAPACITY);
                 d = -1;
             }
+            if (SM && d >= 0 && (e < 0 || e >= a.E)) {
+                raise_status(a.status, MOEDISP_STATUS_BAD_EXPERT_ID);
+                d = -1;
+            }
             if (d < 0) d = -1;
             if (__ballot_sync(0xffffffffu, d >= 0)) {
                 int32_t dk[MOEDISP_MAX_K];
 #pragma unroll
                 for (int k = 0; k < MOEDISP_MAX_K; ++k) dk[k] = __shfl_sync(0xffffffffu, d, k);
+                if (SM) {
+                    // lane 0 publishes the slots' experts with the rows (its barrier arrival
+                    // releases its own writes)
+#pragma unroll
+                    for (int k = 0; k < KS; ++k) {
+                        const int32_t ek = __shfl_sync(0xffffffffu, e, k);
+                        if (lane == 0 && k < K && dk[k] >= 0) dexp[grp][st][k] = ek;
+                    }
+                }
                 if (lane == 0) {
 #pragma unroll
                     for (int k = 0; k < MOEDISP_MAX_K; ++k)
@@ -349,15 +412,48 @@ __global__ void __launch_bounds__(kQuantThreads, 2) dispatch_quant_kernel(Dispat
 #pragma unroll
         for (int k = 0; k < MOEDISP_MAX_K; ++k) d[k] = k < K ? drow[grp][st][k] : -1;
         const uint4* row = reinterpret_cast<const uint4*>(inbuf + (size_t)st * a.in_bytes);
-        float m = 0.0f;
-        for (int c = gt; c < nvec; c += GT) m = fmaxf(m, absmax8(row[c]));
+        // Row maxima: of |x| (one), or of |x * smooth[e_k]| per slot (SM). Expert ids in
+        // dexp are always in [0, E), even in a stage whose token is stale.
+        float m[KS];
+        int32_t ex[KS];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        for (int k = 0; k < KS; ++k) {
+            m[k] = 0.0f;
+            ex[k] = SM ? dexp[grp][st][k] : 0;
+        }
+        for (int c = gt; c < nvec; c += GT) {
+            const uint4 v = row[c];
+            if (SM) {
+#pragma unroll
+                for (int k = 0; k < KS; ++k) {
+                    if (k < K && d[k] >= 0) {
+                        float xs[8];
+                        smooth8(v, a.smooth + (int64_t)ex[k] * a.H + 8 * c, xs);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) m[k] = fmaxf(m[k], fabsf(xs[j]));
+                    }
+                }
+            } else {
+                m[0] = fmaxf(m[0], absmax8(v));
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < KS; ++k) {
+            if (k < (SM ? K : 1)) {
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) m[k] = fmaxf(m[k], __shfl_xor_sync(0xffffffffu, m[k], o));
+            }
+        }
         if (WPT > 1) {
-            if (lane == 0) red[grp][it & 1][gw] = m;
+            if (lane == 0) {
+#pragma unroll
+                for (int k = 0; k < KS; ++k) red[grp][it & 1][k][gw] = m[k];
+            }
             group_barrier(1 + grp, GT);
 #pragma unroll
-            for (int w = 0; w < WPT; ++w) m = fmaxf(m, red[grp][it & 1][w]);
+            for (int k = 0; k < KS; ++k)
+#pragma unroll
+                for (int w = 0; w < WPT; ++w) m[k] = fmaxf(m[k], red[grp][it & 1][k][w]);
         } else {
             __syncwarp();
         }
@@ -368,9 +464,34 @@ __global__ void __launch_bounds__(kQuantThreads, 2) dispatch_quant_kernel(Dispat
         // Every thread of the group is past the previous token: its stage is free.
         if (gw == 0 && it >= 1) fill((it - 1) % S);
         if (g < 0) break;
-        const float scale = __fdiv_rn(m, kQmax);
+        if (SM) {
+            float sc[KS], iv[KS];
+#pragma unroll
+            for (int k = 0; k < KS; ++k) {
+                sc[k] = __fdiv_rn(m[k], kQmax);
+                iv[k] = __frcp_rn(sc[k]);
+            }
+            for (int c = gt; c < nvec; c += GT) {
+                const uint4 v = row[c];
+#pragma unroll
+                for (int k = 0; k < KS; ++k) {
+                    if (k < K && d[k] >= 0) {
+                        float xs[8];
+                        smooth8(v, a.smooth + (int64_t)ex[k] * a.H + 8 * c, xs);
+                        __stcs(reinterpret_cast<uint2*>(a.expand_x + (int64_t)d[k] * a.out_bytes) + c,
+                               quant8f<Q>(xs, sc[k], iv[k], m[k] == 0.0f));
+                    }
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < KS; ++k)
+                if (gt == k && k < K && d[k] >= 0) a.scales[d[k]] = sc[k];
+            continue;
+        }
+        const float m0 = m[0];
+        const float scale = __fdiv_rn(m0, kQmax);
         const float inv = __frcp_rn(scale);
-        const bool zero = m == 0.0f;
+        const bool zero = m0 == 0.0f;
         if (K <= 8) {                          // row bases once per token, 8-way stores
             uint2* dst[8];
 #pragma unroll
@@ -423,7 +544,7 @@ cudaError_t launch_copy(DispatchArgs a, cudaStream_t stream) {
                       1, a);
 }
 
-template <int Q, int WPT>
+template <int Q, int WPT, bool SM>
 cudaError_t launch_quant_w(DispatchArgs a, cudaStream_t stream) {
     constexpr int NG = kQuantThreads / 32 / WPT;
     // Stages per group: two for single-warp groups (small rows: more blocks per SM pays
@@ -431,29 +552,35 @@ cudaError_t launch_quant_w(DispatchArgs a, cudaStream_t stream) {
     a.stages = WPT == 1 ? 2 : 3;
     const size_t smem = (size_t)NG * a.stages * a.in_bytes;
     int per_sm = 1;
-    cudaError_t err = blocks_per_sm((const void*)dispatch_quant_kernel<Q, WPT>, kQuantThreads, smem,
-                                    &per_sm);
+    cudaError_t err = blocks_per_sm((const void*)dispatch_quant_kernel<Q, WPT, SM>, kQuantThreads,
+                                    smem, &per_sm);
     if (err != cudaSuccess) return err;
     int64_t grid = (int64_t)current_sm_count() * per_sm;
     grid = std::min<int64_t>(grid, std::max<int64_t>((a.G + NG - 1) / NG, 1));
-    return launch_pdl(dispatch_quant_kernel<Q, WPT>, dim3((unsigned)grid), dim3(kQuantThreads), smem,
-                      stream, 1, a);
+    return launch_pdl(dispatch_quant_kernel<Q, WPT, SM>, dim3((unsigned)grid), dim3(kQuantThreads),
+                      smem, stream, 1, a);
 }
 
 // Warps per token: the fewest that hold a row in kChunks 16-byte chunks per thread.
+template <int Q, bool SM>
+cudaError_t launch_quant_s(const DispatchArgs& a, cudaStream_t stream) {
+    const int nvec = a.H / 8;
+    if (nvec <= 1 * 32 * kChunks) return launch_quant_w<Q, 1, SM>(a, stream);
+    if (nvec <= 2 * 32 * kChunks) return launch_quant_w<Q, 2, SM>(a, stream);
+    if (nvec <= 4 * 32 * kChunks) return launch_quant_w<Q, 4, SM>(a, stream);
+    return launch_quant_w<Q, 8, SM>(a, stream);
+}
+
 template <int Q>
 cudaError_t launch_quant(const DispatchArgs& a, cudaStream_t stream) {
-    const int nvec = a.H / 8;
-    if (nvec <= 1 * 32 * kChunks) return launch_quant_w<Q, 1>(a, stream);
-    if (nvec <= 2 * 32 * kChunks) return launch_quant_w<Q, 2>(a, stream);
-    if (nvec <= 4 * 32 * kChunks) return launch_quant_w<Q, 4>(a, stream);
-    return launch_quant_w<Q, 8>(a, stream);
+    return a.smooth != nullptr ? launch_quant_s<Q, true>(a, stream) : launch_quant_s<Q, false>(a, stream);
 }
 
 }  // namespace
 
 cudaError_t launch_dispatch(const void* x, int H, const moedisp_dims& dims,
-                            const moedisp_layout& L, int quant_mode, void* expand_x,
+                            const moedisp_layout& L, int quant_mode, const float* smooth_scales,
+                            const int32_t* expert_ids, void* expand_x,
                             float* dynamic_scales, int64_t* expert_token_nums,
                             int expert_token_nums_type, int32_t* ep_recv_counts,
                             int32_t* status, cudaStream_t stream) {
@@ -466,6 +593,8 @@ cudaError_t launch_dispatch(const void* x, int H, const moedisp_dims& dims,
     a.rows_cap = L.rows_cap;
     a.expand_x = static_cast<uint8_t*>(expand_x);
     a.scales = dynamic_scales;
+    a.smooth = smooth_scales;
+    a.ids = expert_ids;
     a.stages = 2;
     a.in_bytes = (uint32_t)H * 2u;
     a.out_bytes = quant_mode == MOEDISP_QUANT_NONE ? (uint32_t)H * 2u : (uint32_t)H;

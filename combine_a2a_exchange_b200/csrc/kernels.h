@@ -70,20 +70,21 @@ struct LayoutGeometry {
 };
 LayoutGeometry layout_geometry(const moedisp_dims& d);
 
-cudaError_t launch_layout(const int32_t* expert_ids, const uint8_t* active,
+cudaError_t launch_layout(const int32_t* expert_ids, const uint8_t* active, int active_dims,
                           const moedisp_dims& dims, const moedisp_layout& layout,
                           void* workspace, int32_t* status, cudaStream_t stream);
 
 // Allocation-free layout: the tiled path on the library's static scratch array.
 size_t layout_noalloc_scratch_bytes();
 cudaError_t launch_layout_noalloc(const int32_t* expert_ids, const uint8_t* active,
-                                  const moedisp_dims& dims, const moedisp_layout& layout,
+                                  int active_dims, const moedisp_dims& dims, const moedisp_layout& layout,
                                   int32_t* status, cudaStream_t stream);
 
 cudaError_t launch_bounded_wait_selftest(uint64_t limit_ns, int32_t* status, cudaStream_t stream);
 
 cudaError_t launch_dispatch(const void* x, int H, const moedisp_dims& dims,
-                            const moedisp_layout& layout, int quant_mode, void* expand_x,
+                            const moedisp_layout& layout, int quant_mode,
+                            const float* smooth_scales, const int32_t* expert_ids, void* expand_x,
                             float* dynamic_scales, int64_t* expert_token_nums,
                             int expert_token_nums_type, int32_t* ep_recv_counts,
                             int32_t* status, cudaStream_t stream);

@@ -57,7 +57,8 @@ constexpr int kCMaxCluster = 16;
 
 struct LayoutArgs {
     const int32_t* ids;
-    const uint8_t* active;
+    const uint8_t* active;     // null, [G] (per token, active_dims 1) or [G*K] (per slot, 2)
+    int active_dims;
     int W, T, K, E, ne;
     int64_t P;                 // slots per source rank, T*K
     int tiles_per_rank;
@@ -81,7 +82,9 @@ struct LayoutArgs {
 __device__ __forceinline__ int slot_expert(const LayoutArgs& a, int64_t s, bool& bad) {
     const int e = __ldg(a.ids + s);
     // s < 2^30 (checked on the host), so a 32-bit division finds the token.
-    if (a.active != nullptr && __ldg(a.active + (uint32_t)s / (uint32_t)a.K) == 0) return -1;
+    if (a.active != nullptr &&
+        __ldg(a.active + (a.active_dims == 1 ? (uint32_t)s / (uint32_t)a.K : (uint32_t)s)) == 0)
+        return -1;
     if (e < 0 || e >= a.E) {
         bad = true;
         return -1;
@@ -550,13 +553,14 @@ LayoutGeometry layout_geometry(const moedisp_dims& d) {
 }
 
 namespace {
-LayoutArgs make_args(const int32_t* expert_ids, const uint8_t* active, const moedisp_dims& dims,
-                     const moedisp_layout& L, void* workspace, int32_t* status,
-                     const LayoutGeometry& g) {
+LayoutArgs make_args(const int32_t* expert_ids, const uint8_t* active, int active_dims,
+                     const moedisp_dims& dims, const moedisp_layout& L, void* workspace,
+                     int32_t* status, const LayoutGeometry& g) {
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     LayoutArgs a;
     a.ids = expert_ids;
     a.active = active;
+    a.active_dims = active_dims;
     a.W = dims.W;
     a.T = dims.T;
     a.K = dims.K;
@@ -581,11 +585,11 @@ LayoutArgs make_args(const int32_t* expert_ids, const uint8_t* active, const moe
 }
 }  // namespace
 
-cudaError_t launch_layout(const int32_t* expert_ids, const uint8_t* active,
+cudaError_t launch_layout(const int32_t* expert_ids, const uint8_t* active, int active_dims,
                           const moedisp_dims& dims, const moedisp_layout& L, void* workspace,
                           int32_t* status, cudaStream_t stream) {
     const LayoutGeometry g = layout_geometry(dims);
-    LayoutArgs a = make_args(expert_ids, active, dims, L, workspace, status, g);
+    LayoutArgs a = make_args(expert_ids, active, active_dims, dims, L, workspace, status, g);
 
     int tpr_c = 0, steps_c = 0;
     int64_t tile_c = 0;
@@ -643,7 +647,8 @@ cudaError_t layout_scratch_address(void** out) {
 size_t layout_noalloc_scratch_bytes() { return MOEDISP_NOALLOC_SCRATCH_BYTES; }
 
 cudaError_t launch_layout_noalloc(const int32_t* expert_ids, const uint8_t* active,
-                                  const moedisp_dims& dims, const moedisp_layout& L,
+                                  int active_dims, const moedisp_dims& dims,
+                                  const moedisp_layout& L,
                                   int32_t* status, cudaStream_t stream) {
     const LayoutGeometry g = layout_geometry(dims);
     void* scratch = nullptr;
@@ -651,7 +656,7 @@ cudaError_t launch_layout_noalloc(const int32_t* expert_ids, const uint8_t* acti
     if (err != cudaSuccess) return err;
     // The array keeps whatever the previous call left; nothing in it has to start at
     // zero: every scratch word is written (tile counts, then offsets) before it is read.
-    LayoutArgs a = make_args(expert_ids, active, dims, L, scratch, status, g);
+    LayoutArgs a = make_args(expert_ids, active, active_dims, dims, L, scratch, status, g);
     return launch_tiled(a, dims, g, stream);
 }
 

@@ -64,7 +64,8 @@ typedef struct CUstream_st *moedisp_stream_t;
 /* Returns a static, human-readable name for a return code (< 0) or status bits (> 0). */
 const char *moedisp_status_string(int code);
 
-/* ABI version, currently 1. */
+/* ABI version, currently 2 (2: active_mask_dims in the layout calls; smoothing scales in
+ * moe_dispatch). */
 int moedisp_version(void);
 
 /* Diagnostic for the time-out path of the device-side waits (this library's own
@@ -148,7 +149,8 @@ int moedisp_layout_workspace_size(moedisp_dims dims, size_t *bytes);
  * Routes the G*K (token, expert) slots into an expert-grouped layout, following the
  * PyTorch symm_mem 2-D exchange plan and index-push dispatch (get_occurrence_numbers,
  * make2dExchangePlan, _allToAllV_2d_index_push_kernel) and the Ascend
- * aclnnMoeDistributeDispatchV2 inputs (expertIds int32 [Bs][K], 1-D xActiveMask):
+ * aclnnMoeDistributeDispatchV2 inputs (expertIds int32 [Bs][K], xActiveMask of shape
+ * (Bs,) or (Bs, K)):
  *   cnt[r][e]   = active slots of rank r with expert e (the 2-D plan's in_splits);
  *   occ[s]      = earlier active slots of s's rank with s's expert (0-based);
  *   rows of expand_x are ordered by destination rank, then local expert, then source
@@ -156,9 +158,12 @@ int moedisp_layout_workspace_size(moedisp_dims dims, size_t *bytes);
  *   all active slots by expert id:
  *     dst_row[s] = expert_base[e] + sum_{r' < r} cnt[r'][e] + occ[s];
  *   assist_info[dst_row[s]] = s.
- * expert_ids: int32 [G][K] device; active_mask: uint8 [G] device or NULL (all active; any
- * pattern of active tokens is accepted). A slot is active when its token is active and
- * its expert id lies in [0, E); an active token's out-of-range id sets
+ * expert_ids: int32 [G][K] device; active_mask: uint8 device or NULL (all active), with
+ * active_mask_dims 1: [G], one flag per token (any pattern of active tokens is
+ * accepted), or 2: [G][K], one flag per slot (a token whose K flags are all zero sends
+ * nothing); active_mask_dims is ignored when active_mask is NULL, else anything but 1 or 2
+ * is MOEDISP_ERR_INVALID. A slot is active when its flag (or its token's) is nonzero and
+ * its expert id lies in [0, E); an active slot's out-of-range id sets
  * MOEDISP_STATUS_BAD_EXPERT_ID and that slot is dropped. If R > rows_cap,
  * MOEDISP_STATUS_CAPACITY is set, every output is still computed, and assist_info is
  * written only below rows_cap.
@@ -170,7 +175,7 @@ int moedisp_layout_workspace_size(moedisp_dims dims, size_t *bytes);
  * three: per-tile warp-aggregated histograms, per-expert scans down the tiles, and a
  * per-tile ranking + scatter. */
 int moedisp_moe_dispatch_layout(const int32_t *expert_ids, const uint8_t *active_mask,
-                                moedisp_dims dims, const moedisp_layout *layout,
+                                int active_mask_dims, moedisp_dims dims, const moedisp_layout *layout,
                                 void *workspace, size_t workspace_bytes, int32_t *status,
                                 moedisp_stream_t stream);
 
@@ -198,7 +203,7 @@ int moedisp_moe_dispatch_layout(const int32_t *expert_ids, const uint8_t *active
  * Other arguments and errors are those of moedisp_moe_dispatch_layout. */
 #define MOEDISP_NOALLOC_SCRATCH_BYTES (2u << 20)
 int moedisp_moe_dispatch_layout_noalloc(const int32_t *expert_ids, const uint8_t *active_mask,
-                                        moedisp_dims dims, const moedisp_layout *layout,
+                                        int active_mask_dims, moedisp_dims dims, const moedisp_layout *layout,
                                         int32_t *status, moedisp_stream_t stream);
 
 /* Quantisation modes of moe_dispatch (the Ascend quantMode values; 3 is this library's
@@ -218,6 +223,12 @@ int moedisp_moe_dispatch_layout_noalloc(const int32_t *expert_ids, const uint8_t
  *   FP8_E4M3: scale = a / 448, q = a == 0 ? 0 : e4m3(x / scale), round to nearest even,
  *         saturating to +-448                                    (e4m3, H bytes/row)
  *   dynamic_scales[dst_row[s]] = scale (quant modes).
+ * smooth_scales (Ascend scalesOptional, the per-expert quantisation smoothing factors):
+ * fp32 [E][H] device, 16-byte aligned, or NULL; quant modes only (with NONE it is
+ * MOEDISP_ERR_INVALID). When given, the copy for slot s = (g, k) with expert
+ * e = expert_ids[s] quantises x[g] * smooth_scales[e] (one fp32 product per element)
+ * instead of x[g], with its own a and scale; expert_ids (int32 [G][K] device, the layout's
+ * input) is then required, and is ignored otherwise.
  * x: bf16 [G][H] device, 16-byte aligned; expand_x: [layout->rows_cap][H] elements of
  * the output type, 16-byte aligned, not overlapping x; dynamic_scales: fp32
  * [rows_cap] (required for quant modes, ignored otherwise). H % 8 == 0 (NONE) or
@@ -228,9 +239,11 @@ int moedisp_moe_dispatch_layout_noalloc(const int32_t *expert_ids, const uint8_t
  *   ep_recv_counts int32 [W][ne][W]: rows expert d*ne+le receives from source rank r.
  * Rows at or beyond rows_cap are not written (MOEDISP_STATUS_CAPACITY).
  * One persistent kernel: each token row is brought into shared memory once by a bulk
- * (TMA) copy, quantised there if asked, and written to its K rows by bulk copies. */
+ * (TMA) copy; unquantised rows leave it as K bulk copies, quantised ones as 8-byte
+ * streaming stores of the codes to the K rows. */
 int moedisp_moe_dispatch(const void *x, int H, moedisp_dims dims,
-                         const moedisp_layout *layout, int quant_mode, void *expand_x,
+                         const moedisp_layout *layout, int quant_mode,
+                         const float *smooth_scales, const int32_t *expert_ids, void *expand_x,
                          float *dynamic_scales, int64_t *expert_token_nums,
                          int expert_token_nums_type, int32_t *ep_recv_counts,
                          int32_t *status, moedisp_stream_t stream);

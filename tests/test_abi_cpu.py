@@ -49,7 +49,7 @@ def test_library_exports_every_declared_symbol(md):
 
 
 def test_status_strings(md):
-    assert md.version() == 1
+    assert md.version() == 2
     assert md.status_string(0) == "ok"
     assert md.status_string(-1) == "null pointer"
     assert md.status_string(md.STATUS_CAPACITY | md.STATUS_TIMEOUT) == "capacity | timeout"
@@ -113,8 +113,8 @@ def test_layout_rejections(md):
     with pytest.raises(md.MoedispError):
         md.layout_workspace_size(4, 8, 17, 8)                # K > 16
     L = _layout(md)
-    call = lambda ids, dims, L, ws, nws, st: md.raw_call(
-        "moedisp_moe_dispatch_layout", ids, None, dims, ctypes.byref(L), ws, nws, st, None)
+    call = lambda ids, dims, L, ws, nws, st, act=None, ad=0: md.raw_call(
+        "moedisp_moe_dispatch_layout", ids, act, ad, dims, ctypes.byref(L), ws, nws, st, None)
     ids, ws, st = FAKE + (64 << 20), FAKE + (128 << 20), FAKE + (256 << 20)
     d = md.Dims(4, 8, 2, 8)
     assert call(ids, d, L, ws, ws_ok - 1, st) == md.MOEDISP_ERR_WORKSPACE
@@ -129,14 +129,20 @@ def test_layout_rejections(md):
     bad = _layout(md, rows_cap=-1)
     assert call(ids, d, bad, ws, ws_ok, st) == md.MOEDISP_ERR_INVALID
     assert call(ids, d, L, L.cnt, ws_ok, st) == md.MOEDISP_ERR_ALIASED   # workspace over cnt
+    act = FAKE + (300 << 20)
+    assert call(ids, d, L, ws, ws_ok, st, act, 0) == md.MOEDISP_ERR_INVALID    # mask dims
+    assert call(ids, d, L, ws, ws_ok, st, act, 3) == md.MOEDISP_ERR_INVALID
+    # a per-slot mask [G][K] spans G*K bytes: one starting G*K - 1 bytes before occ overlaps it
+    G, K = 4 * 8, 2
+    assert call(ids, d, L, ws, ws_ok, st, L.occ - (G * K - 1), 2) == md.MOEDISP_ERR_ALIASED
 
 
 def test_dispatch_and_combine_rejections(md):
     L = _layout(md)
     d = md.Dims(4, 8, 2, 8)
     x, ex, sc, st = FAKE + (64 << 20), FAKE + (128 << 20), FAKE + (192 << 20), FAKE + (256 << 20)
-    disp = lambda x, H, q, ex, sc, st, etn=None, t=1: md.raw_call(
-        "moedisp_moe_dispatch", x, H, d, ctypes.byref(L), q, ex, sc, etn, t, None, st, None)
+    disp = lambda x, H, q, ex, sc, st, etn=None, t=1, sm=None, ids=None: md.raw_call(
+        "moedisp_moe_dispatch", x, H, d, ctypes.byref(L), q, sm, ids, ex, sc, etn, t, None, st, None)
     assert disp(x, 128, 1, ex, sc, st) == md.MOEDISP_ERR_INVALID           # quant mode
     assert disp(x, 120, 2, ex, sc, st) == md.MOEDISP_ERR_MISALIGNED        # H % 16 (quant)
     assert disp(x, 124, 0, ex, sc, st) == md.MOEDISP_ERR_MISALIGNED        # H % 8
@@ -147,6 +153,12 @@ def test_dispatch_and_combine_rejections(md):
     assert disp(x + 8, 128, 0, ex, None, st) == md.MOEDISP_ERR_MISALIGNED
     assert disp(x, 128, 0, ex, None, None) == md.MOEDISP_ERR_NULLPTR
     assert disp(x, 128, 0, ex, None, st, etn=FAKE + (300 << 20), t=5) == md.MOEDISP_ERR_INVALID
+    sm, ids = FAKE + (320 << 20), FAKE + (384 << 20)
+    assert disp(x, 128, 0, ex, None, st, sm=sm, ids=ids) == md.MOEDISP_ERR_INVALID  # smoothing, no quant
+    assert disp(x, 128, 2, ex, sc, st, sm=sm) == md.MOEDISP_ERR_NULLPTR             # no expert ids
+    assert disp(x, 128, 2, ex, sc, st, sm=sm + 4, ids=ids) == md.MOEDISP_ERR_MISALIGNED
+    assert disp(x, 128, 2, ex, sc, st, sm=sm, ids=ids + 2) == md.MOEDISP_ERR_MISALIGNED
+    assert disp(x, 128, 2, sm + 256, sc, st, sm=sm, ids=ids) == md.MOEDISP_ERR_ALIASED  # out over smooth
     comb = lambda eo, H, w, y, st: md.raw_call(
         "moedisp_moe_combine", eo, H, d, ctypes.byref(L), w, y, st, None)
     assert comb(ex, 100, x, sc, st) == md.MOEDISP_ERR_MISALIGNED

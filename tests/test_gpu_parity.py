@@ -193,6 +193,10 @@ LAYOUT_CASES = [
     # one cluster, two tiles per rank and the largest tile
     ("tiny", dict(W=8, T=2048, K=8, E=256, routing="zipf")),
     ("tiny", dict(W=1, T=2048, K=8, E=1024)),
+    # per-slot (2-D) active masks: cluster path, tiled path, K = 1
+    ("tiny", dict(W=3, T=500, K=4, E=12, slot_active_p=0.5)),
+    ("tiny", dict(W=2, T=30000, K=8, E=16, slot_active_p=0.6)),
+    ("tiny", dict(W=4, T=100, K=1, E=8, slot_active_p=0.5)),
     ("cfg2", {}), ("cfg3", {}), ("cfg4", {}),
 ]
 
@@ -241,7 +245,7 @@ def test_layout_capacity_overflow(md):
 
 # ------------------------------------------------------------------ dispatch
 
-def run_dispatch(md, w, L, quant_mode, etn_type=1):
+def run_dispatch(md, w, L, quant_mode, etn_type=1, smooth=None):
     x = bf16_dev(w.x_bits)
     full, scales, gr = alloc_expand(L, w.H, quant_mode)
     ex = full[gr:gr + L.rows_cap]
@@ -251,7 +255,9 @@ def run_dispatch(md, w, L, quant_mode, etn_type=1):
     erc = torch.full((w.W, ne, w.W), -1, dtype=torch.int32, device="cuda")
     st = new_status()
     md.moe_dispatch(x, w.H, L, quant_mode, ex, sc if quant_mode else None, st,
-                    expert_token_nums=etn, expert_token_nums_type=etn_type, ep_recv_counts=erc)
+                    expert_token_nums=etn, expert_token_nums_type=etn_type, ep_recv_counts=erc,
+                    smooth_scales=None if smooth is None else dev(smooth),
+                    expert_ids=None if smooth is None else dev(w.expert_ids))
     torch.cuda.synchronize()
     return full, scales, gr, etn.cpu().numpy(), erc.cpu().numpy(), int(st.item())
 
@@ -265,6 +271,8 @@ DISPATCH_CASES = [
     ("tiny", dict(W=2, T=64, K=16, E=32, H=16384), 0),                # largest H, K
     ("tiny", dict(W=2, T=64, K=16, E=32, H=16384), 2),
     ("tiny", dict(W=4, T=50, K=5, E=8, H=8, routing="dup"), 0),       # smallest H
+    ("tiny", dict(W=3, T=300, K=4, E=12, H=256, slot_active_p=0.5), 0),   # per-slot mask
+    ("tiny", dict(W=3, T=300, K=4, E=12, H=256, slot_active_p=0.5), 3),
 ]
 
 
@@ -293,6 +301,60 @@ def test_dispatch_parity_full(md, name, over, q):
         assert (s[:gr] == -1).all() and (s[gr + R:] == -1).all()
     retn, rerc, _ = oracle.moe_recv_counts(w.W, w.E, ref["cnt"], 1)
     assert np.array_equal(etn, retn) and np.array_equal(erc, rerc)
+
+
+SMOOTH_CASES = [
+    (dict(W=2, T=40, K=2, E=4, H=128), 2),
+    (dict(W=2, T=60, K=8, E=16, H=2048, zero_rows=0.05, outlier_frac=0.05), 3),   # 1 warp/token
+    (dict(W=2, T=50, K=4, E=8, H=4096, slot_active_p=0.6), 2),                   # 2 warps, slot mask
+    (dict(W=2, T=40, K=8, E=16, H=7168, outlier_frac=0.05, zero_rows=0.05), 2),  # 4 warps
+    (dict(W=2, T=20, K=16, E=32, H=16384, routing="dup"), 3),                    # 8 warps, K = 16
+    (dict(W=3, T=333, K=3, E=9, H=512, active_p=0.7), 3),
+]
+
+
+@pytest.mark.parametrize("over,q", SMOOTH_CASES)
+def test_dispatch_smoothing_parity(md, over, q):
+    """Per-expert smoothing before the dynamic quantisation: every row's codes and scale
+    bit-exact against the oracle."""
+    w = wl.moe_workload("tiny", seed=35, **over)
+    sm = wl.smooth_scales(w.E, w.H, seed=36)
+    L, st0 = run_layout(md, w)
+    assert st0 == 0
+    ref = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active)
+    full, scales, gr, _, _, st = run_dispatch(md, w, L, q, smooth=sm)
+    assert st == 0
+    R = ref["R"]
+    rex, rsc, fl = oracle.moe_dispatch(w.x_bits, ref["dst_row"], w.K, ref["rows_cap"], q,
+                                       smooth=sm, expert_ids=w.expert_ids)
+    assert fl == 0
+    got = full.cpu().numpy()
+    assert np.array_equal(got[gr:gr + R], rex[:R])
+    assert (got[:gr] == 0x5A).all() and (got[gr + R:] == 0x5A).all()
+    s = scales.cpu().numpy()
+    assert np.array_equal(s[gr:gr + R].view(np.uint32), rsc[:R].view(np.uint32))
+    assert (s[:gr] == -1).all() and (s[gr + R:] == -1).all()
+
+
+def test_dispatch_smoothing_bad_expert_id_is_flagged(md):
+    """A routed slot whose expert id is out of range (the layout was computed from other
+    ids) is skipped with BAD_EXPERT_ID instead of reading outside the smoothing table."""
+    w = wl.moe_workload("tiny", seed=37, W=2, T=30, K=2, E=4, H=256)
+    sm = wl.smooth_scales(w.E, w.H, seed=38)
+    L, _ = run_layout(md, w)
+    bad = w.expert_ids.copy()
+    bad[3, 1] = 99
+    w2 = wl.MoEWorkload(**{**w.__dict__, "expert_ids": bad})
+    full, scales, gr, _, _, st = run_dispatch(md, w2, L, 2, smooth=sm)
+    assert st & md.STATUS_BAD_EXPERT_ID
+    ref = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active)
+    rex, rsc, fl = oracle.moe_dispatch(w.x_bits, ref["dst_row"], w.K, ref["rows_cap"], 2,
+                                       smooth=sm, expert_ids=bad)
+    assert fl & oracle.ORC_BAD_EXPERT
+    skipped = ref["dst_row"][3 * w.K + 1]
+    got = full.cpu().numpy()[gr:gr + ref["R"]]
+    keep = np.arange(ref["R"]) != skipped
+    assert np.array_equal(got[keep], rex[:ref["R"]][keep]) and (got[skipped] == 0x5A).all()
 
 
 @pytest.mark.parametrize("name,q", [("cfg2", 0), ("cfg3", 2), ("cfg4", 3)])
@@ -589,7 +651,9 @@ def test_combine_rmsnorm_full_size_sampled(md, name):
 
 @pytest.mark.parametrize("name,over,q", [("tiny", {}, 0), ("cfg2", {}, 0),
                                          ("tiny", dict(W=4, T=300, K=4, E=16, H=256, active_p=0.8), 2),
-                                         ("tiny", dict(W=4, T=300, K=4, E=16, H=256, active_p=0.8), 3)])
+                                         ("tiny", dict(W=4, T=300, K=4, E=16, H=256, active_p=0.8), 3),
+                                         ("tiny", dict(W=4, T=300, K=4, E=16, H=256, slot_active_p=0.6), 0),
+                                         ("tiny", dict(W=4, T=300, K=4, E=16, H=256, slot_active_p=0.6), 2)])
 def test_dispatch_then_combine(md, name, over, q):
     """Layout -> dispatch -> identity expert -> combine. For bf16 the expert output is
     expand_x itself; for the quant modes the harness dequantises (q * scale, bf16), on
@@ -627,9 +691,14 @@ def test_dispatch_then_combine(md, name, over, q):
     check_combine(yb, eo_ref, ref["dst_row"], w.weights, w.K, L.rows_cap)
     if q == 0:
         xf = wl.bf16_bits_to_f32(w.x_bits).astype(np.float64)
-        act = np.ones(w.G, bool) if w.active is None else w.active.astype(bool)
-        wsum = w.weights.astype(np.float64).sum(axis=1)
-        exp = xf * (wsum * act)[:, None]
+        if w.active is None:
+            act = np.ones((w.G, w.K), bool)
+        elif w.active.ndim == 1:
+            act = np.repeat(w.active.astype(bool)[:, None], w.K, axis=1)
+        else:
+            act = w.active.astype(bool)
+        wsum = (w.weights.astype(np.float64) * act).sum(axis=1)
+        exp = xf * wsum[:, None]
         yf = wl.bf16_bits_to_f32(yb).astype(np.float64)
         assert (np.abs(yf - exp) <= ATOL + RTOL * np.abs(exp)).all()
 
