@@ -150,8 +150,13 @@ def algorithmic_bytes(op, w=None, R=None, a2a=None):
     if op == "layout":
         return G * K * 4 + (0 if w.active is None else G) + 2 * G * K * 4 + R * 4
     if op == "dispatch_smooth":
-        # the dispatch's bytes + the smoothing table (read once at least) + the expert ids
-        return algorithmic_bytes("dispatch", w, R) + w.E * H * 4 + G * K * 4
+        # the dispatch's bytes + the smoothing table, read once
+        return algorithmic_bytes("dispatch", w, R) + w.E * H * 4
+    if op == "dispatch_smooth_gather":
+        # as walked by the row-order kernel: one token row per output row, the rows'
+        # assist_info, the codes and scales, the smoothing table
+        out_elem = 2 if w.quant_mode == 0 else 1
+        return R * H * 2 + R * 4 + R * H * out_elem + R * 4 + w.E * H * 4
     if op == "combine_rmsnorm":
         # expert rows + residual read, residual_out + y written, gamma, routing
         return R * H * 2 + 3 * G * H * 2 + H * 4 + G * K * 8
@@ -508,7 +513,7 @@ def op_sweep(md, torch, device, hbm, reps=10):
             e0, e1 = Ev(enable_timing=True), Ev(enable_timing=True)
             e0.record()
             md.moe_dispatch(st.x, w.H, st.L, w.quant_mode, st.ex, st.scales, st.status,
-                            smooth_scales=sm, expert_ids=st.ids)
+                            smooth_scales=sm)
             e1.record()
             if r >= 3:
                 pairs.append((e0, e1))
@@ -517,9 +522,11 @@ def op_sweep(md, torch, device, hbm, reps=10):
         ms = statistics.mean(a.elapsed_time(b) for a, b in pairs)
         R = int(st.L.expert_base[-1].item())
         b = algorithmic_bytes("dispatch_smooth", w, R)
+        bg = algorithmic_bytes("dispatch_smooth_gather", w, R)
         out.append({"workload": name, "op": "dispatch_smooth", "us": round(ms * 1e3, 2),
                     "bytes": b, "GB/s": round(b / ms / 1e6, 1),
-                    "frac": round(b / ms / 1e6 / hbm, 4)})
+                    "frac": round(b / ms / 1e6 / hbm, 4),
+                    "gather_bytes": bg, "gather_frac": round(bg / ms / 1e6 / hbm, 4)})
         del st, sm
         torch.cuda.empty_cache()
     # raw all-to-all-v, W = 64

@@ -76,7 +76,7 @@ _layout = _sig("moedisp_moe_dispatch_layout",
 _layout_noalloc = _sig("moedisp_moe_dispatch_layout_noalloc",
                        [_P, _P, _I, Dims, ctypes.POINTER(Layout), _P, _P])
 _dispatch = _sig("moedisp_moe_dispatch",
-                 [_P, _I, Dims, ctypes.POINTER(Layout), _I, _P, _P, _P, _P, _P, _I, _P, _P, _P])
+                 [_P, _I, Dims, ctypes.POINTER(Layout), _I, _P, _P, _P, _P, _I, _P, _P, _P])
 _combine = _sig("moedisp_moe_combine", [_P, _I, Dims, ctypes.POINTER(Layout), _P, _P, _P, _P])
 _combine_rms = _sig("moedisp_moe_combine_rmsnorm",
                     [_P, _I, Dims, ctypes.POINTER(Layout), _P, _P, _P, ctypes.c_float, _P, _P, _P, _P])
@@ -236,12 +236,12 @@ def moe_dispatch_layout_noalloc(expert_ids, active_mask, layout: LayoutBuffers, 
 
 def moe_dispatch(x, H, layout: LayoutBuffers, quant_mode, expand_x, dynamic_scales, status,
                  expert_token_nums=None, expert_token_nums_type=1, ep_recv_counts=None,
-                 stream=None, raise_on_error=True, smooth_scales=None, expert_ids=None) -> int:
+                 stream=None, raise_on_error=True, smooth_scales=None) -> int:
     """smooth_scales: fp32 [E, H] per-expert smoothing before quantisation (quantising
-    modes), with the routing's expert_ids [G, K]."""
+    modes)."""
     L = layout.struct()
     rc = _dispatch(_ptr(x), int(H), layout.dims, ctypes.byref(L), int(quant_mode),
-                   _ptr(smooth_scales), _ptr(expert_ids), _ptr(expand_x),
+                   _ptr(smooth_scales), _ptr(expand_x),
                    _ptr(dynamic_scales), _ptr(expert_token_nums), int(expert_token_nums_type),
                    _ptr(ep_recv_counts), _ptr(status), _stream(stream))
     return _check(rc, "moe_dispatch", raise_on_error)

@@ -225,7 +225,7 @@ int moedisp_moe_dispatch_layout_noalloc(const int32_t* expert_ids, const uint8_t
 
 int moedisp_moe_dispatch(const void* x, int H, moedisp_dims dims,
                          const moedisp_layout* layout, int quant_mode,
-                         const float* smooth_scales, const int32_t* expert_ids, void* expand_x,
+                         const float* smooth_scales, void* expand_x,
                          float* dynamic_scales, int64_t* expert_token_nums,
                          int expert_token_nums_type, int32_t* ep_recv_counts,
                          int32_t* status, moedisp_stream_t stream) {
@@ -246,7 +246,8 @@ int moedisp_moe_dispatch(const void* x, int H, moedisp_dims dims,
     const int64_t G = (int64_t)dims.W * dims.T;
     const int64_t slots = G * dims.K;
     if (G > 0 && (!x || !L.dst_row)) return MOEDISP_ERR_NULLPTR;
-    if (G > 0 && smooth_scales && !expert_ids) return MOEDISP_ERR_NULLPTR;
+    if (smooth_scales && L.rows_cap > 0 && (!L.assist_info || !L.expert_base))
+        return MOEDISP_ERR_NULLPTR;
     if (L.rows_cap > 0 && !expand_x) return MOEDISP_ERR_NULLPTR;
     if (quant_mode != MOEDISP_QUANT_NONE && L.rows_cap > 0 && !dynamic_scales)
         return MOEDISP_ERR_NULLPTR;
@@ -255,7 +256,7 @@ int moedisp_moe_dispatch(const void* x, int H, moedisp_dims dims,
     if (!aligned(x, 16) || !aligned(expand_x, 16) || !aligned(L.dst_row, 4) ||
         !aligned(dynamic_scales, 4) || !aligned(expert_token_nums, 8) ||
         !aligned(ep_recv_counts, 4) || !aligned(status, 4) || !aligned(smooth_scales, 16) ||
-        !aligned(expert_ids, 4))
+        !aligned(L.assist_info, 4) || !aligned(L.expert_base, 8))
         return MOEDISP_ERR_MISALIGNED;
     const size_t out_row = quant_mode == MOEDISP_QUANT_NONE ? (size_t)H * 2 : (size_t)H;
     const int ne = dims.E / dims.W;
@@ -269,13 +270,13 @@ int moedisp_moe_dispatch(const void* x, int H, moedisp_dims dims,
                   {{x, (size_t)G * H * 2},
                    {L.dst_row, (size_t)slots * 4},
                    {smooth_scales, (size_t)dims.E * H * 4},
-                   {smooth_scales ? expert_ids : nullptr, (size_t)slots * 4},
+                   {smooth_scales ? L.assist_info : nullptr, (size_t)L.rows_cap * 4},
                    {L.cnt, (size_t)dims.W * dims.E * 4},
                    {L.expert_base, (size_t)(dims.E + 1) * 8},
                    {L.rank_base, (size_t)(dims.W + 1) * 8}}))
         return MOEDISP_ERR_ALIASED;
-    return rc(moedisp::launch_dispatch(x, H, dims, L, quant_mode, smooth_scales,
-                                       smooth_scales ? expert_ids : nullptr, expand_x, dynamic_scales,
+    return rc(moedisp::launch_dispatch(x, H, dims, L, quant_mode, smooth_scales, expand_x,
+                                       dynamic_scales,
                                        expert_token_nums, expert_token_nums_type, ep_recv_counts,
                                        status, stream));
 }

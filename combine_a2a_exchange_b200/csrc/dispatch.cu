@@ -28,7 +28,7 @@ struct DispatchArgs {
     uint8_t* expand_x;
     float* scales;
     const float* smooth;       // [E][H] per-expert smoothing (quantising modes) or null
-    const int32_t* ids;        // [G][K] expert ids, with smooth
+    const int32_t* assist;     // [rows_cap] slot of each row (the smoothing kernel)
     int stages;
     uint32_t in_bytes, out_bytes;
     // receive counts (optional)
@@ -68,20 +68,21 @@ __device__ __forceinline__ float absmax8(const uint4& v) {
 
 // int8 boundaries are the half-integers; |x/scale| <= ~127, so the bound above is below
 // 2.3e-5 and a margin of 2^-14 from k + 0.5 is safe. Rounding to an integer uses the
-// floating-point adder: for |v| < 2^22, v + 1.5*2^23 rounds v's fraction away to the
-// nearest integer, ties to even, and the integer is read back from the sum's low bits.
-__device__ __forceinline__ int q_int8(float x, float scale, float inv) {
+// floating-point adder: for |v| < 2^22, rr = v + 1.5*2^23 rounds v's fraction away to the
+// nearest integer, ties to even, and rr's bit pattern is that of 1.5*2^23 plus the integer,
+// whose low byte is therefore the integer's two's-complement low byte -- the int8 code.
+// The clamp to +-127 can only act when the scale itself is inexact far beyond fp32's
+// rounding (subnormal scales); the fast path is taken only for |r| < 127.5, where it
+// cannot act, and the slow path clamps. Returns a word whose low byte is the code.
+__device__ __forceinline__ uint32_t q_int8(float x, float scale, float inv) {
     constexpr float kMagic = 12582912.0f;                    // 1.5 * 2^23
-    float v = __fmul_rn(x, inv);
-    float rr = __fadd_rn(v, kMagic);
+    const float v = __fmul_rn(x, inv);
+    const float rr = __fadd_rn(v, kMagic);
     const float t = __fsub_rn(v, __fsub_rn(rr, kMagic));      // v - round(v), in [-0.5, 0.5]
-    if (!(0.5f - fabsf(t) >= 0.00006103515625f)) {            // near k + 0.5, or not finite
-        v = __fdiv_rn(x, scale);
-        if (!(fabsf(v) < 4194304.0f)) return v > 0.0f ? 127 : -127;   // |v| >= 2^22 or NaN
-        rr = __fadd_rn(v, kMagic);
-    }
-    const int q = (int)(__float_as_uint(rr) - __float_as_uint(kMagic));
-    return max(-127, min(127, q));
+    if (0.5f - fabsf(t) >= 0.00006103515625f && fabsf(v) < 127.5f) return __float_as_uint(rr);
+    // near k + 0.5, out of range or not finite: the IEEE quotient, clamped (NaN -> -127)
+    const float q = fminf(fmaxf(__fdiv_rn(x, scale), -127.0f), 127.0f);
+    return __float_as_uint(__fadd_rn(q, kMagic));
 }
 
 // E4M3 keeps 3 mantissa bits: for 2^-6 <= |v| < 448 its rounding boundaries are the fp32
@@ -90,7 +91,8 @@ __device__ __forceinline__ int q_int8(float x, float scale, float inv) {
 // truncating: the code is sign | ((bits + 0x80000) >> 20) - ((127 - 7) << 3), the carry
 // moving into the exponent when the mantissa rounds up. Elsewhere (near a boundary, in
 // E4M3's subnormal range, at the saturation edge, not finite) the IEEE quotient goes
-// through the hardware conversion (round to nearest even, saturating to +-448).
+// through the hardware conversion (round to nearest even, saturating to +-448). Returns a
+// word whose low byte is the code.
 __device__ __forceinline__ uint32_t q_e4m3(float x, float scale, float inv) {
     const float r = __fmul_rn(x, inv);
     const uint32_t b = __float_as_uint(r);
@@ -99,17 +101,17 @@ __device__ __forceinline__ uint32_t q_e4m3(float x, float scale, float inv) {
     if (u - 0x3c800000u < 0x43e00000u - 0x3c800000u && (u & 0xfffffu) - 0x7fff0u > 32u)
         return ((b >> 24) & 0x80u) | (((u + 0x80000u) >> 20) - 0x3c0u);
     const float v = __fdiv_rn(x, scale);
-    return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(v, 0.0f), __NV_SATFINITE, __NV_E4M3) & 0xffu;
+    return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(v, 0.0f), __NV_SATFINITE, __NV_E4M3);
 }
 
-__device__ __forceinline__ uint32_t q_int8_pair(uint32_t w, float scale, float inv) {
-    const int a = q_int8(bf16_lo(w), scale, inv);
-    const int b = q_int8(bf16_hi(w), scale, inv);
-    return (uint32_t)(a & 0xff) | ((uint32_t)(b & 0xff) << 8);
+template <int Q>
+__device__ __forceinline__ uint32_t q_code(float x, float scale, float inv) {
+    return Q == MOEDISP_QUANT_INT8 ? q_int8(x, scale, inv) : q_e4m3(x, scale, inv);
 }
 
-__device__ __forceinline__ uint32_t q_e4m3_pair(uint32_t w, float scale, float inv) {
-    return q_e4m3(bf16_lo(w), scale, inv) | (q_e4m3(bf16_hi(w), scale, inv) << 8);
+// The low bytes of four words, in order, in one word (three byte permutes).
+__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
 
 // Eight fp32 values (a smoothed row chunk) to eight codes.
@@ -118,35 +120,31 @@ __device__ __forceinline__ uint2 quant8f(const float (&v)[8], float scale, float
     if (zero) return make_uint2(0u, 0u);
     uint32_t b[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-        b[j] = Q == MOEDISP_QUANT_INT8 ? (uint32_t)(q_int8(v[j], scale, inv) & 0xff)
-                                       : q_e4m3(v[j], scale, inv);
-    return make_uint2(b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24),
-                      b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24));
+    for (int j = 0; j < 8; ++j) b[j] = q_code<Q>(v[j], scale, inv);
+    return make_uint2(pack_low_bytes(b[0], b[1], b[2], b[3]), pack_low_bytes(b[4], b[5], b[6], b[7]));
 }
 
-// x chunk (8 bf16) times a smoothing chunk (8 fp32), one correctly rounded product each.
-__device__ __forceinline__ void smooth8(const uint4& v, const float* s, float (&o)[8]) {
-    const float4 s0 = __ldg(reinterpret_cast<const float4*>(s));
-    const float4 s1 = __ldg(reinterpret_cast<const float4*>(s) + 1);
+// x chunk (8 bf16) times a smoothing chunk (8 fp32, shared memory), one correctly rounded
+// product each.
+__device__ __forceinline__ void smooth8(const uint4& v, const float4* s, float (&o)[8]) {
+    const float4 s0 = s[0];
+    const float4 s1 = s[1];
     o[0] = __fmul_rn(bf16_lo(v.x), s0.x); o[1] = __fmul_rn(bf16_hi(v.x), s0.y);
     o[2] = __fmul_rn(bf16_lo(v.y), s0.z); o[3] = __fmul_rn(bf16_hi(v.y), s0.w);
     o[4] = __fmul_rn(bf16_lo(v.z), s1.x); o[5] = __fmul_rn(bf16_hi(v.z), s1.y);
     o[6] = __fmul_rn(bf16_lo(v.w), s1.z); o[7] = __fmul_rn(bf16_hi(v.w), s1.w);
 }
 
+// Eight bf16 values (a row chunk) to eight codes.
 template <int Q>
 __device__ __forceinline__ uint2 quant8(const uint4& v, float scale, float inv, bool zero) {
     if (zero) return make_uint2(0u, 0u);
-    uint32_t p0, p1, p2, p3;
-    if (Q == MOEDISP_QUANT_INT8) {
-        p0 = q_int8_pair(v.x, scale, inv); p1 = q_int8_pair(v.y, scale, inv);
-        p2 = q_int8_pair(v.z, scale, inv); p3 = q_int8_pair(v.w, scale, inv);
-    } else {
-        p0 = q_e4m3_pair(v.x, scale, inv); p1 = q_e4m3_pair(v.y, scale, inv);
-        p2 = q_e4m3_pair(v.z, scale, inv); p3 = q_e4m3_pair(v.w, scale, inv);
-    }
-    return make_uint2(p0 | (p1 << 16), p2 | (p3 << 16));
+    const float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                        bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+    uint32_t b[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) b[j] = q_code<Q>(f[j], scale, inv);
+    return make_uint2(pack_low_bytes(b[0], b[1], b[2], b[3]), pack_low_bytes(b[4], b[5], b[6], b[7]));
 }
 
 __device__ void write_recv_counts(const DispatchArgs& a) {
@@ -285,23 +283,16 @@ __device__ __forceinline__ void group_barrier(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-//
-// With per-expert smoothing (SM), the copy for slot k is x * smooth[e_k] quantised on its
-// own: the group reduces K maxima of |x * smooth[e_k]| in one pass over the row, then
-// recomputes the products chunk by chunk (the smoothing rows come from L2) and stores
-// each slot's codes and scale.
-template <int Q, int WPT, bool SM>
+template <int Q, int WPT>
 __global__ void __launch_bounds__(kQuantThreads, 2) dispatch_quant_kernel(DispatchArgs a) {
     constexpr int NG = kQuantThreads / 32 / WPT;     // token groups per block
     constexpr int GT = WPT * 32;                     // threads per group
-    constexpr int KS = SM ? MOEDISP_MAX_K : 1;       // maxima reduced per token
     constexpr float kQmax = Q == MOEDISP_QUANT_INT8 ? 127.0f : 448.0f;
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t bars[NG][kMaxStages];
     __shared__ int64_t tok[NG][kMaxStages];
     __shared__ int32_t drow[NG][kMaxStages][MOEDISP_MAX_K];
-    __shared__ int32_t dexp[NG][kMaxStages][KS];     // expert of each slot (SM)
-    __shared__ float red[NG][2][KS][WPT];
+    __shared__ float red[NG][2][WPT];
     __shared__ int abort_s[NG];
     __shared__ unsigned next_s;                      // the block's next token index
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -315,7 +306,6 @@ __global__ void __launch_bounds__(kQuantThreads, 2) dispatch_quant_kernel(Dispat
         fence_mbar_init();
         abort_s[grp] = 0;
     }
-    if (SM && gt < S * KS) dexp[grp][gt / KS][gt % KS] = 0;   // always a valid expert id
     if (tid == 0) next_s = 0;
     __syncthreads();
     // L2 prefetch of the block's first NG * S token rows (see dispatch_copy_kernel).
@@ -338,24 +328,18 @@ __global__ void __launch_bounds__(kQuantThreads, 2) dispatch_quant_kernel(Dispat
         return (int64_t)blockIdx.x + (int64_t)i * gridDim.x;
     };
     int64_t pf_g = 0;
-    int32_t pf_d = -1, pf_e = 0;
-    auto load_routing = [&]() {
-        const bool mine = pf_g < a.G && lane < K;
-        pf_d = mine ? __ldg(a.dst_row + pf_g * K + lane) : -1;
-        if (SM) pf_e = mine ? __ldg(a.ids + pf_g * K + lane) : 0;
-    };
+    int32_t pf_d = -1;
     if (gw == 0) {
         pf_g = next_token();
-        load_routing();
+        pf_d = (pf_g < a.G && lane < K) ? __ldg(a.dst_row + pf_g * K + lane) : -1;
     }
     auto fill = [&](int st) {
         while (true) {
             const int64_t g = pf_g;
             int32_t d = pf_d;
-            const int32_t e = pf_e;
             if (g < a.G) {
                 pf_g = next_token();
-                load_routing();
+                pf_d = (pf_g < a.G && lane < K) ? __ldg(a.dst_row + pf_g * K + lane) : -1;
             }
             if (g >= a.G) {
                 if (lane == 0) {
@@ -368,24 +352,11 @@ __global__ void __launch_bounds__(kQuantThreads, 2) dispatch_quant_kernel(Dispat
                 raise_status(a.status, MOEDISP_STATUS_CAPACITY);
                 d = -1;
             }
-            if (SM && d >= 0 && (e < 0 || e >= a.E)) {
-                raise_status(a.status, MOEDISP_STATUS_BAD_EXPERT_ID);
-                d = -1;
-            }
             if (d < 0) d = -1;
             if (__ballot_sync(0xffffffffu, d >= 0)) {
                 int32_t dk[MOEDISP_MAX_K];
 #pragma unroll
                 for (int k = 0; k < MOEDISP_MAX_K; ++k) dk[k] = __shfl_sync(0xffffffffu, d, k);
-                if (SM) {
-                    // lane 0 publishes the slots' experts with the rows (its barrier arrival
-                    // releases its own writes)
-#pragma unroll
-                    for (int k = 0; k < KS; ++k) {
-                        const int32_t ek = __shfl_sync(0xffffffffu, e, k);
-                        if (lane == 0 && k < K && dk[k] >= 0) dexp[grp][st][k] = ek;
-                    }
-                }
                 if (lane == 0) {
 #pragma unroll
                     for (int k = 0; k < MOEDISP_MAX_K; ++k)
@@ -412,48 +383,15 @@ __global__ void __launch_bounds__(kQuantThreads, 2) dispatch_quant_kernel(Dispat
 #pragma unroll
         for (int k = 0; k < MOEDISP_MAX_K; ++k) d[k] = k < K ? drow[grp][st][k] : -1;
         const uint4* row = reinterpret_cast<const uint4*>(inbuf + (size_t)st * a.in_bytes);
-        // Row maxima: of |x| (one), or of |x * smooth[e_k]| per slot (SM). Expert ids in
-        // dexp are always in [0, E), even in a stage whose token is stale.
-        float m[KS];
-        int32_t ex[KS];
+        float m = 0.0f;
+        for (int c = gt; c < nvec; c += GT) m = fmaxf(m, absmax8(row[c]));
 #pragma unroll
-        for (int k = 0; k < KS; ++k) {
-            m[k] = 0.0f;
-            ex[k] = SM ? dexp[grp][st][k] : 0;
-        }
-        for (int c = gt; c < nvec; c += GT) {
-            const uint4 v = row[c];
-            if (SM) {
-#pragma unroll
-                for (int k = 0; k < KS; ++k) {
-                    if (k < K && d[k] >= 0) {
-                        float xs[8];
-                        smooth8(v, a.smooth + (int64_t)ex[k] * a.H + 8 * c, xs);
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) m[k] = fmaxf(m[k], fabsf(xs[j]));
-                    }
-                }
-            } else {
-                m[0] = fmaxf(m[0], absmax8(v));
-            }
-        }
-#pragma unroll
-        for (int k = 0; k < KS; ++k) {
-            if (k < (SM ? K : 1)) {
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) m[k] = fmaxf(m[k], __shfl_xor_sync(0xffffffffu, m[k], o));
-            }
-        }
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         if (WPT > 1) {
-            if (lane == 0) {
-#pragma unroll
-                for (int k = 0; k < KS; ++k) red[grp][it & 1][k][gw] = m[k];
-            }
+            if (lane == 0) red[grp][it & 1][gw] = m;
             group_barrier(1 + grp, GT);
 #pragma unroll
-            for (int k = 0; k < KS; ++k)
-#pragma unroll
-                for (int w = 0; w < WPT; ++w) m[k] = fmaxf(m[k], red[grp][it & 1][k][w]);
+            for (int w = 0; w < WPT; ++w) m = fmaxf(m, red[grp][it & 1][w]);
         } else {
             __syncwarp();
         }
@@ -464,34 +402,9 @@ __global__ void __launch_bounds__(kQuantThreads, 2) dispatch_quant_kernel(Dispat
         // Every thread of the group is past the previous token: its stage is free.
         if (gw == 0 && it >= 1) fill((it - 1) % S);
         if (g < 0) break;
-        if (SM) {
-            float sc[KS], iv[KS];
-#pragma unroll
-            for (int k = 0; k < KS; ++k) {
-                sc[k] = __fdiv_rn(m[k], kQmax);
-                iv[k] = __frcp_rn(sc[k]);
-            }
-            for (int c = gt; c < nvec; c += GT) {
-                const uint4 v = row[c];
-#pragma unroll
-                for (int k = 0; k < KS; ++k) {
-                    if (k < K && d[k] >= 0) {
-                        float xs[8];
-                        smooth8(v, a.smooth + (int64_t)ex[k] * a.H + 8 * c, xs);
-                        __stcs(reinterpret_cast<uint2*>(a.expand_x + (int64_t)d[k] * a.out_bytes) + c,
-                               quant8f<Q>(xs, sc[k], iv[k], m[k] == 0.0f));
-                    }
-                }
-            }
-#pragma unroll
-            for (int k = 0; k < KS; ++k)
-                if (gt == k && k < K && d[k] >= 0) a.scales[d[k]] = sc[k];
-            continue;
-        }
-        const float m0 = m[0];
-        const float scale = __fdiv_rn(m0, kQmax);
+        const float scale = __fdiv_rn(m, kQmax);
         const float inv = __frcp_rn(scale);
-        const bool zero = m0 == 0.0f;
+        const bool zero = m == 0.0f;
         if (K <= 8) {                          // row bases once per token, 8-way stores
             uint2* dst[8];
 #pragma unroll
@@ -520,6 +433,107 @@ __global__ void __launch_bounds__(kQuantThreads, 2) dispatch_quant_kernel(Dispat
     }
 }
 
+// Quantising dispatch with per-expert smoothing. The copy of token g for expert e is
+// x[g] * smooth[e] quantised on its own, so the work is per row of expand_x, not per
+// token, and it is arithmetic-heavy (a product, a maximum and a quantisation per output
+// element). Rows are taken in their own order (grouped by expert): a block takes chunks of
+// consecutive rows; for each expert segment of a chunk it copies smooth[e] into shared
+// memory once, and its token groups (WPT warps each) share the segment's rows. A group
+// gathers its row's token x[assist_info[row] / K] straight into registers (CPT 16-byte
+// chunks per thread, all loads issued before the first use), reduces max |x * smooth[e]|
+// (shuffles, plus a named barrier across the group's warps), and stores the codes (8
+// bytes per chunk, coalesced) and the row's scale. No staging buffers, so many warps fit
+// an SM; the smoothing table is read about once; nothing waits on another block.
+template <int Q, int WPT, int CPT>
+__global__ void __launch_bounds__(kQuantThreads, CPT > 4 ? 2 : 4) dispatch_smooth_kernel(DispatchArgs a) {
+    constexpr int NG = kQuantThreads / 32 / WPT;     // groups per block
+    constexpr int GT = WPT * 32;                     // threads per group
+    constexpr float kQmax = Q == MOEDISP_QUANT_INT8 ? 127.0f : 448.0f;
+    extern __shared__ __align__(16) float4 sbuf[];   // [H / 4]: smooth[e]
+    __shared__ float red[NG][2][WPT];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int grp = warp / WPT, gw = warp - grp * WPT, gt = tid - grp * GT;
+    grid_dep_wait();
+    grid_dep_launch_dependents();
+    write_recv_counts(a);
+
+    const int64_t r_all = a.expert_base[a.E];
+    if (blockIdx.x == 0 && tid == 0 && r_all > a.rows_cap)
+        raise_status(a.status, MOEDISP_STATUS_CAPACITY);
+    const int64_t R = min64(r_all, a.rows_cap);
+    const int64_t RC = max64(64, (R + 4 * (int64_t)gridDim.x - 1) / (4 * (int64_t)gridDim.x));
+    const int nvec = a.H >> 3, n4 = a.H >> 2;
+    const int64_t slots = a.G * a.K;
+    const uint4* x4 = reinterpret_cast<const uint4*>(a.x);
+    int parity = 0;
+
+    for (int64_t ch = blockIdx.x; ch * RC < R; ch += gridDim.x) {
+        int64_t r = ch * RC;
+        const int64_t end = min64(R, r + RC);
+        int lo = 0, hi = a.E;                       // expert_base[lo] <= r < expert_base[hi]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (a.expert_base[mid] <= r) lo = mid; else hi = mid;
+        }
+        for (int e = lo; r < end; ++e) {
+            const int64_t seg_end = min64(end, a.expert_base[e + 1]);
+            if (seg_end <= r) continue;
+            __syncthreads();                        // every group is done with the last row
+            const float4* src = reinterpret_cast<const float4*>(a.smooth + (int64_t)e * a.H);
+            for (int i = tid; i < n4; i += kQuantThreads) sbuf[i] = __ldg(src + i);
+            __syncthreads();
+            for (int64_t row = r + grp; row < seg_end; row += NG) {
+                const int32_t slot = __ldg(a.assist + row);          // same for the group
+                if (slot < 0 || (int64_t)slot >= slots) {
+                    if (gt == 0) raise_status(a.status, MOEDISP_STATUS_BAD_EXPERT_ID);
+                    continue;
+                }
+                const uint4* xr = x4 + (int64_t)(slot / a.K) * nvec;
+                uint4 v[CPT];
+#pragma unroll
+                for (int j = 0; j < CPT; ++j) {
+                    const int c = gt + j * GT;
+                    v[j] = c < nvec ? __ldg(xr + c) : make_uint4(0u, 0u, 0u, 0u);
+                }
+                float m = 0.0f;
+#pragma unroll
+                for (int j = 0; j < CPT; ++j) {
+                    const int c = gt + j * GT;
+                    if (c < nvec) {
+                        float xs[8];
+                        smooth8(v[j], sbuf + 2 * c, xs);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) m = fmaxf(m, fabsf(xs[q]));
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                if (WPT > 1) {
+                    if (lane == 0) red[grp][parity][gw] = m;
+                    group_barrier(1 + grp, GT);
+#pragma unroll
+                    for (int w = 0; w < WPT; ++w) m = fmaxf(m, red[grp][parity][w]);
+                    parity ^= 1;
+                }
+                const float scale = __fdiv_rn(m, kQmax);
+                const float inv = __frcp_rn(scale);
+                uint2* dst = reinterpret_cast<uint2*>(a.expand_x + row * a.out_bytes);
+#pragma unroll
+                for (int j = 0; j < CPT; ++j) {
+                    const int c = gt + j * GT;
+                    if (c < nvec) {
+                        float xs[8];
+                        smooth8(v[j], sbuf + 2 * c, xs);
+                        __stcs(dst + c, quant8f<Q>(xs, scale, inv, m == 0.0f));
+                    }
+                }
+                if (gt == 0) a.scales[row] = scale;
+            }
+            r = seg_end;
+        }
+    }
+}
+
 cudaError_t launch_copy(DispatchArgs a, cudaStream_t stream) {
     // Few tokens per block keep the pipeline's serial start short: use the fewest stages
     // (2, 4 or 8) with which one wave of resident blocks gives each block at most about
@@ -544,7 +558,7 @@ cudaError_t launch_copy(DispatchArgs a, cudaStream_t stream) {
                       1, a);
 }
 
-template <int Q, int WPT, bool SM>
+template <int Q, int WPT>
 cudaError_t launch_quant_w(DispatchArgs a, cudaStream_t stream) {
     constexpr int NG = kQuantThreads / 32 / WPT;
     // Stages per group: two for single-warp groups (small rows: more blocks per SM pays
@@ -552,35 +566,58 @@ cudaError_t launch_quant_w(DispatchArgs a, cudaStream_t stream) {
     a.stages = WPT == 1 ? 2 : 3;
     const size_t smem = (size_t)NG * a.stages * a.in_bytes;
     int per_sm = 1;
-    cudaError_t err = blocks_per_sm((const void*)dispatch_quant_kernel<Q, WPT, SM>, kQuantThreads,
+    cudaError_t err = blocks_per_sm((const void*)dispatch_quant_kernel<Q, WPT>, kQuantThreads,
                                     smem, &per_sm);
     if (err != cudaSuccess) return err;
     int64_t grid = (int64_t)current_sm_count() * per_sm;
     grid = std::min<int64_t>(grid, std::max<int64_t>((a.G + NG - 1) / NG, 1));
-    return launch_pdl(dispatch_quant_kernel<Q, WPT, SM>, dim3((unsigned)grid), dim3(kQuantThreads),
+    return launch_pdl(dispatch_quant_kernel<Q, WPT>, dim3((unsigned)grid), dim3(kQuantThreads),
                       smem, stream, 1, a);
 }
 
 // Warps per token: the fewest that hold a row in kChunks 16-byte chunks per thread.
-template <int Q, bool SM>
-cudaError_t launch_quant_s(const DispatchArgs& a, cudaStream_t stream) {
+// Smoothing kernel geometry: CPT chunks of the row per thread and WPT warps per row: the
+// fewest chunks per thread up to four (registers, hence warps per SM, matter most here),
+// then eight for the widest rows.
+template <int Q, int WPT, int CPT>
+cudaError_t launch_smooth_w(DispatchArgs a, cudaStream_t stream) {
+    const size_t smem = (size_t)a.H * 4;
+    int per_sm = 1;
+    cudaError_t err = blocks_per_sm((const void*)dispatch_smooth_kernel<Q, WPT, CPT>, kQuantThreads,
+                                    smem, &per_sm);
+    if (err != cudaSuccess) return err;
+    const int64_t grid = (int64_t)current_sm_count() * per_sm;
+    return launch_pdl(dispatch_smooth_kernel<Q, WPT, CPT>, dim3((unsigned)grid),
+                      dim3(kQuantThreads), smem, stream, 1, a);
+}
+
+template <int Q>
+cudaError_t launch_smooth(const DispatchArgs& a, cudaStream_t stream) {
     const int nvec = a.H / 8;
-    if (nvec <= 1 * 32 * kChunks) return launch_quant_w<Q, 1, SM>(a, stream);
-    if (nvec <= 2 * 32 * kChunks) return launch_quant_w<Q, 2, SM>(a, stream);
-    if (nvec <= 4 * 32 * kChunks) return launch_quant_w<Q, 4, SM>(a, stream);
-    return launch_quant_w<Q, 8, SM>(a, stream);
+    if (nvec <= 32) return launch_smooth_w<Q, 1, 1>(a, stream);
+    if (nvec <= 64) return launch_smooth_w<Q, 1, 2>(a, stream);
+    if (nvec <= 128) return launch_smooth_w<Q, 1, 4>(a, stream);
+    if (nvec <= 256) return launch_smooth_w<Q, 2, 4>(a, stream);
+    if (nvec <= 512) return launch_smooth_w<Q, 4, 4>(a, stream);
+    if (nvec <= 1024) return launch_smooth_w<Q, 8, 4>(a, stream);
+    return launch_smooth_w<Q, 8, 8>(a, stream);
 }
 
 template <int Q>
 cudaError_t launch_quant(const DispatchArgs& a, cudaStream_t stream) {
-    return a.smooth != nullptr ? launch_quant_s<Q, true>(a, stream) : launch_quant_s<Q, false>(a, stream);
+    if (a.smooth != nullptr) return launch_smooth<Q>(a, stream);
+    const int nvec = a.H / 8;
+    if (nvec <= 1 * 32 * kChunks) return launch_quant_w<Q, 1>(a, stream);
+    if (nvec <= 2 * 32 * kChunks) return launch_quant_w<Q, 2>(a, stream);
+    if (nvec <= 4 * 32 * kChunks) return launch_quant_w<Q, 4>(a, stream);
+    return launch_quant_w<Q, 8>(a, stream);
 }
 
 }  // namespace
 
 cudaError_t launch_dispatch(const void* x, int H, const moedisp_dims& dims,
                             const moedisp_layout& L, int quant_mode, const float* smooth_scales,
-                            const int32_t* expert_ids, void* expand_x,
+                            void* expand_x,
                             float* dynamic_scales, int64_t* expert_token_nums,
                             int expert_token_nums_type, int32_t* ep_recv_counts,
                             int32_t* status, cudaStream_t stream) {
@@ -594,7 +631,7 @@ cudaError_t launch_dispatch(const void* x, int H, const moedisp_dims& dims,
     a.expand_x = static_cast<uint8_t*>(expand_x);
     a.scales = dynamic_scales;
     a.smooth = smooth_scales;
-    a.ids = expert_ids;
+    a.assist = L.assist_info;
     a.stages = 2;
     a.in_bytes = (uint32_t)H * 2u;
     a.out_bytes = quant_mode == MOEDISP_QUANT_NONE ? (uint32_t)H * 2u : (uint32_t)H;

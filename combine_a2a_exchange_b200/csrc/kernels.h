@@ -84,7 +84,7 @@ cudaError_t launch_bounded_wait_selftest(uint64_t limit_ns, int32_t* status, cud
 
 cudaError_t launch_dispatch(const void* x, int H, const moedisp_dims& dims,
                             const moedisp_layout& layout, int quant_mode,
-                            const float* smooth_scales, const int32_t* expert_ids, void* expand_x,
+                            const float* smooth_scales, void* expand_x,
                             float* dynamic_scales, int64_t* expert_token_nums,
                             int expert_token_nums_type, int32_t* ep_recv_counts,
                             int32_t* status, cudaStream_t stream);

@@ -225,10 +225,11 @@ int moedisp_moe_dispatch_layout_noalloc(const int32_t *expert_ids, const uint8_t
  *   dynamic_scales[dst_row[s]] = scale (quant modes).
  * smooth_scales (Ascend scalesOptional, the per-expert quantisation smoothing factors):
  * fp32 [E][H] device, 16-byte aligned, or NULL; quant modes only (with NONE it is
- * MOEDISP_ERR_INVALID). When given, the copy for slot s = (g, k) with expert
- * e = expert_ids[s] quantises x[g] * smooth_scales[e] (one fp32 product per element)
- * instead of x[g], with its own a and scale; expert_ids (int32 [G][K] device, the layout's
- * input) is then required, and is ignored otherwise.
+ * MOEDISP_ERR_INVALID). When given, the copy for slot s = (g, k) routed to expert e
+ * quantises x[g] * smooth_scales[e] (one fp32 product per element) instead of x[g], with
+ * its own a and scale. The rows are then produced in expand_x order from the layout's
+ * expert_base and assist_info (a row whose assist_info is outside [0, G*K) is skipped and
+ * sets MOEDISP_STATUS_BAD_EXPERT_ID); dst_row is not read.
  * x: bf16 [G][H] device, 16-byte aligned; expand_x: [layout->rows_cap][H] elements of
  * the output type, 16-byte aligned, not overlapping x; dynamic_scales: fp32
  * [rows_cap] (required for quant modes, ignored otherwise). H % 8 == 0 (NONE) or
@@ -238,12 +239,14 @@ int moedisp_moe_dispatch_layout_noalloc(const int32_t *expert_ids, const uint8_t
  *     over the rank's local experts up to and including le (type 0);
  *   ep_recv_counts int32 [W][ne][W]: rows expert d*ne+le receives from source rank r.
  * Rows at or beyond rows_cap are not written (MOEDISP_STATUS_CAPACITY).
- * One persistent kernel: each token row is brought into shared memory once by a bulk
- * (TMA) copy; unquantised rows leave it as K bulk copies, quantised ones as 8-byte
- * streaming stores of the codes to the K rows. */
+ * One persistent kernel: without smoothing each token row is brought into shared memory
+ * once by a bulk (TMA) copy; unquantised rows leave it as K bulk copies, quantised ones as
+ * 8-byte streaming stores of the codes to the K rows. With smoothing each block walks
+ * runs of consecutive rows, holding one expert's smoothing row in shared memory and
+ * gathering the rows' tokens by bulk copies. */
 int moedisp_moe_dispatch(const void *x, int H, moedisp_dims dims,
                          const moedisp_layout *layout, int quant_mode,
-                         const float *smooth_scales, const int32_t *expert_ids, void *expand_x,
+                         const float *smooth_scales, void *expand_x,
                          float *dynamic_scales, int64_t *expert_token_nums,
                          int expert_token_nums_type, int32_t *ep_recv_counts,
                          int32_t *status, moedisp_stream_t stream);

@@ -141,8 +141,8 @@ def test_dispatch_and_combine_rejections(md):
     L = _layout(md)
     d = md.Dims(4, 8, 2, 8)
     x, ex, sc, st = FAKE + (64 << 20), FAKE + (128 << 20), FAKE + (192 << 20), FAKE + (256 << 20)
-    disp = lambda x, H, q, ex, sc, st, etn=None, t=1, sm=None, ids=None: md.raw_call(
-        "moedisp_moe_dispatch", x, H, d, ctypes.byref(L), q, sm, ids, ex, sc, etn, t, None, st, None)
+    disp = lambda x, H, q, ex, sc, st, etn=None, t=1, sm=None, lay=None: md.raw_call(
+        "moedisp_moe_dispatch", x, H, d, ctypes.byref(lay or L), q, sm, ex, sc, etn, t, None, st, None)
     assert disp(x, 128, 1, ex, sc, st) == md.MOEDISP_ERR_INVALID           # quant mode
     assert disp(x, 120, 2, ex, sc, st) == md.MOEDISP_ERR_MISALIGNED        # H % 16 (quant)
     assert disp(x, 124, 0, ex, sc, st) == md.MOEDISP_ERR_MISALIGNED        # H % 8
@@ -153,12 +153,12 @@ def test_dispatch_and_combine_rejections(md):
     assert disp(x + 8, 128, 0, ex, None, st) == md.MOEDISP_ERR_MISALIGNED
     assert disp(x, 128, 0, ex, None, None) == md.MOEDISP_ERR_NULLPTR
     assert disp(x, 128, 0, ex, None, st, etn=FAKE + (300 << 20), t=5) == md.MOEDISP_ERR_INVALID
-    sm, ids = FAKE + (320 << 20), FAKE + (384 << 20)
-    assert disp(x, 128, 0, ex, None, st, sm=sm, ids=ids) == md.MOEDISP_ERR_INVALID  # smoothing, no quant
-    assert disp(x, 128, 2, ex, sc, st, sm=sm) == md.MOEDISP_ERR_NULLPTR             # no expert ids
-    assert disp(x, 128, 2, ex, sc, st, sm=sm + 4, ids=ids) == md.MOEDISP_ERR_MISALIGNED
-    assert disp(x, 128, 2, ex, sc, st, sm=sm, ids=ids + 2) == md.MOEDISP_ERR_MISALIGNED
-    assert disp(x, 128, 2, sm + 256, sc, st, sm=sm, ids=ids) == md.MOEDISP_ERR_ALIASED  # out over smooth
+    sm = FAKE + (320 << 20)
+    assert disp(x, 128, 0, ex, None, st, sm=sm) == md.MOEDISP_ERR_INVALID   # smoothing, no quant
+    assert disp(x, 128, 2, ex, sc, st, sm=sm + 4) == md.MOEDISP_ERR_MISALIGNED
+    assert disp(x, 128, 2, sm + 256, sc, st, sm=sm) == md.MOEDISP_ERR_ALIASED  # out over smooth
+    noassist = _layout(md); noassist.assist_info = None
+    assert disp(x, 128, 2, ex, sc, st, sm=sm, lay=noassist) == md.MOEDISP_ERR_NULLPTR
     comb = lambda eo, H, w, y, st: md.raw_call(
         "moedisp_moe_combine", eo, H, d, ctypes.byref(L), w, y, st, None)
     assert comb(ex, 100, x, sc, st) == md.MOEDISP_ERR_MISALIGNED

@@ -256,8 +256,7 @@ def run_dispatch(md, w, L, quant_mode, etn_type=1, smooth=None):
     st = new_status()
     md.moe_dispatch(x, w.H, L, quant_mode, ex, sc if quant_mode else None, st,
                     expert_token_nums=etn, expert_token_nums_type=etn_type, ep_recv_counts=erc,
-                    smooth_scales=None if smooth is None else dev(smooth),
-                    expert_ids=None if smooth is None else dev(w.expert_ids))
+                    smooth_scales=None if smooth is None else dev(smooth))
     torch.cuda.synchronize()
     return full, scales, gr, etn.cpu().numpy(), erc.cpu().numpy(), int(st.item())
 
@@ -336,25 +335,50 @@ def test_dispatch_smoothing_parity(md, over, q):
     assert (s[:gr] == -1).all() and (s[gr + R:] == -1).all()
 
 
-def test_dispatch_smoothing_bad_expert_id_is_flagged(md):
-    """A routed slot whose expert id is out of range (the layout was computed from other
-    ids) is skipped with BAD_EXPERT_ID instead of reading outside the smoothing table."""
+@pytest.mark.parametrize("q", [2, 3])
+@pytest.mark.parametrize("smooth", [False, True])
+def test_quant_subnormal_rows(md, q, smooth):
+    """Rows of bf16 subnormals (integers up to 8 times 2^-133). Smoothed by 2^-7 the
+    products sit deep in fp32's subnormal range, where the scale max/127 (max/448) keeps
+    only a few bits: every such row's unclamped quotient passes 127.5 (int8), and half of
+    them pass e4m3's saturation edge, so the clamp and the saturation act. Bit-exact
+    against the oracle."""
+    w = wl.moe_workload("tiny", seed=39, W=2, T=24, K=3, E=6, H=64)
+    rng = np.random.default_rng(40)
+    mag = np.where(np.arange(w.G)[:, None] % 2 == 0, 8, 1)
+    xi = rng.integers(-8, 9, size=(w.G, w.H)) % (mag + 1) * np.sign(rng.standard_normal((w.G, w.H)))
+    w.x_bits = wl.f32_to_bf16_bits((xi * 2.0 ** -133).astype(np.float32))
+    sm = np.full((w.E, w.H), 2.0 ** -7, np.float32) if smooth else None
+    L, _ = run_layout(md, w)
+    ref = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active)
+    full, scales, gr, _, _, st = run_dispatch(md, w, L, q, smooth=sm)
+    assert st == 0
+    R = ref["R"]
+    rex, rsc, _ = oracle.moe_dispatch(w.x_bits, ref["dst_row"], w.K, ref["rows_cap"], q,
+                                      smooth=sm, expert_ids=w.expert_ids if smooth else None)
+    assert np.array_equal(full.cpu().numpy()[gr:gr + R], rex[:R])
+    assert np.array_equal(scales.cpu().numpy()[gr:gr + R].view(np.uint32), rsc[:R].view(np.uint32))
+
+
+def test_dispatch_smoothing_bad_assist_entry_is_flagged(md):
+    """A row whose assist_info entry is out of range is skipped with BAD_EXPERT_ID instead
+    of gathering outside x; every other row is exact."""
     w = wl.moe_workload("tiny", seed=37, W=2, T=30, K=2, E=4, H=256)
     sm = wl.smooth_scales(w.E, w.H, seed=38)
     L, _ = run_layout(md, w)
-    bad = w.expert_ids.copy()
-    bad[3, 1] = 99
-    w2 = wl.MoEWorkload(**{**w.__dict__, "expert_ids": bad})
-    full, scales, gr, _, _, st = run_dispatch(md, w2, L, 2, smooth=sm)
-    assert st & md.STATUS_BAD_EXPERT_ID
     ref = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active)
-    rex, rsc, fl = oracle.moe_dispatch(w.x_bits, ref["dst_row"], w.K, ref["rows_cap"], 2,
-                                       smooth=sm, expert_ids=bad)
-    assert fl & oracle.ORC_BAD_EXPERT
-    skipped = ref["dst_row"][3 * w.K + 1]
-    got = full.cpu().numpy()[gr:gr + ref["R"]]
-    keep = np.arange(ref["R"]) != skipped
-    assert np.array_equal(got[keep], rex[:ref["R"]][keep]) and (got[skipped] == 0x5A).all()
+    R = ref["R"]
+    L.assist_info[5] = w.G * w.K                    # one past the last slot
+    L.assist_info[9] = -7
+    full, scales, gr, _, _, st = run_dispatch(md, w, L, 2, smooth=sm)
+    assert st == md.STATUS_BAD_EXPERT_ID
+    rex, rsc, _ = oracle.moe_dispatch(w.x_bits, ref["dst_row"], w.K, ref["rows_cap"], 2,
+                                      smooth=sm, expert_ids=w.expert_ids)
+    got = full.cpu().numpy()[gr:gr + R]
+    keep = np.ones(R, bool)
+    keep[[5, 9]] = False
+    assert np.array_equal(got[keep], rex[:R][keep])
+    assert (got[5] == 0x5A).all() and (got[9] == 0x5A).all()
 
 
 @pytest.mark.parametrize("name,q", [("cfg2", 0), ("cfg3", 2), ("cfg4", 3)])
