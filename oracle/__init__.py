@@ -61,8 +61,9 @@ def lib() -> ctypes.CDLL:
         L.orc_e4m3_to_f32.restype = ctypes.c_float
         L.orc_a2a_exchange_plan.argtypes = [i32, P, P, P, P]
         L.orc_a2a_v.argtypes = [i32, P, i64, P, i64, i64, P, P, P]
-        L.orc_moe_dispatch_layout.argtypes = [i32, i32, i32, i32, P, P, i32, i64, P, P, P, P, P, P, P]
-        L.orc_moe_recv_counts.argtypes = [i32, i32, P, i32, P, P]
+        L.orc_moe_dispatch_layout.argtypes = [i32, i32, i32, i32, P, P, i32, i64, i64, P, P, P, P, P,
+                                              P, P]
+        L.orc_moe_recv_counts.argtypes = [i32, i32, P, i64, i32, P, P]
         L.orc_moe_dispatch.argtypes = [i32, i32, i32, P, P, i64, i32, P, P, P, i32, P]
         L.orc_quant_row.argtypes = [i32, P, i32, P]
         L.orc_quant_row.restype = ctypes.c_float
@@ -137,9 +138,9 @@ def a2a_v(inp: np.ndarray, out: np.ndarray, src_offsets, out_splits, dst_offsets
 # ----------------------------------------------------------------------- O3
 
 def moe_dispatch_layout(W: int, T: int, K: int, E: int, expert_ids, active=None,
-                        rows_cap: int | None = None) -> dict:
+                        rows_cap: int | None = None, major_align: int = 0) -> dict:
     """active: None, a per-token mask [G], or a per-slot mask [G, K] (told apart by size;
-    with K = 1 the two readings coincide)."""
+    with K = 1 the two readings coincide). major_align >= 2 pads expert segments."""
     ids = _c(expert_ids, np.int32).reshape(-1)
     G = W * T
     assert ids.size == G * K
@@ -147,7 +148,8 @@ def moe_dispatch_layout(W: int, T: int, K: int, E: int, expert_ids, active=None,
     active_dims = 1 if act is None or act.size == G else 2
     assert act is None or act.size == (G if active_dims == 1 else G * K)
     if rows_cap is None:
-        rows_cap = G * K
+        A = max(int(major_align), 1)
+        rows_cap = G * K + (E * A if A > 1 else 0)
     out = dict(
         cnt=np.zeros((W, E), np.int32),
         occ=np.zeros(G * K, np.int32),
@@ -157,7 +159,8 @@ def moe_dispatch_layout(W: int, T: int, K: int, E: int, expert_ids, active=None,
         rank_base=np.zeros(W + 1, np.int64),
         send_splits=np.zeros((W, W), np.int64),
     )
-    fl = lib().orc_moe_dispatch_layout(W, T, K, E, _p(ids), _p(act), active_dims, rows_cap,
+    fl = lib().orc_moe_dispatch_layout(W, T, K, E, _p(ids), _p(act), active_dims, int(major_align),
+                                       rows_cap,
                                        _p(out["cnt"]), _p(out["occ"]), _p(out["dst_row"]),
                                        _p(out["assist_info"]), _p(out["expert_base"]),
                                        _p(out["rank_base"]), _p(out["send_splits"]))
@@ -167,12 +170,13 @@ def moe_dispatch_layout(W: int, T: int, K: int, E: int, expert_ids, active=None,
     return out
 
 
-def moe_recv_counts(W: int, E: int, cnt, expert_token_nums_type: int = 1):
+def moe_recv_counts(W: int, E: int, cnt, expert_token_nums_type: int = 1, major_align: int = 0):
     ne = E // W
     c = _c(cnt, np.int32)
     etn = np.zeros((W, ne), np.int64)
     erc = np.zeros((W, ne, W), np.int32)
-    fl = lib().orc_moe_recv_counts(W, E, _p(c), expert_token_nums_type, _p(etn), _p(erc))
+    fl = lib().orc_moe_recv_counts(W, E, _p(c), int(major_align), expert_token_nums_type,
+                                   _p(etn), _p(erc))
     return etn, erc, fl
 
 

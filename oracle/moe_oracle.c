@@ -158,14 +158,27 @@ int orc_a2a_v(int W, const uint8_t *in, int64_t in_rank_stride_rows, uint8_t *ou
  *        _allToAllV_2d_index_push_kernel), i.e. global row rank_base[d] + that.
  * Inactive slots ([P4] xActiveMask: a 1-D mask [G] of tokens, read as any pattern, or a
  * 2-D mask [G][K] of slots, where a token whose K flags are all false sends nothing) and
- * expert ids outside [0, E) contribute no slot; both get occ = dst_row = -1. */
+ * expert ids outside [0, E) contribute no slot; both get occ = dst_row = -1.
+ * major_align ([P1] all_to_all_vdev_2d major_align, the padding rule of the 2-D plan
+ * test): 0 or 1, no padding; A >= 2, each expert's segment of aggregate[e] rows is
+ * padded to max(A, ceil(aggregate[e] / A) * A) rows, so every expert starts on a multiple
+ * of A; the padding rows follow the expert's real rows and get assist_info -1. */
+static int64_t padded_rows(int64_t n, int64_t A)
+{
+    if (A <= 1) return n;
+    int64_t p = (n + A - 1) / A * A;
+    return p < A ? A : p;
+}
+
 int orc_moe_dispatch_layout(int W, int T, int K, int E, const int32_t *expert_ids,
-                            const uint8_t *active, int active_dims, int64_t rows_cap, int32_t *cnt,
+                            const uint8_t *active, int active_dims, int64_t major_align,
+                            int64_t rows_cap, int32_t *cnt,
                             int32_t *occ, int32_t *dst_row, int32_t *assist_info,
                             int64_t *expert_base, int64_t *rank_base, int64_t *send_splits)
 {
     if (W <= 0 || T < 0 || K <= 0 || E <= 0 || E % W != 0) return ORC_BAD_ARG;
     if (active && active_dims != 1 && active_dims != 2) return ORC_BAD_ARG;
+    if (major_align < 0) return ORC_BAD_ARG;
     int flags = 0;
     int ne = E / W;
     int64_t G = (int64_t)W * T;
@@ -206,7 +219,7 @@ int orc_moe_dispatch_layout(int W, int T, int K, int E, const int32_t *expert_id
         int64_t c = 0;
         for (int le = 0; le < ne; le++) {
             cusum_per_rank[d * ne + le] = c;
-            c += aggregate[d * ne + le];
+            c += padded_rows(aggregate[d * ne + le], major_align);
         }
     }
     for (int r = 0; r < W; r++)
@@ -216,7 +229,7 @@ int orc_moe_dispatch_layout(int W, int T, int K, int E, const int32_t *expert_id
     int64_t acc = 0;
     for (int d = 0; d < W; d++) {
         rank_base[d] = acc;
-        for (int le = 0; le < ne; le++) acc += aggregate[d * ne + le];
+        for (int le = 0; le < ne; le++) acc += padded_rows(aggregate[d * ne + le], major_align);
     }
     rank_base[W] = acc;
     for (int e = 0; e < E; e++) expert_base[e] = rank_base[e / ne] + cusum_per_rank[e];
@@ -242,6 +255,9 @@ int orc_moe_dispatch_layout(int W, int T, int K, int E, const int32_t *expert_id
             if (row < rows_cap) assist_info[row] = (int32_t)s;
         }
     }
+    for (int e = 0; e < E; e++)
+        for (int64_t row = expert_base[e] + aggregate[e]; row < expert_base[e + 1]; row++)
+            if (row < rows_cap) assist_info[row] = -1;
 
     free(cusum_per_expert); free(aggregate); free(cusum_per_rank); free(dst2d); free(running);
     return flags;
@@ -249,11 +265,14 @@ int orc_moe_dispatch_layout(int W, int T, int K, int E, const int32_t *expert_id
 
 /* [P4] expertTokenNumsOut (per local expert: count, or with type 0 the running sum over
  * the rank's local experts, read as inclusive) and epRecvCountsOut (rows received from
- * each source rank, ordered expert-major like [P1]'s 2-D out_splits). */
-int orc_moe_recv_counts(int W, int E, const int32_t *cnt, int expert_token_nums_type,
-                        int64_t *expert_token_nums, int32_t *ep_recv_counts)
+ * each source rank, ordered expert-major like [P1]'s 2-D out_splits). With major_align,
+ * as in [P1]'s 2-D plan, the last source rank's entry absorbs the expert's padding, so
+ * both count the padded segment. */
+int orc_moe_recv_counts(int W, int E, const int32_t *cnt, int64_t major_align,
+                        int expert_token_nums_type, int64_t *expert_token_nums,
+                        int32_t *ep_recv_counts)
 {
-    if (W <= 0 || E <= 0 || E % W != 0) return ORC_BAD_ARG;
+    if (W <= 0 || E <= 0 || E % W != 0 || major_align < 0) return ORC_BAD_ARG;
     int ne = E / W;
     for (int d = 0; d < W; d++) {
         int64_t run = 0;
@@ -265,6 +284,9 @@ int orc_moe_recv_counts(int W, int E, const int32_t *cnt, int expert_token_nums_
                 ep_recv_counts[((int64_t)d * ne + le) * W + r] = c;
                 tot += c;
             }
+            int64_t pad = padded_rows(tot, major_align) - tot;
+            ep_recv_counts[((int64_t)d * ne + le) * W + (W - 1)] += (int32_t)pad;
+            tot += pad;
             run += tot;
             expert_token_nums[(int64_t)d * ne + le] = expert_token_nums_type == 0 ? run : tot;
         }

@@ -46,10 +46,13 @@ int orc_a2a_v(int W, const uint8_t *in, int64_t in_rank_stride_rows, uint8_t *ou
               const int64_t *out_splits, const int64_t *dst_offsets);
 
 /* O3: dispatch layout. active may be NULL (all active); active_dims 1: active[G] per
- * token, 2: active[G][K] per slot. Inactive slots get occ = -1, dst_row = -1. assist_info
- * entries beyond R are left untouched. */
+ * token, 2: active[G][K] per slot. Inactive slots get occ = -1, dst_row = -1. major_align
+ * 0/1: none, A >= 2: expert segments padded to multiples of A (at least A rows), padding
+ * rows get assist_info -1. assist_info entries at or beyond R = expert_base[E] are left
+ * untouched. */
 int orc_moe_dispatch_layout(int W, int T, int K, int E, const int32_t *expert_ids,
-                            const uint8_t *active, int active_dims, int64_t rows_cap, int32_t *cnt,
+                            const uint8_t *active, int active_dims, int64_t major_align,
+                            int64_t rows_cap, int32_t *cnt,
                             int32_t *occ, int32_t *dst_row, int32_t *assist_info,
                             int64_t *expert_base, int64_t *rank_base, int64_t *send_splits);
 
@@ -57,8 +60,9 @@ int orc_moe_dispatch_layout(int W, int T, int K, int E, const int32_t *expert_id
  * expert_token_nums[W][ne] (type 1 counts, type 0 inclusive prefix sum over local
  * experts); ep_recv_counts[W][ne][W] = rows that local expert le of rank d receives
  * from source rank r. */
-int orc_moe_recv_counts(int W, int E, const int32_t *cnt, int expert_token_nums_type,
-                        int64_t *expert_token_nums, int32_t *ep_recv_counts);
+int orc_moe_recv_counts(int W, int E, const int32_t *cnt, int64_t major_align,
+                        int expert_token_nums_type, int64_t *expert_token_nums,
+                        int32_t *ep_recv_counts);
 
 /* O4: dispatch copy with optional per-token dynamic quantisation (0 none, 2 int8,
  * 3 fp8-e4m3). dynamic_scales may be NULL for mode 0. smooth ([E][H] fp32, quantising

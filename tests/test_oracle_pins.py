@@ -299,6 +299,67 @@ def test_layout_closed_form_on_workloads(name, over):
     _check_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active, lay)
 
 
+@pytest.mark.parametrize("A", [2, 3, 8, 128])
+@pytest.mark.parametrize("seed", range(3))
+def test_layout_major_align_properties(A, seed):
+    """[P1] all_to_all_vdev_2d major_align: every expert segment starts on a multiple of A,
+    holds the expert's rows in stable slot order and then padding rows (assist_info -1),
+    is a multiple of A long, never empty, and pads by less than A past its rows; every
+    dst_row moves by its expert's base shift only."""
+    rng = np.random.default_rng(300 + seed)
+    W, ne = int(rng.integers(1, 5)), int(rng.integers(1, 5))
+    E, T, K = W * ne, int(rng.integers(1, 40)), int(rng.integers(1, 4))
+    ids = rng.integers(0, E, size=(W * T, K)).astype(np.int32)
+    ids[ids == E - 1] = 0                                          # expert E-1 stays empty
+    active = (rng.random(W * T) < 0.8).astype(np.uint8)
+    plain = oracle.moe_dispatch_layout(W, T, K, E, ids, active)
+    pad = oracle.moe_dispatch_layout(W, T, K, E, ids, active, major_align=A)
+    assert pad["flags"] == 0
+    eb, eb0 = pad["expert_base"], plain["expert_base"]
+    rows, _ = brute_layout(W, T, K, E, ids.tolist(), active.tolist())
+    pos = 0
+    for e in range(E):
+        n = int(eb0[e + 1] - eb0[e])
+        seg = int(eb[e + 1] - eb[e])
+        assert eb[e] % A == 0 and seg % A == 0 and seg >= n
+        assert seg == A if n == 0 else seg - n < A
+        assert pad["assist_info"][eb[e]:eb[e] + n].tolist() == rows[pos:pos + n]
+        assert (pad["assist_info"][eb[e] + n:eb[e + 1]] == -1).all()
+        pos += n
+    assert eb[E - 1 + 1] - eb[E - 1] == A                          # the empty expert
+    act = plain["dst_row"] >= 0
+    e_of = ids.reshape(-1)
+    assert (pad["dst_row"][~act] == -1).all()
+    assert (pad["dst_row"][act] - plain["dst_row"][act] == (eb - eb0)[e_of[act]]).all()
+    assert pad["rank_base"].tolist() == [int(eb[d * ne]) for d in range(W)] + [int(eb[E])]
+    for k in ("cnt", "occ", "send_splits"):
+        assert np.array_equal(pad[k], plain[k]), k
+
+
+def test_layout_major_align_one_is_no_padding():
+    w = wl.moe_workload("tiny", seed=22, W=3, T=30, E=12, K=3, active_p=0.7)
+    base = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active)
+    for A in (0, 1):
+        o = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active, major_align=A)
+        for k in ("cnt", "occ", "dst_row", "expert_base", "rank_base", "send_splits"):
+            assert np.array_equal(o[k], base[k]), k
+
+
+def test_recv_counts_major_align_absorbed_by_last_rank():
+    """As in [P1]'s 2-D plan test, the last source rank's split absorbs the padding:
+    per expert the received counts sum to the padded segment."""
+    w = wl.moe_workload("tiny", seed=23, W=4, T=9, E=12, K=3)
+    A = 8
+    lay = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active, major_align=A)
+    ne = w.E // w.W
+    etn1, erc, _ = oracle.moe_recv_counts(w.W, w.E, lay["cnt"], 1, major_align=A)
+    etn0, _, _ = oracle.moe_recv_counts(w.W, w.E, lay["cnt"], 0, major_align=A)
+    seg = np.diff(lay["expert_base"]).reshape(w.W, ne)
+    assert (erc.sum(axis=2) == seg).all() and (etn1 == seg).all()
+    assert (erc[:, :, :-1] == lay["cnt"].T.reshape(w.W, ne, w.W)[:, :, :-1]).all()
+    assert (etn0[:, -1] == np.diff(lay["rank_base"])).all()
+
+
 def test_layout_bad_expert_and_capacity():
     ids = np.array([[0, 5], [1, -1], [2, 3]], np.int32)     # W=1, T=3, K=2, E=4
     lay = oracle.moe_dispatch_layout(1, 3, 2, 4, ids)
