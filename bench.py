@@ -529,6 +529,32 @@ def op_sweep(md, torch, device, hbm, reps=10):
                     "gather_bytes": bg, "gather_frac": round(bg / ms / 1e6 / hbm, 4)})
         del st, sm
         torch.cuda.empty_cache()
+    # layout with expert segments padded to multiples of 128 rows (grouped-GEMM tiles),
+    # beside the unpadded layout timed the same way (eager launches, flushed L2)
+    for name, A in (("cfg2", 0), ("cfg2", 128), ("cfg3", 0), ("cfg3", 128)):
+        w = wl.moe_workload(name, seed=0)
+        L = md.LayoutBuffers.allocate(w.W, w.T, w.K, w.E, device=device, major_align=A)
+        ids = torch.from_numpy(w.expert_ids.reshape(-1)).to(device)
+        act = None if w.active is None else torch.from_numpy(w.active).to(device)
+        status = torch.zeros(1, dtype=torch.int32, device=device)
+        Ev = torch.cuda.Event
+        pairs = []
+        for r in range(reps + 3):
+            flush.zero_()
+            e0, e1 = Ev(enable_timing=True), Ev(enable_timing=True)
+            e0.record()
+            md.moe_dispatch_layout(ids, act, L, status)
+            e1.record()
+            if r >= 3:
+                pairs.append((e0, e1))
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0, md.status_string(int(status.item()))
+        ms = statistics.mean(a.elapsed_time(b) for a, b in pairs)
+        R = int(L.expert_base[-1].item())
+        out.append({"workload": name, "op": f"layout_eager_align{A}", "us": round(ms * 1e3, 2),
+                    "rows": R})
+        del L
+        torch.cuda.empty_cache()
     # raw all-to-all-v, W = 64
     a = wl.a2a_workload(seed=0)
     W, E_ = a.W, a.row_elems

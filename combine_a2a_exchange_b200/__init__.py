@@ -72,9 +72,9 @@ _plan = _sig("moedisp_a2a_exchange_plan", [_P, _I, _P, _P, _P, _P, _P])
 _a2a_v = _sig("moedisp_a2a_v", [_P, _I64, _P, _I64, _I64, _I, _P, _P, _P, _P, _P])
 _ws_size = _sig("moedisp_layout_workspace_size", [Dims, ctypes.POINTER(ctypes.c_size_t)])
 _layout = _sig("moedisp_moe_dispatch_layout",
-               [_P, _P, _I, Dims, ctypes.POINTER(Layout), _P, ctypes.c_size_t, _P, _P])
+               [_P, _P, _I, _I, Dims, ctypes.POINTER(Layout), _P, ctypes.c_size_t, _P, _P])
 _layout_noalloc = _sig("moedisp_moe_dispatch_layout_noalloc",
-                       [_P, _P, _I, Dims, ctypes.POINTER(Layout), _P, _P])
+                       [_P, _P, _I, _I, Dims, ctypes.POINTER(Layout), _P, _P])
 _dispatch = _sig("moedisp_moe_dispatch",
                  [_P, _I, Dims, ctypes.POINTER(Layout), _I, _P, _P, _P, _P, _I, _P, _P, _P])
 _combine = _sig("moedisp_moe_combine", [_P, _I, Dims, ctypes.POINTER(Layout), _P, _P, _P, _P])
@@ -169,14 +169,18 @@ class LayoutBuffers:
     rank_base: object
     send_splits: object
     workspace: object
+    major_align: int = 0
 
     @classmethod
-    def allocate(cls, W, T, K, E, rows_cap=None, device="cuda"):
+    def allocate(cls, W, T, K, E, rows_cap=None, device="cuda", major_align=0):
+        """rows_cap defaults to the most rows the layout can produce: G*K, plus E*A with
+        major_align A >= 2."""
         import torch
         G = W * T
-        rows_cap = G * K if rows_cap is None else rows_cap
+        if rows_cap is None:
+            rows_cap = G * K + (E * major_align if major_align > 1 else 0)
         z = dict(device=device)
-        return cls(W=W, T=T, K=K, E=E, rows_cap=rows_cap,
+        return cls(W=W, T=T, K=K, E=E, rows_cap=rows_cap, major_align=major_align,
                    cnt=torch.zeros((W, E), dtype=torch.int32, **z),
                    occ=torch.zeros(G * K, dtype=torch.int32, **z),
                    dst_row=torch.zeros(G * K, dtype=torch.int32, **z),
@@ -218,8 +222,8 @@ def moe_dispatch_layout(expert_ids, active_mask, layout: LayoutBuffers, status, 
     nbytes = (ws.numel() * ws.element_size()) if workspace_bytes is None else workspace_bytes
     L = layout.struct()
     rc = _layout(_ptr(expert_ids), _ptr(active_mask),
-                 _mask_dims(active_mask, layout.dims, active_mask_dims), layout.dims,
-                 ctypes.byref(L), _ptr(ws), int(nbytes), _ptr(status), _stream(stream))
+                 _mask_dims(active_mask, layout.dims, active_mask_dims), int(layout.major_align),
+                 layout.dims, ctypes.byref(L), _ptr(ws), int(nbytes), _ptr(status), _stream(stream))
     return _check(rc, "moe_dispatch_layout", raise_on_error)
 
 
@@ -229,8 +233,9 @@ def moe_dispatch_layout_noalloc(expert_ids, active_mask, layout: LayoutBuffers, 
     library's own device memory (see include/moedisp.h). Allocates nothing."""
     L = layout.struct()
     rc = _layout_noalloc(_ptr(expert_ids), _ptr(active_mask),
-                         _mask_dims(active_mask, layout.dims, active_mask_dims), layout.dims,
-                         ctypes.byref(L), _ptr(status), _stream(stream))
+                         _mask_dims(active_mask, layout.dims, active_mask_dims),
+                         int(layout.major_align), layout.dims, ctypes.byref(L), _ptr(status),
+                         _stream(stream))
     return _check(rc, "moe_dispatch_layout_noalloc", raise_on_error)
 
 

@@ -45,6 +45,16 @@ int check_dims(const moedisp_dims& d) {
     return MOEDISP_OK;
 }
 
+// major_align: 0 or 1 (no padding) up to MOEDISP_MAX_ALIGN; the padded row count
+// (at most G*K + E*align) must stay an int32 row index.
+int check_major_align(int major_align, const moedisp_dims& d) {
+    if (major_align < 0) return MOEDISP_ERR_INVALID;
+    if (major_align > MOEDISP_MAX_ALIGN) return MOEDISP_ERR_UNSUPPORTED;
+    const int64_t worst = (int64_t)d.W * d.T * d.K + (major_align > 1 ? (int64_t)d.E * major_align : 0);
+    if (worst >= (int64_t(1) << 31)) return MOEDISP_ERR_UNSUPPORTED;
+    return MOEDISP_OK;
+}
+
 int check_rows_cap(int64_t rows_cap) {
     if (rows_cap < 0) return MOEDISP_ERR_INVALID;
     if (rows_cap > 0x7fffffffll) return MOEDISP_ERR_UNSUPPORTED;
@@ -89,7 +99,7 @@ const char* moedisp_status_string(int code) {
     return "unknown code";
 }
 
-int moedisp_version(void) { return 2; }
+int moedisp_version(void) { return 3; }
 
 int moedisp_selftest_bounded_wait(uint32_t limit_us, int32_t* status, moedisp_stream_t stream) {
     if (!status) return MOEDISP_ERR_NULLPTR;
@@ -150,7 +160,7 @@ int moedisp_layout_workspace_size(moedisp_dims dims, size_t* bytes) {
 }
 
 int moedisp_moe_dispatch_layout(const int32_t* expert_ids, const uint8_t* active_mask,
-                                int active_mask_dims, moedisp_dims dims, const moedisp_layout* layout,
+                                int active_mask_dims, int major_align, moedisp_dims dims, const moedisp_layout* layout,
                                 void* workspace, size_t workspace_bytes, int32_t* status,
                                 moedisp_stream_t stream) {
     if (!layout || !status) return MOEDISP_ERR_NULLPTR;
@@ -163,6 +173,7 @@ int moedisp_moe_dispatch_layout(const int32_t* expert_ids, const uint8_t* active
     if (slots > 0 && (!expert_ids || !L.occ || !L.dst_row)) return MOEDISP_ERR_NULLPTR;
     if (L.rows_cap > 0 && !L.assist_info) return MOEDISP_ERR_NULLPTR;
     if (active_mask && active_mask_dims != 1 && active_mask_dims != 2) return MOEDISP_ERR_INVALID;
+    if ((c = check_major_align(major_align, dims)) != MOEDISP_OK) return c;
     if (!workspace) return MOEDISP_ERR_WORKSPACE;
     const moedisp::LayoutGeometry g = moedisp::layout_geometry(dims);
     if (workspace_bytes < g.total_bytes) return MOEDISP_ERR_WORKSPACE;
@@ -184,12 +195,12 @@ int moedisp_moe_dispatch_layout(const int32_t* expert_ids, const uint8_t* active
                   {{expert_ids, (size_t)slots * 4},
                    {active_mask, (size_t)(active_mask_dims == 2 ? slots : G)}}))
         return MOEDISP_ERR_ALIASED;
-    return rc(moedisp::launch_layout(expert_ids, active_mask, active_mask_dims, dims, L, workspace,
-                                     status, stream));
+    return rc(moedisp::launch_layout(expert_ids, active_mask, active_mask_dims, major_align, dims,
+                                     L, workspace, status, stream));
 }
 
 int moedisp_moe_dispatch_layout_noalloc(const int32_t* expert_ids, const uint8_t* active_mask,
-                                        int active_mask_dims, moedisp_dims dims, const moedisp_layout* layout,
+                                        int active_mask_dims, int major_align, moedisp_dims dims, const moedisp_layout* layout,
                                         int32_t* status, moedisp_stream_t stream) {
     if (!layout || !status) return MOEDISP_ERR_NULLPTR;
     int c = check_dims(dims);
@@ -201,6 +212,7 @@ int moedisp_moe_dispatch_layout_noalloc(const int32_t* expert_ids, const uint8_t
     if (slots > 0 && (!expert_ids || !L.occ || !L.dst_row)) return MOEDISP_ERR_NULLPTR;
     if (L.rows_cap > 0 && !L.assist_info) return MOEDISP_ERR_NULLPTR;
     if (active_mask && active_mask_dims != 1 && active_mask_dims != 2) return MOEDISP_ERR_INVALID;
+    if ((c = check_major_align(major_align, dims)) != MOEDISP_OK) return c;
     if (moedisp::layout_geometry(dims).total_bytes > moedisp::layout_noalloc_scratch_bytes())
         return MOEDISP_ERR_UNSUPPORTED;
     if (!aligned(expert_ids, 4) || !aligned(L.cnt, 4) || !aligned(L.occ, 4) ||
@@ -219,8 +231,8 @@ int moedisp_moe_dispatch_layout_noalloc(const int32_t* expert_ids, const uint8_t
                   {{expert_ids, (size_t)slots * 4},
                    {active_mask, (size_t)(active_mask_dims == 2 ? slots : G)}}))
         return MOEDISP_ERR_ALIASED;
-    return rc(moedisp::launch_layout_noalloc(expert_ids, active_mask, active_mask_dims, dims, L,
-                                             status, stream));
+    return rc(moedisp::launch_layout_noalloc(expert_ids, active_mask, active_mask_dims,
+                                             major_align, dims, L, status, stream));
 }
 
 int moedisp_moe_dispatch(const void* x, int H, moedisp_dims dims,
@@ -252,7 +264,7 @@ int moedisp_moe_dispatch(const void* x, int H, moedisp_dims dims,
     if (quant_mode != MOEDISP_QUANT_NONE && L.rows_cap > 0 && !dynamic_scales)
         return MOEDISP_ERR_NULLPTR;
     if (expert_token_nums && (!L.expert_base || !L.rank_base)) return MOEDISP_ERR_NULLPTR;
-    if (ep_recv_counts && !L.cnt) return MOEDISP_ERR_NULLPTR;
+    if (ep_recv_counts && (!L.cnt || !L.expert_base)) return MOEDISP_ERR_NULLPTR;
     if (!aligned(x, 16) || !aligned(expand_x, 16) || !aligned(L.dst_row, 4) ||
         !aligned(dynamic_scales, 4) || !aligned(expert_token_nums, 8) ||
         !aligned(ep_recv_counts, 4) || !aligned(status, 4) || !aligned(smooth_scales, 16) ||

@@ -155,7 +155,15 @@ __device__ void write_recv_counts(const DispatchArgs& a) {
         for (int64_t idx = first; idx < n; idx += stride) {
             const int64_t e = idx / a.W;                  // = d*ne + le
             const int r = (int)(idx - e * a.W);
-            a.erc[idx] = a.cnt[(int64_t)r * a.E + e];
+            int32_t v = a.cnt[(int64_t)r * a.E + e];
+            if (r == a.W - 1) {
+                // the last source rank's entry absorbs the expert's padding (major_align):
+                // segment rows minus the rows routed to the expert
+                int64_t routed = 0;
+                for (int q = 0; q < a.W; ++q) routed += a.cnt[(int64_t)q * a.E + e];
+                v += (int32_t)(a.expert_base[e + 1] - a.expert_base[e] - routed);
+            }
+            a.erc[idx] = v;
         }
     }
     if (a.etn != nullptr) {
@@ -484,6 +492,7 @@ __global__ void __launch_bounds__(kQuantThreads, CPT > 4 ? 2 : 4) dispatch_smoot
             __syncthreads();
             for (int64_t row = r + grp; row < seg_end; row += NG) {
                 const int32_t slot = __ldg(a.assist + row);          // same for the group
+                if (slot == -1) continue;                            // a padding row
                 if (slot < 0 || (int64_t)slot >= slots) {
                     if (gt == 0) raise_status(a.status, MOEDISP_STATUS_BAD_EXPERT_ID);
                     continue;

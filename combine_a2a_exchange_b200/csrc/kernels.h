@@ -71,13 +71,13 @@ struct LayoutGeometry {
 LayoutGeometry layout_geometry(const moedisp_dims& d);
 
 cudaError_t launch_layout(const int32_t* expert_ids, const uint8_t* active, int active_dims,
-                          const moedisp_dims& dims, const moedisp_layout& layout,
+                          int major_align, const moedisp_dims& dims, const moedisp_layout& layout,
                           void* workspace, int32_t* status, cudaStream_t stream);
 
 // Allocation-free layout: the tiled path on the library's static scratch array.
 size_t layout_noalloc_scratch_bytes();
 cudaError_t launch_layout_noalloc(const int32_t* expert_ids, const uint8_t* active,
-                                  int active_dims, const moedisp_dims& dims, const moedisp_layout& layout,
+                                  int active_dims, int major_align, const moedisp_dims& dims, const moedisp_layout& layout,
                                   int32_t* status, cudaStream_t stream);
 
 cudaError_t launch_bounded_wait_selftest(uint64_t limit_ns, int32_t* status, cudaStream_t stream);

@@ -60,6 +60,7 @@ struct LayoutArgs {
     const uint8_t* active;     // null, [G] (per token, active_dims 1) or [G*K] (per slot, 2)
     int active_dims;
     int W, T, K, E, ne;
+    int64_t align;             // major_align: expert segments padded to multiples (>= 2)
     int64_t P;                 // slots per source rank, T*K
     int tiles_per_rank;
     int n_tiles;
@@ -106,6 +107,19 @@ __device__ __forceinline__ unsigned peers_by_ballot(unsigned key, int bits) {
         }
     }
     return m;
+}
+
+// Rows of an expert's segment holding n routed rows: n, or with major_align A >= 2 the
+// next multiple of A, at least A (an expert never gets an empty segment).
+__device__ __forceinline__ int64_t padded_rows(int64_t n, int64_t A) {
+    if (A <= 1) return n;
+    const int64_t p = (n + A - 1) / A * A;
+    return p < A ? A : p;
+}
+
+// Marks an expert's padding rows [first, end), below rows_cap, as holding no slot.
+__device__ __forceinline__ void mark_padding(const LayoutArgs& a, int64_t first, int64_t end) {
+    for (int64_t row = first; row < end && row < a.rows_cap; ++row) a.assist[row] = -1;
 }
 
 // Bits needed for the keys 0..E (expert + 1, 0 = no expert).
@@ -301,9 +315,13 @@ __global__ void __launch_bounds__(kThreads) layout_rank_kernel(LayoutArgs a) {
             cntr[e] = __ldcg(tp + row_next + e) - cp;
             tot = __ldcg(tp + row_tot + e);
         }
+        const int64_t seg = e < E ? padded_rows(tot, a.align) : 0;
         int64_t chunk;
-        const int64_t ex = block_exclusive_scan(tot, warp_tot, chunk);
-        if (e < E) ebase[e] = carry + ex;
+        const int64_t ex = block_exclusive_scan(seg, warp_tot, chunk);
+        if (e < E) {
+            ebase[e] = carry + ex;
+            if (tile == 0 && seg > tot) mark_padding(a, carry + ex + tot, carry + ex + seg);
+        }
         carry += chunk;
     }
     if (threadIdx.x == 0) ebase[E] = carry;
@@ -403,9 +421,13 @@ layout_cluster_kernel(LayoutArgs a) {
             colp[e] = cp;
             cntr[e] = cr;
         }
+        const int64_t seg = e < E ? padded_rows(tot, a.align) : 0;
         int64_t chunk;
-        const int64_t ex = block_exclusive_scan(tot, warp_tot, chunk);
-        if (e < E) ebase[e] = carry + ex;
+        const int64_t ex = block_exclusive_scan(seg, warp_tot, chunk);
+        if (e < E) {
+            ebase[e] = carry + ex;
+            if (tile == 0 && seg > tot) mark_padding(a, carry + ex + tot, carry + ex + seg);
+        }
         carry += chunk;
     }
     if (threadIdx.x == 0) ebase[E] = carry;
@@ -554,13 +576,14 @@ LayoutGeometry layout_geometry(const moedisp_dims& d) {
 
 namespace {
 LayoutArgs make_args(const int32_t* expert_ids, const uint8_t* active, int active_dims,
-                     const moedisp_dims& dims, const moedisp_layout& L, void* workspace,
-                     int32_t* status, const LayoutGeometry& g) {
+                     int major_align, const moedisp_dims& dims, const moedisp_layout& L,
+                     void* workspace, int32_t* status, const LayoutGeometry& g) {
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     LayoutArgs a;
     a.ids = expert_ids;
     a.active = active;
     a.active_dims = active_dims;
+    a.align = major_align;
     a.W = dims.W;
     a.T = dims.T;
     a.K = dims.K;
@@ -586,10 +609,11 @@ LayoutArgs make_args(const int32_t* expert_ids, const uint8_t* active, int activ
 }  // namespace
 
 cudaError_t launch_layout(const int32_t* expert_ids, const uint8_t* active, int active_dims,
-                          const moedisp_dims& dims, const moedisp_layout& L, void* workspace,
-                          int32_t* status, cudaStream_t stream) {
+                          int major_align, const moedisp_dims& dims, const moedisp_layout& L,
+                          void* workspace, int32_t* status, cudaStream_t stream) {
     const LayoutGeometry g = layout_geometry(dims);
-    LayoutArgs a = make_args(expert_ids, active, active_dims, dims, L, workspace, status, g);
+    LayoutArgs a = make_args(expert_ids, active, active_dims, major_align, dims, L, workspace,
+                             status, g);
 
     int tpr_c = 0, steps_c = 0;
     int64_t tile_c = 0;
@@ -647,7 +671,7 @@ cudaError_t layout_scratch_address(void** out) {
 size_t layout_noalloc_scratch_bytes() { return MOEDISP_NOALLOC_SCRATCH_BYTES; }
 
 cudaError_t launch_layout_noalloc(const int32_t* expert_ids, const uint8_t* active,
-                                  int active_dims, const moedisp_dims& dims,
+                                  int active_dims, int major_align, const moedisp_dims& dims,
                                   const moedisp_layout& L,
                                   int32_t* status, cudaStream_t stream) {
     const LayoutGeometry g = layout_geometry(dims);
@@ -656,7 +680,8 @@ cudaError_t launch_layout_noalloc(const int32_t* expert_ids, const uint8_t* acti
     if (err != cudaSuccess) return err;
     // The array keeps whatever the previous call left; nothing in it has to start at
     // zero: every scratch word is written (tile counts, then offsets) before it is read.
-    LayoutArgs a = make_args(expert_ids, active, active_dims, dims, L, scratch, status, g);
+    LayoutArgs a = make_args(expert_ids, active, active_dims, major_align, dims, L, scratch,
+                             status, g);
     return launch_tiled(a, dims, g, stream);
 }
 

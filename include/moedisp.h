@@ -60,12 +60,13 @@ typedef struct CUstream_st *moedisp_stream_t;
 #define MOEDISP_MAX_E        1024    /* Ascend A3: moeExpertNum <= 1024 */
 #define MOEDISP_MAX_H        16384   /* hidden size (elements) for dispatch staging */
 #define MOEDISP_MAX_W        65536   /* ranks of an exchange plan */
+#define MOEDISP_MAX_ALIGN    65536   /* major_align of the layout */
 
 /* Returns a static, human-readable name for a return code (< 0) or status bits (> 0). */
 const char *moedisp_status_string(int code);
 
-/* ABI version, currently 2 (2: active_mask_dims in the layout calls; smoothing scales in
- * moe_dispatch). */
+/* ABI version, currently 3 (2: active_mask_dims in the layout calls, smoothing scales in
+ * moe_dispatch; 3: major_align in the layout calls). */
 int moedisp_version(void);
 
 /* Diagnostic for the time-out path of the device-side waits (this library's own
@@ -167,6 +168,14 @@ int moedisp_layout_workspace_size(moedisp_dims dims, size_t *bytes);
  * MOEDISP_STATUS_BAD_EXPERT_ID and that slot is dropped. If R > rows_cap,
  * MOEDISP_STATUS_CAPACITY is set, every output is still computed, and assist_info is
  * written only below rows_cap.
+ * major_align (the PyTorch symm_mem all_to_all_vdev_2d major_align, with the padding rule
+ * of its 2-D exchange-plan test): 0 or 1, no padding; A in [2, MOEDISP_MAX_ALIGN], every
+ * expert's segment of n routed rows is padded to max(A, ceil(n / A) * A) rows, so every
+ * expert starts on a multiple of A and none is empty (as grouped-GEMM kernels want):
+ * expert_base and rank_base then count padded segments, R = expert_base[E] includes the
+ * padding, the padding rows follow each expert's routed rows and get assist_info -1 (below
+ * rows_cap), and moe_dispatch leaves them untouched. Negative: MOEDISP_ERR_INVALID; above
+ * MOEDISP_MAX_ALIGN: MOEDISP_ERR_UNSUPPORTED.
  * workspace: device memory of at least moedisp_layout_workspace_size() bytes, 16-byte
  * aligned; its contents need no initialisation (every word is written before it is
  * read). Calls sharing one workspace must not run concurrently.
@@ -175,7 +184,7 @@ int moedisp_layout_workspace_size(moedisp_dims dims, size_t *bytes);
  * three: per-tile warp-aggregated histograms, per-expert scans down the tiles, and a
  * per-tile ranking + scatter. */
 int moedisp_moe_dispatch_layout(const int32_t *expert_ids, const uint8_t *active_mask,
-                                int active_mask_dims, moedisp_dims dims, const moedisp_layout *layout,
+                                int active_mask_dims, int major_align, moedisp_dims dims, const moedisp_layout *layout,
                                 void *workspace, size_t workspace_bytes, int32_t *status,
                                 moedisp_stream_t stream);
 
@@ -203,7 +212,7 @@ int moedisp_moe_dispatch_layout(const int32_t *expert_ids, const uint8_t *active
  * Other arguments and errors are those of moedisp_moe_dispatch_layout. */
 #define MOEDISP_NOALLOC_SCRATCH_BYTES (2u << 20)
 int moedisp_moe_dispatch_layout_noalloc(const int32_t *expert_ids, const uint8_t *active_mask,
-                                        int active_mask_dims, moedisp_dims dims, const moedisp_layout *layout,
+                                        int active_mask_dims, int major_align, moedisp_dims dims, const moedisp_layout *layout,
                                         int32_t *status, moedisp_stream_t stream);
 
 /* Quantisation modes of moe_dispatch (the Ascend quantMode values; 3 is this library's
@@ -237,7 +246,9 @@ int moedisp_moe_dispatch_layout_noalloc(const int32_t *expert_ids, const uint8_t
  * Optional (NULL to skip), per destination rank d and local expert le:
  *   expert_token_nums int64 [W][ne]: rows of expert d*ne+le (type 1), or the running sum
  *     over the rank's local experts up to and including le (type 0);
- *   ep_recv_counts int32 [W][ne][W]: rows expert d*ne+le receives from source rank r.
+ *   ep_recv_counts int32 [W][ne][W]: rows expert d*ne+le receives from source rank r; with
+ *     major_align the last source rank's entry also counts the expert's padding rows (as
+ *     the 2-D plan's out_splits do), and expert_token_nums counts padded segments.
  * Rows at or beyond rows_cap are not written (MOEDISP_STATUS_CAPACITY).
  * One persistent kernel: without smoothing each token row is brought into shared memory
  * once by a bulk (TMA) copy; unquantised rows leave it as K bulk copies, quantised ones as

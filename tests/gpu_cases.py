@@ -27,10 +27,10 @@ def new_status():
     return torch.zeros(1, dtype=torch.int32, device="cuda")
 
 
-def run_layout(md, w: wl.MoEWorkload, rows_cap=None, ids=None, active="default"):
+def run_layout(md, w: wl.MoEWorkload, rows_cap=None, ids=None, active="default", major_align=0):
     ids = w.expert_ids if ids is None else ids
     act = w.active if isinstance(active, str) else active
-    L = md.LayoutBuffers.allocate(w.W, w.T, w.K, w.E, rows_cap=rows_cap)
+    L = md.LayoutBuffers.allocate(w.W, w.T, w.K, w.E, rows_cap=rows_cap, major_align=major_align)
     st = new_status()
     ids_d = dev(ids.reshape(-1).astype(np.int32))
     act_d = None if act is None else dev(act.astype(np.uint8))

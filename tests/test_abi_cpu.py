@@ -49,7 +49,7 @@ def test_library_exports_every_declared_symbol(md):
 
 
 def test_status_strings(md):
-    assert md.version() == 2
+    assert md.version() == 3
     assert md.status_string(0) == "ok"
     assert md.status_string(-1) == "null pointer"
     assert md.status_string(md.STATUS_CAPACITY | md.STATUS_TIMEOUT) == "capacity | timeout"
@@ -113,8 +113,8 @@ def test_layout_rejections(md):
     with pytest.raises(md.MoedispError):
         md.layout_workspace_size(4, 8, 17, 8)                # K > 16
     L = _layout(md)
-    call = lambda ids, dims, L, ws, nws, st, act=None, ad=0: md.raw_call(
-        "moedisp_moe_dispatch_layout", ids, act, ad, dims, ctypes.byref(L), ws, nws, st, None)
+    call = lambda ids, dims, L, ws, nws, st, act=None, ad=0, al=0: md.raw_call(
+        "moedisp_moe_dispatch_layout", ids, act, ad, al, dims, ctypes.byref(L), ws, nws, st, None)
     ids, ws, st = FAKE + (64 << 20), FAKE + (128 << 20), FAKE + (256 << 20)
     d = md.Dims(4, 8, 2, 8)
     assert call(ids, d, L, ws, ws_ok - 1, st) == md.MOEDISP_ERR_WORKSPACE
@@ -132,6 +132,8 @@ def test_layout_rejections(md):
     act = FAKE + (300 << 20)
     assert call(ids, d, L, ws, ws_ok, st, act, 0) == md.MOEDISP_ERR_INVALID    # mask dims
     assert call(ids, d, L, ws, ws_ok, st, act, 3) == md.MOEDISP_ERR_INVALID
+    assert call(ids, d, L, ws, ws_ok, st, al=-1) == md.MOEDISP_ERR_INVALID        # major_align
+    assert call(ids, d, L, ws, ws_ok, st, al=(1 << 16) + 1) == md.MOEDISP_ERR_UNSUPPORTED
     # a per-slot mask [G][K] spans G*K bytes: one starting G*K - 1 bytes before occ overlaps it
     G, K = 4 * 8, 2
     assert call(ids, d, L, ws, ws_ok, st, L.occ - (G * K - 1), 2) == md.MOEDISP_ERR_ALIASED

@@ -243,6 +243,68 @@ def test_layout_capacity_overflow(md):
     assert_layout_equal(layout_host(L), ref, ref["R"], cap)
 
 
+ALIGN_CASES = [
+    ("tiny", dict(W=3, T=500, K=4, E=12), 16),                        # cluster path
+    ("tiny", dict(W=4, T=300, K=4, E=64, routing="zipf", zipf_zero=20), 8),   # empty experts
+    ("tiny", dict(W=2, T=30000, K=8, E=16, active_p=0.7), 128),       # tiled path
+    ("tiny", dict(W=5, T=700, K=6, E=40, slot_active_p=0.5), 3),
+    ("cfg3", {}, 128),
+]
+
+
+@pytest.mark.parametrize("name,over,A", ALIGN_CASES)
+def test_layout_major_align_parity(md, name, over, A):
+    """Padded expert segments: every layout output, the padding rows' assist_info -1
+    included, bit-exact against the oracle; receive counts too."""
+    w = wl.moe_workload(name, seed=24, **over)
+    L, st = run_layout(md, w, major_align=A)
+    ref = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active, major_align=A)
+    assert st == 0 and ref["flags"] == 0 and L.rows_cap == ref["rows_cap"]
+    assert_layout_equal(layout_host(L), ref, ref["R"], ref["rows_cap"])
+    assert (ref["expert_base"] % A == 0).all()
+    full, scales, gr, etn, erc, st2 = run_dispatch(md, w, L, w.quant_mode, etn_type=1)
+    assert st2 == 0
+    retn, rerc, _ = oracle.moe_recv_counts(w.W, w.E, ref["cnt"], 1, major_align=A)
+    assert np.array_equal(etn, retn) and np.array_equal(erc, rerc)
+
+
+@pytest.mark.parametrize("q", [0, 2, 3])
+def test_dispatch_and_combine_with_major_align(md, q):
+    """Dispatch writes the routed rows of a padded layout and leaves its padding rows
+    untouched; the smoothing kernel, which walks rows, skips them without a status; the
+    combine reads only routed rows."""
+    A = 32
+    w = wl.moe_workload("tiny", seed=25, W=4, T=200, K=4, E=16, H=256, routing="zipf",
+                        zipf_zero=4, active_p=0.8)
+    L, _ = run_layout(md, w, major_align=A)
+    ref = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active, major_align=A)
+    R = ref["R"]
+    pad_rows = np.nonzero(ref["assist_info"][:R] == -1)[0]
+    assert pad_rows.size > 0
+    for smooth in ([None, wl.smooth_scales(w.E, w.H, seed=26)] if q else [None]):
+        full, scales, gr, _, _, st = run_dispatch(md, w, L, q, smooth=smooth)
+        assert st == 0
+        rex, rsc, _ = oracle.moe_dispatch(w.x_bits, ref["dst_row"], w.K, ref["rows_cap"], q,
+                                          smooth=smooth,
+                                          expert_ids=None if smooth is None else w.expert_ids)
+        got = full.cpu().numpy()[gr:gr + R]
+        real = np.ones(R, bool)
+        real[pad_rows] = False
+        if q == 0:
+            got = got.view(np.uint16)
+            assert np.array_equal(got[real], rex[:R][real])
+            assert (got[pad_rows] == np.uint16(-12345 & 0xFFFF)).all()
+        else:
+            assert np.array_equal(got[real], rex[:R][real]) and (got[pad_rows] == 0x5A).all()
+            sc = scales.cpu().numpy()[gr:gr + R]
+            assert np.array_equal(sc[real].view(np.uint32), rsc[:R][real].view(np.uint32))
+            assert (sc[pad_rows] == -1).all()
+    eo = wl.expert_rows(L.rows_cap, w.H, seed=27)
+    y, st = run_combine(md, L, eo, w)
+    assert st == 0
+    check_combine(y, eo, ref["dst_row"], w.weights, w.K, L.rows_cap)
+
+
 # ------------------------------------------------------------------ dispatch
 
 def run_dispatch(md, w, L, quant_mode, etn_type=1, smooth=None):

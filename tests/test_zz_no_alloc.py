@@ -64,6 +64,6 @@ def test_noalloc_layout_rejects_oversized_problems(md):
     L = md.Layout(1 << 40, 1 << 41, 1 << 42, 1 << 43, 1 << 44, 1 << 45, 1 << 46, W * T * K)
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     import ctypes
-    rc = md.raw_call("moedisp_moe_dispatch_layout_noalloc", 1 << 47, None, 0, md.Dims(W, T, K, E),
+    rc = md.raw_call("moedisp_moe_dispatch_layout_noalloc", 1 << 47, None, 0, 0, md.Dims(W, T, K, E),
                      ctypes.byref(L), st.data_ptr(), None)
     assert rc == md.MOEDISP_ERR_UNSUPPORTED
