@@ -73,7 +73,8 @@ def lib() -> ctypes.CDLL:
         L.orc_moe_combine_f32.argtypes = [i32, i32, i32, P, i64, P, P, P]
         L.orc_moe_combine_rmsnorm_f64.argtypes = [i32, i32, i32, P, i64, P, P, P, P, ctypes.c_float, P, P]
         L.orc_moe_combine_rmsnorm_f32.argtypes = [i32, i32, i32, P, i64, P, P, P, P, ctypes.c_float, P, P]
-        for f in ("orc_moe_combine_rmsnorm_f64", "orc_moe_combine_rmsnorm_f32",
+        L.orc_shared_expert_routing.argtypes = [i32, i32, i32, i32, i32, i32, P, P, P, P]
+        for f in ("orc_shared_expert_routing", "orc_moe_combine_rmsnorm_f64", "orc_moe_combine_rmsnorm_f32",
                   "orc_a2a_exchange_plan", "orc_a2a_v", "orc_moe_dispatch_layout",
                   "orc_moe_recv_counts", "orc_moe_dispatch", "orc_moe_combine_f64",
                   "orc_moe_combine_f32"):
@@ -269,3 +270,17 @@ def moe_combine_rmsnorm(expert_out_bits, dst_row, weights, K: int, residual_bits
         fl = lib().orc_moe_combine_rmsnorm_f32(G, K, H, _p(eo), rows_cap, _p(dr), _p(w), _p(res),
                                                _p(gm), eps, _p(rout), _p(y))
     return rout, y, fl
+
+
+# ------------------------------------------------------------ shared experts
+
+def shared_expert_routing(W: int, T: int, K: int, E: int, N: int, S: int, expert_ids, weights):
+    """Returns (ext_ids [G, K+N] int32, ext_w [G, K+N] fp32, E_total, flags)."""
+    ids = _c(expert_ids, np.int32).reshape(-1)
+    w = _c(weights, np.float32).reshape(-1)
+    G = W * T
+    ext_ids = np.zeros((G, K + N), np.int32)
+    ext_w = np.zeros((G, K + N), np.float32)
+    fl = lib().orc_shared_expert_routing(W, T, K, E, N, S, _p(ids), _p(w), _p(ext_ids), _p(ext_w))
+    E_total = W * (E // (W - S)) if 0 <= S < W and E % (W - S) == 0 else 0
+    return ext_ids, ext_w, E_total, fl

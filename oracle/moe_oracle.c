@@ -495,3 +495,51 @@ int orc_moe_combine_rmsnorm_f32(int G, int K, int H, const uint16_t *expert_out,
     free(acc);
     return flags;
 }
+
+/* ------------------------------------------------------ shared experts ([P4]) */
+
+/* [P4] sharedExpertNum N, sharedExpertRankNum S, expertShardType 0: the first S of the W
+ * ranks host shared experts (one replica each, S / N replicas of each of the N shared
+ * experts, replica groups in shared-expert order), the other W - S ranks host the
+ * E routed experts, ne = E / (W - S) each. Every token also goes to each shared expert.
+ * Reading of the pages (which fix only the counts: a shared rank receives
+ * Bs * W * N / S tokens): source rank r's tokens go to replica (r mod (S / N)) of each
+ * shared expert, i.e. rank j * (S / N) + r mod (S / N) for shared expert j.
+ * The result is a routing over a uniform expert space of W * ne experts, ne per rank:
+ * routed expert e becomes S * ne + e; shared expert j's replica on rank d is expert d * ne
+ * (the rank's other ne - 1 expert ids stay unused). ext_ids / ext_w are [G][K + N]: the
+ * K routed slots (weights as given; an id outside [0, E) is mapped to W * ne, still out of
+ * range), then the N shared slots with weight 1. */
+int orc_shared_expert_routing(int W, int T, int K, int E, int N, int S,
+                              const int32_t *expert_ids, const float *w,
+                              int32_t *ext_ids, float *ext_w)
+{
+    if (W <= 0 || T < 0 || K <= 0 || E <= 0 || N < 0 || S < 0 || S >= W) return ORC_BAD_ARG;
+    if ((S == 0) != (N == 0)) return ORC_BAD_ARG;
+    if (S > 0 && (W % S != 0 || S % N != 0)) return ORC_BAD_ARG;
+    if (E % (W - S) != 0) return ORC_BAD_ARG;
+    int ne = E / (W - S);
+    int KN = K + N;
+    int flags = 0;
+    for (int r = 0; r < W; r++)
+        for (int t = 0; t < T; t++) {
+            int64_t g = (int64_t)r * T + t;
+            for (int k = 0; k < K; k++) {
+                int32_t e = expert_ids[g * K + k];
+                if (e < 0 || e >= E) {
+                    flags |= ORC_BAD_EXPERT;
+                    ext_ids[g * KN + k] = W * ne;
+                } else {
+                    ext_ids[g * KN + k] = S * ne + e;
+                }
+                ext_w[g * KN + k] = w[g * K + k];
+            }
+            for (int j = 0; j < N; j++) {
+                int replicas = S / N;
+                int d = j * replicas + r % replicas;
+                ext_ids[g * KN + K + j] = d * ne;
+                ext_w[g * KN + K + j] = 1.0f;
+            }
+        }
+    return flags;
+}

@@ -97,6 +97,13 @@ int orc_moe_combine_rmsnorm_f32(int G, int K, int H, const uint16_t *expert_out,
                                 const uint16_t *residual, const float *gamma, float eps,
                                 uint16_t *residual_out, uint16_t *y);
 
+/* Shared experts ([P4] sharedExpertNum N, sharedExpertRankNum S, expertShardType 0): the
+ * routing widened to K + N slots over W * (E / (W - S)) experts, shared-expert ranks
+ * first; ext_ids / ext_w are [G][K + N]. */
+int orc_shared_expert_routing(int W, int T, int K, int E, int N, int S,
+                              const int32_t *expert_ids, const float *w,
+                              int32_t *ext_ids, float *ext_w);
+
 #ifdef __cplusplus
 }
 #endif

@@ -679,3 +679,56 @@ def test_rmsnorm_closed_form_properties():
     rz, _, _ = oracle.moe_combine_rmsnorm(eo, dr, w, 3, zero, ones, eps)
     yc, _ = oracle.moe_combine_f64(eo, dr, w, 3)
     assert np.allclose(wl.bf16_bits_to_f32(rz), yc, rtol=2 ** -8, atol=1e-30)
+
+
+# ------------------------------------------------------------ shared experts
+
+@pytest.mark.parametrize("W,S,N,ne", [(8, 4, 1, 16), (8, 4, 2, 4), (6, 3, 3, 2), (4, 2, 1, 3)])
+def test_shared_experts_receive_counts_and_rank_order(W, S, N, ne):
+    """[P4]: shared-expert ranks come first (expertShardType 0) and each receives
+    Bs * epWorldSize * sharedExpertNum / sharedExpertRankNum tokens; the routed experts
+    keep their rows on ranks S..W-1; every token reaches each shared expert once."""
+    E = (W - S) * ne
+    T, K = 37, 3
+    w = wl.moe_workload("tiny", seed=60, W=W, T=T, K=K, E=E)
+    ext, extw, E_tot, fl = oracle.shared_expert_routing(W, T, K, E, N, S, w.expert_ids, w.weights)
+    assert fl == 0 and E_tot == W * ne
+    lay = oracle.moe_dispatch_layout(W, T, K + N, E_tot, ext)
+    per_rank = np.diff(lay["rank_base"])
+    assert (per_rank[:S] == T * W * N // S).all()
+    assert per_rank[S:].sum() == W * T * K
+    assert (ext[:, :K] // ne >= S).all() and (ext[:, K:] // ne < S).all()
+    # the N shared slots of a token are N different shared experts (replica groups)
+    grp = (ext[:, K:] // ne) // (S // N)
+    assert all(len(set(row)) == N for row in grp.tolist())
+    assert (extw[:, K:] == 1.0).all() and np.array_equal(extw[:, :K], w.weights)
+    # routed experts keep their relative order: e -> S*ne + e
+    assert np.array_equal(ext[:, :K] - S * ne, w.expert_ids)
+
+
+def test_shared_experts_identity_expert_combine():
+    """Identity experts through the widened routing: y = (sum_k w_k + N) * x."""
+    W, S, N, ne, T, K, H = 4, 2, 2, 3, 9, 2, 24
+    E = (W - S) * ne
+    w = wl.moe_workload("tiny", seed=61, W=W, T=T, K=K, E=E, H=H)
+    ext, extw, E_tot, _ = oracle.shared_expert_routing(W, T, K, E, N, S, w.expert_ids, w.weights)
+    lay = oracle.moe_dispatch_layout(W, T, K + N, E_tot, ext)
+    ex, _, fl = oracle.moe_dispatch(w.x_bits, lay["dst_row"], K + N, lay["rows_cap"], 0)
+    y64, fl2 = oracle.moe_combine_f64(ex, lay["dst_row"], extw, K + N)
+    assert fl == 0 and fl2 == 0
+    xf = wl.bf16_bits_to_f32(w.x_bits).astype(np.float64)
+    exp = xf * (w.weights.astype(np.float64).sum(axis=1) + N)[:, None]
+    assert np.allclose(y64, exp, rtol=1e-12, atol=1e-12)
+
+
+def test_shared_experts_argument_rules():
+    ids = np.zeros((8, 2), np.int32)
+    wts = np.ones((8, 2), np.float32)
+    ok = lambda W, E, N, S: oracle.shared_expert_routing(W, 2, 2, E, N, S, ids[:W * 2], wts[:W * 2])[3]
+    assert ok(4, 4, 0, 0) == 0                                   # no shared experts
+    assert ok(4, 4, 1, 0) & oracle.ORC_BAD_ARG                   # N without shared ranks
+    assert ok(4, 4, 2, 1) & oracle.ORC_BAD_ARG                   # S % N != 0
+    assert ok(4, 3, 1, 2) & oracle.ORC_BAD_ARG                   # E % (W - S) != 0
+    assert ok(4, 4, 1, 3) & oracle.ORC_BAD_ARG                   # W % S != 0
+    ext, _, _, _ = oracle.shared_expert_routing(4, 2, 2, 4, 0, 0, ids, wts)
+    assert np.array_equal(ext, ids)
