@@ -555,6 +555,43 @@ def op_sweep(md, torch, device, hbm, reps=10):
                     "rows": R})
         del L
         torch.cuda.empty_cache()
+    # cfg2 with shared experts: 4 of the 8 ranks host one shared-expert replica each
+    # (sharedExpertNum 1), the 64 routed experts live on the other 4; every token also
+    # goes to its shared replica (9 rows per token). Step: widened routing -> layout ->
+    # dispatch -> combine, one graph.
+    w = wl.moe_workload("cfg2", seed=0)
+    S_, N_ = 4, 1
+    ne_ = w.E // (w.W - S_)
+    Kw, Ew = w.K + N_, w.W * ne_
+    ids = torch.from_numpy(w.expert_ids).to(device)
+    wts = torch.from_numpy(w.weights).to(device)
+    x = torch.from_numpy(w.x_bits.view(np.int16)).to(device).view(torch.bfloat16)
+    ext = torch.empty((w.G, Kw), dtype=torch.int32, device=device)
+    extw = torch.empty((w.G, Kw), dtype=torch.float32, device=device)
+    L = md.LayoutBuffers.allocate(w.W, w.T, Kw, Ew, device=device)
+    ex = torch.empty((L.rows_cap, w.H), dtype=torch.bfloat16, device=device)
+    y = torch.empty((w.G, w.H), dtype=torch.bfloat16, device=device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def shared_step():
+        md.shared_expert_routing(ids, wts, w.W, w.T, w.K, w.E, N_, S_, ext, extw, status)
+        md.moe_dispatch_layout(ext, None, L, status)
+        md.moe_dispatch(x, w.H, L, 0, ex, None, status)
+        md.moe_combine(ex, w.H, L, extw, y, status)
+
+    g = capture(torch, shared_step)
+    t = time_graph(torch, g, reps, 3, flush)
+    del g
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, md.status_string(int(status.item()))
+    ms = statistics.mean(t)
+    R = w.G * Kw
+    b = (w.G * w.H * 2 + R * w.H * 2) * 2 + w.G * w.K * 8 + w.G * Kw * 16
+    out.append({"workload": "cfg2+shared(S=4,N=1)", "op": "step", "us": round(ms * 1e3, 2),
+                "tokens/s": round(w.G / (ms / 1e3), 1), "bytes": b,
+                "frac": round(b / ms / 1e6 / hbm, 4)})
+    del ids, wts, x, ext, extw, L, ex, y
+    torch.cuda.empty_cache()
     # raw all-to-all-v, W = 64
     a = wl.a2a_workload(seed=0)
     W, E_ = a.W, a.row_elems

@@ -78,6 +78,8 @@ _layout_noalloc = _sig("moedisp_moe_dispatch_layout_noalloc",
 _dispatch = _sig("moedisp_moe_dispatch",
                  [_P, _I, Dims, ctypes.POINTER(Layout), _I, _P, _P, _P, _P, _I, _P, _P, _P])
 _combine = _sig("moedisp_moe_combine", [_P, _I, Dims, ctypes.POINTER(Layout), _P, _P, _P, _P])
+_shared = _sig("moedisp_shared_expert_routing",
+               [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P])
 _combine_rms = _sig("moedisp_moe_combine_rmsnorm",
                     [_P, _I, Dims, ctypes.POINTER(Layout), _P, _P, _P, ctypes.c_float, _P, _P, _P, _P])
 
@@ -269,6 +271,17 @@ def moe_combine_rmsnorm(expert_out, H, layout: LayoutBuffers, expert_scales, res
     return _check(rc, "moe_combine_rmsnorm", raise_on_error)
 
 
+def shared_expert_routing(expert_ids, expert_scales, W, T, K, E, shared_expert_num,
+                          shared_expert_rank_num, ext_ids, ext_scales, status, stream=None,
+                          raise_on_error=True) -> int:
+    """Widens the routing with the shared experts: ext_ids / ext_scales are [G, K + N];
+    the layout then takes dims (W, T, K + N, W * (E // (W - S)))."""
+    rc = _shared(_ptr(expert_ids), _ptr(expert_scales), int(W), int(T), int(K), int(E),
+                 int(shared_expert_num), int(shared_expert_rank_num), _ptr(ext_ids),
+                 _ptr(ext_scales), _ptr(status), _stream(stream))
+    return _check(rc, "shared_expert_routing", raise_on_error)
+
+
 def raw_selftest(limit_us, status_ptr) -> int:
     return int(_selftest_wait(int(limit_us), status_ptr, None))
 
@@ -279,13 +292,14 @@ def raw_call(name: str, *args) -> int:
                 "moedisp_moe_dispatch_layout": _layout,
                 "moedisp_moe_dispatch_layout_noalloc": _layout_noalloc,
                 "moedisp_moe_dispatch": _dispatch, "moedisp_moe_combine": _combine,
-                "moedisp_moe_combine_rmsnorm": _combine_rms}[name](*args))
+                "moedisp_moe_combine_rmsnorm": _combine_rms,
+                "moedisp_shared_expert_routing": _shared}[name](*args))
 
 
 __all__ = [
     "a2a_exchange_plan", "a2a_v", "layout_workspace_size", "LayoutBuffers",
     "moe_dispatch_layout", "moe_dispatch_layout_noalloc", "moe_dispatch", "moe_combine",
-    "selftest_bounded_wait", "moe_combine_rmsnorm",
+    "selftest_bounded_wait", "moe_combine_rmsnorm", "shared_expert_routing",
     "status_string", "version", "NOALLOC_SCRATCH_BYTES",
     "Dims", "Layout", "MoedispError", "LIBRARY_PATH",
     "QUANT_NONE", "QUANT_INT8", "QUANT_FP8_E4M3",

@@ -318,6 +318,33 @@ int moedisp_moe_combine(const void* expert_out, int H, moedisp_dims dims,
     return rc(moedisp::launch_combine(expert_out, H, dims, L, expert_scales, y, status, stream));
 }
 
+int moedisp_shared_expert_routing(const int32_t* expert_ids, const float* expert_scales, int W,
+                                  int T, int K, int E, int shared_expert_num,
+                                  int shared_expert_rank_num, int32_t* ext_ids, float* ext_scales,
+                                  int32_t* status, moedisp_stream_t stream) {
+    const int N = shared_expert_num, S = shared_expert_rank_num;
+    if (!status) return MOEDISP_ERR_NULLPTR;
+    if (W < 1 || T < 0 || K < 1 || E < 1 || N < 0 || S < 0 || S >= W) return MOEDISP_ERR_INVALID;
+    if ((S == 0) != (N == 0)) return MOEDISP_ERR_INVALID;
+    if (S > 0 && (W % S != 0 || S % N != 0)) return MOEDISP_ERR_INVALID;
+    if (E % (W - S) != 0) return MOEDISP_ERR_INVALID;
+    if (K + N > MOEDISP_MAX_K) return MOEDISP_ERR_UNSUPPORTED;
+    if ((int64_t)W * (E / (W - S)) > MOEDISP_MAX_E) return MOEDISP_ERR_UNSUPPORTED;
+    const int64_t G = (int64_t)W * T;
+    if (G * (K + N) >= (int64_t(1) << 30)) return MOEDISP_ERR_UNSUPPORTED;
+    if (G == 0) return MOEDISP_OK;
+    if (!expert_ids || !expert_scales || !ext_ids || !ext_scales) return MOEDISP_ERR_NULLPTR;
+    if (!aligned(expert_ids, 4) || !aligned(expert_scales, 4) || !aligned(ext_ids, 4) ||
+        !aligned(ext_scales, 4) || !aligned(status, 4))
+        return MOEDISP_ERR_MISALIGNED;
+    const size_t nin = (size_t)G * K * 4, nout = (size_t)G * (K + N) * 4;
+    if (any_alias({{ext_ids, nout}, {ext_scales, nout}, {status, 4}},
+                  {{expert_ids, nin}, {expert_scales, nin}}))
+        return MOEDISP_ERR_ALIASED;
+    return rc(moedisp::launch_shared_routing(expert_ids, expert_scales, W, T, K, E, N, S, ext_ids,
+                                             ext_scales, status, stream));
+}
+
 int moedisp_moe_combine_rmsnorm(const void* expert_out, int H, moedisp_dims dims,
                                 const moedisp_layout* layout, const float* expert_scales,
                                 const void* residual, const float* gamma, float eps,

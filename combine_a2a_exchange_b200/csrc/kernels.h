@@ -93,6 +93,10 @@ cudaError_t launch_combine(const void* expert_out, int H, const moedisp_dims& di
                            const moedisp_layout& layout, const float* expert_scales, void* y,
                            int32_t* status, cudaStream_t stream);
 
+cudaError_t launch_shared_routing(const int32_t* expert_ids, const float* expert_scales, int W,
+                                  int T, int K, int E, int N, int S, int32_t* ext_ids,
+                                  float* ext_scales, int32_t* status, cudaStream_t stream);
+
 cudaError_t launch_combine_rmsnorm(const void* expert_out, int H, const moedisp_dims& dims,
                                    const moedisp_layout& layout, const float* expert_scales,
                                    const void* residual, const float* gamma, float eps,

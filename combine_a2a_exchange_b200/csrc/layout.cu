@@ -117,9 +117,17 @@ __device__ __forceinline__ int64_t padded_rows(int64_t n, int64_t A) {
     return p < A ? A : p;
 }
 
-// Marks an expert's padding rows [first, end), below rows_cap, as holding no slot.
-__device__ __forceinline__ void mark_padding(const LayoutArgs& a, int64_t first, int64_t end) {
-    for (int64_t row = first; row < end && row < a.rows_cap; ++row) a.assist[row] = -1;
+// Marks the padding rows of experts part, part + parts, ... as holding no slot (below
+// rows_cap): each expert's range [ebase[e] + etot[e], ebase[e + 1]) is written by the whole
+// block, coalesced. A no-op without major_align.
+__device__ __forceinline__ void mark_padding(const LayoutArgs& a, const int64_t* ebase,
+                                             const int32_t* etot, int part, int parts) {
+    if (a.align <= 1) return;
+    for (int e = part; e < a.E; e += parts) {
+        const int64_t end = min64(ebase[e + 1], a.rows_cap);
+        for (int64_t row = ebase[e] + etot[e] + threadIdx.x; row < end; row += blockDim.x)
+            a.assist[row] = -1;
+    }
 }
 
 // Bits needed for the keys 0..E (expert + 1, 0 = no expert).
@@ -273,6 +281,7 @@ __global__ void __launch_bounds__(kThreads) layout_rank_kernel(LayoutArgs a) {
     int32_t* pre = wc + kWarps * ES;                             // [E]
     int32_t* colp = pre + E;                                     // [E]
     int32_t* cntr = colp + E;                                    // [E]
+    int32_t* etot = cntr + E;                                    // [E] rows routed to e
     const int tile = blockIdx.x;
     const int r = tile / tpr, c = tile - r * tpr;
     const int64_t base = (int64_t)r * a.P;
@@ -320,12 +329,13 @@ __global__ void __launch_bounds__(kThreads) layout_rank_kernel(LayoutArgs a) {
         const int64_t ex = block_exclusive_scan(seg, warp_tot, chunk);
         if (e < E) {
             ebase[e] = carry + ex;
-            if (tile == 0 && seg > tot) mark_padding(a, carry + ex + tot, carry + ex + seg);
+            etot[e] = (int32_t)tot;
         }
         carry += chunk;
     }
     if (threadIdx.x == 0) ebase[E] = carry;
     __syncthreads();
+    mark_padding(a, ebase, etot, tile, a.n_tiles);
 
     const int64_t R = ebase[E];
     if (tile == 0) {
@@ -367,6 +377,7 @@ layout_cluster_kernel(LayoutArgs a) {
     int32_t* tpre = tcnt + E;                                    // [E] counts in earlier tiles
     int32_t* colp = tpre + E;                                    // [E] counts in earlier ranks
     int32_t* cntr = colp + E;                                    // [E] counts of this rank
+    int32_t* etot = cntr + E;                                    // [E] rows routed to e
 
     const int tile = (int)cluster.block_rank();
     const int C = (int)cluster.num_blocks();
@@ -426,7 +437,7 @@ layout_cluster_kernel(LayoutArgs a) {
         const int64_t ex = block_exclusive_scan(seg, warp_tot, chunk);
         if (e < E) {
             ebase[e] = carry + ex;
-            if (tile == 0 && seg > tot) mark_padding(a, carry + ex + tot, carry + ex + seg);
+            etot[e] = (int32_t)tot;
         }
         carry += chunk;
     }
@@ -435,6 +446,7 @@ layout_cluster_kernel(LayoutArgs a) {
     // (which the others may still be reading) until the matching wait at the end.
     cluster_arrive_release();
     __syncthreads();
+    mark_padding(a, ebase, etot, tile, C);
 
     const int64_t R = ebase[E];
     if (tile == 0) {
@@ -475,7 +487,7 @@ bool cluster_geometry(const moedisp_dims& d, int* tpr, int64_t* tile_len, int* s
 }
 
 size_t cluster_smem(int E) {
-    return (size_t)(E + 1) * sizeof(int64_t) + ((size_t)kCWarps * (E | 1) + 4 * (size_t)E) * sizeof(int32_t);
+    return (size_t)(E + 1) * sizeof(int64_t) + ((size_t)kCWarps * (E | 1) + 5 * (size_t)E) * sizeof(int32_t);
 }
 
 // Whether a cluster of C blocks of this kernel can be resident on the current device.
@@ -529,7 +541,7 @@ cudaError_t launch_tiled(LayoutArgs& a, const moedisp_dims& dims, const LayoutGe
     const int E = dims.E;
     const size_t smem_count = (size_t)E * sizeof(int32_t);
     const size_t smem_rank = (size_t)(E + 1) * sizeof(int64_t) +
-                             ((size_t)kWarps * (E | 1) + 3 * (size_t)E) * sizeof(int32_t);
+                             ((size_t)kWarps * (E | 1) + 4 * (size_t)E) * sizeof(int32_t);
     void (*count)(LayoutArgs) = nullptr;
     void (*rank)(LayoutArgs) = nullptr;
     switch (g.steps) {

@@ -277,6 +277,30 @@ int moedisp_moe_combine(const void *expert_out, int H, moedisp_dims dims,
                         const moedisp_layout *layout, const float *expert_scales, void *y,
                         int32_t *status, moedisp_stream_t stream);
 
+/* shared_expert_routing
+ *
+ * Shared experts (Ascend aclnnMoeDistributeDispatchV2 sharedExpertNum N,
+ * sharedExpertRankNum S, expertShardType 0: shared-expert ranks before the routed-expert
+ * ranks), expressed as a wider routing that the layout, dispatch and combine take as is.
+ * The first S of the W ranks each host one shared-expert replica (S / N replicas of each of
+ * the N shared experts, grouped by shared expert); the other W - S ranks host the E routed
+ * experts, ne = E / (W - S) each. In the uniform expert space of W * ne experts:
+ *   routed expert e          -> S * ne + e    (an id outside [0, E) -> W * ne, still out
+ *                                              of range: BAD_EXPERT_ID at the layout)
+ *   shared expert j, token of source rank r -> (j * (S / N) + r mod (S / N)) * ne
+ * (the pages fix only the counts -- a shared rank receives T * W * N / S tokens; the
+ * replica of a source rank is this library's choice). Outputs, [G][K + N] each:
+ * ext_ids int32 (the K routed slots, then the N shared ones) and ext_scales fp32 (the
+ * given weights, then 1). Then call moe_dispatch_layout, moe_dispatch and moe_combine with
+ * dims {W, T, K + N, W * ne}; a shared rank's ne - 1 other local experts stay empty.
+ * Rules: N = 0 exactly when S = 0; S < W, W % S == 0, S % N == 0, E % (W - S) == 0
+ * (else MOEDISP_ERR_INVALID); K + N <= MOEDISP_MAX_K and W * ne <= MOEDISP_MAX_E (else
+ * MOEDISP_ERR_UNSUPPORTED). Out-of-range ids set MOEDISP_STATUS_BAD_EXPERT_ID. */
+int moedisp_shared_expert_routing(const int32_t *expert_ids, const float *expert_scales, int W,
+                                  int T, int K, int E, int shared_expert_num,
+                                  int shared_expert_rank_num, int32_t *ext_ids,
+                                  float *ext_scales, int32_t *status, moedisp_stream_t stream);
+
 /* moe_combine_rmsnorm
  *
  * The combine fused with the residual add and RMSNorm that follow it (the FlashInfer

@@ -203,3 +203,23 @@ def test_binding_has_no_fallback():
     for f in glob.glob(os.path.join(ROOT, "combine_a2a_exchange_b200", "**", "*.py"), recursive=True):
         text = open(f).read()
         assert "import oracle" not in text and "from oracle" not in text, f
+
+
+def test_shared_expert_routing_rejections(md):
+    ids, w, eo, ew, st = (FAKE + (i << 20) for i in (64, 128, 192, 256, 320))
+    call = lambda W, T, K, E, N, S, ids=ids, w=w, eo=eo, ew=ew, st=st: md.raw_call(
+        "moedisp_shared_expert_routing", ids, w, W, T, K, E, N, S, eo, ew, st, None)
+    assert call(8, 4, 2, 64, 1, 0) == md.MOEDISP_ERR_INVALID        # N without shared ranks
+    assert call(8, 4, 2, 64, 0, 4) == md.MOEDISP_ERR_INVALID        # shared ranks, N = 0
+    assert call(8, 4, 2, 64, 3, 4) == md.MOEDISP_ERR_INVALID        # S % N
+    assert call(8, 4, 2, 64, 1, 3) == md.MOEDISP_ERR_INVALID        # W % S
+    assert call(8, 4, 2, 62, 1, 4) == md.MOEDISP_ERR_INVALID        # E % (W - S)
+    assert call(8, 4, 2, 64, 1, 8) == md.MOEDISP_ERR_INVALID        # S < W
+    assert call(8, 4, 16, 64, 1, 4) == md.MOEDISP_ERR_UNSUPPORTED   # K + N > 16
+    assert call(8, 4, 2, 1024, 1, 4) == md.MOEDISP_ERR_UNSUPPORTED  # W * ne > 1024
+    assert call(8, 4, 2, 64, 1, 4, ids=None) == md.MOEDISP_ERR_NULLPTR
+    assert call(8, 4, 2, 64, 1, 4, st=None) == md.MOEDISP_ERR_NULLPTR
+    assert call(8, 4, 2, 64, 1, 4, eo=ids + 64) == md.MOEDISP_ERR_ALIASED
+    assert call(8, 4, 2, 64, 1, 4, ew=eo + 4) == md.MOEDISP_ERR_ALIASED   # outputs overlap
+    assert call(8, 4, 2, 64, 1, 4, eo=eo + 2) == md.MOEDISP_ERR_MISALIGNED
+    assert call(8, 0, 2, 64, 1, 4, ids=None, w=None, eo=None, ew=None) == md.MOEDISP_OK

@@ -733,6 +733,63 @@ def test_combine_rmsnorm_full_size_sampled(md, name):
                           w.K, bits_host(res[tk]), gamma.cpu().numpy(), max(rows.size, 1))
 
 
+# ---------------------------------------------------------------- shared experts
+
+SHARED_CASES = [(8, 4, 1, 16, 256, 8, 4096, 0), (8, 4, 2, 4, 100, 6, 512, 2),
+                (6, 3, 3, 2, 77, 3, 2048, 3), (16, 8, 4, 8, 64, 4, 256, 0)]
+
+
+@pytest.mark.parametrize("W,S,N,ne,T,K,H,q", SHARED_CASES)
+def test_shared_experts_end_to_end(md, W, S, N, ne, T, K, H, q):
+    """Widened routing bit-exact against the oracle, then layout, dispatch and combine of
+    the widened problem against the oracle's composition."""
+    E = (W - S) * ne
+    w = wl.moe_workload("tiny", seed=62, W=W, T=T, K=K, E=E, H=H, active_p=0.9)
+    ext_ref, extw_ref, E_tot, fl = oracle.shared_expert_routing(W, T, K, E, N, S, w.expert_ids,
+                                                                w.weights)
+    assert fl == 0
+    G = W * T
+    ext = torch.empty((G, K + N), dtype=torch.int32, device="cuda")
+    extw = torch.empty((G, K + N), dtype=torch.float32, device="cuda")
+    st = new_status()
+    md.shared_expert_routing(dev(w.expert_ids), dev(w.weights), W, T, K, E, N, S, ext, extw, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert np.array_equal(ext.cpu().numpy(), ext_ref)
+    assert np.array_equal(extw.cpu().numpy().view(np.uint32), extw_ref.view(np.uint32))
+    wide = wl.MoEWorkload(**{**w.__dict__, "K": K + N, "E": E_tot, "expert_ids": ext_ref,
+                             "weights": extw_ref, "quant_mode": q})
+    L, st0 = run_layout(md, wide)
+    ref = oracle.moe_dispatch_layout(W, T, K + N, E_tot, ext_ref, w.active)
+    assert st0 == 0
+    assert_layout_equal(layout_host(L), ref, ref["R"], ref["rows_cap"])
+    full, scales, gr, _, _, st1 = run_dispatch(md, wide, L, q)
+    assert st1 == 0
+    rex, rsc, _ = oracle.moe_dispatch(w.x_bits, ref["dst_row"], K + N, ref["rows_cap"], q)
+    R = ref["R"]
+    assert np.array_equal(full.cpu().numpy()[gr:gr + R].view(rex.dtype), rex[:R])
+    eo = wl.expert_rows(L.rows_cap, H, seed=63)
+    y, st2 = run_combine(md, L, eo, wide)
+    assert st2 == 0
+    check_combine(y, eo, ref["dst_row"], extw_ref, K + N, L.rows_cap)
+
+
+def test_shared_experts_bad_id(md):
+    W, S, N, ne, T, K = 4, 2, 1, 3, 10, 2
+    E = (W - S) * ne
+    w = wl.moe_workload("tiny", seed=64, W=W, T=T, K=K, E=E)
+    ids = w.expert_ids.copy()
+    ids[3, 1] = E
+    ext = torch.empty((W * T, K + N), dtype=torch.int32, device="cuda")
+    extw = torch.empty((W * T, K + N), dtype=torch.float32, device="cuda")
+    st = new_status()
+    md.shared_expert_routing(dev(ids), dev(w.weights), W, T, K, E, N, S, ext, extw, st)
+    torch.cuda.synchronize()
+    ref, _, _, fl = oracle.shared_expert_routing(W, T, K, E, N, S, ids, w.weights)
+    assert int(st.item()) == md.STATUS_BAD_EXPERT_ID and fl & oracle.ORC_BAD_EXPERT
+    assert np.array_equal(ext.cpu().numpy(), ref)
+
+
 # --------------------------------------------------------------- end to end
 
 @pytest.mark.parametrize("name,over,q", [("tiny", {}, 0), ("cfg2", {}, 0),
