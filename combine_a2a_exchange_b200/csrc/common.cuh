@@ -116,14 +116,6 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, 
         : "memory");
 }
 
-// Hint: bring a global range into L2. Coherent by construction (L2 is the device's point of
-// coherence), so it may be issued before the grid dependency wait, on data an earlier kernel
-// may still be writing.
-__device__ __forceinline__ void bulk_prefetch_l2(const void* gmem_src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gmem_src), "r"(bytes)
-                 : "memory");
-}
-
 __device__ __forceinline__ void bulk_store(void* gmem_dst, const void* smem_src, uint32_t bytes) {
     asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gmem_dst),
                  "r"(smem_addr(smem_src)), "r"(bytes)

@@ -69,18 +69,34 @@ __device__ __forceinline__ float absmax8(const uint4& v) {
 // int8 boundaries are the half-integers; |x/scale| <= ~127, so the bound above is below
 // 2.3e-5 and a margin of 2^-14 from k + 0.5 is safe. Rounding to an integer uses the
 // floating-point adder: for |v| < 2^22, rr = v + 1.5*2^23 rounds v's fraction away to the
-// nearest integer, ties to even, and rr's bit pattern is that of 1.5*2^23 plus the integer,
-// whose low byte is therefore the integer's two's-complement low byte -- the int8 code.
-// The clamp to +-127 can only act when the scale itself is inexact far beyond fp32's
-// rounding (subnormal scales); the fast path is taken only for |r| < 127.5, where it
-// cannot act, and the slow path clamps. Returns a word whose low byte is the code.
-__device__ __forceinline__ uint32_t q_int8(float x, float scale, float inv) {
+// nearest integer, ties to even, and rr's bit pattern is that of 1.5*2^23 plus the
+// integer. Two exact formulations follow; each kernel uses the one measured faster in it.
+//
+// q_int8: the integer, clamped to +-127 (the clamp acts only when the scale itself is
+// inexact far beyond fp32 rounding, i.e. subnormal).
+__device__ __forceinline__ int q_int8(float x, float scale, float inv) {
     constexpr float kMagic = 12582912.0f;                    // 1.5 * 2^23
+    float v = __fmul_rn(x, inv);
+    float rr = __fadd_rn(v, kMagic);
+    const float t = __fsub_rn(v, __fsub_rn(rr, kMagic));      // v - round(v), in [-0.5, 0.5]
+    if (!(0.5f - fabsf(t) >= 0.00006103515625f)) {            // near k + 0.5, or not finite
+        v = __fdiv_rn(x, scale);
+        if (!(fabsf(v) < 4194304.0f)) return v > 0.0f ? 127 : -127;   // |v| >= 2^22 or NaN
+        rr = __fadd_rn(v, kMagic);
+    }
+    const int q = (int)(__float_as_uint(rr) - __float_as_uint(kMagic));
+    return max(-127, min(127, q));
+}
+
+// q_int8_w: a word whose low byte is the code -- rr's own bits when |r| < 127.5, where
+// the clamp cannot act (the low byte of 1.5*2^23 + q is q's two's-complement low byte);
+// else the IEEE quotient, clamped (NaN -> -127).
+__device__ __forceinline__ uint32_t q_int8_w(float x, float scale, float inv) {
+    constexpr float kMagic = 12582912.0f;
     const float v = __fmul_rn(x, inv);
     const float rr = __fadd_rn(v, kMagic);
-    const float t = __fsub_rn(v, __fsub_rn(rr, kMagic));      // v - round(v), in [-0.5, 0.5]
+    const float t = __fsub_rn(v, __fsub_rn(rr, kMagic));
     if (0.5f - fabsf(t) >= 0.00006103515625f && fabsf(v) < 127.5f) return __float_as_uint(rr);
-    // near k + 0.5, out of range or not finite: the IEEE quotient, clamped (NaN -> -127)
     const float q = fminf(fmaxf(__fdiv_rn(x, scale), -127.0f), 127.0f);
     return __float_as_uint(__fadd_rn(q, kMagic));
 }
@@ -106,7 +122,7 @@ __device__ __forceinline__ uint32_t q_e4m3(float x, float scale, float inv) {
 
 template <int Q>
 __device__ __forceinline__ uint32_t q_code(float x, float scale, float inv) {
-    return Q == MOEDISP_QUANT_INT8 ? q_int8(x, scale, inv) : q_e4m3(x, scale, inv);
+    return Q == MOEDISP_QUANT_INT8 ? q_int8_w(x, scale, inv) : q_e4m3(x, scale, inv);
 }
 
 // The low bytes of four words, in order, in one word (three byte permutes).
@@ -135,15 +151,27 @@ __device__ __forceinline__ void smooth8(const uint4& v, const float4* s, float (
     o[6] = __fmul_rn(bf16_lo(v.w), s1.z); o[7] = __fmul_rn(bf16_hi(v.w), s1.w);
 }
 
-// Eight bf16 values (a row chunk) to eight codes.
+__device__ __forceinline__ uint32_t q_int8_pair(uint32_t w, float scale, float inv) {
+    const int a = q_int8(bf16_lo(w), scale, inv);
+    const int b = q_int8(bf16_hi(w), scale, inv);
+    return (uint32_t)(a & 0xff) | ((uint32_t)(b & 0xff) << 8);
+}
+
+// Eight bf16 values (a row chunk) to eight codes: int8 as pairs of clamped integers,
+// e4m3 through byte permutes (each measured the faster in the token-order kernel).
 template <int Q>
 __device__ __forceinline__ uint2 quant8(const uint4& v, float scale, float inv, bool zero) {
     if (zero) return make_uint2(0u, 0u);
+    if (Q == MOEDISP_QUANT_INT8) {
+        const uint32_t p0 = q_int8_pair(v.x, scale, inv), p1 = q_int8_pair(v.y, scale, inv);
+        const uint32_t p2 = q_int8_pair(v.z, scale, inv), p3 = q_int8_pair(v.w, scale, inv);
+        return make_uint2(p0 | (p1 << 16), p2 | (p3 << 16));
+    }
     const float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
                         bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
     uint32_t b[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) b[j] = q_code<Q>(f[j], scale, inv);
+    for (int j = 0; j < 8; ++j) b[j] = q_e4m3(f[j], scale, inv);
     return make_uint2(pack_low_bytes(b[0], b[1], b[2], b[3]), pack_low_bytes(b[4], b[5], b[6], b[7]));
 }
 
@@ -191,12 +219,6 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
         fence_mbar_init();
     }
     __syncwarp();
-    // The first rows this block will load go to L2 while the kernel this one depends on
-    // (normally the layout, which moves little data) is still running.
-    if (lane < S) {
-        const int64_t g = (int64_t)blockIdx.x + (int64_t)lane * gridDim.x;
-        if (g < a.G) bulk_prefetch_l2(a.x + g * a.in_bytes, a.in_bytes);
-    }
     grid_dep_wait();
     grid_dep_launch_dependents();
     write_recv_counts(a);
@@ -316,11 +338,6 @@ __global__ void __launch_bounds__(kQuantThreads, 2) dispatch_quant_kernel(Dispat
     }
     if (tid == 0) next_s = 0;
     __syncthreads();
-    // L2 prefetch of the block's first NG * S token rows (see dispatch_copy_kernel).
-    if (tid < NG * S) {
-        const int64_t g = (int64_t)blockIdx.x + (int64_t)tid * gridDim.x;
-        if (g < a.G) bulk_prefetch_l2(a.x + g * a.in_bytes, a.in_bytes);
-    }
     grid_dep_wait();
     grid_dep_launch_dependents();
     write_recv_counts(a);

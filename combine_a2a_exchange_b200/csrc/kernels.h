@@ -21,6 +21,15 @@ cudaError_t allow_dynamic_smem(const void* kernel);
 // (at least 1; cached per device). Also calls allow_dynamic_smem.
 cudaError_t blocks_per_sm(const void* kernel, int threads, size_t smem, int* out);
 
+// Grid for `items` equal work items spread by a grid-stride loop over at most `max_grid`
+// resident blocks: the fewest items per block that fit, and the fewest blocks that then
+// cover them, so that every block gets the same count (no last-wave tail).
+inline int64_t balanced_grid(int64_t items, int64_t max_grid) {
+    if (items <= 0 || max_grid <= 0) return 1;
+    const int64_t per = (items + max_grid - 1) / max_grid;
+    return (items + per - 1) / per;
+}
+
 // Launches `kernel` with programmatic stream serialization (and a 1-D cluster of
 // `cluster` blocks when cluster > 1) and returns the launch status.
 template <typename... KArgs, typename... Args>
