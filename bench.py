@@ -592,6 +592,57 @@ def op_sweep(md, torch, device, hbm, reps=10):
                 "frac": round(b / ms / 1e6 / hbm, 4)})
     del ids, wts, x, ext, extw, L, ex, y
     torch.cuda.empty_cache()
+    # exchange -> dispatch: the tokens of W = 8 ranks are first exchanged (splits ~
+    # randint[0, 512)), then dispatched by the receivers' routing (H = 4096 bf16, E = 64,
+    # K = 8). Sequential: a2a_v into a receive buffer, then dispatch from it. Without a
+    # receive buffer: a2a_token_rows, then moe_dispatch_gather straight from the senders'
+    # buffer. Both graphs: plan, receive map (the layout's mask), layout, exchange/dispatch.
+    a = wl.a2a_workload(seed=3, W=8, max_split=512, zero_frac=0.1, row_elems=4096)
+    W_, H_, K_, E_ = a.W, 4096, 8, 64
+    cap_in, T_ = a.cap_in, a.cap_out
+    w = wl.moe_workload("tiny", seed=4, W=W_, T=T_, K=K_, E=E_, H=8)
+    S = torch.from_numpy(a.in_splits).to(device)
+    g0 = torch.Generator(device=device).manual_seed(5)
+    xin = torch.randn((W_ * cap_in, H_), generator=g0, device=device).to(torch.bfloat16)
+    recv = torch.empty((W_ * T_, H_), dtype=torch.bfloat16, device=device)
+    ids = torch.from_numpy(w.expert_ids.reshape(-1)).to(device)
+    plan = [torch.empty((W_, W_), dtype=torch.int64, device=device) for _ in range(3)]
+    tr = torch.empty(W_ * T_, dtype=torch.int64, device=device)
+    act = torch.empty(W_ * T_, dtype=torch.uint8, device=device)
+    L = md.LayoutBuffers.allocate(W_, T_, K_, E_, device=device)
+    ex = torch.empty((L.rows_cap, H_), dtype=torch.bfloat16, device=device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def front():
+        md.a2a_exchange_plan(S, plan[0], plan[1], plan[2], status)
+        md.a2a_token_rows(plan[0], plan[1], plan[2], W_, T_, cap_in, tr, status, active=act)
+        md.moe_dispatch_layout(ids, act, L, status)
+
+    def sequential():
+        front()
+        md.a2a_v(xin, cap_in, recv, T_, 2 * H_, W_, plan[0], plan[1], plan[2], status)
+        md.moe_dispatch(recv, H_, L, 0, ex, None, status)
+
+    def fused():
+        front()
+        md.moe_dispatch_gather(xin, W_ * cap_in, tr, H_, L, 0, ex, None, status)
+
+    res = {}
+    for nm, fn in (("sequential", sequential), ("no_receive_buffer", fused)):
+        g = capture(torch, fn)
+        res[nm] = statistics.mean(time_graph(torch, g, reps, 3, flush))
+        del g
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, md.status_string(int(status.item()))
+    n_recv = int(a.in_splits.sum())
+    R = int(L.expert_base[-1].item())
+    b_fused = n_recv * H_ * 2 + R * H_ * 2
+    for nm, ms in res.items():
+        out.append({"workload": "a2a8->dispatch", "op": nm, "us": round(ms * 1e3, 2),
+                    "tokens/s": round(n_recv / (ms / 1e3), 1),
+                    "bytes_min": b_fused, "frac_of_min": round(b_fused / ms / 1e6 / hbm, 4)})
+    del xin, recv, ex, L
+    torch.cuda.empty_cache()
     # raw all-to-all-v, W = 64
     a = wl.a2a_workload(seed=0)
     W, E_ = a.W, a.row_elems

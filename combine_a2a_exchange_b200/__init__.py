@@ -78,6 +78,11 @@ _layout_noalloc = _sig("moedisp_moe_dispatch_layout_noalloc",
 _dispatch = _sig("moedisp_moe_dispatch",
                  [_P, _I, Dims, ctypes.POINTER(Layout), _I, _P, _P, _P, _P, _I, _P, _P, _P])
 _combine = _sig("moedisp_moe_combine", [_P, _I, Dims, ctypes.POINTER(Layout), _P, _P, _P, _P])
+_dispatch_gather = _sig("moedisp_moe_dispatch_gather",
+                        [_P, ctypes.c_int64, _P, _I, Dims, ctypes.POINTER(Layout), _I, _P, _P, _P,
+                         _P, _I, _P, _P, _P])
+_token_rows = _sig("moedisp_a2a_token_rows",
+                   [_P, _P, _P, _I, ctypes.c_int64, ctypes.c_int64, _P, _P, _P, _P])
 _shared = _sig("moedisp_shared_expert_routing",
                [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P])
 _combine_rms = _sig("moedisp_moe_combine_rmsnorm",
@@ -271,6 +276,29 @@ def moe_combine_rmsnorm(expert_out, H, layout: LayoutBuffers, expert_scales, res
     return _check(rc, "moe_combine_rmsnorm", raise_on_error)
 
 
+def moe_dispatch_gather(x, x_rows, token_rows, H, layout: LayoutBuffers, quant_mode, expand_x,
+                        dynamic_scales, status, expert_token_nums=None, expert_token_nums_type=1,
+                        ep_recv_counts=None, stream=None, raise_on_error=True,
+                        smooth_scales=None) -> int:
+    """moe_dispatch with token g read from row token_rows[g] of x ([x_rows, H])."""
+    L = layout.struct()
+    rc = _dispatch_gather(_ptr(x), int(x_rows), _ptr(token_rows), int(H), layout.dims,
+                          ctypes.byref(L), int(quant_mode), _ptr(smooth_scales), _ptr(expand_x),
+                          _ptr(dynamic_scales), _ptr(expert_token_nums),
+                          int(expert_token_nums_type), _ptr(ep_recv_counts), _ptr(status),
+                          _stream(stream))
+    return _check(rc, "moe_dispatch_gather", raise_on_error)
+
+
+def a2a_token_rows(src_offsets, out_splits, dst_offsets, W, T, in_rank_stride_rows, token_rows,
+                   status, active=None, stream=None, raise_on_error=True) -> int:
+    """Source row of every receive position of an exchange plan (-1 where none)."""
+    rc = _token_rows(_ptr(src_offsets), _ptr(out_splits), _ptr(dst_offsets), int(W), int(T),
+                     int(in_rank_stride_rows), _ptr(token_rows), _ptr(active), _ptr(status),
+                     _stream(stream))
+    return _check(rc, "a2a_token_rows", raise_on_error)
+
+
 def shared_expert_routing(expert_ids, expert_scales, W, T, K, E, shared_expert_num,
                           shared_expert_rank_num, ext_ids, ext_scales, status, stream=None,
                           raise_on_error=True) -> int:
@@ -293,13 +321,16 @@ def raw_call(name: str, *args) -> int:
                 "moedisp_moe_dispatch_layout_noalloc": _layout_noalloc,
                 "moedisp_moe_dispatch": _dispatch, "moedisp_moe_combine": _combine,
                 "moedisp_moe_combine_rmsnorm": _combine_rms,
-                "moedisp_shared_expert_routing": _shared}[name](*args))
+                "moedisp_shared_expert_routing": _shared,
+                "moedisp_moe_dispatch_gather": _dispatch_gather,
+                "moedisp_a2a_token_rows": _token_rows}[name](*args))
 
 
 __all__ = [
     "a2a_exchange_plan", "a2a_v", "layout_workspace_size", "LayoutBuffers",
     "moe_dispatch_layout", "moe_dispatch_layout_noalloc", "moe_dispatch", "moe_combine",
     "selftest_bounded_wait", "moe_combine_rmsnorm", "shared_expert_routing",
+    "moe_dispatch_gather", "a2a_token_rows",
     "status_string", "version", "NOALLOC_SCRATCH_BYTES",
     "Dims", "Layout", "MoedispError", "LIBRARY_PATH",
     "QUANT_NONE", "QUANT_INT8", "QUANT_FP8_E4M3",

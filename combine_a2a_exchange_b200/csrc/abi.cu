@@ -82,6 +82,71 @@ const char* const kStatusNames[16] = {
 
 }  // namespace
 
+namespace {
+// moe_dispatch and moe_dispatch_gather: token g's row is token_rows[g] of x (x_rows rows),
+// or row g when token_rows is null (x_rows = G).
+int dispatch_impl(const void* x, int64_t x_rows, const int64_t* token_rows, int H, moedisp_dims dims,
+                         const moedisp_layout* layout, int quant_mode,
+                         const float* smooth_scales, void* expand_x,
+                         float* dynamic_scales, int64_t* expert_token_nums,
+                         int expert_token_nums_type, int32_t* ep_recv_counts,
+                         int32_t* status, moedisp_stream_t stream) {
+    if (!layout || !status) return MOEDISP_ERR_NULLPTR;
+    int c = check_dims(dims);
+    if (c != MOEDISP_OK) return c;
+    const moedisp_layout& L = *layout;
+    if ((c = check_rows_cap(L.rows_cap)) != MOEDISP_OK) return c;
+    if (quant_mode != MOEDISP_QUANT_NONE && quant_mode != MOEDISP_QUANT_INT8 &&
+        quant_mode != MOEDISP_QUANT_FP8_E4M3)
+        return MOEDISP_ERR_INVALID;
+    if (expert_token_nums && expert_token_nums_type != 0 && expert_token_nums_type != 1)
+        return MOEDISP_ERR_INVALID;
+    if (smooth_scales && quant_mode == MOEDISP_QUANT_NONE) return MOEDISP_ERR_INVALID;
+    if (H <= 0) return MOEDISP_ERR_INVALID;
+    if (H > MOEDISP_MAX_H) return MOEDISP_ERR_UNSUPPORTED;
+    if (H % (quant_mode == MOEDISP_QUANT_NONE ? 8 : 16) != 0) return MOEDISP_ERR_MISALIGNED;
+    const int64_t G = (int64_t)dims.W * dims.T;
+    const int64_t slots = G * dims.K;
+    if (G > 0 && (!x || !L.dst_row)) return MOEDISP_ERR_NULLPTR;
+    if (x_rows < 0) return MOEDISP_ERR_INVALID;
+    if (smooth_scales && L.rows_cap > 0 && (!L.assist_info || !L.expert_base))
+        return MOEDISP_ERR_NULLPTR;
+    if (L.rows_cap > 0 && !expand_x) return MOEDISP_ERR_NULLPTR;
+    if (quant_mode != MOEDISP_QUANT_NONE && L.rows_cap > 0 && !dynamic_scales)
+        return MOEDISP_ERR_NULLPTR;
+    if (expert_token_nums && (!L.expert_base || !L.rank_base)) return MOEDISP_ERR_NULLPTR;
+    if (ep_recv_counts && (!L.cnt || !L.expert_base)) return MOEDISP_ERR_NULLPTR;
+    if (!aligned(x, 16) || !aligned(expand_x, 16) || !aligned(L.dst_row, 4) ||
+        !aligned(dynamic_scales, 4) || !aligned(expert_token_nums, 8) ||
+        !aligned(ep_recv_counts, 4) || !aligned(status, 4) || !aligned(smooth_scales, 16) ||
+        !aligned(L.assist_info, 4) || !aligned(L.expert_base, 8) || !aligned(token_rows, 8))
+        return MOEDISP_ERR_MISALIGNED;
+    const size_t out_row = quant_mode == MOEDISP_QUANT_NONE ? (size_t)H * 2 : (size_t)H;
+    const int ne = dims.E / dims.W;
+    const Span scales{quant_mode == MOEDISP_QUANT_NONE ? nullptr : dynamic_scales,
+                      (size_t)L.rows_cap * 4};
+    if (any_alias({{expand_x, (size_t)L.rows_cap * out_row},
+                   scales,
+                   {expert_token_nums, (size_t)dims.E * 8},
+                   {ep_recv_counts, (size_t)dims.W * ne * dims.W * 4},
+                   {status, 4}},
+                  {{x, (size_t)x_rows * H * 2},
+                   {token_rows, (size_t)G * 8},
+                   {L.dst_row, (size_t)slots * 4},
+                   {smooth_scales, (size_t)dims.E * H * 4},
+                   {smooth_scales ? L.assist_info : nullptr, (size_t)L.rows_cap * 4},
+                   {L.cnt, (size_t)dims.W * dims.E * 4},
+                   {L.expert_base, (size_t)(dims.E + 1) * 8},
+                   {L.rank_base, (size_t)(dims.W + 1) * 8}}))
+        return MOEDISP_ERR_ALIASED;
+    return rc(moedisp::launch_dispatch(x, x_rows, token_rows, H, dims, L, quant_mode, smooth_scales,
+                                       expand_x,
+                                       dynamic_scales,
+                                       expert_token_nums, expert_token_nums_type, ep_recv_counts,
+                                       status, stream));
+}
+}  // namespace
+
 extern "C" {
 
 const char* moedisp_status_string(int code) {
@@ -241,56 +306,42 @@ int moedisp_moe_dispatch(const void* x, int H, moedisp_dims dims,
                          float* dynamic_scales, int64_t* expert_token_nums,
                          int expert_token_nums_type, int32_t* ep_recv_counts,
                          int32_t* status, moedisp_stream_t stream) {
-    if (!layout || !status) return MOEDISP_ERR_NULLPTR;
-    int c = check_dims(dims);
-    if (c != MOEDISP_OK) return c;
-    const moedisp_layout& L = *layout;
-    if ((c = check_rows_cap(L.rows_cap)) != MOEDISP_OK) return c;
-    if (quant_mode != MOEDISP_QUANT_NONE && quant_mode != MOEDISP_QUANT_INT8 &&
-        quant_mode != MOEDISP_QUANT_FP8_E4M3)
-        return MOEDISP_ERR_INVALID;
-    if (expert_token_nums && expert_token_nums_type != 0 && expert_token_nums_type != 1)
-        return MOEDISP_ERR_INVALID;
-    if (smooth_scales && quant_mode == MOEDISP_QUANT_NONE) return MOEDISP_ERR_INVALID;
-    if (H <= 0) return MOEDISP_ERR_INVALID;
-    if (H > MOEDISP_MAX_H) return MOEDISP_ERR_UNSUPPORTED;
-    if (H % (quant_mode == MOEDISP_QUANT_NONE ? 8 : 16) != 0) return MOEDISP_ERR_MISALIGNED;
-    const int64_t G = (int64_t)dims.W * dims.T;
-    const int64_t slots = G * dims.K;
-    if (G > 0 && (!x || !L.dst_row)) return MOEDISP_ERR_NULLPTR;
-    if (smooth_scales && L.rows_cap > 0 && (!L.assist_info || !L.expert_base))
-        return MOEDISP_ERR_NULLPTR;
-    if (L.rows_cap > 0 && !expand_x) return MOEDISP_ERR_NULLPTR;
-    if (quant_mode != MOEDISP_QUANT_NONE && L.rows_cap > 0 && !dynamic_scales)
-        return MOEDISP_ERR_NULLPTR;
-    if (expert_token_nums && (!L.expert_base || !L.rank_base)) return MOEDISP_ERR_NULLPTR;
-    if (ep_recv_counts && (!L.cnt || !L.expert_base)) return MOEDISP_ERR_NULLPTR;
-    if (!aligned(x, 16) || !aligned(expand_x, 16) || !aligned(L.dst_row, 4) ||
-        !aligned(dynamic_scales, 4) || !aligned(expert_token_nums, 8) ||
-        !aligned(ep_recv_counts, 4) || !aligned(status, 4) || !aligned(smooth_scales, 16) ||
-        !aligned(L.assist_info, 4) || !aligned(L.expert_base, 8))
+    return dispatch_impl(x, (int64_t)dims.W * dims.T, nullptr, H, dims, layout, quant_mode,
+                         smooth_scales, expand_x, dynamic_scales, expert_token_nums,
+                         expert_token_nums_type, ep_recv_counts, status, stream);
+}
+
+int moedisp_moe_dispatch_gather(const void* x, int64_t x_rows, const int64_t* token_rows, int H,
+                                moedisp_dims dims, const moedisp_layout* layout, int quant_mode,
+                                const float* smooth_scales, void* expand_x,
+                                float* dynamic_scales, int64_t* expert_token_nums,
+                                int expert_token_nums_type, int32_t* ep_recv_counts,
+                                int32_t* status, moedisp_stream_t stream) {
+    if ((int64_t)dims.W * dims.T > 0 && !token_rows) return MOEDISP_ERR_NULLPTR;
+    return dispatch_impl(x, x_rows, token_rows, H, dims, layout, quant_mode, smooth_scales,
+                         expand_x, dynamic_scales, expert_token_nums, expert_token_nums_type,
+                         ep_recv_counts, status, stream);
+}
+
+int moedisp_a2a_token_rows(const int64_t* src_offsets, const int64_t* out_splits,
+                           const int64_t* dst_offsets, int W, int64_t T,
+                           int64_t in_rank_stride_rows, int64_t* token_rows, uint8_t* active,
+                           int32_t* status, moedisp_stream_t stream) {
+    if (!status) return MOEDISP_ERR_NULLPTR;
+    if (W < 1 || T < 0 || in_rank_stride_rows < 0) return MOEDISP_ERR_INVALID;
+    if (W > MOEDISP_MAX_W) return MOEDISP_ERR_UNSUPPORTED;
+    if ((int64_t)W * T == 0) return MOEDISP_OK;
+    if (!src_offsets || !out_splits || !dst_offsets || !token_rows) return MOEDISP_ERR_NULLPTR;
+    if (!aligned(src_offsets, 8) || !aligned(out_splits, 8) || !aligned(dst_offsets, 8) ||
+        !aligned(token_rows, 8) || !aligned(status, 4))
         return MOEDISP_ERR_MISALIGNED;
-    const size_t out_row = quant_mode == MOEDISP_QUANT_NONE ? (size_t)H * 2 : (size_t)H;
-    const int ne = dims.E / dims.W;
-    const Span scales{quant_mode == MOEDISP_QUANT_NONE ? nullptr : dynamic_scales,
-                      (size_t)L.rows_cap * 4};
-    if (any_alias({{expand_x, (size_t)L.rows_cap * out_row},
-                   scales,
-                   {expert_token_nums, (size_t)dims.E * 8},
-                   {ep_recv_counts, (size_t)dims.W * ne * dims.W * 4},
-                   {status, 4}},
-                  {{x, (size_t)G * H * 2},
-                   {L.dst_row, (size_t)slots * 4},
-                   {smooth_scales, (size_t)dims.E * H * 4},
-                   {smooth_scales ? L.assist_info : nullptr, (size_t)L.rows_cap * 4},
-                   {L.cnt, (size_t)dims.W * dims.E * 4},
-                   {L.expert_base, (size_t)(dims.E + 1) * 8},
-                   {L.rank_base, (size_t)(dims.W + 1) * 8}}))
+    const size_t plan = (size_t)W * W * 8, n = (size_t)W * T;
+    if (any_alias({{token_rows, n * 8}, {active, n}, {status, 4}},
+                  {{src_offsets, plan}, {out_splits, plan}, {dst_offsets, plan}}))
         return MOEDISP_ERR_ALIASED;
-    return rc(moedisp::launch_dispatch(x, H, dims, L, quant_mode, smooth_scales, expand_x,
-                                       dynamic_scales,
-                                       expert_token_nums, expert_token_nums_type, ep_recv_counts,
-                                       status, stream));
+    return rc(moedisp::launch_a2a_token_rows(src_offsets, out_splits, dst_offsets, W, T,
+                                             in_rank_stride_rows, token_rows, active, status,
+                                             stream));
 }
 
 int moedisp_moe_combine(const void* expert_out, int H, moedisp_dims dims,

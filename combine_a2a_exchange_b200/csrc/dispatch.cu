@@ -29,6 +29,8 @@ struct DispatchArgs {
     float* scales;
     const float* smooth;       // [E][H] per-expert smoothing (quantising modes) or null
     const int32_t* assist;     // [rows_cap] slot of each row (the smoothing kernel)
+    const int64_t* rows;       // [G] row of x holding each token, -1 for none; null: row g
+    int64_t x_rows;            // rows of x
     int stages;
     uint32_t in_bytes, out_bytes;
     // receive counts (optional)
@@ -175,6 +177,12 @@ __device__ __forceinline__ uint2 quant8(const uint4& v, float scale, float inv, 
     return make_uint2(pack_low_bytes(b[0], b[1], b[2], b[3]), pack_low_bytes(b[4], b[5], b[6], b[7]));
 }
 
+// Row of x that holds token g (g itself unless a gather map is given), -1 past the end.
+__device__ __forceinline__ int64_t token_source(const DispatchArgs& a, int64_t g) {
+    if (g >= a.G) return -1;
+    return a.rows == nullptr ? g : __ldg(a.rows + g);
+}
+
 __device__ void write_recv_counts(const DispatchArgs& a) {
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     const int64_t first = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -228,12 +236,15 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
     // for a dependent load.
     int64_t pf_g = blockIdx.x;
     int32_t pf_d = (pf_g < a.G && lane < K) ? __ldg(a.dst_row + pf_g * K + lane) : -1;
+    int64_t pf_s = token_source(a, pf_g);
     auto fill = [&](int st) {
         while (true) {
             const int64_t g = pf_g;
             int32_t d = pf_d;
+            const int64_t src = pf_s;
             pf_g = g + gridDim.x;
             pf_d = (pf_g < a.G && lane < K) ? __ldg(a.dst_row + pf_g * K + lane) : -1;
+            pf_s = token_source(a, pf_g);
             if (g >= a.G) {
                 if (lane == 0) {
                     tok[st] = -1;
@@ -247,6 +258,10 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
             }
             if (d < 0) d = -1;
             if (__ballot_sync(0xffffffffu, d >= 0)) {
+                if (src < 0 || src >= a.x_rows) {      // routed, but no row of x holds it
+                    if (lane == 0) raise_status(a.status, MOEDISP_STATUS_BAD_SPLIT);
+                    continue;
+                }
                 int32_t dk[MOEDISP_MAX_K];
 #pragma unroll
                 for (int k = 0; k < MOEDISP_MAX_K; ++k) dk[k] = __shfl_sync(0xffffffffu, d, k);
@@ -256,7 +271,7 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
                         if (k < K) drow[st][k] = dk[k];
                     tok[st] = g;
                     mbar_arrive_expect_tx(&bars[st], a.in_bytes);
-                    bulk_load(inbuf + (size_t)st * a.in_bytes, a.x + g * a.in_bytes, a.in_bytes,
+                    bulk_load(inbuf + (size_t)st * a.in_bytes, a.x + src * a.in_bytes, a.in_bytes,
                               &bars[st]);
                 }
                 return;
@@ -352,19 +367,22 @@ __global__ void __launch_bounds__(kQuantThreads, 2) dispatch_quant_kernel(Dispat
         i = __shfl_sync(0xffffffffu, i, 0);
         return (int64_t)blockIdx.x + (int64_t)i * gridDim.x;
     };
-    int64_t pf_g = 0;
+    int64_t pf_g = 0, pf_s = -1;
     int32_t pf_d = -1;
     if (gw == 0) {
         pf_g = next_token();
         pf_d = (pf_g < a.G && lane < K) ? __ldg(a.dst_row + pf_g * K + lane) : -1;
+        pf_s = token_source(a, pf_g);
     }
     auto fill = [&](int st) {
         while (true) {
             const int64_t g = pf_g;
             int32_t d = pf_d;
+            const int64_t src = pf_s;
             if (g < a.G) {
                 pf_g = next_token();
                 pf_d = (pf_g < a.G && lane < K) ? __ldg(a.dst_row + pf_g * K + lane) : -1;
+                pf_s = token_source(a, pf_g);
             }
             if (g >= a.G) {
                 if (lane == 0) {
@@ -379,6 +397,10 @@ __global__ void __launch_bounds__(kQuantThreads, 2) dispatch_quant_kernel(Dispat
             }
             if (d < 0) d = -1;
             if (__ballot_sync(0xffffffffu, d >= 0)) {
+                if (src < 0 || src >= a.x_rows) {      // routed, but no row of x holds it
+                    if (lane == 0) raise_status(a.status, MOEDISP_STATUS_BAD_SPLIT);
+                    continue;
+                }
                 int32_t dk[MOEDISP_MAX_K];
 #pragma unroll
                 for (int k = 0; k < MOEDISP_MAX_K; ++k) dk[k] = __shfl_sync(0xffffffffu, d, k);
@@ -388,7 +410,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) dispatch_quant_kernel(Dispat
                         if (k < K) drow[grp][st][k] = dk[k];
                     tok[grp][st] = g;
                     mbar_arrive_expect_tx(&gbar[st], a.in_bytes);
-                    bulk_load(inbuf + (size_t)st * a.in_bytes, a.x + g * a.in_bytes, a.in_bytes,
+                    bulk_load(inbuf + (size_t)st * a.in_bytes, a.x + src * a.in_bytes, a.in_bytes,
                               &gbar[st]);
                 }
                 return;
@@ -514,7 +536,12 @@ __global__ void __launch_bounds__(kQuantThreads, CPT > 4 ? 2 : 4) dispatch_smoot
                     if (gt == 0) raise_status(a.status, MOEDISP_STATUS_BAD_EXPERT_ID);
                     continue;
                 }
-                const uint4* xr = x4 + (int64_t)(slot / a.K) * nvec;
+                const int64_t src = token_source(a, slot / a.K);      // same for the group
+                if (src < 0 || src >= a.x_rows) {
+                    if (gt == 0) raise_status(a.status, MOEDISP_STATUS_BAD_SPLIT);
+                    continue;
+                }
+                const uint4* xr = x4 + src * nvec;
                 uint4 v[CPT];
 #pragma unroll
                 for (int j = 0; j < CPT; ++j) {
@@ -641,9 +668,9 @@ cudaError_t launch_quant(const DispatchArgs& a, cudaStream_t stream) {
 
 }  // namespace
 
-cudaError_t launch_dispatch(const void* x, int H, const moedisp_dims& dims,
-                            const moedisp_layout& L, int quant_mode, const float* smooth_scales,
-                            void* expand_x,
+cudaError_t launch_dispatch(const void* x, int64_t x_rows, const int64_t* token_rows, int H,
+                            const moedisp_dims& dims, const moedisp_layout& L, int quant_mode,
+                            const float* smooth_scales, void* expand_x,
                             float* dynamic_scales, int64_t* expert_token_nums,
                             int expert_token_nums_type, int32_t* ep_recv_counts,
                             int32_t* status, cudaStream_t stream) {
@@ -658,6 +685,8 @@ cudaError_t launch_dispatch(const void* x, int H, const moedisp_dims& dims,
     a.scales = dynamic_scales;
     a.smooth = smooth_scales;
     a.assist = L.assist_info;
+    a.rows = token_rows;
+    a.x_rows = x_rows;
     a.stages = 2;
     a.in_bytes = (uint32_t)H * 2u;
     a.out_bytes = quant_mode == MOEDISP_QUANT_NONE ? (uint32_t)H * 2u : (uint32_t)H;

@@ -130,6 +130,63 @@ a2a_v_kernel(const uint8_t* __restrict__ in, int64_t in_stride_rows, uint8_t* __
 
 // ------------------------------------------------------------------ launchers
 
+// Source of every receive position, for a dispatch that reads the exchanged tokens in
+// place (no receive buffer): position p of rank i (p < T, the receive capacity) holds,
+// when it is one of the rows rank i receives, row src_offsets[i][j] + (p - dst_offsets[i][j])
+// of source rank j, where j is the segment holding p (dst_offsets[i] is the exclusive scan
+// of out_splits[i], so j is the last segment starting at or before p); that row is
+// j * in_rank_stride_rows + ... of the concatenated input. Other positions get -1 (and,
+// with an active mask, 0). A segment outside its sender's rows gives -1 and BAD_SPLIT.
+__global__ void __launch_bounds__(kPlanThreads)
+a2a_token_rows_kernel(const int64_t* __restrict__ src_offsets,
+                      const int64_t* __restrict__ out_splits,
+                      const int64_t* __restrict__ dst_offsets, int W, int64_t T,
+                      int64_t in_rank_stride_rows, int64_t* __restrict__ token_rows,
+                      uint8_t* __restrict__ active, int32_t* status) {
+    grid_dep_wait();
+    grid_dep_launch_dependents();
+    const int64_t n = (int64_t)W * T;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    bool bad = false;
+    for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < n; g += stride) {
+        const int i = (int)(g / T);
+        const int64_t p = g - (int64_t)i * T;
+        const int64_t* dst = dst_offsets + (int64_t)i * W;
+        int lo = 0, hi = W;                      // last j with dst[j] <= p (or 0)
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (__ldg(dst + mid) <= p) lo = mid; else hi = mid;
+        }
+        const int64_t q = p - __ldg(dst + lo);
+        const int64_t len = __ldg(out_splits + (int64_t)i * W + lo);
+        int64_t row = -1;
+        if (q >= 0 && q < len) {
+            const int64_t src = __ldg(src_offsets + (int64_t)i * W + lo) + q;
+            if (src >= 0 && src < in_rank_stride_rows) row = (int64_t)lo * in_rank_stride_rows + src;
+            else bad = true;
+        }
+        token_rows[g] = row;
+        if (active != nullptr) active[g] = row >= 0 ? 1 : 0;
+    }
+    if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0)
+        raise_status(status, MOEDISP_STATUS_BAD_SPLIT);
+}
+
+cudaError_t launch_a2a_token_rows(const int64_t* src_offsets, const int64_t* out_splits,
+                                  const int64_t* dst_offsets, int W, int64_t T,
+                                  int64_t in_rank_stride_rows, int64_t* token_rows,
+                                  uint8_t* active, int32_t* status, cudaStream_t stream) {
+    const int64_t n = (int64_t)W * T;
+    int per_sm = 1;
+    cudaError_t err = blocks_per_sm((const void*)a2a_token_rows_kernel, kPlanThreads, 0, &per_sm);
+    if (err != cudaSuccess) return err;
+    int64_t grid = std::max<int64_t>(1, (n + kPlanThreads - 1) / kPlanThreads);
+    grid = std::min<int64_t>(grid, (int64_t)current_sm_count() * per_sm);
+    return launch_pdl(a2a_token_rows_kernel, dim3((unsigned)grid), dim3(kPlanThreads), 0, stream, 1,
+                      src_offsets, out_splits, dst_offsets, W, T, in_rank_stride_rows, token_rows,
+                      active, status);
+}
+
 cudaError_t launch_a2a_plan(const int64_t* in_splits, int W, int64_t* src_offsets,
                             int64_t* out_splits, int64_t* dst_offsets, int32_t* status,
                             cudaStream_t stream) {

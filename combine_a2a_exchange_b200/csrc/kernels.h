@@ -91,7 +91,13 @@ cudaError_t launch_layout_noalloc(const int32_t* expert_ids, const uint8_t* acti
 
 cudaError_t launch_bounded_wait_selftest(uint64_t limit_ns, int32_t* status, cudaStream_t stream);
 
-cudaError_t launch_dispatch(const void* x, int H, const moedisp_dims& dims,
+cudaError_t launch_a2a_token_rows(const int64_t* src_offsets, const int64_t* out_splits,
+                                  const int64_t* dst_offsets, int W, int64_t T,
+                                  int64_t in_rank_stride_rows, int64_t* token_rows,
+                                  uint8_t* active, int32_t* status, cudaStream_t stream);
+
+cudaError_t launch_dispatch(const void* x, int64_t x_rows, const int64_t* token_rows, int H,
+                            const moedisp_dims& dims,
                             const moedisp_layout& layout, int quant_mode,
                             const float* smooth_scales, void* expand_x,
                             float* dynamic_scales, int64_t* expert_token_nums,

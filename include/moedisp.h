@@ -277,6 +277,40 @@ int moedisp_moe_combine(const void *expert_out, int H, moedisp_dims dims,
                         const moedisp_layout *layout, const float *expert_scales, void *y,
                         int32_t *status, moedisp_stream_t stream);
 
+/* moe_dispatch_gather
+ *
+ * moe_dispatch for tokens that stay where they are: token g's row is row token_rows[g]
+ * of x (x: bf16 [x_rows][H]); token_rows int64 [G] device, 8-byte aligned. A routed token
+ * whose token_rows entry is outside [0, x_rows) is skipped and sets
+ * MOEDISP_STATUS_BAD_SPLIT. Everything else is moe_dispatch's (x rows read once, in
+ * place). With a2a_token_rows this is the exchange and the dispatch in one pass: the
+ * PyTorch symm_mem change pipelines its get-style exchange into the index push through
+ * per-block ready counters; on one GPU the received rows need not be materialised at
+ * all, and each row streams from its sender's buffer straight to its K expert rows
+ * (the kernel's own stage barriers are the ready signals). */
+int moedisp_moe_dispatch_gather(const void *x, int64_t x_rows, const int64_t *token_rows, int H,
+                                moedisp_dims dims, const moedisp_layout *layout, int quant_mode,
+                                const float *smooth_scales, void *expand_x,
+                                float *dynamic_scales, int64_t *expert_token_nums,
+                                int expert_token_nums_type, int32_t *ep_recv_counts,
+                                int32_t *status, moedisp_stream_t stream);
+
+/* a2a_token_rows
+ *
+ * The source of every receive position of an exchange plan (a2a_exchange_plan's outputs
+ * src_offsets, out_splits, dst_offsets, [W][W] int64 device), for moe_dispatch_gather over
+ * the received tokens without a receive buffer: position p < T of rank i (T = the
+ * per-rank receive capacity, the dispatch's T) that a2a_v would fill from source rank j
+ * gets row j * in_rank_stride_rows + src_offsets[i][j] + (p - dst_offsets[i][j]) of the
+ * senders' concatenated input (a2a_v's `in`); other positions get -1.
+ * token_rows: int64 [W][T] device; active: uint8 [W][T] device (1 where a row is received,
+ * the layout's per-token mask) or NULL. A segment leaving its sender's rows gives -1 and
+ * MOEDISP_STATUS_BAD_SPLIT. */
+int moedisp_a2a_token_rows(const int64_t *src_offsets, const int64_t *out_splits,
+                           const int64_t *dst_offsets, int W, int64_t T,
+                           int64_t in_rank_stride_rows, int64_t *token_rows, uint8_t *active,
+                           int32_t *status, moedisp_stream_t stream);
+
 /* shared_expert_routing
  *
  * Shared experts (Ascend aclnnMoeDistributeDispatchV2 sharedExpertNum N,

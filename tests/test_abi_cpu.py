@@ -223,3 +223,29 @@ def test_shared_expert_routing_rejections(md):
     assert call(8, 4, 2, 64, 1, 4, ew=eo + 4) == md.MOEDISP_ERR_ALIASED   # outputs overlap
     assert call(8, 4, 2, 64, 1, 4, eo=eo + 2) == md.MOEDISP_ERR_MISALIGNED
     assert call(8, 0, 2, 64, 1, 4, ids=None, w=None, eo=None, ew=None) == md.MOEDISP_OK
+
+
+def test_gather_and_token_rows_rejections(md):
+    L = _layout(md)
+    d = md.Dims(4, 8, 2, 8)
+    x, rows, ex, sc, st = (FAKE + (i << 20) for i in (64, 96, 128, 192, 256))
+    g = lambda x, xr, rows, st=st: md.raw_call(
+        "moedisp_moe_dispatch_gather", x, xr, rows, 128, d, ctypes.byref(L), 0, None, ex, None,
+        None, 1, None, st, None)
+    assert g(x, 100, None) == md.MOEDISP_ERR_NULLPTR                 # no token map
+    assert g(x, -1, rows) == md.MOEDISP_ERR_INVALID                  # x_rows < 0
+    assert g(x, 100, rows + 4) == md.MOEDISP_ERR_MISALIGNED
+    assert g(x, 100, ex + 64) == md.MOEDISP_ERR_ALIASED              # map inside expand_x
+    assert g(x, 1 << 20, rows) == md.MOEDISP_ERR_ALIASED             # x reaches expand_x
+    so, os_, do, tr, act = (FAKE + (i << 20) for i in (300, 320, 340, 360, 380))
+    t = lambda W, T, stride, so=so, tr=tr, act=act, st=st: md.raw_call(
+        "moedisp_a2a_token_rows", so, os_, do, W, T, stride, tr, act, st, None)
+    assert t(0, 4, 10) == md.MOEDISP_ERR_INVALID
+    assert t(4, -1, 10) == md.MOEDISP_ERR_INVALID
+    assert t(4, 4, -1) == md.MOEDISP_ERR_INVALID
+    assert t(4, 4, 10, so=None) == md.MOEDISP_ERR_NULLPTR
+    assert t(4, 4, 10, st=None) == md.MOEDISP_ERR_NULLPTR
+    assert t(4, 4, 10, tr=tr + 4) == md.MOEDISP_ERR_MISALIGNED
+    assert t(4, 4, 10, tr=so) == md.MOEDISP_ERR_ALIASED
+    assert t(4, 4, 10, act=do + 8) == md.MOEDISP_ERR_ALIASED
+    assert t(4, 0, 10, so=None, tr=None) == md.MOEDISP_OK

@@ -733,6 +733,113 @@ def test_combine_rmsnorm_full_size_sampled(md, name):
                           w.K, bits_host(res[tk]), gamma.cpu().numpy(), max(rows.size, 1))
 
 
+# ------------------------------------------- exchange -> dispatch without a receive buffer
+
+def _a2a_case(seed, W, max_split, H, K, ne, zero_frac=0.1):
+    a = wl.a2a_workload(seed=seed, W=W, max_split=max_split, zero_frac=zero_frac, row_elems=H)
+    cap_in, T = a.cap_in, a.cap_out
+    rng = np.random.default_rng(seed + 1)
+    x = wl.f32_to_bf16_bits(rng.standard_normal((W, cap_in, H)).astype(np.float32))
+    w = wl.moe_workload("tiny", seed=seed + 2, W=W, T=T, K=K, E=W * ne, H=H)
+    return a, cap_in, T, x, w
+
+
+def _device_plan(md, S):
+    W = S.shape[0]
+    plan = [torch.empty((W, W), dtype=torch.int64, device="cuda") for _ in range(3)]
+    st = new_status()
+    md.a2a_exchange_plan(dev(S), plan[0], plan[1], plan[2], st)
+    return plan, st
+
+
+@pytest.mark.parametrize("W,max_split,T_extra", [(4, 40, 0), (8, 300, 5), (16, 64, 0), (64, 16, 3)])
+def test_a2a_token_rows_parity(md, W, max_split, T_extra):
+    """The map, checked against the oracle's exchange of an index payload: each input row
+    carries its own row number, so the received buffer holds exactly the map."""
+    a = wl.a2a_workload(seed=W, W=W, max_split=max_split, row_elems=4)
+    cap_in, T = a.cap_in, a.cap_out + T_extra
+    idx = np.arange(W * cap_in, dtype=np.int64).reshape(W, cap_in, 1)
+    src, outs, dsto, fl = oracle.a2a_exchange_plan(a.in_splits)
+    out = np.full((W, T, 1), -1, np.int64)
+    assert oracle.a2a_v(idx, out, src, outs, dsto) == 0 and fl == 0
+    plan, st = _device_plan(md, a.in_splits)
+    tr = torch.full((W, T), -7, dtype=torch.int64, device="cuda")
+    act = torch.full((W, T), 9, dtype=torch.uint8, device="cuda")
+    md.a2a_token_rows(plan[0], plan[1], plan[2], W, T, cap_in, tr, st, active=act)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert np.array_equal(tr.cpu().numpy(), out[:, :, 0])
+    assert np.array_equal(act.cpu().numpy(), (out[:, :, 0] >= 0).astype(np.uint8))
+
+
+@pytest.mark.parametrize("q,smooth", [(0, False), (2, False), (3, False), (2, True)])
+def test_dispatch_of_exchanged_tokens_without_receive_buffer(md, q, smooth):
+    """a2a_token_rows + the layout over the received tokens + moe_dispatch_gather on the
+    senders' buffer equals the oracle's exchange into a receive buffer followed by its
+    dispatch: rows, scales and receive counts bit-exact."""
+    W, K, ne, H = 8, 4, 4, 256
+    a, cap_in, T, x, w = _a2a_case(70, W, 120, H, K, ne)
+    src, outs, dsto, _ = oracle.a2a_exchange_plan(a.in_splits)
+    recv = np.zeros((W, T, H), np.uint16)
+    assert oracle.a2a_v(x, recv, src, outs, dsto) == 0
+    recv_n = outs.sum(axis=1)
+    active = (np.arange(T)[None, :] < recv_n[:, None]).astype(np.uint8).reshape(-1)
+    ref = oracle.moe_dispatch_layout(W, T, K, W * ne, w.expert_ids, active)
+    sm = wl.smooth_scales(W * ne, H, seed=71) if smooth else None
+    rex, rsc, fl = oracle.moe_dispatch(recv.reshape(W * T, H), ref["dst_row"], K, ref["rows_cap"], q,
+                                       smooth=sm, expert_ids=w.expert_ids if smooth else None)
+    assert fl == 0
+    # device: map -> layout (mask from the map) -> gather dispatch from the senders' buffer
+    plan, st = _device_plan(md, a.in_splits)
+    tr = torch.empty(W * T, dtype=torch.int64, device="cuda")
+    act = torch.empty(W * T, dtype=torch.uint8, device="cuda")
+    md.a2a_token_rows(plan[0], plan[1], plan[2], W, T, cap_in, tr, st, active=act)
+    L = md.LayoutBuffers.allocate(W, T, K, W * ne)
+    md.moe_dispatch_layout(dev(w.expert_ids.reshape(-1)), act, L, st)
+    full, scales, gr = alloc_expand(L, H, q)
+    ne_ = ne
+    etn = torch.full((W, ne_), -1, dtype=torch.int64, device="cuda")
+    erc = torch.full((W, ne_, W), -1, dtype=torch.int32, device="cuda")
+    md.moe_dispatch_gather(bf16_dev(x.reshape(W * cap_in, H)), W * cap_in, tr, H, L, q,
+                           full[gr:gr + L.rows_cap], scales[gr:gr + L.rows_cap] if q else None, st,
+                           expert_token_nums=etn, ep_recv_counts=erc,
+                           smooth_scales=None if sm is None else dev(sm))
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert np.array_equal(act.cpu().numpy(), active)
+    R = ref["R"]
+    got = full.cpu().numpy()[gr:gr + R]
+    assert np.array_equal(got.view(rex.dtype) if q == 0 else got, rex[:R])
+    if q:
+        assert np.array_equal(scales.cpu().numpy()[gr:gr + R].view(np.uint32), rsc[:R].view(np.uint32))
+    retn, rerc, _ = oracle.moe_recv_counts(W, W * ne, ref["cnt"], 1)
+    assert np.array_equal(etn.cpu().numpy(), retn) and np.array_equal(erc.cpu().numpy(), rerc)
+
+
+def test_dispatch_gather_bad_rows_are_flagged(md):
+    w = wl.moe_workload("tiny", seed=72, W=2, T=20, K=2, E=4, H=64)
+    L, _ = run_layout(md, w)
+    rows = np.arange(w.G, dtype=np.int64)[::-1].copy()           # reversed gather
+    rows[3] = w.G                                                 # past the end of x
+    rows[7] = -1
+    full, scales, gr = alloc_expand(L, w.H, 0)
+    st = new_status()
+    md.moe_dispatch_gather(bf16_dev(w.x_bits), w.G, dev(rows), w.H, L, 0, full[gr:gr + L.rows_cap],
+                           None, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == md.STATUS_BAD_SPLIT
+    ref = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active)
+    xg = w.x_bits[np.clip(rows, 0, w.G - 1)]
+    rex, _, _ = oracle.moe_dispatch(xg, ref["dst_row"], w.K, ref["rows_cap"], 0)
+    got = full.cpu().numpy().view(np.uint16)[gr:gr + ref["R"]]
+    dr = ref["dst_row"].reshape(w.G, w.K)
+    bad_rows = np.concatenate([dr[3], dr[7]])
+    keep = np.ones(ref["R"], bool)
+    keep[bad_rows[bad_rows >= 0]] = False
+    assert np.array_equal(got[keep], rex[:ref["R"]][keep])
+    assert (got[~keep] == np.uint16(-12345 & 0xFFFF)).all()
+
+
 # ---------------------------------------------------------------- shared experts
 
 SHARED_CASES = [(8, 4, 1, 16, 256, 8, 4096, 0), (8, 4, 2, 4, 100, 6, 512, 2),
