@@ -683,6 +683,54 @@ def op_sweep(md, torch, device, hbm, reps=10):
 
 # ---------------------------------------------------------------------- main
 
+def run_single_op(args, wl, md, torch):
+    """Times one op of the widened path on --workload after the step's layout (and
+    dispatch) ran once: warm-up launches, then --steps launches, each behind an L2 flush.
+    Prints one JSON line. Launch order: the step's kernels once, then the op's."""
+    device = torch.device("cuda", torch.cuda.current_device())
+    w = wl.moe_workload(args.workload, seed=0, **({"T": args.T} if args.T else {}))
+    st = MoEStep(md, torch, w, device)
+    st.run()
+    flush = L2Flush(torch, device)
+    if args.op == "dispatch_smooth":
+        if w.quant_mode == 0:
+            raise SystemExit("dispatch_smooth needs a quantising workload (cfg3, cfg4)")
+        sm = torch.from_numpy(wl.smooth_scales(w.E, w.H, seed=1)).to(device)
+
+        def op():
+            md.moe_dispatch(st.x, w.H, st.L, w.quant_mode, st.ex, st.scales, st.status,
+                            smooth_scales=sm)
+    else:
+        g = torch.Generator(device=device).manual_seed(11)
+        res = torch.randn((w.G, w.H), generator=g, device=device).to(torch.bfloat16)
+        gamma = 0.5 + torch.rand((w.H,), generator=g, device=device)
+        rout = torch.empty_like(res)
+
+        def op():
+            md.moe_combine_rmsnorm(st.expert_out, w.H, st.L, st.wts, res, gamma, 1e-6, st.y,
+                                   st.status, residual_out=rout)
+    Ev = torch.cuda.Event
+    for _ in range(args.warmup):
+        flush.zero_()
+        op()
+    pairs = []
+    for _ in range(args.steps):
+        flush.zero_()
+        a, b = Ev(enable_timing=True), Ev(enable_timing=True)
+        a.record()
+        op()
+        b.record()
+        pairs.append((a, b))
+    torch.cuda.synchronize()
+    stt = int(st.status.item())
+    if stt != 0:
+        raise SystemExit(f"status {md.status_string(stt)}")
+    us = statistics.mean(x.elapsed_time(y) for x, y in pairs) * 1e3
+    print(json.dumps({"op": args.op, "workload": args.workload, "us": round(us, 2),
+                      "steps": args.steps, "warmup": args.warmup}))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -697,6 +745,8 @@ def main():
     ap.add_argument("--no-ops", action="store_true", help="skip the per-op sweep of other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--op", choices=["step", "dispatch_smooth", "combine_rmsnorm"], default="step",
+                    help="time one NEXT-row op alone on --workload (one GPU), e.g. to profile it")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -718,6 +768,8 @@ def main():
     import combine_a2a_exchange_b200 as md
 
     torch.cuda.set_device(local_rank)
+    if args.op != "step":
+        return run_single_op(args, wl, md, torch)
     device = torch.device("cuda", local_rank)
     if world > 1:
         from datetime import timedelta
