@@ -3,12 +3,14 @@
 //
 // The PyTorch symm_mem index push sends one row per (token, expert) with a remote put
 // from the source buffer. On one GPU the K destinations are rows of one expand_x buffer,
-// so each token row is read from HBM exactly once: a persistent block brings the row
-// into shared memory with a 1-D bulk (TMA) load, quantises it there if asked, and the
-// K copies leave shared memory as K bulk stores issued by K lanes in parallel. Each warp
-// runs its own pipeline: it looks ahead through its tokens (skipping tokens with no
-// active slot), keeps up to stages-1 row loads in flight, and reuses a stage only after
-// the bulk stores that read it have drained.
+// so each token row is read from HBM exactly once. Unquantised, a persistent block brings
+// the row into shared memory with a 1-D bulk (TMA) load and the K copies leave as K bulk
+// stores issued by K lanes in parallel; each warp runs its own pipeline, looking ahead
+// through its tokens (skipping tokens with no active slot), keeping up to stages-1 row
+// loads in flight and reusing a stage only after the bulk stores that read it have
+// drained. Quantised, a group of warps gathers the row into registers, quantises it once
+// and writes the codes to the K rows. With per-expert smoothing every output row is
+// quantised on its own, in expand_x's row order.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -314,170 +316,8 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
     if (issuer) bulk_wait<0>();
 }
 
-// Quantising dispatch. A block of kQuantThreads threads is split into token groups of WPT
-// warps; each group is an independent pipeline over the tokens it draws from the block's
-// share, with its own shared-memory stages and barriers. The group's first lane streams token rows into the
-// stages (bulk loads); the group reduces the row's max |x| (warp shuffles, plus a named
-// barrier across the group's warps when WPT > 1 -- that barrier also carries the
-// time-out verdict), then each thread quantises its 16-byte chunks of the row and writes
-// the 8-byte results straight to the token's K rows (a warp covers 256 contiguous bytes
-// of a row per store). The previous token's stage is refilled after the barrier.
-constexpr int kChunks = 8;
-
 __device__ __forceinline__ void group_barrier(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
-}
-
-template <int Q, int WPT>
-__global__ void __launch_bounds__(kQuantThreads, 2) dispatch_quant_kernel(DispatchArgs a) {
-    constexpr int NG = kQuantThreads / 32 / WPT;     // token groups per block
-    constexpr int GT = WPT * 32;                     // threads per group
-    constexpr float kQmax = Q == MOEDISP_QUANT_INT8 ? 127.0f : 448.0f;
-    extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ __align__(8) uint64_t bars[NG][kMaxStages];
-    __shared__ int64_t tok[NG][kMaxStages];
-    __shared__ int32_t drow[NG][kMaxStages][MOEDISP_MAX_K];
-    __shared__ float red[NG][2][WPT];
-    __shared__ int abort_s[NG];
-    __shared__ unsigned next_s;                      // the block's next token index
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int grp = warp / WPT, gw = warp - grp * WPT, gt = tid - grp * GT;
-    const int S = a.stages, K = a.K;
-    uint8_t* inbuf = smem + (size_t)grp * S * a.in_bytes;
-    uint64_t* gbar = bars[grp];
-
-    if (gt == 0) {
-        for (int s = 0; s < S; ++s) mbar_init(&gbar[s], 1);
-        fence_mbar_init();
-        abort_s[grp] = 0;
-    }
-    if (tid == 0) next_s = 0;
-    __syncthreads();
-    grid_dep_wait();
-    grid_dep_launch_dependents();
-    write_recv_counts(a);
-
-    // The group's first warp arms stages. The block's tokens are g = blockIdx.x + i *
-    // gridDim.x; the groups draw i from a shared counter, so a group that meets
-    // inactive tokens simply takes more. The routing (K destination rows) of the token
-    // after the one being armed is loaded one fill ahead.
-    auto next_token = [&]() -> int64_t {
-        unsigned i = 0;
-        if (lane == 0) i = atomicAdd(&next_s, 1u);
-        i = __shfl_sync(0xffffffffu, i, 0);
-        return (int64_t)blockIdx.x + (int64_t)i * gridDim.x;
-    };
-    int64_t pf_g = 0, pf_s = -1;
-    int32_t pf_d = -1;
-    if (gw == 0) {
-        pf_g = next_token();
-        pf_d = (pf_g < a.G && lane < K) ? __ldg(a.dst_row + pf_g * K + lane) : -1;
-        pf_s = token_source(a, pf_g);
-    }
-    auto fill = [&](int st) {
-        while (true) {
-            const int64_t g = pf_g;
-            int32_t d = pf_d;
-            const int64_t src = pf_s;
-            if (g < a.G) {
-                pf_g = next_token();
-                pf_d = (pf_g < a.G && lane < K) ? __ldg(a.dst_row + pf_g * K + lane) : -1;
-                pf_s = token_source(a, pf_g);
-            }
-            if (g >= a.G) {
-                if (lane == 0) {
-                    tok[grp][st] = -1;
-                    mbar_arrive(&gbar[st]);
-                }
-                return;
-            }
-            if (d >= a.rows_cap) {
-                raise_status(a.status, MOEDISP_STATUS_CAPACITY);
-                d = -1;
-            }
-            if (d < 0) d = -1;
-            if (__ballot_sync(0xffffffffu, d >= 0)) {
-                if (src < 0 || src >= a.x_rows) {      // routed, but no row of x holds it
-                    if (lane == 0) raise_status(a.status, MOEDISP_STATUS_BAD_SPLIT);
-                    continue;
-                }
-                int32_t dk[MOEDISP_MAX_K];
-#pragma unroll
-                for (int k = 0; k < MOEDISP_MAX_K; ++k) dk[k] = __shfl_sync(0xffffffffu, d, k);
-                if (lane == 0) {
-#pragma unroll
-                    for (int k = 0; k < MOEDISP_MAX_K; ++k)
-                        if (k < K) drow[grp][st][k] = dk[k];
-                    tok[grp][st] = g;
-                    mbar_arrive_expect_tx(&gbar[st], a.in_bytes);
-                    bulk_load(inbuf + (size_t)st * a.in_bytes, a.x + src * a.in_bytes, a.in_bytes,
-                              &gbar[st]);
-                }
-                return;
-            }
-        }
-    };
-    if (gw == 0)
-        for (int st = 0; st < S; ++st) fill(st);
-
-    const int nvec = a.H >> 3;
-    for (int it = 0;; ++it) {
-        const int st = it % S;
-        const uint32_t par = (uint32_t)((it / S) & 1);
-        if (!mbar_wait(&gbar[st], par)) abort_s[grp] = 1;
-        const int64_t g = tok[grp][st];
-        int32_t d[MOEDISP_MAX_K];
-#pragma unroll
-        for (int k = 0; k < MOEDISP_MAX_K; ++k) d[k] = k < K ? drow[grp][st][k] : -1;
-        const uint4* row = reinterpret_cast<const uint4*>(inbuf + (size_t)st * a.in_bytes);
-        float m = 0.0f;
-        for (int c = gt; c < nvec; c += GT) m = fmaxf(m, absmax8(row[c]));
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if (WPT > 1) {
-            if (lane == 0) red[grp][it & 1][gw] = m;
-            group_barrier(1 + grp, GT);
-#pragma unroll
-            for (int w = 0; w < WPT; ++w) m = fmaxf(m, red[grp][it & 1][w]);
-        } else {
-            __syncwarp();
-        }
-        if (abort_s[grp]) {
-            if (gt == 0) raise_status(a.status, MOEDISP_STATUS_TIMEOUT);
-            break;
-        }
-        // Every thread of the group is past the previous token: its stage is free.
-        if (gw == 0 && it >= 1) fill((it - 1) % S);
-        if (g < 0) break;
-        const float scale = __fdiv_rn(m, kQmax);
-        const float inv = __frcp_rn(scale);
-        const bool zero = m == 0.0f;
-        if (K <= 8) {                          // row bases once per token, 8-way stores
-            uint2* dst[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-                dst[k] = d[k] >= 0 ? reinterpret_cast<uint2*>(a.expand_x + (int64_t)d[k] * a.out_bytes)
-                                   : nullptr;
-            for (int c = gt; c < nvec; c += GT) {
-                const uint2 q = quant8<Q>(row[c], scale, inv, zero);
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    if (dst[k] != nullptr) __stcs(dst[k] + c, q);
-            }
-        } else {
-            for (int c = gt; c < nvec; c += GT) {
-                const uint2 q = quant8<Q>(row[c], scale, inv, zero);
-#pragma unroll
-                for (int k = 0; k < MOEDISP_MAX_K; ++k)
-                    if (d[k] >= 0)
-                        __stcs(reinterpret_cast<uint2*>(a.expand_x + (int64_t)d[k] * a.out_bytes) + c, q);
-            }
-        }
-        if (gt < K) {
-            const int32_t dt = drow[grp][st][gt];
-            if (dt >= 0) a.scales[dt] = scale;
-        }
-    }
 }
 
 // Quantising dispatch with per-expert smoothing. The copy of token g for expert e is
@@ -587,6 +427,80 @@ __global__ void __launch_bounds__(kQuantThreads, CPT > 4 ? 2 : 4) dispatch_smoot
     }
 }
 
+// Quantising dispatch: token order, each row read once and quantised once. A group of
+// WPT warps gathers its token's row straight into registers (CPT 16-byte chunks per
+// thread, all issued together): no shared-memory staging, so that nothing but registers
+// limits the warps per SM (a bulk-copy-staged version was measured 5 % slower on cfg3 and
+// cfg4: its stages capped an SM at ~24 warps). Groups take tokens g = group, group +
+// groups, ...; per token: the K destination rows (lanes 0..K-1, shuffled), skip if none
+// is routed, max |x| (shuffles + a named barrier across the group), then the codes are
+// written to the K rows (8 bytes per chunk, coalesced) with the scale.
+template <int Q, int WPT, int CPT>
+__global__ void __launch_bounds__(kQuantThreads, CPT > 4 ? 2 : 4) dispatch_quant_kernel(DispatchArgs a) {
+    constexpr int NG = kQuantThreads / 32 / WPT;
+    constexpr int GT = WPT * 32;
+    constexpr float kQmax = Q == MOEDISP_QUANT_INT8 ? 127.0f : 448.0f;
+    __shared__ float red[NG][2][WPT];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int grp = warp / WPT, gw = warp - grp * WPT, gt = tid - grp * GT;
+    grid_dep_wait();
+    grid_dep_launch_dependents();
+    write_recv_counts(a);
+    const int K = a.K, nvec = a.H >> 3;
+    const int64_t groups = (int64_t)gridDim.x * NG;
+    int parity = 0;
+    for (int64_t g = (int64_t)blockIdx.x * NG + grp; g < a.G; g += groups) {
+        int32_t d = lane < K ? __ldg(a.dst_row + g * K + lane) : -1;
+        if (d >= a.rows_cap) {
+            raise_status(a.status, MOEDISP_STATUS_CAPACITY);
+            d = -1;
+        }
+        if (d < 0) d = -1;
+        if (!__ballot_sync(0xffffffffu, d >= 0)) continue;          // same in every warp
+        const int64_t src = token_source(a, g);
+        if (src < 0 || src >= a.x_rows) {
+            if (gt == 0) raise_status(a.status, MOEDISP_STATUS_BAD_SPLIT);
+            continue;
+        }
+        const uint4* xr = reinterpret_cast<const uint4*>(a.x) + src * nvec;
+        uint4 v[CPT];
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) {
+            const int c = gt + j * GT;
+            v[j] = c < nvec ? __ldcs(xr + c) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        float m = 0.0f;
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) m = fmaxf(m, absmax8(v[j]));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (WPT > 1) {
+            if (lane == 0) red[grp][parity][gw] = m;
+            group_barrier(1 + grp, GT);
+#pragma unroll
+            for (int w = 0; w < WPT; ++w) m = fmaxf(m, red[grp][parity][w]);
+            parity ^= 1;
+        }
+        const float scale = __fdiv_rn(m, kQmax);
+        const float inv = __frcp_rn(scale);
+        const bool zero = m == 0.0f;
+        uint2 q[CPT];
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) q[j] = quant8<Q>(v[j], scale, inv, zero);
+        for (int k = 0; k < K; ++k) {
+            const int32_t dk = __shfl_sync(0xffffffffu, d, k);
+            if (dk < 0) continue;
+            uint2* dst = reinterpret_cast<uint2*>(a.expand_x + (int64_t)dk * a.out_bytes);
+#pragma unroll
+            for (int j = 0; j < CPT; ++j) {
+                const int c = gt + j * GT;
+                if (c < nvec) __stcs(dst + c, q[j]);
+            }
+            if (gt == 0) a.scales[dk] = scale;
+        }
+    }
+}
+
 cudaError_t launch_copy(DispatchArgs a, cudaStream_t stream) {
     // Few tokens per block keep the pipeline's serial start short: use the fewest stages
     // (2, 4 or 8) with which one wave of resident blocks gives each block at most about
@@ -611,24 +525,6 @@ cudaError_t launch_copy(DispatchArgs a, cudaStream_t stream) {
                       1, a);
 }
 
-template <int Q, int WPT>
-cudaError_t launch_quant_w(DispatchArgs a, cudaStream_t stream) {
-    constexpr int NG = kQuantThreads / 32 / WPT;
-    // Stages per group: two for single-warp groups (small rows: more blocks per SM pays
-    // more), three for wider groups (large rows: deeper look-ahead pays more); measured.
-    a.stages = WPT == 1 ? 2 : 3;
-    const size_t smem = (size_t)NG * a.stages * a.in_bytes;
-    int per_sm = 1;
-    cudaError_t err = blocks_per_sm((const void*)dispatch_quant_kernel<Q, WPT>, kQuantThreads,
-                                    smem, &per_sm);
-    if (err != cudaSuccess) return err;
-    int64_t grid = (int64_t)current_sm_count() * per_sm;
-    grid = std::min<int64_t>(grid, std::max<int64_t>((a.G + NG - 1) / NG, 1));
-    return launch_pdl(dispatch_quant_kernel<Q, WPT>, dim3((unsigned)grid), dim3(kQuantThreads),
-                      smem, stream, 1, a);
-}
-
-// Warps per token: the fewest that hold a row in kChunks 16-byte chunks per thread.
 // Smoothing kernel geometry: CPT chunks of the row per thread and WPT warps per row: the
 // fewest chunks per thread up to four (registers, hence warps per SM, matter most here),
 // then eight for the widest rows.
@@ -656,14 +552,37 @@ cudaError_t launch_smooth(const DispatchArgs& a, cudaStream_t stream) {
     return launch_smooth_w<Q, 8, 8>(a, stream);
 }
 
+template <int Q, int WPT, int CPT>
+cudaError_t launch_quant_w(DispatchArgs a, cudaStream_t stream) {
+    int per_sm = 1;
+    cudaError_t err = blocks_per_sm((const void*)dispatch_quant_kernel<Q, WPT, CPT>,
+                                    kQuantThreads, 0, &per_sm);
+    if (err != cudaSuccess) return err;
+    constexpr int NG = kQuantThreads / 32 / WPT;
+    int64_t grid = (int64_t)current_sm_count() * per_sm;
+    grid = std::min<int64_t>(grid, std::max<int64_t>((a.G + NG - 1) / NG, 1));
+    return launch_pdl(dispatch_quant_kernel<Q, WPT, CPT>, dim3((unsigned)grid),
+                      dim3(kQuantThreads), 0, stream, 1, a);
+}
+
+// Token-order quantising geometry: as the smoothing kernel's (chunks per thread up to four,
+// then eight for the widest rows).
+template <int Q>
+cudaError_t launch_quant_tok(const DispatchArgs& a, cudaStream_t stream) {
+    const int nvec = a.H / 8;
+    if (nvec <= 32) return launch_quant_w<Q, 1, 1>(a, stream);
+    if (nvec <= 64) return launch_quant_w<Q, 1, 2>(a, stream);
+    if (nvec <= 128) return launch_quant_w<Q, 1, 4>(a, stream);
+    if (nvec <= 256) return launch_quant_w<Q, 2, 4>(a, stream);
+    if (nvec <= 512) return launch_quant_w<Q, 4, 4>(a, stream);
+    if (nvec <= 1024) return launch_quant_w<Q, 8, 4>(a, stream);
+    return launch_quant_w<Q, 8, 8>(a, stream);
+}
+
 template <int Q>
 cudaError_t launch_quant(const DispatchArgs& a, cudaStream_t stream) {
     if (a.smooth != nullptr) return launch_smooth<Q>(a, stream);
-    const int nvec = a.H / 8;
-    if (nvec <= 1 * 32 * kChunks) return launch_quant_w<Q, 1>(a, stream);
-    if (nvec <= 2 * 32 * kChunks) return launch_quant_w<Q, 2>(a, stream);
-    if (nvec <= 4 * 32 * kChunks) return launch_quant_w<Q, 4>(a, stream);
-    return launch_quant_w<Q, 8>(a, stream);
+    return launch_quant_tok<Q>(a, stream);
 }
 
 }  // namespace
