@@ -664,6 +664,49 @@ def op_sweep(md, torch, device, hbm, reps=10):
                     "bytes_min": b_fused, "frac_of_min": round(b_fused / ms / 1e6 / hbm, 4)})
     del xin, recv, ex, L
     torch.cuda.empty_cache()
+    # expert parallelism through per-rank buffers: cfg2's 8 ranks each dispatch their own
+    # tokens into the 8 ranks' separate buffers through a pointer table, then each combines
+    # its own tokens from them (one stream per rank; on one GPU the "peers" are local
+    # allocations, so this measures the kernels' addressing, not NVLink)
+    w = wl.moe_workload("cfg2", seed=0)
+    st = MoEStep(md, torch, w, device)
+    st.run()
+    rb = st.L.rank_base.cpu().numpy()
+    cap = int(np.diff(rb).max())
+    bufs = [torch.empty((cap, w.H), dtype=torch.bfloat16, device=device) for _ in range(w.W)]
+    table = torch.tensor([b.data_ptr() for b in bufs], dtype=torch.int64, device=device)
+    ys = [torch.empty((w.T, w.H), dtype=torch.bfloat16, device=device) for _ in range(w.W)]
+    streams = [torch.cuda.Stream(device=device) for _ in range(w.W)]
+    ids = st.ids
+    wts = st.wts.view(w.G, w.K)
+
+    def peers_step():
+        main = torch.cuda.current_stream()
+        for r, s_ in enumerate(streams):
+            s_.wait_stream(main)
+            with torch.cuda.stream(s_):
+                md.moe_dispatch_peers(st.x[r * w.T:(r + 1) * w.T], w.H, st.L, r, ids, 0, table, cap,
+                                      st.status)
+        for s_ in streams:
+            main.wait_stream(s_)
+        for r, s_ in enumerate(streams):
+            s_.wait_stream(main)
+            with torch.cuda.stream(s_):
+                md.moe_combine_peers(table, cap, w.H, st.L, r, ids, wts[r * w.T:(r + 1) * w.T],
+                                     ys[r], st.status)
+        for s_ in streams:
+            main.wait_stream(s_)
+
+    g = capture(torch, peers_step)
+    t = statistics.mean(time_graph(torch, g, reps, 3, flush))
+    del g
+    torch.cuda.synchronize()
+    assert int(st.status.item()) == 0, md.status_string(int(st.status.item()))
+    b = algorithmic_bytes("dispatch", w, w.G * w.K) + algorithmic_bytes("combine", w, w.G * w.K)
+    out.append({"workload": "cfg2 over 8 per-rank buffers", "op": "dispatch_peers+combine_peers",
+                "us": round(t * 1e3, 2), "bytes": b, "frac": round(b / t / 1e6 / hbm, 4)})
+    del st, bufs, ys
+    torch.cuda.empty_cache()
     # raw all-to-all-v, W = 64
     a = wl.a2a_workload(seed=0)
     W, E_ = a.W, a.row_elems

@@ -83,6 +83,12 @@ _dispatch_gather = _sig("moedisp_moe_dispatch_gather",
                          _P, _I, _P, _P, _P])
 _token_rows = _sig("moedisp_a2a_token_rows",
                    [_P, _P, _P, _I, ctypes.c_int64, ctypes.c_int64, _P, _P, _P, _P])
+_dispatch_peers = _sig("moedisp_moe_dispatch_peers",
+                       [_P, _I, Dims, _I, _P, ctypes.POINTER(Layout), _I, _P, _P, ctypes.c_int64,
+                        _P, _P])
+_combine_peers = _sig("moedisp_moe_combine_peers",
+                      [_P, ctypes.c_int64, _I, Dims, _I, _P, ctypes.POINTER(Layout), _P, _P, _P,
+                       _P])
 _shared = _sig("moedisp_shared_expert_routing",
                [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P])
 _combine_rms = _sig("moedisp_moe_combine_rmsnorm",
@@ -299,6 +305,29 @@ def a2a_token_rows(src_offsets, out_splits, dst_offsets, W, T, in_rank_stride_ro
     return _check(rc, "a2a_token_rows", raise_on_error)
 
 
+def moe_dispatch_peers(x, H, layout: LayoutBuffers, rank, expert_ids, quant_mode, peer_expand_x,
+                       peer_rows_cap, status, peer_scales=None, stream=None,
+                       raise_on_error=True) -> int:
+    """Rank `rank`'s dispatch over W GPUs: peer_expand_x / peer_scales are device int64
+    tensors [W] of the ranks' buffer addresses (peer memory mapped into this GPU)."""
+    L = layout.struct()
+    rc = _dispatch_peers(_ptr(x), int(H), layout.dims, int(rank), _ptr(expert_ids),
+                         ctypes.byref(L), int(quant_mode), _ptr(peer_expand_x),
+                         _ptr(peer_scales), int(peer_rows_cap), _ptr(status), _stream(stream))
+    return _check(rc, "moe_dispatch_peers", raise_on_error)
+
+
+def moe_combine_peers(peer_expert_out, peer_rows_cap, H, layout: LayoutBuffers, rank, expert_ids,
+                      expert_scales, y, status, stream=None, raise_on_error=True) -> int:
+    """Rank `rank`'s combine over W GPUs: peer_expert_out is a device int64 tensor [W] of
+    the ranks' expert-output buffer addresses."""
+    L = layout.struct()
+    rc = _combine_peers(_ptr(peer_expert_out), int(peer_rows_cap), int(H), layout.dims, int(rank),
+                        _ptr(expert_ids), ctypes.byref(L), _ptr(expert_scales), _ptr(y),
+                        _ptr(status), _stream(stream))
+    return _check(rc, "moe_combine_peers", raise_on_error)
+
+
 def shared_expert_routing(expert_ids, expert_scales, W, T, K, E, shared_expert_num,
                           shared_expert_rank_num, ext_ids, ext_scales, status, stream=None,
                           raise_on_error=True) -> int:
@@ -323,14 +352,16 @@ def raw_call(name: str, *args) -> int:
                 "moedisp_moe_combine_rmsnorm": _combine_rms,
                 "moedisp_shared_expert_routing": _shared,
                 "moedisp_moe_dispatch_gather": _dispatch_gather,
-                "moedisp_a2a_token_rows": _token_rows}[name](*args))
+                "moedisp_a2a_token_rows": _token_rows,
+                "moedisp_moe_dispatch_peers": _dispatch_peers,
+                "moedisp_moe_combine_peers": _combine_peers}[name](*args))
 
 
 __all__ = [
     "a2a_exchange_plan", "a2a_v", "layout_workspace_size", "LayoutBuffers",
     "moe_dispatch_layout", "moe_dispatch_layout_noalloc", "moe_dispatch", "moe_combine",
     "selftest_bounded_wait", "moe_combine_rmsnorm", "shared_expert_routing",
-    "moe_dispatch_gather", "a2a_token_rows",
+    "moe_dispatch_gather", "a2a_token_rows", "moe_dispatch_peers", "moe_combine_peers",
     "status_string", "version", "NOALLOC_SCRATCH_BYTES",
     "Dims", "Layout", "MoedispError", "LIBRARY_PATH",
     "QUANT_NONE", "QUANT_INT8", "QUANT_FP8_E4M3",

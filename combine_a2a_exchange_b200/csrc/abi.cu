@@ -369,6 +369,62 @@ int moedisp_moe_combine(const void* expert_out, int H, moedisp_dims dims,
     return rc(moedisp::launch_combine(expert_out, H, dims, L, expert_scales, y, status, stream));
 }
 
+int moedisp_moe_dispatch_peers(const void* x, int H, moedisp_dims dims, int rank,
+                               const int32_t* expert_ids, const moedisp_layout* layout,
+                               int quant_mode, void* const* peer_expand_x,
+                               float* const* peer_scales, int64_t peer_rows_cap, int32_t* status,
+                               moedisp_stream_t stream) {
+    if (!layout || !status) return MOEDISP_ERR_NULLPTR;
+    int c = check_dims(dims);
+    if (c != MOEDISP_OK) return c;
+    const moedisp_layout& L = *layout;
+    if ((c = check_rows_cap(L.rows_cap)) != MOEDISP_OK) return c;
+    if (rank < 0 || rank >= dims.W || peer_rows_cap < 0) return MOEDISP_ERR_INVALID;
+    if (quant_mode != MOEDISP_QUANT_NONE && quant_mode != MOEDISP_QUANT_INT8 &&
+        quant_mode != MOEDISP_QUANT_FP8_E4M3)
+        return MOEDISP_ERR_INVALID;
+    if (H <= 0) return MOEDISP_ERR_INVALID;
+    if (H > MOEDISP_MAX_H) return MOEDISP_ERR_UNSUPPORTED;
+    if (H % (quant_mode == MOEDISP_QUANT_NONE ? 8 : 16) != 0) return MOEDISP_ERR_MISALIGNED;
+    if (dims.T == 0) return MOEDISP_OK;
+    if (!x || !expert_ids || !L.dst_row || !L.rank_base || !peer_expand_x) return MOEDISP_ERR_NULLPTR;
+    if (quant_mode != MOEDISP_QUANT_NONE && !peer_scales) return MOEDISP_ERR_NULLPTR;
+    if (!aligned(x, 16) || !aligned(expert_ids, 4) || !aligned(L.dst_row, 4) ||
+        !aligned(L.rank_base, 8) || !aligned(peer_expand_x, 8) || !aligned(peer_scales, 8) ||
+        !aligned(status, 4))
+        return MOEDISP_ERR_MISALIGNED;
+    return rc(moedisp::launch_dispatch_peers(x, H, dims, rank, expert_ids, L, quant_mode,
+                                             peer_expand_x, peer_scales, peer_rows_cap, status,
+                                             stream));
+}
+
+int moedisp_moe_combine_peers(const void* const* peer_expert_out, int64_t peer_rows_cap, int H,
+                              moedisp_dims dims, int rank, const int32_t* expert_ids,
+                              const moedisp_layout* layout, const float* expert_scales, void* y,
+                              int32_t* status, moedisp_stream_t stream) {
+    if (!layout || !status) return MOEDISP_ERR_NULLPTR;
+    int c = check_dims(dims);
+    if (c != MOEDISP_OK) return c;
+    const moedisp_layout& L = *layout;
+    if ((c = check_rows_cap(L.rows_cap)) != MOEDISP_OK) return c;
+    if (rank < 0 || rank >= dims.W || peer_rows_cap < 0 || H <= 0) return MOEDISP_ERR_INVALID;
+    if (H % 8 != 0) return MOEDISP_ERR_MISALIGNED;
+    if (dims.T == 0) return MOEDISP_OK;
+    if (!peer_expert_out || !expert_ids || !L.dst_row || !L.rank_base || !expert_scales || !y)
+        return MOEDISP_ERR_NULLPTR;
+    if (!aligned(peer_expert_out, 8) || !aligned(expert_ids, 4) || !aligned(L.dst_row, 4) ||
+        !aligned(L.rank_base, 8) || !aligned(expert_scales, 4) || !aligned(y, 16) ||
+        !aligned(status, 4))
+        return MOEDISP_ERR_MISALIGNED;
+    const size_t slots = (size_t)dims.W * dims.T * dims.K;
+    if (any_alias({{y, (size_t)dims.T * H * 2}, {status, 4}},
+                  {{expert_ids, slots * 4}, {L.dst_row, slots * 4},
+                   {expert_scales, (size_t)dims.T * dims.K * 4}}))
+        return MOEDISP_ERR_ALIASED;
+    return rc(moedisp::launch_combine_peers(peer_expert_out, peer_rows_cap, H, dims, rank,
+                                            expert_ids, L, expert_scales, y, status, stream));
+}
+
 int moedisp_shared_expert_routing(const int32_t* expert_ids, const float* expert_scales, int W,
                                   int T, int K, int E, int shared_expert_num,
                                   int shared_expert_rank_num, int32_t* ext_ids, float* ext_scales,

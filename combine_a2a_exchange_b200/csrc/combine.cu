@@ -26,6 +26,13 @@ struct CombineArgs {
     int64_t rows_cap;
     uint4* y;
     int32_t* status;
+    // Rows on W separate ranks (PEERS): expert e's rows live in rank e / ne's buffer
+    // peer_eo[e / ne] (peer memory), local row = global row - rank_base[e / ne].
+    const uint4* const* peer_eo;
+    int64_t peer_cap;
+    const int32_t* ids;
+    const int64_t* rank_base;
+    int ne;
 };
 
 __device__ __forceinline__ float lo_f(uint32_t v) { return __uint_as_float(v << 16); }
@@ -36,16 +43,18 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-template <int K>
+template <int K, bool PEERS>
 __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a) {
     grid_dep_wait();
     grid_dep_launch_dependents();
     const int chunks = (a.H8 + kThreads - 1) / kThreads;
     const int64_t items = a.G * chunks;
     // The next item's routing (rows and weights) is loaded while this item's rows are in
-    // flight, so each item costs one dependent round trip instead of two.
+    // flight, so each item costs one dependent round trip instead of two. PEERS: each
+    // row's base address (rank table, local row) is resolved with it.
     int32_t nd[K];
     float nw[K];
+    const uint4* np[PEERS ? K : 1];
     auto load_routing = [&](int64_t item) {
         if (item >= items) return;
         const int64_t g = item / chunks;
@@ -53,6 +62,15 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a) {
         for (int k = 0; k < K; ++k) {
             nd[k] = __ldg(a.dst_row + g * K + k);
             nw[k] = __ldg(a.w + g * K + k);
+            if (PEERS) {
+                np[PEERS ? k : 0] = nullptr;
+                if (nd[k] >= 0 && nd[k] < a.rows_cap) {
+                    const int q = __ldg(a.ids + g * K + k) / a.ne;
+                    const int64_t local = (int64_t)nd[k] - __ldg(a.rank_base + q);
+                    if (local >= 0 && local < a.peer_cap) np[PEERS ? k : 0] = a.peer_eo[q] + local * a.H8;
+                    else nd[k] = a.rows_cap;                 // flagged as beyond capacity below
+                }
+            }
         }
     };
     load_routing(blockIdx.x);
@@ -61,11 +79,13 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a) {
         const int vec = (int)(item - g * chunks) * kThreads + threadIdx.x;
         int32_t d[K];
         float w[K];
+        const uint4* p[PEERS ? K : 1];
         bool over = false;
 #pragma unroll
         for (int k = 0; k < K; ++k) {
             d[k] = nd[k];
             w[k] = nw[k];
+            if (PEERS) p[PEERS ? k : 0] = np[PEERS ? k : 0];
             if (d[k] >= a.rows_cap) {
                 over = true;
                 d[k] = -1;
@@ -76,8 +96,10 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a) {
         if (vec >= a.H8) continue;
         uint4 v[K];
 #pragma unroll
-        for (int k = 0; k < K; ++k)
-            v[k] = d[k] >= 0 ? __ldcs(a.eo + (int64_t)d[k] * a.H8 + vec) : make_uint4(0, 0, 0, 0);
+        for (int k = 0; k < K; ++k) {
+            const uint4* row = PEERS ? p[PEERS ? k : 0] : a.eo + (int64_t)d[k] * a.H8;
+            v[k] = d[k] >= 0 ? __ldcs(row + vec) : make_uint4(0, 0, 0, 0);
+        }
         float acc[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
@@ -105,8 +127,9 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a) {
 
 template <int K>
 cudaError_t launch_k(const CombineArgs& a, cudaStream_t stream) {
+    void (*kernel)(CombineArgs) = a.peer_eo != nullptr ? combine_kernel<K, true> : combine_kernel<K, false>;
     int per_sm = 1;
-    cudaError_t err = blocks_per_sm((const void*)combine_kernel<K>, kThreads, 0, &per_sm);
+    cudaError_t err = blocks_per_sm((const void*)kernel, kThreads, 0, &per_sm);
     if (err != cudaSuccess) return err;
     const int chunks = (a.H8 + kThreads - 1) / kThreads;
     // All resident blocks, even if the last round of items leaves some idle: measured
@@ -114,7 +137,7 @@ cudaError_t launch_k(const CombineArgs& a, cudaStream_t stream) {
     // flight cost more than the tail).
     int64_t grid = (int64_t)current_sm_count() * per_sm;
     grid = std::min<int64_t>(grid, std::max<int64_t>(1, a.G * chunks));
-    return launch_pdl(combine_kernel<K>, dim3((unsigned)grid), dim3(kThreads), 0, stream, 1, a);
+    return launch_pdl(kernel, dim3((unsigned)grid), dim3(kThreads), 0, stream, 1, a);
 }
 
 
@@ -237,6 +260,20 @@ cudaError_t launch_rms_k(const RmsArgs& a, cudaStream_t stream) {
 
 }  // namespace
 
+namespace {
+cudaError_t launch_combine_args(const CombineArgs& a, int K, cudaStream_t stream) {
+    switch (K) {
+#define MOEDISP_K(n) \
+    case n: return launch_k<n>(a, stream);
+        MOEDISP_K(1) MOEDISP_K(2) MOEDISP_K(3) MOEDISP_K(4) MOEDISP_K(5) MOEDISP_K(6)
+        MOEDISP_K(7) MOEDISP_K(8) MOEDISP_K(9) MOEDISP_K(10) MOEDISP_K(11) MOEDISP_K(12)
+        MOEDISP_K(13) MOEDISP_K(14) MOEDISP_K(15) MOEDISP_K(16)
+#undef MOEDISP_K
+        default: return cudaErrorInvalidValue;
+    }
+}
+}  // namespace
+
 cudaError_t launch_combine(const void* expert_out, int H, const moedisp_dims& dims,
                            const moedisp_layout& L, const float* expert_scales, void* y,
                            int32_t* status, cudaStream_t stream) {
@@ -249,15 +286,34 @@ cudaError_t launch_combine(const void* expert_out, int H, const moedisp_dims& di
     a.rows_cap = L.rows_cap;
     a.y = static_cast<uint4*>(y);
     a.status = status;
-    switch (dims.K) {
-#define MOEDISP_K(n) \
-    case n: return launch_k<n>(a, stream);
-        MOEDISP_K(1) MOEDISP_K(2) MOEDISP_K(3) MOEDISP_K(4) MOEDISP_K(5) MOEDISP_K(6)
-        MOEDISP_K(7) MOEDISP_K(8) MOEDISP_K(9) MOEDISP_K(10) MOEDISP_K(11) MOEDISP_K(12)
-        MOEDISP_K(13) MOEDISP_K(14) MOEDISP_K(15) MOEDISP_K(16)
-#undef MOEDISP_K
-        default: return cudaErrorInvalidValue;
-    }
+    a.peer_eo = nullptr;
+    a.peer_cap = 0;
+    a.ids = nullptr;
+    a.rank_base = nullptr;
+    a.ne = 1;
+    return launch_combine_args(a, dims.K, stream);
+}
+
+cudaError_t launch_combine_peers(const void* const* peer_expert_out, int64_t peer_cap, int H,
+                                 const moedisp_dims& dims, int rank, const int32_t* expert_ids,
+                                 const moedisp_layout& L, const float* expert_scales, void* y,
+                                 int32_t* status, cudaStream_t stream) {
+    const int64_t slot0 = (int64_t)rank * dims.T * dims.K;
+    CombineArgs a;
+    a.eo = nullptr;
+    a.G = dims.T;
+    a.H8 = H / 8;
+    a.dst_row = L.dst_row + slot0;
+    a.w = expert_scales;
+    a.rows_cap = L.rows_cap;
+    a.y = static_cast<uint4*>(y);
+    a.status = status;
+    a.peer_eo = reinterpret_cast<const uint4* const*>(peer_expert_out);
+    a.peer_cap = peer_cap;
+    a.ids = expert_ids + slot0;
+    a.rank_base = L.rank_base;
+    a.ne = dims.E / dims.W;
+    return launch_combine_args(a, dims.K, stream);
 }
 
 }  // namespace moedisp

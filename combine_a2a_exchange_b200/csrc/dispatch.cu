@@ -33,6 +33,13 @@ struct DispatchArgs {
     const int32_t* assist;     // [rows_cap] slot of each row (the smoothing kernel)
     const int64_t* rows;       // [G] row of x holding each token, -1 for none; null: row g
     int64_t x_rows;            // rows of x
+    // Destination rows on W separate ranks (PEERS kernels): rank q's expand_x / scales are
+    // peer_out[q] / peer_scales[q] (device pointers reachable from this GPU) with peer_cap
+    // rows; global row d of expert e goes to rank e / ne, local row d - rank_base[e / ne].
+    void* const* peer_out;
+    float* const* peer_scales;
+    int64_t peer_cap;
+    const int32_t* ids;        // [G][K] expert ids of this rank's slots (PEERS)
     int stages;
     uint32_t in_bytes, out_bytes;
     // receive counts (optional)
@@ -179,6 +186,21 @@ __device__ __forceinline__ uint2 quant8(const uint4& v, float scale, float inv, 
     return make_uint2(pack_low_bytes(b[0], b[1], b[2], b[3]), pack_low_bytes(b[4], b[5], b[6], b[7]));
 }
 
+// PEERS: address of global destination row d of slot (g, k), or null (with
+// MOEDISP_STATUS_CAPACITY raised) when it falls beyond its rank's peer_cap rows.
+__device__ __forceinline__ uint8_t* peer_row(const DispatchArgs& a, int64_t g, int k, int32_t d,
+                                             int64_t* local_out) {
+    const int e = __ldg(a.ids + g * a.K + k);
+    const int q = e / a.ne;
+    const int64_t local = (int64_t)d - __ldg(a.rank_base + q);
+    if (local < 0 || local >= a.peer_cap) {
+        raise_status(a.status, MOEDISP_STATUS_CAPACITY);
+        return nullptr;
+    }
+    *local_out = local;
+    return static_cast<uint8_t*>(a.peer_out[q]) + local * a.out_bytes;
+}
+
 // Row of x that holds token g (g itself unless a gather map is given), -1 past the end.
 __device__ __forceinline__ int64_t token_source(const DispatchArgs& a, int64_t g) {
     if (g >= a.G) return -1;
@@ -214,12 +236,15 @@ __device__ void write_recv_counts(const DispatchArgs& a) {
 }
 
 // bf16 dispatch: one warp per block; lane 0 streams token rows in, lanes 0..K-1 write
-// them out.
+// them out. PEERS: the K destinations are rows of the W ranks' own buffers (peer memory),
+// each lane resolving its slot's address one fill ahead.
+template <bool PEERS>
 __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t bars[kMaxStages];
     __shared__ int64_t tok[kMaxStages];
     __shared__ int32_t drow[kMaxStages][MOEDISP_MAX_K];
+    __shared__ uint8_t* dptr[PEERS ? kMaxStages : 1][MOEDISP_MAX_K];   // resolved (PEERS)
     const int lane = threadIdx.x & 31;
     const int S = a.stages, K = a.K;
     uint8_t* inbuf = smem;
@@ -259,11 +284,18 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
                 d = -1;
             }
             if (d < 0) d = -1;
+            uint8_t* ptr = nullptr;
+            if (PEERS && d >= 0) {
+                int64_t local;
+                ptr = peer_row(a, g, lane, d, &local);
+                if (ptr == nullptr) d = -1;
+            }
             if (__ballot_sync(0xffffffffu, d >= 0)) {
                 if (src < 0 || src >= a.x_rows) {      // routed, but no row of x holds it
                     if (lane == 0) raise_status(a.status, MOEDISP_STATUS_BAD_SPLIT);
                     continue;
                 }
+                if (PEERS && lane < K) dptr[PEERS ? st : 0][lane] = ptr;   // read back by this lane
                 int32_t dk[MOEDISP_MAX_K];
 #pragma unroll
                 for (int k = 0; k < MOEDISP_MAX_K; ++k) dk[k] = __shfl_sync(0xffffffffu, d, k);
@@ -303,7 +335,10 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
 
         if (issuer) {
             const int32_t d = drow[st][lane];
-            if (d >= 0) bulk_store(a.expand_x + (int64_t)d * a.out_bytes, row_in, a.in_bytes);
+            if (d >= 0) {
+                uint8_t* dst = PEERS ? dptr[PEERS ? st : 0][lane] : a.expand_x + (int64_t)d * a.out_bytes;
+                bulk_store(dst, row_in, a.in_bytes);
+            }
             bulk_commit();
         }
         // Refill the stage of the previous token once its stores have read it.
@@ -435,7 +470,7 @@ __global__ void __launch_bounds__(kQuantThreads, CPT > 4 ? 2 : 4) dispatch_smoot
 // groups, ...; per token: the K destination rows (lanes 0..K-1, shuffled), skip if none
 // is routed, max |x| (shuffles + a named barrier across the group), then the codes are
 // written to the K rows (8 bytes per chunk, coalesced) with the scale.
-template <int Q, int WPT, int CPT>
+template <int Q, int WPT, int CPT, bool PEERS>
 __global__ void __launch_bounds__(kQuantThreads, CPT > 4 ? 2 : 4) dispatch_quant_kernel(DispatchArgs a) {
     constexpr int NG = kQuantThreads / 32 / WPT;
     constexpr int GT = WPT * 32;
@@ -487,16 +522,35 @@ __global__ void __launch_bounds__(kQuantThreads, CPT > 4 ? 2 : 4) dispatch_quant
         uint2 q[CPT];
 #pragma unroll
         for (int j = 0; j < CPT; ++j) q[j] = quant8<Q>(v[j], scale, inv, zero);
+        // PEERS: lane k resolves slot k's rank and local row (and scale address)
+        uint8_t* myrow = nullptr;
+        float* mysc = nullptr;
+        if (PEERS && d >= 0) {
+            int64_t local = 0;
+            myrow = peer_row(a, g, lane, d, &local);
+            if (myrow != nullptr) mysc = a.peer_scales[__ldg(a.ids + g * K + lane) / a.ne] + local;
+        }
         for (int k = 0; k < K; ++k) {
             const int32_t dk = __shfl_sync(0xffffffffu, d, k);
-            if (dk < 0) continue;
-            uint2* dst = reinterpret_cast<uint2*>(a.expand_x + (int64_t)dk * a.out_bytes);
+            uint2* dst;
+            if (PEERS) {
+                dst = reinterpret_cast<uint2*>(__shfl_sync(0xffffffffu, (unsigned long long)myrow, k));
+                if (dst == nullptr) continue;
+            } else {
+                if (dk < 0) continue;
+                dst = reinterpret_cast<uint2*>(a.expand_x + (int64_t)dk * a.out_bytes);
+            }
 #pragma unroll
             for (int j = 0; j < CPT; ++j) {
                 const int c = gt + j * GT;
                 if (c < nvec) __stcs(dst + c, q[j]);
             }
-            if (gt == 0) a.scales[dk] = scale;
+            if (PEERS) {
+                float* sp = reinterpret_cast<float*>(__shfl_sync(0xffffffffu, (unsigned long long)mysc, k));
+                if (gt == 0) *sp = scale;
+            } else if (gt == 0) {
+                a.scales[dk] = scale;
+            }
         }
     }
 }
@@ -510,7 +564,7 @@ cudaError_t launch_copy(DispatchArgs a, cudaStream_t stream) {
     for (int cand : {2, 4, 8}) {
         if ((size_t)cand * a.in_bytes > 64 * 1024 && cand > 2) break;
         int n = 1;
-        cudaError_t err = blocks_per_sm((const void*)dispatch_copy_kernel, kCopyThreads,
+        cudaError_t err = blocks_per_sm((const void*)dispatch_copy_kernel<false>, kCopyThreads,
                                         (size_t)cand * a.in_bytes, &n);
         if (err != cudaSuccess) return err;
         S = cand;
@@ -521,8 +575,8 @@ cudaError_t launch_copy(DispatchArgs a, cudaStream_t stream) {
     const size_t smem = (size_t)S * a.in_bytes;
     int64_t grid = (int64_t)sms * per_sm;
     grid = std::min<int64_t>(grid, std::max<int64_t>(a.G, 1));
-    return launch_pdl(dispatch_copy_kernel, dim3((unsigned)grid), dim3(kCopyThreads), smem, stream,
-                      1, a);
+    return launch_pdl(a.peer_out != nullptr ? dispatch_copy_kernel<true> : dispatch_copy_kernel<false>,
+                      dim3((unsigned)grid), dim3(kCopyThreads), smem, stream, 1, a);
 }
 
 // Smoothing kernel geometry: CPT chunks of the row per thread and WPT warps per row: the
@@ -554,15 +608,15 @@ cudaError_t launch_smooth(const DispatchArgs& a, cudaStream_t stream) {
 
 template <int Q, int WPT, int CPT>
 cudaError_t launch_quant_w(DispatchArgs a, cudaStream_t stream) {
+    void (*kernel)(DispatchArgs) = a.peer_out != nullptr ? dispatch_quant_kernel<Q, WPT, CPT, true>
+                                                         : dispatch_quant_kernel<Q, WPT, CPT, false>;
     int per_sm = 1;
-    cudaError_t err = blocks_per_sm((const void*)dispatch_quant_kernel<Q, WPT, CPT>,
-                                    kQuantThreads, 0, &per_sm);
+    cudaError_t err = blocks_per_sm((const void*)kernel, kQuantThreads, 0, &per_sm);
     if (err != cudaSuccess) return err;
     constexpr int NG = kQuantThreads / 32 / WPT;
     int64_t grid = (int64_t)current_sm_count() * per_sm;
     grid = std::min<int64_t>(grid, std::max<int64_t>((a.G + NG - 1) / NG, 1));
-    return launch_pdl(dispatch_quant_kernel<Q, WPT, CPT>, dim3((unsigned)grid),
-                      dim3(kQuantThreads), 0, stream, 1, a);
+    return launch_pdl(kernel, dim3((unsigned)grid), dim3(kQuantThreads), 0, stream, 1, a);
 }
 
 // Token-order quantising geometry: as the smoothing kernel's (chunks per thread up to four,
@@ -619,6 +673,57 @@ cudaError_t launch_dispatch(const void* x, int64_t x_rows, const int64_t* token_
     a.etn_type = expert_token_nums_type;
     a.erc = ep_recv_counts;
     a.status = status;
+    a.peer_out = nullptr;
+    a.peer_scales = nullptr;
+    a.peer_cap = 0;
+    a.ids = nullptr;
+    switch (quant_mode) {
+        case MOEDISP_QUANT_NONE: return launch_copy(a, stream);
+        case MOEDISP_QUANT_INT8: return launch_quant<MOEDISP_QUANT_INT8>(a, stream);
+        case MOEDISP_QUANT_FP8_E4M3: return launch_quant<MOEDISP_QUANT_FP8_E4M3>(a, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_dispatch_peers(const void* x, int H, const moedisp_dims& dims, int rank,
+                                  const int32_t* expert_ids, const moedisp_layout& L,
+                                  int quant_mode, void* const* peer_out,
+                                  float* const* peer_scales, int64_t peer_cap, int32_t* status,
+                                  cudaStream_t stream) {
+    const int64_t slot0 = (int64_t)rank * dims.T * dims.K;
+    moedisp_layout Lr = L;
+    Lr.dst_row = L.dst_row + slot0;                 // this rank's slots
+    moedisp_dims d1 = dims;
+    DispatchArgs a;
+    a.x = static_cast<const uint8_t*>(x);
+    a.G = dims.T;
+    a.K = dims.K;
+    a.H = H;
+    a.dst_row = Lr.dst_row;
+    a.rows_cap = L.rows_cap;
+    a.expand_x = nullptr;
+    a.scales = nullptr;
+    a.smooth = nullptr;
+    a.assist = nullptr;
+    a.rows = nullptr;
+    a.x_rows = dims.T;
+    a.stages = 2;
+    a.in_bytes = (uint32_t)H * 2u;
+    a.out_bytes = quant_mode == MOEDISP_QUANT_NONE ? (uint32_t)H * 2u : (uint32_t)H;
+    a.cnt = nullptr;
+    a.expert_base = L.expert_base;
+    a.rank_base = L.rank_base;
+    a.W = d1.W;
+    a.E = d1.E;
+    a.ne = d1.E / d1.W;
+    a.etn = nullptr;
+    a.etn_type = 1;
+    a.erc = nullptr;
+    a.status = status;
+    a.peer_out = peer_out;
+    a.peer_scales = peer_scales;
+    a.peer_cap = peer_cap;
+    a.ids = expert_ids + slot0;
     switch (quant_mode) {
         case MOEDISP_QUANT_NONE: return launch_copy(a, stream);
         case MOEDISP_QUANT_INT8: return launch_quant<MOEDISP_QUANT_INT8>(a, stream);

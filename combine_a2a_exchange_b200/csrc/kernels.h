@@ -104,6 +104,18 @@ cudaError_t launch_dispatch(const void* x, int64_t x_rows, const int64_t* token_
                             int expert_token_nums_type, int32_t* ep_recv_counts,
                             int32_t* status, cudaStream_t stream);
 
+// Rank `rank`'s dispatch when the W ranks are separate GPUs: its T tokens' rows go to
+// rows of the ranks' own buffers through a device table of W pointers (peer memory).
+cudaError_t launch_dispatch_peers(const void* x, int H, const moedisp_dims& dims, int rank,
+                                  const int32_t* expert_ids, const moedisp_layout& layout,
+                                  int quant_mode, void* const* peer_out,
+                                  float* const* peer_scales, int64_t peer_cap, int32_t* status,
+                                  cudaStream_t stream);
+cudaError_t launch_combine_peers(const void* const* peer_expert_out, int64_t peer_cap, int H,
+                                 const moedisp_dims& dims, int rank, const int32_t* expert_ids,
+                                 const moedisp_layout& layout, const float* expert_scales,
+                                 void* y, int32_t* status, cudaStream_t stream);
+
 cudaError_t launch_combine(const void* expert_out, int H, const moedisp_dims& dims,
                            const moedisp_layout& layout, const float* expert_scales, void* y,
                            int32_t* status, cudaStream_t stream);

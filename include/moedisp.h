@@ -311,6 +311,41 @@ int moedisp_a2a_token_rows(const int64_t *src_offsets, const int64_t *out_splits
                            int64_t in_rank_stride_rows, int64_t *token_rows, uint8_t *active,
                            int32_t *status, moedisp_stream_t stream);
 
+/* moe_dispatch_peers / moe_combine_peers
+ *
+ * Expert parallelism over W separate GPUs (one rank each). Every rank all-gathers the
+ * routing (expert_ids [W*T][K], the active mask) -- a few bytes per token -- and computes
+ * the global layout of all W ranks with moe_dispatch_layout (dims {W, T, K, E}); then:
+ *   moe_dispatch_peers: rank `rank` writes its T token rows (x: bf16 [T][H]) straight to
+ *     their K destination rows in the owning ranks' buffers: global row d of expert e
+ *     lands in rank q = e / ne's expand_x, local row d - rank_base[q], through
+ *     peer_expand_x (a device array of W pointers to the ranks' expand_x buffers, each
+ *     [peer_rows_cap][H] of the output type, mapped into this GPU -- its own included),
+ *     with the scales through peer_scales (device array of W float pointers; quant modes)
+ *     -- the dispatch and the exchange in one kernel, each row read from HBM once and sent
+ *     over NVLink once per destination;
+ *   moe_combine_peers: rank `rank` computes y[t] (bf16 [T][H]) of its own tokens by
+ *     gathering each slot's expert-output row from the owning rank's buffer through
+ *     peer_expert_out (device array of W pointers, each [peer_rows_cap][H] bf16), with
+ *     this rank's weights (expert_scales fp32 [T][K]) -- the exchange back and the
+ *     weighted sum in one kernel.
+ * expert_ids: the all-gathered ids the layout was computed from (the owner of each slot).
+ * Results equal moe_dispatch / moe_combine of the single-buffer layout, row for row (local
+ * row = global row - rank_base[q]). A slot whose local row is at or beyond peer_rows_cap
+ * is skipped and sets MOEDISP_STATUS_CAPACITY. Ordering between ranks (expand_x rows
+ * complete before the experts run, expert outputs complete before the combine) is the
+ * caller's: a barrier across the ranks' streams. Not supported with smoothing scales or a
+ * gather map. The pointers in the tables are not checked against each other. */
+int moedisp_moe_dispatch_peers(const void *x, int H, moedisp_dims dims, int rank,
+                               const int32_t *expert_ids, const moedisp_layout *layout,
+                               int quant_mode, void *const *peer_expand_x,
+                               float *const *peer_scales, int64_t peer_rows_cap, int32_t *status,
+                               moedisp_stream_t stream);
+int moedisp_moe_combine_peers(const void *const *peer_expert_out, int64_t peer_rows_cap, int H,
+                              moedisp_dims dims, int rank, const int32_t *expert_ids,
+                              const moedisp_layout *layout, const float *expert_scales, void *y,
+                              int32_t *status, moedisp_stream_t stream);
+
 /* shared_expert_routing
  *
  * Shared experts (Ascend aclnnMoeDistributeDispatchV2 sharedExpertNum N,

@@ -249,3 +249,25 @@ def test_gather_and_token_rows_rejections(md):
     assert t(4, 4, 10, tr=so) == md.MOEDISP_ERR_ALIASED
     assert t(4, 4, 10, act=do + 8) == md.MOEDISP_ERR_ALIASED
     assert t(4, 0, 10, so=None, tr=None) == md.MOEDISP_OK
+
+
+def test_peers_rejections(md):
+    L = _layout(md)
+    d = md.Dims(4, 8, 2, 8)
+    x, ids, tab, stab, st, y, w = (FAKE + (i << 20) for i in (64, 96, 128, 160, 256, 300, 340))
+    disp = lambda rank, q, tab=tab, stab=stab, st=st, H=128: md.raw_call(
+        "moedisp_moe_dispatch_peers", x, H, d, rank, ids, ctypes.byref(L), q, tab, stab, 100, st, None)
+    assert disp(4, 0) == md.MOEDISP_ERR_INVALID                   # rank >= W
+    assert disp(-1, 0) == md.MOEDISP_ERR_INVALID
+    assert disp(0, 1) == md.MOEDISP_ERR_INVALID                   # quant mode
+    assert disp(0, 0, tab=None) == md.MOEDISP_ERR_NULLPTR
+    assert disp(0, 2, stab=None) == md.MOEDISP_ERR_NULLPTR        # scales table for quant
+    assert disp(0, 0, tab=tab + 4) == md.MOEDISP_ERR_MISALIGNED
+    assert disp(0, 0, st=None) == md.MOEDISP_ERR_NULLPTR
+    assert disp(0, 2, H=136) == md.MOEDISP_ERR_MISALIGNED
+    comb = lambda rank, y=y, tab=tab: md.raw_call(
+        "moedisp_moe_combine_peers", tab, 100, 128, d, rank, ids, ctypes.byref(L), w, y, st, None)
+    assert comb(4) == md.MOEDISP_ERR_INVALID
+    assert comb(0, tab=None) == md.MOEDISP_ERR_NULLPTR
+    assert comb(0, y=y + 8) == md.MOEDISP_ERR_MISALIGNED
+    assert comb(0, y=w) == md.MOEDISP_ERR_ALIASED                 # y over the weights

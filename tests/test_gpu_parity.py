@@ -840,6 +840,115 @@ def test_dispatch_gather_bad_rows_are_flagged(md):
     assert (got[~keep] == np.uint16(-12345 & 0xFFFF)).all()
 
 
+# --------------------------------------------- expert parallelism over W separate buffers
+
+def _peer_buffers(W, cap, H, q, fill):
+    """W separate per-rank buffers (each its own allocation, as on W GPUs) with a canary,
+    and the device table of their addresses."""
+    if q == 0:
+        bufs = [torch.full((cap, H), fill, dtype=torch.int16, device="cuda") for _ in range(W)]
+    else:
+        bufs = [torch.full((cap, H), fill & 0xFF, dtype=torch.uint8, device="cuda") for _ in range(W)]
+    table = torch.tensor([b.data_ptr() for b in bufs], dtype=torch.int64, device="cuda")
+    return bufs, table
+
+
+@pytest.mark.parametrize("q", [0, 2, 3])
+@pytest.mark.parametrize("W,T,K,E,H", [(4, 300, 4, 16, 256), (8, 256, 8, 64, 4096), (3, 77, 5, 9, 136)])
+def test_peers_dispatch_and_combine(md, q, W, T, K, E, H):
+    """Each rank dispatches its own tokens into the W ranks' own buffers through a pointer
+    table and combines its own tokens from them: row for row the single-buffer result."""
+    if q and H % 16:
+        pytest.skip("quantised rows need H % 16 == 0")
+    w = wl.moe_workload("tiny", seed=80 + W, W=W, T=T, K=K, E=E, H=H, active_p=0.85)
+    L, st0 = run_layout(md, w)                         # the global layout, as every rank computes it
+    ref = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active)
+    rb = ref["rank_base"]
+    cap = int(np.diff(rb).max()) + 3
+    rex, rsc, _ = oracle.moe_dispatch(w.x_bits, ref["dst_row"], w.K, ref["rows_cap"], q)
+    bufs, table = _peer_buffers(W, cap, H, q, -12345 if q == 0 else 0x5A)
+    sbufs = [torch.full((cap,), -1.0, dtype=torch.float32, device="cuda") for _ in range(W)]
+    stable = torch.tensor([b.data_ptr() for b in sbufs], dtype=torch.int64, device="cuda")
+    ids = dev(w.expert_ids.reshape(-1))
+    st = new_status()
+    x = bf16_dev(w.x_bits)
+    for r in range(W):
+        md.moe_dispatch_peers(x[r * T:(r + 1) * T], H, L, r, ids, q, table, cap, st,
+                              peer_scales=stable if q else None)
+    torch.cuda.synchronize()
+    assert st0 == 0 and int(st.item()) == 0
+    for d in range(W):
+        n = int(rb[d + 1] - rb[d])
+        got = bufs[d].cpu().numpy()
+        if q == 0:
+            got = got.view(np.uint16)
+            assert np.array_equal(got[:n], rex[rb[d]:rb[d + 1]])
+            assert (got[n:] == np.uint16(-12345 & 0xFFFF)).all()
+        else:
+            assert np.array_equal(got[:n], rex[rb[d]:rb[d + 1]]) and (got[n:] == 0x5A).all()
+            sc = sbufs[d].cpu().numpy()
+            assert np.array_equal(sc[:n].view(np.uint32), rsc[rb[d]:rb[d + 1]].view(np.uint32))
+            assert (sc[n:] == -1).all()
+    # combine: expert outputs spread over the ranks' own buffers
+    eo = wl.expert_rows(ref["R"], H, seed=81)
+    ebufs = []
+    for d in range(W):
+        b = torch.zeros((cap, H), dtype=torch.int16, device="cuda")
+        b[:int(rb[d + 1] - rb[d])] = torch.from_numpy(eo[rb[d]:rb[d + 1]].view(np.int16)).cuda()
+        ebufs.append(b)
+    etable = torch.tensor([b.data_ptr() for b in ebufs], dtype=torch.int64, device="cuda")
+    wts = dev(w.weights)
+    ys = []
+    for r in range(W):
+        y = torch.full((T, H), 7, dtype=torch.int16, device="cuda").view(torch.bfloat16)
+        md.moe_combine_peers(etable, cap, H, L, r, ids, wts[r * T:(r + 1) * T], y, st)
+        ys.append(y)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    yb = np.concatenate([bits_host(y) for y in ys])
+    check_combine(yb, eo, ref["dst_row"], w.weights, w.K, ref["R"])
+
+
+def test_peers_capacity(md):
+    """A rank buffer too small for its rows: the rows beyond it are skipped and flagged in
+    both directions; every row that fits is exact."""
+    W, T, K, E, H = 4, 200, 4, 8, 128
+    w = wl.moe_workload("tiny", seed=90, W=W, T=T, K=K, E=E, H=H)
+    L, _ = run_layout(md, w)
+    ref = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active)
+    rb = ref["rank_base"]
+    cap = int(np.diff(rb).min()) - 5
+    bufs, table = _peer_buffers(W, cap, H, 0, -12345)
+    ids = dev(w.expert_ids.reshape(-1))
+    st = new_status()
+    x = bf16_dev(w.x_bits)
+    for r in range(W):
+        md.moe_dispatch_peers(x[r * T:(r + 1) * T], H, L, r, ids, 0, table, cap, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == md.STATUS_CAPACITY
+    rex, _, _ = oracle.moe_dispatch(w.x_bits, ref["dst_row"], w.K, ref["rows_cap"], 0)
+    for d in range(W):
+        assert np.array_equal(bufs[d].cpu().numpy().view(np.uint16), rex[rb[d]:rb[d] + cap])
+    eo = wl.expert_rows(ref["R"], H, seed=91)
+    ebufs = [torch.from_numpy(eo[rb[d]:rb[d] + cap].view(np.int16).copy()).cuda() for d in range(W)]
+    etable = torch.tensor([b.data_ptr() for b in ebufs], dtype=torch.int64, device="cuda")
+    st2 = new_status()
+    wts = dev(w.weights)
+    ys = []
+    for r in range(W):
+        y = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
+        md.moe_combine_peers(etable, cap, H, L, r, ids, wts[r * T:(r + 1) * T], y, st2)
+        ys.append(y)
+    torch.cuda.synchronize()
+    assert int(st2.item()) == md.STATUS_CAPACITY
+    # the oracle with every row beyond a rank's capacity treated as unrouted
+    dr = ref["dst_row"].copy()
+    owner = np.searchsorted(rb, dr, side="right") - 1
+    dr[(dr >= 0) & (dr - rb[np.clip(owner, 0, W - 1)] >= cap)] = -1
+    yb = np.concatenate([bits_host(y) for y in ys])
+    check_combine(yb, eo, dr, w.weights, w.K, ref["R"])
+
+
 # ---------------------------------------------------------------- shared experts
 
 SHARED_CASES = [(8, 4, 1, 16, 256, 8, 4096, 0), (8, 4, 2, 4, 100, 6, 512, 2),
