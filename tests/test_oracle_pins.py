@@ -485,6 +485,47 @@ def test_quant_properties(mode):
             assert (np.abs(deq - v) <= half * (1 + 1e-5) + 1e-6).all()
 
 
+@pytest.mark.parametrize("seed", range(3))
+def test_dispatch_equals_pack_then_exchange(seed):
+    """An independent composition: each source rank packs its active slots' token rows in
+    stable expert order (numpy argsort), the 1-D exchange plan of the layout's send_splits
+    moves them (O1 + O2), and every segment rank d receives from rank r equals expand_x's
+    rows of rank d's experts from rank r (O3 + O4) -- the 2-D plan's expert-major order is
+    the 1-D exchange regrouped within each receiver."""
+    rng = np.random.default_rng(400 + seed)
+    W, ne = int(rng.integers(2, 5)), int(rng.integers(1, 4))
+    E, T, K, H = W * ne, int(rng.integers(1, 30)), int(rng.integers(1, 4)), 8
+    w = wl.moe_workload("tiny", seed=410 + seed, W=W, T=T, K=K, E=E, H=H, active_p=0.8,
+                        routing="dup")
+    lay = oracle.moe_dispatch_layout(W, T, K, E, w.expert_ids, w.active)
+    ex, _, fl = oracle.moe_dispatch(w.x_bits, lay["dst_row"], K, lay["rows_cap"], 0)
+    assert fl == 0
+    ids = w.expert_ids.reshape(W, T * K)
+    act = np.repeat(w.active.astype(bool), K).reshape(W, T * K)
+    packs = []
+    for r in range(W):
+        slots = np.nonzero(act[r])[0]
+        order = slots[np.argsort(ids[r][slots], kind="stable")]
+        packs.append(w.x_bits[r * T + order // K])
+    cap_in = max(1, max(len(pk) for pk in packs))
+    inp = np.zeros((W, cap_in, H), np.uint16)
+    for r, pk in enumerate(packs):
+        inp[r, :len(pk)] = pk
+    S = lay["send_splits"]
+    src, outs, dsto, _ = oracle.a2a_exchange_plan(S)
+    cap_out = max(1, int(outs.sum(axis=1).max()))
+    out = np.zeros((W, cap_out, H), np.uint16)
+    assert oracle.a2a_v(inp, out, src, outs, dsto) == 0
+    cnt, eb = lay["cnt"], lay["expert_base"]
+    for d in range(W):
+        for r in range(W):
+            exp = [ex[eb[e] + cnt[:r, e].sum(): eb[e] + cnt[:r + 1, e].sum()]
+                   for e in range(d * ne, (d + 1) * ne)]
+            exp = np.concatenate(exp) if exp else np.zeros((0, H), np.uint16)
+            got = out[d, dsto[d, r]: dsto[d, r] + outs[d, r]]
+            assert np.array_equal(got, exp), (d, r)
+
+
 def test_dispatch_copy_and_scale_placement():
     w = wl.moe_workload("tiny", seed=4, T=5)
     lay = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active)
