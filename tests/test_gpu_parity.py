@@ -1076,3 +1076,56 @@ def test_bounded_wait_times_out_and_context_survives(md):
     ref = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active)
     assert st2 == 0
     assert_layout_equal(layout_host(L), ref, ref["R"], ref["rows_cap"])
+
+
+# ------------------------------------------------------------- randomised sweep
+
+def _random_case(i):
+    rng = np.random.default_rng(1000 + i)
+    W = int(rng.choice([1, 2, 3, 4, 5, 8, 16]))
+    ne = int(rng.integers(1, 9))
+    E = W * ne
+    K = int(rng.integers(1, min(16, E) + 1)) if rng.random() < 0.8 else int(rng.integers(1, 17))
+    T = int(rng.integers(0, 400))
+    q = int(rng.choice([0, 2, 3]))
+    H = int(rng.choice([16, 32, 48, 128, 272, 1024, 2064])) if q else int(rng.choice([8, 24, 128, 520, 4096]))
+    over = dict(W=W, T=T, K=K, E=E, H=H, routing="dup" if K > E or rng.random() < 0.3 else "uniform")
+    mask = rng.random()
+    if mask < 0.3:
+        over["active_p"] = float(rng.uniform(0.2, 1.0))
+    elif mask < 0.5:
+        over["slot_active_p"] = float(rng.uniform(0.2, 1.0))
+    A = int(rng.choice([0, 0, 0, 2, 5, 16]))
+    smooth = bool(q and rng.random() < 0.3)
+    return over, q, A, smooth
+
+
+@pytest.mark.parametrize("i", range(40))
+def test_random_configurations(md, i):
+    """Seeded random shapes through layout -> dispatch -> combine, every output bit-exact
+    against the oracle (combine against the fixed-order fp32 oracle)."""
+    over, q, A, smooth = _random_case(i)
+    w = wl.moe_workload("tiny", seed=2000 + i, **over)
+    L, st = run_layout(md, w, major_align=A)
+    ref = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active, major_align=A)
+    assert st == 0 and ref["flags"] == 0
+    assert_layout_equal(layout_host(L), ref, ref["R"], ref["rows_cap"])
+    sm = wl.smooth_scales(w.E, w.H, seed=3000 + i) if smooth else None
+    full, scales, gr, etn, erc, st2 = run_dispatch(md, w, L, q, smooth=sm)
+    assert st2 == 0
+    rex, rsc, _ = oracle.moe_dispatch(w.x_bits, ref["dst_row"], w.K, ref["rows_cap"], q, smooth=sm,
+                                      expert_ids=w.expert_ids if smooth else None)
+    real = ref["assist_info"][:ref["R"]] >= 0
+    got = full.cpu().numpy()[gr:gr + ref["R"]]
+    got = got.view(np.uint16) if q == 0 else got
+    assert np.array_equal(got[real], rex[:ref["R"]][real])
+    if q:
+        s = scales.cpu().numpy()[gr:gr + ref["R"]]
+        assert np.array_equal(s[real].view(np.uint32), rsc[:ref["R"]][real].view(np.uint32))
+    retn, rerc, _ = oracle.moe_recv_counts(w.W, w.E, ref["cnt"], 1, major_align=A)
+    assert np.array_equal(etn, retn) and np.array_equal(erc, rerc)
+    if w.G:
+        eo = wl.expert_rows(max(L.rows_cap, 1), w.H, seed=4000 + i)
+        y, st3 = run_combine(md, L, eo, w)
+        assert st3 == 0
+        check_combine(y, eo, ref["dst_row"], w.weights, w.K, L.rows_cap)
