@@ -690,16 +690,13 @@ cudaError_t launch_dispatch_peers(const void* x, int H, const moedisp_dims& dims
                                   int quant_mode, void* const* peer_out,
                                   float* const* peer_scales, int64_t peer_cap, int32_t* status,
                                   cudaStream_t stream) {
-    const int64_t slot0 = (int64_t)rank * dims.T * dims.K;
-    moedisp_layout Lr = L;
-    Lr.dst_row = L.dst_row + slot0;                 // this rank's slots
-    moedisp_dims d1 = dims;
+    const int64_t slot0 = (int64_t)rank * dims.T * dims.K;     // this rank's first slot
     DispatchArgs a;
     a.x = static_cast<const uint8_t*>(x);
     a.G = dims.T;
     a.K = dims.K;
     a.H = H;
-    a.dst_row = Lr.dst_row;
+    a.dst_row = L.dst_row + slot0;
     a.rows_cap = L.rows_cap;
     a.expand_x = nullptr;
     a.scales = nullptr;
@@ -713,9 +710,9 @@ cudaError_t launch_dispatch_peers(const void* x, int H, const moedisp_dims& dims
     a.cnt = nullptr;
     a.expert_base = L.expert_base;
     a.rank_base = L.rank_base;
-    a.W = d1.W;
-    a.E = d1.E;
-    a.ne = d1.E / d1.W;
+    a.W = dims.W;
+    a.E = dims.E;
+    a.ne = dims.E / dims.W;
     a.etn = nullptr;
     a.etn_type = 1;
     a.erc = nullptr;
