@@ -271,3 +271,24 @@ def test_peers_rejections(md):
     assert comb(0, tab=None) == md.MOEDISP_ERR_NULLPTR
     assert comb(0, y=y + 8) == md.MOEDISP_ERR_MISALIGNED
     assert comb(0, y=w) == md.MOEDISP_ERR_ALIASED                 # y over the weights
+
+
+def test_binding_host_logic(md):
+    """Argument marshalling that happens in Python: the active mask's form is read from
+    its shape, and the default capacity covers major_align padding."""
+    import torch
+    d = md.Dims(4, 8, 3, 8)
+    assert md._mask_dims(None, d, None) == 0
+    assert md._mask_dims(torch.zeros(32, dtype=torch.uint8), d, None) == 1
+    assert md._mask_dims(torch.zeros(32, 3, dtype=torch.uint8), d, None) == 2
+    assert md._mask_dims(torch.zeros(96, dtype=torch.uint8), d, None) == 2      # flat [G*K]
+    assert md._mask_dims(torch.zeros(32, dtype=torch.uint8), md.Dims(4, 8, 1, 8), None) == 1
+    assert md._mask_dims(torch.zeros(32, dtype=torch.uint8), d, 2) == 2          # explicit
+    with pytest.raises(ValueError):
+        md._mask_dims(FAKE, d, None)                                           # raw pointer
+    L = md.LayoutBuffers.allocate(4, 8, 3, 8, device="cpu")
+    assert L.rows_cap == 4 * 8 * 3 and L.major_align == 0
+    L = md.LayoutBuffers.allocate(4, 8, 3, 8, device="cpu", major_align=16)
+    assert L.rows_cap == 4 * 8 * 3 + 8 * 16 and L.assist_info.numel() == L.rows_cap
+    L = md.LayoutBuffers.allocate(4, 8, 3, 8, device="cpu", major_align=1)
+    assert L.rows_cap == 4 * 8 * 3
