@@ -747,16 +747,74 @@ def op_sweep(md, torch, device, hbm, reps=10):
 
 # ---------------------------------------------------------------------- main
 
+def run_gather_op(args, wl, md, torch, device, flush):
+    """moe_dispatch_gather of W = 8 ranks' exchanged tokens read in place (splits ~
+    randint[0, 512), H = 4096 bf16, E = 64, K = 8), after the plan, the receive map and the
+    layout ran once."""
+    a = wl.a2a_workload(seed=3, W=8, max_split=512, zero_frac=0.1, row_elems=4096)
+    W_, H_, K_, E_ = a.W, 4096, 8, 64
+    cap_in, T_ = a.cap_in, a.cap_out
+    w = wl.moe_workload("tiny", seed=4, W=W_, T=T_, K=K_, E=E_, H=8)
+    g0 = torch.Generator(device=device).manual_seed(5)
+    xin = torch.randn((W_ * cap_in, H_), generator=g0, device=device).to(torch.bfloat16)
+    plan = [torch.empty((W_, W_), dtype=torch.int64, device=device) for _ in range(3)]
+    tr = torch.empty(W_ * T_, dtype=torch.int64, device=device)
+    act = torch.empty(W_ * T_, dtype=torch.uint8, device=device)
+    L = md.LayoutBuffers.allocate(W_, T_, K_, E_, device=device)
+    ex = torch.empty((L.rows_cap, H_), dtype=torch.bfloat16, device=device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    md.a2a_exchange_plan(torch.from_numpy(a.in_splits).to(device), plan[0], plan[1], plan[2], status)
+    md.a2a_token_rows(plan[0], plan[1], plan[2], W_, T_, cap_in, tr, status, active=act)
+    md.moe_dispatch_layout(torch.from_numpy(w.expert_ids.reshape(-1)).to(device), act, L, status)
+    Ev = torch.cuda.Event
+    for _ in range(args.warmup):
+        flush.zero_()
+        md.moe_dispatch_gather(xin, W_ * cap_in, tr, H_, L, 0, ex, None, status)
+    pairs = []
+    for _ in range(args.steps):
+        flush.zero_()
+        e0, e1 = Ev(enable_timing=True), Ev(enable_timing=True)
+        e0.record()
+        md.moe_dispatch_gather(xin, W_ * cap_in, tr, H_, L, 0, ex, None, status)
+        e1.record()
+        pairs.append((e0, e1))
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise SystemExit(f"status {md.status_string(int(status.item()))}")
+    us = statistics.mean(x.elapsed_time(y) for x, y in pairs) * 1e3
+    print(json.dumps({"op": args.op, "workload": "a2a8->dispatch", "us": round(us, 2),
+                      "steps": args.steps, "warmup": args.warmup}))
+    return 0
+
+
 def run_single_op(args, wl, md, torch):
     """Times one op of the widened path on --workload after the step's layout (and
     dispatch) ran once: warm-up launches, then --steps launches, each behind an L2 flush.
     Prints one JSON line. Launch order: the step's kernels once, then the op's."""
     device = torch.device("cuda", torch.cuda.current_device())
+    flush = L2Flush(torch, device)
+    if args.op == "dispatch_gather":
+        return run_gather_op(args, wl, md, torch, device, flush)
     w = wl.moe_workload(args.workload, seed=0, **({"T": args.T} if args.T else {}))
     st = MoEStep(md, torch, w, device)
     st.run()
-    flush = L2Flush(torch, device)
-    if args.op == "dispatch_smooth":
+    if args.op == "peers":
+        # every rank's dispatch into the W ranks' separate buffers, then every rank's
+        # combine from them (rank by rank on one stream)
+        rb = st.L.rank_base.cpu().numpy()
+        cap = int(np.diff(rb).max())
+        bufs = [torch.empty((cap, w.H), dtype=torch.bfloat16, device=device) for _ in range(w.W)]
+        table = torch.tensor([b.data_ptr() for b in bufs], dtype=torch.int64, device=device)
+        wts = st.wts.view(w.G, w.K)
+
+        def op():
+            for r in range(w.W):
+                md.moe_dispatch_peers(st.x[r * w.T:(r + 1) * w.T], w.H, st.L, r, st.ids, 0, table,
+                                      cap, st.status)
+            for r in range(w.W):
+                md.moe_combine_peers(table, cap, w.H, st.L, r, st.ids, wts[r * w.T:(r + 1) * w.T],
+                                     st.y[r * w.T:(r + 1) * w.T], st.status)
+    elif args.op == "dispatch_smooth":
         if w.quant_mode == 0:
             raise SystemExit("dispatch_smooth needs a quantising workload (cfg3, cfg4)")
         sm = torch.from_numpy(wl.smooth_scales(w.E, w.H, seed=1)).to(device)
@@ -809,7 +867,8 @@ def main():
     ap.add_argument("--no-ops", action="store_true", help="skip the per-op sweep of other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--op", choices=["step", "dispatch_smooth", "combine_rmsnorm"], default="step",
+    ap.add_argument("--op", choices=["step", "dispatch_smooth", "combine_rmsnorm", "dispatch_gather",
+                                     "peers"], default="step",
                     help="time one NEXT-row op alone on --workload (one GPU), e.g. to profile it")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
