@@ -2,7 +2,9 @@
  * moedisp.h -- C ABI of libmoedisp: expert-parallel (EP) MoE token dispatch / combine
  * and the uneven all-to-all-v exchange, for NVIDIA B200 (sm_100a).
  *
- * The W EP ranks of the exchange are "virtual ranks": slices of one GPU's memory.
+ * The W EP ranks of the exchange are "virtual ranks": slices of one GPU's memory --
+ * except in moe_dispatch_peers / moe_combine_peers, where they are W GPUs and the rows
+ * move through a table of the ranks' buffer addresses (peer memory).
  *
  * Conventions shared by every call
  * --------------------------------
