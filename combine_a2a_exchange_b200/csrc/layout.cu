@@ -8,10 +8,11 @@
 // never straddle a source rank, and:
 //
 //  * small problems (at most 16 tiles of at most 2048 slots): one kernel, one thread-block
-//    cluster. Each 256-thread block ranks its tile (below), the blocks exchange their
-//    per-expert tile counts through distributed shared memory across the cluster barrier,
-//    and every block derives its tile offsets, the expert bases and the per-rank counts
-//    from them -- no global scratch, no second launch.
+//    cluster. Each 256-thread block ranks its tile (below) and pushes its per-expert tile
+//    counts into every block's shared memory (distributed shared memory stores, before
+//    the cluster barrier); every block then derives its tile offsets, the expert bases and
+//    the per-rank counts from its local copy -- no global scratch, no second launch, no
+//    remote read after the barrier.
 //  * larger problems: three kernels, each spread over the whole GPU.
 //      count: one block per tile; a warp-aggregated shared-memory histogram -> the tile's
 //             counts per expert;
@@ -356,8 +357,8 @@ __global__ void __launch_bounds__(kThreads) layout_rank_kernel(LayoutArgs a) {
 
 // ------------------------------------------------------------ cluster path
 
-__device__ __forceinline__ void cluster_arrive_release() {
-    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void cluster_wait_acquire() {
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
@@ -373,11 +374,11 @@ layout_cluster_kernel(LayoutArgs a) {
     const int ES = E | 1;                                        // odd row stride: no bank conflicts
     int64_t* ebase = reinterpret_cast<int64_t*>(smem_raw);      // [E + 1]
     int32_t* wc = reinterpret_cast<int32_t*>(ebase + E + 1);    // [kCWarps][ES]
-    int32_t* tcnt = wc + kCWarps * ES;                           // [E] this tile's counts
-    int32_t* tpre = tcnt + E;                                    // [E] counts in earlier tiles
+    int32_t* tpre = wc + kCWarps * ES;                           // [E] counts in earlier tiles
     int32_t* colp = tpre + E;                                    // [E] counts in earlier ranks
     int32_t* cntr = colp + E;                                    // [E] counts of this rank
     int32_t* etot = cntr + E;                                    // [E] rows routed to e
+    int32_t* allc = etot + E;                                    // [C][E] every tile's counts
 
     const int tile = (int)cluster.block_rank();
     const int C = (int)cluster.num_blocks();
@@ -389,12 +390,16 @@ layout_cluster_kernel(LayoutArgs a) {
     grid_dep_wait();
     grid_dep_launch_dependents();
     __syncthreads();
+    // Distributed shared memory of a block may be written only once that block runs: this
+    // arrival is matched by the wait before the counts are pushed (long satisfied by then).
+    cluster_arrive_relaxed();
 
     int32_t* mine = wc + warp * ES;
     const int64_t wlo = lo + (int64_t)warp * STEPS * 32;
     uint32_t pk[STEPS];
     rank_in_warp<STEPS>(a, base, wlo, hi, mine, pk);
     __syncthreads();
+    cluster_wait_acquire();
     // Per expert, an exclusive scan over the warps' counts, in warp order.
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int32_t run = 0;
@@ -404,13 +409,14 @@ layout_cluster_kernel(LayoutArgs a) {
             wc[w * ES + e] = run;
             run += t;
         }
-        tcnt[e] = run;
+        // pushed into row `tile` of every block's copy (remote stores need no round trip)
+        for (int t = 0; t < C; ++t) cluster.map_shared_rank(allc, t)[tile * E + e] = run;
     }
-    cluster.sync();   // every tile's counts are final and visible across the cluster
+    cluster.sync();   // every tile's counts have landed in every block (release / acquire)
 
-    // Counts of every tile, read from the other blocks' shared memory (all reads issued
-    // together): offsets of this tile and of this rank, this rank's row of cnt, and the
-    // expert totals, scanned into expert bases.
+    // Counts of every tile, now local: offsets of this tile and of this rank, this rank's
+    // row of cnt, and the expert totals, scanned into expert bases. No block reads another
+    // block's shared memory after the barrier, so blocks may finish independently.
     int64_t carry = 0;
     for (int b0 = 0; b0 < E; b0 += blockDim.x) {
         const int e = b0 + threadIdx.x;
@@ -419,7 +425,7 @@ layout_cluster_kernel(LayoutArgs a) {
             int32_t v[kCMaxCluster];
 #pragma unroll
             for (int t = 0; t < kCMaxCluster; ++t)
-                v[t] = t < C ? cluster.map_shared_rank(tcnt, t)[e] : 0;
+                v[t] = t < C ? allc[t * E + e] : 0;
             int32_t pre = 0, cp = 0, cr = 0;
 #pragma unroll
             for (int t = 0; t < kCMaxCluster; ++t) {
@@ -442,9 +448,6 @@ layout_cluster_kernel(LayoutArgs a) {
         carry += chunk;
     }
     if (threadIdx.x == 0) ebase[E] = carry;
-    // This block reads no other block's shared memory from here on; it keeps its own
-    // (which the others may still be reading) until the matching wait at the end.
-    cluster_arrive_release();
     __syncthreads();
     mark_padding(a, ebase, etot, tile, C);
 
@@ -463,7 +466,6 @@ layout_cluster_kernel(LayoutArgs a) {
         }
     }
     scatter_slots<STEPS>(a, base, wlo, hi, pk, tpre, colp, mine, ebase);
-    cluster_wait_acquire();
 }
 
 int pow2_at_least(int64_t x) {
@@ -487,7 +489,8 @@ bool cluster_geometry(const moedisp_dims& d, int* tpr, int64_t* tile_len, int* s
 }
 
 size_t cluster_smem(int E) {
-    return (size_t)(E + 1) * sizeof(int64_t) + ((size_t)kCWarps * (E | 1) + 5 * (size_t)E) * sizeof(int32_t);
+    return (size_t)(E + 1) * sizeof(int64_t) +
+           ((size_t)kCWarps * (E | 1) + (4 + kCMaxCluster) * (size_t)E) * sizeof(int32_t);
 }
 
 // Whether a cluster of C blocks of this kernel can be resident on the current device.
