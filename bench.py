@@ -1,12 +1,15 @@
 """Benchmark of the EP MoE dispatch / combine hot path on B200.
 
-One step = one pass of the whole path over one batch of the ``cfg2`` workload (W=8
-virtual EP ranks x T=256 tokens, H=4096 bf16, E=64, K=8): dispatch layout (2 kernels),
-exchange plan of the layout's send counts (1 kernel), dispatch copy (1 kernel), combine
-(1 kernel) with the dispatched rows as the experts' outputs (identity expert). Inputs are
-resident in HBM when the timed region starts; L2 is flushed before every timed step
-(a 512 MiB write, then a 256 MiB read of another buffer so no dirty line is left to be
-written back), outside the per-step CUDA-event pair.
+One step = one pass of the whole path over one batch of the ``cfg3`` workload, the
+largest configuration (W=8 virtual EP ranks x T=4096 tokens, H=7168 bf16 with 1 %
+outlier rows, E=256, K=8 Zipf(1.2)-skewed experts, per-token dynamic int8 quantisation):
+dispatch layout (three kernels: tile histograms, column scans, ranking + scatter),
+exchange plan of the layout's send counts (1 kernel, on a side-stream branch), quantising
+dispatch (1 kernel), combine (1 kernel) of N(0,1) bf16 expert outputs. Inputs are resident
+in HBM when the timed region starts; L2 is flushed before every timed step (a 512 MiB
+write, then a 256 MiB read of another buffer so no dirty line is left to be written
+back), outside the per-step CUDA-event pair. ``--workload cfg2|cfg4`` runs another
+configuration as the step.
 
 Prints ONE JSON line (rank 0). ``value`` = tokens/s over all ranks (each rank runs an
 independent replica: weak scaling, no data-path collective); ``e2e`` = the same metric
@@ -40,7 +43,7 @@ UNIT = "tokens/s"
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 512 << 20     # written, then a separate 256 MiB buffer is read
 L2_READ_BYTES = 256 << 20
-LAUNCHES_PER_STEP = 5          # layout (2 kernels), plan, dispatch, combine
+CPU_SAMPLE_T = 256             # tokens per rank of the oracle's bounded sample
 
 
 def log(*a):
@@ -250,6 +253,35 @@ def capture(torch, fn):
     return g
 
 
+def kernel_launches(torch, fn):
+    """Kernel nodes in a CUDA graph of fn (the library's kernels of one step; the graph
+    holds nothing else), or None if the runtime cannot be asked."""
+    import ctypes
+    try:
+        rt = ctypes.CDLL("libcudart.so.12")
+        g = torch.cuda.CUDAGraph(keep_graph=True)
+        with torch.cuda.graph(g):
+            fn()
+        torch.cuda.synchronize()
+        h = ctypes.c_void_p(g.raw_cuda_graph())
+        n = ctypes.c_size_t(0)
+        if rt.cudaGraphGetNodes(h, None, ctypes.byref(n)) != 0:
+            return None
+        nodes = (ctypes.c_void_p * max(n.value, 1))()
+        if rt.cudaGraphGetNodes(h, nodes, ctypes.byref(n)) != 0:
+            return None
+        kinds = ctypes.c_int(0)
+        k = 0
+        for i in range(n.value):
+            if rt.cudaGraphNodeGetType(ctypes.c_void_p(nodes[i]), ctypes.byref(kinds)) != 0:
+                return None
+            k += kinds.value == 0                    # cudaGraphNodeTypeKernel
+        del g
+        return k
+    except Exception:
+        return None
+
+
 class L2Flush:
     """Writes a 512 MiB buffer (> 4x L2), then reads a separate 256 MiB one: the read
     evicts the dirty lines of the write, so the timed region starts with L2 holding
@@ -439,40 +471,80 @@ def oracle_step(oracle, w):
         oracle.moe_combine_f32(eo, lay["dst_row"], w.weights, w.K)
 
 
+def cpu_sample(w, T_s=CPU_SAMPLE_T):
+    """A bounded sample of workload w for the CPU oracle: the first T_s tokens of every
+    source rank (same ranks, experts, routing, hidden size and quantisation), so that one
+    oracle step takes about a second however large w is."""
+    import workloads as wl
+    if w.T <= T_s:
+        return w
+    rows = np.concatenate([np.arange(r * w.T, r * w.T + T_s) for r in range(w.W)])
+    act = None if w.active is None else np.ascontiguousarray(w.active[rows])
+    return wl.MoEWorkload(name=w.name, W=w.W, T=T_s, H=w.H, E=w.E, K=w.K,
+                          quant_mode=w.quant_mode, x_bits=np.ascontiguousarray(w.x_bits[rows]),
+                          expert_ids=np.ascontiguousarray(w.expert_ids[rows]),
+                          weights=np.ascontiguousarray(w.weights[rows]), active=act,
+                          recipe=dict(w.recipe, sample_T=T_s))
+
+
+def sample_note(w, s):
+    return (f"the first {s.T} of each rank's {w.T} tokens of {w.name} ({s.G} of {w.G} tokens; "
+            f"same W, H, E, K, routing and quantisation), full oracle steps (layout, plan, "
+            f"dispatch, fp32 combine) on one host thread")
+
+
 def cpu_baseline(w, budget_s=10.0):
     import oracle
     cores = len(os.sched_getaffinity(0))
-    oracle_step(oracle, w)                       # warm-up (builds the library if needed)
+    s = cpu_sample(w)
+    oracle_step(oracle, s)                       # warm-up (builds the library if needed)
     t0 = time.perf_counter()
     n = 0
     while True:
-        oracle_step(oracle, w)
+        oracle_step(oracle, s)
         n += 1
         el = time.perf_counter() - t0
         if el >= budget_s:
             break
-    return {"value": n * w.G / el, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{n} full {w.name} steps (layout, plan, dispatch, fp32 combine) on one "
-                      f"host thread, {el:.1f} s; {cores} cores visible"}
+    return {"value": n * s.G / el, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{n} steps of {sample_note(w, s)}, {el:.1f} s; {cores} cores visible"}
 
 
-def config_of(w, flush_note=True):
-    c = {"workload": f"{w.name}: W={w.W} virtual EP ranks x T={w.T} tokens, H={w.H} bf16, "
-                     f"E={w.E}, K={w.K}, quant={'none' if w.quant_mode == 0 else w.quant_mode}",
-         "global_batch": w.G, "seq_len": 1, "parallelism": "ep-virtual (one GPU)"}
-    if flush_note:
-        c["l2"] = "flushed before every timed step (512 MiB write, then 256 MiB read of another buffer)"
-    return c
+def dtype_of(w):
+    """Arithmetic types of the step: bf16 rows, the dispatch codes, fp32 combine sums."""
+    return {0: "bf16", 2: "bf16 in, int8 codes + f32 scales, f32 combine",
+            3: "bf16 in, e4m3 codes + f32 scales, f32 combine"}[w.quant_mode]
+
+
+def config_of(w):
+    return {"workload": f"{w.name}: W={w.W} virtual EP ranks x T={w.T} tokens, H={w.H} bf16, "
+                        f"E={w.E}, K={w.K}, quant={'none' if w.quant_mode == 0 else w.quant_mode}",
+            "global_batch": w.G, "seq_len": 1, "parallelism": "ep-virtual (one GPU)",
+            "l2": "flushed before every timed step (512 MiB write, then 256 MiB read of another buffer)"}
 
 
 # --------------------------------------------------------------- per-op sweep
 
-def op_sweep(md, torch, device, hbm, reps=10):
+def dispatch_kernel_name(w):
+    return {0: "dispatch_copy_kernel", 2: "dispatch_quant_kernel (int8)",
+            3: "dispatch_quant_kernel (e4m3)"}[w.quant_mode]
+
+
+def op_sweep(md, torch, device, hbm, reps=10, main_workload="cfg3"):
     import workloads as wl
     out = []
     flush = L2Flush(torch, device)
-    for name in ("cfg3", "cfg4"):
-        w = wl.moe_workload(name, seed=0)
+    cache = {}
+
+    def moe(name):
+        if name not in cache:
+            cache[name] = wl.moe_workload(name, seed=0)
+        return cache[name]
+
+    for name in ("cfg2", "cfg3", "cfg4"):
+        if name == main_workload:
+            continue
+        w = moe(name)
         st = MoEStep(md, torch, w, device)
         g = capture(torch, st.run)
         t_step = time_graph(torch, g, reps, 3, flush)
@@ -493,7 +565,7 @@ def op_sweep(md, torch, device, hbm, reps=10):
     # fused tail: combine + residual add + RMSNorm (residual_out written), after the step's
     # layout and dispatch
     for name in ("cfg2", "cfg3"):
-        w = wl.moe_workload(name, seed=0)
+        w = moe(name)
         st = MoEStep(md, torch, w, device)
         st.run()
         g = torch.Generator(device=device).manual_seed(11)
@@ -523,7 +595,7 @@ def op_sweep(md, torch, device, hbm, reps=10):
         torch.cuda.empty_cache()
     # dispatch with per-expert smoothing before the dynamic quantisation
     for name in ("cfg3", "cfg4"):
-        w = wl.moe_workload(name, seed=0)
+        w = moe(name)
         st = MoEStep(md, torch, w, device)
         st.run()
         sm = torch.from_numpy(wl.smooth_scales(w.E, w.H, seed=1)).to(device)
@@ -553,7 +625,7 @@ def op_sweep(md, torch, device, hbm, reps=10):
     # layout with expert segments padded to multiples of 128 rows (grouped-GEMM tiles),
     # beside the unpadded layout timed the same way (eager launches, flushed L2)
     for name, A in (("cfg2", 0), ("cfg2", 128), ("cfg3", 0), ("cfg3", 128)):
-        w = wl.moe_workload(name, seed=0)
+        w = moe(name)
         L = md.LayoutBuffers.allocate(w.W, w.T, w.K, w.E, device=device, major_align=A)
         ids = torch.from_numpy(w.expert_ids.reshape(-1)).to(device)
         act = None if w.active is None else torch.from_numpy(w.active).to(device)
@@ -580,7 +652,7 @@ def op_sweep(md, torch, device, hbm, reps=10):
     # (sharedExpertNum 1), the 64 routed experts live on the other 4; every token also
     # goes to its shared replica (9 rows per token). Step: widened routing -> layout ->
     # dispatch -> combine, one graph.
-    w = wl.moe_workload("cfg2", seed=0)
+    w = moe("cfg2")
     S_, N_ = 4, 1
     ne_ = w.E // (w.W - S_)
     Kw, Ew = w.K + N_, w.W * ne_
@@ -668,7 +740,7 @@ def op_sweep(md, torch, device, hbm, reps=10):
     # tokens into the 8 ranks' separate buffers through a pointer table, then each combines
     # its own tokens from them (one stream per rank; on one GPU the "peers" are local
     # allocations, so this measures the kernels' addressing, not NVLink)
-    w = wl.moe_workload("cfg2", seed=0)
+    w = moe("cfg2")
     st = MoEStep(md, torch, w, device)
     st.run()
     rb = st.L.rank_base.cpu().numpy()
@@ -859,7 +931,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="cfg2")
+    ap.add_argument("--workload", default="cfg3")
     ap.add_argument("--T", type=int, default=None,
                     help="tokens per rank override (smaller cases for profiling)")
     ap.add_argument("--a2a-W", type=int, default=64, help="ranks of the a2a64 workload")
@@ -912,6 +984,7 @@ def main():
         pass
     sampler = ClockSampler(enabled=(rank == 0))
 
+    launches = kernel_launches(torch, step.run)
     g_step = capture(torch, step.run)
     sampler.start()                    # clocks sampled over warm-up, timed steps, per-op timing
     for _ in range(args.warmup):
@@ -943,7 +1016,7 @@ def main():
     dom = max(("dispatch", "combine"), key=lambda o: per_op[o])
     dom_bytes = algorithmic_bytes(dom, w, R)
     achieved = dom_bytes / (per_op[dom] * 1e-3) / 1e9
-    kernel_key = {"dispatch": "dispatch_copy_kernel", "combine": f"combine_kernel<{w.K}>"}[dom]
+    kernel_key = {"dispatch": dispatch_kernel_name(w), "combine": f"combine_kernel<{w.K}>"}[dom]
     traffic = ncu_traffic(kernel_key)
 
     e2e = None
@@ -960,7 +1033,7 @@ def main():
     if rank == 0 and world == 1 and not args.no_ops:
         del step
         torch.cuda.empty_cache()
-        ops = op_sweep(md, torch, device, hbm)
+        ops = op_sweep(md, torch, device, hbm, main_workload=w.name)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w)
@@ -983,7 +1056,7 @@ def main():
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": dtype_of(w),
         "data": "synthetic (seeded generator; no dataset)",
         "config": config_of(w),
         "timing": "CUDA-graph replay of the step (exchange plan on a side-stream branch beside "
@@ -997,7 +1070,8 @@ def main():
                      "peak": hbm, "peak_source": peak_src, "unit": "GB/s",
                      "frac": round(achieved / hbm, 4), "traffic": traffic,
                      "algorithmic_bytes": dom_bytes},
-        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "gpu_launches": None if launches is None else launches * args.steps,
+        "launches_per_step": launches,
         "clocks": clocks,
         "e2e": e2e,
         "cpu_baseline": cpu,
@@ -1055,25 +1129,25 @@ def run_a2a(args, wl, world, rank, local_rank):
 def run_reference(args, wl):
     import oracle
     w = wl.moe_workload(args.workload, seed=0)
+    s = cpu_sample(w)
     cores = len(os.sched_getaffinity(0))
     for _ in range(args.warmup):
-        oracle_step(oracle, w)
+        oracle_step(oracle, s)
     ts = []
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        oracle_step(oracle, w)
+        oracle_step(oracle, s)
         ts.append(time.perf_counter() - t0)
     ms = statistics.mean(ts) * 1e3
-    value = round(w.G / (ms / 1e3), 1)
+    value = round(s.G / (ms / 1e3), 1)
     line = {
         "impl": "reference",
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded generator; no dataset)", "config": config_of(w, False),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": dtype_of(w),
+        "data": "synthetic (seeded generator; no dataset)", "config": config_of(w),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": f"each step one full {w.name} pass (layout, plan, dispatch, "
-                                   f"fp32 combine) on one host thread; {cores} cores visible"},
+                         "sample": f"each step: {sample_note(w, s)}; {cores} cores visible"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

@@ -89,6 +89,7 @@ _dispatch_peers = _sig("moedisp_moe_dispatch_peers",
 _combine_peers = _sig("moedisp_moe_combine_peers",
                       [_P, ctypes.c_int64, _I, Dims, _I, _P, ctypes.POINTER(Layout), _P, _P, _P,
                        _P])
+_ep_barrier = _sig("moedisp_ep_barrier", [_P, _I, _I, ctypes.c_uint32, ctypes.c_uint32, _P, _P])
 _shared = _sig("moedisp_shared_expert_routing",
                [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P])
 _combine_rms = _sig("moedisp_moe_combine_rmsnorm",
@@ -317,6 +318,16 @@ def moe_dispatch_peers(x, H, layout: LayoutBuffers, rank, expert_ids, quant_mode
     return _check(rc, "moe_dispatch_peers", raise_on_error)
 
 
+def ep_barrier(peer_signals, W, rank, epoch, timeout_us, status, stream=None,
+               raise_on_error=True) -> int:
+    """Barrier across the W expert-parallel ranks: peer_signals is a device int64 tensor [W]
+    of the ranks' signal-array addresses (uint32 [W] each, peer memory mapped into this
+    GPU); a wait beyond timeout_us sets STATUS_TIMEOUT in `status` instead of hanging."""
+    rc = _ep_barrier(_ptr(peer_signals), int(W), int(rank), ctypes.c_uint32(int(epoch) & 0xFFFFFFFF),
+                     ctypes.c_uint32(int(timeout_us)), _ptr(status), _stream(stream))
+    return _check(rc, "ep_barrier", raise_on_error)
+
+
 def moe_combine_peers(peer_expert_out, peer_rows_cap, H, layout: LayoutBuffers, rank, expert_ids,
                       expert_scales, y, status, stream=None, raise_on_error=True) -> int:
     """Rank `rank`'s combine over W GPUs: peer_expert_out is a device int64 tensor [W] of
@@ -354,7 +365,8 @@ def raw_call(name: str, *args) -> int:
                 "moedisp_moe_dispatch_gather": _dispatch_gather,
                 "moedisp_a2a_token_rows": _token_rows,
                 "moedisp_moe_dispatch_peers": _dispatch_peers,
-                "moedisp_moe_combine_peers": _combine_peers}[name](*args))
+                "moedisp_moe_combine_peers": _combine_peers,
+                "moedisp_ep_barrier": _ep_barrier}[name](*args))
 
 
 __all__ = [

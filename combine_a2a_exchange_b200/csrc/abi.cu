@@ -173,6 +173,17 @@ int moedisp_selftest_bounded_wait(uint32_t limit_us, int32_t* status, moedisp_st
     return rc(moedisp::launch_bounded_wait_selftest((uint64_t)limit_us * 1000ull, status, stream));
 }
 
+int moedisp_ep_barrier(uint32_t* const* peer_signals, int W, int rank, uint32_t epoch,
+                       uint32_t timeout_us, int32_t* status, moedisp_stream_t stream) {
+    if (!peer_signals || !status) return MOEDISP_ERR_NULLPTR;
+    if (W < 1 || rank < 0 || rank >= W) return MOEDISP_ERR_INVALID;
+    if (W > MOEDISP_MAX_W) return MOEDISP_ERR_UNSUPPORTED;
+    if (timeout_us < 1 || timeout_us > 10000000u) return MOEDISP_ERR_INVALID;
+    if (!aligned(peer_signals, 8) || !aligned(status, 4)) return MOEDISP_ERR_MISALIGNED;
+    return rc(moedisp::launch_ep_barrier(peer_signals, W, rank, epoch,
+                                         (uint64_t)timeout_us * 1000ull, status, stream));
+}
+
 int moedisp_a2a_exchange_plan(const int64_t* in_splits, int W, int64_t* src_offsets,
                               int64_t* out_splits, int64_t* dst_offsets, int32_t* status,
                               moedisp_stream_t stream) {
@@ -330,8 +341,11 @@ int moedisp_a2a_token_rows(const int64_t* src_offsets, const int64_t* out_splits
     if (!status) return MOEDISP_ERR_NULLPTR;
     if (W < 1 || T < 0 || in_rank_stride_rows < 0) return MOEDISP_ERR_INVALID;
     if (W > MOEDISP_MAX_W) return MOEDISP_ERR_UNSUPPORTED;
-    if ((int64_t)W * T == 0) return MOEDISP_OK;
-    if (!src_offsets || !out_splits || !dst_offsets || !token_rows) return MOEDISP_ERR_NULLPTR;
+    // With T = 0 there are no positions, but a given plan is still checked for rows that
+    // would need one (CAPACITY).
+    if (T == 0 && (!src_offsets || !out_splits || !dst_offsets)) return MOEDISP_OK;
+    if (!src_offsets || !out_splits || !dst_offsets || (T > 0 && !token_rows))
+        return MOEDISP_ERR_NULLPTR;
     if (!aligned(src_offsets, 8) || !aligned(out_splits, 8) || !aligned(dst_offsets, 8) ||
         !aligned(token_rows, 8) || !aligned(status, 4))
         return MOEDISP_ERR_MISALIGNED;

@@ -105,6 +105,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     return mbar_wait_for(bar, parity, kWaitLimitNs);
 }
 
+// After a wait that timed out: waits, within one more time limit in total, for the loads
+// still armed on the stage barriers of pieces [first, end) -- piece q on barrier
+// q % stages, phase parity (q / stages) & 1 -- so that no bulk copy lands in this block's
+// shared memory after the block has exited. False if some load did not complete in time
+// (the caller has already raised MOEDISP_STATUS_TIMEOUT; the outputs are undefined).
+__device__ __forceinline__ bool mbar_drain(uint64_t* bars, int stages, int64_t first,
+                                           int64_t end) {
+    const uint64_t t0 = global_timer_ns();
+    for (int64_t q = first; q < end; ++q) {
+        const uint64_t spent = global_timer_ns() - t0;
+        if (spent >= kWaitLimitNs) return false;
+        if (!mbar_wait_for(&bars[q % stages], (uint32_t)((q / stages) & 1), kWaitLimitNs - spent))
+            return false;
+    }
+    return true;
+}
+
 // ------------------------------------------------------- 1-D bulk (TMA) copies
 // Addresses must be 16-byte aligned and sizes multiples of 16 bytes.
 

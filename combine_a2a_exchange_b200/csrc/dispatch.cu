@@ -314,6 +314,7 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
     };
 
     for (int st = 0; st < S; ++st) fill(st);
+    int64_t filled = S;                 // pipeline iterations whose stage has been filled
 
     const bool issuer = lane < K;
     for (int it = 0;; ++it) {
@@ -325,7 +326,12 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
         if (lane == 0) ok = mbar_wait(&bars[st], par) ? 1 : 0;
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) {
-            if (lane == 0) raise_status(a.status, MOEDISP_STATUS_TIMEOUT);
+            // Stop filling, and let the row loads already armed land before the block
+            // exits (a stage filled with the end-of-work marker completes at once).
+            if (lane == 0) {
+                raise_status(a.status, MOEDISP_STATUS_TIMEOUT);
+                (void)mbar_drain(bars, S, it, filled);
+            }
             break;
         }
         (void)mbar_wait(&bars[st], par);
@@ -346,6 +352,7 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
             if (issuer) bulk_wait_read<1>();
             __syncwarp();
             fill((it - 1) % S);
+            filled = it - 1 + S + 1;
         }
     }
     if (issuer) bulk_wait<0>();

@@ -110,10 +110,13 @@ a2a_v_kernel(const uint8_t* __restrict__ in, int64_t in_stride_rows, uint8_t* __
 
     const int64_t pro = min64(kA2AStages, mine);
     for (int64_t q = 0; q < pro; ++q) issue(q);
+    int64_t issued = pro;                               // pieces whose loads were armed
     for (int64_t q = 0; q < mine; ++q) {
         const int st = (int)(q % kA2AStages);
         if (!mbar_wait(&bars[st], (uint32_t)((q / kA2AStages) & 1))) {
+            // Stop issuing, and let the loads already armed land before the block exits.
             raise_status(status, MOEDISP_STATUS_TIMEOUT);
+            (void)mbar_drain(bars, kA2AStages, q, issued);
             break;
         }
         bulk_store(dst + piece_off(q), stage_buf + st * kA2APiece, piece_len(q));
@@ -123,6 +126,7 @@ a2a_v_kernel(const uint8_t* __restrict__ in, int64_t in_stride_rows, uint8_t* __
         if (q >= 1 && q - 1 + kA2AStages < mine) {
             bulk_wait_read<1>();
             issue(q - 1 + kA2AStages);
+            issued = q + kA2AStages;
         }
     }
     bulk_wait<0>();
@@ -136,7 +140,9 @@ a2a_v_kernel(const uint8_t* __restrict__ in, int64_t in_stride_rows, uint8_t* __
 // of source rank j, where j is the segment holding p (dst_offsets[i] is the exclusive scan
 // of out_splits[i], so j is the last segment starting at or before p); that row is
 // j * in_rank_stride_rows + ... of the concatenated input. Other positions get -1 (and,
-// with an active mask, 0). A segment outside its sender's rows gives -1 and BAD_SPLIT.
+// with an active mask, 0). A segment outside its sender's rows gives -1 and BAD_SPLIT; a
+// rank that receives more than T rows in total (rows that have no position) sets
+// CAPACITY, as a2a_v flags a receive buffer too small for its rows.
 __global__ void __launch_bounds__(kPlanThreads)
 a2a_token_rows_kernel(const int64_t* __restrict__ src_offsets,
                       const int64_t* __restrict__ out_splits,
@@ -147,8 +153,16 @@ a2a_token_rows_kernel(const int64_t* __restrict__ src_offsets,
     grid_dep_launch_dependents();
     const int64_t n = (int64_t)W * T;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t first = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    // Rows received by rank i end at its last segment's end (dst_offsets[i] is the
+    // exclusive scan of out_splits[i]); beyond T they have no receive position.
+    for (int64_t i = first; i < W; i += stride) {
+        const int64_t last = i * W + W - 1;
+        if (__ldg(dst_offsets + last) + __ldg(out_splits + last) > T)
+            raise_status(status, MOEDISP_STATUS_CAPACITY);
+    }
     bool bad = false;
-    for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < n; g += stride) {
+    for (int64_t g = first; g < n; g += stride) {
         const int i = (int)(g / T);
         const int64_t p = g - (int64_t)i * T;
         const int64_t* dst = dst_offsets + (int64_t)i * W;

@@ -91,6 +91,10 @@ cudaError_t launch_layout_noalloc(const int32_t* expert_ids, const uint8_t* acti
 
 cudaError_t launch_bounded_wait_selftest(uint64_t limit_ns, int32_t* status, cudaStream_t stream);
 
+// Barrier across W ranks over peer-mapped signal words (bounded wait).
+cudaError_t launch_ep_barrier(uint32_t* const* peer_signals, int W, int rank, uint32_t epoch,
+                              uint64_t limit_ns, int32_t* status, cudaStream_t stream);
+
 cudaError_t launch_a2a_token_rows(const int64_t* src_offsets, const int64_t* out_splits,
                                   const int64_t* dst_offsets, int W, int64_t T,
                                   int64_t in_rank_stride_rows, int64_t* token_rows,

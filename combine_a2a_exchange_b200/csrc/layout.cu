@@ -488,9 +488,11 @@ bool cluster_geometry(const moedisp_dims& d, int* tpr, int64_t* tile_len, int* s
     return *steps <= kCMaxSteps;
 }
 
-size_t cluster_smem(int E) {
+// Dynamic shared memory of a cluster of C blocks: expert bases, the warps' counts, four
+// per-expert rows and the C pushed rows of tile counts.
+size_t cluster_smem(int E, int C) {
     return (size_t)(E + 1) * sizeof(int64_t) +
-           ((size_t)kCWarps * (E | 1) + (4 + kCMaxCluster) * (size_t)E) * sizeof(int32_t);
+           ((size_t)kCWarps * (E | 1) + (4 + (size_t)C) * (size_t)E) * sizeof(int32_t);
 }
 
 // Whether a cluster of C blocks of this kernel can be resident on the current device.
@@ -634,7 +636,7 @@ cudaError_t launch_layout(const int32_t* expert_ids, const uint8_t* active, int 
     int64_t tile_c = 0;
     if (cluster_geometry(dims, &tpr_c, &tile_c, &steps_c)) {
         const int C = dims.W * tpr_c;
-        const size_t smem = cluster_smem(dims.E);
+        const size_t smem = cluster_smem(dims.E, C);
         void (*kernel)(LayoutArgs) =
             steps_c == 1 ? layout_cluster_kernel<1> : steps_c == 2 ? layout_cluster_kernel<2>
             : steps_c == 4 ? layout_cluster_kernel<4> : layout_cluster_kernel<8>;

@@ -16,7 +16,9 @@
  *  - Device-detected errors are OR-ed into `*status` (an int32 in device memory that the
  *    caller zeroes) as MOEDISP_STATUS_* bits; read it after the stream completes. No
  *    kernel traps, asserts or waits without bound: every device-side wait gives up after
- *    about two seconds and sets MOEDISP_STATUS_TIMEOUT.
+ *    about two seconds and sets MOEDISP_STATUS_TIMEOUT. A kernel that times out stops
+ *    issuing copies and waits (again with a limit) for the ones in flight before it
+ *    exits; the outputs of a call that reported MOEDISP_STATUS_TIMEOUT are undefined.
  *  - Empty inputs (no rows, no tokens, all splits 0) are valid no-ops.
  *  - Integer, index, copy and quantisation outputs are deterministic and bit-exact
  *    against a plain CPU implementation; combine sums each token's K rows in fp32 in
@@ -307,7 +309,9 @@ int moedisp_moe_dispatch_gather(const void *x, int64_t x_rows, const int64_t *to
  * senders' concatenated input (a2a_v's `in`); other positions get -1.
  * token_rows: int64 [W][T] device; active: uint8 [W][T] device (1 where a row is received,
  * the layout's per-token mask) or NULL. A segment leaving its sender's rows gives -1 and
- * MOEDISP_STATUS_BAD_SPLIT. */
+ * MOEDISP_STATUS_BAD_SPLIT. A rank that receives more than T rows in total (its last
+ * segment ends beyond T) sets MOEDISP_STATUS_CAPACITY: the rows past T have no position
+ * and are not dispatched. */
 int moedisp_a2a_token_rows(const int64_t *src_offsets, const int64_t *out_splits,
                            const int64_t *dst_offsets, int W, int64_t T,
                            int64_t in_rank_stride_rows, int64_t *token_rows, uint8_t *active,
@@ -347,6 +351,28 @@ int moedisp_moe_combine_peers(const void *const *peer_expert_out, int64_t peer_r
                               moedisp_dims dims, int rank, const int32_t *expert_ids,
                               const moedisp_layout *layout, const float *expert_scales, void *y,
                               int32_t *status, moedisp_stream_t stream);
+
+/* ep_barrier
+ *
+ * Orders the W ranks of moe_dispatch_peers / moe_combine_peers on the GPUs themselves,
+ * with a time limit (this library's own addition: the PyTorch symm_mem change orders its
+ * ranks with signal-pad barriers that wait without one). Each rank owns a signal array of
+ * W uint32 words in peer-mappable device memory, zeroed once before the first barrier;
+ * peer_signals is a device array of W pointers to the ranks' arrays as mapped into this
+ * GPU (its own included), 8-byte aligned. Rank `rank`'s call, in stream order:
+ *   - after every earlier kernel on the stream has completed (its writes into peers'
+ *     buffers included), stores `epoch` into word `rank` of every rank's array (a
+ *     system-scope release);
+ *   - waits until every word of its own array has reached `epoch` (acquire loads, compared
+ *     with wrap-around), so that no rank's later kernels start before every rank has
+ *     finished its earlier ones.
+ * epoch: 1, 2, 3, ... in the same sequence on every rank (one per barrier; words are never
+ * reset). A wait longer than timeout_us (1..10^7 microseconds) gives up, ORs
+ * MOEDISP_STATUS_TIMEOUT into *status and returns: a rank that died or fell behind is
+ * reported, not waited for (the caller reads the status and stops). W = 1 only publishes.
+ * One block. */
+int moedisp_ep_barrier(uint32_t *const *peer_signals, int W, int rank, uint32_t epoch,
+                       uint32_t timeout_us, int32_t *status, moedisp_stream_t stream);
 
 /* shared_expert_routing
  *

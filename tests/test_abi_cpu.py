@@ -292,3 +292,19 @@ def test_binding_host_logic(md):
     assert L.rows_cap == 4 * 8 * 3 + 8 * 16 and L.assist_info.numel() == L.rows_cap
     L = md.LayoutBuffers.allocate(4, 8, 3, 8, device="cpu", major_align=1)
     assert L.rows_cap == 4 * 8 * 3
+
+
+def test_ep_barrier_rejections(md):
+    tab, st = FAKE + (1 << 20), FAKE + (2 << 20)
+    b = lambda tab=tab, W=2, rank=0, to=1000, st=st: md.raw_call(
+        "moedisp_ep_barrier", tab, W, rank, 1, to, st, None)
+    assert b(tab=None) == md.MOEDISP_ERR_NULLPTR
+    assert b(st=None) == md.MOEDISP_ERR_NULLPTR
+    assert b(W=0) == md.MOEDISP_ERR_INVALID
+    assert b(rank=2) == md.MOEDISP_ERR_INVALID
+    assert b(rank=-1) == md.MOEDISP_ERR_INVALID
+    assert b(to=0) == md.MOEDISP_ERR_INVALID                   # no limit is not allowed
+    assert b(to=10000001) == md.MOEDISP_ERR_INVALID
+    assert b(W=70000, rank=1) == md.MOEDISP_ERR_UNSUPPORTED
+    assert b(tab=tab + 4) == md.MOEDISP_ERR_MISALIGNED
+    assert b(st=st + 2) == md.MOEDISP_ERR_MISALIGNED

@@ -106,3 +106,58 @@ def test_ep_routing_all_gather_gives_every_rank_the_global_layout():
         assert p.exitcode == 0
     assert all(r[1] and r[2] for r in res)
     assert res[0][3] == res[1][3]                        # the same receive ranges everywhere
+
+
+def _leaving_worker(rank, world, port, out):
+    """Step 1 on every rank; then rank 1 leaves (the process ends without a word) and rank
+    0 runs step 2's routing all-gather, which must fail within the group's timeout."""
+    import time
+    from datetime import timedelta
+
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import workloads as wl
+    from combine_a2a_exchange_b200.ep import gather_routing
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=5))
+    w = wl.moe_workload("tiny", seed=6, W=world, T=16, K=2, E=4)
+    T = w.T
+    ids = torch.from_numpy(w.expert_ids[rank * T:(rank + 1) * T].copy())
+    ids_all, _ = gather_routing(ids, None, None)
+    ok1 = bool((ids_all.numpy() == w.expert_ids).all())
+    if rank == 1:
+        out.put((rank, ok1, None, None))
+        out.close()
+        out.join_thread()                 # the message is out before the process ends
+        os._exit(0)                       # leaves between steps: no goodbye, no destroy
+    time.sleep(1.0)                       # rank 1 is gone by now
+    t0 = time.monotonic()
+    err = None
+    try:
+        gather_routing(ids, None, None)
+    except Exception as e:                # gloo reports the lost peer or the timeout
+        err = type(e).__name__
+    out.put((rank, ok1, err, time.monotonic() - t0))
+    out.close()
+    out.join_thread()
+    os._exit(0)
+
+
+def test_ep_rank_leaving_between_steps_fails_the_survivor_in_bounded_time():
+    """Failure detection on the host: after a completed step one rank exits; the other
+    rank's next routing all-gather raises within the process group's 5 s timeout (plus a
+    margin) instead of waiting for good. No GPU is involved."""
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_leaving_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+    assert res[0][1] and res[1][1]                       # step 1 ran on both ranks
+    rank0 = res[0]
+    assert rank0[2] is not None, "the survivor's all-gather did not fail"
+    assert rank0[3] < 30.0, rank0[3]
