@@ -886,6 +886,15 @@ def run_single_op(args, wl, md, torch):
             for r in range(w.W):
                 md.moe_combine_peers(table, cap, w.H, st.L, r, st.ids, wts[r * w.T:(r + 1) * w.T],
                                      st.y[r * w.T:(r + 1) * w.T], st.status)
+    elif args.op == "combine":
+        def op():
+            st.op_combine()
+    elif args.op == "dispatch":
+        def op():
+            st.op_dispatch()
+    elif args.op == "layout":
+        def op():
+            st.op_layout()
     elif args.op == "dispatch_smooth":
         if w.quant_mode == 0:
             raise SystemExit("dispatch_smooth needs a quantising workload (cfg3, cfg4)")
@@ -920,8 +929,14 @@ def run_single_op(args, wl, md, torch):
     if stt != 0:
         raise SystemExit(f"status {md.status_string(stt)}")
     us = statistics.mean(x.elapsed_time(y) for x, y in pairs) * 1e3
-    print(json.dumps({"op": args.op, "workload": args.workload, "us": round(us, 2),
-                      "steps": args.steps, "warmup": args.warmup}))
+    line = {"op": args.op, "workload": args.workload, "us": round(us, 2),
+            "steps": args.steps, "warmup": args.warmup}
+    if args.op in ("layout", "dispatch", "combine", "dispatch_smooth", "combine_rmsnorm"):
+        hbm, src = measured_peaks()
+        b = algorithmic_bytes(args.op, w, int(st.L.expert_base[-1].item()))
+        line.update({"bytes": b, "GB/s": round(b / us / 1e3, 1),
+                     "frac": round(b / us / 1e3 / hbm, 4), "peak_source": src})
+    print(json.dumps(line))
     return 0
 
 
@@ -939,9 +954,10 @@ def main():
     ap.add_argument("--no-ops", action="store_true", help="skip the per-op sweep of other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--op", choices=["step", "dispatch_smooth", "combine_rmsnorm", "dispatch_gather",
-                                     "peers"], default="step",
-                    help="time one NEXT-row op alone on --workload (one GPU), e.g. to profile it")
+    ap.add_argument("--op", choices=["step", "layout", "dispatch", "combine", "dispatch_smooth",
+                                     "combine_rmsnorm", "dispatch_gather", "peers"], default="step",
+                    help="time one op alone on --workload (one GPU, eager launches behind an L2 "
+                         "flush), e.g. to profile it")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 

@@ -89,6 +89,10 @@ _dispatch_peers = _sig("moedisp_moe_dispatch_peers",
 _combine_peers = _sig("moedisp_moe_combine_peers",
                       [_P, ctypes.c_int64, _I, Dims, _I, _P, ctypes.POINTER(Layout), _P, _P, _P,
                        _P])
+_pipe_ws = _sig("moedisp_a2a_dispatch_pipelined_workspace_size", [_I, ctypes.POINTER(ctypes.c_size_t)])
+_pipe = _sig("moedisp_a2a_dispatch_pipelined",
+             [_P, _I64, _P, _P, _P, _P, _I, Dims, ctypes.POINTER(Layout), _I, _P, _P, _P, _I, _P,
+              _P, ctypes.c_uint32, _I, ctypes.c_uint32, _P, ctypes.c_size_t, _P, _P])
 _ep_barrier = _sig("moedisp_ep_barrier", [_P, _I, _I, ctypes.c_uint32, ctypes.c_uint32, _P, _P])
 _shared = _sig("moedisp_shared_expert_routing",
                [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P])
@@ -318,6 +322,37 @@ def moe_dispatch_peers(x, H, layout: LayoutBuffers, rank, expert_ids, quant_mode
     return _check(rc, "moe_dispatch_peers", raise_on_error)
 
 
+PIPE_PRODUCE = 1
+PIPE_CONSUME = 2
+PIPE_BOTH = 3
+
+
+def a2a_dispatch_pipelined_workspace_size(W: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_pipe_ws(int(W), ctypes.byref(n)), "a2a_dispatch_pipelined_workspace_size", True)
+    return int(n.value)
+
+
+def a2a_dispatch_pipelined(inp, in_rank_stride_rows, src_offsets, out_splits, dst_offsets, recv,
+                           H, layout: LayoutBuffers, quant_mode, expand_x, dynamic_scales, ready,
+                           epoch, workspace, status, roles=PIPE_BOTH, wait_limit_us=2_000_000,
+                           expert_token_nums=None, expert_token_nums_type=1,
+                           ep_recv_counts=None, stream=None, raise_on_error=True) -> int:
+    """The exchange (a2a_v into recv [W][T][H]) and the dispatch of the received tokens
+    (layout over the W*T receive positions), pipelined through per-segment ready words
+    (uint32 [W][W], zeroed once; a new epoch per exchange). workspace: a device buffer of
+    a2a_dispatch_pipelined_workspace_size(W) bytes."""
+    L = layout.struct()
+    rc = _pipe(_ptr(inp), int(in_rank_stride_rows), _ptr(src_offsets), _ptr(out_splits),
+               _ptr(dst_offsets), _ptr(recv), int(H), layout.dims, ctypes.byref(L), int(quant_mode),
+               _ptr(expand_x), _ptr(dynamic_scales), _ptr(expert_token_nums),
+               int(expert_token_nums_type), _ptr(ep_recv_counts), _ptr(ready),
+               ctypes.c_uint32(int(epoch) & 0xFFFFFFFF), int(roles), ctypes.c_uint32(int(wait_limit_us)),
+               _ptr(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
+               _ptr(status), _stream(stream))
+    return _check(rc, "a2a_dispatch_pipelined", raise_on_error)
+
+
 def ep_barrier(peer_signals, W, rank, epoch, timeout_us, status, stream=None,
                raise_on_error=True) -> int:
     """Barrier across the W expert-parallel ranks: peer_signals is a device int64 tensor [W]
@@ -366,7 +401,8 @@ def raw_call(name: str, *args) -> int:
                 "moedisp_a2a_token_rows": _token_rows,
                 "moedisp_moe_dispatch_peers": _dispatch_peers,
                 "moedisp_moe_combine_peers": _combine_peers,
-                "moedisp_ep_barrier": _ep_barrier}[name](*args))
+                "moedisp_ep_barrier": _ep_barrier,
+                "moedisp_a2a_dispatch_pipelined": _pipe}[name](*args))
 
 
 __all__ = [

@@ -334,6 +334,86 @@ int moedisp_moe_dispatch_gather(const void* x, int64_t x_rows, const int64_t* to
                          ep_recv_counts, status, stream);
 }
 
+int moedisp_a2a_dispatch_pipelined_workspace_size(int W, size_t* bytes) {
+    if (!bytes) return MOEDISP_ERR_NULLPTR;
+    if (W < 1) return MOEDISP_ERR_INVALID;
+    if (W > MOEDISP_MAX_W) return MOEDISP_ERR_UNSUPPORTED;
+    *bytes = moedisp::pipeline_workspace_bytes(W);
+    return MOEDISP_OK;
+}
+
+int moedisp_a2a_dispatch_pipelined(const void* in, int64_t in_rank_stride_rows,
+                                   const int64_t* src_offsets, const int64_t* out_splits,
+                                   const int64_t* dst_offsets, void* recv, int H,
+                                   moedisp_dims dims, const moedisp_layout* layout,
+                                   int quant_mode, void* expand_x, float* dynamic_scales,
+                                   int64_t* expert_token_nums, int expert_token_nums_type,
+                                   int32_t* ep_recv_counts, uint32_t* ready, uint32_t epoch,
+                                   int roles, uint32_t wait_limit_us, void* workspace,
+                                   size_t workspace_bytes, int32_t* status,
+                                   moedisp_stream_t stream) {
+    if (!layout || !status) return MOEDISP_ERR_NULLPTR;
+    int c = check_dims(dims);
+    if (c != MOEDISP_OK) return c;
+    const moedisp_layout& L = *layout;
+    if ((c = check_rows_cap(L.rows_cap)) != MOEDISP_OK) return c;
+    if (quant_mode != MOEDISP_QUANT_NONE && quant_mode != MOEDISP_QUANT_INT8 &&
+        quant_mode != MOEDISP_QUANT_FP8_E4M3)
+        return MOEDISP_ERR_INVALID;
+    if (expert_token_nums && expert_token_nums_type != 0 && expert_token_nums_type != 1)
+        return MOEDISP_ERR_INVALID;
+    if (roles != MOEDISP_PIPE_PRODUCE && roles != MOEDISP_PIPE_CONSUME && roles != MOEDISP_PIPE_BOTH)
+        return MOEDISP_ERR_INVALID;
+    if (wait_limit_us < 1 || wait_limit_us > 10000000u) return MOEDISP_ERR_INVALID;
+    if (H <= 0 || in_rank_stride_rows < 0) return MOEDISP_ERR_INVALID;
+    if (H > MOEDISP_MAX_H) return MOEDISP_ERR_UNSUPPORTED;
+    if (H % (quant_mode == MOEDISP_QUANT_NONE ? 8 : 16) != 0) return MOEDISP_ERR_MISALIGNED;
+    const int64_t G = (int64_t)dims.W * dims.T;
+    if (G == 0 && (!src_offsets || !out_splits || !dst_offsets)) return MOEDISP_OK;
+    if (!src_offsets || !out_splits || !dst_offsets || !ready || !workspace)
+        return MOEDISP_ERR_NULLPTR;
+    if (G > 0 && (!recv || !L.dst_row)) return MOEDISP_ERR_NULLPTR;
+    if (in_rank_stride_rows > 0 && !in) return MOEDISP_ERR_NULLPTR;
+    if (L.rows_cap > 0 && !expand_x) return MOEDISP_ERR_NULLPTR;
+    if (quant_mode != MOEDISP_QUANT_NONE && L.rows_cap > 0 && !dynamic_scales)
+        return MOEDISP_ERR_NULLPTR;
+    if (expert_token_nums && (!L.expert_base || !L.rank_base)) return MOEDISP_ERR_NULLPTR;
+    if (ep_recv_counts && (!L.cnt || !L.expert_base)) return MOEDISP_ERR_NULLPTR;
+    if (workspace_bytes < moedisp::pipeline_workspace_bytes(dims.W)) return MOEDISP_ERR_WORKSPACE;
+    if (!aligned(in, 16) || !aligned(recv, 16) || !aligned(expand_x, 16) ||
+        !aligned(src_offsets, 8) || !aligned(out_splits, 8) || !aligned(dst_offsets, 8) ||
+        !aligned(L.dst_row, 4) || !aligned(dynamic_scales, 4) || !aligned(expert_token_nums, 8) ||
+        !aligned(ep_recv_counts, 4) || !aligned(ready, 4) || !aligned(workspace, 16) ||
+        !aligned(status, 4))
+        return MOEDISP_ERR_MISALIGNED;
+    const size_t row = (size_t)H * 2;
+    const size_t out_row = quant_mode == MOEDISP_QUANT_NONE ? row : (size_t)H;
+    const size_t plan = (size_t)dims.W * dims.W * 8;
+    const int ne = dims.E / dims.W;
+    const Span scales{quant_mode == MOEDISP_QUANT_NONE ? nullptr : dynamic_scales,
+                      (size_t)L.rows_cap * 4};
+    if (any_alias({{recv, (size_t)G * row},
+                   {expand_x, (size_t)L.rows_cap * out_row},
+                   scales,
+                   {expert_token_nums, (size_t)dims.E * 8},
+                   {ep_recv_counts, (size_t)dims.W * ne * dims.W * 4},
+                   {ready, (size_t)dims.W * dims.W * 4},
+                   {workspace, moedisp::pipeline_workspace_bytes(dims.W)},
+                   {status, 4}},
+                  {{in, (size_t)dims.W * in_rank_stride_rows * row},
+                   {src_offsets, plan}, {out_splits, plan}, {dst_offsets, plan},
+                   {L.dst_row, (size_t)G * dims.K * 4},
+                   {L.cnt, (size_t)dims.W * dims.E * 4},
+                   {L.expert_base, (size_t)(dims.E + 1) * 8},
+                   {L.rank_base, (size_t)(dims.W + 1) * 8}}))
+        return MOEDISP_ERR_ALIASED;
+    return rc(moedisp::launch_a2a_dispatch_pipelined(
+        in, in_rank_stride_rows, src_offsets, out_splits, dst_offsets, recv, H, dims, L,
+        quant_mode, expand_x, dynamic_scales, expert_token_nums, expert_token_nums_type,
+        ep_recv_counts, ready, epoch, roles, (uint64_t)wait_limit_us * 1000ull, workspace, status,
+        stream));
+}
+
 int moedisp_a2a_token_rows(const int64_t* src_offsets, const int64_t* out_splits,
                            const int64_t* dst_offsets, int W, int64_t T,
                            int64_t in_rank_stride_rows, int64_t* token_rows, uint8_t* active,

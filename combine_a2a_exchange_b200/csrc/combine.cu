@@ -2,11 +2,12 @@
 // in fp32 with fused multiply-adds in ascending k (a fixed order, so the result is
 // deterministic and reproducible bit for bit), skipping slots that were not routed.
 //
-// A thread owns 8 columns (one 16-byte vector) of one token: it issues all K row loads
-// before the first multiply-add, so K independent 16-byte loads per thread are in
-// flight; a warp covers 512 contiguous bytes of each row. Rows are read exactly once
-// (streaming loads), y is written once (streaming stores). The gate weight, the fp32
-// accumulation and the bf16 cast are fused into the gather.
+// A block combines one token at a time: each thread owns 16-byte vectors (8 columns) of
+// the token's row and issues the loads of two of them from all K rows before the first
+// multiply-add, so 2K independent 16-byte loads per thread are in flight; the K rows are
+// read front to back. Rows are read exactly once (streaming loads), y is written once
+// (streaming stores). The gate weight, the fp32 accumulation and the bf16 cast are fused
+// into the gather.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -43,21 +44,49 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+// FMA chain of one 16-byte vector (8 columns) over the K rows, in ascending k; rows that
+// were not routed (d[k] < 0) are skipped.
+template <int K>
+__device__ __forceinline__ uint4 combine_vec(const uint4 (&v)[K], const int32_t (&d)[K],
+                                             const float (&w)[K]) {
+    float acc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+        if (d[k] < 0) continue;
+        const float wk = w[k];
+        acc[0] = __fmaf_rn(wk, lo_f(v[k].x), acc[0]);
+        acc[1] = __fmaf_rn(wk, hi_f(v[k].x), acc[1]);
+        acc[2] = __fmaf_rn(wk, lo_f(v[k].y), acc[2]);
+        acc[3] = __fmaf_rn(wk, hi_f(v[k].y), acc[3]);
+        acc[4] = __fmaf_rn(wk, lo_f(v[k].z), acc[4]);
+        acc[5] = __fmaf_rn(wk, hi_f(v[k].z), acc[5]);
+        acc[6] = __fmaf_rn(wk, lo_f(v[k].w), acc[6]);
+        acc[7] = __fmaf_rn(wk, hi_f(v[k].w), acc[7]);
+    }
+    uint4 o;
+    o.x = pack_bf16(acc[0], acc[1]);
+    o.y = pack_bf16(acc[2], acc[3]);
+    o.z = pack_bf16(acc[4], acc[5]);
+    o.w = pack_bf16(acc[6], acc[7]);
+    return o;
+}
+
+// One token per block at a time (persistent grid-stride over tokens): its routing (K rows
+// and weights; PEERS: each row's base address in its rank's buffer) is loaded once, one
+// token ahead, and the block walks the token's columns in passes of two 16-byte vectors
+// per thread, so 2K row loads per thread are in flight; each of the K rows is read front
+// to back by one block.
 template <int K, bool PEERS>
 __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a) {
     grid_dep_wait();
     grid_dep_launch_dependents();
-    const int chunks = (a.H8 + kThreads - 1) / kThreads;
-    const int64_t items = a.G * chunks;
-    // The next item's routing (rows and weights) is loaded while this item's rows are in
-    // flight, so each item costs one dependent round trip instead of two. PEERS: each
-    // row's base address (rank table, local row) is resolved with it.
     int32_t nd[K];
     float nw[K];
     const uint4* np[PEERS ? K : 1];
-    auto load_routing = [&](int64_t item) {
-        if (item >= items) return;
-        const int64_t g = item / chunks;
+    auto load_routing = [&](int64_t g) {
+        if (g >= a.G) return;
 #pragma unroll
         for (int k = 0; k < K; ++k) {
             nd[k] = __ldg(a.dst_row + g * K + k);
@@ -74,9 +103,7 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a) {
         }
     };
     load_routing(blockIdx.x);
-    for (int64_t item = blockIdx.x; item < items; item += gridDim.x) {
-        const int64_t g = item / chunks;
-        const int vec = (int)(item - g * chunks) * kThreads + threadIdx.x;
+    for (int64_t g = blockIdx.x; g < a.G; g += gridDim.x) {
         int32_t d[K];
         float w[K];
         const uint4* p[PEERS ? K : 1];
@@ -91,37 +118,22 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a) {
                 d[k] = -1;
             }
         }
-        load_routing(item + gridDim.x);
+        load_routing(g + gridDim.x);
         if (over && threadIdx.x == 0) raise_status(a.status, MOEDISP_STATUS_CAPACITY);
-        if (vec >= a.H8) continue;
-        uint4 v[K];
+        uint4* yr = a.y + g * a.H8;
+        for (int c0 = threadIdx.x; c0 < a.H8; c0 += 2 * kThreads) {
+            const int c1 = c0 + kThreads;
+            const bool two = c1 < a.H8;
+            uint4 v0[K], v1[K];
 #pragma unroll
-        for (int k = 0; k < K; ++k) {
-            const uint4* row = PEERS ? p[PEERS ? k : 0] : a.eo + (int64_t)d[k] * a.H8;
-            v[k] = d[k] >= 0 ? __ldcs(row + vec) : make_uint4(0, 0, 0, 0);
+            for (int k = 0; k < K; ++k) {
+                const uint4* row = PEERS ? p[PEERS ? k : 0] : a.eo + (int64_t)d[k] * a.H8;
+                v0[k] = d[k] >= 0 ? __ldcs(row + c0) : make_uint4(0, 0, 0, 0);
+                v1[k] = (d[k] >= 0 && two) ? __ldcs(row + c1) : make_uint4(0, 0, 0, 0);
+            }
+            __stcs(yr + c0, combine_vec<K>(v0, d, w));
+            if (two) __stcs(yr + c1, combine_vec<K>(v1, d, w));
         }
-        float acc[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
-#pragma unroll
-        for (int k = 0; k < K; ++k) {
-            if (d[k] < 0) continue;
-            const float wk = w[k];
-            acc[0] = __fmaf_rn(wk, lo_f(v[k].x), acc[0]);
-            acc[1] = __fmaf_rn(wk, hi_f(v[k].x), acc[1]);
-            acc[2] = __fmaf_rn(wk, lo_f(v[k].y), acc[2]);
-            acc[3] = __fmaf_rn(wk, hi_f(v[k].y), acc[3]);
-            acc[4] = __fmaf_rn(wk, lo_f(v[k].z), acc[4]);
-            acc[5] = __fmaf_rn(wk, hi_f(v[k].z), acc[5]);
-            acc[6] = __fmaf_rn(wk, lo_f(v[k].w), acc[6]);
-            acc[7] = __fmaf_rn(wk, hi_f(v[k].w), acc[7]);
-        }
-        uint4 o;
-        o.x = pack_bf16(acc[0], acc[1]);
-        o.y = pack_bf16(acc[2], acc[3]);
-        o.z = pack_bf16(acc[4], acc[5]);
-        o.w = pack_bf16(acc[6], acc[7]);
-        __stcs(a.y + g * a.H8 + vec, o);
     }
 }
 
@@ -131,12 +143,9 @@ cudaError_t launch_k(const CombineArgs& a, cudaStream_t stream) {
     int per_sm = 1;
     cudaError_t err = blocks_per_sm((const void*)kernel, kThreads, 0, &per_sm);
     if (err != cudaSuccess) return err;
-    const int chunks = (a.H8 + kThreads - 1) / kThreads;
-    // All resident blocks, even if the last round of items leaves some idle: measured
-    // faster on cfg2 than the fewest blocks that divide the items evenly (fewer bytes in
-    // flight cost more than the tail).
+    // All resident blocks (more bytes in flight beat an even last round of tokens).
     int64_t grid = (int64_t)current_sm_count() * per_sm;
-    grid = std::min<int64_t>(grid, std::max<int64_t>(1, a.G * chunks));
+    grid = std::min<int64_t>(grid, std::max<int64_t>(1, a.G));
     return launch_pdl(kernel, dim3((unsigned)grid), dim3(kThreads), 0, stream, 1, a);
 }
 

@@ -1,0 +1,187 @@
+// Helpers shared by the dispatch kernels: per-token dynamic quantisation of bf16 rows
+// (int8 and fp8-e4m3: bf16 unpacking, the row maximum, the exact-but-fast code decision,
+// code packing), named barriers for groups of warps, and the receive counts
+// (expert_token_nums, ep_recv_counts) derived from the layout.
+#pragma once
+
+#include "common.cuh"
+
+namespace moedisp {
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ float absmax8(const uint4& v) {
+    float m = fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x)));
+    m = fmaxf(m, fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y))));
+    m = fmaxf(m, fmaxf(fabsf(bf16_lo(v.z)), fabsf(bf16_hi(v.z))));
+    m = fmaxf(m, fmaxf(fabsf(bf16_lo(v.w)), fabsf(bf16_hi(v.w))));
+    return m;
+}
+
+// Quantisation. The definition is q = clamp(rint(x / scale), -127, 127) for int8 and
+// q = e4m3_rn_satfinite(x / scale) for fp8, with x / scale one IEEE fp32 division. The
+// quotient is only needed near a rounding boundary of q, so it is first approximated
+// by r = x * inv, inv = 1 / scale (both correctly rounded): then
+//   |r - x/scale| <= |x/scale| * (2^-23 + 2^-48)  and  |fl(x/scale) - x/scale| <= |x/scale| * 2^-24,
+// i.e. r and the IEEE quotient differ by at most ~3 units in the last place of fp32.
+// When r is farther than that from every rounding boundary of q, both round to the same
+// q; otherwise (and for inv or r not finite) the IEEE quotient is computed. The result
+// is the definition's bit for bit; the fast test only decides which path gives it.
+
+// int8 boundaries are the half-integers; |x/scale| <= ~127, so the bound above is below
+// 2.3e-5 and a margin of 2^-14 from k + 0.5 is safe. Rounding to an integer uses the
+// floating-point adder: for |v| < 2^22, rr = v + 1.5*2^23 rounds v's fraction away to the
+// nearest integer, ties to even, and rr's bit pattern is that of 1.5*2^23 plus the
+// integer. Two exact formulations follow; each kernel uses the one measured faster in it.
+//
+// q_int8: the integer, clamped to +-127 (the clamp acts only when the scale itself is
+// inexact far beyond fp32 rounding, i.e. subnormal).
+__device__ __forceinline__ int q_int8(float x, float scale, float inv) {
+    constexpr float kMagic = 12582912.0f;                    // 1.5 * 2^23
+    float v = __fmul_rn(x, inv);
+    float rr = __fadd_rn(v, kMagic);
+    const float t = __fsub_rn(v, __fsub_rn(rr, kMagic));      // v - round(v), in [-0.5, 0.5]
+    if (!(0.5f - fabsf(t) >= 0.00006103515625f)) {            // near k + 0.5, or not finite
+        v = __fdiv_rn(x, scale);
+        if (!(fabsf(v) < 4194304.0f)) return v > 0.0f ? 127 : -127;   // |v| >= 2^22 or NaN
+        rr = __fadd_rn(v, kMagic);
+    }
+    const int q = (int)(__float_as_uint(rr) - __float_as_uint(kMagic));
+    return max(-127, min(127, q));
+}
+
+// q_int8_w: a word whose low byte is the code -- rr's own bits when |r| < 127.5, where
+// the clamp cannot act (the low byte of 1.5*2^23 + q is q's two's-complement low byte);
+// else the IEEE quotient, clamped (NaN -> -127).
+__device__ __forceinline__ uint32_t q_int8_w(float x, float scale, float inv) {
+    constexpr float kMagic = 12582912.0f;
+    const float v = __fmul_rn(x, inv);
+    const float rr = __fadd_rn(v, kMagic);
+    const float t = __fsub_rn(v, __fsub_rn(rr, kMagic));
+    if (0.5f - fabsf(t) >= 0.00006103515625f && fabsf(v) < 127.5f) return __float_as_uint(rr);
+    const float q = fminf(fmaxf(__fdiv_rn(x, scale), -127.0f), 127.0f);
+    return __float_as_uint(__fadd_rn(q, kMagic));
+}
+
+// E4M3 keeps 3 mantissa bits: for 2^-6 <= |v| < 448 its rounding boundaries are the fp32
+// values whose 20 low mantissa bits are exactly 0x80000. When r is more than 16 fp32 ulps
+// from such a boundary, rounding to nearest is adding half an E4M3 step to the bits and
+// truncating: the code is sign | ((bits + 0x80000) >> 20) - ((127 - 7) << 3), the carry
+// moving into the exponent when the mantissa rounds up. Elsewhere (near a boundary, in
+// E4M3's subnormal range, at the saturation edge, not finite) the IEEE quotient goes
+// through the hardware conversion (round to nearest even, saturating to +-448). Returns a
+// word whose low byte is the code.
+__device__ __forceinline__ uint32_t q_e4m3(float x, float scale, float inv) {
+    const float r = __fmul_rn(x, inv);
+    const uint32_t b = __float_as_uint(r);
+    const uint32_t u = b & 0x7fffffffu;
+    // (unsigned range tests: 2^-6 <= |r| < 448, and low bits outside [0x80000 +- 16])
+    if (u - 0x3c800000u < 0x43e00000u - 0x3c800000u && (u & 0xfffffu) - 0x7fff0u > 32u)
+        return ((b >> 24) & 0x80u) | (((u + 0x80000u) >> 20) - 0x3c0u);
+    const float v = __fdiv_rn(x, scale);
+    return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(v, 0.0f), __NV_SATFINITE, __NV_E4M3);
+}
+
+template <int Q>
+__device__ __forceinline__ uint32_t q_code(float x, float scale, float inv) {
+    return Q == MOEDISP_QUANT_INT8 ? q_int8_w(x, scale, inv) : q_e4m3(x, scale, inv);
+}
+
+// The low bytes of four words, in order, in one word (three byte permutes).
+__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
+// Eight fp32 values (a smoothed row chunk) to eight codes.
+template <int Q>
+__device__ __forceinline__ uint2 quant8f(const float (&v)[8], float scale, float inv, bool zero) {
+    if (zero) return make_uint2(0u, 0u);
+    uint32_t b[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) b[j] = q_code<Q>(v[j], scale, inv);
+    return make_uint2(pack_low_bytes(b[0], b[1], b[2], b[3]), pack_low_bytes(b[4], b[5], b[6], b[7]));
+}
+
+// x chunk (8 bf16) times a smoothing chunk (8 fp32, shared memory), one correctly rounded
+// product each.
+__device__ __forceinline__ void smooth8(const uint4& v, const float4* s, float (&o)[8]) {
+    const float4 s0 = s[0];
+    const float4 s1 = s[1];
+    o[0] = __fmul_rn(bf16_lo(v.x), s0.x); o[1] = __fmul_rn(bf16_hi(v.x), s0.y);
+    o[2] = __fmul_rn(bf16_lo(v.y), s0.z); o[3] = __fmul_rn(bf16_hi(v.y), s0.w);
+    o[4] = __fmul_rn(bf16_lo(v.z), s1.x); o[5] = __fmul_rn(bf16_hi(v.z), s1.y);
+    o[6] = __fmul_rn(bf16_lo(v.w), s1.z); o[7] = __fmul_rn(bf16_hi(v.w), s1.w);
+}
+
+__device__ __forceinline__ uint32_t q_int8_pair(uint32_t w, float scale, float inv) {
+    const int a = q_int8(bf16_lo(w), scale, inv);
+    const int b = q_int8(bf16_hi(w), scale, inv);
+    return (uint32_t)(a & 0xff) | ((uint32_t)(b & 0xff) << 8);
+}
+
+// Eight bf16 values (a row chunk) to eight codes: int8 as pairs of clamped integers,
+// e4m3 through byte permutes (each measured the faster in the token-order kernel).
+template <int Q>
+__device__ __forceinline__ uint2 quant8(const uint4& v, float scale, float inv, bool zero) {
+    if (zero) return make_uint2(0u, 0u);
+    if (Q == MOEDISP_QUANT_INT8) {
+        const uint32_t p0 = q_int8_pair(v.x, scale, inv), p1 = q_int8_pair(v.y, scale, inv);
+        const uint32_t p2 = q_int8_pair(v.z, scale, inv), p3 = q_int8_pair(v.w, scale, inv);
+        return make_uint2(p0 | (p1 << 16), p2 | (p3 << 16));
+    }
+    const float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                        bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+    uint32_t b[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) b[j] = q_e4m3(f[j], scale, inv);
+    return make_uint2(pack_low_bytes(b[0], b[1], b[2], b[3]), pack_low_bytes(b[4], b[5], b[6], b[7]));
+}
+
+__device__ __forceinline__ void group_barrier(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Receive counts of one layout, written by whichever dispatch kernel runs it.
+struct DispatchCounts {
+    const int32_t* cnt;            // [W][E]
+    const int64_t* expert_base;    // [E + 1]
+    const int64_t* rank_base;      // [W + 1]
+    int W, E, ne;
+    int64_t* etn;                  // [W][ne] or null
+    int etn_type;                  // 0: running sum over the rank's experts, 1: counts
+    int32_t* erc;                  // [W][ne][W] or null
+};
+
+// Grid-stride over the whole grid: ep_recv_counts[d][le][r] = cnt[r][d*ne + le] (the last
+// source rank's entry also holds the expert's padding rows under major_align), and
+// expert_token_nums per destination rank and local expert.
+__device__ __forceinline__ void write_dispatch_counts(const DispatchCounts& a) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t first = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (a.erc != nullptr) {
+        const int64_t n = (int64_t)a.W * a.ne * a.W;
+        for (int64_t idx = first; idx < n; idx += stride) {
+            const int64_t e = idx / a.W;                  // = d*ne + le
+            const int r = (int)(idx - e * a.W);
+            int32_t v = a.cnt[(int64_t)r * a.E + e];
+            if (r == a.W - 1) {
+                // the last source rank's entry absorbs the expert's padding (major_align):
+                // segment rows minus the rows routed to the expert
+                int64_t routed = 0;
+                for (int q = 0; q < a.W; ++q) routed += a.cnt[(int64_t)q * a.E + e];
+                v += (int32_t)(a.expert_base[e + 1] - a.expert_base[e] - routed);
+            }
+            a.erc[idx] = v;
+        }
+    }
+    if (a.etn != nullptr) {
+        for (int64_t e = first; e < a.E; e += stride) {
+            const int d = (int)(e / a.ne);
+            a.etn[e] = a.etn_type == 0 ? a.expert_base[e + 1] - a.rank_base[d]
+                                       : a.expert_base[e + 1] - a.expert_base[e];
+        }
+    }
+}
+
+}  // namespace moedisp

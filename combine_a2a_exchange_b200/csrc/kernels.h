@@ -120,6 +120,18 @@ cudaError_t launch_combine_peers(const void* const* peer_expert_out, int64_t pee
                                  const moedisp_layout& layout, const float* expert_scales,
                                  void* y, int32_t* status, cudaStream_t stream);
 
+// Exchange -> dispatch pipelined through per-segment ready words (set-up + one kernel).
+size_t pipeline_workspace_bytes(int W);
+cudaError_t launch_a2a_dispatch_pipelined(const void* in, int64_t in_rank_stride_rows,
+                                          const int64_t* src_offsets, const int64_t* out_splits,
+                                          const int64_t* dst_offsets, void* recv, int H,
+                                          const moedisp_dims& dims, const moedisp_layout& L,
+                                          int quant_mode, void* expand_x, float* dynamic_scales,
+                                          int64_t* expert_token_nums, int expert_token_nums_type,
+                                          int32_t* ep_recv_counts, uint32_t* ready, uint32_t epoch,
+                                          int roles, uint64_t limit_ns, void* workspace,
+                                          int32_t* status, cudaStream_t stream);
+
 cudaError_t launch_combine(const void* expert_out, int H, const moedisp_dims& dims,
                            const moedisp_layout& layout, const float* expert_scales, void* y,
                            int32_t* status, cudaStream_t stream);

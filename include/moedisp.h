@@ -299,6 +299,56 @@ int moedisp_moe_dispatch_gather(const void *x, int64_t x_rows, const int64_t *to
                                 int expert_token_nums_type, int32_t *ep_recv_counts,
                                 int32_t *status, moedisp_stream_t stream);
 
+/* a2a_dispatch_pipelined
+ *
+ * The exchange and the dispatch of the exchanged tokens overlapped through per-segment
+ * ready words, after the PyTorch symm_mem change's get-style exchange that publishes
+ * (release) how many rows of each peer have arrived while the index-push kernel spins on
+ * those words (acquire) before pushing the rows on to their experts. One call does what
+ * a2a_v followed by moe_dispatch does:
+ *   recv row (i*T + dst_offsets[i][j] + q) = in row (j*in_rank_stride_rows +
+ *       src_offsets[i][j] + q)                         for q < out_splits[i][j]  (a2a_v)
+ *   expand_x / dynamic_scales of every received token, dispatched as moe_dispatch does
+ *       with `layout` (the layout of the W*T receive positions: token g = i*T + p)
+ * but in one persistent kernel: blocks take exchange pieces of segment (i, j) and
+ * dispatch chunks of already received segments from one ticket counter (the pieces of
+ * segment s+1 come before the tokens of segment s), the block landing a segment's last
+ * rows stores ready[i*W + j] = epoch (release), and the tokens of a segment are
+ * dispatched once an acquire load sees it -- each received row is read back from L2
+ * moments after it was written.
+ * in: bf16 [W][in_rank_stride_rows][H]; recv: bf16 [W][T][H] (T = dims.T, the receive
+ * capacity), both 16-byte aligned and not overlapping; plan arrays as for a2a_v; layout,
+ * quant_mode, expand_x, dynamic_scales, expert_token_nums(_type), ep_recv_counts as for
+ * moe_dispatch (no smoothing).
+ * ready: uint32 [W][W] device, zeroed once when allocated and then left to this call;
+ * epoch: 1, 2, 3, ... a new value for every exchange (the ready words keep the last one).
+ * roles: MOEDISP_PIPE_BOTH (the normal case); MOEDISP_PIPE_PRODUCE, the exchange alone,
+ * publishing the ready words; MOEDISP_PIPE_CONSUME, the dispatch alone, for rows that
+ * another party delivered into recv and published with this epoch (a PRODUCE call of
+ * the same epoch before it, or a peer). wait_limit_us (1..10^7): a dispatch chunk whose
+ * segment is not published within this time sets MOEDISP_STATUS_TIMEOUT, and the
+ * kernel stops waiting for any segment (the outputs are then incomplete).
+ * A segment whose ranges leave their buffers (or has a negative size/offset) is neither
+ * exchanged nor dispatched and sets MOEDISP_STATUS_BAD_SPLIT.
+ * workspace: device memory of moedisp_a2a_dispatch_pipelined_workspace_size(W) bytes,
+ * 16-byte aligned, no initialisation needed; calls sharing a workspace or ready words
+ * must not run concurrently. H % 8 == 0 (NONE) or H % 16 == 0, H <= MOEDISP_MAX_H.
+ * Two kernels: a one-block set-up (segment checks, ticket offsets), then the pipeline. */
+#define MOEDISP_PIPE_PRODUCE 1
+#define MOEDISP_PIPE_CONSUME 2
+#define MOEDISP_PIPE_BOTH    3
+int moedisp_a2a_dispatch_pipelined_workspace_size(int W, size_t *bytes);
+int moedisp_a2a_dispatch_pipelined(const void *in, int64_t in_rank_stride_rows,
+                                   const int64_t *src_offsets, const int64_t *out_splits,
+                                   const int64_t *dst_offsets, void *recv, int H,
+                                   moedisp_dims dims, const moedisp_layout *layout,
+                                   int quant_mode, void *expand_x, float *dynamic_scales,
+                                   int64_t *expert_token_nums, int expert_token_nums_type,
+                                   int32_t *ep_recv_counts, uint32_t *ready, uint32_t epoch,
+                                   int roles, uint32_t wait_limit_us, void *workspace,
+                                   size_t workspace_bytes, int32_t *status,
+                                   moedisp_stream_t stream);
+
 /* a2a_token_rows
  *
  * The source of every receive position of an exchange plan (a2a_exchange_plan's outputs

@@ -308,3 +308,38 @@ def test_ep_barrier_rejections(md):
     assert b(W=70000, rank=1) == md.MOEDISP_ERR_UNSUPPORTED
     assert b(tab=tab + 4) == md.MOEDISP_ERR_MISALIGNED
     assert b(st=st + 2) == md.MOEDISP_ERR_MISALIGNED
+
+
+def test_pipelined_rejections(md):
+    L = _layout(md)
+    d = md.Dims(4, 8, 2, 8)
+    ws_need = md.a2a_dispatch_pipelined_workspace_size(4)
+    assert ws_need > 0
+    inp, so, os_, do, recv, ex, sc, ready, ws, st = (FAKE + (i << 20) for i in range(64, 74))
+
+    def p(inp=inp, stride=10, so=so, recv=recv, H=128, d=d, q=0, ex=ex, sc=None, ready=ready,
+          roles=3, lim=1000, ws=ws, wsb=ws_need, st=st):
+        return md.raw_call("moedisp_a2a_dispatch_pipelined", inp, stride, so, os_, do, recv, H, d,
+                           ctypes.byref(L), q, ex, sc, None, 1, None, ready, 1, roles, lim, ws, wsb,
+                           st, None)
+    assert p(st=None) == md.MOEDISP_ERR_NULLPTR
+    assert p(ready=None) == md.MOEDISP_ERR_NULLPTR
+    assert p(ws=None) == md.MOEDISP_ERR_NULLPTR
+    assert p(so=None) == md.MOEDISP_ERR_NULLPTR
+    assert p(recv=None) == md.MOEDISP_ERR_NULLPTR
+    assert p(inp=None) == md.MOEDISP_ERR_NULLPTR
+    assert p(q=2) == md.MOEDISP_ERR_NULLPTR                    # quantising without scales
+    assert p(roles=0) == md.MOEDISP_ERR_INVALID
+    assert p(roles=4) == md.MOEDISP_ERR_INVALID
+    assert p(lim=0) == md.MOEDISP_ERR_INVALID
+    assert p(stride=-1) == md.MOEDISP_ERR_INVALID
+    assert p(q=1) == md.MOEDISP_ERR_INVALID
+    assert p(H=100) == md.MOEDISP_ERR_MISALIGNED
+    assert p(H=136, q=3, sc=sc) == md.MOEDISP_ERR_MISALIGNED   # quantised rows need H % 16
+    assert p(H=32768) == md.MOEDISP_ERR_UNSUPPORTED
+    assert p(wsb=ws_need - 1) == md.MOEDISP_ERR_WORKSPACE
+    assert p(recv=recv + 8) == md.MOEDISP_ERR_MISALIGNED
+    assert p(ws=ws + 8) == md.MOEDISP_ERR_MISALIGNED
+    assert p(recv=inp) == md.MOEDISP_ERR_ALIASED              # receive buffer over the send rows
+    assert p(ready=ex) == md.MOEDISP_ERR_ALIASED              # ready words inside expand_x
+    assert p(d=md.Dims(4, 0, 2, 8), so=None) == md.MOEDISP_OK  # no positions, no plan

@@ -923,6 +923,159 @@ def test_dispatch_of_exchanged_tokens_without_receive_buffer(md, q, smooth):
     assert np.array_equal(etn.cpu().numpy(), retn) and np.array_equal(erc.cpu().numpy(), rerc)
 
 
+def _pipelined_case(md, seed, W, max_split, H, K, ne, corrupt=None):
+    """Oracle and device inputs of one exchange -> dispatch problem: the oracle's exchange
+    into a receive buffer (fill 0x7777), its layout over the received positions and its
+    dispatch; on the device the plan, the receive mask (a2a_token_rows) and the layout.
+    corrupt: (i, j) of a segment whose source offset is pushed past its sender's rows."""
+    a, cap_in, T, x, w = _a2a_case(seed, W, max_split, H, K, ne)
+    src, outs, dsto, _ = oracle.a2a_exchange_plan(a.in_splits)
+    if corrupt is not None:
+        i, j = corrupt
+        src = src.copy()
+        src[i, j] = cap_in
+    recv = np.full((W, T, H), 0x7777, np.uint16)
+    fl = oracle.a2a_v(x, recv, src, outs, dsto)
+    ok = np.zeros((W, T), np.uint8)                   # positions the exchange fills
+    for i in range(W):
+        for j in range(W):
+            n = outs[i, j]
+            if n > 0 and (corrupt is None or (i, j) != tuple(corrupt)):
+                ok[i, dsto[i, j]:dsto[i, j] + n] = 1
+    active = ok.reshape(-1)
+    ref = oracle.moe_dispatch_layout(W, T, K, W * ne, w.expert_ids, active)
+    plan = [dev(z.astype(np.int64)) for z in (src, outs, dsto)]
+    st = new_status()
+    L = md.LayoutBuffers.allocate(W, T, K, W * ne)
+    md.moe_dispatch_layout(dev(w.expert_ids.reshape(-1)), dev(active), L, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    return dict(a=a, cap_in=cap_in, T=T, x=x, w=w, recv=recv, fl=fl, ref=ref, plan=plan, L=L,
+                W=W, H=H, K=K, ne=ne)
+
+
+def _run_pipelined(md, c, q, epoch, ready, ws, roles=None, recv_dev=None, out=None, limit_us=2_000_000):
+    W, T, H, L = c["W"], c["T"], c["H"], c["L"]
+    if recv_dev is None:
+        recv_dev = torch.full((W * T, H), 0x7777, dtype=torch.int16, device="cuda")
+    if out is None:
+        full, scales, gr = alloc_expand(L, H, q)
+        etn = torch.full((W, c["ne"]), -1, dtype=torch.int64, device="cuda")
+        erc = torch.full((W, c["ne"], W), -1, dtype=torch.int32, device="cuda")
+        out = (full, scales, gr, etn, erc)
+    full, scales, gr, etn, erc = out
+    st = new_status()
+    md.a2a_dispatch_pipelined(bf16_dev(c["x"].reshape(-1, H)), c["cap_in"], c["plan"][0], c["plan"][1],
+                              c["plan"][2], recv_dev, H, L, q, full[gr:gr + L.rows_cap],
+                              scales[gr:gr + L.rows_cap] if q else None, ready, epoch, ws, st,
+                              roles=md.PIPE_BOTH if roles is None else roles, wait_limit_us=limit_us,
+                              expert_token_nums=etn, ep_recv_counts=erc)
+    torch.cuda.synchronize()
+    return recv_dev, out, int(st.item())
+
+
+def _check_pipelined(md, c, q, recv_dev, out):
+    full, scales, gr, etn, erc = out
+    W, T, H, ref = c["W"], c["T"], c["H"], c["ref"]
+    assert np.array_equal(recv_dev.cpu().numpy().view(np.uint16), c["recv"].reshape(W * T, H))
+    rex, rsc, fl = oracle.moe_dispatch(c["recv"].reshape(W * T, H), ref["dst_row"], c["K"],
+                                       ref["rows_cap"], q)
+    assert fl == 0
+    R = ref["R"]
+    got = full.cpu().numpy()
+    if q == 0:
+        got = got.view(np.uint16)
+    assert np.array_equal(got[gr:gr + R], rex[:R])
+    canary = 0x5A if q else np.uint16(-12345 & 0xFFFF)
+    assert (got[:gr] == canary).all() and (got[gr + R:] == canary).all()
+    if q:
+        assert np.array_equal(scales.cpu().numpy()[gr:gr + R].view(np.uint32), rsc[:R].view(np.uint32))
+    retn, rerc, _ = oracle.moe_recv_counts(W, W * c["ne"], ref["cnt"], 1)
+    assert np.array_equal(etn.cpu().numpy(), retn) and np.array_equal(erc.cpu().numpy(), rerc)
+
+
+def _pipe_state(md, W):
+    ready = torch.zeros((W, W), dtype=torch.int32, device="cuda")
+    ws = torch.empty(md.a2a_dispatch_pipelined_workspace_size(W), dtype=torch.uint8, device="cuda")
+    return ready, ws
+
+
+@pytest.mark.parametrize("q", [0, 2, 3])
+@pytest.mark.parametrize("W,max_split,H,K,ne", [(8, 120, 256, 4, 4), (4, 300, 2048, 8, 2),
+                                                (16, 40, 7168, 2, 1), (3, 50, 16, 3, 5)])
+def test_pipelined_exchange_and_dispatch(md, q, W, max_split, H, K, ne):
+    """a2a_dispatch_pipelined equals the oracle's exchange into a receive buffer followed by
+    its dispatch: the receive buffer (untouched positions included), every dispatched row,
+    scale and receive count bit-exact -- and again on a second call with the next epoch
+    over the same ready words and workspace."""
+    c = _pipelined_case(md, 90 + W, W, max_split, H, K, ne)
+    assert c["fl"] == 0
+    ready, ws = _pipe_state(md, W)
+    for epoch in (1, 2):
+        recv_dev, out, st = _run_pipelined(md, c, q, epoch, ready, ws)
+        assert st == 0
+        _check_pipelined(md, c, q, recv_dev, out)
+    published = ready.cpu().numpy().reshape(-1)
+    nonempty = (c["a"].in_splits.T.reshape(-1) > 0)
+    assert (published[nonempty] == 2).all() and (published[~nonempty] == 0).all()
+
+
+@pytest.mark.slow
+def test_pipelined_exchange_and_dispatch_benchmark_shape(md):
+    """The benchmark's exchange -> dispatch shape: W = 8, splits ~ randint[0, 512),
+    H = 4096 bf16, E = 64, K = 8."""
+    c = _pipelined_case(md, 3, 8, 512, 4096, 8, 8)
+    ready, ws = _pipe_state(md, 8)
+    recv_dev, out, st = _run_pipelined(md, c, 0, 1, ready, ws)
+    assert st == 0
+    _check_pipelined(md, c, 0, recv_dev, out)
+
+
+@pytest.mark.parametrize("q", [0, 3])
+def test_pipelined_produce_then_consume(md, q):
+    """The two roles as separate calls of one epoch: the exchange alone publishes the ready
+    words, the dispatch alone then finds them published -- the same result as both in one."""
+    c = _pipelined_case(md, 95, 8, 100, 512, 4, 2)
+    ready, ws = _pipe_state(md, 8)
+    recv_dev, out, st = _run_pipelined(md, c, q, 5, ready, ws, roles=md.PIPE_PRODUCE)
+    assert st == 0
+    assert out[0].cpu().numpy()[out[2]:].max() == out[0].cpu().numpy()[out[2]:].min()   # no dispatch yet
+    recv_dev, out, st = _run_pipelined(md, c, q, 5, ready, ws, roles=md.PIPE_CONSUME,
+                                       recv_dev=recv_dev, out=out)
+    assert st == 0
+    _check_pipelined(md, c, q, recv_dev, out)
+
+
+def test_pipelined_consumer_whose_producer_never_publishes_times_out(md):
+    """The dispatch alone, for an epoch nobody published: every wait gives up after the
+    20 ms limit (the first one to run out stops the others), the call reports TIMEOUT, the
+    GPU context stays usable and the next full call of the pipeline is exact."""
+    import time
+    c = _pipelined_case(md, 96, 8, 100, 256, 4, 2)
+    ready, ws = _pipe_state(md, 8)
+    t0 = time.monotonic()
+    _, _, st = _run_pipelined(md, c, 2, 9, ready, ws, roles=md.PIPE_CONSUME, limit_us=20000)
+    assert st == md.STATUS_TIMEOUT
+    assert time.monotonic() - t0 < 10.0
+    recv_dev, out, st = _run_pipelined(md, c, 2, 10, ready, ws)
+    assert st == 0
+    _check_pipelined(md, c, 2, recv_dev, out)
+
+
+def test_pipelined_bad_segment_is_skipped_and_flagged(md):
+    """A segment whose source range leaves its sender's rows is neither exchanged nor
+    dispatched (BAD_SPLIT, as a2a_v); every other segment is exact and nothing waits."""
+    W = 8
+    a = wl.a2a_workload(seed=97, W=W, max_split=60, row_elems=256)
+    i, j = [(i, j) for i in range(W) for j in range(W) if a.in_splits[j, i] > 0][3]
+    c = _pipelined_case(md, 97, W, 60, 256, 4, 2, corrupt=(i, j))
+    assert c["fl"] & oracle.ORC_BAD_SPLIT
+    ready, ws = _pipe_state(md, W)
+    recv_dev, out, st = _run_pipelined(md, c, 0, 1, ready, ws)
+    assert st == md.STATUS_BAD_SPLIT
+    _check_pipelined(md, c, 0, recv_dev, out)
+
+
 def test_dispatch_gather_bad_rows_are_flagged(md):
     w = wl.moe_workload("tiny", seed=72, W=2, T=20, K=2, E=4, H=64)
     L, _ = run_layout(md, w)
