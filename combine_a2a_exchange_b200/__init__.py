@@ -93,6 +93,10 @@ _pipe_ws = _sig("moedisp_a2a_dispatch_pipelined_workspace_size", [_I, ctypes.POI
 _pipe = _sig("moedisp_a2a_dispatch_pipelined",
              [_P, _I64, _P, _P, _P, _P, _I, Dims, ctypes.POINTER(Layout), _I, _P, _P, _P, _I, _P,
               _P, ctypes.c_uint32, _I, ctypes.c_uint32, _P, ctypes.c_size_t, _P, _P])
+IPC_HANDLE_BYTES = 64
+_ipc_export = _sig("moedisp_ipc_export", [_P, _P, ctypes.POINTER(ctypes.c_int64)])
+_ipc_import = _sig("moedisp_ipc_import", [_P, ctypes.c_int64, ctypes.POINTER(ctypes.c_void_p)])
+_ipc_close = _sig("moedisp_ipc_close", [_P])
 _ep_barrier = _sig("moedisp_ep_barrier", [_P, _I, _I, ctypes.c_uint32, ctypes.c_uint32, _P, _P])
 _shared = _sig("moedisp_shared_expert_routing",
                [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P])
@@ -351,6 +355,27 @@ def a2a_dispatch_pipelined(inp, in_rank_stride_rows, src_offsets, out_splits, ds
                _ptr(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
                _ptr(status), _stream(stream))
     return _check(rc, "a2a_dispatch_pipelined", raise_on_error)
+
+
+def ipc_export(t) -> tuple[bytes, int]:
+    """(IPC handle bytes, byte offset) of a device tensor's memory, for another process."""
+    buf = ctypes.create_string_buffer(IPC_HANDLE_BYTES)
+    off = ctypes.c_int64(0)
+    _check(_ipc_export(_ptr(t), buf, ctypes.byref(off)), "ipc_export", True)
+    return bytes(buf.raw), int(off.value)
+
+
+def ipc_import(handle: bytes, offset: int) -> int:
+    """Address, in this process, of a buffer another process exported (a plain peer
+    mapping, no multicast); release it with ipc_close."""
+    assert len(handle) == IPC_HANDLE_BYTES
+    p = ctypes.c_void_p(0)
+    _check(_ipc_import(ctypes.c_char_p(handle), int(offset), ctypes.byref(p)), "ipc_import", True)
+    return int(p.value)
+
+
+def ipc_close(ptr: int) -> None:
+    _check(_ipc_close(ctypes.c_void_p(int(ptr))), "ipc_close", True)
 
 
 def ep_barrier(peer_signals, W, rank, epoch, timeout_us, status, stream=None,

@@ -402,6 +402,29 @@ int moedisp_moe_combine_peers(const void *const *peer_expert_out, int64_t peer_r
                               const moedisp_layout *layout, const float *expert_scales, void *y,
                               int32_t *status, moedisp_stream_t stream);
 
+/* ipc_export / ipc_import / ipc_close
+ *
+ * Peer mappings for moe_dispatch_peers / moe_combine_peers / ep_barrier when the ranks are
+ * processes (one per GPU, or several on one GPU): plain CUDA IPC mappings, so no memory is
+ * bound to an NVLink multicast object (the PyTorch symm_mem change maps its buffers with
+ * NVSHMEM instead). Host-side calls on the current device; no kernel, no allocation.
+ *   ipc_export: for a device buffer of this process (any pointer into a cudaMalloc
+ *     allocation, e.g. a caching allocator's segment), writes the allocation's IPC handle
+ *     (MOEDISP_IPC_HANDLE_BYTES bytes, host memory) and the buffer's byte offset in it.
+ *     Send both to the other ranks (they are plain bytes). Pointers that are not device
+ *     memory of this process: MOEDISP_ERR_INVALID; a CUDA refusal: MOEDISP_ERR_CUDA
+ *     (memory from a virtual-memory allocator cannot be exported this way).
+ *   ipc_import: in another process, maps the allocation (once per process, shared by
+ *     every buffer imported from it) and returns the buffer's address in this process.
+ *     A handle of this same process cannot be opened (MOEDISP_ERR_CUDA): use the buffer
+ *     itself. Importing one buffer twice: MOEDISP_ERR_INVALID.
+ *   ipc_close: releases a pointer ipc_import returned (the mapping goes with its last
+ *     buffer); the peer's buffers must not be used after it. */
+#define MOEDISP_IPC_HANDLE_BYTES 64
+int moedisp_ipc_export(const void *dev_ptr, void *handle, int64_t *offset);
+int moedisp_ipc_import(const void *handle, int64_t offset, void **dev_ptr);
+int moedisp_ipc_close(void *dev_ptr);
+
 /* ep_barrier
  *
  * Orders the W ranks of moe_dispatch_peers / moe_combine_peers on the GPUs themselves,

@@ -343,3 +343,21 @@ def test_pipelined_rejections(md):
     assert p(recv=inp) == md.MOEDISP_ERR_ALIASED              # receive buffer over the send rows
     assert p(ready=ex) == md.MOEDISP_ERR_ALIASED              # ready words inside expand_x
     assert p(d=md.Dims(4, 0, 2, 8), so=None) == md.MOEDISP_OK  # no positions, no plan
+
+
+def test_ipc_rejections(md):
+    h = ctypes.create_string_buffer(64)
+    off = ctypes.c_int64(0)
+    p = ctypes.c_void_p(0)
+    lib = ctypes.CDLL(md.LIBRARY_PATH)
+    lib.moedisp_ipc_export.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(ctypes.c_int64)]
+    lib.moedisp_ipc_import.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(ctypes.c_void_p)]
+    lib.moedisp_ipc_close.argtypes = [ctypes.c_void_p]
+    assert lib.moedisp_ipc_export(None, h, ctypes.byref(off)) == md.MOEDISP_ERR_NULLPTR
+    assert lib.moedisp_ipc_export(FAKE, None, ctypes.byref(off)) == md.MOEDISP_ERR_NULLPTR
+    assert lib.moedisp_ipc_export(FAKE, h, None) == md.MOEDISP_ERR_NULLPTR
+    assert lib.moedisp_ipc_import(None, 0, ctypes.byref(p)) == md.MOEDISP_ERR_NULLPTR
+    assert lib.moedisp_ipc_import(h, 0, None) == md.MOEDISP_ERR_NULLPTR
+    assert lib.moedisp_ipc_import(h, -1, ctypes.byref(p)) == md.MOEDISP_ERR_INVALID
+    assert lib.moedisp_ipc_close(None) == md.MOEDISP_ERR_NULLPTR
+    assert lib.moedisp_ipc_close(FAKE) == md.MOEDISP_ERR_INVALID       # never imported

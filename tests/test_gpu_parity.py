@@ -1403,6 +1403,21 @@ def test_ep_dispatcher_one_rank_end_to_end(md, q):
     assert res["ok"] and res["epoch"] == 6, res
 
 
+@pytest.mark.parametrize("q", [0, 2])
+def test_ep_two_processes_share_one_gpu_through_ipc_mappings(md, q):
+    """Two EP ranks as two processes on this GPU: buffers mapped across the processes with
+    the library's IPC calls, host barriers only (no kernel waits for the other process);
+    each rank's dispatched rows and combined tokens against the oracle, two steps."""
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "tests", "ep_two_ranks_one_gpu.py"), str(q)],
+                       capture_output=True, text=True, timeout=400)
+    assert r.returncode == 0, (r.stdout[-3000:], r.stderr[-4000:])
+    lines = [json.loads(l) for l in r.stdout.strip().splitlines() if l.startswith("{")]
+    assert len(lines) == 2 and all(l["ok"] for l in lines), lines
+
+
 # ------------------------------------------------------------- randomised sweep
 
 def _random_case(i):
