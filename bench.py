@@ -952,6 +952,9 @@ def main():
     ap.add_argument("--a2a-W", type=int, default=64, help="ranks of the a2a64 workload")
     ap.add_argument("--a2a-max-split", type=int, default=512, help="split bound of a2a64")
     ap.add_argument("--no-ops", action="store_true", help="skip the per-op sweep of other workloads")
+    ap.add_argument("--ep", action="store_true",
+                    help="expert parallelism across the N GPUs (the real exchange over NVLink) "
+                         "instead of one independent replica per GPU")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--op", choices=["step", "layout", "dispatch", "combine", "dispatch_smooth",
@@ -973,6 +976,8 @@ def main():
         return run_reference(args, wl)
     if args.workload == "a2a64":
         return run_a2a(args, wl, world, rank, local_rank)
+    if args.ep:
+        return run_ep(args, wl, world, rank, local_rank)
 
     import torch
     import torch.distributed as dist
@@ -1139,6 +1144,95 @@ def run_a2a(args, wl, world, rank, local_rank):
                                    f"zeros, rows of {E_} bf16", "moved_rows": a.moved_rows()},
             "hbm_GBps": round(b / (ms * 1e-3) / 1e9, 1), "peak": hbm, "peak_source": peak_src,
             "gpu_launches": 2 * args.steps}), flush=True)
+    return 0
+
+
+def run_ep(args, wl, world, rank, local_rank):
+    """Expert parallelism across the GPUs: the workload's W virtual ranks are spread over
+    the N processes (W/N each, so GPU r holds tokens [r*G/N, (r+1)*G/N) and experts
+    [r*E/N, (r+1)*E/N)), and one step is EPDispatcher's real exchange -- routing
+    all-gather (NCCL), global layout, peer-table dispatch into the owners' buffers, bounded
+    device barriers, peer-table combine -- with the experts' outputs fixed (N(0,1) rows).
+    Strong scaling: the total work is the configuration's at every N. Inputs are larger
+    than L2 on every GPU, so no flush between steps; device time per step is the max over
+    ranks. NVLink bytes are the rows this rank sends to other GPUs in the dispatch plus the
+    rows it reads from other GPUs in the combine."""
+    from datetime import timedelta
+
+    import torch
+    import torch.distributed as dist
+    import combine_a2a_exchange_b200 as md
+    from combine_a2a_exchange_b200.ep import EPDispatcher
+
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    os.environ.setdefault("MASTER_PORT", "29517")
+    os.environ.setdefault("RANK", str(rank))
+    os.environ.setdefault("WORLD_SIZE", str(world))
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+    w = wl.moe_workload(args.workload, seed=0)
+    if w.W % world or w.E % world:
+        raise SystemExit(f"--ep needs N dividing W={w.W} and E={w.E}")
+    Tr = w.G // world
+    sl = slice(rank * Tr, (rank + 1) * Tr)
+    ep = EPDispatcher(md, dist.group.WORLD, Tr, w.K, w.E, w.H, quant_mode=w.quant_mode,
+                      device=device)
+    x = torch.from_numpy(np.ascontiguousarray(w.x_bits[sl]).view(np.int16)).to(device).view(torch.bfloat16)
+    ids = torch.from_numpy(np.ascontiguousarray(w.expert_ids[sl])).to(device)
+    act = None if w.active is None else torch.from_numpy(np.ascontiguousarray(w.active[sl])).to(device)
+    wts = torch.from_numpy(np.ascontiguousarray(w.weights[sl])).to(device)
+    y = torch.empty((Tr, w.H), dtype=torch.bfloat16, device=device)
+    g = torch.Generator(device=device).manual_seed(7 + rank)
+    ep.expert_out.copy_(torch.randn(ep.expert_out.shape, generator=g, device=device).to(torch.bfloat16))
+
+    def step():
+        ep.dispatch(x, ids, act)
+        ep.combine(wts, y, check=False)
+
+    for _ in range(args.warmup):
+        step()
+    ep.check()
+    dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    ep.check()
+    dist.barrier()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(torch, e0.elapsed_time(e1) / args.steps, device)
+    # bytes this rank moves over NVLink per step
+    ne = w.E // world
+    mine = w.expert_ids[sl]
+    live = np.ones(mine.shape, bool) if w.active is None else (
+        np.broadcast_to(w.active[sl][:, None], mine.shape).astype(bool) if w.active.ndim == 1
+        else w.active[sl].astype(bool))
+    remote = int(((mine // ne != rank) & live).sum())
+    out_row = w.H * (2 if w.quant_mode == 0 else 1) + (4 if w.quant_mode else 0)
+    nvl = remote * (out_row + 2 * w.H)
+    nvl_t = torch.tensor([float(nvl)], dtype=torch.float64, device=device)
+    dist.all_reduce(nvl_t, op=dist.ReduceOp.MAX)
+    ep.close()
+    dist.barrier()
+    dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    print(json.dumps({
+        "metric": METRIC, "value": round(w.G / (ms / 1e3), 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": dtype_of(w),
+        "data": "synthetic (seeded generator; no dataset)",
+        "config": dict(config_of(w), parallelism=f"ep{world} (expert parallel over GPUs)",
+                       l2="inputs larger than L2 on every GPU; no flush"),
+        "mode": "ep: routing all-gather, global layout, peer-table dispatch and combine over "
+                "IPC-mapped buffers, bounded device barriers",
+        "nvlink_bytes_per_rank_step_max": int(nvl_t.item()),
+        "nvlink_GBps_per_rank": round(nvl_t.item() / (ms * 1e-3) / 1e9, 1),
+        "gpu_launches": None}), flush=True)
     return 0
 
 

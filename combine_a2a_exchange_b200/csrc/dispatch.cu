@@ -327,11 +327,9 @@ __global__ void __launch_bounds__(kQuantThreads, CPT > 4 ? 2 : 4) dispatch_smoot
 // thread, all issued together): no shared-memory staging, so that nothing but registers
 // limits the warps per SM (a bulk-copy-staged version was measured 5 % slower on cfg3 and
 // cfg4: its stages capped an SM at ~24 warps). Groups take tokens g = group, group +
-// groups, ...; per token: the K destination rows (lanes 0..K-1, shuffled), max |x|
-// (shuffles + a named barrier across the group), the codes, and then -- before the codes
-// are written to the K rows (8 bytes per chunk, coalesced) with the scale -- the loads of
-// the group's next routed token are issued into the registers the row just left, so that
-// its latency hides behind this token's stores.
+// groups, ...; per token: the K destination rows (lanes 0..K-1, shuffled), skip if none
+// is routed, max |x| (shuffles + a named barrier across the group), then the codes are
+// written to the K rows (8 bytes per chunk, coalesced) with the scale.
 template <int Q, int WPT, int CPT, bool PEERS>
 __global__ void __launch_bounds__(kQuantThreads, CPT > 4 ? 2 : 4) dispatch_quant_kernel(DispatchArgs a) {
     constexpr int NG = kQuantThreads / 32 / WPT;
@@ -346,40 +344,26 @@ __global__ void __launch_bounds__(kQuantThreads, CPT > 4 ? 2 : 4) dispatch_quant
     const int K = a.K, nvec = a.H >> 3;
     const int64_t groups = (int64_t)gridDim.x * NG;
     int parity = 0;
-    // The group's next token from g on that has a routed slot whose row of x exists (its
-    // destination rows in d, this lane's slot), or a.G; skipped tokens are flagged.
-    auto next_token = [&](int64_t g, int32_t& d, int64_t& src) -> int64_t {
-        for (; g < a.G; g += groups) {
-            d = lane < K ? __ldg(a.dst_row + g * K + lane) : -1;
-            if (d >= a.rows_cap) {
-                raise_status(a.status, MOEDISP_STATUS_CAPACITY);
-                d = -1;
-            }
-            if (d < 0) d = -1;
-            if (!__ballot_sync(0xffffffffu, d >= 0)) continue;      // same in every warp
-            src = token_source(a, g);
-            if (src < 0 || src >= a.x_rows) {
-                if (gt == 0) raise_status(a.status, MOEDISP_STATUS_BAD_SPLIT);
-                continue;
-            }
-            return g;
+    for (int64_t g = (int64_t)blockIdx.x * NG + grp; g < a.G; g += groups) {
+        int32_t d = lane < K ? __ldg(a.dst_row + g * K + lane) : -1;
+        if (d >= a.rows_cap) {
+            raise_status(a.status, MOEDISP_STATUS_CAPACITY);
+            d = -1;
         }
-        return a.G;
-    };
-    uint4 v[CPT];
-    auto load_row = [&](int64_t src) {
+        if (d < 0) d = -1;
+        if (!__ballot_sync(0xffffffffu, d >= 0)) continue;          // same in every warp
+        const int64_t src = token_source(a, g);
+        if (src < 0 || src >= a.x_rows) {
+            if (gt == 0) raise_status(a.status, MOEDISP_STATUS_BAD_SPLIT);
+            continue;
+        }
         const uint4* xr = reinterpret_cast<const uint4*>(a.x) + src * nvec;
+        uint4 v[CPT];
 #pragma unroll
         for (int j = 0; j < CPT; ++j) {
             const int c = gt + j * GT;
             v[j] = c < nvec ? __ldcs(xr + c) : make_uint4(0u, 0u, 0u, 0u);
         }
-    };
-    int32_t d = -1;
-    int64_t src = 0;
-    int64_t g = next_token((int64_t)blockIdx.x * NG + grp, d, src);
-    if (g < a.G) load_row(src);
-    while (g < a.G) {
         float m = 0.0f;
 #pragma unroll
         for (int j = 0; j < CPT; ++j) m = fmaxf(m, absmax8(v[j]));
@@ -406,11 +390,6 @@ __global__ void __launch_bounds__(kQuantThreads, CPT > 4 ? 2 : 4) dispatch_quant
             myrow = peer_row(a, g, lane, d, &local);
             if (myrow != nullptr) mysc = a.peer_scales[__ldg(a.ids + g * K + lane) / a.ne] + local;
         }
-        // the next token's row is on its way while this token's codes are stored
-        int32_t d2 = -1;
-        int64_t src2 = 0;
-        const int64_t g2 = next_token(g + groups, d2, src2);
-        if (g2 < a.G) load_row(src2);
         for (int k = 0; k < K; ++k) {
             const int32_t dk = __shfl_sync(0xffffffffu, d, k);
             uint2* dst;
@@ -433,9 +412,6 @@ __global__ void __launch_bounds__(kQuantThreads, CPT > 4 ? 2 : 4) dispatch_quant
                 a.scales[dk] = scale;
             }
         }
-        g = g2;
-        d = d2;
-        src = src2;
     }
 }
 

@@ -206,6 +206,11 @@ LAYOUT_CASES = [
     # one cluster, two tiles per rank and the largest tile
     ("tiny", dict(W=8, T=2048, K=8, E=256, routing="zipf")),
     ("tiny", dict(W=1, T=2048, K=8, E=1024)),
+    # one cluster of 1024-thread blocks (tiles of up to 16384 slots): E = 1024 near the
+    # shared-memory limit, a per-token mask with ragged tiles, a per-slot mask
+    ("tiny", dict(W=4, T=4096, K=4, E=1024)),
+    ("tiny", dict(W=16, T=1000, K=8, E=128, active_p=0.6)),
+    ("tiny", dict(W=8, T=3001, K=5, E=64, slot_active_p=0.7)),
     # per-slot (2-D) active masks: cluster path, tiled path, K = 1
     ("tiny", dict(W=3, T=500, K=4, E=12, slot_active_p=0.5)),
     ("tiny", dict(W=2, T=30000, K=8, E=16, slot_active_p=0.6)),
