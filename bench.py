@@ -65,14 +65,15 @@ def source_sha(path):
     return hashlib.sha256(open(os.path.join(ROOT, path), "rb").read()).hexdigest()[:16]
 
 
-def ncu_traffic(kernel_key):
-    """dram read+write bytes per launch from a committed ncu capture, when the kernel's
-    source has not changed since (else None)."""
+def ncu_traffic(kernel_key, workload):
+    """dram read+write bytes per launch of `kernel_key` on `workload` from a committed ncu
+    capture (scaled to the full launch when the capture ran a smaller case), when the
+    kernel's source has not changed since (else None)."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
     try:
-        d = json.load(open(p)).get(kernel_key)
+        d = json.load(open(p)).get(f"{kernel_key} @ {workload}")
         if not d or d.get("source_sha") != source_sha(d["source"]):
             return None
         return float(d["bytes_per_launch"])
@@ -720,21 +721,46 @@ def op_sweep(md, torch, device, hbm, reps=10, main_workload="cfg3"):
         front()
         md.moe_dispatch_gather(xin, W_ * cap_in, tr, H_, L, 0, ex, None, status)
 
+    ready = torch.zeros((W_, W_), dtype=torch.int32, device=device)
+    pws = torch.empty(md.a2a_dispatch_pipelined_workspace_size(W_), dtype=torch.uint8, device=device)
+    epoch = [0]
+
+    def pipelined():
+        front()
+        epoch[0] += 1           # a new epoch per exchange (the graph replays this value)
+        md.a2a_dispatch_pipelined(xin, cap_in, plan[0], plan[1], plan[2], recv, H_, L, 0, ex, None,
+                                  ready, epoch[0], pws, status)
+
     res = {}
     for nm, fn in (("sequential", sequential), ("no_receive_buffer", fused)):
         g = capture(torch, fn)
         res[nm] = statistics.mean(time_graph(torch, g, reps, 3, flush))
         del g
+    # the pipelined call publishes its epoch into the ready words, so each timed call needs
+    # a new epoch: eager launches (the host enqueues them behind the flush)
+    Ev = torch.cuda.Event
+    pairs = []
+    for r in range(reps + 3):
+        flush.zero_()
+        e0, e1 = Ev(enable_timing=True), Ev(enable_timing=True)
+        e0.record()
+        pipelined()
+        e1.record()
+        if r >= 3:
+            pairs.append((e0, e1))
     torch.cuda.synchronize()
+    res["pipelined_ready_words"] = statistics.mean(x.elapsed_time(y) for x, y in pairs)
     assert int(status.item()) == 0, md.status_string(int(status.item()))
     n_recv = int(a.in_splits.sum())
     R = int(L.expert_base[-1].item())
     b_fused = n_recv * H_ * 2 + R * H_ * 2
+    b_recv = b_fused + n_recv * H_ * 2          # the receive buffer is an output too
     for nm, ms in res.items():
+        bm = b_recv if nm != "no_receive_buffer" else b_fused
         out.append({"workload": "a2a8->dispatch", "op": nm, "us": round(ms * 1e3, 2),
                     "tokens/s": round(n_recv / (ms / 1e3), 1),
-                    "bytes_min": b_fused, "frac_of_min": round(b_fused / ms / 1e6 / hbm, 4)})
-    del xin, recv, ex, L
+                    "bytes_min": bm, "frac_of_min": round(bm / ms / 1e6 / hbm, 4)})
+    del xin, recv, ex, L, ready, pws
     torch.cuda.empty_cache()
     # expert parallelism through per-rank buffers: cfg2's 8 ranks each dispatch their own
     # tokens into the 8 ranks' separate buffers through a pointer table, then each combines
@@ -820,9 +846,11 @@ def op_sweep(md, torch, device, hbm, reps=10, main_workload="cfg3"):
 # ---------------------------------------------------------------------- main
 
 def run_gather_op(args, wl, md, torch, device, flush):
-    """moe_dispatch_gather of W = 8 ranks' exchanged tokens read in place (splits ~
-    randint[0, 512), H = 4096 bf16, E = 64, K = 8), after the plan, the receive map and the
-    layout ran once."""
+    """The dispatch of W = 8 ranks' exchanged tokens (splits ~ randint[0, 512), H = 4096
+    bf16, E = 64, K = 8) after the plan, the receive map and the layout ran once:
+    moe_dispatch_gather reading the tokens in place, or (--op dispatch_pipelined) the
+    exchange into a receive buffer and the dispatch pipelined through ready words, a new
+    epoch per call."""
     a = wl.a2a_workload(seed=3, W=8, max_split=512, zero_frac=0.1, row_elems=4096)
     W_, H_, K_, E_ = a.W, 4096, 8, 64
     cap_in, T_ = a.cap_in, a.cap_out
@@ -839,15 +867,29 @@ def run_gather_op(args, wl, md, torch, device, flush):
     md.a2a_token_rows(plan[0], plan[1], plan[2], W_, T_, cap_in, tr, status, active=act)
     md.moe_dispatch_layout(torch.from_numpy(w.expert_ids.reshape(-1)).to(device), act, L, status)
     Ev = torch.cuda.Event
+    if args.op == "dispatch_pipelined":
+        recv = torch.empty((W_ * T_, H_), dtype=torch.bfloat16, device=device)
+        ready = torch.zeros((W_, W_), dtype=torch.int32, device=device)
+        pws = torch.empty(md.a2a_dispatch_pipelined_workspace_size(W_), dtype=torch.uint8,
+                          device=device)
+        epoch = [0]
+
+        def op():
+            epoch[0] += 1
+            md.a2a_dispatch_pipelined(xin, cap_in, plan[0], plan[1], plan[2], recv, H_, L, 0, ex,
+                                      None, ready, epoch[0], pws, status)
+    else:
+        def op():
+            md.moe_dispatch_gather(xin, W_ * cap_in, tr, H_, L, 0, ex, None, status)
     for _ in range(args.warmup):
         flush.zero_()
-        md.moe_dispatch_gather(xin, W_ * cap_in, tr, H_, L, 0, ex, None, status)
+        op()
     pairs = []
     for _ in range(args.steps):
         flush.zero_()
         e0, e1 = Ev(enable_timing=True), Ev(enable_timing=True)
         e0.record()
-        md.moe_dispatch_gather(xin, W_ * cap_in, tr, H_, L, 0, ex, None, status)
+        op()
         e1.record()
         pairs.append((e0, e1))
     torch.cuda.synchronize()
@@ -865,7 +907,7 @@ def run_single_op(args, wl, md, torch):
     Prints one JSON line. Launch order: the step's kernels once, then the op's."""
     device = torch.device("cuda", torch.cuda.current_device())
     flush = L2Flush(torch, device)
-    if args.op == "dispatch_gather":
+    if args.op in ("dispatch_gather", "dispatch_pipelined"):
         return run_gather_op(args, wl, md, torch, device, flush)
     w = wl.moe_workload(args.workload, seed=0, **({"T": args.T} if args.T else {}))
     st = MoEStep(md, torch, w, device)
@@ -958,7 +1000,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--op", choices=["step", "layout", "dispatch", "combine", "dispatch_smooth",
-                                     "combine_rmsnorm", "dispatch_gather", "peers"], default="step",
+                                     "combine_rmsnorm", "dispatch_gather", "dispatch_pipelined",
+                                     "peers"], default="step",
                     help="time one op alone on --workload (one GPU, eager launches behind an L2 "
                          "flush), e.g. to profile it")
     args = ap.parse_args()
@@ -1038,7 +1081,7 @@ def main():
     dom_bytes = algorithmic_bytes(dom, w, R)
     achieved = dom_bytes / (per_op[dom] * 1e-3) / 1e9
     kernel_key = {"dispatch": dispatch_kernel_name(w), "combine": f"combine_kernel<{w.K}>"}[dom]
-    traffic = ncu_traffic(kernel_key)
+    traffic = ncu_traffic(kernel_key, w.name)
 
     e2e = None
     if not args.no_e2e:

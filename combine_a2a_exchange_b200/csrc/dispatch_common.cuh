@@ -93,25 +93,70 @@ __device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint3
     return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
 
-// Eight fp32 values (a smoothed row chunk) to eight codes.
+// Eight fp32 values (a smoothed row chunk) to eight codes. The floating-point steps of the
+// fast test run on pairs with the packed fp32x2 instructions (each lane an IEEE
+// round-to-nearest operation, the same result as the scalar one): for int8 the shortcut
+// r = x * inv, rr = r + 1.5*2^23, t = r - (rr - 1.5*2^23); for e4m3 the product r. The
+// decisions, the slow path and the encoding are q_int8_w's and q_e4m3's, element by
+// element.
 template <int Q>
 __device__ __forceinline__ uint2 quant8f(const float (&v)[8], float scale, float inv, bool zero) {
     if (zero) return make_uint2(0u, 0u);
+    constexpr float kMagic = 12582912.0f;                    // 1.5 * 2^23
+    const float2 inv2 = make_float2(inv, inv);
     uint32_t b[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) b[j] = q_code<Q>(v[j], scale, inv);
+    for (int p = 0; p < 4; ++p) {
+        const float x0 = v[2 * p], x1 = v[2 * p + 1];
+        const float2 r = __fmul2_rn(make_float2(x0, x1), inv2);
+        if (Q == MOEDISP_QUANT_INT8) {
+            const float2 rr = __fadd2_rn(r, make_float2(kMagic, kMagic));
+            const float2 back = __fadd2_rn(rr, make_float2(-kMagic, -kMagic));
+            const float2 t = __fadd2_rn(r, make_float2(-back.x, -back.y));
+            const float xs[2] = {x0, x1};
+            const float rs[2] = {r.x, r.y};
+            const float rrs[2] = {rr.x, rr.y};
+            const float ts[2] = {t.x, t.y};
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                if (0.5f - fabsf(ts[h]) >= 0.00006103515625f && fabsf(rs[h]) < 127.5f) {
+                    b[2 * p + h] = __float_as_uint(rrs[h]);
+                } else {
+                    const float q = fminf(fmaxf(__fdiv_rn(xs[h], scale), -127.0f), 127.0f);
+                    b[2 * p + h] = __float_as_uint(__fadd_rn(q, kMagic));
+                }
+            }
+        } else {
+            const float xs[2] = {x0, x1};
+            const float rs[2] = {r.x, r.y};
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t bb = __float_as_uint(rs[h]);
+                const uint32_t u = bb & 0x7fffffffu;
+                if (u - 0x3c800000u < 0x43e00000u - 0x3c800000u && (u & 0xfffffu) - 0x7fff0u > 32u) {
+                    b[2 * p + h] = ((bb >> 24) & 0x80u) | (((u + 0x80000u) >> 20) - 0x3c0u);
+                } else {
+                    const float q = __fdiv_rn(xs[h], scale);
+                    b[2 * p + h] = (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(q, 0.0f), __NV_SATFINITE,
+                                                                      __NV_E4M3);
+                }
+            }
+        }
+    }
     return make_uint2(pack_low_bytes(b[0], b[1], b[2], b[3]), pack_low_bytes(b[4], b[5], b[6], b[7]));
 }
 
 // x chunk (8 bf16) times a smoothing chunk (8 fp32, shared memory), one correctly rounded
-// product each.
+// product each (four packed fp32x2 multiplies).
 __device__ __forceinline__ void smooth8(const uint4& v, const float4* s, float (&o)[8]) {
     const float4 s0 = s[0];
     const float4 s1 = s[1];
-    o[0] = __fmul_rn(bf16_lo(v.x), s0.x); o[1] = __fmul_rn(bf16_hi(v.x), s0.y);
-    o[2] = __fmul_rn(bf16_lo(v.y), s0.z); o[3] = __fmul_rn(bf16_hi(v.y), s0.w);
-    o[4] = __fmul_rn(bf16_lo(v.z), s1.x); o[5] = __fmul_rn(bf16_hi(v.z), s1.y);
-    o[6] = __fmul_rn(bf16_lo(v.w), s1.z); o[7] = __fmul_rn(bf16_hi(v.w), s1.w);
+    const float2 p0 = __fmul2_rn(make_float2(bf16_lo(v.x), bf16_hi(v.x)), make_float2(s0.x, s0.y));
+    const float2 p1 = __fmul2_rn(make_float2(bf16_lo(v.y), bf16_hi(v.y)), make_float2(s0.z, s0.w));
+    const float2 p2 = __fmul2_rn(make_float2(bf16_lo(v.z), bf16_hi(v.z)), make_float2(s1.x, s1.y));
+    const float2 p3 = __fmul2_rn(make_float2(bf16_lo(v.w), bf16_hi(v.w)), make_float2(s1.z, s1.w));
+    o[0] = p0.x; o[1] = p0.y; o[2] = p1.x; o[3] = p1.y;
+    o[4] = p2.x; o[5] = p2.y; o[6] = p3.x; o[7] = p3.y;
 }
 
 __device__ __forceinline__ uint32_t q_int8_pair(uint32_t w, float scale, float inv) {
