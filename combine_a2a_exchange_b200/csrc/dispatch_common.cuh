@@ -33,7 +33,10 @@ __device__ __forceinline__ float absmax8(const uint4& v) {
 // 2.3e-5 and a margin of 2^-14 from k + 0.5 is safe. Rounding to an integer uses the
 // floating-point adder: for |v| < 2^22, rr = v + 1.5*2^23 rounds v's fraction away to the
 // nearest integer, ties to even, and rr's bit pattern is that of 1.5*2^23 plus the
-// integer. Two exact formulations follow; each kernel uses the one measured faster in it.
+// integer. Two exact formulations are used, each where it measured faster: q_int8 below
+// (the clamped integer, token-order dispatch) and, in quant8f, rr's own bits as a word
+// whose low byte is the code when |r| < 127.5 (where the clamp cannot act: the low byte
+// of 1.5*2^23 + q is q's two's-complement low byte), else the IEEE quotient, clamped.
 //
 // q_int8: the integer, clamped to +-127 (the clamp acts only when the scale itself is
 // inexact far beyond fp32 rounding, i.e. subnormal).
@@ -51,41 +54,22 @@ __device__ __forceinline__ int q_int8(float x, float scale, float inv) {
     return max(-127, min(127, q));
 }
 
-// q_int8_w: a word whose low byte is the code -- rr's own bits when |r| < 127.5, where
-// the clamp cannot act (the low byte of 1.5*2^23 + q is q's two's-complement low byte);
-// else the IEEE quotient, clamped (NaN -> -127).
-__device__ __forceinline__ uint32_t q_int8_w(float x, float scale, float inv) {
-    constexpr float kMagic = 12582912.0f;
-    const float v = __fmul_rn(x, inv);
-    const float rr = __fadd_rn(v, kMagic);
-    const float t = __fsub_rn(v, __fsub_rn(rr, kMagic));
-    if (0.5f - fabsf(t) >= 0.00006103515625f && fabsf(v) < 127.5f) return __float_as_uint(rr);
-    const float q = fminf(fmaxf(__fdiv_rn(x, scale), -127.0f), 127.0f);
-    return __float_as_uint(__fadd_rn(q, kMagic));
-}
-
 // E4M3 keeps 3 mantissa bits: for 2^-6 <= |v| < 448 its rounding boundaries are the fp32
-// values whose 20 low mantissa bits are exactly 0x80000. When r is more than 16 fp32 ulps
-// from such a boundary, rounding to nearest is adding half an E4M3 step to the bits and
-// truncating: the code is sign | ((bits + 0x80000) >> 20) - ((127 - 7) << 3), the carry
-// moving into the exponent when the mantissa rounds up. Elsewhere (near a boundary, in
-// E4M3's subnormal range, at the saturation edge, not finite) the IEEE quotient goes
-// through the hardware conversion (round to nearest even, saturating to +-448). Returns a
-// word whose low byte is the code.
-__device__ __forceinline__ uint32_t q_e4m3(float x, float scale, float inv) {
-    const float r = __fmul_rn(x, inv);
-    const uint32_t b = __float_as_uint(r);
-    const uint32_t u = b & 0x7fffffffu;
-    // (unsigned range tests: 2^-6 <= |r| < 448, and low bits outside [0x80000 +- 16])
-    if (u - 0x3c800000u < 0x43e00000u - 0x3c800000u && (u & 0xfffffu) - 0x7fff0u > 32u)
-        return ((b >> 24) & 0x80u) | (((u + 0x80000u) >> 20) - 0x3c0u);
-    const float v = __fdiv_rn(x, scale);
-    return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(v, 0.0f), __NV_SATFINITE, __NV_E4M3);
+// values whose 20 low mantissa bits are exactly 0x80000. A shortcut quotient r that lies in
+// that range and more than 16 fp32 ulps from such a boundary rounds like the IEEE quotient
+// (the unsigned tests below); elsewhere (near a boundary, in E4M3's subnormal range, at
+// the saturation edge, not finite) the IEEE quotient is used. Two codes come from one
+// hardware conversion of the pair (round to nearest even, saturating to +-448), x0's in
+// the low byte; r0, r1 are the shortcut quotients x * inv.
+__device__ __forceinline__ bool e4m3_shortcut_ok(float r) {
+    const uint32_t u = __float_as_uint(r) & 0x7fffffffu;
+    return u - 0x3c800000u < 0x43e00000u - 0x3c800000u && (u & 0xfffffu) - 0x7fff0u > 32u;
 }
 
-template <int Q>
-__device__ __forceinline__ uint32_t q_code(float x, float scale, float inv) {
-    return Q == MOEDISP_QUANT_INT8 ? q_int8_w(x, scale, inv) : q_e4m3(x, scale, inv);
+__device__ __forceinline__ uint32_t q_e4m3_pair(float x0, float x1, float r0, float r1, float scale) {
+    if (!e4m3_shortcut_ok(r0)) r0 = __fdiv_rn(x0, scale);
+    if (!e4m3_shortcut_ok(r1)) r1 = __fdiv_rn(x1, scale);
+    return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(r0, r1), __NV_SATFINITE, __NV_E4M3);
 }
 
 // The low bytes of four words, in order, in one word (three byte permutes).
@@ -94,11 +78,10 @@ __device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint3
 }
 
 // Eight fp32 values (a smoothed row chunk) to eight codes. The floating-point steps of the
-// fast test run on pairs with the packed fp32x2 instructions (each lane an IEEE
-// round-to-nearest operation, the same result as the scalar one): for int8 the shortcut
-// r = x * inv, rr = r + 1.5*2^23, t = r - (rr - 1.5*2^23); for e4m3 the product r. The
-// decisions, the slow path and the encoding are q_int8_w's and q_e4m3's, element by
-// element.
+// shortcut run on pairs with the packed fp32x2 instructions (each lane an IEEE
+// round-to-nearest operation, the same result as the scalar one): for int8 r = x * inv,
+// rr = r + 1.5*2^23, t = r - (rr - 1.5*2^23), then the code word or the IEEE quotient
+// element by element; for e4m3 the product r, then q_e4m3_pair.
 template <int Q>
 __device__ __forceinline__ uint2 quant8f(const float (&v)[8], float scale, float inv, bool zero) {
     if (zero) return make_uint2(0u, 0u);
@@ -127,20 +110,9 @@ __device__ __forceinline__ uint2 quant8f(const float (&v)[8], float scale, float
                 }
             }
         } else {
-            const float xs[2] = {x0, x1};
-            const float rs[2] = {r.x, r.y};
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const uint32_t bb = __float_as_uint(rs[h]);
-                const uint32_t u = bb & 0x7fffffffu;
-                if (u - 0x3c800000u < 0x43e00000u - 0x3c800000u && (u & 0xfffffu) - 0x7fff0u > 32u) {
-                    b[2 * p + h] = ((bb >> 24) & 0x80u) | (((u + 0x80000u) >> 20) - 0x3c0u);
-                } else {
-                    const float q = __fdiv_rn(xs[h], scale);
-                    b[2 * p + h] = (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(q, 0.0f), __NV_SATFINITE,
-                                                                      __NV_E4M3);
-                }
-            }
+            const uint32_t pr = q_e4m3_pair(x0, x1, r.x, r.y, scale);
+            b[2 * p] = pr & 0xffu;
+            b[2 * p + 1] = pr >> 8;
         }
     }
     return make_uint2(pack_low_bytes(b[0], b[1], b[2], b[3]), pack_low_bytes(b[4], b[5], b[6], b[7]));
@@ -165,8 +137,8 @@ __device__ __forceinline__ uint32_t q_int8_pair(uint32_t w, float scale, float i
     return (uint32_t)(a & 0xff) | ((uint32_t)(b & 0xff) << 8);
 }
 
-// Eight bf16 values (a row chunk) to eight codes: int8 as pairs of clamped integers,
-// e4m3 through byte permutes (each measured the faster in the token-order kernel).
+// Eight bf16 values (a row chunk) to eight codes: int8 as pairs of clamped integers (each
+// formulation measured the faster in the token-order kernel), e4m3 two by two.
 template <int Q>
 __device__ __forceinline__ uint2 quant8(const uint4& v, float scale, float inv, bool zero) {
     if (zero) return make_uint2(0u, 0u);
@@ -177,10 +149,12 @@ __device__ __forceinline__ uint2 quant8(const uint4& v, float scale, float inv, 
     }
     const float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
                         bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
-    uint32_t b[8];
+    uint32_t h[4];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) b[j] = q_e4m3(f[j], scale, inv);
-    return make_uint2(pack_low_bytes(b[0], b[1], b[2], b[3]), pack_low_bytes(b[4], b[5], b[6], b[7]));
+    for (int p = 0; p < 4; ++p)
+        h[p] = q_e4m3_pair(f[2 * p], f[2 * p + 1], __fmul_rn(f[2 * p], inv), __fmul_rn(f[2 * p + 1], inv),
+                           scale);
+    return make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
 }
 
 __device__ __forceinline__ void group_barrier(int id, int threads) {
