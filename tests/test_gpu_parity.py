@@ -1051,6 +1051,49 @@ def test_pipelined_produce_then_consume(md, q):
     _check_pipelined(md, c, q, recv_dev, out)
 
 
+@pytest.mark.parametrize("q", [0, 2])
+def test_pipelined_with_major_align_padding(md, q):
+    """The layout of the received tokens padded to multiples of 16 rows per expert: every
+    routed row as the oracle's exchange + dispatch gives it, the padding rows (assist_info
+    -1) left untouched."""
+    W, K, ne, H = 4, 4, 3, 256
+    a, cap_in, T, x, w = _a2a_case(98, W, 90, H, K, ne)
+    src, outs, dsto, _ = oracle.a2a_exchange_plan(a.in_splits)
+    recv = np.full((W, T, H), 0x7777, np.uint16)
+    assert oracle.a2a_v(x, recv, src, outs, dsto) == 0
+    active = (np.arange(T)[None, :] < outs.sum(axis=1)[:, None]).astype(np.uint8).reshape(-1)
+    A = 16
+    ref = oracle.moe_dispatch_layout(W, T, K, W * ne, w.expert_ids, active, major_align=A)
+    plan = [dev(z.astype(np.int64)) for z in (src, outs, dsto)]
+    L = md.LayoutBuffers.allocate(W, T, K, W * ne, major_align=A)
+    st = new_status()
+    md.moe_dispatch_layout(dev(w.expert_ids.reshape(-1)), dev(active), L, st)
+    full, scales, gr = alloc_expand(L, H, q)
+    recv_dev = torch.full((W * T, H), 0x7777, dtype=torch.int16, device="cuda")
+    ready, ws = _pipe_state(md, W)
+    md.a2a_dispatch_pipelined(bf16_dev(x.reshape(-1, H)), cap_in, plan[0], plan[1], plan[2], recv_dev,
+                              H, L, q, full[gr:gr + L.rows_cap], scales[gr:gr + L.rows_cap] if q else None,
+                              ready, 1, ws, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert np.array_equal(recv_dev.cpu().numpy().view(np.uint16), recv.reshape(W * T, H))
+    rex, rsc, fl = oracle.moe_dispatch(recv.reshape(W * T, H), ref["dst_row"], K, ref["rows_cap"], q)
+    assert fl == 0
+    R = ref["R"]
+    got = full.cpu().numpy()[gr:gr + R]
+    if q == 0:
+        got = got.view(np.uint16)
+    routed = ref["assist_info"][:R] >= 0
+    assert (~routed).any()                                       # there is padding
+    assert np.array_equal(got[routed], rex[:R][routed])
+    canary = 0x5A if q else np.uint16(-12345 & 0xFFFF)
+    assert (got[~routed] == canary).all()
+    if q:
+        sc = scales.cpu().numpy()[gr:gr + R]
+        assert np.array_equal(sc[routed].view(np.uint32), rsc[:R][routed].view(np.uint32))
+        assert (sc[~routed] == -1).all()
+
+
 def test_pipelined_consumer_whose_producer_never_publishes_times_out(md):
     """The dispatch alone, for an epoch nobody published: every wait gives up after the
     20 ms limit (the first one to run out stops the others), the call reports TIMEOUT, the
@@ -1408,7 +1451,7 @@ def test_ep_dispatcher_one_rank_end_to_end(md, q):
     assert res["ok"] and res["epoch"] == 6, res
 
 
-@pytest.mark.parametrize("q", [0, 2])
+@pytest.mark.parametrize("q", [0, 2, 3])
 def test_ep_two_processes_share_one_gpu_through_ipc_mappings(md, q):
     """Two EP ranks as two processes on this GPU: buffers mapped across the processes with
     the library's IPC calls, host barriers only (no kernel waits for the other process);
