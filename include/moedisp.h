@@ -329,7 +329,10 @@ int moedisp_moe_dispatch_gather(const void *x, int64_t x_rows, const int64_t *to
  * segment is not published within this time sets MOEDISP_STATUS_TIMEOUT, and the
  * kernel stops waiting for any segment (the outputs are then incomplete).
  * A segment whose ranges leave their buffers (or has a negative size/offset) is neither
- * exchanged nor dispatched and sets MOEDISP_STATUS_BAD_SPLIT.
+ * exchanged nor dispatched and sets MOEDISP_STATUS_BAD_SPLIT. Tokens are dispatched segment
+ * by segment: a receive position that no valid segment covers is not dispatched even if
+ * the layout routes it (build the layout with the received positions as its mask, e.g.
+ * from a2a_token_rows, and the two agree).
  * workspace: device memory of moedisp_a2a_dispatch_pipelined_workspace_size(W) bytes,
  * 16-byte aligned, no initialisation needed; calls sharing a workspace or ready words
  * must not run concurrently. H % 8 == 0 (NONE) or H % 16 == 0, H <= MOEDISP_MAX_H.

@@ -1094,6 +1094,31 @@ def test_pipelined_with_major_align_padding(md, q):
         assert (sc[~routed] == -1).all()
 
 
+def _random_pipe_case(i):
+    rng = np.random.default_rng(500 + i)
+    W = int(rng.choice([1, 2, 3, 5, 8, 12]))
+    q = int(rng.choice([0, 2, 3]))
+    H = int(rng.choice([16, 48, 256, 1024, 2064] if q else [8, 24, 256, 1000, 2048]))
+    K = int(rng.integers(1, 9))
+    ne = int(rng.integers(1, 5))
+    max_split = int(rng.choice([1, 7, 60, 200]))
+    return W, max_split, H, K, ne, q
+
+
+@pytest.mark.parametrize("i", range(16))
+def test_pipelined_random_configurations(md, i):
+    """Seeded random exchange -> dispatch problems (W from 1 to 12, splits from 0 up to 200
+    rows with zeros, H from 8 to 2064, K from 1 to 8, every quant mode): the pipelined call
+    against the oracle's exchange then dispatch, every output bit-exact."""
+    W, max_split, H, K, ne, q = _random_pipe_case(i)
+    c = _pipelined_case(md, 600 + i, W, max_split, H, K, ne)
+    assert c["fl"] == 0
+    ready, ws = _pipe_state(md, W)
+    recv_dev, out, st = _run_pipelined(md, c, q, 3 + i, ready, ws)
+    assert st == 0, md.status_string(st)
+    _check_pipelined(md, c, q, recv_dev, out)
+
+
 def test_pipelined_consumer_whose_producer_never_publishes_times_out(md):
     """The dispatch alone, for an epoch nobody published: every wait gives up after the
     20 ms limit (the first one to run out stops the others), the call reports TIMEOUT, the
