@@ -62,6 +62,7 @@ struct PipeArgs {
     uint32_t* abort_flag;
     uint32_t* landed;          // [W*W]
     int64_t* item_off;         // [2*W*W + 2]
+    bool offsets_in_smem;      // the main kernel keeps a 32-bit copy of item_off in shared memory
     // dispatch
     const int32_t* dst_row;
     int64_t rows_cap;
@@ -291,6 +292,7 @@ __device__ void consume(const PipeArgs& a, int64_t s, int64_t c, float (&red)[kP
 template <int Q, int WPT, int CPT>
 __global__ void __launch_bounds__(kPipeThreads, CPT > 4 ? 2 : 4) pipe_main_kernel(PipeArgs a, DispatchCounts rc) {
     constexpr int NG = kPipeThreads / 32 / WPT;
+    extern __shared__ int32_t off_sh[];                  // [U + 1] the ticket-slot offsets
     __shared__ float red[NG][2][WPT];
     __shared__ long long t_sh;
     grid_dep_wait();
@@ -298,7 +300,16 @@ __global__ void __launch_bounds__(kPipeThreads, CPT > 4 ? 2 : 4) pipe_main_kerne
     if (a.roles & MOEDISP_PIPE_CONSUME) write_dispatch_counts(rc);
     const int64_t S = (int64_t)a.W * a.W;
     const int64_t U = 2 * S + 1;
-    const int64_t total = __ldcg(a.item_off + U);
+    // Every work item looks its ticket up among the slot offsets: unless W is large, a block
+    // copies them into shared memory once (there are at most 2*W*T items, below 2^31 by the
+    // host's bound on W*T*K), so the lookups are not chains of dependent global loads.
+    const bool sh = a.offsets_in_smem;
+    if (sh) {
+        for (int64_t u = threadIdx.x; u <= U; u += blockDim.x) off_sh[u] = (int32_t)__ldcg(a.item_off + u);
+        __syncthreads();
+    }
+    auto off = [&](int64_t u) -> int64_t { return sh ? (int64_t)off_sh[u] : __ldcg(a.item_off + u); };
+    const int64_t total = off(U);
     int parity = 0;
     while (true) {
         __syncthreads();                                   // t_sh of the last item is read
@@ -306,15 +317,15 @@ __global__ void __launch_bounds__(kPipeThreads, CPT > 4 ? 2 : 4) pipe_main_kerne
         __syncthreads();
         const int64_t t = t_sh;
         if (t >= total) break;
-        int64_t lo = 0, hi = U;                            // item_off[lo] <= t < item_off[hi]
+        int64_t lo = 0, hi = U;                            // off(lo) <= t < off(hi)
         while (hi - lo > 1) {
             const int64_t mid = (lo + hi) >> 1;
-            if (__ldcg(a.item_off + mid) <= t) lo = mid; else hi = mid;
+            if (off(mid) <= t) lo = mid; else hi = mid;
         }
         bool prod;
         int64_t s;
         slot_of(lo, &prod, &s);
-        const int64_t k = t - __ldcg(a.item_off + lo);
+        const int64_t k = t - off(lo);
         if (prod) produce(a, s, k);
         else consume<Q, WPT, CPT>(a, s, k, red, parity);
     }
@@ -325,12 +336,15 @@ cudaError_t launch_pipe_w(PipeArgs a, const DispatchCounts& rc, cudaStream_t str
     constexpr int NG = kPipeThreads / 32 / WPT;
     a.tokens_per_item = (int64_t)NG * kConsumerRounds;
     int per_sm = 1;
-    cudaError_t err = blocks_per_sm((const void*)pipe_main_kernel<Q, WPT, CPT>, kPipeThreads, 0, &per_sm);
+    const size_t table = (size_t)(2 * (int64_t)a.W * a.W + 2) * sizeof(int32_t);
+    a.offsets_in_smem = table <= 48 * 1024;                      // W <= 78
+    const size_t smem = a.offsets_in_smem ? table : 0;
+    cudaError_t err = blocks_per_sm((const void*)pipe_main_kernel<Q, WPT, CPT>, kPipeThreads, smem, &per_sm);
     if (err != cudaSuccess) return err;
     err = launch_pdl(pipe_setup_kernel, dim3(1), dim3(kSetupThreads), 0, stream, 1, a);
     if (err != cudaSuccess) return err;
     const int64_t grid = (int64_t)current_sm_count() * per_sm;
-    return launch_pdl(pipe_main_kernel<Q, WPT, CPT>, dim3((unsigned)grid), dim3(kPipeThreads), 0,
+    return launch_pdl(pipe_main_kernel<Q, WPT, CPT>, dim3((unsigned)grid), dim3(kPipeThreads), smem,
                       stream, 1, a, rc);
 }
 
@@ -378,6 +392,7 @@ cudaError_t launch_a2a_dispatch_pipelined(const void* in, int64_t in_rank_stride
     a.H8 = H / 8;
     a.rows_per_piece = std::max<int64_t>(1, kPieceBytes / ((int64_t)H * 2));
     a.tokens_per_item = 1;
+    a.offsets_in_smem = false;
     a.roles = roles;
     a.epoch = epoch;
     a.ready = ready;

@@ -1007,7 +1007,8 @@ def _pipe_state(md, W):
 
 @pytest.mark.parametrize("q", [0, 2, 3])
 @pytest.mark.parametrize("W,max_split,H,K,ne", [(8, 120, 256, 4, 4), (4, 300, 2048, 8, 2),
-                                                (16, 40, 7168, 2, 1), (3, 50, 16, 3, 5)])
+                                                (16, 40, 7168, 2, 1), (3, 50, 16, 3, 5),
+                                                (96, 4, 64, 2, 1)])   # W = 96: offsets in global memory
 def test_pipelined_exchange_and_dispatch(md, q, W, max_split, H, K, ne):
     """a2a_dispatch_pipelined equals the oracle's exchange into a receive buffer followed by
     its dispatch: the receive buffer (untouched positions included), every dispatched row,
