@@ -723,33 +723,21 @@ def op_sweep(md, torch, device, hbm, reps=10, main_workload="cfg3"):
 
     ready = torch.zeros((W_, W_), dtype=torch.int32, device=device)
     pws = torch.empty(md.a2a_dispatch_pipelined_workspace_size(W_), dtype=torch.uint8, device=device)
-    epoch = [0]
 
     def pipelined():
         front()
-        epoch[0] += 1           # a new epoch per exchange (the graph replays this value)
+        # the graph replays one epoch: the ready words are zeroed in stream order first
+        ready.zero_()
         md.a2a_dispatch_pipelined(xin, cap_in, plan[0], plan[1], plan[2], recv, H_, L, 0, ex, None,
-                                  ready, epoch[0], pws, status)
+                                  ready, 1, pws, status)
 
     res = {}
-    for nm, fn in (("sequential", sequential), ("no_receive_buffer", fused)):
+    for nm, fn in (("sequential", sequential), ("no_receive_buffer", fused),
+                   ("pipelined_ready_words", pipelined)):
         g = capture(torch, fn)
         res[nm] = statistics.mean(time_graph(torch, g, reps, 3, flush))
         del g
-    # the pipelined call publishes its epoch into the ready words, so each timed call needs
-    # a new epoch: eager launches (the host enqueues them behind the flush)
-    Ev = torch.cuda.Event
-    pairs = []
-    for r in range(reps + 3):
-        flush.zero_()
-        e0, e1 = Ev(enable_timing=True), Ev(enable_timing=True)
-        e0.record()
-        pipelined()
-        e1.record()
-        if r >= 3:
-            pairs.append((e0, e1))
     torch.cuda.synchronize()
-    res["pipelined_ready_words"] = statistics.mean(x.elapsed_time(y) for x, y in pairs)
     assert int(status.item()) == 0, md.status_string(int(status.item()))
     n_recv = int(a.in_splits.sum())
     R = int(L.expert_base[-1].item())

@@ -344,8 +344,9 @@ def a2a_dispatch_pipelined(inp, in_rank_stride_rows, src_offsets, out_splits, ds
                            ep_recv_counts=None, stream=None, raise_on_error=True) -> int:
     """The exchange (a2a_v into recv [W][T][H]) and the dispatch of the received tokens
     (layout over the W*T receive positions), pipelined through per-segment ready words
-    (uint32 [W][W], zeroed once; a new epoch per exchange). workspace: a device buffer of
-    a2a_dispatch_pipelined_workspace_size(W) bytes."""
+    (uint32 [W][W], zeroed once; a new epoch 1, 2, ... per exchange -- or, for a CUDA
+    graph, ready zeroed in stream order before every call and epoch 1 each time).
+    workspace: a device buffer of a2a_dispatch_pipelined_workspace_size(W) bytes."""
     L = layout.struct()
     rc = _pipe(_ptr(inp), int(in_rank_stride_rows), _ptr(src_offsets), _ptr(out_splits),
                _ptr(dst_offsets), _ptr(recv), int(H), layout.dims, ctypes.byref(L), int(quant_mode),

@@ -176,7 +176,7 @@ int moedisp_selftest_bounded_wait(uint32_t limit_us, int32_t* status, moedisp_st
 int moedisp_ep_barrier(uint32_t* const* peer_signals, int W, int rank, uint32_t epoch,
                        uint32_t timeout_us, int32_t* status, moedisp_stream_t stream) {
     if (!peer_signals || !status) return MOEDISP_ERR_NULLPTR;
-    if (W < 1 || rank < 0 || rank >= W) return MOEDISP_ERR_INVALID;
+    if (W < 1 || rank < 0 || rank >= W || epoch == 0) return MOEDISP_ERR_INVALID;
     if (W > MOEDISP_MAX_W) return MOEDISP_ERR_UNSUPPORTED;
     if (timeout_us < 1 || timeout_us > 10000000u) return MOEDISP_ERR_INVALID;
     if (!aligned(peer_signals, 8) || !aligned(status, 4)) return MOEDISP_ERR_MISALIGNED;
@@ -365,6 +365,7 @@ int moedisp_a2a_dispatch_pipelined(const void* in, int64_t in_rank_stride_rows,
     if (roles != MOEDISP_PIPE_PRODUCE && roles != MOEDISP_PIPE_CONSUME && roles != MOEDISP_PIPE_BOTH)
         return MOEDISP_ERR_INVALID;
     if (wait_limit_us < 1 || wait_limit_us > 10000000u) return MOEDISP_ERR_INVALID;
+    if (epoch == 0) return MOEDISP_ERR_INVALID;        // zeroed words would read as published
     if (H <= 0 || in_rank_stride_rows < 0) return MOEDISP_ERR_INVALID;
     if (H > MOEDISP_MAX_H) return MOEDISP_ERR_UNSUPPORTED;
     if (H % (quant_mode == MOEDISP_QUANT_NONE ? 8 : 16) != 0) return MOEDISP_ERR_MISALIGNED;

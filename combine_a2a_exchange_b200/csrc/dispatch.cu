@@ -218,23 +218,130 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
 // Quantising dispatch with per-expert smoothing. The copy of token g for expert e is
 // x[g] * smooth[e] quantised on its own, so the work is per row of expand_x, not per
 // token, and it is arithmetic-heavy (a product, a maximum and a quantisation per output
-// element). Rows are taken in their own order (grouped by expert): a block takes chunks of
-// consecutive rows; for each expert segment of a chunk it copies smooth[e] into shared
-// memory once, and its token groups (WPT warps each) share the segment's rows. A group
-// gathers its row's token x[assist_info[row] / K] straight into registers (CPT 16-byte
-// chunks per thread, all loads issued before the first use), reduces max |x * smooth[e]|
-// (shuffles, plus a named barrier across the group's warps), and stores the codes (8
-// bytes per chunk, coalesced) and the row's scale. No staging buffers, so many warps fit
-// an SM; the smoothing table is read about once; nothing waits on another block.
+// element). A block takes chunks of rows of one expert at a time: it copies smooth[e] into
+// shared memory once per run of rows, and its token groups (WPT warps each) share the
+// rows. A group gathers its row's token x[assist_info[row] / K] straight into registers
+// (CPT 16-byte chunks per thread, all loads issued before the first use), reduces
+// max |x * smooth[e]| (shuffles, plus a named barrier across the group's warps), and
+// stores the codes (8 bytes per chunk, coalesced) and the row's scale. No staging
+// buffers, so many warps fit an SM; nothing waits on another block.
+//
+// Order of the rows. Within an expert's segment the rows are in slot order, hence grouped
+// by source rank: rank r's rows of expert e start at expert_base[e] + sum_{r'<r} cnt[r'][e].
+// RANK_ORDER walks the rows rank by rank (for each rank, its part of every expert's
+// segment), so that all K copies of a token are quantised while its x row is still in L2:
+// the whole grid works on one or two ranks' tokens at a time instead of on every token
+// (each row of x is then read from DRAM about once rather than up to K times). Without
+// RANK_ORDER (cnt absent or the tables too large) the rows go in expand_x order.
+
+// Rows [row, seg_end) of expert e; smooth[e] is loaded into sbuf first.
+// max(|a|, |b|, |c|) in one instruction (the three-input form of max, sm_100 and later);
+// like fmaxf, a NaN input is passed over in favour of the others.
+__device__ __forceinline__ float fmax3_abs(float a, float b, float c) {
+    float r;
+    asm("max.abs.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 template <int Q, int WPT, int CPT>
-__global__ void __launch_bounds__(kQuantThreads, CPT > 4 ? 2 : 4) dispatch_smooth_kernel(DispatchArgs a) {
+__device__ __forceinline__ void smooth_rows(const DispatchArgs& a, float4* sbuf, float (*red)[2][WPT],
+                                            int e, int64_t row, int64_t seg_end, int& parity) {
     constexpr int NG = kQuantThreads / 32 / WPT;     // groups per block
     constexpr int GT = WPT * 32;                     // threads per group
     constexpr float kQmax = Q == MOEDISP_QUANT_INT8 ? 127.0f : 448.0f;
-    extern __shared__ __align__(16) float4 sbuf[];   // [H / 4]: smooth[e]
-    __shared__ float red[NG][2][WPT];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int grp = warp / WPT, gw = warp - grp * WPT, gt = tid - grp * GT;
+    const int nvec = a.H >> 3, n4 = a.H >> 2;
+    const int64_t slots = a.G * a.K;
+    const uint4* x4 = reinterpret_cast<const uint4*>(a.x);
+    // smooth[e] in two planes: chunk c's first four values at sbuf[c], its last four at
+    // sbuf[nvec + c], so that a warp's 16-byte reads of consecutive chunks are contiguous
+    // (interleaved, they would span twice the banks' width: two wavefronts per read)
+    __syncthreads();                                 // every group is done with the last rows
+    const float4* src = reinterpret_cast<const float4*>(a.smooth + (int64_t)e * a.H);
+    for (int i = tid; i < n4; i += kQuantThreads) sbuf[(i & 1) * nvec + (i >> 1)] = __ldg(src + i);
+    __syncthreads();
+    for (row += grp; row < seg_end; row += NG) {
+        const int32_t slot = __ldg(a.assist + row);          // same for the group
+        if (slot == -1) continue;                            // a padding row
+        if (slot < 0 || (int64_t)slot >= slots) {
+            if (gt == 0) raise_status(a.status, MOEDISP_STATUS_BAD_EXPERT_ID);
+            continue;
+        }
+        const int64_t xrow = token_source(a, slot / a.K);     // same for the group
+        if (xrow < 0 || xrow >= a.x_rows) {
+            if (gt == 0) raise_status(a.status, MOEDISP_STATUS_BAD_SPLIT);
+            continue;
+        }
+        const uint4* xr = x4 + xrow * nvec;
+        uint4 v[CPT];
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) {
+            const int c = gt + j * GT;
+            v[j] = c < nvec ? __ldg(xr + c) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        float mq[2] = {0.0f, 0.0f};                 // independent partial maxima
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) {
+            const int c = gt + j * GT;
+            if (c < nvec) {
+                float xs[8];
+                smooth8(v[j], sbuf[c], sbuf[nvec + c], xs);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) mq[q & 1] = fmax3_abs(mq[q & 1], xs[2 * q], xs[2 * q + 1]);
+            }
+        }
+        float m = fmaxf(mq[0], mq[1]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (WPT > 1) {
+            if (lane == 0) red[grp][parity][gw] = m;
+            group_barrier(1 + grp, GT);
+#pragma unroll
+            for (int w = 0; w < WPT; ++w) m = fmaxf(m, red[grp][parity][w]);
+            parity ^= 1;
+        }
+        const float scale = __fdiv_rn(m, kQmax);
+        const float inv = __frcp_rn(scale);
+        uint2* dst = reinterpret_cast<uint2*>(a.expand_x + row * a.out_bytes);
+        // the window decides (nearly) every code; a thread with an undecided one rewrites
+        // its chunks element by element (same thread, same addresses: the later stores are
+        // the ones that stay)
+        uint32_t amb = window_ok(scale) ? 0u : 1u;
+        if (amb == 0u) {
+            const float2 lo = window_lo(inv), hi = window_hi(inv);
+#pragma unroll
+            for (int j = 0; j < CPT; ++j) {
+                const int c = gt + j * GT;
+                if (c < nvec) {
+                    float xs[8];
+                    smooth8(v[j], sbuf[c], sbuf[nvec + c], xs);
+                    __stcs(dst + c, quant8w<Q>(xs, lo, hi, amb));
+                }
+            }
+        }
+        if (amb != 0u) {
+#pragma unroll
+            for (int j = 0; j < CPT; ++j) {
+                const int c = gt + j * GT;
+                if (c < nvec) {
+                    float xs[8];
+                    smooth8(v[j], sbuf[c], sbuf[nvec + c], xs);
+                    __stcs(dst + c, quant8f<Q>(xs, scale, inv, m == 0.0f));
+                }
+            }
+        }
+        if (gt == 0) a.scales[row] = scale;
+    }
+}
+
+template <int Q, int WPT, int CPT, bool RANK_ORDER>
+__global__ void __launch_bounds__(kQuantThreads, CPT > 4 ? 3 : 4) dispatch_smooth_kernel(DispatchArgs a) {
+    constexpr int NG = kQuantThreads / 32 / WPT;
+    extern __shared__ __align__(16) float4 sbuf[];   // [H / 4]: smooth[e]; then the tables
+    __shared__ float red[NG][2][WPT];
+    __shared__ int64_t warp_tot[32];
+    const int tid = threadIdx.x;
     grid_dep_wait();
     grid_dep_launch_dependents();
     write_recv_counts(a);
@@ -243,81 +350,76 @@ __global__ void __launch_bounds__(kQuantThreads, CPT > 4 ? 2 : 4) dispatch_smoot
     if (blockIdx.x == 0 && tid == 0 && r_all > a.rows_cap)
         raise_status(a.status, MOEDISP_STATUS_CAPACITY);
     const int64_t R = min64(r_all, a.rows_cap);
-    const int64_t RC = max64(64, (R + 4 * (int64_t)gridDim.x - 1) / (4 * (int64_t)gridDim.x));
-    const int nvec = a.H >> 3, n4 = a.H >> 2;
-    const int64_t slots = a.G * a.K;
-    const uint4* x4 = reinterpret_cast<const uint4*>(a.x);
     int parity = 0;
 
-    for (int64_t ch = blockIdx.x; ch * RC < R; ch += gridDim.x) {
-        int64_t r = ch * RC;
-        const int64_t end = min64(R, r + RC);
-        int lo = 0, hi = a.E;                       // expert_base[lo] <= r < expert_base[hi]
+    if (!RANK_ORDER) {
+        const int64_t RC = max64(64, (R + 4 * (int64_t)gridDim.x - 1) / (4 * (int64_t)gridDim.x));
+        for (int64_t ch = blockIdx.x; ch * RC < R; ch += gridDim.x) {
+            int64_t r = ch * RC;
+            const int64_t end = min64(R, r + RC);
+            int lo = 0, hi = a.E;                   // expert_base[lo] <= r < expert_base[hi]
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (a.expert_base[mid] <= r) lo = mid; else hi = mid;
+            }
+            for (int e = lo; r < end; ++e) {
+                const int64_t seg_end = min64(end, a.expert_base[e + 1]);
+                if (seg_end <= r) continue;
+                smooth_rows<Q, WPT, CPT>(a, sbuf, red, e, r, seg_end, parity);
+                r = seg_end;
+            }
+        }
+        return;
+    }
+
+    // Tables over the W*E (rank, expert) parts, rank-major: vpre[i] = routed rows of the
+    // parts before part i (vpre[W*E] = all of them), cpre[i] = offset of part i in its
+    // expert's segment (sum of cnt over the lower ranks).
+    const int WE = a.W * a.E;
+    int32_t* vpre = reinterpret_cast<int32_t*>(sbuf + (a.H >> 2));
+    int32_t* cpre = vpre + WE + 1;
+    for (int e = tid; e < a.E; e += kQuantThreads) {
+        int32_t run = 0;
+        for (int q = 0; q < a.W; ++q) {
+            const int32_t c = __ldg(a.cnt + (int64_t)q * a.E + e);
+            cpre[q * a.E + e] = run;
+            vpre[q * a.E + e + 1] = c;
+            run += c;
+        }
+    }
+    __syncthreads();
+    {
+        const int per = (WE + kQuantThreads - 1) / kQuantThreads;
+        const int i0 = min(WE, tid * per), i1 = min(WE, i0 + per);
+        int64_t part = 0;
+        for (int i = i0; i < i1; ++i) part += vpre[i + 1];
+        int64_t total;
+        int64_t run = block_exclusive_scan(part, warp_tot, total);
+        for (int i = i0; i < i1; ++i) {
+            run += vpre[i + 1];
+            vpre[i + 1] = (int32_t)run;
+        }
+        if (tid == 0) vpre[0] = 0;
+    }
+    __syncthreads();
+    const int64_t Rv = vpre[WE];
+    const int64_t RC = max64(64, (Rv + 4 * (int64_t)gridDim.x - 1) / (4 * (int64_t)gridDim.x));
+    for (int64_t ch = blockIdx.x; ch * RC < Rv; ch += gridDim.x) {
+        int64_t v = ch * RC;
+        const int64_t vend = min64(Rv, v + RC);
+        int lo = 0, hi = WE;                        // vpre[lo] <= v < vpre[hi]
         while (hi - lo > 1) {
             const int mid = (lo + hi) >> 1;
-            if (a.expert_base[mid] <= r) lo = mid; else hi = mid;
+            if (vpre[mid] <= v) lo = mid; else hi = mid;
         }
-        for (int e = lo; r < end; ++e) {
-            const int64_t seg_end = min64(end, a.expert_base[e + 1]);
-            if (seg_end <= r) continue;
-            __syncthreads();                        // every group is done with the last row
-            const float4* src = reinterpret_cast<const float4*>(a.smooth + (int64_t)e * a.H);
-            for (int i = tid; i < n4; i += kQuantThreads) sbuf[i] = __ldg(src + i);
-            __syncthreads();
-            for (int64_t row = r + grp; row < seg_end; row += NG) {
-                const int32_t slot = __ldg(a.assist + row);          // same for the group
-                if (slot == -1) continue;                            // a padding row
-                if (slot < 0 || (int64_t)slot >= slots) {
-                    if (gt == 0) raise_status(a.status, MOEDISP_STATUS_BAD_EXPERT_ID);
-                    continue;
-                }
-                const int64_t src = token_source(a, slot / a.K);      // same for the group
-                if (src < 0 || src >= a.x_rows) {
-                    if (gt == 0) raise_status(a.status, MOEDISP_STATUS_BAD_SPLIT);
-                    continue;
-                }
-                const uint4* xr = x4 + src * nvec;
-                uint4 v[CPT];
-#pragma unroll
-                for (int j = 0; j < CPT; ++j) {
-                    const int c = gt + j * GT;
-                    v[j] = c < nvec ? __ldg(xr + c) : make_uint4(0u, 0u, 0u, 0u);
-                }
-                float m = 0.0f;
-#pragma unroll
-                for (int j = 0; j < CPT; ++j) {
-                    const int c = gt + j * GT;
-                    if (c < nvec) {
-                        float xs[8];
-                        smooth8(v[j], sbuf + 2 * c, xs);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) m = fmaxf(m, fabsf(xs[q]));
-                    }
-                }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-                if (WPT > 1) {
-                    if (lane == 0) red[grp][parity][gw] = m;
-                    group_barrier(1 + grp, GT);
-#pragma unroll
-                    for (int w = 0; w < WPT; ++w) m = fmaxf(m, red[grp][parity][w]);
-                    parity ^= 1;
-                }
-                const float scale = __fdiv_rn(m, kQmax);
-                const float inv = __frcp_rn(scale);
-                uint2* dst = reinterpret_cast<uint2*>(a.expand_x + row * a.out_bytes);
-#pragma unroll
-                for (int j = 0; j < CPT; ++j) {
-                    const int c = gt + j * GT;
-                    if (c < nvec) {
-                        float xs[8];
-                        smooth8(v[j], sbuf + 2 * c, xs);
-                        __stcs(dst + c, quant8f<Q>(xs, scale, inv, m == 0.0f));
-                    }
-                }
-                if (gt == 0) a.scales[row] = scale;
-            }
-            r = seg_end;
+        for (int i = lo; v < vend; ++i) {
+            const int64_t part_end = min64(vend, vpre[i + 1]);
+            if (part_end <= v) continue;
+            const int e = i % a.E;
+            const int64_t row = __ldg(a.expert_base + e) + cpre[i] + (v - vpre[i]);
+            const int64_t row_end = min64(R, row + (part_end - v));
+            if (row < row_end) smooth_rows<Q, WPT, CPT>(a, sbuf, red, e, row, row_end, parity);
+            v = part_end;
         }
     }
 }
@@ -378,10 +480,24 @@ __global__ void __launch_bounds__(kQuantThreads, CPT > 4 ? 2 : 4) dispatch_quant
         }
         const float scale = __fdiv_rn(m, kQmax);
         const float inv = __frcp_rn(scale);
-        const bool zero = m == 0.0f;
         uint2 q[CPT];
+        // e4m3: the window of the smoothing kernel (cfg4 fp8 96.7 -> 94.4 us); int8 keeps
+        // the element-by-element decision, which measured faster here (400 vs 436 us on
+        // cfg3) although the window wins in the smoothing kernel
+        uint32_t amb = Q == MOEDISP_QUANT_FP8_E4M3 && window_ok(scale) ? 0u : 1u;
+        if (amb == 0u) {
+            const float2 lo = window_lo(inv), hi = window_hi(inv);
 #pragma unroll
-        for (int j = 0; j < CPT; ++j) q[j] = quant8<Q>(v[j], scale, inv, zero);
+            for (int j = 0; j < CPT; ++j) {
+                float f[8];
+                unpack8(v[j], f);
+                q[j] = quant8w<Q>(f, lo, hi, amb);
+            }
+        }
+        if (amb != 0u) {
+#pragma unroll
+            for (int j = 0; j < CPT; ++j) q[j] = quant8<Q>(v[j], scale, inv, m == 0.0f);
+        }
         // PEERS: lane k resolves slot k's rank and local row (and scale address)
         uint8_t* myrow = nullptr;
         float* mysc = nullptr;
@@ -439,18 +555,37 @@ cudaError_t launch_copy(DispatchArgs a, cudaStream_t stream) {
                       dim3((unsigned)grid), dim3(kCopyThreads), smem, stream, 1, a);
 }
 
-// Smoothing kernel geometry: CPT chunks of the row per thread and WPT warps per row: the
-// fewest chunks per thread up to four (registers, hence warps per SM, matter most here),
-// then eight for the widest rows.
+// Smoothing kernel geometry: CPT chunks of the row per thread and WPT warps per row. Each
+// warp of a row's group repeats the row's own work (its routing and token lookups, checks,
+// the scale's division and reciprocal, the group maximum), so few warps per row with many
+// chunks each (up to 8; 80 registers, 3 blocks per SM) beat many warps with few chunks:
+// cfg3 (H = 7168: 4 warps x 7 chunks, an exact fit) 1430 -> 1083 us against 8 x 4; cfg4
+// (H = 2048: 1 warp x 8) 282 -> 248 us against 2 x 4; 2 blocks per SM (105 registers)
+// measured in between.
+//
+// Rank order (see the kernel) when x is well beyond the L2 (up to about twice its size
+// most of the K re-reads of a row hit it anyway, and the tables cost more than they save:
+// cfg4, 134 MB of x, 250 vs 235 us; cfg3, 470 MB, 1085 vs 1161 us), the layout's counts
+// are given, their tables fit in shared memory beside the smoothing row and the row
+// counts fit in 32 bits.
+constexpr int kSmoothMaxParts = 4096;
+
 template <int Q, int WPT, int CPT>
 cudaError_t launch_smooth_w(DispatchArgs a, cudaStream_t stream) {
-    const size_t smem = (size_t)a.H * 4;
+    const int64_t WE = (int64_t)a.W * a.E;
+    const bool ranked = a.cnt != nullptr && WE <= kSmoothMaxParts && a.G * a.K < (int64_t)INT32_MAX &&
+                        a.x_rows * (int64_t)a.in_bytes > 2 * current_l2_bytes();
+    const size_t smem = (size_t)a.H * 4 + (ranked ? (size_t)(2 * WE + 1) * 4 : 0);
+    const void* fn = ranked ? (const void*)dispatch_smooth_kernel<Q, WPT, CPT, true>
+                            : (const void*)dispatch_smooth_kernel<Q, WPT, CPT, false>;
     int per_sm = 1;
-    cudaError_t err = blocks_per_sm((const void*)dispatch_smooth_kernel<Q, WPT, CPT>, kQuantThreads,
-                                    smem, &per_sm);
+    cudaError_t err = blocks_per_sm(fn, kQuantThreads, smem, &per_sm);
     if (err != cudaSuccess) return err;
     const int64_t grid = (int64_t)current_sm_count() * per_sm;
-    return launch_pdl(dispatch_smooth_kernel<Q, WPT, CPT>, dim3((unsigned)grid),
+    if (ranked)
+        return launch_pdl(dispatch_smooth_kernel<Q, WPT, CPT, true>, dim3((unsigned)grid),
+                          dim3(kQuantThreads), smem, stream, 1, a);
+    return launch_pdl(dispatch_smooth_kernel<Q, WPT, CPT, false>, dim3((unsigned)grid),
                       dim3(kQuantThreads), smem, stream, 1, a);
 }
 
@@ -460,9 +595,10 @@ cudaError_t launch_smooth(const DispatchArgs& a, cudaStream_t stream) {
     if (nvec <= 32) return launch_smooth_w<Q, 1, 1>(a, stream);
     if (nvec <= 64) return launch_smooth_w<Q, 1, 2>(a, stream);
     if (nvec <= 128) return launch_smooth_w<Q, 1, 4>(a, stream);
-    if (nvec <= 256) return launch_smooth_w<Q, 2, 4>(a, stream);
-    if (nvec <= 512) return launch_smooth_w<Q, 4, 4>(a, stream);
-    if (nvec <= 1024) return launch_smooth_w<Q, 8, 4>(a, stream);
+    if (nvec <= 256) return launch_smooth_w<Q, 1, 8>(a, stream);
+    if (nvec <= 512) return launch_smooth_w<Q, 2, 8>(a, stream);
+    if (nvec <= 896) return launch_smooth_w<Q, 4, 7>(a, stream);
+    if (nvec <= 1024) return launch_smooth_w<Q, 4, 8>(a, stream);
     return launch_smooth_w<Q, 8, 8>(a, stream);
 }
 

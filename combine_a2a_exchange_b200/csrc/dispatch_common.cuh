@@ -11,6 +11,11 @@ namespace moedisp {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+__device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
+    f[0] = bf16_lo(v.x); f[1] = bf16_hi(v.x); f[2] = bf16_lo(v.y); f[3] = bf16_hi(v.y);
+    f[4] = bf16_lo(v.z); f[5] = bf16_hi(v.z); f[6] = bf16_lo(v.w); f[7] = bf16_hi(v.w);
+}
+
 __device__ __forceinline__ float absmax8(const uint4& v) {
     float m = fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x)));
     m = fmaxf(m, fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y))));
@@ -118,11 +123,68 @@ __device__ __forceinline__ uint2 quant8f(const float (&v)[8], float scale, float
     return make_uint2(pack_low_bytes(b[0], b[1], b[2], b[3]), pack_low_bytes(b[4], b[5], b[6], b[7]));
 }
 
-// x chunk (8 bf16) times a smoothing chunk (8 fp32, shared memory), one correctly rounded
-// product each (four packed fp32x2 multiplies).
-__device__ __forceinline__ void smooth8(const uint4& v, const float4* s, float (&o)[8]) {
-    const float4 s0 = s[0];
-    const float4 s1 = s[1];
+// Window quantisation: the code of every element of a row at once, for a row whose scale
+// is a normal number. With inv = RN(1/scale), lo = RN(inv * (1 - 2^-22)) and
+// hi = RN(inv * (1 + 2^-22)) satisfy
+//   lo <= (1/scale) (1 + 2^-24)^2 (1 - 2^-22) < (1/scale) (1 - 2^-24)   and
+//   hi >= (1/scale) (1 - 2^-24)^2 (1 + 2^-22) > (1/scale) (1 + 2^-24),
+// while the IEEE quotient RN(x/scale) lies within (x/scale) (1 +- 2^-24) (or is below
+// every rounding boundary, when it is subnormal). So the exact products x*lo and x*hi
+// bracket RN(x/scale); both encodings are monotone (non-decreasing) functions of their
+// input, so where the two ends give the same code, that code is RN(x/scale)'s. For int8
+// an end is one fused multiply-add, RN(x*lo + 1.5*2^23), whose bits are those of
+// 1.5*2^23 + rint(x*lo) (|x*lo| <= 127.0001 with a normal scale, so no clamp can act; the
+// low byte is the code); for E4M3 an end is the rounded product RN(x*lo) (rounding is
+// monotone too) converted by the hardware pair conversion. `amb` collects the bits in
+// which the two ends differ: zero when every code was decided. An end's rounding
+// window is |v| * 2^-21 wide, so a code is left undecided about once per 10^5 elements.
+template <int Q>
+__device__ __forceinline__ uint2 quant8w(const float (&v)[8], float2 lo, float2 hi, uint32_t& amb) {
+    if constexpr (Q == MOEDISP_QUANT_INT8) {
+        constexpr float kMagic = 12582912.0f;                    // 1.5 * 2^23
+        const float2 mg = make_float2(kMagic, kMagic);
+        uint32_t b[8];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const float2 x = make_float2(v[2 * p], v[2 * p + 1]);
+            const float2 a = __ffma2_rn(x, lo, mg);
+            const float2 c = __ffma2_rn(x, hi, mg);
+            b[2 * p] = __float_as_uint(a.x);
+            b[2 * p + 1] = __float_as_uint(a.y);
+            amb |= (b[2 * p] ^ __float_as_uint(c.x)) | (b[2 * p + 1] ^ __float_as_uint(c.y));
+        }
+        return make_uint2(pack_low_bytes(b[0], b[1], b[2], b[3]), pack_low_bytes(b[4], b[5], b[6], b[7]));
+    } else {
+        uint32_t h[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const float2 x = make_float2(v[2 * p], v[2 * p + 1]);
+            const uint32_t a = (uint32_t)__nv_cvt_float2_to_fp8x2(__fmul2_rn(x, lo), __NV_SATFINITE, __NV_E4M3);
+            const uint32_t c = (uint32_t)__nv_cvt_float2_to_fp8x2(__fmul2_rn(x, hi), __NV_SATFINITE, __NV_E4M3);
+            h[p] = a;
+            amb |= a ^ c;
+        }
+        return make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
+    }
+}
+
+// Whether a row's codes can come from the window (its scale a normal, finite number), and
+// the two ends of the window.
+__device__ __forceinline__ bool window_ok(float scale) {
+    return scale >= 1.17549435e-38f && scale <= 3.40282347e38f;
+}
+__device__ __forceinline__ float2 window_lo(float inv) {
+    const float t = __fmul_rn(inv, 0.999999761581420898f);    // 1 - 2^-22
+    return make_float2(t, t);
+}
+__device__ __forceinline__ float2 window_hi(float inv) {
+    const float t = __fmul_rn(inv, 1.00000023841857910f);     // 1 + 2^-22
+    return make_float2(t, t);
+}
+
+// x chunk (8 bf16) times a smoothing chunk (8 fp32: s0 its first four, s1 its last four),
+// one correctly rounded product each (four packed fp32x2 multiplies).
+__device__ __forceinline__ void smooth8(const uint4& v, const float4& s0, const float4& s1, float (&o)[8]) {
     const float2 p0 = __fmul2_rn(make_float2(bf16_lo(v.x), bf16_hi(v.x)), make_float2(s0.x, s0.y));
     const float2 p1 = __fmul2_rn(make_float2(bf16_lo(v.y), bf16_hi(v.y)), make_float2(s0.z, s0.w));
     const float2 p2 = __fmul2_rn(make_float2(bf16_lo(v.z), bf16_hi(v.z)), make_float2(s1.x, s1.y));

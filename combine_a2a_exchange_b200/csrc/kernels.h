@@ -13,6 +13,7 @@ namespace moedisp {
 
 // Streaming-multiprocessor count of the current device (cached per device).
 int current_sm_count();
+int64_t current_l2_bytes();     // L2 cache size of the current device
 
 // Lets `kernel` use the device's full opt-in dynamic shared memory (once per device).
 cudaError_t allow_dynamic_smem(const void* kernel);

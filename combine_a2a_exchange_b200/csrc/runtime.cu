@@ -33,6 +33,19 @@ int current_sm_count() {
     return n;
 }
 
+int64_t current_l2_bytes() {
+    static std::map<int, int64_t> cache;
+    const int dev = current_device();
+    std::lock_guard<std::mutex> lock(g_mu);
+    auto it = cache.find(dev);
+    if (it != cache.end()) return it->second;
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrL2CacheSize, dev) != cudaSuccess || n <= 0)
+        n = 126 << 20;
+    cache[dev] = n;
+    return n;
+}
+
 cudaError_t allow_dynamic_smem(const void* kernel) {
     static std::set<std::pair<int, const void*>> done;
     const int dev = current_device();

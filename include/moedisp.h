@@ -321,7 +321,11 @@ int moedisp_moe_dispatch_gather(const void *x, int64_t x_rows, const int64_t *to
  * quant_mode, expand_x, dynamic_scales, expert_token_nums(_type), ep_recv_counts as for
  * moe_dispatch (no smoothing).
  * ready: uint32 [W][W] device, zeroed once when allocated and then left to this call;
- * epoch: 1, 2, 3, ... a new value for every exchange (the ready words keep the last one).
+ * epoch: 1, 2, 3, ... a new value for every exchange (the ready words keep the last one;
+ * compared for equality, so after 2^32 - 1 the sequence goes on with 1).
+ * Equally valid, and the form a CUDA graph can replay: zero the ready words in stream
+ * order before every call and pass the same epoch each time (say 1). epoch 0 is rejected
+ * (MOEDISP_ERR_INVALID): zeroed words would read as already published.
  * roles: MOEDISP_PIPE_BOTH (the normal case); MOEDISP_PIPE_PRODUCE, the exchange alone,
  * publishing the ready words; MOEDISP_PIPE_CONSUME, the dispatch alone, for rows that
  * another party delivered into recv and published with this epoch (a PRODUCE call of
@@ -443,7 +447,9 @@ int moedisp_ipc_close(void *dev_ptr);
  *     with wrap-around), so that no rank's later kernels start before every rank has
  *     finished its earlier ones.
  * epoch: 1, 2, 3, ... in the same sequence on every rank (one per barrier; words are never
- * reset). A wait longer than timeout_us (1..10^7 microseconds) gives up, ORs
+ * reset); 0 is rejected (MOEDISP_ERR_INVALID: it would pass zeroed words), so after
+ * 2^32 - 1 the sequence goes on with 1 (the wrap-around compare holds while no rank is
+ * 2^31 barriers ahead of another). A wait longer than timeout_us (1..10^7 microseconds) gives up, ORs
  * MOEDISP_STATUS_TIMEOUT into *status and returns: a rank that died or fell behind is
  * reported, not waited for (the caller reads the status and stops). W = 1 only publishes.
  * One block. */

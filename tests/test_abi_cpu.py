@@ -296,9 +296,10 @@ def test_binding_host_logic(md):
 
 def test_ep_barrier_rejections(md):
     tab, st = FAKE + (1 << 20), FAKE + (2 << 20)
-    b = lambda tab=tab, W=2, rank=0, to=1000, st=st: md.raw_call(
-        "moedisp_ep_barrier", tab, W, rank, 1, to, st, None)
+    b = lambda tab=tab, W=2, rank=0, to=1000, st=st, ep=1: md.raw_call(
+        "moedisp_ep_barrier", tab, W, rank, ep, to, st, None)
     assert b(tab=None) == md.MOEDISP_ERR_NULLPTR
+    assert b(ep=0) == md.MOEDISP_ERR_INVALID                   # zeroed words would pass
     assert b(st=None) == md.MOEDISP_ERR_NULLPTR
     assert b(W=0) == md.MOEDISP_ERR_INVALID
     assert b(rank=2) == md.MOEDISP_ERR_INVALID
@@ -318,10 +319,11 @@ def test_pipelined_rejections(md):
     inp, so, os_, do, recv, ex, sc, ready, ws, st = (FAKE + (i << 20) for i in range(64, 74))
 
     def p(inp=inp, stride=10, so=so, recv=recv, H=128, d=d, q=0, ex=ex, sc=None, ready=ready,
-          roles=3, lim=1000, ws=ws, wsb=ws_need, st=st):
+          roles=3, lim=1000, ws=ws, wsb=ws_need, st=st, ep=1):
         return md.raw_call("moedisp_a2a_dispatch_pipelined", inp, stride, so, os_, do, recv, H, d,
-                           ctypes.byref(L), q, ex, sc, None, 1, None, ready, 1, roles, lim, ws, wsb,
-                           st, None)
+                           ctypes.byref(L), q, ex, sc, None, 1, None, ready, ep, roles, lim, ws,
+                           wsb, st, None)
+    assert p(ep=0) == md.MOEDISP_ERR_INVALID                   # zeroed words would read as published
     assert p(st=None) == md.MOEDISP_ERR_NULLPTR
     assert p(ready=None) == md.MOEDISP_ERR_NULLPTR
     assert p(ws=None) == md.MOEDISP_ERR_NULLPTR

@@ -393,6 +393,12 @@ SMOOTH_CASES = [
     (dict(W=2, T=40, K=8, E=16, H=7168, outlier_frac=0.05, zero_rows=0.05), 2),  # 4 warps
     (dict(W=2, T=20, K=16, E=32, H=16384, routing="dup"), 3),                    # 8 warps, K = 16
     (dict(W=3, T=333, K=3, E=9, H=512, active_p=0.7), 3),
+    # rows taken rank by rank over many chunks, Zipf routing (rare experts: tiny parts)
+    (dict(W=8, T=600, K=8, E=64, H=1024, routing="zipf"), 2),
+    (dict(W=16, T=100, K=6, E=256, H=256, routing="zipf", active_p=0.7), 3),   # W*E = 4096
+    (dict(W=1, T=500, K=4, E=16, H=256, slot_active_p=0.8), 3),
+    # W*E above the rank-order tables' limit: rows taken in expand_x order
+    (dict(W=8, T=30, K=4, E=1024, H=128), 2),
 ]
 
 
@@ -608,19 +614,24 @@ def test_int8_half_integer_ties(md):
     assert np.array_equal(full.cpu().numpy()[gr:gr + ref["R"]], rex[:ref["R"]])
 
 
-def test_dispatch_capacity_guard(md):
+@pytest.mark.parametrize("q,smooth", [(2, False), (2, True), (3, True)])
+def test_dispatch_capacity_guard(md, q, smooth):
     w = wl.moe_workload("tiny", seed=8, W=2, T=100, K=4, E=8, H=64)
     cap = 500                                                      # R = 800
+    sm = wl.smooth_scales(w.E, w.H, seed=9) if smooth else None
     L, st = run_layout(md, w, rows_cap=cap)
     assert st == md.STATUS_CAPACITY
-    full, scales, gr, _, _, st = run_dispatch(md, w, L, 2)
+    full, scales, gr, _, _, st = run_dispatch(md, w, L, q, smooth=sm)
     assert st & md.STATUS_CAPACITY
     got = full.cpu().numpy()
     assert (got[:gr] == 0x5A).all() and (got[gr + cap:] == 0x5A).all()
     ref = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, None, rows_cap=cap)
-    rex, rsc, fl = oracle.moe_dispatch(w.x_bits, ref["dst_row"], w.K, cap, 2)
+    rex, rsc, fl = oracle.moe_dispatch(w.x_bits, ref["dst_row"], w.K, cap, q, smooth=sm,
+                                       expert_ids=w.expert_ids if smooth else None)
     assert fl & oracle.ORC_CAPACITY
     assert np.array_equal(got[gr:gr + cap], rex[:cap])
+    s_ = scales.cpu().numpy()
+    assert np.array_equal(s_[gr:gr + cap].view(np.uint32), rsc[:cap].view(np.uint32))
 
 
 # ------------------------------------------------------------------- combine
@@ -1024,6 +1035,48 @@ def test_pipelined_exchange_and_dispatch(md, q, W, max_split, H, K, ne):
     published = ready.cpu().numpy().reshape(-1)
     nonempty = (c["a"].in_splits.T.reshape(-1) > 0)
     assert (published[nonempty] == 2).all() and (published[~nonempty] == 0).all()
+
+
+@pytest.mark.parametrize("q", [0, 2])
+def test_pipelined_graph_replay_with_zeroed_ready_words(md, q):
+    """The form a CUDA graph replays: the ready words zeroed in stream order, then the call
+    with the same epoch (1) every time. Three replays of one captured graph over new token
+    values (same plan and layout) each equal the oracle's exchange and dispatch of them."""
+    c = _pipelined_case(md, 97, 8, 100, 512, 4, 2)
+    W, T, H, L = c["W"], c["T"], c["H"], c["L"]
+    src, outs, dsto, _ = oracle.a2a_exchange_plan(c["a"].in_splits)
+    ready, ws = _pipe_state(md, W)
+    ready.fill_(7)                                   # stale words from some earlier use
+    x_dev = bf16_dev(c["x"].reshape(-1, H))
+    recv_dev = torch.empty((W * T, H), dtype=torch.int16, device="cuda")
+    full, scales, gr = alloc_expand(L, H, q)
+    etn = torch.empty((W, c["ne"]), dtype=torch.int64, device="cuda")
+    erc = torch.empty((W, c["ne"], W), dtype=torch.int32, device="cuda")
+    st = new_status()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        ready.zero_()
+        md.a2a_dispatch_pipelined(x_dev, c["cap_in"], c["plan"][0], c["plan"][1], c["plan"][2],
+                                  recv_dev, H, L, q, full[gr:gr + L.rows_cap],
+                                  scales[gr:gr + L.rows_cap] if q else None, ready, 1, ws, st,
+                                  expert_token_nums=etn, ep_recv_counts=erc)
+    rng = np.random.default_rng(98)
+    for rep in range(3):
+        x = c["x"] if rep == 0 else wl.f32_to_bf16_bits(
+            (rng.standard_normal(c["x"].shape) * (1 + rep)).astype(np.float32))
+        x_dev.copy_(bf16_dev(x.reshape(-1, H)))
+        recv_dev.fill_(0x7777)
+        full.fill_(0x5A if q else -12345)
+        scales.fill_(-1.0)
+        etn.fill_(-1)
+        erc.fill_(-1)
+        g.replay()
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        recv = np.full((W, T, H), 0x7777, np.uint16)
+        assert oracle.a2a_v(x, recv, src, outs, dsto) == 0
+        _check_pipelined(md, dict(c, x=x, recv=recv), q, recv_dev, (full, scales, gr, etn, erc))
+    del g
 
 
 @pytest.mark.slow
