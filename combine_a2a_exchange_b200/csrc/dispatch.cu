@@ -48,6 +48,7 @@ struct DispatchArgs {
     const int64_t* expert_base;
     const int64_t* rank_base;
     int W, E, ne;
+    uint64_t kmagic;           // ceil(2^34 / K): slot / K = (slot * kmagic) >> 34 for slots < 2^30
     int64_t* etn;
     int etn_type;
     int32_t* erc;
@@ -243,7 +244,7 @@ __device__ __forceinline__ float fmax3_abs(float a, float b, float c) {
     return r;
 }
 
-template <int Q, int WPT, int CPT>
+template <int Q, int WPT, int CPT, bool EXACT>
 __device__ __forceinline__ void smooth_rows(const DispatchArgs& a, float4* sbuf, float (*red)[2][WPT],
                                             int e, int64_t row, int64_t seg_end, int& parity) {
     constexpr int NG = kQuantThreads / 32 / WPT;     // groups per block
@@ -251,7 +252,8 @@ __device__ __forceinline__ void smooth_rows(const DispatchArgs& a, float4* sbuf,
     constexpr float kQmax = Q == MOEDISP_QUANT_INT8 ? 127.0f : 448.0f;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int grp = warp / WPT, gw = warp - grp * WPT, gt = tid - grp * GT;
-    const int nvec = a.H >> 3, n4 = a.H >> 2;
+    // an exact fit (nvec == CPT * GT) makes every bounds test below a compile-time true
+    const int nvec = EXACT ? CPT * GT : a.H >> 3, n4 = 2 * nvec;
     const int64_t slots = a.G * a.K;
     const uint4* x4 = reinterpret_cast<const uint4*>(a.x);
     // smooth[e] in two planes: chunk c's first four values at sbuf[c], its last four at
@@ -268,7 +270,7 @@ __device__ __forceinline__ void smooth_rows(const DispatchArgs& a, float4* sbuf,
             if (gt == 0) raise_status(a.status, MOEDISP_STATUS_BAD_EXPERT_ID);
             continue;
         }
-        const int64_t xrow = token_source(a, slot / a.K);     // same for the group
+        const int64_t xrow = token_source(a, (int64_t)(((uint64_t)(uint32_t)slot * a.kmagic) >> 34));
         if (xrow < 0 || xrow >= a.x_rows) {
             if (gt == 0) raise_status(a.status, MOEDISP_STATUS_BAD_SPLIT);
             continue;
@@ -335,8 +337,9 @@ __device__ __forceinline__ void smooth_rows(const DispatchArgs& a, float4* sbuf,
     }
 }
 
-template <int Q, int WPT, int CPT, bool RANK_ORDER>
-__global__ void __launch_bounds__(kQuantThreads, CPT > 4 ? 3 : 4) dispatch_smooth_kernel(DispatchArgs a) {
+template <int Q, int WPT, int CPT, bool RANK_ORDER, bool EXACT>
+__global__ void __launch_bounds__(kQuantThreads, EXACT && WPT == 1 ? 2 : (CPT > 4 ? 3 : 4))
+dispatch_smooth_kernel(DispatchArgs a) {
     constexpr int NG = kQuantThreads / 32 / WPT;
     extern __shared__ __align__(16) float4 sbuf[];   // [H / 4]: smooth[e]; then the tables
     __shared__ float red[NG][2][WPT];
@@ -365,7 +368,7 @@ __global__ void __launch_bounds__(kQuantThreads, CPT > 4 ? 3 : 4) dispatch_smoot
             for (int e = lo; r < end; ++e) {
                 const int64_t seg_end = min64(end, a.expert_base[e + 1]);
                 if (seg_end <= r) continue;
-                smooth_rows<Q, WPT, CPT>(a, sbuf, red, e, r, seg_end, parity);
+                smooth_rows<Q, WPT, CPT, EXACT>(a, sbuf, red, e, r, seg_end, parity);
                 r = seg_end;
             }
         }
@@ -418,7 +421,7 @@ __global__ void __launch_bounds__(kQuantThreads, CPT > 4 ? 3 : 4) dispatch_smoot
             const int e = i % a.E;
             const int64_t row = __ldg(a.expert_base + e) + cpre[i] + (v - vpre[i]);
             const int64_t row_end = min64(R, row + (part_end - v));
-            if (row < row_end) smooth_rows<Q, WPT, CPT>(a, sbuf, red, e, row, row_end, parity);
+            if (row < row_end) smooth_rows<Q, WPT, CPT, EXACT>(a, sbuf, red, e, row, row_end, parity);
             v = part_end;
         }
     }
@@ -561,7 +564,12 @@ cudaError_t launch_copy(DispatchArgs a, cudaStream_t stream) {
 // chunks each (up to 8; 80 registers, 3 blocks per SM) beat many warps with few chunks:
 // cfg3 (H = 7168: 4 warps x 7 chunks, an exact fit) 1430 -> 1083 us against 8 x 4; cfg4
 // (H = 2048: 1 warp x 8) 282 -> 248 us against 2 x 4; 2 blocks per SM (105 registers)
-// measured in between.
+// measured in between. When the row fits the group exactly (H / 8 == CPT * WPT * 32) the
+// kernel is built with every bounds test resolved at compile time (EXACT), which lets the
+// compiler overlap the chunks' loads and arithmetic freely: cfg3 1089 -> 997 us (with a
+// few spilled registers at 80, still the faster), cfg4 237 -> 218 us, and 202 us with one
+// warp per row at 2 blocks per SM (no spills); with 4-warp rows 2 blocks per SM lost
+// (1153 us).
 //
 // Rank order (see the kernel) when x is well beyond the L2 (up to about twice its size
 // most of the K re-reads of a row hit it anyway, and the tables cost more than they save:
@@ -570,23 +578,29 @@ cudaError_t launch_copy(DispatchArgs a, cudaStream_t stream) {
 // counts fit in 32 bits.
 constexpr int kSmoothMaxParts = 4096;
 
-template <int Q, int WPT, int CPT>
-cudaError_t launch_smooth_w(DispatchArgs a, cudaStream_t stream) {
+template <int Q, int WPT, int CPT, bool EXACT>
+cudaError_t launch_smooth_x(DispatchArgs a, cudaStream_t stream) {
     const int64_t WE = (int64_t)a.W * a.E;
     const bool ranked = a.cnt != nullptr && WE <= kSmoothMaxParts && a.G * a.K < (int64_t)INT32_MAX &&
                         a.x_rows * (int64_t)a.in_bytes > 2 * current_l2_bytes();
     const size_t smem = (size_t)a.H * 4 + (ranked ? (size_t)(2 * WE + 1) * 4 : 0);
-    const void* fn = ranked ? (const void*)dispatch_smooth_kernel<Q, WPT, CPT, true>
-                            : (const void*)dispatch_smooth_kernel<Q, WPT, CPT, false>;
+    const void* fn = ranked ? (const void*)dispatch_smooth_kernel<Q, WPT, CPT, true, EXACT>
+                            : (const void*)dispatch_smooth_kernel<Q, WPT, CPT, false, EXACT>;
     int per_sm = 1;
     cudaError_t err = blocks_per_sm(fn, kQuantThreads, smem, &per_sm);
     if (err != cudaSuccess) return err;
     const int64_t grid = (int64_t)current_sm_count() * per_sm;
     if (ranked)
-        return launch_pdl(dispatch_smooth_kernel<Q, WPT, CPT, true>, dim3((unsigned)grid),
+        return launch_pdl(dispatch_smooth_kernel<Q, WPT, CPT, true, EXACT>, dim3((unsigned)grid),
                           dim3(kQuantThreads), smem, stream, 1, a);
-    return launch_pdl(dispatch_smooth_kernel<Q, WPT, CPT, false>, dim3((unsigned)grid),
+    return launch_pdl(dispatch_smooth_kernel<Q, WPT, CPT, false, EXACT>, dim3((unsigned)grid),
                       dim3(kQuantThreads), smem, stream, 1, a);
+}
+
+template <int Q, int WPT, int CPT>
+cudaError_t launch_smooth_w(DispatchArgs a, cudaStream_t stream) {
+    if (a.H / 8 == CPT * WPT * 32) return launch_smooth_x<Q, WPT, CPT, true>(a, stream);
+    return launch_smooth_x<Q, WPT, CPT, false>(a, stream);
 }
 
 template <int Q>
@@ -660,6 +674,7 @@ cudaError_t launch_dispatch(const void* x, int64_t x_rows, const int64_t* token_
     a.in_bytes = (uint32_t)H * 2u;
     a.out_bytes = quant_mode == MOEDISP_QUANT_NONE ? (uint32_t)H * 2u : (uint32_t)H;
     a.cnt = L.cnt;
+    a.kmagic = ((uint64_t(1) << 34) + (uint64_t)dims.K - 1) / (uint64_t)dims.K;
     a.expert_base = L.expert_base;
     a.rank_base = L.rank_base;
     a.W = dims.W;
@@ -704,6 +719,7 @@ cudaError_t launch_dispatch_peers(const void* x, int H, const moedisp_dims& dims
     a.in_bytes = (uint32_t)H * 2u;
     a.out_bytes = quant_mode == MOEDISP_QUANT_NONE ? (uint32_t)H * 2u : (uint32_t)H;
     a.cnt = nullptr;
+    a.kmagic = ((uint64_t(1) << 34) + (uint64_t)dims.K - 1) / (uint64_t)dims.K;
     a.expert_base = L.expert_base;
     a.rank_base = L.rank_base;
     a.W = dims.W;

@@ -7,6 +7,7 @@ import os
 import re
 import subprocess
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -363,3 +364,16 @@ def test_ipc_rejections(md):
     assert lib.moedisp_ipc_import(h, -1, ctypes.byref(p)) == md.MOEDISP_ERR_INVALID
     assert lib.moedisp_ipc_close(None) == md.MOEDISP_ERR_NULLPTR
     assert lib.moedisp_ipc_close(FAKE) == md.MOEDISP_ERR_INVALID       # never imported
+
+
+def test_slot_division_by_k_multiply_shift():
+    """The smoothing dispatch divides a slot (< 2^30) by K (<= 16) as (slot * ceil(2^34 / K))
+    >> 34: with M = 2^34 / K + e (0 <= e < 1) the quotient is slot / K + slot * e / 2^34, whose
+    excess stays below 2^-4 <= 1 / K, so the floor is exact. Every K, both ends of the slot
+    range and a seeded sample between them."""
+    rng = np.random.default_rng(5)
+    slots = np.concatenate([np.arange(0, 4096), (1 << 30) - 1 - np.arange(0, 4096),
+                            rng.integers(0, 1 << 30, 50000)]).astype(object)
+    for K in range(1, 17):
+        M = ((1 << 34) + K - 1) // K
+        assert all((int(s) * M) >> 34 == int(s) // K for s in slots), K
