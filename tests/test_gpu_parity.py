@@ -590,6 +590,41 @@ def test_fp8_conversion_exhaustive_over_bf16(md):
     assert np.array_equal(got, exp)
 
 
+def test_fp8_ties_with_an_inexact_reciprocal(md):
+    """Rows whose largest magnitude is 672 have scale exactly 672 / 448 = 1.5 while 1 / 1.5
+    is not a binary fraction, so the shortcut product x * (1 / scale) is off the true
+    quotient by an ulp or so. x = 1.5 * b for every E4M3 rounding midpoint b that bf16
+    holds exactly makes x / scale an exact tie (round half to even), with the values one
+    bf16 ulp either side next to it: each must come out as the oracle's code, i.e. the
+    undecided window must fall back to the IEEE quotient."""
+    mids = _rounding_boundaries(3)
+    xs = (1.5 * mids).astype(np.float32)
+    bits = wl.f32_to_bf16_bits(xs)
+    exact = wl.bf16_bits_to_f32(bits).astype(np.float64) == 1.5 * mids
+    b = bits[exact]
+    vals = np.concatenate([b, b + 1, b - 1]).astype(np.uint16)     # bf16 neighbours
+    assert b.size > 100
+    H = 256
+    per = H - 1
+    n_rows = -(-vals.size // per)
+    x = np.zeros((n_rows, H), np.uint16)
+    x[:, 0] = wl.f32_to_bf16_bits(np.float32(672.0))
+    flat = np.zeros(n_rows * per, np.uint16)
+    flat[:vals.size] = vals
+    x[:, 1:] = flat.reshape(n_rows, per)
+    T = n_rows
+    w = wl.MoEWorkload(name="e4m3_ties", W=1, T=T, H=H, E=1, K=1, quant_mode=3, x_bits=x,
+                       expert_ids=np.zeros((T, 1), np.int32),
+                       weights=np.ones((T, 1), np.float32), active=None)
+    L, _ = run_layout(md, w)
+    ref = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, None)
+    full, scales, gr, _, _, st = run_dispatch(md, w, L, 3)
+    assert st == 0
+    assert (scales.cpu().numpy()[gr:gr + T] == 1.5).all()
+    rex, rsc, _ = oracle.moe_dispatch(x, ref["dst_row"], w.K, ref["rows_cap"], 3)
+    assert np.array_equal(full.cpu().numpy()[gr:gr + T], rex[:T])
+
+
 def test_int8_half_integer_ties(md):
     """Rows whose largest magnitude is 127 have scale exactly 1, so x / scale = x: rows of
     half-integers k + 0.5 sit exactly on int8 rounding boundaries (round half to even)
