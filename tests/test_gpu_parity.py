@@ -200,14 +200,13 @@ LAYOUT_CASES = [
     ("tiny", dict(W=64, T=33, K=8, E=1024)),              # many experts and ranks
     # beyond one 16-block cluster: the tiled (count, scan, rank) path
     ("tiny", dict(W=2, T=40000, K=8, E=16)),              # 158 tiles of up to 4096 slots
-    ("tiny", dict(W=4, T=70000, K=8, E=64)),              # > kScanRows tiles: multi-pass scan
+    ("tiny", dict(W=4, T=70000, K=8, E=64)),              # 548 tiles: two passes of the scan
     ("tiny", dict(W=20, T=300, K=4, E=40, active_p=0.5)),
     ("tiny", dict(W=3, T=30000, K=6, E=300, routing="zipf", zipf_zero=30)),
     # one cluster, two tiles per rank and the largest tile
     ("tiny", dict(W=8, T=2048, K=8, E=256, routing="zipf")),
     ("tiny", dict(W=1, T=2048, K=8, E=1024)),
-    # one cluster of 1024-thread blocks (tiles of up to 16384 slots): E = 1024 near the
-    # shared-memory limit, a per-token mask with ragged tiles, a per-slot mask
+    # the tiled path at E = 1024, a per-token mask with ragged tiles, a per-slot mask
     ("tiny", dict(W=4, T=4096, K=4, E=1024)),
     ("tiny", dict(W=16, T=1000, K=8, E=128, active_p=0.6)),
     ("tiny", dict(W=8, T=3001, K=5, E=64, slot_active_p=0.7)),
