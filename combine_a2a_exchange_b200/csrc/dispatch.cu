@@ -216,26 +216,6 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
     if (issuer) bulk_wait<0>();
 }
 
-// Quantising dispatch with per-expert smoothing. The copy of token g for expert e is
-// x[g] * smooth[e] quantised on its own, so the work is per row of expand_x, not per
-// token, and it is arithmetic-heavy (a product, a maximum and a quantisation per output
-// element). A block takes chunks of rows of one expert at a time: it copies smooth[e] into
-// shared memory once per run of rows, and its token groups (WPT warps each) share the
-// rows. A group gathers its row's token x[assist_info[row] / K] straight into registers
-// (CPT 16-byte chunks per thread, all loads issued before the first use), reduces
-// max |x * smooth[e]| (shuffles, plus a named barrier across the group's warps), and
-// stores the codes (8 bytes per chunk, coalesced) and the row's scale. No staging
-// buffers, so many warps fit an SM; nothing waits on another block.
-//
-// Order of the rows. Within an expert's segment the rows are in slot order, hence grouped
-// by source rank: rank r's rows of expert e start at expert_base[e] + sum_{r'<r} cnt[r'][e].
-// RANK_ORDER walks the rows rank by rank (for each rank, its part of every expert's
-// segment), so that all K copies of a token are quantised while its x row is still in L2:
-// the whole grid works on one or two ranks' tokens at a time instead of on every token
-// (each row of x is then read from DRAM about once rather than up to K times). Without
-// RANK_ORDER (cnt absent or the tables too large) the rows go in expand_x order.
-
-// Rows [row, seg_end) of expert e; smooth[e] is loaded into sbuf first.
 // max(|a|, |b|, |c|) in one instruction (the three-input form of max, sm_100 and later);
 // like fmaxf, a NaN input is passed over in favour of the others.
 __device__ __forceinline__ float fmax3_abs(float a, float b, float c) {
@@ -244,6 +224,27 @@ __device__ __forceinline__ float fmax3_abs(float a, float b, float c) {
     return r;
 }
 
+// Quantising dispatch with per-expert smoothing. The copy of token g for expert e is
+// x[g] * smooth[e] quantised on its own, so the work is per row of expand_x, not per
+// token, and it is arithmetic-heavy (a product, a maximum and a quantisation per output
+// element). A block takes chunks of rows of one expert at a time: it copies smooth[e] into
+// shared memory once per run of rows, and its token groups (WPT warps each) share the
+// rows. A group gathers its row's token x[assist_info[row] / K] straight into registers
+// (CPT 16-byte chunks per thread, all loads issued before the first use), reduces
+// max |x * smooth[e]| (shuffles, plus a named barrier across the group's warps), and
+// stores the codes (window quantisation, 8 bytes per chunk, coalesced) and the row's
+// scale. No staging buffers; nothing waits on another block.
+//
+// Order of the rows. Within an expert's segment the rows are in slot order, hence grouped
+// by source rank: rank r's rows of expert e start at expert_base[e] + sum_{r'<r} cnt[r'][e].
+// RANK_ORDER walks the rows rank by rank (for each rank, its part of every expert's
+// segment), so that all K copies of a token are quantised while its x row is still in L2:
+// the whole grid works on one or two ranks' tokens at a time instead of on every token
+// (each row of x is then read from DRAM about once rather than up to K times). Without
+// RANK_ORDER (x within twice the L2, cnt absent or the tables too large) the rows go in
+// expand_x order.
+
+// Rows [row, seg_end) of expert e; smooth[e] is loaded into sbuf first.
 template <int Q, int WPT, int CPT, bool EXACT>
 __device__ __forceinline__ void smooth_rows(const DispatchArgs& a, float4* sbuf, float (*red)[2][WPT],
                                             int e, int32_t row, int32_t seg_end, int& parity) {
