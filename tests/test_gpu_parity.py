@@ -424,6 +424,35 @@ def test_dispatch_smoothing_parity(md, over, q):
     assert (s[:gr] == -1).all() and (s[gr + R:] == -1).all()
 
 
+@pytest.mark.parametrize("q,W,H,E", [(2, 8, 7168, 32), (3, 16, 2048, 64)])
+def test_dispatch_smoothing_rank_order(md, q, W, H, E):
+    """The smoothing kernel walks its rows rank by rank when the token rows are well beyond
+    the L2 (more than twice its size): T is chosen from this device's L2 so that they are,
+    with cfg3's row width in int8 and cfg4's in e4m3 (the benchmark's instantiations), K = 2
+    and Zipf routing. Every row's codes and scale bit-exact against the oracle."""
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    T = int(2.3 * l2 / (W * H * 2)) + 1
+    w = wl.moe_workload("tiny", seed=44, W=W, T=T, K=2, E=E, H=H, routing="zipf", zipf_zero=2,
+                        active_p=0.9)
+    assert w.G * H * 2 > 2 * l2
+    sm = wl.smooth_scales(w.E, w.H, seed=45)
+    L, st0 = run_layout(md, w)
+    assert st0 == 0
+    ref = oracle.moe_dispatch_layout(w.W, w.T, w.K, w.E, w.expert_ids, w.active)
+    full, scales, gr, _, _, st = run_dispatch(md, w, L, q, smooth=sm)
+    assert st == 0
+    R = ref["R"]
+    rex, rsc, fl = oracle.moe_dispatch(w.x_bits, ref["dst_row"], w.K, ref["rows_cap"], q,
+                                       smooth=sm, expert_ids=w.expert_ids)
+    assert fl == 0
+    got = full.cpu().numpy()
+    del full
+    assert np.array_equal(got[gr:gr + R], rex[:R])
+    assert (got[:gr] == 0x5A).all() and (got[gr + R:] == 0x5A).all()
+    del got, rex
+    assert np.array_equal(scales.cpu().numpy()[gr:gr + R].view(np.uint32), rsc[:R].view(np.uint32))
+
+
 def _rounding_boundaries(q):
     """The quantiser's rounding boundaries below its largest code: int8, the half-integers
     k + 0.5 with |k + 0.5| < 127; e4m3, the midpoints between neighbouring finite codes
