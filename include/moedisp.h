@@ -240,9 +240,10 @@ int moedisp_moe_dispatch_layout_noalloc(const int32_t *expert_ids, const uint8_t
  * fp32 [E][H] device, 16-byte aligned, or NULL; quant modes only (with NONE it is
  * MOEDISP_ERR_INVALID). When given, the copy for slot s = (g, k) routed to expert e
  * quantises x[g] * smooth_scales[e] (one fp32 product per element) instead of x[g], with
- * its own a and scale. The rows are then produced in expand_x order from the layout's
- * expert_base and assist_info (a row whose assist_info is outside [0, G*K) is skipped and
- * sets MOEDISP_STATUS_BAD_EXPERT_ID); dst_row is not read.
+ * its own a and scale. The rows are then produced from the layout's expert_base,
+ * assist_info and, when it is given, cnt (which orders the work rank by rank when x is
+ * large; a row whose assist_info is outside [0, G*K) is skipped and sets
+ * MOEDISP_STATUS_BAD_EXPERT_ID); dst_row is not read.
  * x: bf16 [G][H] device, 16-byte aligned; expand_x: [layout->rows_cap][H] elements of
  * the output type, 16-byte aligned, not overlapping x; dynamic_scales: fp32
  * [rows_cap] (required for quant modes, ignored otherwise). H % 8 == 0 (NONE) or
@@ -254,11 +255,13 @@ int moedisp_moe_dispatch_layout_noalloc(const int32_t *expert_ids, const uint8_t
  *     major_align the last source rank's entry also counts the expert's padding rows (as
  *     the 2-D plan's out_splits do), and expert_token_nums counts padded segments.
  * Rows at or beyond rows_cap are not written (MOEDISP_STATUS_CAPACITY).
- * One persistent kernel: without smoothing each token row is brought into shared memory
- * once by a bulk (TMA) copy; unquantised rows leave it as K bulk copies, quantised ones as
- * 8-byte streaming stores of the codes to the K rows. With smoothing each block walks
- * runs of consecutive rows, holding one expert's smoothing row in shared memory and
- * gathering the rows' tokens by bulk copies. */
+ * One persistent kernel: an unquantised token row is brought into shared memory once by
+ * a bulk (TMA) copy and leaves it as K bulk copies; a quantised one is read once into
+ * registers and its codes leave as 8-byte streaming stores to the K rows. With smoothing
+ * each block walks runs of rows of one expert, holding that expert's smoothing row in
+ * shared memory and gathering each row's token into registers. The codes are those of the
+ * IEEE quotient x / scale bit for bit (a faster decision is used only where it provably
+ * agrees). */
 int moedisp_moe_dispatch(const void *x, int H, moedisp_dims dims,
                          const moedisp_layout *layout, int quant_mode,
                          const float *smooth_scales, void *expand_x,
