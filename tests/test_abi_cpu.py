@@ -377,3 +377,32 @@ def test_slot_division_by_k_multiply_shift():
     for K in range(1, 17):
         M = ((1 << 34) + K - 1) // K
         assert all((int(s) * M) >> 34 == int(s) // K for s in slots), K
+
+
+def test_window_quantisation_brackets_the_ieee_quotient():
+    """The quantisers' window: with inv = RN(1/scale), lo = RN(inv * RN(1 - 2^-22)) and
+    hi = RN(inv * RN(1 + 2^-22)) in fp32, the exact products x*lo and x*hi must bracket the
+    IEEE quotient RN(x/scale) for every normal scale: lo < (1/scale)(1 - 2^-24) and
+    hi > (1/scale)(1 + 2^-24), which the quotient's own rounding (|RN(q) - q| <= q 2^-24)
+    cannot cross. Checked in exact rational arithmetic on seeded scales spanning the normal
+    range (both ends included) and on mantissas next to powers of two."""
+    from fractions import Fraction
+    rng = np.random.default_rng(11)
+    f32 = np.float32
+    one_m, one_p = f32(1 - 2.0 ** -22), f32(1 + 2.0 ** -22)
+    assert Fraction(float(one_m)) == 1 - Fraction(1, 2 ** 22)
+    assert Fraction(float(one_p)) == 1 + Fraction(1, 2 ** 22)
+    exps = rng.integers(-126, 122, 3000)
+    mant = rng.random(3000) + 1.0
+    scales = np.concatenate([(mant * 2.0 ** exps).astype(f32),
+                             np.array([np.finfo(f32).tiny, f32(2.0 ** 121), f32(1.0), f32(1.5),
+                                       np.nextafter(f32(1.0), f32(2.0)), np.nextafter(f32(2.0), f32(1.0))],
+                                      f32)])
+    eps = Fraction(1, 2 ** 24)
+    for sc in scales:
+        assert np.isfinite(sc) and sc >= np.finfo(f32).tiny
+        inv = f32(1.0) / sc                                   # IEEE round to nearest
+        lo, hi = inv * one_m, inv * one_p
+        q = 1 / Fraction(float(sc))
+        assert Fraction(float(lo)) < q * (1 - eps), sc
+        assert Fraction(float(hi)) > q * (1 + eps), sc
