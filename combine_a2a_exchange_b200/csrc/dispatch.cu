@@ -425,7 +425,10 @@ dispatch_smooth_kernel(DispatchArgs a) {
             const int e = i % a.E;
             const int32_t row = (int32_t)__ldg(a.expert_base + e) + cpre[i] + (v - vpre[i]);
             const int32_t row_end = min(R, row + (part_end - v));
-            if (row < row_end) smooth_rows<Q, WPT, CPT, EXACT>(a, sbuf, red, e, row, row_end, parity);
+            // (a layout whose counts disagree with its bases yields rows outside [0, R):
+            // none of them is touched)
+            if (row >= 0 && row < row_end)
+                smooth_rows<Q, WPT, CPT, EXACT>(a, sbuf, red, e, row, row_end, parity);
             v = part_end;
         }
     }
