@@ -773,3 +773,42 @@ def test_shared_experts_argument_rules():
     assert ok(4, 4, 1, 3) & oracle.ORC_BAD_ARG                   # W % S != 0
     ext, _, _, _ = oracle.shared_expert_routing(4, 2, 2, 4, 0, 0, ids, wts)
     assert np.array_equal(ext, ids)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_layout_segments_are_grouped_by_source_rank(seed):
+    """The order the smoothing dispatch may walk rows in rests on this property of the
+    layout: within expert e's segment the routed rows come rank by rank, rank r's part
+    starting at expert_base[e] + sum_{r'<r} cnt[r'][e] and holding cnt[r][e] rows, and any
+    major_align padding follows all of them. Checked on the oracle's layouts (masks,
+    duplicates, padding): the parts enumerate every routed row once and each part's rows
+    belong to tokens of its rank."""
+    rng = np.random.default_rng(700 + seed)
+    W = int(rng.integers(1, 9))
+    ne = int(rng.integers(1, 6))
+    E, K, T = W * ne, int(rng.integers(1, 9)), int(rng.integers(0, 120))
+    over = dict(W=W, T=T, K=K, E=E, H=8, routing="dup" if K > E or seed % 2 else "uniform")
+    if seed % 3 == 1:
+        over["active_p"] = 0.7
+    elif seed % 3 == 2:
+        over["slot_active_p"] = 0.6
+    w = wl.moe_workload("tiny", seed=seed, **over)
+    A = [0, 4, 16][seed % 3]
+    ref = oracle.moe_dispatch_layout(W, T, K, E, w.expert_ids, w.active, major_align=A)
+    cnt, eb, assist = ref["cnt"], ref["expert_base"], ref["assist_info"]
+    seen = []
+    for e in range(E):
+        start = int(eb[e])
+        for r in range(W):
+            n = int(cnt[r, e])
+            rows = np.arange(start, start + n)
+            slots = assist[rows]
+            assert (slots >= 0).all()
+            assert ((slots // K) // T == r).all()               # tokens of rank r
+            assert (w.expert_ids.reshape(-1)[slots] == e).all()
+            seen.append(rows)
+            start += n
+        assert (assist[start:int(eb[e + 1])] == -1).all()       # padding after every part
+    seen = np.concatenate(seen) if seen else np.zeros(0, np.int64)
+    routed = np.nonzero(assist[:ref["R"]] >= 0)[0]
+    assert np.array_equal(np.sort(seen), routed)
