@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(kCopyThreads) dispatch_copy_kernel(DispatchArg
     for (int it = 0;; ++it) {
         const int st = it % S;
         const uint32_t par = (uint32_t)((it / S) & 1);
-        // Lane 0 waits with a time limit and shares the verdict; then every lane observes
+        // Lane 0 waits with a time limit and shares the outcome; then every lane observes
         // the already completed phase itself.
         int ok = 1;
         if (lane == 0) ok = mbar_wait(&bars[st], par) ? 1 : 0;
